@@ -1,0 +1,179 @@
+/*
+ * q4.h -- C ABI of the group-wise INT4 linear layers and the INT4 MoE expert FFN for NVIDIA B200
+ * (sm_100a).  Library: moe_linear_layers_b200/libq4.so.
+ *
+ * The calls follow the problem as the source pages state it:
+ *   - "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" (below: the W4A8 page) §2.3: weights are
+ *     quantized offline to INT4 with a scale and a zero point; at run time INT4 is widened to INT8,
+ *     multiplied with INT8 activations into INT32, and rescaled by scale_w*scale_a; §3.1: per-token
+ *     activation quantization from amax/127; §2.1: 4-bit storage restored to a 16-bit type for
+ *     W4A16;
+ *   - "从FP32到INT4：大语言模型量化压缩实战指南" §1.3: group-wise quantization, each group its own
+ *     range, a zero point only for the asymmetric form;
+ *   - "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" (INT4 group quantization; MoE experts
+ *     are small SwiGLU FFNs behind a gating network) and "大模型之Dense、MoE与量化" section
+ *     混合专家架构 MoE (a Linear router scores experts, a few are chosen, their outputs are
+ *     recombined in proportion).
+ *
+ * Conventions for every call:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The caller owns every
+ *     buffer; the library allocates no device memory.  Scratch space of the MoE layer is the
+ *     caller's workspace.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every call is
+ *     asynchronous on it.
+ *   - The return value reports errors the host can see before launching (null pointers, shapes,
+ *     alignment, unsupported options, workspace too small, a failed launch).  When it is not Q4_OK
+ *     nothing was launched (except Q4_ERR_CUDA, which reports a failed launch).
+ *   - `dev_status` (nullable) is a device int32 the kernels set, with the first error seen, when
+ *     they detect a problem in the data: Q4_ERR_NONFINITE for a non-finite input group/row,
+ *     Q4_ERR_TIMEOUT when a bounded wait inside a kernel ran out.  The library never clears it;
+ *     the caller zeroes it and reads it when convenient.  Outputs are undefined when it is set.
+ *   - fp16 and bf16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Matrices are row-major.
+ *
+ * Data layout of an INT4 weight W [n][k] (groups of `group` consecutive elements along k):
+ *   packed [n][k/2] u8   element k of a row is in byte k/2, even k in the low nibble;
+ *                        symmetric codes are 4-bit two's complement (-8..7, -8 never produced),
+ *                        asymmetric codes are 0..15;
+ *   scales [n][k/group]  fp16;
+ *   zeros  [n][k/group]  fp16 holding an integer 0..15 (asymmetric only; NULL when symmetric).
+ * Dequantized weight = (code - zero) * scale.
+ */
+#ifndef Q4_H
+#define Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_ERR_NULL = -1,        /* a required pointer is NULL */
+    Q4_ERR_SHAPE = -2,       /* a size is out of range or inconsistent */
+    Q4_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+    Q4_ERR_UNSUPPORTED = -4, /* an option this build does not implement */
+    Q4_ERR_WORKSPACE = -5,   /* workspace too small */
+    Q4_ERR_CUDA = -6,        /* a CUDA call failed (launch error) */
+    Q4_ERR_NONFINITE = -7,   /* (device) non-finite input, or a scale that overflows fp16 */
+    Q4_ERR_TIMEOUT = -8      /* (device) a bounded wait inside a kernel gave up */
+} q4_status;
+
+enum { Q4_OUT_F32 = 0, Q4_OUT_BF16 = 1 };
+
+/* Descriptor of one INT4 weight matrix (all pointers device pointers, 16-byte aligned). */
+typedef struct q4_weight {
+    int32_t n, k;        /* rows (output features) and columns (input features) */
+    int32_t group;       /* 64 or 128; k % group == 0 */
+    int32_t symmetric;   /* 1: codes -8..7, zeros == NULL; 0: codes 0..15 with zeros */
+    const uint8_t* packed;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+} q4_weight;
+
+/* Human-readable name of a status code (static string). */
+const char* q4_status_string(int status);
+
+/* Library version (increments with the ABI). */
+int q4_version(void);
+
+/*
+ * q4_quantize_pack -- round-to-nearest group quantization and packing of an fp32 matrix.
+ * Source: the W4A8 page §2.3 (offline INT4 quantization keeping scale and zero point) and §2.1
+ * (4-bit storage); "从FP32到INT4" §1.3 (per-group range; zero point only when asymmetric).
+ *   symmetric:  S = fp16(amax/7);            code = clamp(rne(w/S), -8, 7)
+ *   asymmetric: mn = min(min w, 0), mx = max(max w, 0), S = fp16((mx-mn)/15),
+ *               z = clamp(rne(-mn/S), 0, 15), code = clamp(rne(w/S) + z, 0, 15)
+ * All divisions are IEEE fp32; rne = round half to even; the STORED fp16 scale codes the group;
+ * a group whose scale is 0 codes to its zero point.
+ * w [n][k] fp32 (16-byte aligned); packed [n][k/2]; scales [n][k/group]; zeros [n][k/group]
+ * (required when symmetric == 0, ignored otherwise).  group in {64, 128}; k % group == 0.
+ * dev_status: Q4_ERR_NONFINITE when a group holds a non-finite value or its scale overflows fp16.
+ */
+int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t group, int32_t symmetric,
+                     uint8_t* packed, uint16_t* scales, uint16_t* zeros,
+                     int32_t* dev_status, void* stream);
+
+/*
+ * q4_linear_w4a16 -- y = x . dequant(W)^T with the dequantization fused in the kernel.
+ * Source: the W4A8 page §2.1 (4-bit storage restored to a 16-bit compute type) and §1 (small batch:
+ * memory bound; larger batch: compute bound).
+ * x [m][k] bf16; y [m][n] fp32 (out_dtype Q4_OUT_F32) or bf16 (Q4_OUT_BF16, round to nearest even of
+ * the fp32 result).  m >= 1.  Small m runs the memory-bound GEMV kernel (CUDA cores, in-register
+ * dequant); larger m runs the tcgen05 tensor-core GEMM (exact integer codes in bf16, fp32
+ * accumulation per group, scale applied per group in the epilogue).  The choice is by shape only.
+ * Requires k % 32 == 0 for the GEMV and k % 128 == 0 for the GEMM (see q4_linear_w4a16_max_gemv_m).
+ * dev_status: Q4_ERR_NONFINITE when x holds a non-finite value (GEMV path).
+ */
+int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
+                    int32_t* dev_status, void* stream);
+
+/* Largest m that q4_linear_w4a16 serves with the GEMV kernel. */
+int q4_linear_w4a16_max_gemv_m(void);
+
+/*
+ * act_quant_per_token -- per-token INT8 quantization of bf16 activations.
+ * Source: the W4A8 page §3.1: amax over the token, scale = amax/127, round half to even, clamp to
+ * [-128, 127].  scale_a[m] = amax/127 (fp32 division); xq = clamp(rne(x / scale_a), -128, 127);
+ * a token with amax == 0 gets scale 0 and all-zero codes.
+ * x [m][k] bf16; xq [m][k] int8; scale_a [m] fp32.  k % 8 == 0.
+ * dev_status: Q4_ERR_NONFINITE when a token holds a non-finite value.
+ */
+int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                        int32_t* dev_status, void* stream);
+
+/*
+ * q4_linear_w4a8 -- INT8 activations x INT4 weights widened to INT8, INT32 accumulation, rescale.
+ * Source: the W4A8 page §2.3 (three steps and the pseudo-code: dequant_int4_to_int8, int8 matmul
+ * into int32, rescale by scale_w * scale_a).  With one weight scale per group of 128 (or 64) the
+ * INT32 partial is kept per (token, row, group):
+ *   acc[m][n][g] = sum_{k in g} xq[m][k] * code[n][k]            (exact int32)
+ *   y[m][n]      = scale_a[m] * sum_g scale_w[n][g] * acc[m][n][g]  (fp32)
+ * W must be symmetric.  y [m][n] fp32 or bf16.  acc_dbg (nullable): [m][n][k/group] int32 copy of the
+ * partials, for verification only (slow).  k % 128 == 0.
+ */
+int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
+                   int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream);
+
+/*
+ * moe_q4_workspace_size -- bytes of device workspace moe_q4_forward needs for these sizes.
+ */
+size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk);
+
+/*
+ * moe_q4_forward -- top-k routed MoE layer of SwiGLU experts with INT4 weights (W4A16).
+ * Source: "大模型之Dense、MoE与量化" 混合专家架构 MoE (Linear router, a few experts per token,
+ * proportional recombination); the W4A8 page §3.2 (router kept in high precision, softmax output)
+ * and §1 (dispatch and merge cost); "高效大语言模型推理实践" MoE架构设计 (each expert a small FFN,
+ * SwiGLU as in the base model).
+ *   logits[t][e] = fp32 dot(x_t, router_w[e]) in a pinned order (+ router_bias[e]):
+ *                  32 partial sums over k = l (mod 32), each an fma chain with k ascending,
+ *                  combined by the butterfly p_l + p_(l xor s), s = 16, 8, 4, 2, 1;
+ *   ids[t][j]    = the topk experts by (logit descending, id ascending), slot j = j-th best;
+ *   w[t][j]      = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the chosen (= softmax, renormalised);
+ *   perm/offsets = stable counting sort of the pairs (t, j) by expert (tokens ascending);
+ *   h            = SiLU(x . Wg_e^T) * (x . Wu_e^T), kept as fp16;  o = h . Wd_e^T;
+ *   y[t]         = sum_j w[t][j] * o_(t,j).
+ * x [T][H] bf16; router_w [E][H] fp32; router_bias [E] fp32 or NULL.
+ * experts[3] = {gate, up, down}: gate and up are [E*I][H] stacked by expert (rows e*I .. e*I+I-1),
+ * down is [E*H][I]; all three with the same group (128 or 64) and symmetry.
+ * y [T][H] fp32 or bf16.  Optional outputs (nullable): topk_ids [T][topk] int32, topk_w [T][topk]
+ * fp32, perm [T*topk] int32 (value t*topk+j), offsets [E+1] int32, expert_counts [E] int32.
+ * workspace: device memory of at least moe_q4_workspace_size(T, H, I, E, topk) bytes, 256-byte
+ * aligned, owned by the caller; contents on entry are ignored.
+ * Limits: E <= 256, topk <= 16, H % 128 == 0, I % 128 == 0.
+ */
+int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H,
+                   const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                   const q4_weight* experts, int32_t I,
+                   void* y, int32_t out_dtype,
+                   int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                   void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H */

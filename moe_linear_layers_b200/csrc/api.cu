@@ -1,0 +1,76 @@
+// Host side of the C ABI: argument validation and dispatch by shape.  See include/q4.h.
+#include "q4_common.cuh"
+
+int q4_gemv_w4a16_launch(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
+                         int32_t* dev_status, cudaStream_t stream);
+int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_weight* w, void* y,
+                      int32_t out_dtype, int32_t* acc_dbg, bool int8_path, int32_t* dev_status,
+                      cudaStream_t stream);
+
+namespace {
+constexpr int kMaxGemvM = 4;
+
+int check_weight(const q4_weight* w, bool need_sym)
+{
+    if (!w || !w->packed || !w->scales) return Q4_ERR_NULL;
+    if (!w->symmetric && !w->zeros) return Q4_ERR_NULL;
+    if (w->n < 0 || w->k <= 0 || (w->group != 64 && w->group != 128) || w->k % w->group) return Q4_ERR_SHAPE;
+    if (need_sym && !w->symmetric) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(w->packed) || !q4_aligned16(w->scales) || (!w->symmetric && !q4_aligned16(w->zeros)))
+        return Q4_ERR_ALIGN;
+    return Q4_OK;
+}
+}  // namespace
+
+extern "C" const char* q4_status_string(int status)
+{
+    switch (status) {
+        case Q4_OK: return "ok";
+        case Q4_ERR_NULL: return "null pointer";
+        case Q4_ERR_SHAPE: return "bad shape";
+        case Q4_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case Q4_ERR_UNSUPPORTED: return "unsupported option";
+        case Q4_ERR_WORKSPACE: return "workspace too small";
+        case Q4_ERR_CUDA: return "CUDA error";
+        case Q4_ERR_NONFINITE: return "non-finite input or scale";
+        case Q4_ERR_TIMEOUT: return "bounded wait timed out";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int q4_version(void) { return 1; }
+
+extern "C" int q4_linear_w4a16_max_gemv_m(void) { return kMaxGemvM; }
+
+extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
+                               int32_t* dev_status, void* stream)
+{
+    int rc = check_weight(w, false);
+    if (rc) return rc;
+    if (!x || !y) return Q4_ERR_NULL;
+    if (m < 0) return Q4_ERR_SHAPE;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(x) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
+    if (m == 0 || w->n == 0) return Q4_OK;
+    if (m <= kMaxGemvM) {
+        if (w->k % 32 || w->k > 16384) return Q4_ERR_UNSUPPORTED;
+        return q4_gemv_w4a16_launch(x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
+    }
+    if (w->k % 128) return Q4_ERR_UNSUPPORTED;
+    return q4_gemm_tc_launch(x, nullptr, m, w, y, out_dtype, nullptr, false, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
+                              int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream)
+{
+    int rc = check_weight(w, true);
+    if (rc) return rc;
+    if (!xq || !scale_a || !y) return Q4_ERR_NULL;
+    if (m < 0) return Q4_ERR_SHAPE;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(xq) || !q4_aligned16(y) || ((uintptr_t)scale_a & 3u) || ((uintptr_t)acc_dbg & 3u))
+        return Q4_ERR_ALIGN;
+    if (m == 0 || w->n == 0) return Q4_OK;
+    if (w->k % 128) return Q4_ERR_UNSUPPORTED;
+    return q4_gemm_tc_launch(xq, scale_a, m, w, y, out_dtype, acc_dbg, true, dev_status, (cudaStream_t)stream);
+}

@@ -1,0 +1,204 @@
+"""Thin Python binding of the C ABI in include/q4.h (argument marshalling only).
+
+Every step of the computation runs in the CUDA library ``libq4.so``; this module only passes device
+pointers (``tensor.data_ptr()``), sizes and the current CUDA stream.  PyTorch provides device memory
+and streams.  There is no fallback: if the library is missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq4.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_linear_layers_b200.build_lib`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+Q4_OK = 0
+Q4_ERR_NULL = -1
+Q4_ERR_SHAPE = -2
+Q4_ERR_ALIGN = -3
+Q4_ERR_UNSUPPORTED = -4
+Q4_ERR_WORKSPACE = -5
+Q4_ERR_CUDA = -6
+Q4_ERR_NONFINITE = -7
+Q4_ERR_TIMEOUT = -8
+Q4_OUT_F32 = 0
+Q4_OUT_BF16 = 1
+
+EXPORTED = ("q4_status_string", "q4_version", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
+            "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward")
+
+
+class q4_weight(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("k", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("symmetric", ctypes.c_int32), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p)]
+
+
+_i32, _p, _sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+_lib.q4_status_string.restype = ctypes.c_char_p
+_lib.q4_status_string.argtypes = [ctypes.c_int]
+_lib.q4_version.restype = ctypes.c_int
+_lib.q4_linear_w4a16_max_gemv_m.restype = ctypes.c_int
+_lib.q4_quantize_pack.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p]
+_lib.q4_linear_w4a16.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p]
+_lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
+_lib.q4_linear_w4a8.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _p]
+_lib.moe_q4_workspace_size.restype = _sz
+_lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
+_lib.moe_q4_forward.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p, _i32,
+                                _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status} ({_lib.q4_status_string(status).decode()})")
+        self.status = status
+
+
+def _check(rc: int, what: str):
+    if rc != Q4_OK:
+        raise Q4Error(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def status_string(status: int) -> str:
+    return _lib.q4_status_string(status).decode()
+
+
+def version() -> int:
+    return _lib.q4_version()
+
+
+class Q4Weight:
+    """Device buffers of one INT4 weight matrix [n][k] plus its C descriptor."""
+
+    def __init__(self, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor | None, n: int, k: int,
+                 group: int, symmetric: bool):
+        self.packed, self.scales, self.zeros = packed, scales, zeros
+        self.n, self.k, self.group, self.symmetric = n, k, group, bool(symmetric)
+        self.desc = q4_weight(n, k, group, int(bool(symmetric)), packed.data_ptr(), scales.data_ptr(),
+                              zeros.data_ptr() if zeros is not None else None)
+
+    @staticmethod
+    def empty(n: int, k: int, group: int, symmetric: bool, device="cuda") -> "Q4Weight":
+        packed = torch.empty((n, k // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty((n, k // group), dtype=torch.float16, device=device)
+        zeros = None if symmetric else torch.empty((n, k // group), dtype=torch.float16, device=device)
+        return Q4Weight(packed, scales, zeros, n, k, group, symmetric)
+
+
+def q4_quantize_pack(w: torch.Tensor, group: int, symmetric: bool, dev_status: torch.Tensor | None = None,
+                     out: Q4Weight | None = None, stream=None) -> Q4Weight:
+    """RTN group quantization + packing of an fp32 [n][k] CUDA tensor."""
+    _dev(w, torch.float32, "w")
+    n, k = w.shape
+    q = out or Q4Weight.empty(n, k, group, symmetric, device=w.device)
+    _check(_lib.q4_quantize_pack(_ptr(w), n, k, group, int(bool(symmetric)), _ptr(q.packed), _ptr(q.scales),
+                                 _ptr(q.zeros), _ptr(dev_status), _stream(stream)), "q4_quantize_pack")
+    return q
+
+
+def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor."""
+    _dev(x, torch.bfloat16, "x")
+    m = x.numel() // w.k
+    if y is None:
+        y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
+           "q4_linear_w4a16")
+    return y
+
+
+def q4_linear_w4a16_max_gemv_m() -> int:
+    return _lib.q4_linear_w4a16_max_gemv_m()
+
+
+def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a: torch.Tensor | None = None,
+                        dev_status: torch.Tensor | None = None, stream=None):
+    """Per-token INT8 quantization of a bf16 [m][k] CUDA tensor -> (xq int8 [m][k], scale_a fp32 [m])."""
+    _dev(x, torch.bfloat16, "x")
+    m, k = x.shape
+    xq = torch.empty((m, k), dtype=torch.int8, device=x.device) if xq is None else xq
+    scale_a = torch.empty((m,), dtype=torch.float32, device=x.device) if scale_a is None else scale_a
+    _check(_lib.act_quant_per_token(_ptr(x), m, k, _ptr(xq), _ptr(scale_a), _ptr(dev_status), _stream(stream)),
+           "act_quant_per_token")
+    return xq, scale_a
+
+
+def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dtype=torch.float32,
+                   y: torch.Tensor | None = None, acc_dbg: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . code)_g; symmetric W."""
+    _dev(xq, torch.int8, "xq")
+    _dev(scale_a, torch.float32, "scale_a")
+    m = xq.shape[0]
+    if y is None:
+        y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
+                               _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
+    return y
+
+
+def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int) -> int:
+    return int(_lib.moe_q4_workspace_size(T, H, I, E, topk))
+
+
+def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                   experts: tuple, I: int, out_dtype=torch.float32, y: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, want_routing: bool = False,
+                   dev_status: torch.Tensor | None = None, stream=None):
+    """Top-k routed MoE SwiGLU layer with INT4 experts.  experts = (gate, up, down) Q4Weight, stacked by expert.
+    Returns y, or (y, topk_ids, topk_w, perm, offsets, counts) when want_routing."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    dev = x.device
+    if y is None:
+        y = torch.empty((T, H), dtype=out_dtype, device=dev)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    ws_bytes = moe_q4_workspace_size(T, H, I, E, topk)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    descs = (q4_weight * 3)(*[e.desc for e in experts])
+    ids = wts = perm = offs = cnts = None
+    if want_routing:
+        ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, topk), dtype=torch.float32, device=dev)
+        perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
+        offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+        cnts = torch.empty((E,), dtype=torch.int32, device=dev)
+    _check(_lib.moe_q4_forward(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, _ptr(y), od,
+                               _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts), _ptr(workspace),
+                               workspace.numel(), _ptr(dev_status), _stream(stream)), "moe_q4_forward")
+    if want_routing:
+        return y, ids, wts, perm, offs, cnts
+    return y

@@ -1,0 +1,87 @@
+"""The C ABI library loads, exports every function include/q4.h declares, and rejects bad arguments on
+the host before any CUDA call (no GPU needed: every call below returns before touching the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_linear_layers_b200 import q4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_exports_every_declared_function():
+    names = _declared_functions()
+    assert {"q4_quantize_pack", "q4_linear_w4a16", "act_quant_per_token", "q4_linear_w4a8",
+            "moe_q4_forward", "moe_q4_workspace_size"} <= set(names)
+    lib = ctypes.CDLL(q4.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(q4.EXPORTED)
+
+
+def test_status_strings():
+    assert q4.status_string(0) == "ok"
+    assert "aligned" in q4.status_string(q4.Q4_ERR_ALIGN)
+    assert q4.version() >= 1
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _w(n=128, k=256, group=64, sym=1, packed=FAKE, scales=FAKE, zeros=None):
+    return q4.q4_weight(n, k, group, sym, packed, scales, zeros)
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(w=None), q4.Q4_ERR_NULL),
+    (dict(w=_w(packed=None)), q4.Q4_ERR_NULL),
+    (dict(w=_w(sym=0, zeros=None)), q4.Q4_ERR_NULL),
+    (dict(w=_w(group=32)), q4.Q4_ERR_SHAPE),
+    (dict(w=_w(k=200)), q4.Q4_ERR_SHAPE),
+    (dict(w=_w(packed=FAKE + 4)), q4.Q4_ERR_ALIGN),
+    (dict(x=FAKE + 2), q4.Q4_ERR_ALIGN),
+    (dict(x=None), q4.Q4_ERR_NULL),
+    (dict(m=-1), q4.Q4_ERR_SHAPE),
+    (dict(out_dtype=7), q4.Q4_ERR_UNSUPPORTED),
+])
+def test_linear_w4a16_validation(args, expect):
+    a = dict(x=FAKE, m=1, w=_w(), y=FAKE, out_dtype=0)
+    a.update(args)
+    w = a["w"]
+    rc = q4._lib.q4_linear_w4a16(a["x"], a["m"], ctypes.byref(w) if w is not None else None, a["y"],
+                                 a["out_dtype"], None, None)
+    assert rc == expect
+
+
+def test_w4a8_needs_symmetric_weights():
+    w = _w(sym=0, zeros=FAKE)
+    rc = q4._lib.q4_linear_w4a8(FAKE, FAKE, 16, ctypes.byref(w), FAKE, 0, None, None, None)
+    assert rc == q4.Q4_ERR_UNSUPPORTED
+
+
+def test_quantize_validation():
+    L = q4._lib
+    assert L.q4_quantize_pack(None, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_NULL
+    assert L.q4_quantize_pack(FAKE, 4, 128, 48, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_quantize_pack(FAKE, 4, 100, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_quantize_pack(FAKE + 8, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_ALIGN
+    assert L.q4_quantize_pack(FAKE, 4, 128, 64, 0, FAKE, FAKE, None, None, None) == q4.Q4_ERR_NULL
+
+
+def test_act_quant_validation():
+    L = q4._lib
+    assert L.act_quant_per_token(None, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_NULL
+    assert L.act_quant_per_token(FAKE, 4, 12, FAKE, FAKE, None, None) == q4.Q4_ERR_SHAPE
+    assert L.act_quant_per_token(FAKE + 2, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_ALIGN

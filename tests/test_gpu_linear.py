@@ -1,0 +1,158 @@
+"""GPU parity: quantize/pack, W4A16 GEMV and per-token act-quant against the oracle, through the C ABI.
+
+Integer outputs (codes, packed bytes, scales, zeros, INT8 activations and their scales) must be
+bit-exact; floating outputs within max|err| <= 1e-2 * rms(reference) of the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_linear_layers_b200 import synth
+from tests._util import assert_close, bf16_rne, cpu_u16, cuda_u16_as, upload_weight
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from moe_linear_layers_b200 import q4 as mod
+    assert torch.cuda.is_available()
+    return mod
+
+
+# ---------------------------------------------------------------------------------------------- #
+# quantize + pack (bit-exact)
+# ---------------------------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("n,k,group,sym", [
+    (128, 256, 64, True),      # the tiny single-linear workload
+    (512, 2048, 128, False),   # k/v projection shape
+    (77, 384, 128, False),     # ragged row count, 3 groups
+    (3, 8192, 128, True),      # down projection width
+    (1, 64, 64, False),        # a single group
+    (8192, 2048, 128, False),  # a full gate projection
+])
+def test_quantize_bitexact(q4, n, k, group, sym):
+    W = synth.weights(("test", "quant", n, k, group, sym), n, k)
+    pk, sc, zr = oracle.quantize(W, group, sym)
+    qw = q4.q4_quantize_pack(torch.from_numpy(W).cuda(), group, sym)
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.packed.cpu().numpy(), pk)
+    assert np.array_equal(cpu_u16(qw.scales), sc)
+    if not sym:
+        assert np.array_equal(cpu_u16(qw.zeros), zr)
+
+
+def test_quantize_golden_and_edge_groups(q4):
+    """Zero groups, all-positive groups and exact ties run through the kernel too."""
+    W = np.zeros((4, 128), np.float32)
+    W[1, :64] = np.linspace(0.1, 3.0, 64, dtype=np.float32)
+    W[2] = np.repeat(np.array([1.75, -0.875, 0.5, 0.0], np.float32), 32)
+    W[3, 64:] = -0.25
+    for sym in (True, False):
+        pk, sc, zr = oracle.quantize(W, 64, sym)
+        qw = q4.q4_quantize_pack(torch.from_numpy(W).cuda(), 64, sym)
+        assert np.array_equal(qw.packed.cpu().numpy(), pk)
+        assert np.array_equal(cpu_u16(qw.scales), sc)
+        if not sym:
+            assert np.array_equal(cpu_u16(qw.zeros), zr)
+
+
+def test_quantize_nonfinite_sets_status(q4):
+    W = np.zeros((2, 128), np.float32)
+    W[1, 3] = np.inf
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.q4_quantize_pack(torch.from_numpy(W).cuda(), 64, True, dev_status=st)
+    assert int(st.item()) == q4.Q4_ERR_NONFINITE
+
+
+# ---------------------------------------------------------------------------------------------- #
+# W4A16 GEMV (m <= 4)
+# ---------------------------------------------------------------------------------------------- #
+
+def _gemv_case(q4, n, k, group, sym, m, tag, out=torch.float32):
+    W = synth.weights(("test", "gemv", tag, n, k), n, k)
+    pk, sc, zr = oracle.quantize(W, group, sym)
+    x = synth.activations(("test", "gemv-x", tag, m, k), m, k)
+    ref = oracle.linear_w4a16(x, pk, sc, zr, n, k, group, sym)
+    w = upload_weight(q4, pk, sc, zr, n, k, group, sym)
+    y = q4.q4_linear_w4a16(cuda_u16_as(x, torch.bfloat16), w, out_dtype=out)
+    torch.cuda.synchronize()
+    return y, ref, w, x
+
+
+def test_gemv_tiny_workload(q4):
+    """W fp32 128x256 N(0, 0.02) with 0.1% outliers x20, symmetric g64; x bf16 1x256; seed 0."""
+    W = synth.weights((0, "tiny-linear", "W"), 128, 256)
+    x = synth.activations((0, "tiny-linear", "x"), 1, 256)
+    pk, sc, zr = oracle.quantize(W, 64, True)
+    ref = oracle.linear_w4a16(x, pk, sc, zr, 128, 256, 64, True)
+    qw = q4.q4_quantize_pack(torch.from_numpy(W).cuda(), 64, True)   # the product path end to end
+    y = q4.q4_linear_w4a16(cuda_u16_as(x, torch.bfloat16), qw)
+    assert_close(y.cpu().numpy(), ref, what="tiny")
+
+
+@pytest.mark.parametrize("n,k,group,sym", [
+    (2048, 2048, 128, False), (512, 2048, 128, False), (8192, 2048, 128, False), (2048, 8192, 128, False),
+    (2048, 2048, 128, True), (77, 256, 64, False), (300, 16384, 128, True), (1000, 4096, 64, False),
+    (5, 1024, 128, True), (1, 32 * 64, 64, False),
+])
+def test_gemv_m1(q4, n, k, group, sym):
+    y, ref, *_ = _gemv_case(q4, n, k, group, sym, 1, "m1")
+    assert_close(y.cpu().numpy(), ref, what=f"gemv {n}x{k}")
+
+
+@pytest.mark.parametrize("m", [2, 3, 4])
+@pytest.mark.parametrize("n,k,group,sym", [(2048, 2048, 128, False), (333, 8192, 128, True), (64, 256, 64, False)])
+def test_gemv_small_m(q4, m, n, k, group, sym):
+    y, ref, *_ = _gemv_case(q4, n, k, group, sym, m, "sm")
+    assert_close(y.cpu().numpy(), ref, what=f"gemv m={m} {n}x{k}")
+
+
+def test_gemv_bf16_out_is_rounded_fp32(q4):
+    y32, ref, w, x = _gemv_case(q4, 1024, 2048, 128, False, 1, "bf16")
+    y16 = q4.q4_linear_w4a16(cuda_u16_as(x, torch.bfloat16), w, out_dtype=torch.bfloat16)
+    assert np.array_equal(cpu_u16(y16), bf16_rne(y32.cpu().numpy()))
+
+
+def test_gemv_nonfinite_x_sets_status(q4):
+    W = synth.weights(("test", "nan"), 64, 256)
+    pk, sc, zr = oracle.quantize(W, 64, True)
+    w = upload_weight(q4, pk, sc, zr, 64, 256, 64, True)
+    x = torch.zeros((1, 256), dtype=torch.bfloat16, device="cuda")
+    x[0, 17] = float("nan")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.q4_linear_w4a16(x, w, dev_status=st)
+    assert int(st.item()) == q4.Q4_ERR_NONFINITE
+
+
+# ---------------------------------------------------------------------------------------------- #
+# per-token INT8 activation quantization (bit-exact)
+# ---------------------------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("m,k", [(16, 2048), (256, 8192), (7, 24), (4096, 2048), (1, 8)])
+def test_act_quant_bitexact(q4, m, k):
+    x = synth.activations(("test", "aq", m, k), m, k, "student_t3")
+    if m > 2:
+        x[1] = 0           # an all-zero token
+        x[2, : k // 2] = 0
+    q_ref, s_ref = oracle.act_quant(x, k)
+    xq, s = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+
+
+def test_act_quant_golden_rows(q4):
+    x = synth.to_bf16_bits(np.array([[127, -63.5, 0.5, 2, 0, 0, 0, 0], [-127, 2.5, -2.5, 1.5, 0, 0, 0, 0]], np.float32))
+    xq, s = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
+    assert s.cpu().tolist() == [1.0, 1.0]
+    assert xq.cpu().numpy()[:, :4].tolist() == [[127, -64, 0, 2], [-127, 2, -2, 2]]
+
+
+def test_act_quant_nonfinite_sets_status(q4):
+    x = torch.ones((3, 64), dtype=torch.bfloat16, device="cuda")
+    x[2, 5] = float("inf")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.act_quant_per_token(x, dev_status=st)
+    assert int(st.item()) == q4.Q4_ERR_NONFINITE
