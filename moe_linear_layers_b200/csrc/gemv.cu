@@ -119,6 +119,18 @@ __device__ __forceinline__ void load_x_chunk(const uint16_t* xc, float p, __half
     }
 }
 
+// Programmatic dependent launch: let the next kernel on the stream start launching, and wait for the
+// previous one (its writes become visible) only before reading data it may produce.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Bring a contiguous byte range into L2 (a hint: it neither reads into registers nor can it observe
+// stale data, L2 being the device's point of coherence).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 template <int KSPLIT, int J, int ROWS, bool SYM>
 __global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_m1_kernel(GemvParams p)
 {
@@ -128,26 +140,70 @@ __global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_m1_kernel(GemvParams p
     const int team = warp / KSPLIT, wit = warp % KSPLIT;
     const int C = p.k / 32, ng = p.k / p.group, cpg = p.group / 32;
     const int64_t rowbytes = p.k / 2;
+    const int rows_per_cta = TEAMS * ROWS;
+    const int64_t stride = (int64_t)gridDim.x * rows_per_cta;
 
-    const float amax = block_amax(p.x, p.k, p.status, red);
-    const float ps = prescale_for(amax);
-    const float inv_ps = 1.0f / ps;
+    pdl_launch_dependents();
+    // The weights do not depend on the previous kernel: start pulling this CTA's rows into L2 now.
+    if (threadIdx.x == 0) {
+        for (int64_t rb = (int64_t)blockIdx.x * rows_per_cta; rb < p.n; rb += stride) {
+            const int64_t rows = min((int64_t)rows_per_cta, (int64_t)p.n - rb);
+            prefetch_l2(p.packed + rb * rowbytes, (uint32_t)(rows * rowbytes));
+        }
+    }
+    pdl_wait();
 
     int cidx[J];
     bool cval[J];
-    __half2 X[J][16];
+    uint4 xraw[J][4];
+    float amax = 0.0f;
+    bool finite = true;
 #pragma unroll
     for (int j = 0; j < J; j++) {
         cidx[j] = wit * 32 * J + 32 * j + lane;
         cval[j] = cidx[j] < C;
-        if (cval[j]) load_x_chunk(p.x + 32 * cidx[j], ps, X[j]);
-        else {
 #pragma unroll
-            for (int i = 0; i < 16; i++) X[j][i] = __float2half2_rn(0.0f);
+        for (int w = 0; w < 4; w++) {
+            xraw[j][w] = cval[j] ? __ldg(reinterpret_cast<const uint4*>(p.x + 32 * cidx[j]) + w) : make_uint4(0, 0, 0, 0);
+            const uint32_t e[4] = {xraw[j][w].x, xraw[j][w].y, xraw[j][w].z, xraw[j][w].w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float a = __uint_as_float(e[i] << 16), b = __uint_as_float(e[i] & 0xFFFF0000u);
+                finite &= isfinite(a) && isfinite(b);
+                amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+            }
+        }
+    }
+    if (!finite) q4_set_status(p.status, Q4_ERR_NONFINITE);
+    // every team covers the whole row of x, so the block max over all warps is max|x|
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kWarps; i++) amax = fmaxf(amax, red[i]);
+    __syncthreads();
+    const float ps = prescale_for(amax);
+    const float inv_ps = 1.0f / ps;
+
+    __half2 X[J][16];
+#pragma unroll
+    for (int j = 0; j < J; j++) {
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            const uint32_t e[4] = {xraw[j][w].x, xraw[j][w].y, xraw[j][w].z, xraw[j][w].w};
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                f[2 * i] = __uint_as_float(e[i] << 16) * ps;
+                f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * ps;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; q++) X[j][4 * w + q] = __floats2half2_rn(f[q], f[q + 4]);
         }
     }
 
-    const int rows_per_cta = TEAMS * ROWS;
     // Row block in flight: the next block is fetched into (nw, ns, nz) while (cw, cs, cz) is used.
     uint4 cw[ROWS][J], nw[ROWS][J];
     __half cs[ROWS][J], ns[ROWS][J], cz[ROWS][J], nz[ROWS][J];
@@ -171,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_m1_kernel(GemvParams p
         }
     };
 
-    const int64_t stride = (int64_t)gridDim.x * rows_per_cta;
     int64_t rb = (int64_t)blockIdx.x * rows_per_cta;
     if (rb < p.n) fetch(cw, cs, cz, rb);
     for (; rb < p.n; rb += stride) {
@@ -342,12 +397,24 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_small_m_kernel(GemvPar
     }
 }
 
+// Launched with programmatic stream serialization: the kernel may begin (and prefetch weights into
+// L2) while the previous kernel on the stream drains; it reads x only after griddepcontrol.wait.
 template <int KSPLIT, int J, int ROWS>
 int launch_m1(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
 {
-    if (symmetric) w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, true><<<grid, kThreads, 0, s>>>(p);
-    else w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, false><<<grid, kThreads, 0, s>>>(p);
-    return q4_launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = symmetric ? cudaLaunchKernelEx(&cfg, w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, true>, p)
+                              : cudaLaunchKernelEx(&cfg, w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, false>, p);
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
 template <int KSPLIT, int J>
@@ -356,7 +423,9 @@ int launch_m1_rows(const GemvParams& p, int symmetric, cudaStream_t s)
     constexpr int TEAMS = kWarps / KSPLIT;
     const int64_t target = (int64_t)q4_num_sms() * 2;  // two resident CTAs per SM
     auto ctas = [&](int rows) { return ((int64_t)p.n + TEAMS * rows - 1) / (TEAMS * rows); };
-    if (ctas(4) >= target) return launch_m1<KSPLIT, J, 4>(p, symmetric, (int)std::min<int64_t>(ctas(4), target), s);
+    // four rows in flight only with one chunk per lane (two chunks x four rows exceed 128 registers)
+    if constexpr (J == 1)
+        if (ctas(4) >= target) return launch_m1<KSPLIT, J, 4>(p, symmetric, (int)std::min<int64_t>(ctas(4), target), s);
     if (ctas(2) >= target) return launch_m1<KSPLIT, J, 2>(p, symmetric, (int)std::min<int64_t>(ctas(2), target), s);
     return launch_m1<KSPLIT, J, 1>(p, symmetric, (int)std::min<int64_t>(ctas(1), target), s);
 }
@@ -368,7 +437,8 @@ int launch_small(const GemvParams& p, int symmetric, cudaStream_t s)
     const size_t smem = (size_t)MT * p.k * 2;
     const int grid = (int)std::min<int64_t>(((int64_t)p.n + TEAMS - 1) / TEAMS, (int64_t)q4_num_sms());
     auto kern = symmetric ? w4a16_gemv_small_m_kernel<KSPLIT, J, MT, true> : w4a16_gemv_small_m_kernel<KSPLIT, J, MT, false>;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (smem > 200 * 1024) return Q4_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return Q4_ERR_CUDA;
     kern<<<grid, kThreads, smem, s>>>(p);
     return q4_launch_status();

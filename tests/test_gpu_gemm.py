@@ -1,0 +1,99 @@
+"""GPU parity of the tcgen05 tensor-core GEMMs (W4A16 bf16 MMA, W4A8 int8 MMA) against the oracle.
+
+Floating outputs: max|err| <= 1e-2 * rms(fp64 oracle).  bf16 outputs equal the round-to-nearest-even of
+the fp32 outputs bit for bit.  W4A8's per-group INT32 partials (debug output) are bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_linear_layers_b200 import synth
+from tests._util import assert_close, bf16_rne, cpu_u16, cuda_u16_as, upload_weight
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from moe_linear_layers_b200 import q4 as mod
+    return mod
+
+
+def _w4a16(q4, m, n, k, group, sym, kind="normal", tag="", rows_m=None):
+    W = synth.weights(("test", "gemm", tag, n, k, group, sym), n, k)
+    pk, sc, zr = oracle.quantize(W, group, sym)
+    x = synth.activations(("test", "gemm-x", tag, m, k), m, k, kind)
+    ref = oracle.linear_w4a16(x, pk, sc, zr, n, k, group, sym, rows_m=rows_m)
+    w = upload_weight(q4, pk, sc, zr, n, k, group, sym)
+    xd = cuda_u16_as(x, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.q4_linear_w4a16(xd, w, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    yn = y.cpu().numpy()
+    if rows_m is not None:
+        yn = yn[rows_m]
+    return yn, ref, w, xd, y
+
+
+def test_w4a16_single_tile(q4):
+    yn, ref, *_ = _w4a16(q4, 128, 128, 128, 128, False, tag="tile")
+    assert_close(yn, ref, what="one tile")
+
+
+@pytest.mark.parametrize("m,n,k,group,sym", [
+    (5, 128, 128, 128, True),          # smallest m on the tensor-core path, one tile
+    (64, 2048, 2048, 128, False),      # prefill m=64
+    (200, 333, 256, 64, False),        # ragged m and n, group 64
+    (130, 1000, 2048, 128, True),      # ragged, symmetric
+    (512, 512, 8192, 128, False),      # long K (64 groups)
+    (256, 8192, 2048, 128, False),     # many n tiles
+    (1024, 256, 1024, 64, True),
+])
+def test_w4a16_gemm(q4, m, n, k, group, sym):
+    yn, ref, *_ = _w4a16(q4, m, n, k, group, sym, tag="g")
+    assert_close(yn, ref, what=f"w4a16 {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(512, 2048, 2048), (2048, 2048, 8192)])
+def test_w4a16_prefill_outlier_channels(q4, m, n, k):
+    """Prefill shapes with 1% of activation channels x10; sampled rows of the oracle at full size."""
+    rows = np.arange(0, m, max(1, m // 48))
+    yn, ref, w, xd, y = _w4a16(q4, m, n, k, 128, False, kind="outlier_channels", tag="pre", rows_m=rows)
+    assert_close(yn, ref, what=f"prefill {m}x{n}x{k}")
+    y16 = q4.q4_linear_w4a16(xd, w, out_dtype=torch.bfloat16)
+    assert np.array_equal(cpu_u16(y16), bf16_rne(y.cpu().numpy()))
+
+
+def _w4a8(q4, m, n, k, group, tag, want_acc=False):
+    W = synth.weights(("test", "w4a8", tag, n, k, group), n, k)
+    pk, sc, _ = oracle.quantize(W, group, True)
+    x = synth.activations(("test", "w4a8-x", tag, m, k), m, k, "student_t3")
+    xq_ref, sa_ref = oracle.act_quant(x, k)
+    w = upload_weight(q4, pk, sc, None, n, k, group, True)
+    xq, sa = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
+    acc = torch.zeros((m, n, k // group), dtype=torch.int32, device="cuda") if want_acc else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.q4_linear_w4a8(xq, sa, w, acc_dbg=acc, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    return y, acc, (xq_ref, sa_ref, pk, sc), w, xq, sa
+
+
+@pytest.mark.parametrize("m,n,k,group", [(16, 128, 128, 128), (130, 333, 512, 128), (64, 256, 256, 64)])
+def test_w4a8_int32_partials_bitexact(q4, m, n, k, group):
+    y, acc, (xq, sa, pk, sc), *_ = _w4a8(q4, m, n, k, group, "acc", want_acc=True)
+    ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_close(y.cpu().numpy(), ref, what="w4a8")
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 2048, 2048), (256, 8192, 2048), (4096, 2048, 8192), (4096, 512, 2048)])
+def test_w4a8_workload_shapes(q4, m, n, k):
+    y, _, (xq, sa, pk, sc), w, xqd, sad = _w4a8(q4, m, n, k, 128, "shape")
+    rows = np.arange(0, m, max(1, m // 32))
+    ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, 128, rows_m=rows)
+    assert_close(y.cpu().numpy()[rows], ref, what=f"w4a8 {m}x{n}x{k}")
+    y16 = q4.q4_linear_w4a8(xqd, sad, w, out_dtype=torch.bfloat16)
+    assert np.array_equal(cpu_u16(y16), bf16_rne(y.cpu().numpy()))
