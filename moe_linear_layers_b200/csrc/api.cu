@@ -52,9 +52,9 @@ extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w,
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(x) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
     if (m == 0 || w->n == 0) return Q4_OK;
-    if (m <= kMaxGemvM) {
-        if (w->k % 32 || w->k > 16384) return Q4_ERR_UNSUPPORTED;
-        return q4_gemv_w4a16_launch(x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
+    if (m <= kMaxGemvM && w->k % 32 == 0) {
+        const int rc = q4_gemv_w4a16_launch(x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
+        if (rc != Q4_ERR_UNSUPPORTED) return rc;  // shapes the GEMV cannot stage go to the GEMM
     }
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
     return q4_gemm_tc_launch(x, nullptr, m, w, y, out_dtype, nullptr, false, dev_status, (cudaStream_t)stream);

@@ -3,26 +3,34 @@
 // Source: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" §2.1 (4-bit storage restored to a
 // 16-bit type before the multiply) and §1 (small model, small batch: memory bound).
 //
-// Design (HBM-bound; the packed weights are streamed once):
-//  * a warp walks weight rows; lane l owns 16-byte chunks (32 codes) at fixed k positions, so its
-//    slice of x stays in registers (m == 1) or is read from shared memory (m > 1) for every row;
-//  * loads are 128-bit ld.global.nc, coalesced (a warp reads 512 contiguous bytes of a row), with
-//    the next row block prefetched while the current one is computed;
-//  * dequant in registers: one LOP3 turns two nibbles into an fp16x2 "1024 + code" (the exponent
-//    of 1024 makes the code the low mantissa bits); an HSUB2 of (1024 + zero) leaves the exact
-//    integer (code - zero) in fp16; nibbles 1, 3, 5, 7 of a word are used in place (16 * code) and
-//    accumulate separately, scaled by 1/16 once per chunk;
-//  * products accumulate in fp16x2 over one chunk (8 per half) and then in fp32, scaled by the
-//    group scale once per chunk; x is pre-scaled by a power of two so |x| < 2 (exact), which keeps
-//    every fp16 partial far from overflow;
-//  * rows that need more than 64 chunks (k > 2048) are split over a team of 2..8 warps, reduced
-//    through shared memory.
+// HBM-bound design (the packed weights are streamed exactly once):
+//  * persistent CTAs, one per SM, each owning a contiguous block of weight rows;
+//  * a producer thread streams the block through a 5-stage shared-memory ring with cp.async.bulk
+//    (16 KB per stage: whole rows are contiguous in memory), completion tracked by mbarriers, so
+//    ~80 KB per SM are in flight without any register-held loads;
+//  * programmatic dependent launch: the CTA pulls its rows into L2 (a coherent prefetch) before it
+//    waits for the previous kernel on the stream, so consecutive GEMVs keep HBM busy across the
+//    kernel boundary; x (which the previous kernel may produce) is read only after the wait;
+//  * x is converted once per CTA into fp16 pairs (power-of-two prescale so max|x| < 2, exact) and
+//    held in registers by the lanes that use it;
+//  * in-register dequant: one LOP3 turns two nibbles into fp16x2 "1024 + code"; an HSUB2 of
+//    (1024 + zero) leaves the exact integer (code - zero); nibbles 1, 3, 5, 7 of a word are used in
+//    place (16 * code) and accumulate separately (scaled by 1/16 once per chunk); products accumulate
+//    in fp16x2 over one 32-code chunk (8 products per half) and then in fp32 times the group scale;
+//  * lanes split a row into 16-byte chunks (coalesced, bank-conflict-free shared reads); rows longer
+//    than 2048 codes are split over 2..8 warps and combined through shared memory.
 #include "q4_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kComputeWarps = 16;
+constexpr int kComputeThreads = kComputeWarps * 32;
+constexpr int kThreads = kComputeThreads + 32;      // + one producer warp
+constexpr int kStageBytes = 16384;
+constexpr int kStages = 5;
+constexpr int kScaleBytes = 16384;                  // the CTA's scales (+ zeros) in shared memory
+constexpr int kMaxM = 4;
 
 struct GemvParams {
     const uint16_t* x;
@@ -32,10 +40,12 @@ struct GemvParams {
     void* y;
     int32_t* status;
     int m, n, k, group, out_bf16;
+    int rows_per_cta;    // contiguous weight rows per CTA
+    int rows_per_stage;  // rows per 16 KB stage
 };
 
-// Nibble -> fp16x2 magic: (u & mask) ^ key, key = 0x6400 (1024.0) in both halves, plus the sign
-// flip 8 of symmetric codes (two's complement -> offset binary: c + 8 = nibble ^ 8).
+// Nibble -> fp16x2 magic: (u & mask) ^ key, key = 0x6400 (1024.0) in both halves, plus the flip of
+// bit 3 of symmetric codes (two's complement -> offset binary: code + 8 = nibble ^ 8).
 template <bool SYM> struct Keys;
 template <> struct Keys<true> {
     static constexpr uint32_t k1 = 0x64006400u ^ 0x00080008u, k16 = 0x64006400u ^ 0x00800080u;
@@ -43,6 +53,37 @@ template <> struct Keys<true> {
 template <> struct Keys<false> {
     static constexpr uint32_t k1 = 0x64006400u, k16 = 0x64006400u;
 };
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Bring a byte range into L2 (coherent: it cannot observe stale data).  Needs 16-byte alignment.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2_range(const uint8_t* lo, const uint8_t* hi)
+{
+    const uintptr_t a = ((uintptr_t)lo + 15) & ~(uintptr_t)15, b = (uintptr_t)hi & ~(uintptr_t)15;
+    for (uintptr_t q = a; q < b; q += 65536) prefetch_l2((const void*)q, (uint32_t)min((uintptr_t)65536, b - q));
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory"); }
+
+__device__ __forceinline__ uint4 lds128(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(tc::smem_u32(p)));
+    return v;
+}
 
 // Power-of-two prescale p with max|x| * p in [1, 2): exact, and every fp16 partial stays small.
 __device__ __forceinline__ float prescale_for(float amax)
@@ -53,119 +94,91 @@ __device__ __forceinline__ float prescale_for(float amax)
     return ldexpf(1.0f, 1 - e);
 }
 
-// Block-wide max of |x| over one token row; also flags non-finite values.
-__device__ float block_amax(const uint16_t* xr, int k, int32_t* status, float* red)
-{
-    float a = 0.0f;
-    bool finite = true;
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        float v = bf16_bits_to_float(xr[i]);
-        finite &= isfinite(v);
-        a = fmaxf(a, fabsf(v));
-    }
-    if (!finite) q4_set_status(status, Q4_ERR_NONFINITE);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = a;
-    __syncthreads();
-    float r = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kWarps; i++) r = fmaxf(r, red[i]);
-    return r;
-}
-
-// One chunk (32 codes) against the x pairs of that chunk; returns the fp32 dot product of
-// (code - zero) and the pre-scaled x (not yet multiplied by the group scale).
+// The 8 codes of one 32-bit word against the x pairs of that word.
+// X = {(x0,x4), (x1,x5), (x2,x6), (x3,x7)} as half2 bit patterns.
 template <bool SYM>
-__device__ __forceinline__ float chunk_dot(const uint4& wv, __half2 bias1, __half2 bias16, const __half2 (&X)[16])
+__device__ __forceinline__ void word_dot(uint32_t u, __half2 b1, __half2 b16, const uint4& X, __half2& acc1,
+                                         __half2& acc16)
 {
-    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-    __half2 acc1 = __float2half2_rn(0.0f), acc16 = __float2half2_rn(0.0f);
-#pragma unroll
-    for (int w = 0; w < 4; w++) {
-        const uint32_t u = words[w], u8 = u >> 8;
-        const __half2 d0 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x000F000Fu, Keys<SYM>::k1)), bias1);
-        const __half2 d1 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x00F000F0u, Keys<SYM>::k16)), bias16);
-        const __half2 d2 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x000F000Fu, Keys<SYM>::k1)), bias1);
-        const __half2 d3 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x00F000F0u, Keys<SYM>::k16)), bias16);
-        acc1 = __hfma2(d0, X[4 * w + 0], acc1);
-        acc16 = __hfma2(d1, X[4 * w + 1], acc16);
-        acc1 = __hfma2(d2, X[4 * w + 2], acc1);
-        acc16 = __hfma2(d3, X[4 * w + 3], acc16);
-    }
-    const float2 f1 = __half22float2(acc1), f16 = __half22float2(acc16);
-    return (f1.x + f1.y) + 0.0625f * (f16.x + f16.y);
+    const uint32_t u8 = u >> 8;
+    const __half2 d0 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x000F000Fu, Keys<SYM>::k1)), b1);
+    const __half2 d1 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x00F000F0u, Keys<SYM>::k16)), b16);
+    const __half2 d2 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x000F000Fu, Keys<SYM>::k1)), b1);
+    const __half2 d3 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x00F000F0u, Keys<SYM>::k16)), b16);
+    acc1 = __hfma2(d0, u32_as_h2(X.x), acc1);
+    acc16 = __hfma2(d1, u32_as_h2(X.y), acc16);
+    acc1 = __hfma2(d2, u32_as_h2(X.z), acc1);
+    acc16 = __hfma2(d3, u32_as_h2(X.w), acc16);
 }
 
-// x pairs of one chunk in the order chunk_dot consumes them: for word w,
-// X[4w+0] = (x[8w], x[8w+4]), X[4w+1] = (x[8w+1], x[8w+5]), X[4w+2] = (x[8w+2], x[8w+6]),
-// X[4w+3] = (x[8w+3], x[8w+7]); each value times the power-of-two prescale p.
-__device__ __forceinline__ void load_x_chunk(const uint16_t* xc, float p, __half2 (&X)[16])
+__device__ __forceinline__ float fold(__half2 acc1, __half2 acc16)
 {
-    const uint4* v = reinterpret_cast<const uint4*>(xc);
-#pragma unroll
-    for (int w = 0; w < 4; w++) {
-        const uint4 q = __ldg(v + w);
-        const uint32_t e[4] = {q.x, q.y, q.z, q.w};
-        float f[8];
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            f[2 * i] = __uint_as_float(e[i] << 16) * p;
-            f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * p;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; j++) X[4 * w + j] = __floats2half2_rn(f[j], f[j + 4]);
-    }
+    const float2 f = __half22float2(__hfma2(acc16, __float2half2_rn(0.0625f), acc1));
+    return f.x + f.y;
 }
 
-// Programmatic dependent launch: let the next kernel on the stream start launching, and wait for the
-// previous one (its writes become visible) only before reading data it may produce.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// Bring a contiguous byte range into L2 (a hint: it neither reads into registers nor can it observe
-// stale data, L2 being the device's point of coherence).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
+template <int KSPLIT, int J, int MT, bool SYM>
+__global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
 {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-template <int KSPLIT, int J, int ROWS, bool SYM>
-__global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_m1_kernel(GemvParams p)
-{
-    constexpr int TEAMS = kWarps / KSPLIT;
-    __shared__ float red[kWarps * ROWS];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-    const int team = warp / KSPLIT, wit = warp % KSPLIT;
+    constexpr int TEAMS = kComputeWarps / KSPLIT;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* stages = smem;                                                   // kStages x kStageBytes
+    uint4* xs = reinterpret_cast<uint4*>(smem + kStages * kStageBytes);       // [MT][4][C] x pairs
     const int C = p.k / 32, ng = p.k / p.group, cpg = p.group / 32;
-    const int64_t rowbytes = p.k / 2;
-    const int rows_per_cta = TEAMS * ROWS;
-    const int64_t stride = (int64_t)gridDim.x * rows_per_cta;
+    __half* ssc = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(xs) + (size_t)MT * p.k * 2);
+    __half* szr = ssc + p.rows_per_cta * ng;
+    float* red = reinterpret_cast<float*>(smem + kStages * kStageBytes + (size_t)MT * p.k * 2 + kScaleBytes);
+    float* pscale = red + 2 * 16 * kMaxM;
+    uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * 16 * kMaxM + 8 * kMaxM);
+    uint64_t* empty = full + kStages;
 
-    pdl_launch_dependents();
-    // The weights do not depend on the previous kernel: start pulling this CTA's rows into L2 now.
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int64_t rowbytes = p.k / 2;
+    const int r0 = blockIdx.x * p.rows_per_cta;
+    const int r1 = min(p.n, r0 + p.rows_per_cta);
+    const int nstages = (r1 - r0 + p.rows_per_stage - 1) / p.rows_per_stage;
+
     if (threadIdx.x == 0) {
-        for (int64_t rb = (int64_t)blockIdx.x * rows_per_cta; rb < p.n; rb += stride) {
-            const int64_t rows = min((int64_t)rows_per_cta, (int64_t)p.n - rb);
-            prefetch_l2(p.packed + rb * rowbytes, (uint32_t)(rows * rowbytes));
-        }
+        for (int i = 0; i < kStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kComputeWarps); }
+        tc::fence_mbar_init();
     }
+    if (warp == kComputeWarps && lane == 0 && r0 < r1) {
+        // weights do not depend on the previous kernel: start pulling them into L2 now
+        prefetch_l2_range(p.packed + (int64_t)r0 * rowbytes, p.packed + (int64_t)r1 * rowbytes);
+        prefetch_l2_range(reinterpret_cast<const uint8_t*>(p.scales + (int64_t)r0 * ng),
+                          reinterpret_cast<const uint8_t*>(p.scales + (int64_t)r1 * ng));
+        if constexpr (!SYM)
+            prefetch_l2_range(reinterpret_cast<const uint8_t*>(p.zeros + (int64_t)r0 * ng),
+                              reinterpret_cast<const uint8_t*>(p.zeros + (int64_t)r1 * ng));
+    }
+    __syncthreads();
+    pdl_launch_dependents();
     pdl_wait();
 
-    int cidx[J];
-    bool cval[J];
-    uint4 xraw[J][4];
-    float amax = 0.0f;
-    bool finite = true;
-#pragma unroll
-    for (int j = 0; j < J; j++) {
-        cidx[j] = wit * 32 * J + 32 * j + lane;
-        cval[j] = cidx[j] < C;
-#pragma unroll
-        for (int w = 0; w < 4; w++) {
-            xraw[j][w] = cval[j] ? __ldg(reinterpret_cast<const uint4*>(p.x + 32 * cidx[j]) + w) : make_uint4(0, 0, 0, 0);
-            const uint32_t e[4] = {xraw[j][w].x, xraw[j][w].y, xraw[j][w].z, xraw[j][w].w};
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            for (int st = 0; st < nstages; st++) {
+                const int s = st % kStages;
+                if (!tc::mbar_wait(&empty[s], ((st / kStages) & 1) ^ 1, p.status, nullptr)) break;
+                const int rs = r0 + st * p.rows_per_stage;
+                const uint32_t bytes = (uint32_t)(min(p.rows_per_stage, r1 - rs) * rowbytes);
+                tc::mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_g2s(stages + s * kStageBytes, p.packed + (int64_t)rs * rowbytes, bytes, &full[s]);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------------- compute warps
+    // x -> fp16 pairs with a power-of-two prescale per token; the CTA's scales and zeros -> smem
+    for (int mm = 0; mm < MT; mm++) {
+        const uint4* xr = reinterpret_cast<const uint4*>(p.x + (int64_t)mm * p.k);
+        float amax = 0.0f;
+        bool finite = true;
+        for (int u = threadIdx.x; u < p.k / 8; u += kComputeThreads) {
+            const uint4 v = __ldg(xr + u);
+            const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 const float a = __uint_as_float(e[i] << 16), b = __uint_as_float(e[i] & 0xFFFF0000u);
@@ -173,303 +186,179 @@ __global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_m1_kernel(GemvParams p
                 amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
             }
         }
-    }
-    if (!finite) q4_set_status(p.status, Q4_ERR_NONFINITE);
-    // every team covers the whole row of x, so the block max over all warps is max|x|
+        if (!finite) q4_set_status(p.status, Q4_ERR_NONFINITE);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kWarps; i++) amax = fmaxf(amax, red[i]);
-    __syncthreads();
-    const float ps = prescale_for(amax);
-    const float inv_ps = 1.0f / ps;
-
-    __half2 X[J][16];
-#pragma unroll
-    for (int j = 0; j < J; j++) {
-#pragma unroll
-        for (int w = 0; w < 4; w++) {
-            const uint32_t e[4] = {xraw[j][w].x, xraw[j][w].y, xraw[j][w].z, xraw[j][w].w};
+        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) red[warp] = amax;
+        compute_bar();
+        if (threadIdx.x == 0) {
+            float a = 0.0f;
+            for (int i = 0; i < kComputeWarps; i++) a = fmaxf(a, red[i]);
+            pscale[mm] = prescale_for(a);
+        }
+        compute_bar();
+        const float ps = pscale[mm];
+        for (int u = threadIdx.x; u < p.k / 8; u += kComputeThreads) {
+            const uint4 v = __ldg(xr + u);
+            const uint32_t e[4] = {v.x, v.y, v.z, v.w};
             float f[8];
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 f[2 * i] = __uint_as_float(e[i] << 16) * ps;
                 f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * ps;
             }
-#pragma unroll
-            for (int q = 0; q < 4; q++) X[j][4 * w + q] = __floats2half2_rn(f[q], f[q + 4]);
+            uint4 o;
+            o.x = h2_as_u32(__floats2half2_rn(f[0], f[4]));
+            o.y = h2_as_u32(__floats2half2_rn(f[1], f[5]));
+            o.z = h2_as_u32(__floats2half2_rn(f[2], f[6]));
+            o.w = h2_as_u32(__floats2half2_rn(f[3], f[7]));
+            xs[((int64_t)mm * 4 + (u & 3)) * C + (u >> 2)] = o;   // word u&3 of chunk u>>2
         }
     }
+    for (int i = threadIdx.x; i < (r1 - r0) * ng; i += kComputeThreads) {
+        ssc[i] = p.scales[(int64_t)r0 * ng + i];
+        if constexpr (!SYM) szr[i] = p.zeros[(int64_t)r0 * ng + i];
+    }
+    compute_bar();
 
-    // Row block in flight: the next block is fetched into (nw, ns, nz) while (cw, cs, cz) is used.
-    uint4 cw[ROWS][J], nw[ROWS][J];
-    __half cs[ROWS][J], ns[ROWS][J], cz[ROWS][J], nz[ROWS][J];
-    auto fetch = [&](uint4 (&wv)[ROWS][J], __half (&sc)[ROWS][J], __half (&zc)[ROWS][J], int64_t rb) {
+    const int team = warp / KSPLIT, ks = warp % KSPLIT;
+    int cidx[J];
+    uint4 X[J][4];
 #pragma unroll
-        for (int rr = 0; rr < ROWS; rr++) {
-            const int64_t r = rb + team * ROWS + rr;
+    for (int j = 0; j < J; j++) {
+        cidx[j] = ks * 32 * J + 32 * j + lane;
+#pragma unroll
+        for (int w = 0; w < 4; w++)
+            X[j][w] = (MT == 1 && cidx[j] < C) ? xs[(int64_t)w * C + cidx[j]] : make_uint4(0, 0, 0, 0);
+    }
+
+    for (int st = 0; st < nstages; st++) {
+        const int s = st % kStages;
+        const int rs = r0 + st * p.rows_per_stage;
+        const int rows_here = min(p.rows_per_stage, r1 - rs);
+        if (!tc::mbar_wait(&full[s], (st / kStages) & 1, p.status, nullptr)) break;
+        const uint8_t* sbase = stages + s * kStageBytes;
+        float* redb = red + (st & 1) * 16 * kMaxM;
+        for (int rr = team; rr < rows_here; rr += TEAMS) {
+            const int row = rs + rr;
+            const int lrow = row - r0;
+            float part[MT];
+#pragma unroll
+            for (int mm = 0; mm < MT; mm++) part[mm] = 0.0f;
 #pragma unroll
             for (int j = 0; j < J; j++) {
-                if (r < p.n && cval[j]) {
-                    wv[rr][j] = ldg_nc_v4(p.packed + r * rowbytes + (int64_t)cidx[j] * 16);
-                    const int64_t gi = r * ng + cidx[j] / cpg;
-                    sc[rr][j] = p.scales[gi];
-                    zc[rr][j] = SYM ? __float2half_rn(8.0f) : p.zeros[gi];
-                } else {
-                    wv[rr][j] = make_uint4(0, 0, 0, 0);
-                    sc[rr][j] = __float2half_rn(0.0f);
-                    zc[rr][j] = __float2half_rn(0.0f);
+                const int c = cidx[j];
+                if (c < C) {
+                    const uint4 wv = lds128(sbase + rr * rowbytes + c * 16);
+                    const int gidx = lrow * ng + c / cpg;
+                    const float sc = __half2float(ssc[gidx]);
+                    __half2 b1, b16;
+                    if constexpr (SYM) {
+                        b1 = __float2half2_rn(1032.0f);
+                        b16 = __float2half2_rn(1152.0f);
+                    } else {
+                        const __half z = szr[gidx];
+                        b1 = __half2half2(__hadd(z, __float2half_rn(1024.0f)));
+                        b16 = __half2half2(__hfma(z, __float2half_rn(16.0f), __float2half_rn(1024.0f)));
+                    }
+                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int mm = 0; mm < MT; mm++) {
+                        __half2 acc1 = __float2half2_rn(0.0f), acc16 = __float2half2_rn(0.0f);
+#pragma unroll
+                        for (int w = 0; w < 4; w++) {
+                            const uint4 xv = MT == 1 ? X[j][w] : xs[((int64_t)mm * 4 + w) * C + c];
+                            word_dot<SYM>(words[w], b1, b16, xv, acc1, acc16);
+                        }
+                        part[mm] += sc * fold(acc1, acc16);
+                    }
                 }
             }
-        }
-    };
-
-    int64_t rb = (int64_t)blockIdx.x * rows_per_cta;
-    if (rb < p.n) fetch(cw, cs, cz, rb);
-    for (; rb < p.n; rb += stride) {
-        if (rb + stride < p.n) fetch(nw, ns, nz, rb + stride);
-        float part[ROWS];
-#pragma unroll
-        for (int rr = 0; rr < ROWS; rr++) {
-            part[rr] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < J; j++) {
-                __half2 b1, b16;
-                if constexpr (SYM) {
-                    b1 = __float2half2_rn(1032.0f);
-                    b16 = __float2half2_rn(1152.0f);
-                } else {
-                    const __half z = cz[rr][j];
-                    b1 = __half2half2(__hadd(z, __float2half_rn(1024.0f)));
-                    b16 = __half2half2(__hfma(z, __float2half_rn(16.0f), __float2half_rn(1024.0f)));
-                }
-                part[rr] += __half2float(cs[rr][j]) * chunk_dot<SYM>(cw[rr][j], b1, b16, X[j]);
-            }
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) part[rr] += __shfl_xor_sync(0xffffffffu, part[rr], off);
-        }
-        if constexpr (KSPLIT == 1) {
-            if (lane < ROWS) {
-                float v = part[0];
-#pragma unroll
-                for (int rr = 1; rr < ROWS; rr++) if (lane == rr) v = part[rr];
-                const int64_t r = rb + team * ROWS + lane;
-                if (r < p.n) {
-                    v *= inv_ps;
-                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[r] = __float2bfloat16_rn(v);
-                    else reinterpret_cast<float*>(p.y)[r] = v;
-                }
-            }
-        } else {
-            if (lane == 0) {
-#pragma unroll
-                for (int rr = 0; rr < ROWS; rr++) red[warp * ROWS + rr] = part[rr];
-            }
-            __syncthreads();
-            if (wit == 0 && lane < ROWS) {
-                float v = 0.0f;
-#pragma unroll
-                for (int t = 0; t < KSPLIT; t++) v += red[(team * KSPLIT + t) * ROWS + lane];
-                const int64_t r = rb + team * ROWS + lane;
-                if (r < p.n) {
-                    v *= inv_ps;
-                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[r] = __float2bfloat16_rn(v);
-                    else reinterpret_cast<float*>(p.y)[r] = v;
-                }
-            }
-            __syncthreads();
-        }
-#pragma unroll
-        for (int rr = 0; rr < ROWS; rr++)
-#pragma unroll
-            for (int j = 0; j < J; j++) { cw[rr][j] = nw[rr][j]; cs[rr][j] = ns[rr][j]; cz[rr][j] = nz[rr][j]; }
-    }
-}
-
-// m in 2..4: the dequantized pairs of a chunk are reused for every token; x pairs come from shared
-// memory laid out [m][word][chunk] (16 bytes each) so that a warp's reads are conflict-free.
-template <int KSPLIT, int J, int MT, bool SYM>
-__global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_small_m_kernel(GemvParams p)
-{
-    constexpr int TEAMS = kWarps / KSPLIT;
-    extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ float red[kWarps * MT];
-    __shared__ float pscale[MT];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-    const int team = warp / KSPLIT, wit = warp % KSPLIT;
-    const int C = p.k / 32, ng = p.k / p.group, cpg = p.group / 32;
-    const int64_t rowbytes = p.k / 2;
-    uint4* xs = reinterpret_cast<uint4*>(smem);  // [MT][4][C] of 4 half2
-
-    for (int mm = 0; mm < MT; mm++) {
-        const float amax = block_amax(p.x + (int64_t)mm * p.k, p.k, p.status, red);
-        if (threadIdx.x == 0) pscale[mm] = prescale_for(amax);
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < MT * C; idx += blockDim.x) {
-        const int mm = idx / C, c = idx % C;
-        __half2 X[16];
-        load_x_chunk(p.x + (int64_t)mm * p.k + 32 * c, pscale[mm], X);
-#pragma unroll
-        for (int w = 0; w < 4; w++) {
-            uint4 v;
-            v.x = h2_as_u32(X[4 * w]); v.y = h2_as_u32(X[4 * w + 1]);
-            v.z = h2_as_u32(X[4 * w + 2]); v.w = h2_as_u32(X[4 * w + 3]);
-            xs[((int64_t)mm * 4 + w) * C + c] = v;
-        }
-    }
-    __syncthreads();
-
-    for (int64_t rb = (int64_t)blockIdx.x * TEAMS; rb < p.n; rb += (int64_t)gridDim.x * TEAMS) {
-        const int64_t r = rb + team;
-        float part[MT];
-#pragma unroll
-        for (int mm = 0; mm < MT; mm++) part[mm] = 0.0f;
-        uint4 wv[J];
-        __half scv[J], zcv[J];
-#pragma unroll
-        for (int j = 0; j < J; j++) {
-            const int c = wit * 32 * J + 32 * j + lane;
-            if (r < p.n && c < C) {
-                wv[j] = ldg_nc_v4(p.packed + r * rowbytes + (int64_t)c * 16);
-                scv[j] = p.scales[r * ng + c / cpg];
-                zcv[j] = SYM ? __float2half_rn(8.0f) : p.zeros[r * ng + c / cpg];
-            } else {
-                wv[j] = make_uint4(0, 0, 0, 0);
-                scv[j] = __float2half_rn(0.0f);
-                zcv[j] = __float2half_rn(0.0f);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < J; j++) {
-            const int c = wit * 32 * J + 32 * j + lane;
-            if (c >= C) continue;
-            const __half2 b1 = __half2half2(__hadd(zcv[j], __float2half_rn(1024.0f)));
-            const __half2 b16 = __half2half2(__hfma(zcv[j], __float2half_rn(16.0f), __float2half_rn(1024.0f)));
-            const uint32_t words[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
-            __half2 acc1[MT], acc16[MT];
-#pragma unroll
-            for (int mm = 0; mm < MT; mm++) { acc1[mm] = __float2half2_rn(0.0f); acc16[mm] = acc1[mm]; }
-#pragma unroll
-            for (int w = 0; w < 4; w++) {
-                const uint32_t u = words[w], u8 = u >> 8;
-                const __half2 d0 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x000F000Fu, Keys<SYM>::k1)), b1);
-                const __half2 d1 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x00F000F0u, Keys<SYM>::k16)), b16);
-                const __half2 d2 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x000F000Fu, Keys<SYM>::k1)), b1);
-                const __half2 d3 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x00F000F0u, Keys<SYM>::k16)), b16);
-#pragma unroll
-                for (int mm = 0; mm < MT; mm++) {
-                    const uint4 xv = xs[((int64_t)mm * 4 + w) * C + c];
-                    acc1[mm] = __hfma2(d0, u32_as_h2(xv.x), acc1[mm]);
-                    acc16[mm] = __hfma2(d1, u32_as_h2(xv.y), acc16[mm]);
-                    acc1[mm] = __hfma2(d2, u32_as_h2(xv.z), acc1[mm]);
-                    acc16[mm] = __hfma2(d3, u32_as_h2(xv.w), acc16[mm]);
-                }
-            }
-            const float s = __half2float(scv[j]);
 #pragma unroll
             for (int mm = 0; mm < MT; mm++) {
-                const float2 f1 = __half22float2(acc1[mm]), f16 = __half22float2(acc16[mm]);
-                part[mm] += s * ((f1.x + f1.y) + 0.0625f * (f16.x + f16.y));
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) part[mm] += __shfl_xor_sync(0xffffffffu, part[mm], off);
+            }
+            if constexpr (KSPLIT == 1) {
+                if (lane < MT) {
+                    float v = part[0];
+#pragma unroll
+                    for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
+                    v /= pscale[lane];
+                    const int64_t o = (int64_t)lane * p.n + row;
+                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
+                    else reinterpret_cast<float*>(p.y)[o] = v;
+                }
+            } else {
+                // rows_per_stage == TEAMS here: one row per team per stage
+                if (lane < MT) {
+                    float v = part[0];
+#pragma unroll
+                    for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
+                    redb[(team * KSPLIT + ks) * MT + lane] = v;
+                }
             }
         }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&empty[s]);
+        if constexpr (KSPLIT > 1) {
+            compute_bar();
+            if (ks == 0 && team < rows_here && lane < MT) {
+                float v = 0.0f;
 #pragma unroll
-        for (int mm = 0; mm < MT; mm++)
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) part[mm] += __shfl_xor_sync(0xffffffffu, part[mm], off);
-        if (lane == 0) {
-#pragma unroll
-            for (int mm = 0; mm < MT; mm++) red[warp * MT + mm] = part[mm];
+                for (int t = 0; t < KSPLIT; t++) v += redb[(team * KSPLIT + t) * MT + lane];
+                v /= pscale[lane];
+                const int64_t o = (int64_t)lane * p.n + (rs + team);
+                if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
+                else reinterpret_cast<float*>(p.y)[o] = v;
+            }
         }
-        __syncthreads();
-        if (wit == 0 && lane < MT && r < p.n) {
-            float v = 0.0f;
-            for (int t = 0; t < KSPLIT; t++) v += red[(team * KSPLIT + t) * MT + lane];
-            v /= pscale[lane];
-            const int64_t o = (int64_t)lane * p.n + r;
-            if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
-            else reinterpret_cast<float*>(p.y)[o] = v;
-        }
-        __syncthreads();
     }
 }
 
-// Launched with programmatic stream serialization: the kernel may begin (and prefetch weights into
-// L2) while the previous kernel on the stream drains; it reads x only after griddepcontrol.wait.
-template <int KSPLIT, int J, int ROWS>
-int launch_m1(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
+template <int KSPLIT, int J, int MT>
+int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
 {
+    const size_t smem = (size_t)kStages * kStageBytes + (size_t)MT * p.k * 2 + kScaleBytes +
+                        (2 * 16 * kMaxM + 8 * kMaxM) * sizeof(float) + 2 * kStages * sizeof(uint64_t);
+    if (smem > 227 * 1024) return Q4_ERR_UNSUPPORTED;
+    auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, J, MT, true> : w4a16_gemv_kernel<KSPLIT, J, MT, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    // Programmatic stream serialization: the kernel may start (and prefetch its weights into L2) while
+    // the previous kernel on the stream drains; it reads x only after griddepcontrol.wait.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = symmetric ? cudaLaunchKernelEx(&cfg, w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, true>, p)
-                              : cudaLaunchKernelEx(&cfg, w4a16_gemv_m1_kernel<KSPLIT, J, ROWS, false>, p);
-    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
 template <int KSPLIT, int J>
-int launch_m1_rows(const GemvParams& p, int symmetric, cudaStream_t s)
-{
-    constexpr int TEAMS = kWarps / KSPLIT;
-    const int64_t target = (int64_t)q4_num_sms() * 2;  // two resident CTAs per SM
-    auto ctas = [&](int rows) { return ((int64_t)p.n + TEAMS * rows - 1) / (TEAMS * rows); };
-    // four rows in flight only with one chunk per lane (two chunks x four rows exceed 128 registers)
-    if constexpr (J == 1)
-        if (ctas(4) >= target) return launch_m1<KSPLIT, J, 4>(p, symmetric, (int)std::min<int64_t>(ctas(4), target), s);
-    if (ctas(2) >= target) return launch_m1<KSPLIT, J, 2>(p, symmetric, (int)std::min<int64_t>(ctas(2), target), s);
-    return launch_m1<KSPLIT, J, 1>(p, symmetric, (int)std::min<int64_t>(ctas(1), target), s);
-}
-
-template <int KSPLIT, int J, int MT>
-int launch_small(const GemvParams& p, int symmetric, cudaStream_t s)
-{
-    constexpr int TEAMS = kWarps / KSPLIT;
-    const size_t smem = (size_t)MT * p.k * 2;
-    const int grid = (int)std::min<int64_t>(((int64_t)p.n + TEAMS - 1) / TEAMS, (int64_t)q4_num_sms());
-    auto kern = symmetric ? w4a16_gemv_small_m_kernel<KSPLIT, J, MT, true> : w4a16_gemv_small_m_kernel<KSPLIT, J, MT, false>;
-    if (smem > 200 * 1024) return Q4_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return Q4_ERR_CUDA;
-    kern<<<grid, kThreads, smem, s>>>(p);
-    return q4_launch_status();
-}
-
-template <int KSPLIT, int J>
-int launch_small_m(const GemvParams& p, int symmetric, cudaStream_t s)
+int launch_m(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
 {
     switch (p.m) {
-        case 2: return launch_small<KSPLIT, J, 2>(p, symmetric, s);
-        case 3: return launch_small<KSPLIT, J, 3>(p, symmetric, s);
-        default: return launch_small<KSPLIT, J, 4>(p, symmetric, s);
+        case 1: return launch<KSPLIT, J, 1>(p, symmetric, grid, s);
+        case 2: return launch<KSPLIT, J, 2>(p, symmetric, grid, s);
+        case 3: return launch<KSPLIT, J, 3>(p, symmetric, grid, s);
+        default: return launch<KSPLIT, J, 4>(p, symmetric, grid, s);
     }
 }
 
 template <int J>
-int dispatch_ksplit(const GemvParams& p, int symmetric, int ksplit, cudaStream_t s)
+int launch_ksplit(const GemvParams& p, int symmetric, int ksplit, int grid, cudaStream_t s)
 {
-    if (p.m == 1) {
-        switch (ksplit) {
-            case 1: return launch_m1_rows<1, J>(p, symmetric, s);
-            case 2: return launch_m1_rows<2, J>(p, symmetric, s);
-            case 4: return launch_m1_rows<4, J>(p, symmetric, s);
-            default: return launch_m1_rows<8, J>(p, symmetric, s);
-        }
-    }
     switch (ksplit) {
-        case 1: return launch_small_m<1, J>(p, symmetric, s);
-        case 2: return launch_small_m<2, J>(p, symmetric, s);
-        case 4: return launch_small_m<4, J>(p, symmetric, s);
-        default: return launch_small_m<8, J>(p, symmetric, s);
+        case 1: return launch_m<1, J>(p, symmetric, grid, s);
+        case 2: return launch_m<2, J>(p, symmetric, grid, s);
+        case 4: return launch_m<4, J>(p, symmetric, grid, s);
+        default: return launch_m<8, J>(p, symmetric, grid, s);
     }
 }
 
@@ -479,7 +368,7 @@ int dispatch_ksplit(const GemvParams& p, int symmetric, int ksplit, cudaStream_t
 int q4_gemv_w4a16_launch(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
                          int32_t* dev_status, cudaStream_t stream)
 {
-    if (w->k % 32 || w->k > 16384 || m < 1 || m > 4) return Q4_ERR_UNSUPPORTED;
+    if (w->k % 32 || w->k > 16384 || m < 1 || m > kMaxM) return Q4_ERR_UNSUPPORTED;
     GemvParams p;
     p.x = x;
     p.packed = w->packed;
@@ -493,10 +382,22 @@ int q4_gemv_w4a16_launch(const uint16_t* x, int32_t m, const q4_weight* w, void*
     p.group = w->group;
     p.out_bf16 = out_dtype == Q4_OUT_BF16;
     const int C = w->k / 32;
-    const int J = C >= 64 ? 2 : 1;
     int ksplit = 1;
-    while (ksplit * 32 * J < C) ksplit *= 2;
+    while (ksplit * 64 < C) ksplit *= 2;                     // at most two chunks per lane
     if (ksplit > 8) return Q4_ERR_UNSUPPORTED;
-    return J == 2 ? dispatch_ksplit<2>(p, w->symmetric, ksplit, stream)
-                  : dispatch_ksplit<1>(p, w->symmetric, ksplit, stream);
+    const int J = (C + 32 * ksplit - 1) / (32 * ksplit);
+    const int teams = kComputeWarps / ksplit;
+    const int rowbytes = w->k / 2;
+    int rps = kStageBytes / rowbytes;
+    if (ksplit > 1) rps = teams;                             // one row per team per stage
+    const int ng = w->k / w->group;
+    const int sbytes_row = ng * 2 * (w->symmetric ? 1 : 2);
+    const int sms = q4_num_sms();
+    int rpc = (w->n + sms - 1) / sms;
+    rpc = std::max(1, std::min(rpc, kScaleBytes / sbytes_row));
+    p.rows_per_cta = rpc;
+    p.rows_per_stage = std::max(1, rps);
+    const int grid = (w->n + rpc - 1) / rpc;
+    return J == 2 ? launch_ksplit<2>(p, w->symmetric, ksplit, grid, stream)
+                  : launch_ksplit<1>(p, w->symmetric, ksplit, grid, stream);
 }

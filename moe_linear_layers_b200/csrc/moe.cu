@@ -1,11 +1,369 @@
-// Top-k routed MoE layer with INT4 SwiGLU experts (in progress).
-#include "q4_common.cuh"
+// Top-k routed MoE layer of SwiGLU experts with INT4 weights (moe_q4_forward).
+//
+// Sources: "大模型之Dense、MoE与量化" 混合专家架构 MoE (a Linear router scores the experts, a few are chosen,
+// their outputs are recombined in proportion); "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" §3.2
+// (router output through softmax, kept in high precision) and §1 (dispatch and merge cost extra);
+// "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" MoE架构设计 (experts are small FFNs behind a gating
+// network, SwiGLU as in the base model).
+//
+// Launch sequence (one stream, no host synchronisation):
+//   1. route     fp32 logits in a pinned reduction order, top-k by (logit desc, id asc), softmax
+//                weights over the chosen logits, per-chunk expert histograms (16 tokens per chunk);
+//   2. scan      expert counts and offsets, per-chunk bases (a column scan of the histograms), and the
+//                tile counts of both grouped GEMMs;
+//   3. scatter   stable counting sort: every (token, slot) pair gets its row in the permuted order
+//                (expert, token ascending), and the token's activation row is gathered there;
+//   4. gate/up   grouped tcgen05 GEMM over (expert, token tile, 64 intermediate rows) tiles with the
+//                SwiGLU epilogue, h in fp16;
+//   5. down      grouped tcgen05 GEMM over (expert, token tile, 128 hidden rows) tiles whose epilogue
+//                adds w[t][j] * out into the fp32 output (float atomics: the sum order is not fixed);
+//   6. (bf16 output) a conversion pass.
+#include "tc_host.cuh"
 
-extern "C" size_t moe_q4_workspace_size(int32_t, int32_t, int32_t, int32_t, int32_t) { return 0; }
+namespace {
 
-extern "C" int moe_q4_forward(const uint16_t*, int32_t, int32_t, const float*, const float*, int32_t, int32_t,
-                              const q4_weight*, int32_t, void*, int32_t, int32_t*, float*, int32_t*, int32_t*,
-                              int32_t*, void*, size_t, int32_t*, void*)
+constexpr int kRouteTok = 16;           // tokens per route CTA (= one histogram chunk)
+constexpr int kRouteWarps = 16;
+constexpr int kRouteKC = 64;            // K columns staged per step
+constexpr int kMaxTopk = 16;
+
+// ---------------------------------------------------------------------------------------------- //
+// 1. route
+// ---------------------------------------------------------------------------------------------- //
+// Warp w computes 4 tokens x 16 experts: lane l owns the k = l (mod 32) partial sums, each an fma chain
+// with k ascending; the 32 partials are combined by an xor butterfly (s = 16, 8, 4, 2, 1), which gives
+// every lane the same value.  This is the pinned order the oracle reproduces bit for bit.
+__global__ void __launch_bounds__(kRouteWarps * 32, 1)
+moe_route_kernel(const uint16_t* __restrict__ x, int T, int H, const float* __restrict__ Wr,
+                 const float* __restrict__ bias, int E, int topk, int32_t* __restrict__ ids, float* __restrict__ wts,
+                 int32_t* __restrict__ hist, int32_t* status)
 {
-    return Q4_ERR_UNSUPPORTED;
+    __shared__ float xs[kRouteTok][kRouteKC];
+    __shared__ float ws[64][kRouteKC];
+    __shared__ float logits[kRouteTok][tcg::kMaxExperts];
+    __shared__ int hcount[tcg::kMaxExperts];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kRouteTok;
+    const int tg = warp / 4, eg = warp % 4;
+
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hcount[e] = 0;
+    for (int eb = 0; eb < E; eb += 64) {
+        float acc[4][16];
+#pragma unroll
+        for (int a = 0; a < 4; a++)
+#pragma unroll
+            for (int b = 0; b < 16; b++) acc[a][b] = 0.0f;
+        for (int k0 = 0; k0 < H; k0 += kRouteKC) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < kRouteTok * kRouteKC; i += blockDim.x) {
+                const int a = i / kRouteKC, c = i % kRouteKC;
+                const int t = t0 + a;
+                xs[a][c] = t < T ? bf16_bits_to_float(x[(int64_t)t * H + k0 + c]) : 0.0f;
+            }
+            for (int i = threadIdx.x; i < 64 * kRouteKC; i += blockDim.x) {
+                const int b = i / kRouteKC, c = i % kRouteKC;
+                const int e = eb + b;
+                ws[b][c] = e < E ? Wr[(int64_t)e * H + k0 + c] : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < kRouteKC / 32; i++) {
+                const int c = lane + 32 * i;
+                float xv[4], wv[16];
+#pragma unroll
+                for (int a = 0; a < 4; a++) xv[a] = xs[4 * tg + a][c];
+#pragma unroll
+                for (int b = 0; b < 16; b++) wv[b] = ws[16 * eg + b][c];
+#pragma unroll
+                for (int a = 0; a < 4; a++)
+#pragma unroll
+                    for (int b = 0; b < 16; b++) acc[a][b] = fmaf(xv[a], wv[b], acc[a][b]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; a++)
+#pragma unroll
+            for (int b = 0; b < 16; b++) {
+                float v = acc[a][b];
+#pragma unroll
+                for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+                const int e = eb + 16 * eg + b;
+                if (lane == 0 && e < E) logits[4 * tg + a][e] = bias ? v + bias[e] : v;
+            }
+    }
+    __syncthreads();
+
+    // top-k per token (warp w handles token w of the chunk)
+    const int t = t0 + warp;
+    if (warp < kRouteTok && t < T) {
+        constexpr int PER = tcg::kMaxExperts / 32;
+        float v[PER];
+        bool finite = true;
+#pragma unroll
+        for (int q = 0; q < PER; q++) {
+            const int e = lane + 32 * q;
+            v[q] = e < E ? logits[warp][e] : -INFINITY;
+            if (e < E) finite &= isfinite(v[q]);
+        }
+        if (!__all_sync(0xffffffffu, finite)) {
+            if (lane == 0) q4_set_status(status, Q4_ERR_NONFINITE);
+        }
+        float sel_l[kMaxTopk];
+        int sel_e[kMaxTopk];
+        for (int j = 0; j < topk; j++) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int q = 0; q < PER; q++) {
+                const int e = lane + 32 * q;
+                if (e < E && (v[q] > bv || (v[q] == bv && e < be))) { bv = v[q]; be = e; }
+            }
+#pragma unroll
+            for (int s = 16; s >= 1; s >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, s);
+                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+            }
+            sel_l[j] = bv;
+            sel_e[j] = be;
+#pragma unroll
+            for (int q = 0; q < PER; q++)
+                if (lane + 32 * q == be) v[q] = -INFINITY;
+        }
+        if (lane == 0) {
+            float den = 0.0f;
+            for (int j = 0; j < topk; j++) den += expf(sel_l[j] - sel_l[0]);
+            for (int j = 0; j < topk; j++) {
+                ids[(int64_t)t * topk + j] = sel_e[j];
+                wts[(int64_t)t * topk + j] = expf(sel_l[j] - sel_l[0]) / den;
+                atomicAdd(&hcount[sel_e[j]], 1);
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = hcount[e];
+}
+
+// ---------------------------------------------------------------------------------------------- //
+// 2. scan (one CTA, one thread per expert)
+// ---------------------------------------------------------------------------------------------- //
+__global__ void moe_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E, int I, int H,
+                                int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
+                                int32_t* __restrict__ counts, int32_t* __restrict__ tiles_gu,
+                                int32_t* __restrict__ tiles_dn)
+{
+    __shared__ int cnt[tcg::kMaxExperts];
+    const int e = threadIdx.x;
+    int c_e = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; c++) c_e += hist[(int64_t)c * E + e];
+        cnt[e] = c_e;
+        if (counts) counts[e] = c_e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int off = 0, tg = 0, td = 0;
+        for (int q = 0; q < E; q++) {
+            offsets[q] = off;
+            tiles_gu[q] = tg;
+            tiles_dn[q] = td;
+            const int mt = (cnt[q] + tcg::BN - 1) / tcg::BN;
+            off += cnt[q];
+            tg += mt * (I / 64);
+            td += mt * (H / tcg::BM);
+        }
+        offsets[E] = off;
+        tiles_gu[E] = tg;
+        tiles_dn[E] = td;
+    }
+    __syncthreads();
+    if (e < E) {
+        int run = offsets[e];
+        for (int c = 0; c < nchunks; c++) {
+            chunk_base[(int64_t)c * E + e] = run;
+            run += hist[(int64_t)c * E + e];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------------- //
+// 3. scatter + gather (one CTA per chunk of 16 tokens)
+// ---------------------------------------------------------------------------------------------- //
+__global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int E, int topk,
+                                                          const int32_t* __restrict__ ids,
+                                                          const int32_t* __restrict__ chunk_base,
+                                                          int32_t* __restrict__ perm, uint16_t* __restrict__ xperm)
+{
+    __shared__ int pos[kRouteTok * kMaxTopk];
+    const int c = blockIdx.x;
+    const int t0 = c * kRouteTok;
+    const int npairs = min(kRouteTok, T - t0) * topk;
+    for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
+        const int tl = q / topk, j = q % topk;
+        const int e = ids[(int64_t)(t0 + tl) * topk + j];
+        int rank = 0;  // earlier tokens of this chunk that chose the same expert (a token picks an expert once)
+        for (int u = 0; u < tl; u++)
+            for (int jj = 0; jj < topk; jj++) rank += ids[(int64_t)(t0 + u) * topk + jj] == e;
+        const int p = chunk_base[(int64_t)c * E + e] + rank;
+        pos[q] = p;
+        perm[p] = (t0 + tl) * topk + j;
+    }
+    __syncthreads();
+    const int vec = H / 8;  // 16-byte units per row
+    for (int i = threadIdx.x; i < npairs * vec; i += blockDim.x) {
+        const int q = i / vec, u = i % vec;
+        const int t = t0 + q / topk;
+        reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * H)[u] = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)t * H) + u);
+    }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ a, __nv_bfloat16* __restrict__ b, int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        b[i] = __float2bfloat16_rn(a[i]);
+}
+
+struct Workspace {
+    uint16_t* xperm;
+    __half* h;
+    float* y32;
+    int32_t *ids, *perm, *offsets, *counts, *hist, *chunk_base, *tiles_gu, *tiles_dn;
+    float* wts;
+    size_t bytes;
+};
+
+inline size_t al(size_t v) { return (v + 255) & ~(size_t)255; }
+
+Workspace carve(void* base, int T, int H, int I, int E, int topk)
+{
+    Workspace w = {};
+    const size_t P = (size_t)T * topk;
+    const size_t nch = (size_t)(T + kRouteTok - 1) / kRouteTok;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { uint8_t* q = p ? p + o : nullptr; o += al(bytes); return q; };
+    w.xperm = reinterpret_cast<uint16_t*>(take(P * H * 2));
+    w.h = reinterpret_cast<__half*>(take(P * I * 2));
+    w.y32 = reinterpret_cast<float*>(take((size_t)T * H * 4));
+    w.ids = reinterpret_cast<int32_t*>(take(P * 4));
+    w.wts = reinterpret_cast<float*>(take(P * 4));
+    w.perm = reinterpret_cast<int32_t*>(take(P * 4));
+    w.offsets = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    w.counts = reinterpret_cast<int32_t*>(take(E * 4));
+    w.hist = reinterpret_cast<int32_t*>(take(nch * E * 4));
+    w.chunk_base = reinterpret_cast<int32_t*>(take(nch * E * 4));
+    w.tiles_gu = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    w.tiles_dn = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    w.bytes = o;
+    return w;
+}
+
+template <int G, bool SYM>
+int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I, int E, int topk, float* y32,
+                   int32_t* status, cudaStream_t s)
+{
+    using namespace tcg;
+    const int P = T * topk;
+    const int sms = q4_num_sms();
+    CUtensorMap mx, mg, mu, mh, md;
+    if (!make_act_map(&mx, ws.xperm, H, P, 2, false) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
+        !make_packed_map(&mu, ex[1].packed, H, (uint64_t)E * I, 64) || !make_act_map(&mh, ws.h, I, P, 2, true) ||
+        !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
+        return Q4_ERR_CUDA;
+    Args a = {};
+    a.M = P;
+    a.N = I;
+    a.K = H;
+    a.scales_a = reinterpret_cast<const __half*>(ex[0].scales);
+    a.zeros_a = reinterpret_cast<const __half*>(ex[0].zeros);
+    a.scales_b = reinterpret_cast<const __half*>(ex[1].scales);
+    a.zeros_b = reinterpret_cast<const __half*>(ex[1].zeros);
+    a.status = status;
+    a.expert_tiles = ws.tiles_gu;
+    a.offsets = ws.offsets;
+    a.h = ws.h;
+    a.E = E;
+    a.topk = topk;
+    int rc = launch<false, G, SYM, Mode::GateUp>(mx, mg, mu, a, sms, s);
+    if (rc) return rc;
+    Args d = {};
+    d.M = P;
+    d.N = H;
+    d.K = I;
+    d.scales_a = reinterpret_cast<const __half*>(ex[2].scales);
+    d.zeros_a = reinterpret_cast<const __half*>(ex[2].zeros);
+    d.y = y32;
+    d.status = status;
+    d.expert_tiles = ws.tiles_dn;
+    d.offsets = ws.offsets;
+    d.perm = ws.perm;
+    d.topk_w = ws.wts;
+    d.E = E;
+    d.topk = topk;
+    return launch<false, G, SYM, Mode::Down>(mh, md, md, d, sms, s);
+}
+
+}  // namespace
+
+extern "C" size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk)
+{
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || topk <= 0) return 0;
+    return carve(nullptr, T, H, I, E, topk).bytes;
+}
+
+extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
+                              int32_t E, int32_t topk, const q4_weight* experts, int32_t I, void* y, int32_t out_dtype,
+                              int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                              void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
+    if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
+        return Q4_ERR_SHAPE;
+    if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    const q4_weight& g = experts[0];
+    const q4_weight& u = experts[1];
+    const q4_weight& d = experts[2];
+    for (int i = 0; i < 3; i++) {
+        const q4_weight& w = experts[i];
+        if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
+        if (w.group != g.group || w.symmetric != g.symmetric) return Q4_ERR_UNSUPPORTED;
+        if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
+            return Q4_ERR_ALIGN;
+    }
+    if (g.group != 64 && g.group != 128) return Q4_ERR_UNSUPPORTED;
+    if (g.n != E * I || g.k != H || u.n != E * I || u.k != H || d.n != E * H || d.k != I) return Q4_ERR_SHAPE;
+    if (!q4_aligned16(x) || !q4_aligned16(y) || ((uintptr_t)workspace & 255u) || ((uintptr_t)router_w & 15u))
+        return Q4_ERR_ALIGN;
+    Workspace ws = carve(workspace, T, H, I, E, topk);
+    if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
+    if (T == 0) return Q4_OK;
+    if (topk_ids) ws.ids = topk_ids;
+    if (topk_w) ws.wts = topk_w;
+    if (perm) ws.perm = perm;
+    if (offsets) ws.offsets = offsets;
+    if (expert_counts) ws.counts = expert_counts;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int nch = (T + kRouteTok - 1) / kRouteTok;
+    float* y32 = out_dtype == Q4_OUT_F32 ? reinterpret_cast<float*>(y) : ws.y32;
+
+    moe_route_kernel<<<nch, kRouteWarps * 32, 0, s>>>(x, T, H, router_w, router_bias, E, topk, ws.ids, ws.wts, ws.hist,
+                                                      dev_status);
+    moe_scan_kernel<<<1, tcg::kMaxExperts, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
+                                                   ws.tiles_gu, ws.tiles_dn);
+    moe_scatter_kernel<<<nch, 256, 0, s>>>(x, T, H, E, topk, ws.ids, ws.chunk_base, ws.perm, ws.xperm);
+    if (cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess) return Q4_ERR_CUDA;
+    int rc = q4_launch_status();
+    if (rc) return rc;
+    if (g.group == 128) rc = g.symmetric ? launch_experts<128, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)
+                                         : launch_experts<128, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s);
+    else rc = g.symmetric ? launch_experts<64, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)
+                          : launch_experts<64, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s);
+    if (rc) return rc;
+    if (out_dtype == Q4_OUT_BF16) {
+        const int64_t n = (int64_t)T * H;
+        f32_to_bf16_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, s>>>(y32, reinterpret_cast<__nv_bfloat16*>(y), n);
+        rc = q4_launch_status();
+    }
+    return rc;
 }

@@ -1,0 +1,498 @@
+// Tensor-core (tcgen05) GEMM with INT4 weights widened into TMEM, shared by the dense linear layers
+// (W4A16 and W4A8) and by the two grouped expert GEMMs of the MoE layer.
+//
+// Sources: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" §2.1 (4-bit storage restored to a 16-bit
+// type for W4A16), §2.3 (INT4 widened to INT8, INT8 x INT8 into INT32, rescale by scale_w*scale_a),
+// §2.2 (INT8 tensor cores at twice the FP16 rate); "从FP32到INT4" §1.3 (one scale per group);
+// "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" MoE架构设计 (experts are small SwiGLU FFNs);
+// "大模型之Dense、MoE与量化" 混合专家架构 MoE (expert outputs recombined in proportion to the router).
+//
+// Every mode computes, for a tile of 128 weight rows (the MMA's M, one TMEM lane each) and 128
+// activation rows (the MMA's N), D_g = sum_{k in g} (code - zero)[row][k] * act[m][k] exactly (integer
+// codes are exact in bf16 / fp16 / int8) one quantization group at a time, and the epilogue
+// accumulates s[row][g] * D_g in fp32.  Group accumulators are double-buffered in TMEM so the MMA of
+// group g+1 overlaps the epilogue's drain of group g.
+//
+// Data flow: TMA brings the packed nibbles (64-byte swizzle) and the activation tile (128-byte
+// swizzle, K-major, the MMA's B operand) into a 4-stage shared-memory ring.  Converter warps widen the
+// nibbles in registers and write them into TMEM with tcgen05.st (the MMA's A operand), so widened
+// weights never use shared-memory bandwidth.  One thread issues tcgen05.mma and commits to mbarriers.
+//
+// Modes:
+//   Dense   y[m][n] = sum_g s[n][g] * D_g (W4A16, bf16 MMA) or y = s_a[m] * sum_g s[n][g] * D_g / 16
+//           (W4A8, int8 MMA on 16*code).
+//   GateUp  A rows 0-63 = gate rows i0..i0+63 of expert e, rows 64-127 = the same rows of up; B = the
+//           expert's rows of the permuted activations; epilogue h = SiLU(gate) * up -> fp16.
+//   Down    A = 128 rows of the expert's down projection (fp16 codes), B = h (fp16); epilogue
+//           y[token][n] += w[token][slot] * out (fp32 reduction into the output).
+//
+// Warp roles (448 threads): warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-5
+// converters (TMEM lanes 32*(warp%4) ...), warps 6-13 epilogue (two warps per TMEM lane quarter, each
+// draining 64 of the 128 columns).  Persistent CTAs walk tiles with a stride of gridDim.x; the rings
+// carry their phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
+#pragma once
+
+#include "tc_ptx.cuh"
+
+namespace tcg {
+
+enum class Mode { Dense, GateUp, Down };
+
+constexpr int BM = 128;                  // weight rows per tile
+constexpr int BN = 128;                  // activation rows per tile
+constexpr int KBLK = 128;                // K per stage
+constexpr int NS = 4;                    // shared-memory stages
+constexpr int NA = 4;                    // TMEM stages of widened weights
+constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
+constexpr int kThreads = 448;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxExperts = 256;
+
+template <bool INT8, Mode MODE> struct Cfg {
+    static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2);   // activation bytes per stage
+    static constexpr int ACOLS = KBLK / (INT8 ? 4 : 2);         // TMEM columns of one widened stage
+    static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
+    static constexpr uint32_t A_COL0 = 2 * BN;                  // widened weights after the 2 D buffers
+    static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
+    static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 2048;
+};
+
+struct Args {
+    int M, N, K;              // Dense: M activation rows, N weight rows.  MoE: N = rows per expert matrix
+    int out_bf16;
+    const __half* scales_a;   // Dense: W; GateUp: gate; Down: down
+    const __half* zeros_a;
+    const __half* scales_b;   // GateUp: up
+    const __half* zeros_b;
+    const float* scale_a;     // W4A8 per-token scales
+    void* y;                  // Dense: [M][N]; Down: fp32 [T][N] (reduction target)
+    int32_t* acc_dbg;         // W4A8 debug partials (nullable)
+    int32_t* status;
+    // MoE
+    const int32_t* expert_tiles;   // [E+1] prefix sums of tiles per expert
+    const int32_t* offsets;        // [E+1] first permuted row of each expert
+    const int32_t* perm;           // [P] pair index t*topk + j of each permuted row
+    const float* topk_w;           // [T*topk] routing weights
+    __half* h;                     // GateUp output [P][N]
+    int E, topk;
+};
+
+struct Tile {
+    int m0, m_end;    // activation rows [m0, m0+128) of which rows < m_end are valid
+    int n0;           // Dense/Down: first weight row of the tile inside the (expert) matrix; GateUp: i0
+    int wrow_a, wrow_b;  // packed rows of the TMA boxes
+    int e;
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// 8 nibbles (k = 0..7, even k in the low nibble of each byte) -> 4 words of 16-bit pairs holding the
+// exact integers (code - zero) in natural k order.  A PRMT puts nibble 2b at bits 0-3 and nibble 2b+1
+// at bits 16-19; one LOP3 ORs in the exponent of 128.0 (bf16) or 1024.0 (fp16), which makes the
+// nibble the low mantissa bits, and flips bit 3 of symmetric two's-complement codes (code + 8); one
+// packed subtract removes the magic plus the zero point (bias2 = magic + zero in both halves).
+template <bool SYM, bool F16>
+__device__ __forceinline__ void widen16(uint32_t w, uint32_t bias2, uint32_t (&o)[4])
+{
+    constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
+    constexpr uint32_t key = SYM ? (magic ^ 0x00080008u) : magic;
+    const uint32_t u = w >> 4;
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        const uint32_t sel = (uint32_t)b | ((uint32_t)b << 4) | ((uint32_t)(4 + b) << 8) | ((uint32_t)(4 + b) << 12);
+        const uint32_t t = lop3_and_xor(prmt(w, u, sel), 0x000F000Fu, key);
+        o[b] = F16 ? f16x2_sub(t, bias2) : bf16x2_sub(t, bias2);
+    }
+}
+
+// 8 symmetric nibbles -> 8 int8 of value 16*code in natural k order (two words): the nibble goes to the
+// high half of its byte, which makes the byte the two's-complement value 16*code; the factor 1/16 is
+// folded into the (power-of-two exact) scale.
+__device__ __forceinline__ void widen_s8x16(uint32_t w, uint32_t& o0, uint32_t& o1)
+{
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;
+    const uint32_t hi = w & 0xF0F0F0F0u;
+    o0 = prmt(lo, hi, 0x5140u);
+    o1 = prmt(lo, hi, 0x7362u);
+}
+
+__device__ __forceinline__ uint32_t pair16_bits(float v, bool f16)
+{
+    if (f16) {
+        const __half2 h = __floats2half2_rn(v, v);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v, v);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+struct Shared {
+    uint64_t xw_full[NS], xw_empty[NS], a_full[NA], a_empty[NA], d_full[2], d_empty[2], done;
+    uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
+    uint32_t tmem_base;
+    int abort_flag;
+    int total_tiles;
+    int expert_tiles[kMaxExperts + 1];
+};
+
+template <Mode MODE>
+__device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
+{
+    Tile T;
+    if constexpr (MODE == Mode::Dense) {
+        T.e = 0;
+        T.m0 = (t % tiles_m) * BN;
+        T.m_end = p.M;
+        T.n0 = (t / tiles_m) * BM;
+        T.wrow_a = T.n0;
+        T.wrow_b = 0;
+    } else {
+        int e = 0;
+        while (e + 1 < p.E && sh->expert_tiles[e + 1] <= t) e++;
+        const int local = t - sh->expert_tiles[e];
+        const int nt_per = MODE == Mode::GateUp ? p.N / 64 : p.N / BM;
+        const int mt = local / nt_per, nt = local % nt_per;
+        T.e = e;
+        T.m0 = p.offsets[e] + mt * BN;
+        T.m_end = p.offsets[e + 1];
+        T.n0 = MODE == Mode::GateUp ? nt * 64 : nt * BM;
+        T.wrow_a = e * p.N + T.n0;
+        T.wrow_b = T.wrow_a;
+    }
+    return T;
+}
+
+// Scale and zero rows of tile row r (one TMEM lane); nullptr when the row is outside the matrix.
+template <Mode MODE>
+__device__ __forceinline__ void row_params(const Args& p, const Tile& T, int r, int ng, const __half*& srow,
+                                           const __half*& zrow)
+{
+    if constexpr (MODE == Mode::Dense) {
+        const int n = T.n0 + r;
+        srow = n < p.N ? p.scales_a + (int64_t)n * ng : nullptr;
+        zrow = (n < p.N && p.zeros_a) ? p.zeros_a + (int64_t)n * ng : nullptr;
+    } else if constexpr (MODE == Mode::GateUp) {
+        const int64_t row = (int64_t)T.e * p.N + T.n0 + (r & 63);
+        srow = (r < 64 ? p.scales_a : p.scales_b) + row * ng;
+        const __half* z = r < 64 ? p.zeros_a : p.zeros_b;
+        zrow = z ? z + row * ng : nullptr;
+    } else {
+        const int64_t row = (int64_t)T.e * p.N + T.n0 + r;
+        srow = p.scales_a + row * ng;
+        zrow = p.zeros_a ? p.zeros_a + row * ng : nullptr;
+    }
+}
+
+template <bool INT8, int G, bool SYM, Mode MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
+               const __grid_constant__ CUtensorMap tm_wb, Args p)
+{
+    using C = Cfg<INT8, MODE>;
+    constexpr bool F16 = MODE == Mode::Down;   // the down projection consumes fp16 h
+    constexpr int GPK = KBLK / G;               // groups per K stage
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* xs = smem;                          // NS x XSTAGE (1024-aligned stages)
+    uint8_t* wsm = smem + NS * C::XSTAGE;        // NS x WSTAGE
+    float* xchg = reinterpret_cast<float*>(wsm + NS * WSTAGE);   // GateUp only
+    Shared* sh = reinterpret_cast<Shared*>(wsm + NS * WSTAGE + C::XCHG);
+    volatile int* abort_flag = &sh->abort_flag;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int kblocks = p.K / KBLK, ngroups = p.K / G;
+    const int tiles_m = (p.M + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; i++) { tc::mbar_init(&sh->xw_full[i], 1); tc::mbar_init(&sh->xw_empty[i], 1 + 4); }
+        for (int i = 0; i < NA; i++) { tc::mbar_init(&sh->a_full[i], 4); tc::mbar_init(&sh->a_empty[i], 1); }
+        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->d_full[i], 1); tc::mbar_init(&sh->d_empty[i], 8); }
+        tc::mbar_init(&sh->done, 1);
+        tc::mbar_init(&sh->up_ready, 4);
+        tc::mbar_init(&sh->gate_done, 4);
+        sh->abort_flag = 0;
+        if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
+        else sh->total_tiles = p.expert_tiles[p.E];
+        tc::fence_mbar_init();
+    }
+    if constexpr (MODE != Mode::Dense)
+        for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sh->expert_tiles[i] = p.expert_tiles[i];
+    if (warp == 0 && lane == 0) {
+        tc::tma_prefetch_desc(&tm_x);
+        tc::tma_prefetch_desc(&tm_wa);
+        if constexpr (MODE == Mode::GateUp) tc::tma_prefetch_desc(&tm_wb);
+    }
+    if (warp == 1) tc::tmem_alloc(&sh->tmem_base, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = sh->tmem_base;
+    const int total = sh->total_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+                for (int kb = 0; kb < kblocks; kb++, it++) {
+                    const int s = it % NS;
+                    if (!tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag)) break;
+                    tc::mbar_arrive_expect_tx(&sh->xw_full[s], C::XSTAGE + WSTAGE);
+                    uint8_t* xdst = xs + s * C::XSTAGE;
+                    tc::tma_load_2d(xdst, &tm_x, &sh->xw_full[s], kb * KBLK, T.m0);
+                    if constexpr (!INT8) tc::tma_load_2d(xdst + BN * 128, &tm_x, &sh->xw_full[s], kb * KBLK + 64, T.m0);
+                    uint8_t* wdst = wsm + s * WSTAGE;
+                    if constexpr (MODE == Mode::GateUp) {
+                        tc::tma_load_2d(wdst, &tm_wa, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_a);
+                        tc::tma_load_2d(wdst + 64 * 64, &tm_wb, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_b);
+                    } else {
+                        tc::tma_load_2d(wdst, &tm_wa, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_a);
+                    }
+                }
+            }
+            if (*abort_flag) {  // let every copy this thread issued land before the CTA can exit
+                const uint32_t first = it > (uint32_t)NS ? it - NS : 0;
+                for (uint32_t j = first; j < it; j++)
+                    tc::mbar_wait(&sh->xw_full[j % NS], (j / NS) & 1, p.status, abort_flag, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = INT8 ? tc::idesc_s8_s32(BN) : (F16 ? tc::idesc_f16_f32(BN) : tc::idesc_bf16_f32(BN));
+            uint32_t it = 0, g = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                for (int kb = 0; kb < kblocks && ok; kb++, it++) {
+                    const int s = it % NS, sa = it % NA;
+                    ok = tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag) &&
+                         tc::mbar_wait(&sh->a_full[sa], (it / NA) & 1, p.status, abort_flag);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    const uint32_t xaddr = tc::smem_u32(xs + s * C::XSTAGE);
+#pragma unroll
+                    for (int gi = 0; gi < GPK; gi++, g++) {
+                        const uint32_t db = g & 1;
+                        if (!(ok = tc::mbar_wait(&sh->d_empty[db], ((g >> 1) & 1) ^ 1, p.status, abort_flag))) break;
+                        tc::fence_after_sync();
+#pragma unroll
+                        for (int i = 0; i < G / C::KI; i++) {
+                            const int kk = gi * G + i * C::KI;   // k offset inside the stage
+                            const uint32_t a_tmem = tbase + C::A_COL0 + sa * C::ACOLS + (INT8 ? kk / 4 : kk / 2);
+                            uint32_t boff;
+                            if constexpr (INT8) boff = kk;                              // one 128-byte row box
+                            else boff = (kk / 64) * (BN * 128) + (kk % 64) * 2;          // two 64-column boxes
+                            const uint64_t bdesc = tc::smem_desc_sw128(xaddr + (boff & ~127u)) + ((boff & 127u) >> 4);
+                            if constexpr (INT8) tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                            else tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                        }
+                        tc::mma_commit(&sh->d_full[db]);
+                    }
+                    tc::mma_commit(&sh->xw_empty[s]);
+                    tc::mma_commit(&sh->a_empty[sa]);
+                }
+            }
+            tc::mma_commit(&sh->done);   // every MMA issued so far has completed once `done` flips
+            tc::mbar_wait(&sh->done, 0, p.status, abort_flag, 100000000ull);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------------ converters
+        const int sub = warp & 3;
+        const int r = 32 * sub + lane;                 // row in tile == TMEM lane
+        const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
+        constexpr float kMagic = F16 ? 1024.0f : 128.0f;
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+            const __half *srow, *zrow;
+            row_params<MODE>(p, T, r, ngroups, srow, zrow);
+            // zero points of the next stage are fetched one stage ahead
+            float znext[GPK];
+#pragma unroll
+            for (int gi = 0; gi < GPK; gi++) znext[gi] = SYM ? 8.0f : (zrow ? __half2float(zrow[gi]) : 0.0f);
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % NS, sa = it % NA;
+                float zcur[GPK];
+#pragma unroll
+                for (int gi = 0; gi < GPK; gi++) {
+                    zcur[gi] = znext[gi];
+                    if constexpr (!SYM)
+                        if (kb + 1 < kblocks) znext[gi] = zrow ? __half2float(zrow[(kb + 1) * GPK + gi]) : 0.0f;
+                }
+                if (!tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
+                uint4 v[4];
+                const uint32_t wrow = tc::smem_u32(wsm + s * WSTAGE) + r * 64;
+#pragma unroll
+                for (int c = 0; c < 4; c++) v[c] = lds128(wrow + ((c ^ ((r >> 1) & 3)) << 4));
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->xw_empty[s]);
+                if (!tc::mbar_wait(&sh->a_empty[sa], ((it / NA) & 1) ^ 1, p.status, abort_flag)) goto conv_done;
+                __syncwarp();
+                tc::fence_after_sync();
+                const uint32_t words[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                                            v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+                const uint32_t acol = tbase + lane_field + C::A_COL0 + sa * C::ACOLS;
+                if constexpr (INT8) {
+                    uint32_t o[32];
+#pragma unroll
+                    for (int w = 0; w < 16; w++) widen_s8x16(words[w], o[2 * w], o[2 * w + 1]);
+                    tc::tmem_st32(acol, o);
+                } else {
+                    uint32_t bias[GPK];
+#pragma unroll
+                    for (int gi = 0; gi < GPK; gi++) bias[gi] = pair16_bits(kMagic + zcur[gi], F16);
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        uint32_t o[32];
+#pragma unroll
+                        for (int w = 0; w < 8; w++) {
+                            const int ww = 8 * h + w;                  // word: k = 8*ww .. 8*ww+7
+                            uint32_t q[4];
+                            widen16<SYM, F16>(words[ww], bias[(8 * ww) / G], q);
+#pragma unroll
+                            for (int b = 0; b < 4; b++) o[4 * w + b] = q[b];
+                        }
+                        tc::tmem_st32(acol + 32 * h, o);
+                    }
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->a_full[sa]);
+            }
+        }
+    conv_done:;
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int ew = warp - 6;
+        const int sub = warp & 3, half = ew >> 2;
+        const int r = 32 * sub + lane;
+        const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
+        uint32_t g = 0, tl = 0;
+        float acc[64];
+        for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
+            const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+            const __half *srow, *zrow;
+            row_params<MODE>(p, T, r, ngroups, srow, zrow);
+#pragma unroll
+            for (int j = 0; j < 64; j++) acc[j] = 0.0f;
+            float s_next = srow ? __half2float(srow[0]) : 0.0f;
+            for (int gl = 0; gl < ngroups; gl++, g++) {
+                const uint32_t db = g & 1;
+                float s = s_next;
+                if (gl + 1 < ngroups) s_next = srow ? __half2float(srow[gl + 1]) : 0.0f;
+                if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
+                if (!tc::mbar_wait(&sh->d_full[db], (g >> 1) & 1, p.status, abort_flag)) goto epi_done;
+                __syncwarp();
+                tc::fence_after_sync();
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(tbase + lane_field + db * BN + half * 64 + 32 * h, v);
+                    tc::tmem_wait_ld();
+                    if constexpr (INT8) {
+                        if (p.acc_dbg && srow) {
+#pragma unroll
+                            for (int j = 0; j < 32; j++) {
+                                const int m = T.m0 + half * 64 + 32 * h + j;
+                                if (m < T.m_end) p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)v[j]) >> 4;
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; j++) acc[32 * h + j] = fmaf(s, (float)(int32_t)v[j], acc[32 * h + j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++) acc[32 * h + j] = fmaf(s, __uint_as_float(v[j]), acc[32 * h + j]);
+                    }
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->d_empty[db]);
+            }
+            // ---------------------------------------------------------- tile output
+            if constexpr (MODE == Mode::Dense) {
+                const int n = T.n0 + r;
+                if (n < p.N) {
+#pragma unroll
+                    for (int j = 0; j < 64; j++) {
+                        const int m = T.m0 + half * 64 + j;
+                        if (m < p.M) {
+                            float v = acc[j];
+                            if constexpr (INT8) v *= p.scale_a[m];
+                            const int64_t o = (int64_t)m * p.N + n;
+                            if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
+                            else reinterpret_cast<float*>(p.y)[o] = v;
+                        }
+                    }
+                }
+            } else if constexpr (MODE == Mode::GateUp) {
+                // rows 64..127 (up) hand their values to rows 0..63 (gate) of the same intermediate index
+                float* xb = xchg + half * 64 * 64;
+                if (r >= 64) {
+                    // the buffer is free once the gate rows consumed the previous tile's values
+                    if (!tc::mbar_wait(&sh->gate_done, (tl & 1) ^ 1, p.status, abort_flag)) goto epi_done;
+#pragma unroll
+                    for (int j = 0; j < 64; j++) xb[j * 64 + (r - 64)] = acc[j];
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sh->up_ready);
+                } else {
+                    if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
+                    const int i = T.n0 + r;
+#pragma unroll
+                    for (int j = 0; j < 64; j++) {
+                        const int m = T.m0 + half * 64 + j;
+                        if (m < T.m_end) {
+                            const float gv = acc[j], uv = xb[j * 64 + r];
+                            const float hv = gv / (1.0f + expf(-gv)) * uv;
+                            p.h[(int64_t)m * p.N + i] = __float2half_rn(hv);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sh->gate_done);
+                }
+            } else {
+                const int n = T.n0 + r;
+                float* yv = reinterpret_cast<float*>(p.y);
+#pragma unroll
+                for (int j = 0; j < 64; j++) {
+                    const int m = T.m0 + half * 64 + j;
+                    if (m < T.m_end) {
+                        const int pair = p.perm[m];
+                        atomicAdd(yv + (int64_t)(pair / p.topk) * p.N + n, p.topk_w[pair] * acc[j]);
+                    }
+                }
+            }
+        }
+    epi_done:;
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+}  // namespace tcg

@@ -1,0 +1,66 @@
+// Host helpers of the tensor-core kernels: TMA tensor-map encoding (driver entry point fetched
+// through the runtime, so the library does not link libcuda) and kernel launch with the opt-in
+// shared-memory size.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "tc_gemm.cuh"
+
+namespace tcg {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 2-D tensor map: `inner` contiguous elements per row, `outer` rows, row pitch in bytes.
+inline bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Activation tile map: [rows][k] of bf16 / fp16 (two 64-column boxes per stage) or int8 (one box).
+inline bool make_act_map(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, int elem_bytes, bool f16)
+{
+    if (elem_bytes == 1)
+        return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, k, rows, k, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    return make_map(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, k, rows,
+                    2 * k, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Packed weight map: [rows][k/2] bytes, boxes of 64 bytes (one K stage) x box_rows rows, 64-byte swizzle.
+inline bool make_packed_map(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, uint32_t box_rows)
+{
+    return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, k / 2, rows, k / 2, KBLK / 2, box_rows,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <bool INT8, int G, bool SYM, Mode MODE>
+int launch(const CUtensorMap& mx, const CUtensorMap& ma, const CUtensorMap& mb, const Args& p, int grid,
+           cudaStream_t s)
+{
+    auto kern = tc_gemm_kernel<INT8, G, SYM, MODE>;
+    constexpr int smem = Cfg<INT8, MODE>::SMEM;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return Q4_ERR_CUDA;
+    kern<<<grid, kThreads, smem, s>>>(mx, ma, mb, p);
+    return q4_launch_status();
+}
+
+}  // namespace tcg

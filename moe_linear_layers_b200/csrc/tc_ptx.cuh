@@ -62,18 +62,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after `limit_ns` of wall time:
-// records Q4_ERR_TIMEOUT in the status word, raises the CTA's abort flag and returns false.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int32_t* status,
+// records Q4_ERR_TIMEOUT in the status word, raises the CTA's abort flag (nullable) and returns false.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int32_t* status,
                                             volatile int* abort_flag, uint64_t limit_ns)
 {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u) {
-            if (*abort_flag) return false;
+            if (abort_flag && *abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 q4_set_status(status, Q4_ERR_TIMEOUT);
-                *abort_flag = 1;
+                if (abort_flag) *abort_flag = 1;
                 return false;
             }
         }
@@ -126,8 +126,9 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate (cta_group::1).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[tmem] * B[smem]^T, 16-bit inputs (bf16 or fp16 per the instruction descriptor),
+// fp32 accumulate (cta_group::1).
+__device__ __forceinline__ void mma_16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate)
 {
     asm volatile(
@@ -203,11 +204,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
 }
 
 // Instruction descriptor: dense, K-major A and B, M = 128, N = n.
-//   c_format bits [4,6): 1 = f32, 2 = s32;  a/b_format bits [7,10)/[10,13): bf16 = 1, s8 = 1 (signed);
+//   c_format bits [4,6): 1 = f32, 2 = s32;  a/b_format bits [7,10)/[10,13): f16 = 0, bf16 = 1, s8 = 1 (signed);
 //   N >> 3 in bits [17,23);  M >> 4 in bits [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t n)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t n)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_s8_s32(uint32_t n)
 {

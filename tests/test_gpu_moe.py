@@ -1,0 +1,97 @@
+"""GPU parity of the MoE layer (route -> permute -> grouped gate/up SwiGLU -> grouped down + combine)
+against the oracle, through the C ABI.
+
+Expert ids, permutation, offsets and counts are bit-exact (the router logits follow a pinned fp32
+reduction order on both sides).  Routing weights: fp32 expf against the fp64 oracle, rtol 1e-5.
+Outputs: max|y - y_ref| <= 1e-2 * rms(y_ref) (fp32 output; the down projection's combine uses float
+atomics, so the last bits vary with the summation order)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_linear_layers_b200 import synth
+from tests._util import REL_TOL, assert_close, cpu_u16, cuda_u16_as, rel_err, upload_weight
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from moe_linear_layers_b200 import q4 as mod
+    return mod
+
+
+def _experts(tag, E, H, I, group, sym):
+    """Stacked expert weights: gate/up [E*I][H], down [E*H][I], quantized by the oracle."""
+    Wg = synth.weights(("moe", tag, "gate"), E * I, H)
+    Wu = synth.weights(("moe", tag, "up"), E * I, H)
+    Wd = synth.weights(("moe", tag, "down"), E * H, I)
+    return [oracle.quantize(W, group, sym) for W in (Wg, Wu, Wd)]
+
+
+def _run(q4, T, H, I, E, topk, group, sym, tag, skew=1.1, tokens=None, out=torch.float32):
+    x = synth.activations(("moe", tag, "x"), T, H)
+    Wr, bias = synth.router(("moe", tag), E, H, skew=skew)
+    qs = _experts(tag, E, H, I, group, sym)
+    logits, ids, w, counts = oracle.route(x, H, Wr, bias, topk)
+    offsets, perm = oracle.permute(ids, E)
+    ref = oracle.moe_experts(x, H, ids, w, qs[0], qs[1], qs[2], I, group, sym, tokens=tokens)
+    ex = (upload_weight(q4, *qs[0], E * I, H, group, sym), upload_weight(q4, *qs[1], E * I, H, group, sym),
+          upload_weight(q4, *qs[2], E * H, I, group, sym))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y, ids_d, w_d, perm_d, off_d, cnt_d = q4.moe_q4_forward(
+        cuda_u16_as(x, torch.bfloat16), torch.from_numpy(Wr).cuda(), torch.from_numpy(bias).cuda(), topk, ex, I,
+        out_dtype=out, want_routing=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(ids_d.cpu().numpy(), ids), "expert ids differ"
+    np.testing.assert_allclose(w_d.cpu().numpy(), w, rtol=1e-5, atol=1e-7)
+    assert np.array_equal(off_d.cpu().numpy(), offsets)
+    assert np.array_equal(perm_d.cpu().numpy(), perm)
+    assert np.array_equal(cnt_d.cpu().numpy(), counts)
+    yn = y.float().cpu().numpy()
+    if tokens is not None:
+        yn = yn[tokens]
+    return yn, ref, counts
+
+
+@pytest.mark.parametrize("T,H,I,E,topk,group,sym", [
+    (64, 256, 128, 8, 2, 128, False),     # small, every expert busy
+    (37, 256, 256, 5, 3, 64, True),       # ragged token count, group 64, symmetric
+    (16, 128, 128, 1, 1, 128, False),     # a single expert: a dense SwiGLU FFN
+    (200, 512, 256, 64, 8, 128, False),   # the workload's expert count / top-8, skewed: some experts empty
+])
+def test_moe_small(q4, T, H, I, E, topk, group, sym):
+    yn, ref, counts = _run(q4, T, H, I, E, topk, group, sym, f"s{T}-{E}")
+    assert_close(yn, ref, what="moe")
+
+
+def test_moe_bf16_output(q4):
+    yn, ref, _ = _run(q4, 48, 256, 128, 8, 2, 128, False, "bf16", out=torch.bfloat16)
+    # bf16 rounding of the output adds at most 2^-8 |y| on top of the stated bar
+    err = np.abs(yn.astype(np.float64) - ref)
+    rms = np.sqrt(np.mean(ref * ref))
+    assert np.all(err <= REL_TOL * rms + 2.0 ** -8 * np.abs(ref))
+
+
+def test_moe_workload_full_size(q4):
+    """4096 tokens, hidden 2048, 64 experts of intermediate 1024, top-8, asymmetric group 128, router
+    logits Zipf-skewed (bias -1.1 ln(e+1)): routing checked for every token, outputs on a sample."""
+    tokens = np.arange(0, 4096, 97)
+    yn, ref, counts = _run(q4, 4096, 2048, 1024, 64, 8, 128, False, "full", tokens=tokens)
+    assert_close(yn, ref, what="moe full")
+    assert counts[0] > counts[-1]    # the skew is visible
+
+
+def test_moe_workspace_too_small(q4):
+    from moe_linear_layers_b200.q4 import Q4Error, Q4_ERR_WORKSPACE
+    T, H, I, E, topk = 32, 128, 128, 4, 2
+    qs = _experts("ws", E, H, I, 128, True)
+    ex = tuple(upload_weight(q4, *qq, n, k, 128, True) for qq, n, k in zip(qs, (E * I, E * I, E * H), (H, H, I)))
+    x = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    Wr = torch.zeros((E, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Q4Error) as ei:
+        q4.moe_q4_forward(x, Wr, None, topk, ex, I, workspace=ws)
+    assert ei.value.status == Q4_ERR_WORKSPACE
