@@ -172,6 +172,36 @@ int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H,
                    int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/*
+ * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate device memory.
+ * No counterpart in the source pages: this is a library convenience, not part of the method.
+ *
+ * Some callers have no way to obtain device memory for the workspace: a plugin loaded into a host
+ * application that owns all device memory and hands out no allocator, or a latency-critical loop in
+ * which a cudaMalloc (which can synchronise the device) is not acceptable.  This entry point takes the
+ * same arguments as moe_q4_forward minus the workspace, and uses instead one fixed scratch array that
+ * the library holds in device memory (a file-scope __device__ array of Q4_MOE_NOALLOC_SCRATCH_BYTES,
+ * 256-byte aligned).  Every GPU on which the library is loaded holds that array until the process
+ * exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Sizes whose moe_q4_workspace_size(T, H, I, E, topk) exceeds Q4_MOE_NOALLOC_SCRATCH_BYTES are
+ *     rejected with Q4_ERR_WORKSPACE before anything is launched (for H = 2048, I = 1024, top-8 that
+ *     is roughly T > 580 tokens).
+ *   - The first call on a device looks up the array's device address with cudaGetSymbolAddress while
+ *     that device is current, and caches it; make that first call on each device before any stream
+ *     capture begins.
+ *   - All calls share the one array, which keeps the last call's contents (every call overwrites
+ *     what it reads).  Calls that overlap on the GPU (for example on two streams) race on it: keep
+ *     them ordered on one stream or serialise them.
+ */
+#define Q4_MOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+int moe_q4_forward_noalloc(const uint16_t* x, int32_t T, int32_t H,
+                           const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                           const q4_weight* experts, int32_t I,
+                           void* y, int32_t out_dtype,
+                           int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                           int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,6 +18,8 @@
 //   5. down      grouped tcgen05 GEMM over (expert, token tile, 128 hidden rows) tiles whose epilogue
 //                adds w[t][j] * out into the fp32 output (float atomics: the sum order is not fixed);
 //   6. (bf16 output) a conversion pass.
+#include <mutex>
+
 #include "tc_host.cuh"
 
 namespace {
@@ -366,4 +368,43 @@ extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const flo
         rc = q4_launch_status();
     }
     return rc;
+}
+
+// ---------------------------------------------------------------------------------------------- //
+// moe_q4_forward without a caller workspace (for callers that cannot allocate device memory; see
+// include/q4.h).  The scratch is one file-scope device array shared by every call; its device address
+// is looked up once per device with cudaGetSymbolAddress (host code must not use the array's name
+// as a device pointer) and then passed to moe_q4_forward as the workspace.
+// ---------------------------------------------------------------------------------------------- //
+static __device__ __align__(256) uint8_t q4_moe_noalloc_scratch[Q4_MOE_NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_scratch_address(void** out)
+{
+    static void* cache[64] = {nullptr};
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return Q4_ERR_CUDA;
+    std::lock_guard<std::mutex> guard(lock);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, q4_moe_noalloc_scratch) != cudaSuccess || !p) return Q4_ERR_CUDA;
+        cache[dev] = p;
+    }
+    *out = cache[dev];
+    return Q4_OK;
+}
+
+extern "C" int moe_q4_forward_noalloc(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                      const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts,
+                                      int32_t I, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
+                                      int32_t* perm, int32_t* offsets, int32_t* expert_counts, int32_t* dev_status,
+                                      void* stream)
+{
+    const size_t need = moe_q4_workspace_size(T, H, I, E, topk);
+    if (need > Q4_MOE_NOALLOC_SCRATCH_BYTES) return Q4_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch_address(&scratch);
+    if (rc) return rc;
+    return moe_q4_forward(x, T, H, router_w, router_bias, E, topk, experts, I, y, out_dtype, topk_ids, topk_w, perm,
+                          offsets, expert_counts, scratch, Q4_MOE_NOALLOC_SCRATCH_BYTES, dev_status, stream);
 }

@@ -32,7 +32,9 @@ Q4_OUT_F32 = 0
 Q4_OUT_BF16 = 1
 
 EXPORTED = ("q4_status_string", "q4_version", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
-            "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward")
+            "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
+            "moe_q4_forward_noalloc")
+Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class q4_weight(ctypes.Structure):
@@ -54,6 +56,8 @@ _lib.moe_q4_workspace_size.restype = _sz
 _lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p, _i32,
                                 _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
+                                        _i32, _p, _p, _p, _p, _p, _p, _p]
 
 
 class Q4Error(RuntimeError):
@@ -201,4 +205,25 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
                                workspace.numel(), _ptr(dev_status), _stream(stream)), "moe_q4_forward")
     if want_routing:
         return y, ids, wts, perm, offs, cnts
+    return y
+
+
+def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                           experts: tuple, I: int, out_dtype=torch.float32, y: torch.Tensor | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_q4_forward using the library's fixed device scratch instead of a caller workspace, for callers
+    that cannot allocate device memory (see include/q4.h).  Sizes needing more than
+    Q4_MOE_NOALLOC_SCRATCH_BYTES of scratch raise Q4Error(Q4_ERR_WORKSPACE).  Calls share the scratch:
+    keep them ordered on one stream."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    if y is None:
+        y = torch.empty((T, H), dtype=out_dtype, device=x.device)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _check(_lib.moe_q4_forward_noalloc(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, _ptr(y),
+                                       od, None, None, None, None, None, _ptr(dev_status), _stream(stream)),
+           "moe_q4_forward_noalloc")
     return y
