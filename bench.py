@@ -1,14 +1,22 @@
-"""Benchmark of the INT4 linear-layer hot path on B200.
+"""Benchmark of the INT4 linear-layer hot path on B200 (one JSON line on rank 0).
 
-Default workload (one JSON line): the LLaMA-3.2-1B-shaped decode step, W4A16 at m = 1: 16 layers x
-{q 2048x2048, k 512x2048, v 512x2048, o 2048x2048, gate 8192x2048, up 8192x2048, down 2048x8192},
-asymmetric group-128 INT4, bf16 activations ~N(0,1), fp32 outputs.  One step = the 112 GEMVs.
-Metric: HBM GB/s = algorithmic bytes (packed weights + scales + zeros + x + y) / step time.
+Headline workload: the LLaMA-3.2-1B-shaped decode step, W4A16 at m = 1 -- 16 layers x {q 2048x2048,
+k 512x2048, v 512x2048, o 2048x2048, gate 8192x2048, up 8192x2048, down 2048x8192}, asymmetric
+group-128 INT4 weights ~N(0, 0.02^2) with 0.1% outliers x20, bf16 activations ~N(0, 1), fp32
+outputs.  One step = the 112 GEMVs (q4_linear_w4a16), replayed as a CUDA graph.
+Metric: HBM GB/s = algorithmic bytes (packed weights + fp16 scales + fp16 zeros + bf16 x + fp32 y)
+of the step / device time of the step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+At one GPU the line also carries "components", the other rows of the hot path on their workloads:
+  prefill  W4A16 GEMM, m = 2048, the same 112 weight matrices, x with 1% of channels x10 (TFLOP/s);
+  w4a8     per-token INT8 act-quant + W4A8 GEMM, m = 4096, the same shapes quantized symmetrically,
+           Student-t(3) activations (TOPS);
+  moe      the MoE layer: 4096 tokens, hidden 2048, 64 experts of intermediate 1024, top-8 (tokens/s).
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs an independent replica of the step (the
-decode step has no data exchange); value = bytes of all ranks / max-over-ranks time.
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
+
+Multi-GPU (torchrun): every rank runs an independent replica of the decode step (the step has no data
+exchange); value = bytes of all ranks / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -16,7 +24,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -30,6 +37,7 @@ sys.path.insert(0, ROOT)
 from moe_linear_layers_b200 import synth  # noqa: E402
 
 METRIC = "INT4 GEMV HBM GB/s (M=1); W4A16/W4A8 GEMM TOPS; MoE layer tokens/s"
+MOE = dict(T=4096, H=2048, I=1024, E=64, topk=8)
 
 
 # ------------------------------------------------------------------------------------------------ #
@@ -56,154 +64,172 @@ def barrier(ws):
 
 
 def max_over_ranks(v: float, ws: int) -> float:
+    """The largest value over all ranks (every rank takes part; NCCL on GPUs, gloo on CPU)."""
     if ws == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
 
 # ------------------------------------------------------------------------------------------------ #
-# clocks sampled during the timed region
+# clocks sampled during the timed region (NVML, every 10 ms)
 # ------------------------------------------------------------------------------------------------ #
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, device: int):
-        # nvidia-smi numbers GPUs differently from CUDA under CUDA_VISIBLE_DEVICES: select by UUID
+    def __init__(self, device: int, period_s: float = 0.01):
+        self.period, self.samples, self.reasons, self.handle, self.max_mhz = period_s, [], set(), None, None
+        self.power = []
         try:
-            u = str(torch.cuda.get_device_properties(device).uuid)
-            self.index = u if u.startswith("GPU-") else f"GPU-{u}"
-        except Exception:
-            self.index = str(device)
-        self.proc, self.lines = None, []
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.nv = nv
+            self.handle = nv.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.error = repr(e)
+            self.handle = None
+
+    def _run(self):
+        nv = self.nv
+        names = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                 "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        while not self.stop:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+                self.power.append(nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+        self.stop = False
+        if self.handle is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
-        except OSError:
-            self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop = True
+        if self.handle is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "power_w_max": round(max(self.power), 1) if self.power else None}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained") or d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def traffic_from_profiles(name):
+    """DRAM bytes per launch recorded from an ncu capture of the current kernel, or None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        return json.load(open(p)).get(name)
+    return None
+
+
+def graph_of(fn):
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_replays(g, steps, ws, sampler=None):
+    stream = torch.cuda.current_stream()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with (sampler if sampler is not None else _Null()):
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    return max_over_ranks(e0.elapsed_time(e1), ws)
+
+
+def dev_bf16(a_u16, dev):
+    return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).to(dev).view(torch.bfloat16)
 
 
 # ------------------------------------------------------------------------------------------------ #
-# the decode workload (LLaMA-3.2-1B shapes, W4A16, m = 1)
+# workloads
 # ------------------------------------------------------------------------------------------------ #
-
-def decode_bytes(layers):
-    """Algorithmic HBM bytes of one decode step: packed weights, fp16 scales and zeros, bf16 x, fp32 y."""
-    total = 0
-    for (_, n, k) in layers:
-        total += n * k // 2 + 2 * 2 * n * (k // 128) + 2 * k + 4 * n
-    return total
-
 
 def decode_layers(n_layers=synth.LLAMA_1B_LAYERS):
     return [(f"L{l}.{nm}", n, k) for l in range(n_layers) for (nm, n, k) in synth.LLAMA_1B_LINEARS]
 
 
-def build_decode(q4, dev, seed=0):
-    """Quantize the 112 weight matrices on the device (the product's quantizer) and make the inputs."""
-    weights, xs, ys = [], [], []
+def decode_bytes(layers):
+    """Algorithmic HBM bytes of one decode step: packed weights, fp16 scales and zeros, bf16 x, fp32 y."""
+    return sum(n * k // 2 + 2 * 2 * n * (k // 128) + 2 * k + 4 * n for (_, n, k) in layers)
+
+
+def build_weights(q4, dev, symmetric_too: bool, seed=0):
+    """The 112 weight matrices quantized on the device (asymmetric, and symmetric when asked)."""
+    asym, sym = [], []
     for (name, n, k) in decode_layers():
         W = torch.from_numpy(synth.weights((seed, "llama1b", name), n, k)).to(dev)
-        weights.append(q4.q4_quantize_pack(W, 128, False))
+        asym.append(q4.q4_quantize_pack(W, 128, False))
+        if symmetric_too:
+            sym.append(q4.q4_quantize_pack(W, 128, True))
         del W
-        x = synth.activations((seed, "llama1b-decode-x", name), 1, k)
-        xs.append(torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16))
-        ys.append(torch.empty((1, n), dtype=torch.float32, device=dev))
     torch.cuda.synchronize()
-    return weights, xs, ys
+    return asym, sym
 
 
-def run_decode(args, ws, rank):
-    from moe_linear_layers_b200 import q4
-    dev = torch.device("cuda", torch.cuda.current_device())
+def run_decode(q4, args, ws, weights, dev):
     layers = decode_layers()
-    weights, xs, ys = build_decode(q4, dev)
+    xs = [dev_bf16(synth.activations((0, "llama1b-decode-x", name), 1, k), dev) for (name, n, k) in layers]
+    ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for (_, n, k) in layers]
     bytes_step = decode_bytes(layers)
-    stream = torch.cuda.current_stream()
 
     def step():
         for w, x, y in zip(weights, xs, ys):
             q4.q4_linear_w4a16(x, w, y=y)
 
-    # CUDA graph of one step (112 launches of the public call), replayed K times.
-    for _ in range(2):
-        step()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        step()
+    g = graph_of(step)
     for _ in range(args.warmup):
         g.replay()
     torch.cuda.synchronize()
-
-    # per-launch durations of the dominant kernel (events around each launch, outside the timed region)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(weights) + 1)]
-    for rep in range(3):
-        ev[0].record()
-        for i, (w, x, y) in enumerate(zip(weights, xs, ys)):
-            q4.q4_linear_w4a16(x, w, y=y)
-            ev[i + 1].record()
-    torch.cuda.synchronize()
-    per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(weights))]
-
-    barrier(ws)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    ms = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms, ws)
+    clk = ClockSampler(torch.cuda.current_device())
+    ms = time_replays(g, args.steps, ws, clk)
     ms_step = ms / args.steps
     value = ws * bytes_step * args.steps / (ms * 1e-3) / 1e9
 
-    # end to end through the public call with host buffers: pinned x in, y back to the host
+    # end to end through the public call with host buffers: pinned x in, y back to the host, eager
     hx = [x.cpu().pin_memory() for x in xs]
     hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
     h2d = sum(t.numel() * t.element_size() for t in hx)
@@ -220,6 +246,7 @@ def run_decode(args, ws, rank):
         e2e_step()
     torch.cuda.synchronize()
     barrier(ws)
+    stream = torch.cuda.current_stream()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(args.steps):
@@ -230,48 +257,131 @@ def run_decode(args, ws, rank):
     e2e_val = ws * bytes_step * args.steps / (ms_e2e * 1e-3) / 1e9
 
     peaks = load_peaks()
-    # dominant kernel: the GEMV; achieved = algorithmic bytes of the step / step time of the graph
-    roof = {"bound": "hbm", "achieved": round(value / ws, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(value / ws / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles("gemv_decode"),
-            "peak_source": peaks["source"],
-            "per_launch_us": {"mean": round(1e3 * float(np.mean(per_launch_ms)), 3),
-                              "gate_up_8192x2048": round(1e3 * float(np.mean([per_launch_ms[i] for i, l in
-                                                                               enumerate(layers) if l[0].endswith(('gate', 'up'))])), 3),
-                              "kv_512x2048": round(1e3 * float(np.mean([per_launch_ms[i] for i, l in
-                                                                         enumerate(layers) if l[0].endswith(('.k', '.v'))])), 3)}}
-    line = {
+    per_gpu = value / ws
+    return {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "llama-3.2-1b-shaped decode step, W4A16 GEMV m=1, 16 layers x 7 linears, "
-                               "asymmetric INT4 group 128, fp32 out",
+        "config": {"workload": "llama-3.2-1b-shaped decode step: W4A16 GEMV m=1 over 16 layers x 7 linears "
+                               "(q,k,v,o 2048/512/512/2048 x 2048, gate/up 8192x2048, down 2048x8192), "
+                               "asymmetric INT4 group 128, bf16 x ~N(0,1), fp32 y",
                    "linears_per_step": len(layers), "bytes_per_step": bytes_step,
-                   "l2": "working set %.0f MB > 126 MB L2; no flush needed" % (bytes_step / 1e6),
-                   "parallelism": f"replicas x{ws}", "launch": "CUDA graph of 112 q4_linear_w4a16 calls"},
-        "roofline": roof,
+                   "l2": "no flush: the step streams %.0f MB of weights, > 126 MB L2" % (bytes_step / 1e6),
+                   "launch": "CUDA graph of 112 q4_linear_w4a16 calls (programmatic dependent launch)",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(per_gpu / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles("gemv_decode"),
+                     "peak_source": peaks["source"] + " (HBM copy bandwidth)",
+                     "kernel": "w4a16_gemv_kernel; achieved = algorithmic bytes of the step / step time = "
+                               "bytes per launch / mean launch duration (graph replay, gaps included)",
+                     "mean_launch_us": round(1e3 * ms_step / len(layers), 3)},
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "eager public-API calls, pinned host x copied in and y copied out every step"},
-        "gpu_launches": len(weights) * args.steps,
+                "how": "eager public-API calls per linear; pinned host x copied in and y copied out every step"},
+        "gpu_launches": len(layers) * args.steps,
         "clocks": clk.summary(),
     }
-    return line
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+def run_prefill(q4, args, weights, dev, m=2048):
+    layers = decode_layers()
+    xk = {k: dev_bf16(synth.activations((0, "llama1b-prefill-x", k), m, k, "outlier_channels"), dev)
+          for k in sorted({k for (_, _, k) in layers})}
+    yn = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in sorted({n for (_, n, _) in layers})}
+
+    def step():
+        for w, (_, n, k) in zip(weights, layers):
+            q4.q4_linear_w4a16(xk[k], w, y=yn[n])
+
+    g = graph_of(step)
+    for _ in range(3):
+        g.replay()
+    steps = max(3, min(args.steps, 10))
+    clk = ClockSampler(torch.cuda.current_device())
+    ms = time_replays(g, steps, 1, clk) / steps
+    flops = 2 * m * sum(n * k for (_, n, k) in layers)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    return {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 3), "m": m,
+            "workload": "W4A16 GEMM over the 112 decode-step matrices at m=2048, x with 1% channels x10, bf16 out",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+                         "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4),
+                         "peak_source": peaks["source"] + " (cuBLAS bf16, sustained)"},
+            "gpu_launches": len(layers) * steps, "clocks": clk.summary()}
 
 
-def traffic_from_profiles(name):
-    """DRAM bytes per launch recorded from an ncu capture of the current kernel (profiles/*.json), or None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        return json.load(open(p)).get(name)
-    return None
+def run_w4a8(q4, args, weights_sym, dev, m=4096):
+    layers = decode_layers()
+    xk = {k: dev_bf16(synth.activations((0, "llama1b-w4a8-x", k), m, k, "student_t3"), dev)
+          for k in sorted({k for (_, _, k) in layers})}
+    xq = {k: torch.empty((m, k), dtype=torch.int8, device=dev) for k in xk}
+    sa = torch.empty((m,), dtype=torch.float32, device=dev)
+    yn = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in sorted({n for (_, n, _) in layers})}
+
+    def step():
+        for w, (_, n, k) in zip(weights_sym, layers):
+            q4.act_quant_per_token(xk[k], xq=xq[k], scale_a=sa)
+            q4.q4_linear_w4a8(xq[k], sa, w, y=yn[n])
+
+    g = graph_of(step)
+    for _ in range(3):
+        g.replay()
+    steps = max(3, min(args.steps, 10))
+    clk = ClockSampler(torch.cuda.current_device())
+    ms = time_replays(g, steps, 1, clk) / steps
+    ops = 2 * m * sum(n * k for (_, n, k) in layers)
+    tops = ops / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    int8_peak = 2 * peaks["bf16_tflops_sustained"]
+    return {"value": round(tops, 1), "unit": "TOPS", "ms_per_step": round(ms, 3), "m": m,
+            "workload": "per-token INT8 act-quant + W4A8 GEMM over the 112 matrices (symmetric INT4 g128), "
+                        "m=4096, Student-t(3) activations, bf16 out; act-quant time included",
+            "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
+                         "frac": round(tops / int8_peak, 4),
+                         "peak_source": peaks["source"] + " bf16 sustained x 2 (nominal int8:bf16 dense ratio)"},
+            "gpu_launches": 2 * len(layers) * steps, "clocks": clk.summary()}
+
+
+def build_moe(q4, dev, seed=0):
+    T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+    ex = []
+    for nm, n, k in (("gate", E * I, H), ("up", E * I, H), ("down", E * H, I)):
+        W = torch.from_numpy(synth.weights((seed, "moe", nm), n, k)).to(dev)
+        ex.append(q4.q4_quantize_pack(W, 128, False))
+        del W
+    x = dev_bf16(synth.activations((seed, "moe", "x"), T, H), dev)
+    Wr, bias = synth.router((seed, "moe"), E, H)
+    return x, torch.from_numpy(Wr).to(dev), torch.from_numpy(bias).to(dev), tuple(ex)
+
+
+def run_moe(q4, args, dev):
+    T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+    x, Wr, bias, ex = build_moe(q4, dev)
+    ws_t = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+
+    g = graph_of(lambda: q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_t))
+    for _ in range(3):
+        g.replay()
+    steps = max(3, min(args.steps, 20))
+    clk = ClockSampler(torch.cuda.current_device())
+    ms = time_replays(g, steps, 1, clk) / steps
+    _, ids, _, _, _, counts = q4.moe_q4_forward(x, Wr, bias, topk, ex, I, workspace=ws_t, want_routing=True)
+    c = counts.cpu().numpy()
+    flops = 2 * T * topk * 3 * H * I
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "workload": "MoE layer: 4096 tokens, hidden 2048, 64 SwiGLU experts of intermediate 1024, top-8, "
+                        "asymmetric INT4 g128, fp32 router with Zipf-skewed logits (bias -1.1 ln(e+1)), fp32 out",
+            "tflops": round(tf, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+                         "peak_source": peaks["source"] + " (cuBLAS bf16, sustained)",
+                         "algorithmic_flop": flops},
+            "expert_counts": {"max": int(c.max()), "mean": float(c.mean()), "min": int(c.min()),
+                              "empty": int((c == 0).sum())},
+            "gpu_launches": 6 * steps, "clocks": clk.summary()}
 
 
 # ------------------------------------------------------------------------------------------------ #
@@ -280,7 +390,7 @@ def traffic_from_profiles(name):
 
 def oracle_decode_sample(rows_per_linear=128):
     """The oracle over the first rows of layer 0's seven linears (same weights and x as the device run).
-    Returns (bytes processed, seconds, threads)."""
+    Returns (bytes processed, seconds)."""
     import oracle
     jobs = []
     for (name, n, k) in decode_layers(1):
@@ -293,21 +403,24 @@ def oracle_decode_sample(rows_per_linear=128):
         oracle.linear_w4a16(x, pk, sc, zr, n, k, 128, False)
     dt = time.perf_counter() - t0
     nbytes = sum(n * k // 2 + 4 * n * (k // 128) + 2 * k + 4 * n for (_, _, _, _, n, k) in jobs)
-    return nbytes, dt, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return nbytes, dt
 
 
-def cpu_baseline_decode():
-    nbytes, dt, cores = oracle_decode_sample()
-    reps = max(1, int(10.0 / max(dt, 1e-3)))
-    reps = min(reps, 200)
-    total_b, total_t = 0, 0.0
+def oracle_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline_decode(budget_s=10.0):
+    b, t = oracle_decode_sample()
+    reps = int(min(200, max(1, budget_s / max(t, 1e-3))))
+    tb, tt = 0, 0.0
     for _ in range(reps):
-        b, t, _ = oracle_decode_sample()
-        total_b += b
-        total_t += t
-    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} passes of the oracle over the first 128 rows of layer 0's 7 linears "
-                      "(W4A16 m=1, fp64 accumulation)"}
+        b, t = oracle_decode_sample()
+        tb += b
+        tt += t
+    return {"value": round(tb / tt / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{reps} passes of the oracle (fp64, OpenMP over output rows) over the first 128 rows of "
+                      "layer 0's 7 linears, W4A16 m=1"}
 
 
 def run_reference(args, ws, rank):
@@ -318,17 +431,18 @@ def run_reference(args, ws, rank):
         oracle_decode_sample()
     tb, tt = 0, 0.0
     for _ in range(args.steps):
-        b, t, cores = oracle_decode_sample()
+        b, t = oracle_decode_sample()
         tb += b
         tt += t
     v = tb / tt / 1e9
+    sample = "first 128 rows of layer 0's 7 linears per step (W4A16 m=1, fp64)"
     return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tt / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama-3.2-1b-shaped decode step, W4A16 GEMV m=1 (oracle sample: first 128 rows "
-                                   "of layer 0's 7 linears per step)", "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": "first 128 rows of layer 0's 7 linears per step"},
+            "config": {"workload": "llama-3.2-1b-shaped decode step, W4A16 GEMV m=1 (oracle on a sample: "
+                                   + sample + ")", "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -338,21 +452,29 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
     if args.impl == "reference":
-        ws = int(os.environ.get("WORLD_SIZE", "1"))
-        rank = int(os.environ.get("RANK", "0"))
-        line = run_reference(args, ws, rank)
+        line = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         if line is not None:
             print(json.dumps(line), flush=True)
         return
 
+    args.warmup = max(args.warmup, 3)
     ws, rank, local = dist_setup()
-    line = run_decode(args, ws, rank)
+    from moe_linear_layers_b200 import q4
+    dev = torch.device("cuda", torch.cuda.current_device())
+    components = ws == 1 and not args.no_components
+    asym, sym = build_weights(q4, dev, symmetric_too=components)
+    line = run_decode(q4, args, ws, asym, dev)
+    if components:
+        line["components"] = {"prefill_w4a16_m2048": run_prefill(q4, args, asym, dev),
+                              "w4a8_m4096": run_w4a8(q4, args, sym, dev)}
+        del sym
+        torch.cuda.empty_cache()
+        line["components"]["moe_layer"] = run_moe(q4, args, dev)
     if rank == 0:
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_decode()
