@@ -104,11 +104,24 @@ int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t group, int32_
  * the fp32 result).  m >= 1.  Small m runs the memory-bound GEMV kernel (CUDA cores, in-register
  * dequant); larger m runs the tcgen05 tensor-core GEMM (exact integer codes in bf16, fp32
  * accumulation per group, scale applied per group in the epilogue).  The choice is by shape only.
- * Requires k % 32 == 0 for the GEMV and k % 128 == 0 for the GEMM (see q4_linear_w4a16_max_gemv_m).
+ * The GEMV serves k % 64 == 0, k <= 16384; the GEMM serves k % 128 == 0 (see q4_linear_w4a16_max_gemv_m).
+ * The GEMV may begin streaming W into L2 before the previous kernel on the stream has finished
+ * (programmatic dependent launch); it reads x only after that kernel's writes are visible.
  * dev_status: Q4_ERR_NONFINITE when x holds a non-finite value (GEMV path).
  */
 int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
                     int32_t* dev_status, void* stream);
+
+/*
+ * q4_linear_w4a16_grouped -- up to 8 independent small-m W4A16 products in one launch:
+ * y[i] = x[i] . dequant(W[i])^T for i < count, each exactly as q4_linear_w4a16 with m <= 4 computes it.
+ * Source: as q4_linear_w4a16; the grouping is a launch-level choice (independent linears of one layer
+ * -- q, k, v, or gate and up -- need not wait for each other), not part of the method.
+ * x, w, y are HOST arrays of `count` entries (device pointers / descriptors).  Every w[i] has the
+ * same k (k % 64 == 0, k <= 16384), group and symmetry; n may differ.  1 <= m <= 4, the same for all.
+ */
+int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, int32_t m, const q4_weight* w,
+                            void* const* y, int32_t out_dtype, int32_t* dev_status, void* stream);
 
 /* Largest m that q4_linear_w4a16 serves with the GEMV kernel. */
 int q4_linear_w4a16_max_gemv_m(void);

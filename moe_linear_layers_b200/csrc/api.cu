@@ -1,8 +1,8 @@
 // Host side of the C ABI: argument validation and dispatch by shape.  See include/q4.h.
 #include "q4_common.cuh"
 
-int q4_gemv_w4a16_launch(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
-                         int32_t* dev_status, cudaStream_t stream);
+int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, const q4_weight* w, void* const* y,
+                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream);
 int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                       int32_t out_dtype, int32_t* acc_dbg, bool int8_path, int32_t* dev_status,
                       cudaStream_t stream);
@@ -52,12 +52,30 @@ extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w,
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(x) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
     if (m == 0 || w->n == 0) return Q4_OK;
-    if (m <= kMaxGemvM && w->k % 32 == 0) {
-        const int rc = q4_gemv_w4a16_launch(x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
+    if (m <= kMaxGemvM && w->k % 64 == 0) {
+        void* ys[1] = {y};
+        const int rc = q4_gemv_w4a16_launch_group(1, &x, m, w, ys, out_dtype, dev_status, (cudaStream_t)stream);
         if (rc != Q4_ERR_UNSUPPORTED) return rc;  // shapes the GEMV cannot stage go to the GEMM
     }
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
     return q4_gemm_tc_launch(x, nullptr, m, w, y, out_dtype, nullptr, false, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, int32_t m, const q4_weight* w,
+                                       void* const* y, int32_t out_dtype, int32_t* dev_status, void* stream)
+{
+    if (!x || !w || !y) return Q4_ERR_NULL;
+    if (count < 1 || count > 8 || m < 1 || m > kMaxGemvM) return Q4_ERR_SHAPE;
+    for (int i = 0; i < count; i++) {
+        const int rc = check_weight(&w[i], false);
+        if (rc) return rc;
+        if (!x[i] || !y[i]) return Q4_ERR_NULL;
+        if (!q4_aligned16(x[i]) || !q4_aligned16(y[i])) return Q4_ERR_ALIGN;
+        if (w[i].k != w[0].k || w[i].group != w[0].group || w[i].symmetric != w[0].symmetric) return Q4_ERR_SHAPE;
+    }
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (w[0].k % 64 || w[0].k > 16384) return Q4_ERR_UNSUPPORTED;
+    return q4_gemv_w4a16_launch_group(count, x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
 }
 
 extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,

@@ -1,47 +1,58 @@
-// W4A16 GEMV for small m (decode): y[m][n] = sum_g s[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x[m][k].
+// W4A16 GEMV for small m (decode): y[m][n] = sum_g s[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x[m][k],
+// for one weight matrix or a group of independent ones in a single launch.
 //
 // Source: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" §2.1 (4-bit storage restored to a
 // 16-bit type before the multiply) and §1 (small model, small batch: memory bound).
 //
 // HBM-bound design (the packed weights are streamed exactly once):
-//  * persistent CTAs, one per SM, each owning a contiguous block of weight rows;
-//  * a producer thread streams the block through a 5-stage shared-memory ring with cp.async.bulk
-//    (16 KB per stage: whole rows are contiguous in memory), completion tracked by mbarriers, so
-//    ~80 KB per SM are in flight without any register-held loads;
+//  * each CTA owns a contiguous block of weight rows of one problem; a producer thread streams the
+//    block (packed rows, and their scales and zeros, all contiguous in memory) through a 4-stage
+//    shared-memory ring with cp.async.bulk, completion tracked by mbarriers;
 //  * programmatic dependent launch: the CTA pulls its rows into L2 (a coherent prefetch) before it
-//    waits for the previous kernel on the stream, so consecutive GEMVs keep HBM busy across the
+//    waits for the previous kernel on the stream, so consecutive launches keep HBM busy across the
 //    kernel boundary; x (which the previous kernel may produce) is read only after the wait;
-//  * x is converted once per CTA into fp16 pairs (power-of-two prescale so max|x| < 2, exact) and
-//    held in registers by the lanes that use it;
+//  * small CTAs (8 compute warps + 1 producer, few registers, ~70 KB shared memory) so that the next
+//    launch's CTAs can be resident, and prefetching, while this launch finishes;
+//  * every lane converts its own 64 values of x to fp16 pairs with its own power-of-two prescale
+//    (max |x| * p in [1, 2): exact), so no block-wide reduction precedes the weight stream;
 //  * in-register dequant: one LOP3 turns two nibbles into fp16x2 "1024 + code"; an HSUB2 of
 //    (1024 + zero) leaves the exact integer (code - zero); nibbles 1, 3, 5, 7 of a word are used in
-//    place (16 * code) and accumulate separately (scaled by 1/16 once per chunk); products accumulate
-//    in fp16x2 over one 32-code chunk (8 products per half) and then in fp32 times the group scale;
-//  * lanes split a row into 16-byte chunks (coalesced, bank-conflict-free shared reads); rows longer
-//    than 2048 codes are split over 2..8 warps and combined through shared memory.
+//    place (16 * code) and accumulate separately (scaled by 1/16 once per group); products accumulate
+//    in fp16x2 over the lane's 2 chunks of one group (16 products per half), then in fp32 times the
+//    group scale; a lane's two 16-byte chunks are adjacent, so they share one group and one scale;
+//  * rows longer than 2048 codes are split over 2..8 warps and combined through shared memory.
 #include "q4_common.cuh"
 #include "tc_ptx.cuh"
 
 namespace {
 
-constexpr int kComputeWarps = 16;
+constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = kComputeWarps * 32;
 constexpr int kThreads = kComputeThreads + 32;      // + one producer warp
-constexpr int kStageBytes = 16384;
-constexpr int kStages = 5;
-constexpr int kScaleBytes = 16384;                  // the CTA's scales (+ zeros) in shared memory
+constexpr int kWeightStage = 16384;                 // packed bytes per stage
+constexpr int kStages = 4;
 constexpr int kMaxM = 4;
+constexpr int kMaxProblems = 8;
+
+struct Problem {
+    const uint16_t* x;       // [m][k] bf16
+    const uint8_t* packed;   // [n][k/2]
+    const __half* scales;    // [n][k/group]
+    const __half* zeros;     // [n][k/group] or null
+    void* y;                 // [m][n]
+    int n;
+    int cta_begin;           // first CTA of this problem
+};
 
 struct GemvParams {
-    const uint16_t* x;
-    const uint8_t* packed;
-    const __half* scales;
-    const __half* zeros;
-    void* y;
+    Problem prob[kMaxProblems];
+    int count;
+    int m, k, group, out_bf16;
+    int rows_per_cta;        // contiguous weight rows per CTA
+    int rows_per_stage;
+    int stage_bytes;         // weights + scales (+ zeros) of one stage, 16-byte multiple
+    int bulk_scales;         // scales/zeros travel in the stages (16-byte aligned rows of scales)
     int32_t* status;
-    int m, n, k, group, out_bf16;
-    int rows_per_cta;    // contiguous weight rows per CTA
-    int rows_per_stage;  // rows per 16 KB stage
 };
 
 // Nibble -> fp16x2 magic: (u & mask) ^ key, key = 0x6400 (1024.0) in both halves, plus the flip of
@@ -63,9 +74,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2_range(const uint8_t* lo, const uint8_t* hi)
+__device__ __forceinline__ void prefetch_l2_range(const void* lo_, const void* hi_)
 {
-    const uintptr_t a = ((uintptr_t)lo + 15) & ~(uintptr_t)15, b = (uintptr_t)hi & ~(uintptr_t)15;
+    const uintptr_t a = ((uintptr_t)lo_ + 15) & ~(uintptr_t)15, b = (uintptr_t)hi_ & ~(uintptr_t)15;
     for (uintptr_t q = a; q < b; q += 65536) prefetch_l2((const void*)q, (uint32_t)min((uintptr_t)65536, b - q));
 }
 
@@ -111,32 +122,59 @@ __device__ __forceinline__ void word_dot(uint32_t u, __half2 b1, __half2 b16, co
     acc16 = __hfma2(d3, u32_as_h2(X.w), acc16);
 }
 
-__device__ __forceinline__ float fold(__half2 acc1, __half2 acc16)
+// x pairs of one word (8 bf16 values e[0..3]) with prescale p, in the order word_dot consumes them.
+__device__ __forceinline__ uint4 x_pairs(const uint4& v, float p)
 {
-    const float2 f = __half22float2(__hfma2(acc16, __float2half2_rn(0.0625f), acc1));
-    return f.x + f.y;
+    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        f[2 * i] = __uint_as_float(e[i] << 16) * p;
+        f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * p;
+    }
+    uint4 o;
+    o.x = h2_as_u32(__floats2half2_rn(f[0], f[4]));
+    o.y = h2_as_u32(__floats2half2_rn(f[1], f[5]));
+    o.z = h2_as_u32(__floats2half2_rn(f[2], f[6]));
+    o.w = h2_as_u32(__floats2half2_rn(f[3], f[7]));
+    return o;
+}
+
+__device__ __forceinline__ float bf16_amax(const uint4& v, bool& finite)
+{
+    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float lo = __uint_as_float(e[i] << 16), hi = __uint_as_float(e[i] & 0xFFFF0000u);
+        finite &= isfinite(lo) && isfinite(hi);
+        a = fmaxf(a, fmaxf(fabsf(lo), fabsf(hi)));
+    }
+    return a;
 }
 
 template <int KSPLIT, int J, int MT, bool SYM>
-__global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
+__global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_kernel(const __grid_constant__ GemvParams p)
 {
     constexpr int TEAMS = kComputeWarps / KSPLIT;
     extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* stages = smem;                                                   // kStages x kStageBytes
-    uint4* xs = reinterpret_cast<uint4*>(smem + kStages * kStageBytes);       // [MT][4][C] x pairs
-    const int C = p.k / 32, ng = p.k / p.group, cpg = p.group / 32;
-    __half* ssc = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(xs) + (size_t)MT * p.k * 2);
-    __half* szr = ssc + p.rows_per_cta * ng;
-    float* red = reinterpret_cast<float*>(smem + kStages * kStageBytes + (size_t)MT * p.k * 2 + kScaleBytes);
-    float* pscale = red + 2 * 16 * kMaxM;
-    uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * 16 * kMaxM + 8 * kMaxM);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kStages;
+    float* red = reinterpret_cast<float*>(empty + kStages);          // [2][TEAMS][KSPLIT][MT]
+    uint8_t* stages = smem + 1024;
 
+    // this CTA's problem and rows
+    int pi = 0;
+    while (pi + 1 < p.count && (int)blockIdx.x >= p.prob[pi + 1].cta_begin) pi++;
+    const Problem& P = p.prob[pi];
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int ng = p.k / p.group, cpg = p.group / 32, C = p.k / 32;
     const int64_t rowbytes = p.k / 2;
-    const int r0 = blockIdx.x * p.rows_per_cta;
-    const int r1 = min(p.n, r0 + p.rows_per_cta);
+    const int r0 = ((int)blockIdx.x - P.cta_begin) * p.rows_per_cta;
+    const int r1 = min(P.n, r0 + p.rows_per_cta);
     const int nstages = (r1 - r0 + p.rows_per_stage - 1) / p.rows_per_stage;
+    const int wbytes = p.rows_per_stage * (int)rowbytes;            // weight part of a stage
+    const int sbytes = p.rows_per_stage * ng * 2;                   // scale part of a stage
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kComputeWarps); }
@@ -144,12 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
     }
     if (warp == kComputeWarps && lane == 0 && r0 < r1) {
         // weights do not depend on the previous kernel: start pulling them into L2 now
-        prefetch_l2_range(p.packed + (int64_t)r0 * rowbytes, p.packed + (int64_t)r1 * rowbytes);
-        prefetch_l2_range(reinterpret_cast<const uint8_t*>(p.scales + (int64_t)r0 * ng),
-                          reinterpret_cast<const uint8_t*>(p.scales + (int64_t)r1 * ng));
-        if constexpr (!SYM)
-            prefetch_l2_range(reinterpret_cast<const uint8_t*>(p.zeros + (int64_t)r0 * ng),
-                              reinterpret_cast<const uint8_t*>(p.zeros + (int64_t)r1 * ng));
+        prefetch_l2_range(P.packed + (int64_t)r0 * rowbytes, P.packed + (int64_t)r1 * rowbytes);
+        prefetch_l2_range(P.scales + (int64_t)r0 * ng, P.scales + (int64_t)r1 * ng);
+        if constexpr (!SYM) prefetch_l2_range(P.zeros + (int64_t)r0 * ng, P.zeros + (int64_t)r1 * ng);
     }
     __syncthreads();
     pdl_launch_dependents();
@@ -162,74 +197,51 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
                 const int s = st % kStages;
                 if (!tc::mbar_wait(&empty[s], ((st / kStages) & 1) ^ 1, p.status, nullptr)) break;
                 const int rs = r0 + st * p.rows_per_stage;
-                const uint32_t bytes = (uint32_t)(min(p.rows_per_stage, r1 - rs) * rowbytes);
+                const int rows = min(p.rows_per_stage, r1 - rs);
+                uint8_t* dst = stages + s * p.stage_bytes;
+                uint32_t bytes = (uint32_t)(rows * rowbytes);
+                if (p.bulk_scales) bytes += (uint32_t)(rows * ng * 2 * (SYM ? 1 : 2));
                 tc::mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s(stages + s * kStageBytes, p.packed + (int64_t)rs * rowbytes, bytes, &full[s]);
+                bulk_g2s(dst, P.packed + (int64_t)rs * rowbytes, (uint32_t)(rows * rowbytes), &full[s]);
+                if (p.bulk_scales) {
+                    bulk_g2s(dst + wbytes, P.scales + (int64_t)rs * ng, (uint32_t)(rows * ng * 2), &full[s]);
+                    if constexpr (!SYM)
+                        bulk_g2s(dst + wbytes + sbytes, P.zeros + (int64_t)rs * ng, (uint32_t)(rows * ng * 2), &full[s]);
+                }
             }
         }
         return;
     }
 
     // ---------------------------------------------------------------------- compute warps
-    // x -> fp16 pairs with a power-of-two prescale per token; the CTA's scales and zeros -> smem
+    const int team = warp / KSPLIT, ks = warp % KSPLIT;
+    const int c0 = ks * 32 * J + J * lane;          // the lane's first chunk (J adjacent chunks)
+    const bool cvalid = c0 < C;
+    const int gl = c0 / cpg;                        // their group (J <= cpg, c0 % J == 0)
+
+    // x of the lane's chunks -> fp16 pairs with the lane's own power-of-two prescale
+    uint4 X[MT][J][4];
+    float inv_ps[MT];
+#pragma unroll
     for (int mm = 0; mm < MT; mm++) {
-        const uint4* xr = reinterpret_cast<const uint4*>(p.x + (int64_t)mm * p.k);
+        uint4 raw[J][4];
         float amax = 0.0f;
         bool finite = true;
-        for (int u = threadIdx.x; u < p.k / 8; u += kComputeThreads) {
-            const uint4 v = __ldg(xr + u);
-            const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float a = __uint_as_float(e[i] << 16), b = __uint_as_float(e[i] & 0xFFFF0000u);
-                finite &= isfinite(a) && isfinite(b);
-                amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+        for (int j = 0; j < J; j++)
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                raw[j][w] = cvalid ? __ldg(reinterpret_cast<const uint4*>(P.x + (int64_t)mm * p.k + 32 * (c0 + j)) + w)
+                                   : make_uint4(0, 0, 0, 0);
+                amax = fmaxf(amax, bf16_amax(raw[j][w], finite));
             }
-        }
         if (!finite) q4_set_status(p.status, Q4_ERR_NONFINITE);
+        const float ps = prescale_for(amax);
+        inv_ps[mm] = 1.0f / ps;
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (lane == 0) red[warp] = amax;
-        compute_bar();
-        if (threadIdx.x == 0) {
-            float a = 0.0f;
-            for (int i = 0; i < kComputeWarps; i++) a = fmaxf(a, red[i]);
-            pscale[mm] = prescale_for(a);
-        }
-        compute_bar();
-        const float ps = pscale[mm];
-        for (int u = threadIdx.x; u < p.k / 8; u += kComputeThreads) {
-            const uint4 v = __ldg(xr + u);
-            const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-            float f[8];
+        for (int j = 0; j < J; j++)
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                f[2 * i] = __uint_as_float(e[i] << 16) * ps;
-                f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * ps;
-            }
-            uint4 o;
-            o.x = h2_as_u32(__floats2half2_rn(f[0], f[4]));
-            o.y = h2_as_u32(__floats2half2_rn(f[1], f[5]));
-            o.z = h2_as_u32(__floats2half2_rn(f[2], f[6]));
-            o.w = h2_as_u32(__floats2half2_rn(f[3], f[7]));
-            xs[((int64_t)mm * 4 + (u & 3)) * C + (u >> 2)] = o;   // word u&3 of chunk u>>2
-        }
-    }
-    for (int i = threadIdx.x; i < (r1 - r0) * ng; i += kComputeThreads) {
-        ssc[i] = p.scales[(int64_t)r0 * ng + i];
-        if constexpr (!SYM) szr[i] = p.zeros[(int64_t)r0 * ng + i];
-    }
-    compute_bar();
-
-    const int team = warp / KSPLIT, ks = warp % KSPLIT;
-    int cidx[J];
-    uint4 X[J][4];
-#pragma unroll
-    for (int j = 0; j < J; j++) {
-        cidx[j] = ks * 32 * J + 32 * j + lane;
-#pragma unroll
-        for (int w = 0; w < 4; w++)
-            X[j][w] = (MT == 1 && cidx[j] < C) ? xs[(int64_t)w * C + cidx[j]] : make_uint4(0, 0, 0, 0);
+            for (int w = 0; w < 4; w++) X[mm][j][w] = x_pairs(raw[j][w], ps);
     }
 
     for (int st = 0; st < nstages; st++) {
@@ -237,41 +249,42 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
         const int rs = r0 + st * p.rows_per_stage;
         const int rows_here = min(p.rows_per_stage, r1 - rs);
         if (!tc::mbar_wait(&full[s], (st / kStages) & 1, p.status, nullptr)) break;
-        const uint8_t* sbase = stages + s * kStageBytes;
-        float* redb = red + (st & 1) * 16 * kMaxM;
+        const uint8_t* sb = stages + s * p.stage_bytes;
+        const __half* ssc = reinterpret_cast<const __half*>(sb + wbytes);
+        const __half* szr = reinterpret_cast<const __half*>(sb + wbytes + sbytes);
+        float* redb = red + (st & 1) * TEAMS * KSPLIT * MT;
         for (int rr = team; rr < rows_here; rr += TEAMS) {
             const int row = rs + rr;
-            const int lrow = row - r0;
             float part[MT];
 #pragma unroll
             for (int mm = 0; mm < MT; mm++) part[mm] = 0.0f;
+            if (cvalid) {
+                float sc;
+                __half z;
+                if (p.bulk_scales) {
+                    sc = __half2float(ssc[rr * ng + gl]);
+                    z = SYM ? __float2half_rn(8.0f) : szr[rr * ng + gl];
+                } else {
+                    sc = __half2float(P.scales[(int64_t)row * ng + gl]);
+                    z = SYM ? __float2half_rn(8.0f) : P.zeros[(int64_t)row * ng + gl];
+                }
+                const __half2 b1 = __half2half2(__hadd(z, __float2half_rn(1024.0f)));
+                const __half2 b16 = __half2half2(__hfma(z, __float2half_rn(16.0f), __float2half_rn(1024.0f)));
+                uint4 wv[J];
 #pragma unroll
-            for (int j = 0; j < J; j++) {
-                const int c = cidx[j];
-                if (c < C) {
-                    const uint4 wv = lds128(sbase + rr * rowbytes + c * 16);
-                    const int gidx = lrow * ng + c / cpg;
-                    const float sc = __half2float(ssc[gidx]);
-                    __half2 b1, b16;
-                    if constexpr (SYM) {
-                        b1 = __float2half2_rn(1032.0f);
-                        b16 = __float2half2_rn(1152.0f);
-                    } else {
-                        const __half z = szr[gidx];
-                        b1 = __half2half2(__hadd(z, __float2half_rn(1024.0f)));
-                        b16 = __half2half2(__hfma(z, __float2half_rn(16.0f), __float2half_rn(1024.0f)));
+                for (int j = 0; j < J; j++) wv[j] = lds128(sb + rr * rowbytes + (c0 + j) * 16);
+#pragma unroll
+                for (int mm = 0; mm < MT; mm++) {
+                    __half2 acc1 = __float2half2_rn(0.0f), acc16 = __float2half2_rn(0.0f);
+#pragma unroll
+                    for (int j = 0; j < J; j++) {
+                        word_dot<SYM>(wv[j].x, b1, b16, X[mm][j][0], acc1, acc16);
+                        word_dot<SYM>(wv[j].y, b1, b16, X[mm][j][1], acc1, acc16);
+                        word_dot<SYM>(wv[j].z, b1, b16, X[mm][j][2], acc1, acc16);
+                        word_dot<SYM>(wv[j].w, b1, b16, X[mm][j][3], acc1, acc16);
                     }
-                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                    for (int mm = 0; mm < MT; mm++) {
-                        __half2 acc1 = __float2half2_rn(0.0f), acc16 = __float2half2_rn(0.0f);
-#pragma unroll
-                        for (int w = 0; w < 4; w++) {
-                            const uint4 xv = MT == 1 ? X[j][w] : xs[((int64_t)mm * 4 + w) * C + c];
-                            word_dot<SYM>(words[w], b1, b16, xv, acc1, acc16);
-                        }
-                        part[mm] += sc * fold(acc1, acc16);
-                    }
+                    const float2 f = __half22float2(__hfma2(acc16, __float2half2_rn(0.0625f), acc1));
+                    part[mm] = sc * (f.x + f.y) * inv_ps[mm];
                 }
             }
 #pragma unroll
@@ -279,23 +292,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
 #pragma unroll
                 for (int off = 16; off >= 1; off >>= 1) part[mm] += __shfl_xor_sync(0xffffffffu, part[mm], off);
             }
-            if constexpr (KSPLIT == 1) {
-                if (lane < MT) {
-                    float v = part[0];
+            if (lane < MT) {
+                float v = part[0];
 #pragma unroll
-                    for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
-                    v /= pscale[lane];
-                    const int64_t o = (int64_t)lane * p.n + row;
-                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
-                    else reinterpret_cast<float*>(p.y)[o] = v;
-                }
-            } else {
-                // rows_per_stage == TEAMS here: one row per team per stage
-                if (lane < MT) {
-                    float v = part[0];
-#pragma unroll
-                    for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
-                    redb[(team * KSPLIT + ks) * MT + lane] = v;
+                for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
+                if constexpr (KSPLIT == 1) {
+                    const int64_t o = (int64_t)lane * P.n + row;
+                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
+                    else reinterpret_cast<float*>(P.y)[o] = v;
+                } else {
+                    redb[(team * KSPLIT + ks) * MT + lane] = v;   // one row per team per stage
                 }
             }
         }
@@ -307,10 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
                 float v = 0.0f;
 #pragma unroll
                 for (int t = 0; t < KSPLIT; t++) v += redb[(team * KSPLIT + t) * MT + lane];
-                v /= pscale[lane];
-                const int64_t o = (int64_t)lane * p.n + (rs + team);
-                if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
-                else reinterpret_cast<float*>(p.y)[o] = v;
+                const int64_t o = (int64_t)lane * P.n + (rs + team);
+                if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
+                else reinterpret_cast<float*>(P.y)[o] = v;
             }
         }
     }
@@ -319,8 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_kernel(GemvParams p)
 template <int KSPLIT, int J, int MT>
 int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
 {
-    const size_t smem = (size_t)kStages * kStageBytes + (size_t)MT * p.k * 2 + kScaleBytes +
-                        (2 * 16 * kMaxM + 8 * kMaxM) * sizeof(float) + 2 * kStages * sizeof(uint64_t);
+    const size_t smem = 1024 + (size_t)kStages * p.stage_bytes;
     if (smem > 227 * 1024) return Q4_ERR_UNSUPPORTED;
     auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, J, MT, true> : w4a16_gemv_kernel<KSPLIT, J, MT, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -364,40 +368,55 @@ int launch_ksplit(const GemvParams& p, int symmetric, int ksplit, int grid, cuda
 
 }  // namespace
 
-// Host entry used by q4_linear_w4a16 for m <= 4.  Requires k % 32 == 0 and k <= 16384.
-int q4_gemv_w4a16_launch(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
-                         int32_t* dev_status, cudaStream_t stream)
+// Host entry used by q4_linear_w4a16 (count == 1) and q4_linear_w4a16_grouped: m <= 4, and every
+// problem with the same k (a multiple of 64, at most 16384), group and symmetry.
+int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, const q4_weight* w, void* const* y,
+                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream)
 {
-    if (w->k % 32 || w->k > 16384 || m < 1 || m > kMaxM) return Q4_ERR_UNSUPPORTED;
-    GemvParams p;
-    p.x = x;
-    p.packed = w->packed;
-    p.scales = reinterpret_cast<const __half*>(w->scales);
-    p.zeros = reinterpret_cast<const __half*>(w->zeros);
-    p.y = y;
-    p.status = dev_status;
+    if (count < 1 || count > kMaxProblems || m < 1 || m > kMaxM) return Q4_ERR_UNSUPPORTED;
+    const int k = w[0].k, group = w[0].group, sym = w[0].symmetric;
+    if (k % 64 || k > 16384) return Q4_ERR_UNSUPPORTED;
+    for (int i = 1; i < count; i++)
+        if (w[i].k != k || w[i].group != group || w[i].symmetric != sym) return Q4_ERR_UNSUPPORTED;
+    GemvParams p = {};
+    p.count = count;
     p.m = m;
-    p.n = w->n;
-    p.k = w->k;
-    p.group = w->group;
+    p.k = k;
+    p.group = group;
     p.out_bf16 = out_dtype == Q4_OUT_BF16;
-    const int C = w->k / 32;
+    p.status = dev_status;
+    const int C = k / 32;
+    const int J = 2;                                   // two adjacent chunks (64 codes) per lane
     int ksplit = 1;
-    while (ksplit * 64 < C) ksplit *= 2;                     // at most two chunks per lane
+    while (ksplit * 32 * J < C) ksplit *= 2;
     if (ksplit > 8) return Q4_ERR_UNSUPPORTED;
-    const int J = (C + 32 * ksplit - 1) / (32 * ksplit);
     const int teams = kComputeWarps / ksplit;
-    const int rowbytes = w->k / 2;
-    int rps = kStageBytes / rowbytes;
-    if (ksplit > 1) rps = teams;                             // one row per team per stage
-    const int ng = w->k / w->group;
-    const int sbytes_row = ng * 2 * (w->symmetric ? 1 : 2);
-    const int sms = q4_num_sms();
-    int rpc = (w->n + sms - 1) / sms;
-    rpc = std::max(1, std::min(rpc, kScaleBytes / sbytes_row));
+    const int rowbytes = k / 2;
+    const int ng = k / group;
+    int rps = ksplit > 1 ? teams : std::max(1, kWeightStage / rowbytes);
+    p.rows_per_stage = rps;
+    p.bulk_scales = (ng * 2) % 16 == 0;
+    p.stage_bytes = rps * rowbytes + (p.bulk_scales ? rps * ng * 2 * (sym ? 1 : 2) : 0);
+    p.stage_bytes = (p.stage_bytes + 15) & ~15;
+    // rows per CTA: about two CTAs per SM over the whole group, whole stages where possible
+    int64_t rows_total = 0;
+    for (int i = 0; i < count; i++) rows_total += w[i].n;
+    const int64_t target_ctas = 2LL * q4_num_sms();
+    int rpc = (int)std::max<int64_t>(1, (rows_total + target_ctas - 1) / target_ctas);
+    if (rpc > rps) rpc = (rpc + rps - 1) / rps * rps;
     p.rows_per_cta = rpc;
-    p.rows_per_stage = std::max(1, rps);
-    const int grid = (w->n + rpc - 1) / rpc;
-    return J == 2 ? launch_ksplit<2>(p, w->symmetric, ksplit, grid, stream)
-                  : launch_ksplit<1>(p, w->symmetric, ksplit, grid, stream);
+    int ctas = 0;
+    for (int i = 0; i < count; i++) {
+        Problem& P = p.prob[i];
+        P.x = x[i];
+        P.packed = w[i].packed;
+        P.scales = reinterpret_cast<const __half*>(w[i].scales);
+        P.zeros = reinterpret_cast<const __half*>(w[i].zeros);
+        P.y = y[i];
+        P.n = w[i].n;
+        P.cta_begin = ctas;
+        ctas += (w[i].n + rpc - 1) / rpc;
+    }
+    if (ctas == 0) return Q4_OK;
+    return launch_ksplit<2>(p, sym, ksplit, ctas, stream);
 }

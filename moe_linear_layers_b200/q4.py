@@ -32,6 +32,7 @@ Q4_OUT_F32 = 0
 Q4_OUT_BF16 = 1
 
 EXPORTED = ("q4_status_string", "q4_version", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
+            "q4_linear_w4a16_grouped",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -50,6 +51,8 @@ _lib.q4_version.restype = ctypes.c_int
 _lib.q4_linear_w4a16_max_gemv_m.restype = ctypes.c_int
 _lib.q4_quantize_pack.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p]
 _lib.q4_linear_w4a16.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p]
+_lib.q4_linear_w4a16_grouped.argtypes = [_i32, ctypes.POINTER(_p), _i32, ctypes.POINTER(q4_weight),
+                                         ctypes.POINTER(_p), _i32, _p, _p]
 _lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
 _lib.q4_linear_w4a8.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _p]
 _lib.moe_q4_workspace_size.restype = _sz
@@ -138,6 +141,32 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
     _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
            "q4_linear_w4a16")
     return y
+
+
+class GroupedGemv:
+    """Host-side argument arrays for q4_linear_w4a16_grouped, built once and reused (e.g. per layer)."""
+
+    def __init__(self, xs, ws, ys):
+        assert len(xs) == len(ws) == len(ys) and 1 <= len(xs) <= 8
+        self.count = len(xs)
+        self.m = xs[0].numel() // ws[0].k
+        self.keep = (xs, ws, ys)
+        self.x = (_p * self.count)(*[t.data_ptr() for t in xs])
+        self.w = (q4_weight * self.count)(*[w.desc for w in ws])
+        self.y = (_p * self.count)(*[t.data_ptr() for t in ys])
+        self.od = Q4_OUT_BF16 if ys[0].dtype == torch.bfloat16 else Q4_OUT_F32
+
+    def __call__(self, dev_status: torch.Tensor | None = None, stream=None):
+        _check(_lib.q4_linear_w4a16_grouped(self.count, self.x, self.m, self.w, self.y, self.od, _ptr(dev_status),
+                                            _stream(stream)), "q4_linear_w4a16_grouped")
+
+
+def q4_linear_w4a16_grouped(xs, ws, ys, dev_status: torch.Tensor | None = None, stream=None):
+    """y[i] = x[i] . dequant(W[i])^T for up to 8 independent small-m problems with the same k, in one launch."""
+    for t in xs:
+        _dev(t, torch.bfloat16, "x")
+    GroupedGemv(xs, ws, ys)(dev_status=dev_status, stream=stream)
+    return ys
 
 
 def q4_linear_w4a16_max_gemv_m() -> int:

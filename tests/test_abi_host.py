@@ -85,3 +85,16 @@ def test_act_quant_validation():
     assert L.act_quant_per_token(None, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_NULL
     assert L.act_quant_per_token(FAKE, 4, 12, FAKE, FAKE, None, None) == q4.Q4_ERR_SHAPE
     assert L.act_quant_per_token(FAKE + 2, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_ALIGN
+
+
+def test_grouped_validation():
+    L = q4._lib
+    ws = (q4.q4_weight * 2)(_w(), _w(k=512))
+    xs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    ys = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert L.q4_linear_w4a16_grouped(2, xs, 1, ws, ys, 0, None, None) == q4.Q4_ERR_SHAPE   # k differs
+    ws2 = (q4.q4_weight * 2)(_w(), _w())
+    assert L.q4_linear_w4a16_grouped(9, xs, 1, ws2, ys, 0, None, None) == q4.Q4_ERR_SHAPE  # too many
+    assert L.q4_linear_w4a16_grouped(2, xs, 5, ws2, ys, 0, None, None) == q4.Q4_ERR_SHAPE  # m > 4
+    xs_bad = (ctypes.c_void_p * 2)(FAKE, FAKE + 2)
+    assert L.q4_linear_w4a16_grouped(2, xs_bad, 1, ws2, ys, 0, None, None) == q4.Q4_ERR_ALIGN

@@ -95,7 +95,7 @@ def test_gemv_tiny_workload(q4):
 @pytest.mark.parametrize("n,k,group,sym", [
     (2048, 2048, 128, False), (512, 2048, 128, False), (8192, 2048, 128, False), (2048, 8192, 128, False),
     (2048, 2048, 128, True), (77, 256, 64, False), (300, 16384, 128, True), (1000, 4096, 64, False),
-    (5, 1024, 128, True), (1, 32 * 64, 64, False),
+    (5, 1024, 128, True), (1, 32 * 64, 64, False), (3000, 1024 + 64, 64, True),
 ])
 def test_gemv_m1(q4, n, k, group, sym):
     y, ref, *_ = _gemv_case(q4, n, k, group, sym, 1, "m1")
@@ -107,6 +107,28 @@ def test_gemv_m1(q4, n, k, group, sym):
 def test_gemv_small_m(q4, m, n, k, group, sym):
     y, ref, *_ = _gemv_case(q4, n, k, group, sym, m, "sm")
     assert_close(y.cpu().numpy(), ref, what=f"gemv m={m} {n}x{k}")
+
+
+@pytest.mark.parametrize("m", [1, 3])
+def test_gemv_grouped_matches_oracle(q4, m):
+    """q, k, v of one layer (same k, different n) in one launch, each with its own x."""
+    shapes = [(2048, 2048), (512, 2048), (512, 2048)]
+    xs, ws, ys, refs = [], [], [], []
+    for i, (n, k) in enumerate(shapes):
+        W = synth.weights(("test", "grp", i), n, k)
+        pk, sc, zr = oracle.quantize(W, 128, False)
+        x = synth.activations(("test", "grp-x", i, m), m, k)
+        refs.append(oracle.linear_w4a16(x, pk, sc, zr, n, k, 128, False))
+        ws.append(upload_weight(q4, pk, sc, zr, n, k, 128, False))
+        xs.append(cuda_u16_as(x, torch.bfloat16))
+        ys.append(torch.empty((m, n), dtype=torch.float32, device="cuda"))
+    q4.q4_linear_w4a16_grouped(xs, ws, ys)
+    torch.cuda.synchronize()
+    for i in range(len(shapes)):
+        assert_close(ys[i].cpu().numpy(), refs[i], what=f"grouped problem {i}")
+        # the grouped result is the single-call result, bit for bit
+        y1 = q4.q4_linear_w4a16(xs[i], ws[i])
+        assert torch.equal(y1, ys[i])
 
 
 def test_gemv_bf16_out_is_rounded_fp32(q4):
