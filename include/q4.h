@@ -79,6 +79,9 @@ const char* q4_status_string(int status);
 /* Library version (increments with the ABI). */
 int q4_version(void);
 
+/* Description of the last CUDA error behind a Q4_ERR_CUDA return on the calling host thread. */
+const char* q4_last_cuda_error_string(void);
+
 /*
  * q4_quantize_pack -- round-to-nearest group quantization and packing of an fp32 matrix.
  * Source: the W4A8 page §2.3 (offline INT4 quantization keeping scale and zero point) and §2.1

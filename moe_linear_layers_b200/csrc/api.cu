@@ -40,6 +40,15 @@ extern "C" const char* q4_status_string(int status)
 
 extern "C" int q4_version(void) { return 1; }
 
+static thread_local cudaError_t q4_last_error = cudaSuccess;
+
+void q4_record_cuda_error(cudaError_t e) { q4_last_error = e; }
+
+extern "C" const char* q4_last_cuda_error_string(void)
+{
+    return q4_last_error == cudaSuccess ? "no error" : cudaGetErrorString(q4_last_error);
+}
+
 extern "C" int q4_linear_w4a16_max_gemv_m(void) { return kMaxGemvM; }
 
 extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,

@@ -327,8 +327,8 @@ int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
     const size_t smem = 1024 + (size_t)kStages * p.stage_bytes;
     if (smem > 227 * 1024) return Q4_ERR_UNSUPPORTED;
     auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, J, MT, true> : w4a16_gemv_kernel<KSPLIT, J, MT, false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return Q4_ERR_CUDA;
+    if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+        return q4_cuda_status(e);
     // Programmatic stream serialization: the kernel may start (and prefetch its weights into L2) while
     // the previous kernel on the stream drains; it reads x only after griddepcontrol.wait.
     cudaLaunchConfig_t cfg = {};
@@ -341,7 +341,7 @@ int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return q4_cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
 template <int KSPLIT, int J>

@@ -32,66 +32,110 @@ constexpr int kMaxTopk = 16;
 // ---------------------------------------------------------------------------------------------- //
 // 1. route
 // ---------------------------------------------------------------------------------------------- //
-// Warp w computes 4 tokens x 16 experts: lane l owns the k = l (mod 32) partial sums, each an fma chain
-// with k ascending; the 32 partials are combined by an xor butterfly (s = 16, 8, 4, 2, 1), which gives
-// every lane the same value.  This is the pinned order the oracle reproduces bit for bit.
-__global__ void __launch_bounds__(kRouteWarps * 32, 1)
-moe_route_kernel(const uint16_t* __restrict__ x, int T, int H, const float* __restrict__ Wr,
+// A CTA scores one chunk of 16 tokens against 64 experts at a time.  Warp w owns 4 tokens x 16 experts;
+// lane l owns the k = l (mod 32) partial sums, each an fma chain with k ascending (two experts per
+// packed fma.rn.f32x2, which rounds each half exactly like fmaf); the 32 partials are combined by an
+// xor butterfly (s = 16, 8, 4, 2, 1), which leaves the same value in every lane.  This is the pinned
+// order the oracle reproduces bit for bit.  A producer warp streams 64-column tiles of Wr (fp32) and x
+// (bf16) through a 4-stage TMA ring.
+constexpr int kRouteStages = 4;
+constexpr int kRouteThreads = (kRouteWarps + 1) * 32;
+constexpr int kRouteWTile = 64 * kRouteKC * 4;       // 64 experts x 64 columns, fp32
+constexpr int kRouteXTile = kRouteTok * kRouteKC * 2;  // 16 tokens x 64 columns, bf16
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+
+__global__ void __launch_bounds__(kRouteThreads, 1)
+moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, int T, int H,
                  const float* __restrict__ bias, int E, int topk, int32_t* __restrict__ ids, float* __restrict__ wts,
                  int32_t* __restrict__ hist, int32_t* status)
 {
-    __shared__ float xs[kRouteTok][kRouteKC];
-    __shared__ float ws[64][kRouteKC];
+    extern __shared__ __align__(128) uint8_t rsm[];
+    float* wst = reinterpret_cast<float*>(rsm);                                       // [stage][64][KC]
+    uint16_t* xst = reinterpret_cast<uint16_t*>(rsm + kRouteStages * kRouteWTile);    // [stage][16][KC]
     __shared__ float logits[kRouteTok][tcg::kMaxExperts];
     __shared__ int hcount[tcg::kMaxExperts];
+    __shared__ uint64_t full[kRouteStages], empty[kRouteStages];
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kRouteTok;
-    const int tg = warp / 4, eg = warp % 4;
+    const int nk = H / kRouteKC;
+    const int neb = (E + 63) / 64;
+    const int nsteps = neb * nk;          // (expert block, k chunk) pairs in order
 
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRouteStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kRouteWarps); }
+        tc::fence_mbar_init();
+    }
     for (int e = threadIdx.x; e < E; e += blockDim.x) hcount[e] = 0;
-    for (int eb = 0; eb < E; eb += 64) {
-        float acc[4][16];
-#pragma unroll
-        for (int a = 0; a < 4; a++)
-#pragma unroll
-            for (int b = 0; b < 16; b++) acc[a][b] = 0.0f;
-        for (int k0 = 0; k0 < H; k0 += kRouteKC) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < kRouteTok * kRouteKC; i += blockDim.x) {
-                const int a = i / kRouteKC, c = i % kRouteKC;
-                const int t = t0 + a;
-                xs[a][c] = t < T ? bf16_bits_to_float(x[(int64_t)t * H + k0 + c]) : 0.0f;
-            }
-            for (int i = threadIdx.x; i < 64 * kRouteKC; i += blockDim.x) {
-                const int b = i / kRouteKC, c = i % kRouteKC;
-                const int e = eb + b;
-                ws[b][c] = e < E ? Wr[(int64_t)e * H + k0 + c] : 0.0f;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < kRouteKC / 32; i++) {
-                const int c = lane + 32 * i;
-                float xv[4], wv[16];
-#pragma unroll
-                for (int a = 0; a < 4; a++) xv[a] = xs[4 * tg + a][c];
-#pragma unroll
-                for (int b = 0; b < 16; b++) wv[b] = ws[16 * eg + b][c];
-#pragma unroll
-                for (int a = 0; a < 4; a++)
-#pragma unroll
-                    for (int b = 0; b < 16; b++) acc[a][b] = fmaf(xv[a], wv[b], acc[a][b]);
+    __syncthreads();
+
+    if (warp == kRouteWarps) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            for (int st = 0; st < nsteps; st++) {
+                const int s = st % kRouteStages;
+                if (!tc::mbar_wait(&empty[s], ((st / kRouteStages) & 1) ^ 1, status, nullptr)) break;
+                const int eb = st / nk, kc = st % nk;
+                tc::mbar_arrive_expect_tx(&full[s], kRouteWTile + kRouteXTile);
+                tc::tma_load_2d(wst + s * (kRouteWTile / 4), &tm_w, &full[s], kc * kRouteKC, eb * 64);
+                tc::tma_load_2d(xst + s * (kRouteXTile / 2), &tm_x, &full[s], kc * kRouteKC, t0);
             }
         }
+    } else {
+        // ------------------------------------------------------------------ 16 compute warps
+        const int tg = warp / 4, eg = warp % 4;
+        for (int eb = 0; eb < neb; eb++) {
+            uint64_t acc[4][8];
 #pragma unroll
-        for (int a = 0; a < 4; a++)
+            for (int a = 0; a < 4; a++)
 #pragma unroll
-            for (int b = 0; b < 16; b++) {
-                float v = acc[a][b];
+                for (int b = 0; b < 8; b++) acc[a][b] = 0;
+            for (int kc = 0; kc < nk; kc++) {
+                const int st = eb * nk + kc, s = st % kRouteStages;
+                if (!tc::mbar_wait(&full[s], (st / kRouteStages) & 1, status, nullptr)) break;
+                const float* wt = wst + s * (kRouteWTile / 4);
+                const uint16_t* xt = xst + s * (kRouteXTile / 2);
 #pragma unroll
-                for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
-                const int e = eb + 16 * eg + b;
-                if (lane == 0 && e < E) logits[4 * tg + a][e] = bias ? v + bias[e] : v;
+                for (int i = 0; i < kRouteKC / 32; i++) {
+                    const int c = lane + 32 * i;
+                    uint64_t xv[4];
+#pragma unroll
+                    for (int a = 0; a < 4; a++) {
+                        const float f = bf16_bits_to_float(xt[(4 * tg + a) * kRouteKC + c]);
+                        xv[a] = pack2(f, f);
+                    }
+#pragma unroll
+                    for (int b = 0; b < 8; b++) {
+                        const uint64_t wv = pack2(wt[(16 * eg + 2 * b) * kRouteKC + c], wt[(16 * eg + 2 * b + 1) * kRouteKC + c]);
+#pragma unroll
+                        for (int a = 0; a < 4; a++) acc[a][b] = ffma2(xv[a], wv, acc[a][b]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&empty[s]);
             }
+#pragma unroll
+            for (int a = 0; a < 4; a++)
+#pragma unroll
+                for (int b = 0; b < 8; b++)
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        float v = __uint_as_float((uint32_t)(acc[a][b] >> (32 * h)));
+#pragma unroll
+                        for (int sft = 16; sft >= 1; sft >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sft);
+                        const int e = eb * 64 + 16 * eg + 2 * b + h;
+                        if (lane == 0 && e < E) logits[4 * tg + a][e] = bias ? v + bias[e] : v;
+                    }
+        }
     }
     __syncthreads();
 
@@ -121,9 +165,9 @@ moe_route_kernel(const uint16_t* __restrict__ x, int T, int H, const float* __re
                 if (e < E && (v[q] > bv || (v[q] == bv && e < be))) { bv = v[q]; be = e; }
             }
 #pragma unroll
-            for (int s = 16; s >= 1; s >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, s);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, s);
+            for (int sft = 16; sft >= 1; sft >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, sft);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, sft);
                 if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
             }
             sel_l[j] = bv;
@@ -192,9 +236,10 @@ __global__ void moe_scan_kernel(const int32_t* __restrict__ hist, int nchunks, i
 // 3. scatter + gather (one CTA per chunk of 16 tokens)
 // ---------------------------------------------------------------------------------------------- //
 __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int E, int topk,
-                                                          const int32_t* __restrict__ ids,
+                                                          const int32_t* __restrict__ ids, const float* __restrict__ wts,
                                                           const int32_t* __restrict__ chunk_base,
-                                                          int32_t* __restrict__ perm, uint16_t* __restrict__ xperm)
+                                                          int32_t* __restrict__ perm, int32_t* __restrict__ row_tok,
+                                                          float* __restrict__ row_w, uint16_t* __restrict__ xperm)
 {
     __shared__ int pos[kRouteTok * kMaxTopk];
     const int c = blockIdx.x;
@@ -209,6 +254,8 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __rest
         const int p = chunk_base[(int64_t)c * E + e] + rank;
         pos[q] = p;
         perm[p] = (t0 + tl) * topk + j;
+        row_tok[p] = t0 + tl;
+        row_w[p] = wts[(int64_t)(t0 + tl) * topk + j];
     }
     __syncthreads();
     const int vec = H / 8;  // 16-byte units per row
@@ -229,8 +276,8 @@ struct Workspace {
     uint16_t* xperm;
     __half* h;
     float* y32;
-    int32_t *ids, *perm, *offsets, *counts, *hist, *chunk_base, *tiles_gu, *tiles_dn;
-    float* wts;
+    int32_t *ids, *perm, *offsets, *counts, *hist, *chunk_base, *tiles_gu, *tiles_dn, *row_tok;
+    float *wts, *row_w;
     size_t bytes;
 };
 
@@ -250,6 +297,8 @@ Workspace carve(void* base, int T, int H, int I, int E, int topk)
     w.ids = reinterpret_cast<int32_t*>(take(P * 4));
     w.wts = reinterpret_cast<float*>(take(P * 4));
     w.perm = reinterpret_cast<int32_t*>(take(P * 4));
+    w.row_tok = reinterpret_cast<int32_t*>(take(P * 4));
+    w.row_w = reinterpret_cast<float*>(take(P * 4));
     w.offsets = reinterpret_cast<int32_t*>(take((E + 1) * 4));
     w.counts = reinterpret_cast<int32_t*>(take(E * 4));
     w.hist = reinterpret_cast<int32_t*>(take(nch * E * 4));
@@ -298,8 +347,8 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     d.status = status;
     d.expert_tiles = ws.tiles_dn;
     d.offsets = ws.offsets;
-    d.perm = ws.perm;
-    d.topk_w = ws.wts;
+    d.row_tok = ws.row_tok;
+    d.row_w = ws.row_w;
     d.E = E;
     d.topk = topk;
     return launch<false, G, SYM, Mode::Down>(mh, md, md, d, sms, s);
@@ -349,12 +398,22 @@ extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const flo
     const int nch = (T + kRouteTok - 1) / kRouteTok;
     float* y32 = out_dtype == Q4_OUT_F32 ? reinterpret_cast<float*>(y) : ws.y32;
 
-    moe_route_kernel<<<nch, kRouteWarps * 32, 0, s>>>(x, T, H, router_w, router_bias, E, topk, ws.ids, ws.wts, ws.hist,
-                                                      dev_status);
+    CUtensorMap mrx, mrw;
+    if (!tcg::make_map(&mrx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, T, (uint64_t)H * 2, kRouteKC, kRouteTok,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !tcg::make_map(&mrw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, router_w, H, E, (uint64_t)H * 4, kRouteKC, 64,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    constexpr int route_smem = kRouteStages * (kRouteWTile + kRouteXTile);
+    if (const cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, route_smem))
+        return q4_cuda_status(e);
+    moe_route_kernel<<<nch, kRouteThreads, route_smem, s>>>(mrx, mrw, T, H, router_bias, E, topk, ws.ids, ws.wts,
+                                                            ws.hist, dev_status);
     moe_scan_kernel<<<1, tcg::kMaxExperts, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
                                                    ws.tiles_gu, ws.tiles_dn);
-    moe_scatter_kernel<<<nch, 256, 0, s>>>(x, T, H, E, topk, ws.ids, ws.chunk_base, ws.perm, ws.xperm);
-    if (cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess) return Q4_ERR_CUDA;
+    moe_scatter_kernel<<<nch, 256, 0, s>>>(x, T, H, E, topk, ws.ids, ws.wts, ws.chunk_base, ws.perm, ws.row_tok,
+                                           ws.row_w, ws.xperm);
+    if (const cudaError_t e = cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s)) return q4_cuda_status(e);
     int rc = q4_launch_status();
     if (rc) return rc;
     if (g.group == 128) rc = g.symmetric ? launch_experts<128, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)

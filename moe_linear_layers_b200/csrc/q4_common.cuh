@@ -47,12 +47,18 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Host side: error mapping for launches.
-static inline int q4_launch_status()
+// Host side: error mapping for launches.  The last CUDA error is kept per host thread for
+// q4_last_cuda_error_string().
+void q4_record_cuda_error(cudaError_t e);
+
+static inline int q4_cuda_status(cudaError_t e)
 {
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    if (e == cudaSuccess) return Q4_OK;
+    q4_record_cuda_error(e);
+    return Q4_ERR_CUDA;
 }
+
+static inline int q4_launch_status() { return q4_cuda_status(cudaGetLastError()); }
 
 static inline bool q4_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

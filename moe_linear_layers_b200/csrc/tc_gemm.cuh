@@ -54,7 +54,7 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     static constexpr uint32_t A_COL0 = 2 * BN;                  // widened weights after the 2 D buffers
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
-    static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 2048;
+    static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144;
 };
 
 struct Args {
@@ -71,8 +71,8 @@ struct Args {
     // MoE
     const int32_t* expert_tiles;   // [E+1] prefix sums of tiles per expert
     const int32_t* offsets;        // [E+1] first permuted row of each expert
-    const int32_t* perm;           // [P] pair index t*topk + j of each permuted row
-    const float* topk_w;           // [T*topk] routing weights
+    const int32_t* row_tok;        // Down: [P] token of each permuted row
+    const float* row_w;            // Down: [P] routing weight of each permuted row
     __half* h;                     // GateUp output [P][N]
     int E, topk;
 };
@@ -152,7 +152,19 @@ struct Shared {
     int abort_flag;
     int total_tiles;
     int expert_tiles[kMaxExperts + 1];
+    int comb_tok[8 * 64];      // Down: token of each activation row of the tile, per epilogue warp
+    float comb_w[8 * 64];      // Down: its routing weight
 };
+
+constexpr int ZD = 4;   // depth of the converters' zero-point FIFO (K stages)
+constexpr int SD = 4;   // depth of the epilogue's scale FIFO (groups)
+
+// Pull a row of group parameters (n fp16 values) toward L2 ahead of use.
+__device__ __forceinline__ void prefetch_row_l2(const __half* row, int n)
+{
+    for (int b = 0; b < n * 2; b += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(row) + b));
+}
 
 template <Mode MODE>
 __device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
@@ -217,6 +229,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     float* xchg = reinterpret_cast<float*>(wsm + NS * WSTAGE);   // GateUp only
     Shared* sh = reinterpret_cast<Shared*>(wsm + NS * WSTAGE + C::XCHG);
     volatile int* abort_flag = &sh->abort_flag;
+    int* comb_tok = sh->comb_tok;
+    float* comb_w = sh->comb_w;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
     const int kblocks = p.K / KBLK, ngroups = p.K / G;
@@ -326,18 +340,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
-            // zero points of the next stage are fetched one stage ahead
-            float znext[GPK];
+            if (t + (int)gridDim.x < total) {  // warm L2 with the next tile's scale/zero row
+                const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
+                const __half *sn, *zn;
+                row_params<MODE>(p, Tn, r, ngroups, sn, zn);
+                if (zn) prefetch_row_l2(zn, ngroups);
+            }
+            // zero points travel through a register FIFO ZD stages deep (global loads, latency hidden)
+            float zq[ZD][GPK];
 #pragma unroll
-            for (int gi = 0; gi < GPK; gi++) znext[gi] = SYM ? 8.0f : (zrow ? __half2float(zrow[gi]) : 0.0f);
+            for (int d = 0; d < ZD; d++)
+#pragma unroll
+                for (int gi = 0; gi < GPK; gi++)
+                    zq[d][gi] = SYM ? 8.0f : ((zrow && d < kblocks) ? __half2float(zrow[d * GPK + gi]) : 0.0f);
             for (int kb = 0; kb < kblocks; kb++, it++) {
                 const int s = it % NS, sa = it % NA;
                 float zcur[GPK];
 #pragma unroll
-                for (int gi = 0; gi < GPK; gi++) {
-                    zcur[gi] = znext[gi];
-                    if constexpr (!SYM)
-                        if (kb + 1 < kblocks) znext[gi] = zrow ? __half2float(zrow[(kb + 1) * GPK + gi]) : 0.0f;
+                for (int gi = 0; gi < GPK; gi++) zcur[gi] = zq[0][gi];
+                if constexpr (!SYM) {
+#pragma unroll
+                    for (int d = 0; d + 1 < ZD; d++)
+#pragma unroll
+                        for (int gi = 0; gi < GPK; gi++) zq[d][gi] = zq[d + 1][gi];
+#pragma unroll
+                    for (int gi = 0; gi < GPK; gi++)
+                        zq[ZD - 1][gi] = (zrow && kb + ZD < kblocks) ? __half2float(zrow[(kb + ZD) * GPK + gi]) : 0.0f;
                 }
                 if (!tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
                 uint4 v[4];
@@ -396,11 +424,31 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
 #pragma unroll
             for (int j = 0; j < 64; j++) acc[j] = 0.0f;
-            float s_next = srow ? __half2float(srow[0]) : 0.0f;
+            if (t + (int)gridDim.x < total) {  // warm L2 with the next tile's scale row
+                const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
+                const __half *sn, *zn;
+                row_params<MODE>(p, Tn, r, ngroups, sn, zn);
+                if (sn) prefetch_row_l2(sn, ngroups);
+            }
+            if constexpr (MODE == Mode::Down) {
+                // token and routing weight of this warp's 64 activation rows, staged for the tile's output
+                for (int j = lane; j < 64; j += 32) {
+                    const int m = T.m0 + half * 64 + j;
+                    const bool ok = m < T.m_end;
+                    comb_tok[ew * 64 + j] = ok ? p.row_tok[m] : 0;
+                    comb_w[ew * 64 + j] = ok ? p.row_w[m] : 0.0f;
+                }
+            }
+            // group scales travel through a register FIFO SD groups deep
+            float sq[SD];
+#pragma unroll
+            for (int d = 0; d < SD; d++) sq[d] = (srow && d < ngroups) ? __half2float(srow[d]) : 0.0f;
             for (int gl = 0; gl < ngroups; gl++, g++) {
                 const uint32_t db = g & 1;
-                float s = s_next;
-                if (gl + 1 < ngroups) s_next = srow ? __half2float(srow[gl + 1]) : 0.0f;
+                float s = sq[0];
+#pragma unroll
+                for (int d = 0; d + 1 < SD; d++) sq[d] = sq[d + 1];
+                sq[SD - 1] = (srow && gl + SD < ngroups) ? __half2float(srow[gl + SD]) : 0.0f;
                 if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
                 if (!tc::mbar_wait(&sh->d_full[db], (g >> 1) & 1, p.status, abort_flag)) goto epi_done;
                 __syncwarp();
@@ -473,14 +521,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             } else {
                 const int n = T.n0 + r;
                 float* yv = reinterpret_cast<float*>(p.y);
+                __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 64; j++) {
                     const int m = T.m0 + half * 64 + j;
-                    if (m < T.m_end) {
-                        const int pair = p.perm[m];
-                        atomicAdd(yv + (int64_t)(pair / p.topk) * p.N + n, p.topk_w[pair] * acc[j]);
-                    }
+                    if (m < T.m_end)
+                        atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N + n, comb_w[ew * 64 + j] * acc[j]);
                 }
+                __syncwarp();
             }
         }
     epi_done:;

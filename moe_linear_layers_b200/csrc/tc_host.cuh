@@ -58,7 +58,7 @@ int launch(const CUtensorMap& mx, const CUtensorMap& ma, const CUtensorMap& mb, 
 {
     auto kern = tc_gemm_kernel<INT8, G, SYM, MODE>;
     constexpr int smem = Cfg<INT8, MODE>::SMEM;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return Q4_ERR_CUDA;
+    if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return q4_cuda_status(e);
     kern<<<grid, kThreads, smem, s>>>(mx, ma, mb, p);
     return q4_launch_status();
 }

@@ -31,7 +31,7 @@ Q4_ERR_TIMEOUT = -8
 Q4_OUT_F32 = 0
 Q4_OUT_BF16 = 1
 
-EXPORTED = ("q4_status_string", "q4_version", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
+EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
             "q4_linear_w4a16_grouped",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc")
@@ -48,6 +48,7 @@ _i32, _p, _sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
 _lib.q4_status_string.restype = ctypes.c_char_p
 _lib.q4_status_string.argtypes = [ctypes.c_int]
 _lib.q4_version.restype = ctypes.c_int
+_lib.q4_last_cuda_error_string.restype = ctypes.c_char_p
 _lib.q4_linear_w4a16_max_gemv_m.restype = ctypes.c_int
 _lib.q4_quantize_pack.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p]
 _lib.q4_linear_w4a16.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p]
@@ -65,7 +66,10 @@ _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctyp
 
 class Q4Error(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {status} ({_lib.q4_status_string(status).decode()})")
+        msg = f"{what}: {status} ({_lib.q4_status_string(status).decode()})"
+        if status == Q4_ERR_CUDA:
+            msg += ": " + _lib.q4_last_cuda_error_string().decode()
+        super().__init__(msg)
         self.status = status
 
 
