@@ -26,9 +26,12 @@
 //   Down    A = 128 rows of the expert's down projection (fp16 codes), B = h (fp16); epilogue
 //           y[token][n] += w[token][slot] * out (fp32 reduction into the output).
 //
-// Warp roles (448 threads): warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-5
-// converters (TMEM lanes 32*(warp%4) ...), warps 6-13 epilogue (two warps per TMEM lane quarter, each
-// draining 64 of the 128 columns).  Persistent CTAs walk tiles with a stride of gridDim.x; the rings
+// Warp roles (480 threads): warp 0 TMA producer, warps 1-2 MMA issuers (warp 1 also owns TMEM), warps
+// 3-6 converters (TMEM lanes 32*(warp%4) ...), warps 7-14 epilogue (two warps per TMEM lane quarter,
+// each draining 64 of the 128 columns).  The two MMA issuers take alternate K stages: a thread that
+// waits on an mbarrier stalls until the MMAs it issued have retired, so a single issuer would leave
+// the tensor pipe idle at every stage boundary; with two, one issuer's MMAs keep the pipe busy while
+// the other waits.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings
 // carry their phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
 #pragma once
 
@@ -44,7 +47,7 @@ constexpr int KBLK = 128;                // K per stage
 constexpr int NS = 4;                    // shared-memory stages
 constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
 
@@ -240,7 +243,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = 0; i < NS; i++) { tc::mbar_init(&sh->xw_full[i], 1); tc::mbar_init(&sh->xw_empty[i], 1 + 4); }
         for (int i = 0; i < NA; i++) { tc::mbar_init(&sh->a_full[i], 4); tc::mbar_init(&sh->a_empty[i], 1); }
         for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->d_full[i], 1); tc::mbar_init(&sh->d_empty[i], 8); }
-        tc::mbar_init(&sh->done, 1);
+        tc::mbar_init(&sh->done, 2);
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
@@ -290,14 +293,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tc::mbar_wait(&sh->xw_full[j % NS], (j / NS) & 1, p.status, abort_flag, 100000000ull);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp <= 2) {
+        // ------------------------------------------------------------------ MMA issuers (alternate K stages)
         if (lane == 0) {
             constexpr uint32_t idesc = INT8 ? tc::idesc_s8_s32(BN) : (F16 ? tc::idesc_f16_f32(BN) : tc::idesc_bf16_f32(BN));
+            const uint32_t parity = warp - 1;
             uint32_t it = 0, g = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 for (int kb = 0; kb < kblocks && ok; kb++, it++) {
+                    if ((it & 1) != parity) {   // the other issuer's stage
+                        g += GPK;
+                        continue;
+                    }
                     const int s = it % NS, sa = it % NA;
                     ok = tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag) &&
                          tc::mbar_wait(&sh->a_full[sa], (it / NA) & 1, p.status, abort_flag);
@@ -329,7 +337,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mma_commit(&sh->done);   // every MMA issued so far has completed once `done` flips
             tc::mbar_wait(&sh->done, 0, p.status, abort_flag, 100000000ull);
         }
-    } else if (warp < 6) {
+    } else if (warp < 7) {
         // ------------------------------------------------------------------ converters
         const int sub = warp & 3;
         const int r = 32 * sub + lane;                 // row in tile == TMEM lane
@@ -412,7 +420,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     conv_done:;
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int ew = warp - 6;
+        const int ew = warp - 7;
         const int sub = warp & 3, half = ew >> 2;
         const int r = 32 * sub + lane;
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
