@@ -6,23 +6,41 @@
 //
 // HBM-bound design (the packed weights are streamed exactly once):
 //  * each CTA owns a contiguous block of weight rows of one problem; a producer thread streams the
-//    block (packed rows, and their scales and zeros, all contiguous in memory) through a 4-stage
-//    shared-memory ring with cp.async.bulk, completion tracked by mbarriers;
-//  * programmatic dependent launch: the CTA pulls its rows into L2 (a coherent prefetch) before it
-//    waits for the previous kernel on the stream, so consecutive launches keep HBM busy across the
-//    kernel boundary; x (which the previous kernel may produce) is read only after the wait;
-//  * small CTAs (8 compute warps + 1 producer, few registers, ~70 KB shared memory) so that the next
-//    launch's CTAs can be resident, and prefetching, while this launch finishes;
-//  * every lane converts its own 64 values of x to fp16 pairs with its own power-of-two prescale
-//    (max |x| * p in [1, 2): exact), so no block-wide reduction precedes the weight stream;
-//  * in-register dequant: one LOP3 turns two nibbles into fp16x2 "1024 + code"; an HSUB2 of
-//    (1024 + zero) leaves the exact integer (code - zero); nibbles 1, 3, 5, 7 of a word are used in
-//    place (16 * code) and accumulate separately (scaled by 1/16 once per group); products accumulate
-//    in fp16x2 over the lane's 2 chunks of one group (16 products per half), then in fp32 times the
-//    group scale; a lane's two 16-byte chunks are adjacent, so they share one group and one scale;
-//  * rows longer than 2048 codes are split over 2..8 warps and combined through shared memory.
+//    block (packed rows, and their scales and zeros, all contiguous in memory) through a shared-memory
+//    ring with cp.async.bulk, completion tracked by mbarriers;
+//  * programmatic dependent launch, weights first: the weights never depend on the previous kernel on
+//    the stream, so the producer fills the whole ring (and pulls the rest of the CTA's rows into L2)
+//    BEFORE anything waits for that kernel.  CTAs are small enough that the next launch's CTAs are
+//    resident, filling their rings, while this launch computes: HBM stays busy across the chain of
+//    dependent launches of a decode step.  Only the compute warps wait, and only they read x and
+//    write y;
+//  * after the wait, x is converted once per CTA: each thread turns one 16-byte word (8 values) into
+//    int16 with the power-of-two scale of its 64-value block (max |x| * 2^e in [2^14, 2^15): every
+//    bf16 value is kept to 2^-15 of the block maximum), staged in shared memory (XOR-swizzled); every
+//    lane then loads its 64 values and takes their integer sum with DP2A against ones.  (Loading a
+//    lane's 64 contiguous values straight from global memory instead is uncoalesced and slower;)
+//  * integer dot products: a LOP3 spreads the low (high) nibbles of a packed word over four bytes and
+//    two DP2A instructions multiply them with int16 x pairs into an int32 accumulator, so a row's
+//    dot product with the lane's 64 x values (one group) is exact; the zero point comes out as
+//    z * sum(x) in the same integers, and one conversion and one multiply by (group scale * 2^-e)
+//    give the lane's fp32 share.  (DP2A sustains about twice the code rate of an fp16 dequant-and-HFMA2
+//    loop on this GPU, which alone would barely keep up with HBM;)
+//  * a warp handles two rows at a time; their lane sums are reduced together (one exchange, then a
+//    4-step butterfly), so a row costs half the shuffles;
+//  * rows longer than 2048 codes are split over 2..8 warps; their partial sums meet in shared memory
+//    once, at the end of the CTA.
 #include "q4_common.cuh"
 #include "tc_ptx.cuh"
+
+#ifndef Q4_GEMV_STAGES
+#define Q4_GEMV_STAGES 6
+#endif
+#ifndef Q4_GEMV_CTAS_PER_SM
+#define Q4_GEMV_CTAS_PER_SM 1
+#endif
+#ifndef Q4_GEMV_MIN_BLOCKS
+#define Q4_GEMV_MIN_BLOCKS 2
+#endif
 
 namespace {
 
@@ -30,9 +48,12 @@ constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = kComputeWarps * 32;
 constexpr int kThreads = kComputeThreads + 32;      // + one producer warp
 constexpr int kWeightStage = 16384;                 // packed bytes per stage
-constexpr int kStages = 4;
+constexpr int kStages = Q4_GEMV_STAGES;
 constexpr int kMaxM = 4;
 constexpr int kMaxProblems = 8;
+constexpr int kLaneK = 64;                          // k values per lane: two adjacent 16-byte chunks
+constexpr int kWarpK = 32 * kLaneK;                 // 2048
+constexpr int kRedBytesMax = 16384;                 // split-k partial sums per CTA
 
 struct Problem {
     const uint16_t* x;       // [m][k] bf16
@@ -52,17 +73,18 @@ struct GemvParams {
     int rows_per_stage;
     int stage_bytes;         // weights + scales (+ zeros) of one stage, 16-byte multiple
     int bulk_scales;         // scales/zeros travel in the stages (16-byte aligned rows of scales)
+    int xs_off, ips_off, red_off, ring_off;   // shared-memory carve, bytes
     int32_t* status;
 };
 
-// Nibble -> fp16x2 magic: (u & mask) ^ key, key = 0x6400 (1024.0) in both halves, plus the flip of
-// bit 3 of symmetric codes (two's complement -> offset binary: code + 8 = nibble ^ 8).
+// Codes -> bytes: (u & mask) ^ key keeps the low (or high) nibble of every byte of a packed word; for
+// symmetric codes the key flips bit 3 of each nibble (two's complement -> offset binary: code + 8).
 template <bool SYM> struct Keys;
 template <> struct Keys<true> {
-    static constexpr uint32_t k1 = 0x64006400u ^ 0x00080008u, k16 = 0x64006400u ^ 0x00800080u;
+    static constexpr uint32_t lo = 0x08080808u, hi = 0x80808080u, zero = 8;
 };
 template <> struct Keys<false> {
-    static constexpr uint32_t k1 = 0x64006400u, k16 = 0x64006400u;
+    static constexpr uint32_t lo = 0u, hi = 0u, zero = 0;
 };
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
@@ -96,109 +118,155 @@ __device__ __forceinline__ uint4 lds128(const void* p)
     return v;
 }
 
-// Power-of-two prescale p with max|x| * p in [1, 2): exact, and every fp16 partial stays small.
-__device__ __forceinline__ float prescale_for(float amax)
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c)
 {
-    if (!(amax > 0.0f) || !isfinite(amax)) return 1.0f;
-    int e;
-    frexpf(amax, &e);  // amax = f * 2^e, f in [0.5, 1)
-    return ldexpf(1.0f, 1 - e);
+    int d;
+    asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
-// The 8 codes of one 32-bit word against the x pairs of that word.
-// X = {(x0,x4), (x1,x5), (x2,x6), (x3,x7)} as half2 bit patterns.
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// The 8 codes of one 32-bit word against the int16 x of that word, exactly, in int32: the low nibbles
+// (codes 0, 2, 4, 6) as bytes into acc1, the high nibbles in place (16 * code) into acc16.
+// X = {(x0,x2), (x4,x6), (x1,x3), (x5,x7)} as int16 pairs.
 template <bool SYM>
-__device__ __forceinline__ void word_dot(uint32_t u, __half2 b1, __half2 b16, const uint4& X, __half2& acc1,
-                                         __half2& acc16)
+__device__ __forceinline__ void word_dot(uint32_t u, const uint4& X, int& acc1, int& acc16)
 {
-    const uint32_t u8 = u >> 8;
-    const __half2 d0 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x000F000Fu, Keys<SYM>::k1)), b1);
-    const __half2 d1 = __hsub2(u32_as_h2(lop3_and_xor(u, 0x00F000F0u, Keys<SYM>::k16)), b16);
-    const __half2 d2 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x000F000Fu, Keys<SYM>::k1)), b1);
-    const __half2 d3 = __hsub2(u32_as_h2(lop3_and_xor(u8, 0x00F000F0u, Keys<SYM>::k16)), b16);
-    acc1 = __hfma2(d0, u32_as_h2(X.x), acc1);
-    acc16 = __hfma2(d1, u32_as_h2(X.y), acc16);
-    acc1 = __hfma2(d2, u32_as_h2(X.z), acc1);
-    acc16 = __hfma2(d3, u32_as_h2(X.w), acc16);
+    const uint32_t lo = lop3_and_xor(u, 0x0F0F0F0Fu, Keys<SYM>::lo);
+    const uint32_t hi = lop3_and_xor(u, 0xF0F0F0F0u, Keys<SYM>::hi);
+    acc1 = dp2a_lo(X.x, lo, acc1);
+    acc1 = dp2a_hi(X.y, lo, acc1);
+    acc16 = dp2a_lo(X.z, hi, acc16);
+    acc16 = dp2a_hi(X.w, hi, acc16);
 }
 
-// x pairs of one word (8 bf16 values e[0..3]) with prescale p, in the order word_dot consumes them.
-__device__ __forceinline__ uint4 x_pairs(const uint4& v, float p)
+// Power-of-two scale 2^e of a 64-value block with max|x| * 2^e in [2^14, 2^15) (bf16 bits of the max
+// magnitude in, e clamped so that 2^e and 2^-e are normal floats), and its inverse.
+__device__ __forceinline__ float2 block_scale(uint32_t amax_bits)
+{
+    const int ex = (int)((amax_bits >> 7) & 0xFFu);
+    if (amax_bits == 0 || ex == 0xFF) return make_float2(1.0f, 1.0f);
+    const int e = min(126, max(-126, 141 - ex));
+    return make_float2(__uint_as_float((uint32_t)(127 + e) << 23), __uint_as_float((uint32_t)(127 - e) << 23));
+}
+
+// x of one word (8 bf16 values) -> int16 rne(x * scale), in the pair order word_dot consumes.  Adding
+// 1.5 * 2^23 rounds to an integer that sits in the low mantissa bits.
+__device__ __forceinline__ uint4 x_ints(const uint4& v, float scale)
 {
     const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-    float f[8];
+    constexpr float kMagic = 12582912.0f;
+    uint32_t b[8];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        f[2 * i] = __uint_as_float(e[i] << 16) * p;
-        f[2 * i + 1] = __uint_as_float(e[i] & 0xFFFF0000u) * p;
+        b[2 * i] = __float_as_uint(fmaf(__uint_as_float(e[i] << 16), scale, kMagic));
+        b[2 * i + 1] = __float_as_uint(fmaf(__uint_as_float(e[i] & 0xFFFF0000u), scale, kMagic));
     }
     uint4 o;
-    o.x = h2_as_u32(__floats2half2_rn(f[0], f[4]));
-    o.y = h2_as_u32(__floats2half2_rn(f[1], f[5]));
-    o.z = h2_as_u32(__floats2half2_rn(f[2], f[6]));
-    o.w = h2_as_u32(__floats2half2_rn(f[3], f[7]));
+    o.x = prmt(b[0], b[2], 0x5410u);
+    o.y = prmt(b[4], b[6], 0x5410u);
+    o.z = prmt(b[1], b[3], 0x5410u);
+    o.w = prmt(b[5], b[7], 0x5410u);
     return o;
 }
 
-__device__ __forceinline__ float bf16_amax(const uint4& v, bool& finite)
+// Per-halfword max of the bf16 magnitudes of a word (integer order = magnitude order for non-NaN),
+// and a flag for an all-ones exponent (inf or NaN) in any of its 8 values.
+__device__ __forceinline__ uint32_t bf16_mag_max(const uint4& v, uint32_t& bad)
 {
     const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-    float a = 0.0f;
+    uint32_t a = 0;
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        const float lo = __uint_as_float(e[i] << 16), hi = __uint_as_float(e[i] & 0xFFFF0000u);
-        finite &= isfinite(lo) && isfinite(hi);
-        a = fmaxf(a, fmaxf(fabsf(lo), fabsf(hi)));
+        a = __vmaxu2(a, e[i] & 0x7FFF7FFFu);
+        bad |= ((e[i] & 0x7F807F80u) + 0x00800080u) & 0x80008000u;   // carry into bit 15 iff exponent all ones
     }
     return a;
 }
 
-template <int KSPLIT, int J, int MT, bool SYM>
-__global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_kernel(const __grid_constant__ GemvParams p)
+// Dot product of one weight row (in the stage) with the lane's 64 x values, per activation row:
+// sum_k (c_k - z) xi_k = sum_k c_k xi_k - z * sum_k xi_k, exact in int32, then one conversion and the
+// group scale times the block's inverse x scale.
+template <bool SYM, int MT>
+__device__ __forceinline__ void row_dot(const uint8_t* wrow, const __half* srow, const __half* zrow, int gl,
+                                        const uint4 (&X)[MT][8], const float (&inv_xs)[MT], const int (&xsum)[MT],
+                                        float (&part)[MT])
+{
+    const float sc = __half2float(srow[gl]);
+    int z = Keys<SYM>::zero;
+    if constexpr (!SYM) z = (int)(__half_as_ushort(__hadd(zrow[gl], __float2half_rn(1024.0f))) & 0x3FFu);
+    const uint4 w0 = lds128(wrow), w1 = lds128(wrow + 16);
+#pragma unroll
+    for (int mm = 0; mm < MT; mm++) {
+        int a1 = 0, a16 = 0, c1 = 0, c16 = 0;
+        word_dot<SYM>(w0.x, X[mm][0], a1, a16);
+        word_dot<SYM>(w0.y, X[mm][1], c1, c16);
+        word_dot<SYM>(w0.z, X[mm][2], a1, a16);
+        word_dot<SYM>(w0.w, X[mm][3], c1, c16);
+        word_dot<SYM>(w1.x, X[mm][4], a1, a16);
+        word_dot<SYM>(w1.y, X[mm][5], c1, c16);
+        word_dot<SYM>(w1.z, X[mm][6], a1, a16);
+        word_dot<SYM>(w1.w, X[mm][7], c1, c16);
+        const int t = (a1 + c1) + ((a16 + c16) >> 4) - z * xsum[mm];   // a16, c16: multiples of 16
+        part[mm] = (float)t * (sc * inv_xs[mm]);
+    }
+}
+
+__device__ __forceinline__ void store_y(void* y, int64_t o, float v, int out_bf16)
+{
+    if (out_bf16) reinterpret_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+    else reinterpret_cast<float*>(y)[o] = v;
+}
+
+template <int KSPLIT, int MT, bool SYM>
+__global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4a16_gemv_kernel(const __grid_constant__ GemvParams p)
 {
     constexpr int TEAMS = kComputeWarps / KSPLIT;
-    extern __shared__ __align__(16) uint8_t smem[];
+    constexpr bool PAIR = MT <= 2;                  // two rows per warp iteration
+    extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kStages;
-    float* red = reinterpret_cast<float*>(empty + kStages);          // [2][TEAMS][KSPLIT][MT]
-    uint8_t* stages = smem + 1024;
+    uint4* xs = reinterpret_cast<uint4*>(smem + p.xs_off);      // [MT][k/8] int16 x pairs, swizzled
+    float* xinv = reinterpret_cast<float*>(smem + p.ips_off);   // [MT][k/64] 2^-e of each block
+    float* red = reinterpret_cast<float*>(smem + p.red_off);    // [rows_per_cta][KSPLIT][MT]
+    uint8_t* ring = smem + p.ring_off;
 
     // this CTA's problem and rows
     int pi = 0;
     while (pi + 1 < p.count && (int)blockIdx.x >= p.prob[pi + 1].cta_begin) pi++;
     const Problem& P = p.prob[pi];
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-    const int ng = p.k / p.group, cpg = p.group / 32, C = p.k / 32;
+    const int ng = p.k / p.group, C = p.k / 32, nw = p.k / 8;
     const int64_t rowbytes = p.k / 2;
+    const int rps = p.rows_per_stage;
     const int r0 = ((int)blockIdx.x - P.cta_begin) * p.rows_per_cta;
     const int r1 = min(P.n, r0 + p.rows_per_cta);
-    const int nstages = (r1 - r0 + p.rows_per_stage - 1) / p.rows_per_stage;
-    const int wbytes = p.rows_per_stage * (int)rowbytes;            // weight part of a stage
-    const int sbytes = p.rows_per_stage * ng * 2;                   // scale part of a stage
+    const int nstages = (r1 - r0 + rps - 1) / rps;
+    const int wbytes = rps * (int)rowbytes;                     // weight part of a stage
+    const int sbytes = rps * ng * 2;                            // scale part of a stage
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kComputeWarps); }
         tc::fence_mbar_init();
     }
-    if (warp == kComputeWarps && lane == 0 && r0 < r1) {
-        // weights do not depend on the previous kernel: start pulling them into L2 now
-        prefetch_l2_range(P.packed + (int64_t)r0 * rowbytes, P.packed + (int64_t)r1 * rowbytes);
-        prefetch_l2_range(P.scales + (int64_t)r0 * ng, P.scales + (int64_t)r1 * ng);
-        if constexpr (!SYM) prefetch_l2_range(P.zeros + (int64_t)r0 * ng, P.zeros + (int64_t)r1 * ng);
-    }
     __syncthreads();
     pdl_launch_dependents();
-    pdl_wait();
 
     if (warp == kComputeWarps) {
-        // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            for (int st = 0; st < nstages; st++) {
+        // ------------------------------------------------------------------ producer (never waits for
+        // the previous kernel: it reads only weights)
+        if (lane == 0 && nstages > 0) {
+            auto issue = [&](int st) {
                 const int s = st % kStages;
-                if (!tc::mbar_wait(&empty[s], ((st / kStages) & 1) ^ 1, p.status, nullptr)) break;
-                const int rs = r0 + st * p.rows_per_stage;
-                const int rows = min(p.rows_per_stage, r1 - rs);
-                uint8_t* dst = stages + s * p.stage_bytes;
+                const int rs = r0 + st * rps;
+                const int rows = min(rps, r1 - rs);
+                uint8_t* dst = ring + s * p.stage_bytes;
                 uint32_t bytes = (uint32_t)(rows * rowbytes);
                 if (p.bulk_scales) bytes += (uint32_t)(rows * ng * 2 * (SYM ? 1 : 2));
                 tc::mbar_arrive_expect_tx(&full[s], bytes);
@@ -208,129 +276,182 @@ __global__ void __launch_bounds__(kThreads, 2) w4a16_gemv_kernel(const __grid_co
                     if constexpr (!SYM)
                         bulk_g2s(dst + wbytes + sbytes, P.zeros + (int64_t)rs * ng, (uint32_t)(rows * ng * 2), &full[s]);
                 }
+            };
+            const int pre = min(nstages, kStages);
+            for (int st = 0; st < pre; st++) issue(st);
+            // x too: an L2 prefetch is coherent, so it is safe before the wait and shortens the read after it
+            prefetch_l2(P.x, (uint32_t)(p.m * p.k * 2));
+            if (nstages > kStages) {
+                const int rl = r0 + kStages * rps;
+                prefetch_l2_range(P.packed + (int64_t)rl * rowbytes, P.packed + (int64_t)r1 * rowbytes);
+                if (p.bulk_scales) {
+                    prefetch_l2_range(P.scales + (int64_t)rl * ng, P.scales + (int64_t)r1 * ng);
+                    if constexpr (!SYM) prefetch_l2_range(P.zeros + (int64_t)rl * ng, P.zeros + (int64_t)r1 * ng);
+                }
+            }
+            for (int st = kStages; st < nstages; st++) {
+                if (!tc::mbar_wait(&empty[st % kStages], ((st / kStages) & 1) ^ 1, p.status, nullptr)) break;
+                issue(st);
             }
         }
         return;
     }
 
     // ---------------------------------------------------------------------- compute warps
-    const int team = warp / KSPLIT, ks = warp % KSPLIT;
-    const int c0 = ks * 32 * J + J * lane;          // the lane's first chunk (J adjacent chunks)
-    const bool cvalid = c0 < C;
-    const int gl = c0 / cpg;                        // their group (J <= cpg, c0 % J == 0)
+    pdl_wait();   // x (and the y buffer) may belong to the previous kernel on the stream
 
-    // x of the lane's chunks -> fp16 pairs with the lane's own power-of-two prescale
-    uint4 X[MT][J][4];
-    float inv_ps[MT];
+    // x -> int16 with the power-of-two scale of its 64-value block: one 16-byte word (8 values) per
+    // thread and pass (coalesced), all loads issued first and the passes independent of one another;
+    // the 8 threads of a block share its scale.  Word w of block L is staged at 8L + ((w % 8) ^ (L % 8)):
+    // conflict-free lane loads.
+    {
+        constexpr int kMaxPasses = 16384 / 8 / kComputeThreads;
+        uint32_t bad = 0;
+#pragma unroll
+        for (int mm = 0; mm < MT; mm++) {
+            const uint4* xrow = reinterpret_cast<const uint4*>(P.x + (int64_t)mm * p.k);
+            uint4 raw[kMaxPasses];
+#pragma unroll
+            for (int i = 0; i < kMaxPasses; i++) {
+                const int w = i * kComputeThreads + threadIdx.x;
+                raw[i] = w < nw ? __ldg(xrow + w) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < kMaxPasses; i++) {
+                if (i * kComputeThreads < nw) {   // uniform; nw % 8 == 0 keeps blocks of 8 threads together
+                    const int w = i * kComputeThreads + threadIdx.x;
+                    uint32_t a = bf16_mag_max(raw[i], bad);
+                    a = __vmaxu2(a, __shfl_xor_sync(0xffffffffu, a, 1));
+                    a = __vmaxu2(a, __shfl_xor_sync(0xffffffffu, a, 2));
+                    a = __vmaxu2(a, __shfl_xor_sync(0xffffffffu, a, 4));
+                    const float2 sc = block_scale(max(a & 0xFFFFu, a >> 16));
+                    if (w < nw) {
+                        const int L = w >> 3, j = w & 7;
+                        xs[mm * nw + (L << 3) + (j ^ (L & 7))] = x_ints(raw[i], sc.x);
+                        if (j == 0) xinv[mm * (nw / 8) + L] = sc.y;
+                    }
+                }
+            }
+        }
+        if (bad) q4_set_status(p.status, Q4_ERR_NONFINITE);
+    }
+    compute_bar();
+
+    const int team = warp / KSPLIT, ks = warp % KSPLIT;
+    const int L = ks * 32 + lane;                   // the lane's 64-value block of k
+    const int c0 = 2 * L;                           // its first 16-byte chunk
+    const bool cvalid = c0 < C;
+    const int gl = L * kLaneK / p.group;            // its group
+    uint4 X[MT][8];
+    float inv_xs[MT];
+    int xsum[MT];
 #pragma unroll
     for (int mm = 0; mm < MT; mm++) {
-        uint4 raw[J][4];
-        float amax = 0.0f;
-        bool finite = true;
 #pragma unroll
-        for (int j = 0; j < J; j++)
+        for (int i = 0; i < 8; i++)
+            X[mm][i] = cvalid ? xs[mm * nw + (L << 3) + (i ^ (L & 7))] : make_uint4(0, 0, 0, 0);
+        inv_xs[mm] = cvalid ? xinv[mm * (nw / 8) + L] : 0.0f;
+        // the lane's integer sum of x, for the zero point: DP2A against ones, four chains
+        int s4[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int w = 0; w < 4; w++) {
-                raw[j][w] = cvalid ? __ldg(reinterpret_cast<const uint4*>(P.x + (int64_t)mm * p.k + 32 * (c0 + j)) + w)
-                                   : make_uint4(0, 0, 0, 0);
-                amax = fmaxf(amax, bf16_amax(raw[j][w], finite));
-            }
-        if (!finite) q4_set_status(p.status, Q4_ERR_NONFINITE);
-        const float ps = prescale_for(amax);
-        inv_ps[mm] = 1.0f / ps;
-#pragma unroll
-        for (int j = 0; j < J; j++)
-#pragma unroll
-            for (int w = 0; w < 4; w++) X[mm][j][w] = x_pairs(raw[j][w], ps);
+        for (int i = 0; i < 8; i++) {
+            s4[0] = dp2a_lo(X[mm][i].x, 0x01010101u, s4[0]);
+            s4[1] = dp2a_lo(X[mm][i].y, 0x01010101u, s4[1]);
+            s4[2] = dp2a_lo(X[mm][i].z, 0x01010101u, s4[2]);
+            s4[3] = dp2a_lo(X[mm][i].w, 0x01010101u, s4[3]);
+        }
+        xsum[mm] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     }
 
     for (int st = 0; st < nstages; st++) {
         const int s = st % kStages;
-        const int rs = r0 + st * p.rows_per_stage;
-        const int rows_here = min(p.rows_per_stage, r1 - rs);
+        const int rs = r0 + st * rps;
+        const int rows_here = min(rps, r1 - rs);
         if (!tc::mbar_wait(&full[s], (st / kStages) & 1, p.status, nullptr)) break;
-        const uint8_t* sb = stages + s * p.stage_bytes;
-        const __half* ssc = reinterpret_cast<const __half*>(sb + wbytes);
-        const __half* szr = reinterpret_cast<const __half*>(sb + wbytes + sbytes);
-        float* redb = red + (st & 1) * TEAMS * KSPLIT * MT;
-        for (int rr = team; rr < rows_here; rr += TEAMS) {
-            const int row = rs + rr;
-            float part[MT];
+        const uint8_t* sb = ring + s * p.stage_bytes;
+        for (int ra = team; ra < rows_here; ra += (PAIR ? 2 : 1) * TEAMS) {
+            const int rb = ra + TEAMS;
+            const bool hasb = PAIR && rb < rows_here;
+            float pa[MT], pb[MT];
 #pragma unroll
-            for (int mm = 0; mm < MT; mm++) part[mm] = 0.0f;
+            for (int mm = 0; mm < MT; mm++) pa[mm] = pb[mm] = 0.0f;
             if (cvalid) {
-                float sc;
-                __half z;
-                if (p.bulk_scales) {
-                    sc = __half2float(ssc[rr * ng + gl]);
-                    z = SYM ? __float2half_rn(8.0f) : szr[rr * ng + gl];
-                } else {
-                    sc = __half2float(P.scales[(int64_t)row * ng + gl]);
-                    z = SYM ? __float2half_rn(8.0f) : P.zeros[(int64_t)row * ng + gl];
+                const __half* sa = p.bulk_scales ? reinterpret_cast<const __half*>(sb + wbytes) + ra * ng
+                                                 : P.scales + (int64_t)(rs + ra) * ng;
+                const __half* za = p.bulk_scales ? reinterpret_cast<const __half*>(sb + wbytes + sbytes) + ra * ng
+                                                 : P.zeros + (int64_t)(rs + ra) * ng;
+                row_dot<SYM, MT>(sb + ra * rowbytes + c0 * 16, sa, za, gl, X, inv_xs, xsum, pa);
+                if (hasb) {
+                    const int d = (rb - ra) * ng;
+                    row_dot<SYM, MT>(sb + rb * rowbytes + c0 * 16, sa + d, SYM ? za : za + d, gl, X, inv_xs, xsum, pb);
                 }
-                const __half2 b1 = __half2half2(__hadd(z, __float2half_rn(1024.0f)));
-                const __half2 b16 = __half2half2(__hfma(z, __float2half_rn(16.0f), __float2half_rn(1024.0f)));
-                uint4 wv[J];
-#pragma unroll
-                for (int j = 0; j < J; j++) wv[j] = lds128(sb + rr * rowbytes + (c0 + j) * 16);
+            }
+            if constexpr (PAIR) {
+                // lanes 0-15 end with row a, lanes 16-31 with row b
+                const bool hi = lane & 16;
 #pragma unroll
                 for (int mm = 0; mm < MT; mm++) {
-                    __half2 acc1 = __float2half2_rn(0.0f), acc16 = __float2half2_rn(0.0f);
+                    float v = hi ? pb[mm] : pa[mm];
+                    v += __shfl_xor_sync(0xffffffffu, hi ? pa[mm] : pb[mm], 16);
 #pragma unroll
-                    for (int j = 0; j < J; j++) {
-                        word_dot<SYM>(wv[j].x, b1, b16, X[mm][j][0], acc1, acc16);
-                        word_dot<SYM>(wv[j].y, b1, b16, X[mm][j][1], acc1, acc16);
-                        word_dot<SYM>(wv[j].z, b1, b16, X[mm][j][2], acc1, acc16);
-                        word_dot<SYM>(wv[j].w, b1, b16, X[mm][j][3], acc1, acc16);
-                    }
-                    const float2 f = __half22float2(__hfma2(acc16, __float2half2_rn(0.0625f), acc1));
-                    part[mm] = sc * (f.x + f.y) * inv_ps[mm];
+                    for (int off = 8; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    pa[mm] = v;
                 }
-            }
+                if ((lane & 15) == 0 && (!hi || hasb)) {
+                    const int rr = hi ? rb : ra;
 #pragma unroll
-            for (int mm = 0; mm < MT; mm++) {
+                    for (int mm = 0; mm < MT; mm++) {
+                        if constexpr (KSPLIT == 1) store_y(P.y, (int64_t)mm * P.n + rs + rr, pa[mm], p.out_bf16);
+                        else red[((rs - r0 + rr) * KSPLIT + ks) * MT + mm] = pa[mm];
+                    }
+                }
+            } else {
 #pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) part[mm] += __shfl_xor_sync(0xffffffffu, part[mm], off);
-            }
-            if (lane < MT) {
-                float v = part[0];
+                for (int mm = 0; mm < MT; mm++)
 #pragma unroll
-                for (int mm = 1; mm < MT; mm++) if (lane == mm) v = part[mm];
-                if constexpr (KSPLIT == 1) {
-                    const int64_t o = (int64_t)lane * P.n + row;
-                    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
-                    else reinterpret_cast<float*>(P.y)[o] = v;
-                } else {
-                    redb[(team * KSPLIT + ks) * MT + lane] = v;   // one row per team per stage
+                    for (int off = 16; off >= 1; off >>= 1) pa[mm] += __shfl_xor_sync(0xffffffffu, pa[mm], off);
+                if (lane < MT) {
+                    float v = pa[0];
+#pragma unroll
+                    for (int mm = 1; mm < MT; mm++) if (lane == mm) v = pa[mm];
+                    if constexpr (KSPLIT == 1) store_y(P.y, (int64_t)lane * P.n + rs + ra, v, p.out_bf16);
+                    else red[((rs - r0 + ra) * KSPLIT + ks) * MT + lane] = v;
                 }
             }
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&empty[s]);
-        if constexpr (KSPLIT > 1) {
-            compute_bar();
-            if (ks == 0 && team < rows_here && lane < MT) {
-                float v = 0.0f;
+    }
+
+    if constexpr (KSPLIT > 1) {
+        compute_bar();
+        const int rows = r1 - r0;
+        for (int i = threadIdx.x; i < rows * MT; i += kComputeThreads) {
+            const int rr = i / MT, mm = i % MT;
+            float v = 0.0f;
 #pragma unroll
-                for (int t = 0; t < KSPLIT; t++) v += redb[(team * KSPLIT + t) * MT + lane];
-                const int64_t o = (int64_t)lane * P.n + (rs + team);
-                if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
-                else reinterpret_cast<float*>(P.y)[o] = v;
-            }
+            for (int t = 0; t < KSPLIT; t++) v += red[(rr * KSPLIT + t) * MT + mm];
+            store_y(P.y, (int64_t)mm * P.n + r0 + rr, v, p.out_bf16);
         }
     }
 }
 
-template <int KSPLIT, int J, int MT>
-int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
+template <int KSPLIT, int MT>
+int launch(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStream_t s)
 {
-    const size_t smem = 1024 + (size_t)kStages * p.stage_bytes;
-    if (smem > 227 * 1024) return Q4_ERR_UNSUPPORTED;
-    auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, J, MT, true> : w4a16_gemv_kernel<KSPLIT, J, MT, false>;
-    if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
-        return q4_cuda_status(e);
-    // Programmatic stream serialization: the kernel may start (and prefetch its weights into L2) while
-    // the previous kernel on the stream drains; it reads x only after griddepcontrol.wait.
+    auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, MT, true> : w4a16_gemv_kernel<KSPLIT, MT, false>;
+    // the shared-memory opt-in is set once per device and instantiation (it does not affect occupancy)
+    static uint64_t opted[2] = {0, 0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(opted[symmetric ? 1 : 0] & bit)) {
+        if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024))
+            return q4_cuda_status(e);
+        opted[symmetric ? 1 : 0] |= bit;
+    }
+    // Programmatic stream serialization: the kernel may start, and fill its weight ring, while the
+    // previous kernel on the stream runs; x is read only after griddepcontrol.wait.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -344,25 +465,14 @@ int launch(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
     return q4_cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
-template <int KSPLIT, int J>
-int launch_m(const GemvParams& p, int symmetric, int grid, cudaStream_t s)
+template <int KSPLIT>
+int launch_m(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStream_t s)
 {
     switch (p.m) {
-        case 1: return launch<KSPLIT, J, 1>(p, symmetric, grid, s);
-        case 2: return launch<KSPLIT, J, 2>(p, symmetric, grid, s);
-        case 3: return launch<KSPLIT, J, 3>(p, symmetric, grid, s);
-        default: return launch<KSPLIT, J, 4>(p, symmetric, grid, s);
-    }
-}
-
-template <int J>
-int launch_ksplit(const GemvParams& p, int symmetric, int ksplit, int grid, cudaStream_t s)
-{
-    switch (ksplit) {
-        case 1: return launch_m<1, J>(p, symmetric, grid, s);
-        case 2: return launch_m<2, J>(p, symmetric, grid, s);
-        case 4: return launch_m<4, J>(p, symmetric, grid, s);
-        default: return launch_m<8, J>(p, symmetric, grid, s);
+        case 1: return launch<KSPLIT, 1>(p, symmetric, grid, smem, s);
+        case 2: return launch<KSPLIT, 2>(p, symmetric, grid, smem, s);
+        case 3: return launch<KSPLIT, 3>(p, symmetric, grid, smem, s);
+        default: return launch<KSPLIT, 4>(p, symmetric, grid, smem, s);
     }
 }
 
@@ -385,26 +495,32 @@ int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, c
     p.group = group;
     p.out_bf16 = out_dtype == Q4_OUT_BF16;
     p.status = dev_status;
-    const int C = k / 32;
-    const int J = 2;                                   // two adjacent chunks (64 codes) per lane
     int ksplit = 1;
-    while (ksplit * 32 * J < C) ksplit *= 2;
+    while (ksplit * kWarpK < k) ksplit *= 2;
     if (ksplit > 8) return Q4_ERR_UNSUPPORTED;
-    const int teams = kComputeWarps / ksplit;
     const int rowbytes = k / 2;
     const int ng = k / group;
-    int rps = ksplit > 1 ? teams : std::max(1, kWeightStage / rowbytes);
+    const int rps = std::max(1, kWeightStage / rowbytes);
     p.rows_per_stage = rps;
     p.bulk_scales = (ng * 2) % 16 == 0;
     p.stage_bytes = rps * rowbytes + (p.bulk_scales ? rps * ng * 2 * (sym ? 1 : 2) : 0);
     p.stage_bytes = (p.stage_bytes + 15) & ~15;
-    // rows per CTA: about two CTAs per SM over the whole group, whole stages where possible
+    // rows per CTA: a fixed number of CTAs per SM over the whole group
     int64_t rows_total = 0;
     for (int i = 0; i < count; i++) rows_total += w[i].n;
-    const int64_t target_ctas = 2LL * q4_num_sms();
+    const int64_t target_ctas = (int64_t)Q4_GEMV_CTAS_PER_SM * q4_num_sms();
+    // (balanced over the SMs: a CTA's last stage may be partial)
     int rpc = (int)std::max<int64_t>(1, (rows_total + target_ctas - 1) / target_ctas);
-    if (rpc > rps) rpc = (rpc + rps - 1) / rps * rps;
+    if (ksplit > 1) rpc = std::min(rpc, std::max(rps, kRedBytesMax / (ksplit * m * 4)));
     p.rows_per_cta = rpc;
+    // shared memory: barriers | int16 x | per-block inverse scale | split-k partials | weight ring
+    p.xs_off = 128;
+    p.ips_off = p.xs_off + m * k * 2;
+    p.red_off = p.ips_off + m * (k / 64) * 4;
+    const int red_bytes = ksplit > 1 ? rpc * ksplit * m * 4 : 0;
+    p.ring_off = (p.red_off + red_bytes + 127) & ~127;
+    const size_t smem = (size_t)p.ring_off + (size_t)kStages * p.stage_bytes;
+    if (smem > 227 * 1024) return Q4_ERR_UNSUPPORTED;
     int ctas = 0;
     for (int i = 0; i < count; i++) {
         Problem& P = p.prob[i];
@@ -418,5 +534,10 @@ int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, c
         ctas += (w[i].n + rpc - 1) / rpc;
     }
     if (ctas == 0) return Q4_OK;
-    return launch_ksplit<2>(p, sym, ksplit, ctas, stream);
+    switch (ksplit) {
+        case 1: return launch_m<1>(p, sym, ctas, smem, stream);
+        case 2: return launch_m<2>(p, sym, ctas, smem, stream);
+        case 4: return launch_m<4>(p, sym, ctas, smem, stream);
+        default: return launch_m<8>(p, sym, ctas, smem, stream);
+    }
 }
