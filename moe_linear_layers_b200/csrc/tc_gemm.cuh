@@ -26,13 +26,18 @@
 //   Down    A = 128 rows of the expert's down projection (fp16 codes), B = h (fp16); epilogue
 //           y[token][n] += w[token][slot] * out (fp32 reduction into the output).
 //
-// Warp roles (480 threads): warp 0 TMA producer, warps 1-2 MMA issuers (warp 1 also owns TMEM), warps
-// 3-6 converters (TMEM lanes 32*(warp%4) ...), warps 7-14 epilogue (two warps per TMEM lane quarter,
-// each draining 64 of the 128 columns).  The two MMA issuers take alternate K stages: a thread that
-// waits on an mbarrier stalls until the MMAs it issued have retired, so a single issuer would leave
-// the tensor pipe idle at every stage boundary; with two, one issuer's MMAs keep the pipe busy while
-// the other waits.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings
-// carry their phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
+// Warp roles (512 threads, 16 warps = 4 per SM sub-partition at 128 registers): warps 0 and 15 TMA
+// producers (alternate stages), warps 1-2 MMA issuers (warp 1 also owns TMEM), warps 3-6 converters
+// (TMEM lanes 32*(warp%4) ...), warps 7-14 epilogue (two warps per TMEM lane quarter, each draining 64
+// of the 128 columns).  A thread that waits on an mbarrier stalls until the asynchronous operations it
+// issued (bulk copies, MMAs) have completed, so every asynchronous stream is split over two threads in
+// different warps that take alternate stages: one keeps the TMA engine (or the tensor pipe) busy while
+// the other waits.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their phases
+// across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
+//
+// Epilogue arithmetic runs on packed fp32 pairs (FFMA2).  For W4A8 every int32 accumulator is preloaded
+// with the bit pattern of 1.5 * 2^23, so the accumulated bits are the float 1.5 * 2^23 + acc and one
+// packed subtraction replaces an integer-to-float conversion per value.
 #pragma once
 
 #include "tc_ptx.cuh"
@@ -44,12 +49,14 @@ enum class Mode { Dense, GateUp, Down };
 constexpr int BM = 128;                  // weight rows per tile
 constexpr int BN = 128;                  // activation rows per tile
 constexpr int KBLK = 128;                // K per stage
-constexpr int NS = 4;                    // shared-memory stages
+constexpr int NS = 4;                    // shared-memory stages (activations + packed weights)
 constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
-constexpr int kThreads = 480;
+constexpr int kThreads = 512;            // 16 warps: 4 per SM sub-partition, 128 registers each
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
+constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
+constexpr float kAccBiasF = 12582912.0f;
 
 template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2);   // activation bytes per stage
@@ -57,6 +64,7 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     static constexpr uint32_t A_COL0 = 2 * BN;                  // widened weights after the 2 D buffers
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
+    static_assert(NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144 <= 227 * 1024, "shared memory");
     static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144;
 };
 
@@ -158,6 +166,8 @@ struct Shared {
     int comb_tok[8 * 64];      // Down: token of each activation row of the tile, per epilogue warp
     float comb_w[8 * 64];      // Down: its routing weight
 };
+static_assert(sizeof(Shared) <= 6144, "Shared must fit the space reserved in Cfg::SMEM");
+
 
 constexpr int ZD = 4;   // depth of the converters' zero-point FIFO (K stages)
 constexpr int SD = 4;   // depth of the epilogue's scale FIFO (groups)
@@ -265,15 +275,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t tbase = sh->tmem_base;
     const int total = sh->total_tiles;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == kThreads / 32 - 1) {
+        // ------------------------------------------------------------------ TMA producers
+        // Two producer threads in different warps take alternate stages: a thread that waits on an
+        // mbarrier stalls until its own outstanding bulk copies have landed, so one thread alone would
+        // issue only one stage per L2 round trip.
         if (lane == 0) {
+            const uint32_t parity = warp == 0 ? 0u : 1u;
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
                 for (int kb = 0; kb < kblocks; kb++, it++) {
+                    if ((it & 1u) != parity) continue;
                     const int s = it % NS;
-                    if (!tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag)) break;
+                    if (!(ok = tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag))) break;
                     tc::mbar_arrive_expect_tx(&sh->xw_full[s], C::XSTAGE + WSTAGE);
                     uint8_t* xdst = xs + s * C::XSTAGE;
                     tc::tma_load_2d(xdst, &tm_x, &sh->xw_full[s], kb * KBLK, T.m0);
@@ -287,10 +303,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                 }
             }
-            if (*abort_flag) {  // let every copy this thread issued land before the CTA can exit
-                const uint32_t first = it > (uint32_t)NS ? it - NS : 0;
-                for (uint32_t j = first; j < it; j++)
-                    tc::mbar_wait(&sh->xw_full[j % NS], (j / NS) & 1, p.status, abort_flag, 100000000ull);
+            if (!ok || *abort_flag) {  // let every copy this thread issued land before the CTA can exit
+                for (uint32_t j = it > (uint32_t)NS ? it - NS : 0; j < it; j++)
+                    if ((j & 1u) == parity)
+                        tc::mbar_wait(&sh->xw_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
             }
         }
     } else if (warp <= 2) {
@@ -315,7 +331,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++, g++) {
                         const uint32_t db = g & 1;
-                        if (!(ok = tc::mbar_wait(&sh->d_empty[db], ((g >> 1) & 1) ^ 1, p.status, abort_flag))) break;
+                        // INT8: the epilogue pre-loads the accumulator (see below) and releases it once first
+                        const uint32_t dpar = INT8 ? ((g >> 1) & 1) : (((g >> 1) & 1) ^ 1);
+                        if (!(ok = tc::mbar_wait(&sh->d_empty[db], dpar, p.status, abort_flag))) break;
                         tc::fence_after_sync();
 #pragma unroll
                         for (int i = 0; i < G / C::KI; i++) {
@@ -325,7 +343,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             if constexpr (INT8) boff = kk;                              // one 128-byte row box
                             else boff = (kk / 64) * (BN * 128) + (kk % 64) * 2;          // two 64-column boxes
                             const uint64_t bdesc = tc::smem_desc_sw128(xaddr + (boff & ~127u)) + ((boff & 127u) >> 4);
-                            if constexpr (INT8) tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                            if constexpr (INT8) tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, true);
                             else tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
                         }
                         tc::mma_commit(&sh->d_full[db]);
@@ -425,13 +443,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int r = 32 * sub + lane;
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
         uint32_t g = 0, tl = 0;
-        float acc[64];
+        // fp32 accumulators in packed pairs: acc2[j] holds the values of columns 2j and 2j+1
+        uint64_t acc2[32];
+        auto accv = [&](int j) { return (j & 1) ? tc::f2_hi(acc2[j >> 1]) : tc::f2_lo(acc2[j >> 1]); };
+        if constexpr (INT8) {
+            // Every int32 accumulator starts at the bit pattern of 1.5 * 2^23 (as a float), so after the
+            // group's MMAs its bits ARE the float 1.5 * 2^23 + acc (|acc| < 2^22): the epilogue converts
+            // with one packed subtraction instead of an integer-to-float conversion per value.
+#pragma unroll
+            for (int d = 0; d < 2; d++)
+#pragma unroll
+                for (int h = 0; h < 2; h++) tc::tmem_fill32(tbase + lane_field + d * BN + half * 64 + 32 * h, kAccBias);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) { tc::mbar_arrive(&sh->d_empty[0]); tc::mbar_arrive(&sh->d_empty[1]); }
+        }
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
 #pragma unroll
-            for (int j = 0; j < 64; j++) acc[j] = 0.0f;
+            for (int j = 0; j < 32; j++) acc2[j] = 0;
             if (t + (int)gridDim.x < total) {  // warm L2 with the next tile's scale row
                 const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
                 const __half *sn, *zn;
@@ -458,6 +491,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 for (int d = 0; d + 1 < SD; d++) sq[d] = sq[d + 1];
                 sq[SD - 1] = (srow && gl + SD < ngroups) ? __half2float(srow[gl + SD]) : 0.0f;
                 if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
+                const uint64_t s2 = tc::f2_pack(__float_as_uint(s), __float_as_uint(s));
                 if (!tc::mbar_wait(&sh->d_full[db], (g >> 1) & 1, p.status, abort_flag)) goto epi_done;
                 __syncwarp();
                 tc::fence_after_sync();
@@ -471,33 +505,74 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
-                                if (m < T.m_end) p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)v[j]) >> 4;
+                                if (m < T.m_end)
+                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)(v[j] - kAccBias)) >> 4;
                             }
                         }
+                        const uint64_t nb2 = tc::f2_pack(__float_as_uint(-kAccBiasF), __float_as_uint(-kAccBiasF));
 #pragma unroll
-                        for (int j = 0; j < 32; j++) acc[32 * h + j] = fmaf(s, (float)(int32_t)v[j], acc[32 * h + j]);
+                        for (int j = 0; j < 16; j++)
+                            acc2[16 * h + j] = tc::f2_fma(s2, tc::f2_add(tc::f2_pack(v[2 * j], v[2 * j + 1]), nb2), acc2[16 * h + j]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; j++) acc[32 * h + j] = fmaf(s, __uint_as_float(v[j]), acc[32 * h + j]);
+                        for (int j = 0; j < 16; j++)
+                            acc2[16 * h + j] = tc::f2_fma(s2, tc::f2_pack(v[2 * j], v[2 * j + 1]), acc2[16 * h + j]);
                     }
+                }
+                if constexpr (INT8) {
+                    // hand the columns back pre-loaded for the next group in this buffer
+                    tc::tmem_fill32(tbase + lane_field + db * BN + half * 64, kAccBias);
+                    tc::tmem_fill32(tbase + lane_field + db * BN + half * 64 + 32, kAccBias);
+                    tc::tmem_wait_st();
                 }
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sh->d_empty[db]);
             }
             // ---------------------------------------------------------- tile output
+            // (every loop below has a branch-free path for a full 64-row block: a conditional branch per
+            // row costs more than the store it guards)
             if constexpr (MODE == Mode::Dense) {
                 const int n = T.n0 + r;
-                if (n < p.N) {
+                const int mb = T.m0 + half * 64;
+                const int rows = min(64, p.M - mb);
+                if (n < p.N && rows > 0) {
+                    const int64_t base = (int64_t)mb * p.N + n;
+                    if (p.out_bf16) {
+                        __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(p.y) + base;
+                        if (rows == 64) {
 #pragma unroll
-                    for (int j = 0; j < 64; j++) {
-                        const int m = T.m0 + half * 64 + j;
-                        if (m < p.M) {
-                            float v = acc[j];
-                            if constexpr (INT8) v *= p.scale_a[m];
-                            const int64_t o = (int64_t)m * p.N + n;
-                            if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
-                            else reinterpret_cast<float*>(p.y)[o] = v;
+                            for (int j = 0; j < 64; j++) {
+                                float v = accv(j);
+                                if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
+                                yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 64; j++)
+                                if (j < rows) {
+                                    float v = accv(j);
+                                    if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
+                                    yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
+                                }
+                        }
+                    } else {
+                        float* yf = reinterpret_cast<float*>(p.y) + base;
+                        if (rows == 64) {
+#pragma unroll
+                            for (int j = 0; j < 64; j++) {
+                                float v = accv(j);
+                                if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
+                                yf[(int64_t)j * p.N] = v;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 64; j++)
+                                if (j < rows) {
+                                    float v = accv(j);
+                                    if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
+                                    yf[(int64_t)j * p.N] = v;
+                                }
                         }
                     }
                 }
@@ -508,33 +583,43 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     // the buffer is free once the gate rows consumed the previous tile's values
                     if (!tc::mbar_wait(&sh->gate_done, (tl & 1) ^ 1, p.status, abort_flag)) goto epi_done;
 #pragma unroll
-                    for (int j = 0; j < 64; j++) xb[j * 64 + (r - 64)] = acc[j];
+                    for (int j = 0; j < 64; j++) xb[j * 64 + (r - 64)] = accv(j);
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&sh->up_ready);
                 } else {
                     if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
                     const int i = T.n0 + r;
+                    const int mb = T.m0 + half * 64;
+                    const int rows = min(64, T.m_end - mb);
+                    __half* hb = p.h + (int64_t)mb * p.N + i;
+                    auto swiglu = [&](int j) {
+                        const float gv = accv(j), uv = xb[j * 64 + r];
+                        return __float2half_rn(gv * __frcp_rn(1.0f + __expf(-gv)) * uv);
+                    };
+                    if (rows == 64) {
 #pragma unroll
-                    for (int j = 0; j < 64; j++) {
-                        const int m = T.m0 + half * 64 + j;
-                        if (m < T.m_end) {
-                            const float gv = acc[j], uv = xb[j * 64 + r];
-                            const float hv = gv / (1.0f + expf(-gv)) * uv;
-                            p.h[(int64_t)m * p.N + i] = __float2half_rn(hv);
-                        }
+                        for (int j = 0; j < 64; j++) hb[(int64_t)j * p.N] = swiglu(j);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; j++)
+                            if (j < rows) hb[(int64_t)j * p.N] = swiglu(j);
                     }
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&sh->gate_done);
                 }
             } else {
                 const int n = T.n0 + r;
-                float* yv = reinterpret_cast<float*>(p.y);
+                float* yv = reinterpret_cast<float*>(p.y) + n;
+                const int rows = min(64, T.m_end - (T.m0 + half * 64));
                 __syncwarp();
+                if (rows == 64) {
 #pragma unroll
-                for (int j = 0; j < 64; j++) {
-                    const int m = T.m0 + half * 64 + j;
-                    if (m < T.m_end)
-                        atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N + n, comb_w[ew * 64 + j] * acc[j]);
+                    for (int j = 0; j < 64; j++)
+                        atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; j++)
+                        if (j < rows) atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
                 }
                 __syncwarp();
             }

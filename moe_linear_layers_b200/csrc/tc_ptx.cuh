@@ -189,6 +189,45 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// ---------------------------------------------------------------------------------------------- //
+// packed fp32 pairs (sm_100 f32x2 arithmetic; each half rounds exactly like the scalar instruction)
+// ---------------------------------------------------------------------------------------------- //
+
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Warp-wide: thread t fills TMEM lane (lane field of taddr) + t, 32 consecutive columns, with one value.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+        "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};"
+        ::"r"(taddr), "r"(v)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major tile written by TMA with 128-byte swizzle:
 // rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset), base 1024-byte aligned.
 // Advancing along K inside the 128-byte row adds (bytes >> 4) to the start address.
