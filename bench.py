@@ -17,6 +17,7 @@ At one GPU the line also carries "components", the other rows of the hot path on
   moe      the MoE layer: 4096 tokens, hidden 2048, 64 experts of intermediate 1024, top-8 (tokens/s).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
+    python bench.py --ncu-case {decode-layer,gemm,moe}     (small launch sequences for ncu captures)
 
 Multi-GPU (torchrun): every rank runs an independent replica of the decode step (the step has no data
 exchange); value = bytes of all ranks / max-over-ranks time.
@@ -144,10 +145,18 @@ def load_peaks():
 
 
 def traffic_from_profiles(name):
-    """DRAM bytes per launch recorded from an ncu capture of the current kernel, or None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        return json.load(open(p)).get(name)
+    """DRAM bytes per launch from an ncu capture (profiles/traffic.txt: `name bytes sha256-of-source
+    source-path`), or None when there is none or the kernel source has changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        f = line.split()
+        if len(f) == 4 and f[0] == name:
+            src = os.path.join(ROOT, f[3])
+            if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == f[2]:
+                return int(float(f[1]))
     return None
 
 
@@ -215,8 +224,17 @@ def build_weights(q4, dev, symmetric_too: bool, seed=0):
 
 def run_decode(q4, args, ws, weights, dev):
     layers = decode_layers()
-    xs = [dev_bf16(synth.activations((0, "llama1b-decode-x", name), 1, k), dev) for (name, n, k) in layers]
-    ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for (_, n, k) in layers]
+    # every linear has its own x and y; they live in two contiguous buffers (one host copy each way per
+    # step for the end-to-end number), each slice 16-byte aligned
+    x_all = dev_bf16(np.concatenate([synth.activations((0, "llama1b-decode-x", name), 1, k).reshape(-1)
+                                     for (name, n, k) in layers]), dev)
+    y_all = torch.empty(sum(n for (_, n, _) in layers), dtype=torch.float32, device=dev)
+    xs, ys, ox, oy = [], [], 0, 0
+    for (_, n, k) in layers:
+        xs.append(x_all[ox:ox + k].view(1, k))
+        ys.append(y_all[oy:oy + n].view(1, n))
+        ox += k
+        oy += n
     bytes_step = decode_bytes(layers)
 
     # per layer: [q, k, v] grouped, o, [gate, up] grouped, down (the dependency structure of a layer)
@@ -252,18 +270,17 @@ def run_decode(q4, args, ws, weights, dev):
         gu.replay()
     ms_u = time_replays(gu, args.steps, ws) / args.steps
 
-    # end to end through the public call with host buffers: pinned x in, y back to the host, eager
-    hx = [x.cpu().pin_memory() for x in xs]
-    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
-    h2d = sum(t.numel() * t.element_size() for t in hx)
-    d2h = sum(t.numel() * t.element_size() for t in hy)
+    # end to end through the public calls with host buffers: the step's x (pinned host memory) copied
+    # in, the 64 calls issued eagerly, every y copied back to pinned host memory
+    hx = x_all.cpu().pin_memory()
+    hy = torch.empty(y_all.shape, dtype=y_all.dtype).pin_memory()
+    h2d = hx.numel() * hx.element_size()
+    d2h = hy.numel() * hy.element_size()
 
     def e2e_step():
-        for hxi, x in zip(hx, xs):
-            x.copy_(hxi, non_blocking=True)
+        x_all.copy_(hx, non_blocking=True)
         step()
-        for y, hyi in zip(ys, hy):
-            hyi.copy_(y, non_blocking=True)
+        hy.copy_(y_all, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         e2e_step()
@@ -302,7 +319,8 @@ def run_decode(q4, args, ws, weights, dev):
                                "bytes per launch / mean launch duration (graph replay, gaps included)",
                      "mean_launch_us": round(1e3 * ms_step / len(calls), 3)},
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "eager public-API calls per linear; pinned host x copied in and y copied out every step"},
+                "how": "eager public-API calls (64 per step); all x of the step copied in from pinned host memory "
+                       "and all y copied back to pinned host memory every step"},
         "gpu_launches": len(calls) * args.steps,
         "clocks": clk.summary(),
     }
@@ -472,6 +490,52 @@ def run_reference(args, ws, rank):
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def ncu_case(case):
+    """Small, fixed launch sequences for ncu captures (each runs twice and exits; nothing is timed)."""
+    from moe_linear_layers_b200 import q4
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if case == "decode-layer":
+        # six distinct layers (195 MB of weights > L2): [q,k,v] grouped, o, [gate,up] grouped, down
+        layers = decode_layers(6)
+        ws = []
+        for (name, n, k) in layers:
+            ws.append(q4.q4_quantize_pack(torch.from_numpy(synth.weights((0, "llama1b", name), n, k)).to(dev), 128, False))
+        xs = [dev_bf16(synth.activations((0, "llama1b-decode-x", name), 1, k), dev) for (name, n, k) in layers]
+        ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for (_, n, _) in layers]
+        torch.cuda.synchronize()
+        for _ in range(2):
+            for l in range(6):
+                b = 7 * l
+                q4.q4_linear_w4a16_grouped(xs[b:b + 3], ws[b:b + 3], ys[b:b + 3])
+                q4.q4_linear_w4a16(xs[b + 3], ws[b + 3], y=ys[b + 3])
+                q4.q4_linear_w4a16_grouped(xs[b + 4:b + 6], ws[b + 4:b + 6], ys[b + 4:b + 6])
+                q4.q4_linear_w4a16(xs[b + 6], ws[b + 6], y=ys[b + 6])
+    elif case == "gemm":
+        # W4A16 m=2048 gate-shaped (8192x2048), then act-quant + W4A8 m=4096 of the same shape
+        W = torch.from_numpy(synth.weights((0, "llama1b", "L0.gate"), 8192, 2048)).to(dev)
+        wa, ws_ = q4.q4_quantize_pack(W, 128, False), q4.q4_quantize_pack(W, 128, True)
+        x = dev_bf16(synth.activations((0, "llama1b-prefill-x", 2048), 2048, 2048, "outlier_channels"), dev)
+        x8 = dev_bf16(synth.activations((0, "llama1b-w4a8-x", 2048), 4096, 2048, "student_t3"), dev)
+        y = torch.empty((2048, 8192), dtype=torch.bfloat16, device=dev)
+        y8 = torch.empty((4096, 8192), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            q4.q4_linear_w4a16(x, wa, y=y)
+        for _ in range(2):
+            xq, sa = q4.act_quant_per_token(x8)
+            q4.q4_linear_w4a8(xq, sa, ws_, y=y8)
+    elif case == "moe":
+        T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+        x, Wr, bias, ex = build_moe(q4, dev)
+        ws_t = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk), dtype=torch.uint8, device=dev)
+        y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_t)
+    torch.cuda.synchronize()
+    print(f"ncu case {case}: done", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -480,7 +544,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=["decode-layer", "gemm", "moe"],
+                    help="run a small fixed launch sequence for an ncu capture and exit (no JSON line)")
     args = ap.parse_args()
+    if args.ncu_case:
+        ncu_case(args.ncu_case)
+        return
 
     if args.impl == "reference":
         line = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))

@@ -49,8 +49,8 @@ enum class Mode { Dense, GateUp, Down };
 constexpr int BM = 128;                  // weight rows per tile
 constexpr int BN = 128;                  // activation rows per tile
 constexpr int KBLK = 128;                // K per stage
-constexpr int NS = 4;                    // shared-memory stages (activations + packed weights)
 constexpr int NA = 4;                    // TMEM stages of widened weights
+constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
 constexpr int kThreads = 512;            // 16 warps: 4 per SM sub-partition, 128 registers each
 constexpr uint32_t kTmemCols = 512;
@@ -64,6 +64,10 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     static constexpr uint32_t A_COL0 = 2 * BN;                  // widened weights after the 2 D buffers
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
+    // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
+    // in flight to cover the latency of the activation copies
+    static constexpr int NS = INT8 ? 8 : (MODE == Mode::GateUp ? 4 : 5);
+    static_assert(NS <= kMaxStages, "ring depth");
     static_assert(NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144 <= 227 * 1024, "shared memory");
     static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144;
 };
@@ -157,7 +161,10 @@ __device__ __forceinline__ uint32_t pair16_bits(float v, bool f16)
 }
 
 struct Shared {
-    uint64_t xw_full[NS], xw_empty[NS], a_full[NA], a_empty[NA], d_full[2], d_empty[2], done;
+    // per stage: packed weights landed (converters wait), activations landed (MMA issuers wait), and
+    // the slot free again (MMA commit + the four converter warps)
+    uint64_t w_full[kMaxStages], x_full[kMaxStages], xw_empty[kMaxStages];
+    uint64_t a_full[NA], a_empty[NA], d_full[2], d_empty[2], done;
     uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
     uint32_t tmem_base;
     int abort_flag;
@@ -169,15 +176,39 @@ struct Shared {
 static_assert(sizeof(Shared) <= 6144, "Shared must fit the space reserved in Cfg::SMEM");
 
 
-constexpr int ZD = 4;   // depth of the converters' zero-point FIFO (K stages)
-constexpr int SD = 4;   // depth of the epilogue's scale FIFO (groups)
-
 // Pull a row of group parameters (n fp16 values) toward L2 ahead of use.
 __device__ __forceinline__ void prefetch_row_l2(const __half* row, int n)
 {
     for (int b = 0; b < n * 2; b += 128)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(row) + b));
 }
+
+// fp16 values of one row (scales or zeros, n of them) read 4 at a time, one 8-byte block ahead: the
+// block for positions [4j, 4j+4) is loaded when position 4j-4 is taken, so a register that is still
+// loading is touched (moved) only 4 positions later.  n % 4 != 0 falls back to direct loads.
+struct QuadRing {
+    const __half* row;
+    int n;
+    uint2 cur, nxt;
+    __device__ __forceinline__ void start(const __half* r, int count)
+    {
+        row = r;
+        n = count;
+        cur = nxt = make_uint2(0u, 0u);
+        if (row && (n & 3) == 0) nxt = __ldg(reinterpret_cast<const uint2*>(row));
+    }
+    __device__ __forceinline__ float get(int i)   // positions in increasing order, from 0
+    {
+        if (!row) return 0.0f;
+        if (n & 3) return __half2float(row[i]);
+        if ((i & 3) == 0) {
+            cur = nxt;
+            nxt = i + 4 < n ? __ldg(reinterpret_cast<const uint2*>(row + i + 4)) : make_uint2(0u, 0u);
+        }
+        const uint32_t w = (i & 2) ? cur.y : cur.x;
+        return __half2float(__ushort_as_half((unsigned short)((i & 1) ? (w >> 16) : (w & 0xFFFFu))));
+    }
+};
 
 template <Mode MODE>
 __device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
@@ -237,6 +268,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     constexpr int GPK = KBLK / G;               // groups per K stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    constexpr int NS = C::NS;
     uint8_t* xs = smem;                          // NS x XSTAGE (1024-aligned stages)
     uint8_t* wsm = smem + NS * C::XSTAGE;        // NS x WSTAGE
     float* xchg = reinterpret_cast<float*>(wsm + NS * WSTAGE);   // GateUp only
@@ -250,7 +282,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const int tiles_m = (p.M + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; i++) { tc::mbar_init(&sh->xw_full[i], 1); tc::mbar_init(&sh->xw_empty[i], 1 + 4); }
+        for (int i = 0; i < NS; i++) {
+            tc::mbar_init(&sh->w_full[i], 1);
+            tc::mbar_init(&sh->x_full[i], 1);
+            tc::mbar_init(&sh->xw_empty[i], 1 + 4);
+        }
         for (int i = 0; i < NA; i++) { tc::mbar_init(&sh->a_full[i], 4); tc::mbar_init(&sh->a_empty[i], 1); }
         for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->d_full[i], 1); tc::mbar_init(&sh->d_empty[i], 8); }
         tc::mbar_init(&sh->done, 2);
@@ -290,23 +326,27 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if ((it & 1u) != parity) continue;
                     const int s = it % NS;
                     if (!(ok = tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag))) break;
-                    tc::mbar_arrive_expect_tx(&sh->xw_full[s], C::XSTAGE + WSTAGE);
-                    uint8_t* xdst = xs + s * C::XSTAGE;
-                    tc::tma_load_2d(xdst, &tm_x, &sh->xw_full[s], kb * KBLK, T.m0);
-                    if constexpr (!INT8) tc::tma_load_2d(xdst + BN * 128, &tm_x, &sh->xw_full[s], kb * KBLK + 64, T.m0);
+                    // weights first (small; the converters start on them while the activations land)
+                    tc::mbar_arrive_expect_tx(&sh->w_full[s], WSTAGE);
                     uint8_t* wdst = wsm + s * WSTAGE;
                     if constexpr (MODE == Mode::GateUp) {
-                        tc::tma_load_2d(wdst, &tm_wa, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_a);
-                        tc::tma_load_2d(wdst + 64 * 64, &tm_wb, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_b);
+                        tc::tma_load_2d(wdst, &tm_wa, &sh->w_full[s], kb * (KBLK / 2), T.wrow_a);
+                        tc::tma_load_2d(wdst + 64 * 64, &tm_wb, &sh->w_full[s], kb * (KBLK / 2), T.wrow_b);
                     } else {
-                        tc::tma_load_2d(wdst, &tm_wa, &sh->xw_full[s], kb * (KBLK / 2), T.wrow_a);
+                        tc::tma_load_2d(wdst, &tm_wa, &sh->w_full[s], kb * (KBLK / 2), T.wrow_a);
                     }
+                    tc::mbar_arrive_expect_tx(&sh->x_full[s], C::XSTAGE);
+                    uint8_t* xdst = xs + s * C::XSTAGE;
+                    if constexpr (INT8) tc::tma_load_2d(xdst, &tm_x, &sh->x_full[s], kb * KBLK, T.m0);
+                    else tc::tma_load_3d(xdst, &tm_x, &sh->x_full[s], 0, T.m0, kb * 2);   // both 64-column halves
                 }
             }
             if (!ok || *abort_flag) {  // let every copy this thread issued land before the CTA can exit
                 for (uint32_t j = it > (uint32_t)NS ? it - NS : 0; j < it; j++)
-                    if ((j & 1u) == parity)
-                        tc::mbar_wait(&sh->xw_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
+                    if ((j & 1u) == parity) {
+                        tc::mbar_wait(&sh->w_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
+                        tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
+                    }
             }
         }
     } else if (warp <= 2) {
@@ -323,7 +363,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         continue;
                     }
                     const int s = it % NS, sa = it % NA;
-                    ok = tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag) &&
+                    ok = tc::mbar_wait(&sh->x_full[s], (it / NS) & 1, p.status, abort_flag) &&
                          tc::mbar_wait(&sh->a_full[sa], (it / NA) & 1, p.status, abort_flag);
                     if (!ok) break;
                     tc::fence_after_sync();
@@ -372,28 +412,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 row_params<MODE>(p, Tn, r, ngroups, sn, zn);
                 if (zn) prefetch_row_l2(zn, ngroups);
             }
-            // zero points travel through a register FIFO ZD stages deep (global loads, latency hidden)
-            float zq[ZD][GPK];
-#pragma unroll
-            for (int d = 0; d < ZD; d++)
-#pragma unroll
-                for (int gi = 0; gi < GPK; gi++)
-                    zq[d][gi] = SYM ? 8.0f : ((zrow && d < kblocks) ? __half2float(zrow[d * GPK + gi]) : 0.0f);
-            for (int kb = 0; kb < kblocks; kb++, it++) {
+            // zero points: read a few stages ahead through a QuadRing (no stall on the loads)
+            QuadRing zr;
+            zr.start(SYM ? nullptr : zrow, ngroups);
+            for (int kb = 0; kb < kblocks; kb++) {
                 const int s = it % NS, sa = it % NA;
                 float zcur[GPK];
 #pragma unroll
-                for (int gi = 0; gi < GPK; gi++) zcur[gi] = zq[0][gi];
-                if constexpr (!SYM) {
-#pragma unroll
-                    for (int d = 0; d + 1 < ZD; d++)
-#pragma unroll
-                        for (int gi = 0; gi < GPK; gi++) zq[d][gi] = zq[d + 1][gi];
-#pragma unroll
-                    for (int gi = 0; gi < GPK; gi++)
-                        zq[ZD - 1][gi] = (zrow && kb + ZD < kblocks) ? __half2float(zrow[(kb + ZD) * GPK + gi]) : 0.0f;
-                }
-                if (!tc::mbar_wait(&sh->xw_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
+                for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : zr.get(kb * GPK + gi);
+                if (!tc::mbar_wait(&sh->w_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
                 uint4 v[4];
                 const uint32_t wrow = tc::smem_u32(wsm + s * WSTAGE) + r * 64;
 #pragma unroll
@@ -433,6 +460,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sh->a_full[sa]);
+                it++;
             }
         }
     conv_done:;
@@ -480,16 +508,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     comb_w[ew * 64 + j] = ok ? p.row_w[m] : 0.0f;
                 }
             }
-            // group scales travel through a register FIFO SD groups deep
-            float sq[SD];
-#pragma unroll
-            for (int d = 0; d < SD; d++) sq[d] = (srow && d < ngroups) ? __half2float(srow[d]) : 0.0f;
-            for (int gl = 0; gl < ngroups; gl++, g++) {
+            // group scales through a QuadRing (read ahead, no stall on the loads)
+            QuadRing sr;
+            sr.start(srow, ngroups);
+            for (int gl = 0; gl < ngroups; gl++) {
                 const uint32_t db = g & 1;
-                float s = sq[0];
-#pragma unroll
-                for (int d = 0; d + 1 < SD; d++) sq[d] = sq[d + 1];
-                sq[SD - 1] = (srow && gl + SD < ngroups) ? __half2float(srow[gl + SD]) : 0.0f;
+                float s = sr.get(gl);
                 if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
                 const uint64_t s2 = tc::f2_pack(__float_as_uint(s), __float_as_uint(s));
                 if (!tc::mbar_wait(&sh->d_full[db], (g >> 1) & 1, p.status, abort_flag)) goto epi_done;
@@ -528,6 +552,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sh->d_empty[db]);
+                g++;
             }
             // ---------------------------------------------------------- tile output
             // (every loop below has a branch-free path for a full 64-row block: a conditional branch per
