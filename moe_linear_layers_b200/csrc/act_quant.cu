@@ -4,55 +4,106 @@
 // round half to even, clamp to [-128, 127].  The division by the scale is IEEE fp32; a token whose
 // amax is 0 gets scale 0 and all-zero codes.
 //
-// HBM-bound (2 B read + 1 B written per element): one CTA per token, 16-byte loads, a block-wide
-// max, then a second pass over the (cache-resident) row that writes 8 codes per 8-byte store.
+// HBM-bound (2 B read + 1 B written per element): one CTA per token, the row held in registers between
+// the max pass and the coding pass (one read of x), 16-byte loads and 8-byte stores.  The quotient
+// x / s is formed without a division per element: with r = RN(1/s), t = RN(x*r), e = x - s*t exact by
+// FMA, q = RN(t + e*r) is the correctly rounded quotient RN(x/s) (Markstein's theorem for round to
+// nearest; every residual that can decide a rounding stays a normal float when s >= 2^-100), so the codes
+// equal those of an IEEE division bit for bit.  Rows with a smaller scale take the division itself.
 #include "q4_common.cuh"
 
 namespace {
 
-__global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restrict__ x, int k,
-                                                        int8_t* __restrict__ xq, float* __restrict__ scale_a,
-                                                        int32_t* status)
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int code8(float x, float s, float r, bool exact_div)
 {
-    __shared__ float red[8];
+    float q;
+    if (exact_div) {
+        q = x / s;
+    } else {
+        const float t = x * r;
+        const float e = fmaf(-s, t, x);
+        q = fmaf(e, r, t);
+    }
+    return (int)fminf(fmaxf(rintf(q), -128.0f), 127.0f);
+}
+
+// codes of one 16-byte word (8 bf16 values) as 8 bytes
+__device__ __forceinline__ uint2 code_word(const uint4& v, float s, float r, bool exact_div)
+{
+    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const int qa = code8(__uint_as_float(e[j] << 16), s, r, exact_div);
+        const int qb = code8(__uint_as_float(e[j] & 0xFFFF0000u), s, r, exact_div);
+        packed[j / 2] |= ((uint32_t)(qa & 0xFF) | ((uint32_t)(qb & 0xFF) << 8)) << (16 * (j & 1));
+    }
+    return make_uint2(packed[0], packed[1]);
+}
+
+// per-halfword max of bf16 magnitudes (integer order = magnitude order for non-NaN) and a flag for an
+// all-ones exponent (inf or NaN) anywhere in the word
+__device__ __forceinline__ uint32_t word_amax(const uint4& v, uint32_t& bad)
+{
+    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t a = 0;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        a = __vmaxu2(a, e[j] & 0x7FFF7FFFu);
+        bad |= ((e[j] & 0x7F807F80u) + 0x00800080u) & 0x80008000u;
+    }
+    return a;
+}
+
+// W = 16-byte words per thread kept in registers (k <= 8 * kThreads * W); W = 0: any k, two passes.
+template <int W>
+__global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __restrict__ x, int k,
+                                                             int8_t* __restrict__ xq, float* __restrict__ scale_a,
+                                                             int32_t* status)
+{
+    __shared__ uint32_t red[kThreads / 32];
     const int64_t row = blockIdx.x;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * k);
+    uint2* out = reinterpret_cast<uint2*>(xq + row * k);
     const int n8 = k / 8;
-    float amax = 0.0f;
-    bool finite = true;
-    for (int i = threadIdx.x; i < n8; i += blockDim.x) {
-        const uint4 v = __ldg(xr + i);
-        const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t a = 0, bad = 0;
+    uint4 v[W > 0 ? W : 1];
+    if constexpr (W > 0) {
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float a = __uint_as_float(e[j] << 16), b = __uint_as_float(e[j] & 0xFFFF0000u);
-            finite &= isfinite(a) && isfinite(b);
-            amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+        for (int i = 0; i < W; i++) {
+            const int w = i * kThreads + threadIdx.x;
+            v[i] = w < n8 ? __ldg(xr + w) : make_uint4(0u, 0u, 0u, 0u);
         }
+#pragma unroll
+        for (int i = 0; i < W; i++) a = __vmaxu2(a, word_amax(v[i], bad));
+    } else {
+        for (int w = threadIdx.x; w < n8; w += kThreads) a = __vmaxu2(a, word_amax(__ldg(xr + w), bad));
     }
-    if (!finite) q4_set_status(status, Q4_ERR_NONFINITE);
+    if (bad) q4_set_status(status, Q4_ERR_NONFINITE);
+    a = max(a & 0xFFFFu, a >> 16);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = amax;
+    for (int off = 16; off >= 1; off >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = a;
     __syncthreads();
-    float m = 0.0f;
+    uint32_t mb = 0;
 #pragma unroll
-    for (int i = 0; i < 8; i++) m = fmaxf(m, red[i]);
+    for (int i = 0; i < kThreads / 32; i++) mb = max(mb, red[i]);
+    const float m = __uint_as_float(mb << 16);
     const float s = m / 127.0f;
     if (threadIdx.x == 0) scale_a[row] = s;
-    uint2* out = reinterpret_cast<uint2*>(xq + row * k);
-    for (int i = threadIdx.x; i < n8; i += blockDim.x) {
-        const uint4 v = __ldg(xr + i);
-        const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-        uint32_t packed[2] = {0u, 0u};
+    const bool exact_div = !(s >= 0x1p-100f);           // tiny (or zero / NaN) scale: divide directly
+    const float r = exact_div ? 0.0f : 1.0f / s;
+    if constexpr (W > 0) {
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float a = __uint_as_float(e[j] << 16), b = __uint_as_float(e[j] & 0xFFFF0000u);
-            const int qa = s == 0.0f ? 0 : (int)fminf(fmaxf(rintf(a / s), -128.0f), 127.0f);
-            const int qb = s == 0.0f ? 0 : (int)fminf(fmaxf(rintf(b / s), -128.0f), 127.0f);
-            packed[j / 2] |= ((uint32_t)(qa & 0xFF) | ((uint32_t)(qb & 0xFF) << 8)) << (16 * (j & 1));
+        for (int i = 0; i < W; i++) {
+            const int w = i * kThreads + threadIdx.x;
+            if (w < n8) out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word(v[i], s, r, exact_div);
         }
-        out[i] = make_uint2(packed[0], packed[1]);
+    } else {
+        for (int w = threadIdx.x; w < n8; w += kThreads)
+            out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word(__ldg(xr + w), s, r, exact_div);
     }
 }
 
@@ -65,6 +116,12 @@ extern "C" int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8
     if (m < 0 || k <= 0 || k % 8) return Q4_ERR_SHAPE;
     if (!q4_aligned16(x) || !q4_aligned16(xq) || ((uintptr_t)scale_a & 3u)) return Q4_ERR_ALIGN;
     if (m == 0) return Q4_OK;
-    act_quant_kernel<<<m, 256, 0, (cudaStream_t)stream>>>(x, k, xq, scale_a, dev_status);
+    const int n8 = k / 8;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n8 <= kThreads) act_quant_kernel<1><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 2 * kThreads) act_quant_kernel<2><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 4 * kThreads) act_quant_kernel<4><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 8 * kThreads) act_quant_kernel<8><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else act_quant_kernel<0><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
     return q4_launch_status();
 }

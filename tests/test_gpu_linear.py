@@ -165,6 +165,36 @@ def test_act_quant_bitexact(q4, m, k):
     assert np.array_equal(xq.cpu().numpy(), q_ref)
 
 
+def test_act_quant_rounding_stress(q4):
+    """Quotients at and next to half-integers, scales with full mantissas, and extreme magnitudes (tiny
+    rows take the kernel's division path, the rest the reciprocal-and-FMA path): codes and scales
+    bit-exact against the oracle's IEEE division."""
+    rng = np.random.default_rng(7)
+    k = 2048
+    rows = []
+    # the quotient grid itself: amax 127 gives s = 1, values on and between half-integers
+    g = np.arange(-127.0, 127.5, 0.5, dtype=np.float32)
+    rows.append(np.resize(g, k))
+    # random magnitudes spanning the bf16 exponent range, with the amax chosen to give awkward scales
+    for e in (-130, -110, -100, -99, -96, -95, -60, -20, -3, 0, 5, 30, 90, 120):
+        r = rng.standard_normal(k).astype(np.float32) * np.float32(2.0 ** e)
+        r[rng.integers(k)] = np.float32(1.37 * 2.0 ** (e + 2))
+        rows.append(r)
+    # values placed right at q + 0.5 of a non-power-of-two scale, and one bf16 ulp to either side
+    s = np.float32(100.0) / np.float32(127.0)
+    base = (np.arange(k) % 255 - 127).astype(np.float32)
+    for d in (0.5, 0.49, 0.51):
+        r = ((base + np.float32(d)) * s).astype(np.float32)
+        r[0] = np.float32(100.0)
+        rows.append(r)
+    x = synth.to_bf16_bits(np.stack(rows).astype(np.float32))
+    q_ref, s_ref = oracle.act_quant(x, k)
+    xq, sc = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
+    torch.cuda.synchronize()
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+
+
 def test_act_quant_golden_rows(q4):
     x = synth.to_bf16_bits(np.array([[127, -63.5, 0.5, 2, 0, 0, 0, 0], [-127, 2.5, -2.5, 1.5, 0, 0, 0, 0]], np.float32))
     xq, s = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
