@@ -16,7 +16,8 @@
 // Data flow: TMA brings the packed nibbles (64-byte swizzle) and the activation tile (128-byte
 // swizzle, K-major, the MMA's B operand) into a 4-stage shared-memory ring.  Converter warps widen the
 // nibbles in registers and write them into TMEM with tcgen05.st (the MMA's A operand), so widened
-// weights never use shared-memory bandwidth.  One thread issues tcgen05.mma and commits to mbarriers.
+// weights never use shared-memory bandwidth.  Four threads in four warps issue tcgen05.mma for
+// alternate K stages and commit to mbarriers.
 //
 // Modes:
 //   Dense   y[m][n] = sum_g s[n][g] * D_g (W4A16, bf16 MMA) or y = s_a[m] * sum_g s[n][g] * D_g / 16
@@ -26,14 +27,18 @@
 //   Down    A = 128 rows of the expert's down projection (fp16 codes), B = h (fp16); epilogue
 //           y[token][n] += w[token][slot] * out (fp32 reduction into the output).
 //
-// Warp roles (512 threads, 16 warps = 4 per SM sub-partition at 128 registers): warps 0 and 15 TMA
-// producers (alternate stages), warps 1-2 MMA issuers (warp 1 also owns TMEM), warps 3-6 converters
-// (TMEM lanes 32*(warp%4) ...), warps 7-14 epilogue (two warps per TMEM lane quarter, each draining 64
-// of the 128 columns).  A thread that waits on an mbarrier stalls until the asynchronous operations it
-// issued (bulk copies, MMAs) have completed, so every asynchronous stream is split over two threads in
-// different warps that take alternate stages: one keeps the TMA engine (or the tensor pipe) busy while
-// the other waits.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their phases
-// across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
+// Warp roles (640 threads = 5 warpgroups, launched at 96 registers and re-partitioned with setmaxnreg):
+//   warps 0-3    MMA issuers, one thread each, stage it issued by warp it % 4 (warp 1 also owns TMEM);
+//   warps 4-7    converters (TMEM lanes 32*(warp%4) ...);
+//   warps 8-9    TMA producers (alternate stages); warps 10-11 idle;
+//   warps 12-19  epilogue (two warps per TMEM lane quarter, each draining 64 of the 128 columns).
+// Measured on B200: one thread issues an M128 N128 K16 MMA only every ~120 cycles, half the tensor
+// pipe's rate, and any strong memory operation in that thread (an mbarrier wait included) stalls it
+// until its MMAs have retired; four issuer threads in different warps that only poll progress counters
+// with weak loads keep the pipe at one MMA per 64 cycles, commits included.  A thread that waits on an
+// mbarrier also stalls until its own bulk copies have landed, so the TMA stream is split over two
+// producer threads too.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their
+// phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
 //
 // Epilogue arithmetic runs on packed fp32 pairs (FFMA2).  For W4A8 every int32 accumulator is preloaded
 // with the bit pattern of 1.5 * 2^23, so the accumulated bits are the float 1.5 * 2^23 + acc and one
@@ -52,7 +57,15 @@ constexpr int KBLK = 128;                // K per stage
 constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
-constexpr int kThreads = 512;            // 16 warps: 4 per SM sub-partition, 128 registers each
+constexpr int kThreads = 640;            // 20 warps = 5 warpgroups
+constexpr int kIssuers = 4;              // MMA issuer threads (warps 0-3)
+// registers per thread: the launch allocation (65536 / 640, rounded down to a multiple of 8) and the
+// per-warpgroup split after setmaxnreg; the split may not exceed the launch allocation
+constexpr int kLaunchRegs = 96;
+constexpr int kRegsLight = 48;           // issuers, producers
+constexpr int kRegsConv = 88;            // converters
+constexpr int kRegsEpi = 144;            // epilogue (two warpgroups)
+static_assert(128 * kRegsLight * 2 + 128 * kRegsConv + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
 constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
@@ -161,10 +174,13 @@ __device__ __forceinline__ uint32_t pair16_bits(float v, bool f16)
 }
 
 struct Shared {
-    // per stage: packed weights landed (converters wait), activations landed (MMA issuers wait), and
-    // the slot free again (MMA commit + the four converter warps)
+    // per stage: packed weights landed, activations landed (converters wait on both), and the slot
+    // free again (MMA commit + the four converter warps; it also frees the stage's TMEM A slot)
     uint64_t w_full[kMaxStages], x_full[kMaxStages], xw_empty[kMaxStages];
-    uint64_t a_full[NA], a_empty[NA], d_full[2], d_empty[2], done;
+    uint64_t d_full[2], done;
+    // progress counters read by the MMA issuer (weak loads): stages converted (and activations landed)
+    // per converter warp, groups drained per epilogue warp, W4A8 accumulator preload done per epilogue warp
+    uint32_t conv_done[4], epi_done[8], epi_init[8];
     uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
     uint32_t tmem_base;
     int abort_flag;
@@ -287,9 +303,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->x_full[i], 1);
             tc::mbar_init(&sh->xw_empty[i], 1 + 4);
         }
-        for (int i = 0; i < NA; i++) { tc::mbar_init(&sh->a_full[i], 4); tc::mbar_init(&sh->a_empty[i], 1); }
-        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->d_full[i], 1); tc::mbar_init(&sh->d_empty[i], 8); }
-        tc::mbar_init(&sh->done, 2);
+        for (int i = 0; i < 2; i++) tc::mbar_init(&sh->d_full[i], 1);
+        for (int i = 0; i < 4; i++) sh->conv_done[i] = 0;
+        for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
+        tc::mbar_init(&sh->done, kIssuers);
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
@@ -311,13 +328,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const uint32_t tbase = sh->tmem_base;
     const int total = sh->total_tiles;
 
-    if (warp == 0 || warp == kThreads / 32 - 1) {
-        // ------------------------------------------------------------------ TMA producers
+    const int wg = warp / 4;
+    if (wg == 2) {
+        tc::setmaxnreg_dec<kRegsLight>();
+        // ------------------------------------------------------------------ TMA producers (warps 8, 9)
         // Two producer threads in different warps take alternate stages: a thread that waits on an
         // mbarrier stalls until its own outstanding bulk copies have landed, so one thread alone would
         // issue only one stage per L2 round trip.
-        if (lane == 0) {
-            const uint32_t parity = warp == 0 ? 0u : 1u;
+        if (lane == 0 && warp < 10) {
+            const uint32_t parity = warp - 8;
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
@@ -349,31 +368,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
             }
         }
-    } else if (warp <= 2) {
-        // ------------------------------------------------------------------ MMA issuers (alternate K stages)
+    } else if (wg == 0) {
+        tc::setmaxnreg_dec<kRegsLight>();
+        // ------------------------------------------------------------------ MMA issuers (warps 0-3)
+        // They wait only by polling progress counters with weak loads (tc::poll_counters), so the tensor
+        // pipe never drains between stages; their completions go out through tcgen05.commit, which tracks
+        // the issuing thread's own MMAs: every stage is issued and committed by one thread.
         if (lane == 0) {
             constexpr uint32_t idesc = INT8 ? tc::idesc_s8_s32(BN) : (F16 ? tc::idesc_f16_f32(BN) : tc::idesc_bf16_f32(BN));
-            const uint32_t parity = warp - 1;
             uint32_t it = 0, g = 0;
             bool ok = true;
+            if constexpr (INT8) ok = tc::poll_counters<8>(sh->epi_init, 1, p.status, abort_flag);
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 for (int kb = 0; kb < kblocks && ok; kb++, it++) {
-                    if ((it & 1) != parity) {   // the other issuer's stage
+                    if (it % kIssuers != (uint32_t)warp) {   // another issuer's stage
                         g += GPK;
                         continue;
                     }
                     const int s = it % NS, sa = it % NA;
-                    ok = tc::mbar_wait(&sh->x_full[s], (it / NS) & 1, p.status, abort_flag) &&
-                         tc::mbar_wait(&sh->a_full[sa], (it / NA) & 1, p.status, abort_flag);
-                    if (!ok) break;
+                    // the stage's weights are widened into TMEM and its activations have landed
+                    if (!(ok = tc::poll_counters<4>(sh->conv_done, it + 1, p.status, abort_flag))) break;
                     tc::fence_after_sync();
                     const uint32_t xaddr = tc::smem_u32(xs + s * C::XSTAGE);
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++, g++) {
                         const uint32_t db = g & 1;
-                        // INT8: the epilogue pre-loads the accumulator (see below) and releases it once first
-                        const uint32_t dpar = INT8 ? ((g >> 1) & 1) : (((g >> 1) & 1) ^ 1);
-                        if (!(ok = tc::mbar_wait(&sh->d_empty[db], dpar, p.status, abort_flag))) break;
+                        // accumulator db is free once group g-2 has been drained
+                        if (!(ok = tc::poll_counters<8>(sh->epi_done, g >= 2 ? g - 1 : 0, p.status, abort_flag))) break;
                         tc::fence_after_sync();
 #pragma unroll
                         for (int i = 0; i < G / C::KI; i++) {
@@ -389,14 +410,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tc::mma_commit(&sh->d_full[db]);
                     }
                     tc::mma_commit(&sh->xw_empty[s]);
-                    tc::mma_commit(&sh->a_empty[sa]);
                 }
             }
-            tc::mma_commit(&sh->done);   // every MMA issued so far has completed once `done` flips
+            tc::mma_commit(&sh->done);   // every MMA of this thread has completed once `done` flips
             tc::mbar_wait(&sh->done, 0, p.status, abort_flag, 100000000ull);
         }
-    } else if (warp < 7) {
-        // ------------------------------------------------------------------ converters
+    } else if (wg == 1) {
+        tc::setmaxnreg_dec<kRegsConv>();
+        // ------------------------------------------------------------------ converters (warps 4-7)
         const int sub = warp & 3;
         const int r = 32 * sub + lane;                 // row in tile == TMEM lane
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
@@ -427,7 +448,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 for (int c = 0; c < 4; c++) v[c] = lds128(wrow + ((c ^ ((r >> 1) & 3)) << 4));
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sh->xw_empty[s]);
-                if (!tc::mbar_wait(&sh->a_empty[sa], ((it / NA) & 1) ^ 1, p.status, abort_flag)) goto conv_done;
+                // TMEM slot sa is free once the MMAs of stage it - NA have completed: that stage's slot of the
+                // ring has been released (its phase cannot be older: this warp has converted stage it - NA,
+                // so the producer refilled it; nor newer: that needs this warp's arrival for it - NA + NS)
+                if (it >= (uint32_t)NA) {
+                    const uint32_t j = it - NA;
+                    if (!tc::mbar_wait(&sh->xw_empty[j % NS], (j / NS) & 1, p.status, abort_flag)) goto conv_done;
+                }
                 __syncwarp();
                 tc::fence_after_sync();
                 const uint32_t words[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
@@ -458,15 +485,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
+                // publish: this warp's rows of the stage are in TMEM, and the stage's activations landed
+                if (!tc::mbar_wait(&sh->x_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sh->a_full[sa]);
+                if (lane == 0) tc::sts_release(&sh->conv_done[sub], it + 1);
                 it++;
             }
         }
     conv_done:;
     } else {
-        // ------------------------------------------------------------------ epilogue
-        const int ew = warp - 7;
+        tc::setmaxnreg_inc<kRegsEpi>();
+        // ------------------------------------------------------------------ epilogue (warps 12-19)
+        const int ew = warp - 12;
         const int sub = warp & 3, half = ew >> 2;
         const int r = 32 * sub + lane;
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
@@ -485,7 +515,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) { tc::mbar_arrive(&sh->d_empty[0]); tc::mbar_arrive(&sh->d_empty[1]); }
+            if (lane == 0) tc::sts_release(&sh->epi_init[ew], 1);
         }
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
@@ -551,7 +581,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sh->d_empty[db]);
+                if (lane == 0) tc::sts_release(&sh->epi_done[ew], g + 1);   // group g drained
                 g++;
             }
             // ---------------------------------------------------------- tile output

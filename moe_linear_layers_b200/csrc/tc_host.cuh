@@ -69,6 +69,14 @@ int launch(const CUtensorMap& mx, const CUtensorMap& ma, const CUtensorMap& mb, 
     auto kern = tc_gemm_kernel<INT8, G, SYM, MODE>;
     constexpr int smem = Cfg<INT8, MODE>::SMEM;
     if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return q4_cuda_status(e);
+    // The kernel re-partitions its registers between warpgroups (setmaxnreg) assuming a launch
+    // allocation of kLaunchRegs per thread; a build that allocated fewer would make the increase wait
+    // forever, so it is refused.
+    static const int nregs = [&] {
+        cudaFuncAttributes fa{};
+        return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (nregs != kLaunchRegs) return Q4_ERR_UNSUPPORTED;
     kern<<<grid, kThreads, smem, s>>>(mx, ma, mb, p);
     return q4_launch_status();
 }

@@ -63,8 +63,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 
 // Wait for the phase with the given parity to complete.  Gives up after `limit_ns` of wall time:
 // records Q4_ERR_TIMEOUT in the status word, raises the CTA's abort flag (nullable) and returns false.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int32_t* status,
-                                            volatile int* abort_flag, uint64_t limit_ns)
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int32_t* status,
+                                               volatile int* abort_flag, uint64_t limit_ns)
 {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0;; i++) {
@@ -197,6 +197,80 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
           "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------- //
+// progress counters for a thread that issues tcgen05.mma
+//
+// Any strong memory operation in an MMA-issuing thread -- an mbarrier wait, even on a completed phase,
+// or a relaxed / acquire / volatile load -- stalls that thread until the MMAs it issued have retired,
+// which leaves the tensor pipe idle (measured: 64 cycles per M128 N128 K16 MMA without, ~155 with one
+// such wait per 8 MMAs).  Weak loads do not.  So the issuer polls monotonic counters with weak loads;
+// the threads that publish them (converters, epilogue) do the mbarrier waits and TMEM waits first and
+// store the counter with release semantics.
+// ---------------------------------------------------------------------------------------------- //
+
+// Register re-partition between warpgroups (every warp of a warpgroup executes the same one).  An
+// increase waits until other warpgroups have released enough registers of the CTA's launch allocation.
+template <uint32_t N> __device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N> __device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+#ifndef Q4_POLL_SLEEP_NS
+#define Q4_POLL_SLEEP_NS 0
+#endif
+
+__device__ __forceinline__ uint32_t lds_weak(const void* p)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void sts_release(void* p, uint32_t v)
+{
+    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Spin until each of the n counters at c is >= target.  The fast path makes weak loads only; after a
+// few thousand unsuccessful rounds it also watches the wall clock (2 s: Q4_ERR_TIMEOUT, raise the abort
+// flag, return false) and the abort flag.
+__device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uint32_t target, int32_t* status,
+                                                   volatile int* abort_flag)
+{
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        bool ok = true;
+        for (int i = 0; i < n; i++) ok &= lds_weak(c + i) >= target;
+        if (ok) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer_ns() - t0 > 2000000000ull) {
+            q4_set_status(status, Q4_ERR_TIMEOUT);
+            if (abort_flag) *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <int N>
+__device__ __forceinline__ bool poll_counters(const uint32_t* c, uint32_t target, int32_t* status,
+                                              volatile int* abort_flag)
+{
+    for (int round = 0; round < 4096; round++) {
+        bool ok = true;
+#pragma unroll
+        for (int i = 0; i < N; i++) ok &= lds_weak(c + i) >= target;
+        if (ok) return true;
+#if Q4_POLL_SLEEP_NS > 0
+        __nanosleep(Q4_POLL_SLEEP_NS);
+#endif
+    }
+    return poll_counters_slow(c, N, target, status, abort_flag);
 }
 
 // ---------------------------------------------------------------------------------------------- //
