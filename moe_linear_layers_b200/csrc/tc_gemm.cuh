@@ -10,8 +10,8 @@
 // Every mode computes, for a tile of 128 weight rows (the MMA's M, one TMEM lane each) and 128
 // activation rows (the MMA's N), D_g = sum_{k in g} (code - zero)[row][k] * act[m][k] exactly (integer
 // codes are exact in bf16 / fp16 / int8) one quantization group at a time, and the epilogue
-// accumulates s[row][g] * D_g in fp32.  Group accumulators are double-buffered in TMEM so the MMA of
-// group g+1 overlaps the epilogue's drain of group g.
+// accumulates s[row][g] * D_g in fp32.  Group accumulators rotate through two TMEM buffers (three for
+// W4A8) so the MMAs of the next groups overlap the epilogue's drain of group g.
 //
 // Data flow: TMA brings the packed nibbles (64-byte swizzle) and the activation tile (128-byte
 // swizzle, K-major, the MMA's B operand) into a 4-stage shared-memory ring.  Converter warps widen the
@@ -62,12 +62,14 @@ constexpr int kIssuers = 4;              // MMA issuer threads (warps 0-3)
 // registers per thread: the launch allocation (65536 / 640, rounded down to a multiple of 8) and the
 // per-warpgroup split after setmaxnreg; the split may not exceed the launch allocation
 constexpr int kLaunchRegs = 96;
-constexpr int kRegsLight = 48;           // issuers, producers
+constexpr int kRegsIssue = 48;           // MMA issuers
+constexpr int kRegsProd = 56;            // TMA producers, parameter loader
 constexpr int kRegsConv = 88;            // converters
 constexpr int kRegsEpi = 144;            // epilogue (two warpgroups)
-static_assert(128 * kRegsLight * 2 + 128 * kRegsConv + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
+static_assert(128 * (kRegsIssue + kRegsProd + kRegsConv) + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
+constexpr int PW = 16;                   // quantization groups per window of the parameter ring
 constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
 constexpr float kAccBiasF = 12582912.0f;
 
@@ -75,14 +77,23 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2);   // activation bytes per stage
     static constexpr int ACOLS = KBLK / (INT8 ? 4 : 2);         // TMEM columns of one widened stage
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
-    static constexpr uint32_t A_COL0 = 2 * BN;                  // widened weights after the 2 D buffers
+    // group accumulators in TMEM: three for W4A8 (its MMAs are twice as fast, so the epilogue needs more
+    // slack), two otherwise; the widened weights follow them (NA * ACOLS columns)
+    static constexpr int ND = INT8 ? 3 : 2;
+    static constexpr uint32_t A_COL0 = ND * BN;
+    static_assert(ND * BN + NA * ACOLS <= (int)kTmemCols, "TMEM columns");
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
+    // group parameters staged in shared memory: 2 slots, each PW groups x 128 rows of fp16 scales
+    // (and, for 16-bit modes, zero points), group-major so a warp reads 32 consecutive rows
+    static constexpr int PTENS = INT8 ? 1 : 2;                  // scales (+ zero points)
+    static constexpr int PSLOT = PW * BM * 2;                   // bytes of one tensor in one slot
+    static constexpr int PARAMS = 2 * PSLOT * PTENS;
     // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
     // in flight to cover the latency of the activation copies
     static constexpr int NS = INT8 ? 8 : (MODE == Mode::GateUp ? 4 : 5);
     static_assert(NS <= kMaxStages, "ring depth");
-    static_assert(NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144 <= 227 * 1024, "shared memory");
-    static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + 1024 + 6144;
+    static_assert(NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144 <= 227 * 1024, "shared memory");
+    static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144;
 };
 
 struct Args {
@@ -177,11 +188,12 @@ struct Shared {
     // per stage: packed weights landed, activations landed (converters wait on both), and the slot
     // free again (MMA commit + the four converter warps; it also frees the stage's TMEM A slot)
     uint64_t w_full[kMaxStages], x_full[kMaxStages], xw_empty[kMaxStages];
-    uint64_t d_full[2], done;
+    uint64_t d_full[3], done;
     // progress counters read by the MMA issuer (weak loads): stages converted (and activations landed)
     // per converter warp, groups drained per epilogue warp, W4A8 accumulator preload done per epilogue warp
     uint32_t conv_done[4], epi_done[8], epi_init[8];
     uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
+    uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
     int abort_flag;
     int total_tiles;
@@ -191,40 +203,6 @@ struct Shared {
 };
 static_assert(sizeof(Shared) <= 6144, "Shared must fit the space reserved in Cfg::SMEM");
 
-
-// Pull a row of group parameters (n fp16 values) toward L2 ahead of use.
-__device__ __forceinline__ void prefetch_row_l2(const __half* row, int n)
-{
-    for (int b = 0; b < n * 2; b += 128)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(row) + b));
-}
-
-// fp16 values of one row (scales or zeros, n of them) read 4 at a time, one 8-byte block ahead: the
-// block for positions [4j, 4j+4) is loaded when position 4j-4 is taken, so a register that is still
-// loading is touched (moved) only 4 positions later.  n % 4 != 0 falls back to direct loads.
-struct QuadRing {
-    const __half* row;
-    int n;
-    uint2 cur, nxt;
-    __device__ __forceinline__ void start(const __half* r, int count)
-    {
-        row = r;
-        n = count;
-        cur = nxt = make_uint2(0u, 0u);
-        if (row && (n & 3) == 0) nxt = __ldg(reinterpret_cast<const uint2*>(row));
-    }
-    __device__ __forceinline__ float get(int i)   // positions in increasing order, from 0
-    {
-        if (!row) return 0.0f;
-        if (n & 3) return __half2float(row[i]);
-        if ((i & 3) == 0) {
-            cur = nxt;
-            nxt = i + 4 < n ? __ldg(reinterpret_cast<const uint2*>(row + i + 4)) : make_uint2(0u, 0u);
-        }
-        const uint32_t w = (i & 2) ? cur.y : cur.x;
-        return __half2float(__ushort_as_half((unsigned short)((i & 1) ? (w >> 16) : (w & 0xFFFFu))));
-    }
-};
 
 template <Mode MODE>
 __device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
@@ -274,6 +252,28 @@ __device__ __forceinline__ void row_params(const Args& p, const Tile& T, int r, 
     }
 }
 
+// PW consecutive fp16 group parameters of one row, from group g0 (zeros past the row's end or for a
+// missing row), stored group-major at dst[j * BM].
+__device__ __forceinline__ void stage_params(const __half* row, int g0, int ng, __half* dst)
+{
+    uint16_t* d = reinterpret_cast<uint16_t*>(dst);
+    if (row && (ng & 7) == 0 && ((uintptr_t)row & 15) == 0) {
+#pragma unroll
+        for (int q = 0; q < PW / 8; q++) {
+            const uint4 u = g0 + 8 * q < ng ? __ldg(reinterpret_cast<const uint4*>(row + g0 + 8 * q)) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                d[(8 * q + 2 * j) * BM] = (uint16_t)(e[j] & 0xFFFFu);
+                d[(8 * q + 2 * j + 1) * BM] = (uint16_t)(e[j] >> 16);
+            }
+        }
+    } else {
+#pragma unroll 4
+        for (int j = 0; j < PW; j++) d[j * BM] = (row && g0 + j < ng) ? __half_as_ushort(row[g0 + j]) : (uint16_t)0;
+    }
+}
+
 template <bool INT8, int G, bool SYM, Mode MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
@@ -288,7 +288,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     uint8_t* xs = smem;                          // NS x XSTAGE (1024-aligned stages)
     uint8_t* wsm = smem + NS * C::XSTAGE;        // NS x WSTAGE
     float* xchg = reinterpret_cast<float*>(wsm + NS * WSTAGE);   // GateUp only
-    Shared* sh = reinterpret_cast<Shared*>(wsm + NS * WSTAGE + C::XCHG);
+    __half* params = reinterpret_cast<__half*>(wsm + NS * WSTAGE + C::XCHG);   // [slot][scale|zero][PW][BM]
+    Shared* sh = reinterpret_cast<Shared*>(wsm + NS * WSTAGE + C::XCHG + C::PARAMS);
     volatile int* abort_flag = &sh->abort_flag;
     int* comb_tok = sh->comb_tok;
     float* comb_w = sh->comb_w;
@@ -303,10 +304,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->x_full[i], 1);
             tc::mbar_init(&sh->xw_empty[i], 1 + 4);
         }
-        for (int i = 0; i < 2; i++) tc::mbar_init(&sh->d_full[i], 1);
+        for (int i = 0; i < C::ND; i++) tc::mbar_init(&sh->d_full[i], 1);
         for (int i = 0; i < 4; i++) sh->conv_done[i] = 0;
         for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
         tc::mbar_init(&sh->done, kIssuers);
+        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->p_full[i], 32); tc::mbar_init(&sh->p_empty[i], 4 + 8); }
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
@@ -330,7 +332,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
     const int wg = warp / 4;
     if (wg == 2) {
-        tc::setmaxnreg_dec<kRegsLight>();
+        tc::setmaxnreg_dec<kRegsProd>();
         // ------------------------------------------------------------------ TMA producers (warps 8, 9)
         // Two producer threads in different warps take alternate stages: a thread that waits on an
         // mbarrier stalls until its own outstanding bulk copies have landed, so one thread alone would
@@ -367,9 +369,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
                     }
             }
+        } else if (warp == 10) {
+            // -------------------------------------------------------------- parameter loader (warp 10)
+            // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
+            // ahead of the converters and the epilogue, so that their loops make no global loads.
+            const int nwin = (ngroups + PW - 1) / PW;
+            uint32_t wi = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+                for (int w = 0; w < nwin; w++, wi++) {
+                    if (!tc::mbar_wait(&sh->p_empty[wi & 1], ((wi >> 1) & 1) ^ 1, p.status, abort_flag)) goto load_done;
+                    __half* ps = params + (wi & 1) * C::PTENS * PW * BM;
+#pragma unroll 1
+                    for (int i = 0; i < BM / 32; i++) {
+                        const int r = 32 * i + lane;
+                        const __half *srow, *zrow;
+                        row_params<MODE>(p, T, r, ngroups, srow, zrow);
+                        stage_params(srow, w * PW, ngroups, ps + r);
+                        if constexpr (!INT8) stage_params(zrow, w * PW, ngroups, ps + PW * BM + r);
+                    }
+                    tc::mbar_arrive(&sh->p_full[wi & 1]);   // every lane: its stores are visible
+                }
+            }
+        load_done:;
         }
     } else if (wg == 0) {
-        tc::setmaxnreg_dec<kRegsLight>();
+        tc::setmaxnreg_dec<kRegsIssue>();
         // ------------------------------------------------------------------ MMA issuers (warps 0-3)
         // They wait only by polling progress counters with weak loads (tc::poll_counters), so the tensor
         // pipe never drains between stages; their completions go out through tcgen05.commit, which tracks
@@ -392,9 +417,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const uint32_t xaddr = tc::smem_u32(xs + s * C::XSTAGE);
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++, g++) {
-                        const uint32_t db = g & 1;
-                        // accumulator db is free once group g-2 has been drained
-                        if (!(ok = tc::poll_counters<8>(sh->epi_done, g >= 2 ? g - 1 : 0, p.status, abort_flag))) break;
+                        const uint32_t db = g % C::ND;
+                        // accumulator db is free once group g-ND has been drained
+                        if (!(ok = tc::poll_counters<8>(sh->epi_done, g >= (uint32_t)C::ND ? g - C::ND + 1 : 0, p.status, abort_flag))) break;
                         tc::fence_after_sync();
 #pragma unroll
                         for (int i = 0; i < G / C::KI; i++) {
@@ -422,39 +447,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int r = 32 * sub + lane;                 // row in tile == TMEM lane
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
         constexpr float kMagic = F16 ? 1024.0f : 128.0f;
-        uint32_t it = 0;
+        uint32_t it = 0, wi = 0;   // stage and parameter-window counters (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-            const __half *srow, *zrow;
-            row_params<MODE>(p, T, r, ngroups, srow, zrow);
-            if (t + (int)gridDim.x < total) {  // warm L2 with the next tile's scale/zero row
-                const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
-                const __half *sn, *zn;
-                row_params<MODE>(p, Tn, r, ngroups, sn, zn);
-                if (zn) prefetch_row_l2(zn, ngroups);
-            }
-            // zero points: read a few stages ahead through a QuadRing (no stall on the loads)
-            QuadRing zr;
-            zr.start(SYM ? nullptr : zrow, ngroups);
             for (int kb = 0; kb < kblocks; kb++) {
                 const int s = it % NS, sa = it % NA;
+                // zero points of the stage's groups from the parameter ring
+                const int g0 = kb * GPK;
+                if (g0 % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto conv_done;
                 float zcur[GPK];
+                const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
 #pragma unroll
-                for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : zr.get(kb * GPK + gi);
-                if (!tc::mbar_wait(&sh->w_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
+                for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
+                if ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups) {   // the window's last stage: release it
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
+                    wi++;
+                }
+                // one combined wait: the stage's packed weights and activations have landed, and TMEM slot
+                // sa is free -- the MMAs of stage it - NA have completed, i.e. that stage's slot of the ring
+                // has been released (its phase cannot be older: this warp has converted stage it - NA, so the
+                // producer refilled it; nor newer: that needs this warp's arrival for it - NA + NS)
+                {
+                    const uint32_t j = it >= (uint32_t)NA ? it - NA : it;
+                    uint64_t* slot_bar = it >= (uint32_t)NA ? &sh->xw_empty[j % NS] : &sh->w_full[s];
+                    const uint32_t slot_par = it >= (uint32_t)NA ? (j / NS) & 1 : (it / NS) & 1;
+                    if (!tc::mbar_wait3(&sh->w_full[s], (it / NS) & 1, &sh->x_full[s], (it / NS) & 1, slot_bar, slot_par,
+                                        p.status, abort_flag))
+                        goto conv_done;
+                }
                 uint4 v[4];
                 const uint32_t wrow = tc::smem_u32(wsm + s * WSTAGE) + r * 64;
 #pragma unroll
                 for (int c = 0; c < 4; c++) v[c] = lds128(wrow + ((c ^ ((r >> 1) & 3)) << 4));
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sh->xw_empty[s]);
-                // TMEM slot sa is free once the MMAs of stage it - NA have completed: that stage's slot of the
-                // ring has been released (its phase cannot be older: this warp has converted stage it - NA,
-                // so the producer refilled it; nor newer: that needs this warp's arrival for it - NA + NS)
-                if (it >= (uint32_t)NA) {
-                    const uint32_t j = it - NA;
-                    if (!tc::mbar_wait(&sh->xw_empty[j % NS], (j / NS) & 1, p.status, abort_flag)) goto conv_done;
-                }
+                if (lane == 0) tc::mbar_arrive_relaxed(&sh->xw_empty[s]);
                 __syncwarp();
                 tc::fence_after_sync();
                 const uint32_t words[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
@@ -486,9 +512,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
                 // publish: this warp's rows of the stage are in TMEM, and the stage's activations landed
-                if (!tc::mbar_wait(&sh->x_full[s], (it / NS) & 1, p.status, abort_flag)) goto conv_done;
                 __syncwarp();
-                if (lane == 0) tc::sts_release(&sh->conv_done[sub], it + 1);
+                if (lane == 0) tc::sts_publish(&sh->conv_done[sub], it + 1);
                 it++;
             }
         }
@@ -509,26 +534,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // group's MMAs its bits ARE the float 1.5 * 2^23 + acc (|acc| < 2^22): the epilogue converts
             // with one packed subtraction instead of an integer-to-float conversion per value.
 #pragma unroll
-            for (int d = 0; d < 2; d++)
+            for (int d = 0; d < C::ND; d++)
 #pragma unroll
                 for (int h = 0; h < 2; h++) tc::tmem_fill32(tbase + lane_field + d * BN + half * 64 + 32 * h, kAccBias);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::sts_release(&sh->epi_init[ew], 1);
+            if (lane == 0) tc::sts_publish(&sh->epi_init[ew], 1);
         }
+        uint32_t wi = 0;   // parameter-window counter (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
 #pragma unroll
             for (int j = 0; j < 32; j++) acc2[j] = 0;
-            if (t + (int)gridDim.x < total) {  // warm L2 with the next tile's scale row
-                const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
-                const __half *sn, *zn;
-                row_params<MODE>(p, Tn, r, ngroups, sn, zn);
-                if (sn) prefetch_row_l2(sn, ngroups);
-            }
             if constexpr (MODE == Mode::Down) {
                 // token and routing weight of this warp's 64 activation rows, staged for the tile's output
                 for (int j = lane; j < 64; j += 32) {
@@ -538,15 +558,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     comb_w[ew * 64 + j] = ok ? p.row_w[m] : 0.0f;
                 }
             }
-            // group scales through a QuadRing (read ahead, no stall on the loads)
-            QuadRing sr;
-            sr.start(srow, ngroups);
             for (int gl = 0; gl < ngroups; gl++) {
-                const uint32_t db = g & 1;
-                float s = sr.get(gl);
+                const uint32_t db = g % C::ND;
+                // group scale from the parameter ring
+                if (gl % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto epi_done;
+                float s = __half2float(params[(wi & 1) * C::PTENS * PW * BM + (gl % PW) * BM + r]);
+                if ((gl + 1) % PW == 0 || gl + 1 == ngroups) {   // the window's last group: release it
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
+                    wi++;
+                }
                 if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
                 const uint64_t s2 = tc::f2_pack(__float_as_uint(s), __float_as_uint(s));
-                if (!tc::mbar_wait(&sh->d_full[db], (g >> 1) & 1, p.status, abort_flag)) goto epi_done;
+                if (!tc::mbar_wait(&sh->d_full[db], (g / C::ND) & 1, p.status, abort_flag)) goto epi_done;
                 __syncwarp();
                 tc::fence_after_sync();
 #pragma unroll
@@ -581,7 +605,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) tc::sts_release(&sh->epi_done[ew], g + 1);   // group g drained
+                if (lane == 0) tc::sts_publish(&sh->epi_done[ew], g + 1);   // group g drained
                 g++;
             }
             // ---------------------------------------------------------- tile output

@@ -35,6 +35,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive without release semantics: the arrival does not wait for this thread's outstanding global
+// loads.  For a consumer that read its operands from shared memory (ld.shared has completed once the
+// values are in registers) and releases the buffer.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -87,6 +95,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     for (int i = 0; i < 64; i++)
         if (mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, status, abort_flag, limit_ns);
+}
+
+// Wait for three phases at once.  The three tests go out back to back, so a consumer that usually
+// finds every phase complete pays one shared-memory round trip instead of three; an incomplete phase
+// falls back to mbar_wait.
+__device__ __forceinline__ bool mbar_wait3(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                           uint32_t p2, int32_t* status, volatile int* abort_flag)
+{
+    uint32_t ok0, ok1, ok2;
+    asm volatile(
+        "{\n\t.reg .pred q0, q1, q2;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q0, [%3], %4;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q1, [%5], %6;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q2, [%7], %8;\n\t"
+        "selp.u32 %0, 1, 0, q0;\n\t"
+        "selp.u32 %1, 1, 0, q1;\n\t"
+        "selp.u32 %2, 1, 0, q2;\n\t}"
+        : "=r"(ok0), "=r"(ok1), "=r"(ok2)
+        : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1), "r"(smem_u32(b2)), "r"(p2)
+        : "memory");
+    if (ok0 & ok1 & ok2) return true;
+    return (ok0 || mbar_wait(b0, p0, status, abort_flag)) && (ok1 || mbar_wait(b1, p1, status, abort_flag)) &&
+           (ok2 || mbar_wait(b2, p2, status, abort_flag));
 }
 
 // ---------------------------------------------------------------------------------------------- //
@@ -206,8 +237,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // or a relaxed / acquire / volatile load -- stalls that thread until the MMAs it issued have retired,
 // which leaves the tensor pipe idle (measured: 64 cycles per M128 N128 K16 MMA without, ~155 with one
 // such wait per 8 MMAs).  Weak loads do not.  So the issuer polls monotonic counters with weak loads;
-// the threads that publish them (converters, epilogue) do the mbarrier waits and TMEM waits first and
-// store the counter with release semantics.
+// the threads that publish them (converters, epilogue) first complete what the counter announces --
+// tcgen05.wait::st / wait::ld, so the TMEM accesses are done, and the mbarrier waits for the data the
+// MMA will read -- and then store the counter with a plain shared-memory store: a release (or even a
+// relaxed) store would also wait for the publisher's unrelated global loads in flight (the scale
+// read-ahead).
 // ---------------------------------------------------------------------------------------------- //
 
 // Register re-partition between warpgroups (every warp of a warpgroup executes the same one).  An
@@ -232,9 +266,9 @@ __device__ __forceinline__ uint32_t lds_weak(const void* p)
     return v;
 }
 
-__device__ __forceinline__ void sts_release(void* p, uint32_t v)
+__device__ __forceinline__ void sts_publish(void* p, uint32_t v)
 {
-    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
 // Spin until each of the n counters at c is >= target.  The fast path makes weak loads only; after a
