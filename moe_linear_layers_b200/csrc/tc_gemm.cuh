@@ -85,9 +85,10 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
     // group parameters staged in shared memory: 2 slots, each PW groups x 128 rows of fp16 scales
     // (and, for 16-bit modes, zero points), group-major so a warp reads 32 consecutive rows
-    static constexpr int PTENS = INT8 ? 1 : 2;                  // scales (+ zero points)
+    // (16-bit modes only; W4A8 has no zero points and its epilogue reads its scales directly)
+    static constexpr int PTENS = 2;                             // scales, zero points
     static constexpr int PSLOT = PW * BM * 2;                   // bytes of one tensor in one slot
-    static constexpr int PARAMS = 2 * PSLOT * PTENS;
+    static constexpr int PARAMS = INT8 ? 0 : 2 * PSLOT * PTENS;
     // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
     // in flight to cover the latency of the activation copies
     static constexpr int NS = INT8 ? 8 : (MODE == Mode::GateUp ? 4 : 5);
@@ -252,6 +253,40 @@ __device__ __forceinline__ void row_params(const Args& p, const Tile& T, int r, 
     }
 }
 
+// W4A8 epilogue: fp16 scales of one row, n of them, read 4 at a time, one 8-byte block ahead: the
+// block for positions [4j, 4j+4) is loaded when position 4j-4 is taken, so a register that is still
+// loading is touched (moved) only 4 positions later.  n % 4 != 0 falls back to direct loads.
+// preload() issues the first block of the next row one tile early, so start() does not wait for it.
+struct QuadRing {
+    const __half* row = nullptr;
+    const __half* pre_row = nullptr;
+    int n = 0;
+    uint2 cur, nxt, pre;
+    __device__ __forceinline__ void preload(const __half* r, int count)
+    {
+        pre_row = (r && (count & 3) == 0) ? r : nullptr;
+        if (pre_row) pre = __ldg(reinterpret_cast<const uint2*>(r));
+    }
+    __device__ __forceinline__ void start(const __half* r, int count)
+    {
+        row = r;
+        n = count;
+        cur = nxt = make_uint2(0u, 0u);
+        if (row && (n & 3) == 0) nxt = row == pre_row ? pre : __ldg(reinterpret_cast<const uint2*>(row));
+    }
+    __device__ __forceinline__ float get(int i)   // positions in increasing order, from 0
+    {
+        if (!row) return 0.0f;
+        if (n & 3) return __half2float(row[i]);
+        if ((i & 3) == 0) {
+            cur = nxt;
+            nxt = i + 4 < n ? __ldg(reinterpret_cast<const uint2*>(row + i + 4)) : make_uint2(0u, 0u);
+        }
+        const uint32_t w = (i & 2) ? cur.y : cur.x;
+        return __half2float(__ushort_as_half((unsigned short)((i & 1) ? (w >> 16) : (w & 0xFFFFu))));
+    }
+};
+
 // PW consecutive fp16 group parameters of one row, from group g0 (zeros past the row's end or for a
 // missing row), stored group-major at dst[j * BM].
 __device__ __forceinline__ void stage_params(const __half* row, int g0, int ng, __half* dst)
@@ -369,7 +404,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
                     }
             }
-        } else if (warp == 10) {
+        } else if (!INT8 && warp == 10) {
             // -------------------------------------------------------------- parameter loader (warp 10)
             // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
             // ahead of the converters and the epilogue, so that their loops make no global loads.
@@ -451,17 +486,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             for (int kb = 0; kb < kblocks; kb++) {
                 const int s = it % NS, sa = it % NA;
-                // zero points of the stage's groups from the parameter ring
-                const int g0 = kb * GPK;
-                if (g0 % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto conv_done;
+                // zero points of the stage's groups from the parameter ring (16-bit modes)
                 float zcur[GPK];
-                const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
 #pragma unroll
-                for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
-                if ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups) {   // the window's last stage: release it
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
-                    wi++;
+                for (int gi = 0; gi < GPK; gi++) zcur[gi] = 8.0f;
+                if constexpr (!INT8) {
+                    const int g0 = kb * GPK;
+                    if (g0 % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto conv_done;
+                    const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
+#pragma unroll
+                    for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
+                    if ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups) {   // the window's last stage: release it
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
+                        wi++;
+                    }
                 }
                 // one combined wait: the stage's packed weights and activations have landed, and TMEM slot
                 // sa is free -- the MMAs of stage it - NA have completed, i.e. that stage's slot of the ring
@@ -542,11 +581,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             __syncwarp();
             if (lane == 0) tc::sts_publish(&sh->epi_init[ew], 1);
         }
-        uint32_t wi = 0;   // parameter-window counter (running across tiles)
+        uint32_t wi = 0;   // parameter-window counter (running across tiles; 16-bit modes)
+        QuadRing sr;       // W4A8: group scales read a few groups ahead
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
+            if constexpr (INT8) {
+                sr.start(srow, ngroups);
+                if (t + (int)gridDim.x < total) {   // load the next tile's first block of scales now
+                    const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
+                    const __half *sn, *zn;
+                    row_params<MODE>(p, Tn, r, ngroups, sn, zn);
+                    sr.preload(sn, ngroups);
+                }
+            }
 #pragma unroll
             for (int j = 0; j < 32; j++) acc2[j] = 0;
             if constexpr (MODE == Mode::Down) {
@@ -560,13 +609,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             }
             for (int gl = 0; gl < ngroups; gl++) {
                 const uint32_t db = g % C::ND;
-                // group scale from the parameter ring
-                if (gl % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto epi_done;
-                float s = __half2float(params[(wi & 1) * C::PTENS * PW * BM + (gl % PW) * BM + r]);
-                if ((gl + 1) % PW == 0 || gl + 1 == ngroups) {   // the window's last group: release it
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
-                    wi++;
+                // group scale: W4A8 from its read-ahead ring, 16-bit modes from the parameter ring
+                float s;
+                if constexpr (INT8) {
+                    s = sr.get(gl);
+                } else {
+                    if (gl % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto epi_done;
+                    s = __half2float(params[(wi & 1) * C::PTENS * PW * BM + (gl % PW) * BM + r]);
+                    if ((gl + 1) % PW == 0 || gl + 1 == ngroups) {   // the window's last group: release it
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
+                        wi++;
+                    }
                 }
                 if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
                 const uint64_t s2 = tc::f2_pack(__float_as_uint(s), __float_as_uint(s));
