@@ -25,19 +25,22 @@
 namespace {
 
 constexpr int kRouteTok = 16;           // tokens per route CTA (= one histogram chunk)
-constexpr int kRouteWarps = 16;
+constexpr int kRouteWarps = 8;
 constexpr int kRouteKC = 64;            // K columns staged per step
 constexpr int kMaxTopk = 16;
 
 // ---------------------------------------------------------------------------------------------- //
 // 1. route
 // ---------------------------------------------------------------------------------------------- //
-// A CTA scores one chunk of 16 tokens against 64 experts at a time.  Warp w owns 4 tokens x 16 experts;
-// lane l owns the k = l (mod 32) partial sums, each an fma chain with k ascending (two experts per
-// packed fma.rn.f32x2, which rounds each half exactly like fmaf); the 32 partials are combined by an
-// xor butterfly (s = 16, 8, 4, 2, 1), which leaves the same value in every lane.  This is the pinned
-// order the oracle reproduces bit for bit.  A producer warp streams 64-column tiles of Wr (fp32) and x
-// (bf16) through a 4-stage TMA ring.
+// A CTA scores one chunk of 16 tokens against 64 experts at a time.  Warp w owns 8 tokens x 16 experts
+// (128 register partials per lane, so each staged value feeds 8 or 16 FMAs); lane l owns the
+// k = l (mod 32) partial sums, each an fma chain with k ascending (two experts per packed
+// fma.rn.f32x2, which rounds each half exactly like fmaf); the 32 partials of a logit are combined by
+// the xor butterfly s = 16, 8, 4, 2, 1 -- computed as a transposing reduction (at each level a lane
+// keeps half of its values and adds its partner's copy of them, 124 shuffles for 128 logits instead of
+// 640), which adds exactly the same pairs as the butterfly.  This is the pinned order the oracle
+// reproduces bit for bit.  A producer warp streams 64-column tiles of Wr (fp32) and x (bf16) through a
+// 4-stage TMA ring.
 constexpr int kRouteStages = 4;
 constexpr int kRouteThreads = (kRouteWarps + 1) * 32;
 constexpr int kRouteWTile = 64 * kRouteKC * 4;       // 64 experts x 64 columns, fp32
@@ -91,12 +94,12 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             }
         }
     } else {
-        // ------------------------------------------------------------------ 16 compute warps
-        const int tg = warp / 4, eg = warp % 4;
+        // ------------------------------------------------------------------ 8 compute warps
+        const int tg = warp / 4, eg = warp % 4;   // tokens 8*tg.., experts 16*eg.. of the 64-block
         for (int eb = 0; eb < neb; eb++) {
-            uint64_t acc[4][8];
+            uint64_t acc[8][8];   // [token][expert pair]
 #pragma unroll
-            for (int a = 0; a < 4; a++)
+            for (int a = 0; a < 8; a++)
 #pragma unroll
                 for (int b = 0; b < 8; b++) acc[a][b] = 0;
             for (int kc = 0; kc < nk; kc++) {
@@ -107,48 +110,68 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < kRouteKC / 32; i++) {
                     const int c = lane + 32 * i;
-                    uint64_t xv[4];
+                    uint64_t wv[8];
 #pragma unroll
-                    for (int a = 0; a < 4; a++) {
-                        const float f = bf16_bits_to_float(xt[(4 * tg + a) * kRouteKC + c]);
-                        xv[a] = pack2(f, f);
-                    }
+                    for (int b = 0; b < 8; b++)
+                        wv[b] = pack2(wt[(16 * eg + 2 * b) * kRouteKC + c], wt[(16 * eg + 2 * b + 1) * kRouteKC + c]);
 #pragma unroll
-                    for (int b = 0; b < 8; b++) {
-                        const uint64_t wv = pack2(wt[(16 * eg + 2 * b) * kRouteKC + c], wt[(16 * eg + 2 * b + 1) * kRouteKC + c]);
+                    for (int a = 0; a < 8; a++) {
+                        const float f = bf16_bits_to_float(xt[(8 * tg + a) * kRouteKC + c]);
+                        const uint64_t xv = pack2(f, f);
 #pragma unroll
-                        for (int a = 0; a < 4; a++) acc[a][b] = ffma2(xv[a], wv, acc[a][b]);
+                        for (int b = 0; b < 8; b++) acc[a][b] = ffma2(xv, wv[b], acc[a][b]);
                     }
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&empty[s]);
             }
+            // transposing butterfly over the 128 partials j = 16 * token + expert (packed in expert pairs):
+            // at the level on lane bit q the lane keeps the half of its values selected by that bit and adds
+            // its partner's copy of them; lane l ends with j = 4l .. 4l+3 in acc[0][0], acc[0][1]
+            auto level = [&](uint64_t& x, uint64_t& y, int bit) {   // x: lower index, y: upper index
+                const bool upper = (lane >> bit) & 1;
+                const uint64_t keep = upper ? y : x, send = upper ? x : y;
+                const uint32_t r0 = __shfl_xor_sync(0xffffffffu, (uint32_t)send, 1 << bit);
+                const uint32_t r1 = __shfl_xor_sync(0xffffffffu, (uint32_t)(send >> 32), 1 << bit);
+                x = pack2(__uint_as_float((uint32_t)keep) + __uint_as_float(r0),
+                          __uint_as_float((uint32_t)(keep >> 32)) + __uint_as_float(r1));
+            };
 #pragma unroll
             for (int a = 0; a < 4; a++)
 #pragma unroll
-                for (int b = 0; b < 8; b++)
+                for (int b = 0; b < 8; b++) level(acc[a][b], acc[a + 4][b], 4);   // j, j + 64
 #pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        float v = __uint_as_float((uint32_t)(acc[a][b] >> (32 * h)));
+            for (int a = 0; a < 2; a++)
 #pragma unroll
-                        for (int sft = 16; sft >= 1; sft >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sft);
-                        const int e = eb * 64 + 16 * eg + 2 * b + h;
-                        if (lane == 0 && e < E) logits[4 * tg + a][e] = bias ? v + bias[e] : v;
-                    }
+                for (int b = 0; b < 8; b++) level(acc[a][b], acc[a + 2][b], 3);   // j, j + 32
+#pragma unroll
+            for (int b = 0; b < 8; b++) level(acc[0][b], acc[1][b], 2);            // j, j + 16
+#pragma unroll
+            for (int b = 0; b < 4; b++) level(acc[0][b], acc[0][b + 4], 1);        // j, j + 8
+#pragma unroll
+            for (int b = 0; b < 2; b++) level(acc[0][b], acc[0][b + 2], 0);        // j, j + 4
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const int j = 4 * lane + q;
+                const int e = eb * 64 + 16 * eg + (j & 15);
+                const float lv = __uint_as_float((uint32_t)(acc[0][q >> 1] >> (32 * (q & 1))));
+                if (e < E) logits[8 * tg + (j >> 4)][e] = bias ? lv + bias[e] : lv;
+            }
         }
     }
     __syncthreads();
 
-    // top-k per token (warp w handles token w of the chunk)
-    const int t = t0 + warp;
-    if (warp < kRouteTok && t < T) {
+    // top-k per token (warp w handles tokens w, w + 9 of the chunk)
+    for (int tt = warp; tt < kRouteTok; tt += kRouteWarps + 1) {
+        const int t = t0 + tt;
+        if (t >= T) break;
         constexpr int PER = tcg::kMaxExperts / 32;
         float v[PER];
         bool finite = true;
 #pragma unroll
         for (int q = 0; q < PER; q++) {
             const int e = lane + 32 * q;
-            v[q] = e < E ? logits[warp][e] : -INFINITY;
+            v[q] = e < E ? logits[tt][e] : -INFINITY;
             if (e < E) finite &= isfinite(v[q]);
         }
         if (!__all_sync(0xffffffffu, finite)) {
