@@ -214,41 +214,55 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 }
 
 // ---------------------------------------------------------------------------------------------- //
-// 2. scan (one CTA, one thread per expert)
+// 2. scan (one CTA of 1024 threads: P = 1024 / E threads per expert, each over a range of chunks)
 // ---------------------------------------------------------------------------------------------- //
-__global__ void moe_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E, int I, int H,
-                                int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
-                                int32_t* __restrict__ counts, int32_t* __restrict__ tiles_gu,
-                                int32_t* __restrict__ tiles_dn)
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) moe_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E,
+                                                               int I, int H, int32_t* __restrict__ chunk_base,
+                                                               int32_t* __restrict__ offsets, int32_t* __restrict__ counts,
+                                                               int32_t* __restrict__ tiles_gu, int32_t* __restrict__ tiles_dn)
 {
-    __shared__ int cnt[tcg::kMaxExperts];
-    const int e = threadIdx.x;
-    int c_e = 0;
-    if (e < E) {
-        for (int c = 0; c < nchunks; c++) c_e += hist[(int64_t)c * E + e];
-        cnt[e] = c_e;
-        if (counts) counts[e] = c_e;
+    __shared__ int part[kScanThreads];
+    __shared__ int cnt[tcg::kMaxExperts], off[tcg::kMaxExperts];
+    const int P = kScanThreads / E;                  // >= 4 (E <= 256)
+    const int e = threadIdx.x % E, pi = threadIdx.x / E;
+    const int per = (nchunks + P - 1) / P;
+    const int c0 = min(nchunks, pi * per), c1 = min(nchunks, c0 + per);
+    int sum = 0;
+    if (pi < P)
+        for (int c = c0; c < c1; c++) sum += hist[(int64_t)c * E + e];   // coalesced across e
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x < E) {   // expert totals
+        int cq = 0;
+        for (int u = 0; u < P; u++) cq += part[u * E + threadIdx.x];
+        cnt[threadIdx.x] = cq;
+        if (counts) counts[threadIdx.x] = cq;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        int off = 0, tg = 0, td = 0;
+        int o = 0, tg = 0, td = 0;
         for (int q = 0; q < E; q++) {
-            offsets[q] = off;
+            const int cq = cnt[q];
+            off[q] = o;
+            offsets[q] = o;
             tiles_gu[q] = tg;
             tiles_dn[q] = td;
-            const int mt = (cnt[q] + tcg::BN - 1) / tcg::BN;
-            off += cnt[q];
+            const int mt = (cq + tcg::BN - 1) / tcg::BN;
+            o += cq;
             tg += mt * (I / 64);
             td += mt * (H / tcg::BM);
         }
-        offsets[E] = off;
+        offsets[E] = o;
         tiles_gu[E] = tg;
         tiles_dn[E] = td;
     }
     __syncthreads();
-    if (e < E) {
-        int run = offsets[e];
-        for (int c = 0; c < nchunks; c++) {
+    if (pi < P) {
+        int run = off[e];
+        for (int u = 0; u < pi; u++) run += part[u * E + e];
+        for (int c = c0; c < c1; c++) {
             chunk_base[(int64_t)c * E + e] = run;
             run += hist[(int64_t)c * E + e];
         }
@@ -265,15 +279,17 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __rest
                                                           float* __restrict__ row_w, uint16_t* __restrict__ xperm)
 {
     __shared__ int pos[kRouteTok * kMaxTopk];
+    __shared__ int cid[kRouteTok * kMaxTopk];   // the chunk's expert ids, token-major
     const int c = blockIdx.x;
     const int t0 = c * kRouteTok;
     const int npairs = min(kRouteTok, T - t0) * topk;
+    for (int q = threadIdx.x; q < npairs; q += blockDim.x) cid[q] = ids[(int64_t)t0 * topk + q];
+    __syncthreads();
     for (int q = threadIdx.x; q < npairs; q += blockDim.x) {
         const int tl = q / topk, j = q % topk;
-        const int e = ids[(int64_t)(t0 + tl) * topk + j];
+        const int e = cid[q];
         int rank = 0;  // earlier tokens of this chunk that chose the same expert (a token picks an expert once)
-        for (int u = 0; u < tl; u++)
-            for (int jj = 0; jj < topk; jj++) rank += ids[(int64_t)(t0 + u) * topk + jj] == e;
+        for (int u = 0; u < tl * topk; u++) rank += cid[u] == e;
         const int p = chunk_base[(int64_t)c * E + e] + rank;
         pos[q] = p;
         perm[p] = (t0 + tl) * topk + j;
@@ -281,11 +297,21 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __rest
         row_w[p] = wts[(int64_t)(t0 + tl) * topk + j];
     }
     __syncthreads();
+    // gather: a warp copies whole rows, eight 16-byte loads in flight per lane before the stores
     const int vec = H / 8;  // 16-byte units per row
-    for (int i = threadIdx.x; i < npairs * vec; i += blockDim.x) {
-        const int q = i / vec, u = i % vec;
-        const int t = t0 + q / topk;
-        reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * H)[u] = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)t * H) + u);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nwarps = blockDim.x / 32;
+    for (int q = warp; q < npairs; q += nwarps) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + q / topk) * H);
+        uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * H);
+        int u = lane;
+        for (; u + 7 * 32 < vec; u += 8 * 32) {
+            uint4 r[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) r[j] = __ldg(src + u + 32 * j);
+#pragma unroll
+            for (int j = 0; j < 8; j++) dst[u + 32 * j] = r[j];
+        }
+        for (; u < vec; u += 32) dst[u] = __ldg(src + u);
     }
 }
 
@@ -432,7 +458,7 @@ extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const flo
         return q4_cuda_status(e);
     moe_route_kernel<<<nch, kRouteThreads, route_smem, s>>>(mrx, mrw, T, H, router_bias, E, topk, ws.ids, ws.wts,
                                                             ws.hist, dev_status);
-    moe_scan_kernel<<<1, tcg::kMaxExperts, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
+    moe_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
                                                    ws.tiles_gu, ws.tiles_dn);
     moe_scatter_kernel<<<nch, 256, 0, s>>>(x, T, H, E, topk, ws.ids, ws.wts, ws.chunk_base, ws.perm, ws.row_tok,
                                            ws.row_w, ws.xperm);
