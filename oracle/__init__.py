@@ -126,7 +126,7 @@ def act_quant(x_bf16_bits, k: int):
 
 
 def linear_w4a8(xq, s_a, packed, scales, n: int, k: int, group: int, rows_m=None, rows_n=None,
-                want_acc: bool = False):
+                want_acc: bool = False, zeros=None, symmetric: bool = True):
     xq = _c(xq, np.int8).reshape(-1, k)
     s_a = _c(s_a, np.float32)
     rm = _c(rows_m, np.int32)
@@ -135,8 +135,10 @@ def linear_w4a8(xq, s_a, packed, scales, n: int, k: int, group: int, rows_m=None
     cn = n if rn is None else len(rn)
     y = np.empty((cm, cn), np.float64)
     acc = np.empty((cm, cn, k // group), np.int32) if want_acc else None
+    if not symmetric and zeros is None:
+        raise OracleError("asymmetric W4A8 needs the zero points")
     lib().orc_linear_w4a8(_p(xq), _p(s_a), xq.shape[0], k, _p(_c(packed, np.uint8)), _p(_c(scales, np.uint16)),
-                          n, group, _p(rm), 0 if rm is None else len(rm), _p(rn), 0 if rn is None else len(rn),
+                          _p(None if symmetric else _c(zeros, np.uint16)), int(bool(symmetric)), n, group, _p(rm), 0 if rm is None else len(rm), _p(rn), 0 if rn is None else len(rn),
                           _p(acc), _p(y))
     return (y, acc) if want_acc else y
 

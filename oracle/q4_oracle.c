@@ -279,13 +279,15 @@ int orc_act_quant(const uint16_t* x, int M, int k, int8_t* q, float* s)
  * W4A8 linear.  [W4A8] §2.3: INT4 codes widened to INT8, INT8 x INT8 products accumulated in
  * INT32, result rescaled by scale_w * scale_a.  With one weight scale per group the INT32 partial
  * is kept per (token, row, group):
- *   acc[m][n][g] = sum_{k in g} xq[m][k] * q[n][k]          (exact int32)
+ *   acc[m][n][g] = sum_{k in g} xq[m][k] * (q[n][k] - z[n][g])     (exact int32)
  *   y[m][n]      = sum_g acc[m][n][g] * scale_w[n][g] * scale_a[m]   (fp64)
- * Symmetric weights (codes -8..7) only; zeros are not used.
+ * Symmetric weights: codes -8..7, z = 0.  Asymmetric weights ([W4A8] §2.3's pseudo-code carries a
+ * weight zero point next to the scale): codes 0..15 and the group's integer zero point z, so the
+ * widened INT8 weight is q - z in [-15, 15].
  * ------------------------------------------------------------------------------------------- */
 void orc_linear_w4a8(const int8_t* xq, const float* s_a, int M, int k,
-                     const uint8_t* packed, const uint16_t* scales, int n, int group,
-                     const int32_t* rows_m, int n_m, const int32_t* rows_n, int n_n,
+                     const uint8_t* packed, const uint16_t* scales, const uint16_t* zeros, int symmetric,
+                     int n, int group, const int32_t* rows_m, int n_m, const int32_t* rows_n, int n_n,
                      int32_t* acc_out, double* y)
 {
     int cm = rows_m ? n_m : M, cn = rows_n ? n_n : n, ng = k / group;
@@ -297,8 +299,9 @@ void orc_linear_w4a8(const int8_t* xq, const float* s_a, int M, int k,
             double sum = 0.0;
             for (int g = 0; g < ng; g++) {
                 int32_t acc = 0;
+                const int32_t z = symmetric ? 0 : (int32_t)orc_f16_to_f32(zeros[(size_t)r * ng + g]);
                 for (int kk = g * group; kk < (g + 1) * group; kk++)
-                    acc += (int32_t)xq[(size_t)mi * k + kk] * (int32_t)code_at(packed, k, r, kk, 1);
+                    acc += (int32_t)xq[(size_t)mi * k + kk] * ((int32_t)code_at(packed, k, r, kk, symmetric) - z);
                 if (acc_out) acc_out[((size_t)im * cn + jn) * ng + g] = acc;
                 sum += (double)acc * (double)orc_f16_to_f32(scales[(size_t)r * ng + g]) * (double)s_a[mi];
             }

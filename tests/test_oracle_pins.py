@@ -37,6 +37,10 @@ def _f16(bits):
     return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
+def _f16_bits(values):
+    return np.asarray(values, dtype=np.float16).view(np.uint16)
+
+
 # ---------------------------------------------------------------------------------------------- #
 # number formats
 # ---------------------------------------------------------------------------------------------- #
@@ -285,6 +289,55 @@ def test_w4a8_scaling():
     x = synth.activations(("pins", "w4a8"), m, k, "student_t3")
     xq, s_a = oracle.act_quant(x, k)
     y = oracle.linear_w4a8(xq, s_a, pk, sc, n, k, group)
+    ref = (xq.astype(np.float64) * s_a[:, None].astype(np.float64)) @ W.astype(np.float64).T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_w4a8_asym_unit_scales_is_integer_matmul_with_zero_points():
+    """Asymmetric weights: the widened INT8 weight is q - z (q in 0..15, z the group's zero point)."""
+    n, k, group, m = 21, 256, 64, 5
+    rng = np.random.default_rng(6)
+    codes = rng.integers(0, 16, size=(n, k))
+    z = rng.integers(0, 16, size=(n, k // group))
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.full((n, k // group), 0x3C00, np.uint16)     # fp16 1.0
+    zeros = _f16_bits(z.astype(np.float32))
+    xq = rng.integers(-128, 128, size=(m, k)).astype(np.int8)
+    s_a = np.ones(m, np.float32)
+    y, acc = oracle.linear_w4a8(xq, s_a, packed, scales, n, k, group, want_acc=True, zeros=zeros, symmetric=False)
+    w_int = codes - np.repeat(z, group, axis=1)
+    assert np.array_equal(y, (xq.astype(np.int64) @ w_int.T.astype(np.int64)).astype(np.float64))
+    for g in range(k // group):
+        sl = slice(g * group, (g + 1) * group)
+        assert np.array_equal(acc[:, :, g], xq[:, sl].astype(np.int64) @ w_int[:, sl].T.astype(np.int64))
+
+
+def test_w4a8_asym_zero_eight_equals_symmetric():
+    """Codes c in -8..7 stored symmetric, or as c + 8 with zero point 8, give the same partials."""
+    n, k, group, m = 13, 256, 128, 4
+    rng = np.random.default_rng(7)
+    c = rng.integers(-8, 8, size=(n, k))
+    sym_packed = ((c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+    u = c + 8
+    asym_packed = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+    sbits = rng.integers(0x1400, 0x3000, size=(n, k // group)).astype(np.uint16)
+    zeros = np.full((n, k // group), 0x4800, np.uint16)      # fp16 8.0
+    x = synth.activations(("pins", "w4a8-z8"), m, k, "student_t3")
+    xq, s_a = oracle.act_quant(x, k)
+    y1, a1 = oracle.linear_w4a8(xq, s_a, sym_packed, sbits, n, k, group, want_acc=True)
+    y2, a2 = oracle.linear_w4a8(xq, s_a, asym_packed, sbits, n, k, group, want_acc=True, zeros=zeros,
+                                symmetric=False)
+    assert np.array_equal(a1, a2) and np.array_equal(y1, y2)
+
+
+def test_w4a8_asym_scaling():
+    """Asymmetric W4A8 equals the fp64 product of the dequantized activations and weights."""
+    n, k, group, m = 9, 256, 128, 3
+    W, q, sbits, z = _exact_grid(n, k, group, False, seed=22)
+    pk, sc, zr = oracle.quantize(W, group, False)
+    x = synth.activations(("pins", "w4a8-asym"), m, k, "student_t3")
+    xq, s_a = oracle.act_quant(x, k)
+    y = oracle.linear_w4a8(xq, s_a, pk, sc, n, k, group, zeros=zr, symmetric=False)
     ref = (xq.astype(np.float64) * s_a[:, None].astype(np.float64)) @ W.astype(np.float64).T
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
 
