@@ -149,10 +149,12 @@ int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, flo
  * Source: the W4A8 page §2.3 (three steps and the pseudo-code: dequant_int4_to_int8, int8 matmul
  * into int32, rescale by scale_w * scale_a).  With one weight scale per group of 128 (or 64) the
  * INT32 partial is kept per (token, row, group):
- *   acc[m][n][g] = sum_{k in g} xq[m][k] * code[n][k]            (exact int32)
- *   y[m][n]      = scale_a[m] * sum_g scale_w[n][g] * acc[m][n][g]  (fp32)
- * W must be symmetric.  y [m][n] fp32 or bf16.  acc_dbg (nullable): [m][n][k/group] int32 copy of the
- * partials, for verification only (slow).  k % 128 == 0.
+ *   acc[m][n][g] = sum_{k in g} xq[m][k] * (code[n][k] - zero[n][g])   (exact int32)
+ *   y[m][n]      = scale_a[m] * sum_g scale_w[n][g] * acc[m][n][g]     (fp32)
+ * Symmetric W: codes -8..7, zero 0.  Asymmetric W (the page's pseudo-code keeps a weight zero point
+ * beside the scale): codes 0..15 and integer zero points 0..15, so the widened INT8 weight is
+ * code - zero in [-15, 15].  y [m][n] fp32 or bf16.  acc_dbg (nullable): [m][n][k/group] int32 copy
+ * of the partials, for verification only (slow).  k % 128 == 0.
  */
 int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                    int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream);

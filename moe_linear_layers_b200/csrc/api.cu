@@ -90,7 +90,7 @@ extern "C" int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, 
 extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                               int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream)
 {
-    int rc = check_weight(w, true);
+    int rc = check_weight(w, false);
     if (rc) return rc;
     if (!xq || !scale_a || !y) return Q4_ERR_NULL;
     if (m < 0) return Q4_ERR_SHAPE;

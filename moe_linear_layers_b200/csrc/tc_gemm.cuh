@@ -73,7 +73,8 @@ constexpr int PW = 16;                   // quantization groups per window of th
 constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
 constexpr float kAccBiasF = 12582912.0f;
 
-template <bool INT8, Mode MODE> struct Cfg {
+// PRING: the group parameters go through the shared-memory ring (every mode except symmetric W4A8)
+template <bool INT8, Mode MODE, bool PRING> struct Cfg {
     static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2);   // activation bytes per stage
     static constexpr int ACOLS = KBLK / (INT8 ? 4 : 2);         // TMEM columns of one widened stage
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
@@ -83,12 +84,12 @@ template <bool INT8, Mode MODE> struct Cfg {
     static constexpr uint32_t A_COL0 = ND * BN;
     static_assert(ND * BN + NA * ACOLS <= (int)kTmemCols, "TMEM columns");
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
-    // group parameters staged in shared memory: 2 slots, each PW groups x 128 rows of fp16 scales
-    // (and, for 16-bit modes, zero points), group-major so a warp reads 32 consecutive rows
-    // (16-bit modes only; W4A8 has no zero points and its epilogue reads its scales directly)
+    // group parameters staged in shared memory: 2 slots, each PW groups x 128 rows of fp16 scales and
+    // zero points, group-major so a warp reads 32 consecutive rows (W4A8's epilogue reads its scales
+    // through a register read-ahead instead, so symmetric W4A8 needs no ring at all)
     static constexpr int PTENS = 2;                             // scales, zero points
     static constexpr int PSLOT = PW * BM * 2;                   // bytes of one tensor in one slot
-    static constexpr int PARAMS = INT8 ? 0 : 2 * PSLOT * PTENS;
+    static constexpr int PARAMS = PRING ? 2 * PSLOT * PTENS : 0;
     // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
     // in flight to cover the latency of the activation copies
     static constexpr int NS = INT8 ? 8 : (MODE == Mode::GateUp ? 4 : 5);
@@ -173,6 +174,18 @@ __device__ __forceinline__ void widen_s8x16(uint32_t w, uint32_t& o0, uint32_t& 
     const uint32_t hi = w & 0xF0F0F0F0u;
     o0 = prmt(lo, hi, 0x5140u);
     o1 = prmt(lo, hi, 0x7362u);
+}
+
+// 8 asymmetric nibbles (codes 0..15) -> 8 int8 of value code - z in natural k order (two words).
+// zb holds 128 - z in every byte: code + (128 - z) lies in 113..143, so a plain 32-bit add has no
+// carries between bytes, and flipping bit 7 of each byte turns the biased value into the two's
+// complement byte of code - z.
+__device__ __forceinline__ void widen_s8_asym(uint32_t w, uint32_t zb, uint32_t& o0, uint32_t& o1)
+{
+    const uint32_t lo = (w & 0x0F0F0F0Fu) + zb;          // codes of even k
+    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) + zb;   // codes of odd k
+    o0 = prmt(lo, hi, 0x5140u) ^ 0x80808080u;
+    o1 = prmt(lo, hi, 0x7362u) ^ 0x80808080u;
 }
 
 __device__ __forceinline__ uint32_t pair16_bits(float v, bool f16)
@@ -314,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
                const __grid_constant__ CUtensorMap tm_wb, Args p)
 {
-    using C = Cfg<INT8, MODE>;
+    constexpr bool PRING = !INT8 || !SYM;
+    using C = Cfg<INT8, MODE, PRING>;
     constexpr bool F16 = MODE == Mode::Down;   // the down projection consumes fp16 h
     constexpr int GPK = KBLK / G;               // groups per K stage
     extern __shared__ uint8_t smem_raw[];
@@ -343,7 +357,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = 0; i < 4; i++) sh->conv_done[i] = 0;
         for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
         tc::mbar_init(&sh->done, kIssuers);
-        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->p_full[i], 32); tc::mbar_init(&sh->p_empty[i], 4 + 8); }
+        // consumers: the converters, and the epilogue unless it is W4A8's
+        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->p_full[i], 32); tc::mbar_init(&sh->p_empty[i], INT8 ? 4 : 4 + 8); }
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
@@ -404,7 +419,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
                     }
             }
-        } else if (!INT8 && warp == 10) {
+        } else if (PRING && warp == 10) {
             // -------------------------------------------------------------- parameter loader (warp 10)
             // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
             // ahead of the converters and the epilogue, so that their loops make no global loads.
@@ -421,7 +436,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         const __half *srow, *zrow;
                         row_params<MODE>(p, T, r, ngroups, srow, zrow);
                         stage_params(srow, w * PW, ngroups, ps + r);
-                        if constexpr (!INT8) stage_params(zrow, w * PW, ngroups, ps + PW * BM + r);
+                        if constexpr (!SYM) stage_params(zrow, w * PW, ngroups, ps + PW * BM + r);
                     }
                     tc::mbar_arrive(&sh->p_full[wi & 1]);   // every lane: its stores are visible
                 }
@@ -486,11 +501,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             for (int kb = 0; kb < kblocks; kb++) {
                 const int s = it % NS, sa = it % NA;
-                // zero points of the stage's groups from the parameter ring (16-bit modes)
+                // zero points of the stage's groups from the parameter ring
                 float zcur[GPK];
 #pragma unroll
                 for (int gi = 0; gi < GPK; gi++) zcur[gi] = 8.0f;
-                if constexpr (!INT8) {
+                if constexpr (PRING) {
                     const int g0 = kb * GPK;
                     if (g0 % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto conv_done;
                     const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
@@ -527,8 +542,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const uint32_t acol = tbase + lane_field + C::A_COL0 + sa * C::ACOLS;
                 if constexpr (INT8) {
                     uint32_t o[32];
+                    if constexpr (SYM) {
 #pragma unroll
-                    for (int w = 0; w < 16; w++) widen_s8x16(words[w], o[2 * w], o[2 * w + 1]);
+                        for (int w = 0; w < 16; w++) widen_s8x16(words[w], o[2 * w], o[2 * w + 1]);
+                    } else {
+                        uint32_t zb[GPK];   // 128 - z in every byte
+#pragma unroll
+                        for (int gi = 0; gi < GPK; gi++) zb[gi] = (uint32_t)(128 - (int)zcur[gi]) * 0x01010101u;
+#pragma unroll
+                        for (int w = 0; w < 16; w++) widen_s8_asym(words[w], zb[(8 * w) / G], o[2 * w], o[2 * w + 1]);
+                    }
                     tc::tmem_st32(acol, o);
                 } else {
                     uint32_t bias[GPK];
@@ -622,7 +645,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         wi++;
                     }
                 }
-                if constexpr (INT8) s *= 0.0625f;   // the MMA saw 16 * code
+                if constexpr (INT8 && SYM) s *= 0.0625f;   // the MMA saw 16 * code
                 const uint64_t s2 = tc::f2_pack(__float_as_uint(s), __float_as_uint(s));
                 if (!tc::mbar_wait(&sh->d_full[db], (g / C::ND) & 1, p.status, abort_flag)) goto epi_done;
                 __syncwarp();
@@ -638,7 +661,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
                                 if (m < T.m_end)
-                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)(v[j] - kAccBias)) >> 4;
+                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
                             }
                         }
                         const uint64_t nb2 = tc::f2_pack(__float_as_uint(-kAccBiasF), __float_as_uint(-kAccBiasF));

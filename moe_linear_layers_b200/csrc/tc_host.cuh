@@ -67,7 +67,7 @@ int launch(const CUtensorMap& mx, const CUtensorMap& ma, const CUtensorMap& mb, 
            cudaStream_t s)
 {
     auto kern = tc_gemm_kernel<INT8, G, SYM, MODE>;
-    constexpr int smem = Cfg<INT8, MODE>::SMEM;
+    constexpr int smem = Cfg<INT8, MODE, !INT8 || !SYM>::SMEM;
     if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return q4_cuda_status(e);
     // The kernel re-partitions its registers between warpgroups (setmaxnreg) assuming a launch
     // allocation of kLaunchRegs per thread; a build that allocated fewer would make the increase wait

@@ -192,7 +192,7 @@ def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a
 def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dtype=torch.float32,
                    y: torch.Tensor | None = None, acc_dbg: torch.Tensor | None = None,
                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . code)_g; symmetric W."""
+    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . (code - zero))_g; zero = 0 for symmetric W."""
     _dev(xq, torch.int8, "xq")
     _dev(scale_a, torch.float32, "scale_a")
     m = xq.shape[0]

@@ -65,10 +65,10 @@ def test_linear_w4a16_validation(args, expect):
     assert rc == expect
 
 
-def test_w4a8_needs_symmetric_weights():
-    w = _w(sym=0, zeros=FAKE)
+def test_w4a8_asymmetric_weights_need_zero_points():
+    w = _w(sym=0, zeros=None)
     rc = q4._lib.q4_linear_w4a8(FAKE, FAKE, 16, ctypes.byref(w), FAKE, 0, None, None, None)
-    assert rc == q4.Q4_ERR_UNSUPPORTED
+    assert rc == q4.Q4_ERR_NULL
 
 
 def test_quantize_validation():

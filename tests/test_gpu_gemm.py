@@ -65,12 +65,12 @@ def test_w4a16_prefill_outlier_channels(q4, m, n, k):
     assert np.array_equal(cpu_u16(y16), bf16_rne(y.cpu().numpy()))
 
 
-def _w4a8(q4, m, n, k, group, tag, want_acc=False):
+def _w4a8(q4, m, n, k, group, tag, want_acc=False, sym=True):
     W = synth.weights(("test", "w4a8", tag, n, k, group), n, k)
-    pk, sc, _ = oracle.quantize(W, group, True)
+    pk, sc, zr = oracle.quantize(W, group, sym)
     x = synth.activations(("test", "w4a8-x", tag, m, k), m, k, "student_t3")
     xq_ref, sa_ref = oracle.act_quant(x, k)
-    w = upload_weight(q4, pk, sc, None, n, k, group, True)
+    w = upload_weight(q4, pk, sc, None if sym else zr, n, k, group, sym)
     xq, sa = q4.act_quant_per_token(cuda_u16_as(x, torch.bfloat16))
     acc = torch.zeros((m, n, k // group), dtype=torch.int32, device="cuda") if want_acc else None
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -78,12 +78,12 @@ def _w4a8(q4, m, n, k, group, tag, want_acc=False):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
-    return y, acc, (xq_ref, sa_ref, pk, sc), w, xq, sa
+    return y, acc, (xq_ref, sa_ref, pk, sc, zr), w, xq, sa
 
 
 @pytest.mark.parametrize("m,n,k,group", [(16, 128, 128, 128), (130, 333, 512, 128), (64, 256, 256, 64)])
 def test_w4a8_int32_partials_bitexact(q4, m, n, k, group):
-    y, acc, (xq, sa, pk, sc), *_ = _w4a8(q4, m, n, k, group, "acc", want_acc=True)
+    y, acc, (xq, sa, pk, sc, _), *_ = _w4a8(q4, m, n, k, group, "acc", want_acc=True)
     ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True)
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert_close(y.cpu().numpy(), ref, what="w4a8")
@@ -91,9 +91,27 @@ def test_w4a8_int32_partials_bitexact(q4, m, n, k, group):
 
 @pytest.mark.parametrize("m,n,k", [(16, 2048, 2048), (256, 8192, 2048), (4096, 2048, 8192), (4096, 512, 2048)])
 def test_w4a8_workload_shapes(q4, m, n, k):
-    y, _, (xq, sa, pk, sc), w, xqd, sad = _w4a8(q4, m, n, k, 128, "shape")
+    y, _, (xq, sa, pk, sc, _), w, xqd, sad = _w4a8(q4, m, n, k, 128, "shape")
     rows = np.arange(0, m, max(1, m // 32))
     ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, 128, rows_m=rows)
     assert_close(y.cpu().numpy()[rows], ref, what=f"w4a8 {m}x{n}x{k}")
     y16 = q4.q4_linear_w4a8(xqd, sad, w, out_dtype=torch.bfloat16)
     assert np.array_equal(cpu_u16(y16), bf16_rne(y.cpu().numpy()))
+
+
+@pytest.mark.parametrize("m,n,k,group", [(16, 128, 128, 128), (130, 333, 512, 128), (64, 256, 256, 64),
+                                         (200, 1000, 2048, 64)])
+def test_w4a8_asym_int32_partials_bitexact(q4, m, n, k, group):
+    """Asymmetric weights: the widened INT8 weight is code - zero; partials bit-exact."""
+    y, acc, (xq, sa, pk, sc, zr), *_ = _w4a8(q4, m, n, k, group, "asym", want_acc=True, sym=False)
+    ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True, zeros=zr, symmetric=False)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_close(y.cpu().numpy(), ref, what="w4a8 asym")
+
+
+@pytest.mark.parametrize("m,n,k", [(4096, 2048, 2048), (256, 8192, 2048)])
+def test_w4a8_asym_workload_shapes(q4, m, n, k):
+    y, _, (xq, sa, pk, sc, zr), w, xqd, sad = _w4a8(q4, m, n, k, 128, "asym-shape", sym=False)
+    rows = np.arange(0, m, max(1, m // 32))
+    ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, 128, rows_m=rows, zeros=zr, symmetric=False)
+    assert_close(y.cpu().numpy()[rows], ref, what=f"w4a8 asym {m}x{n}x{k}")
