@@ -114,6 +114,22 @@ def linear_w4a16(x_bf16_bits, packed, scales, zeros, n: int, k: int, group: int,
     return y
 
 
+def silu_mul(gate_f32, up_f32):
+    """h = silu(g) * u = g / (1 + e^-g) * u in fp64 from fp32 inputs (the SwiGLU gating of the dense FFN
+    and of every expert: "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" MoE架构设计)."""
+    g = np.asarray(gate_f32, np.float32).astype(np.float64)
+    u = np.asarray(up_f32, np.float32).astype(np.float64)
+    return g / (1.0 + np.exp(-g)) * u
+
+
+def linear_w4a16_swiglu(gate_f32, up_f32, packed, scales, zeros, n: int, k: int, group: int,
+                        symmetric: bool) -> np.ndarray:
+    """fp64 y[m][n] = sum_k silu(g) * u * dequant(W): the dense FFN's down projection on its gated input."""
+    h = silu_mul(gate_f32, up_f32).reshape(-1, k)
+    w = dequant(packed, scales, zeros, k, group, symmetric).astype(np.float64)
+    return h @ w.T
+
+
 def act_quant(x_bf16_bits, k: int):
     x = _c(x_bf16_bits, np.uint16).reshape(-1, k)
     m = x.shape[0]

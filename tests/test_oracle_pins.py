@@ -343,6 +343,36 @@ def test_w4a8_asym_scaling():
 
 
 # ---------------------------------------------------------------------------------------------- #
+# SwiGLU-gated input of the dense FFN's down projection
+# ---------------------------------------------------------------------------------------------- #
+
+def test_silu_mul_identities():
+    """silu(g) - silu(-g) = g (sigmoid(-g) = 1 - sigmoid(g)); silu(0) = 0; u scales linearly."""
+    g = np.linspace(-30, 30, 2001, dtype=np.float32)
+    one = np.ones_like(g)
+    d = oracle.silu_mul(g, one) - oracle.silu_mul(-g, one)
+    np.testing.assert_allclose(d, g.astype(np.float64), rtol=1e-14, atol=1e-14)
+    assert oracle.silu_mul(np.float32(0), np.float32(5)) == 0.0
+    u = np.float32(3.0)
+    np.testing.assert_allclose(oracle.silu_mul(g, u * one), 3.0 * oracle.silu_mul(g, one), rtol=1e-15)
+
+
+def test_swiglu_linear_reduces_to_plain_linear_for_saturated_gate():
+    """With gate = 32 (sigmoid(32) = 1 - 1.3e-14) and up = x / 32 (exact), h = x to 1e-13: the fused
+    product equals the plain W4A16 product on x."""
+    n, k, group, m = 24, 512, 128, 2
+    W = synth.weights(("pins", "swiglu"), n, k)
+    pk, sc, zr = oracle.quantize(W, group, False)
+    x = synth.activations(("pins", "swiglu-x"), m, k)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    gate = np.full((m, k), 32.0, np.float32)
+    up = (xf / np.float32(32.0)).astype(np.float32)
+    y = oracle.linear_w4a16_swiglu(gate, up, pk, sc, zr, n, k, group, False)
+    ref = oracle.linear_w4a16(x, pk, sc, zr, n, k, group, False)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------------------------------------- #
 # router and permutation
 # ---------------------------------------------------------------------------------------------- #
 
