@@ -130,6 +130,19 @@ int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, i
 int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, int32_t m, const q4_weight* w,
                             void* const* y, int32_t out_dtype, int32_t* dev_status, void* stream);
 
+/*
+ * q4_linear_w4a16_swiglu -- the down projection of a dense SwiGLU FFN at small m, with the gating
+ * fused into its input: y[m][n] = sum_k h[m][k] * dequant(W)[n][k], h = silu(gate) * up =
+ * gate / (1 + e^-gate) * up, computed in fp32 from the gate and up projections' fp32 outputs.
+ * Source: "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" MoE架构设计 (experts and the base
+ * model's FFN are SwiGLU); the fusion is a launch-level choice (h is never written to memory).
+ * gate, up: fp32 [m][k], 16-byte aligned; 1 <= m <= 4; k % 64 == 0, k <= 16384.  h is carried like
+ * x in q4_linear_w4a16's GEMV (int16 per 64-value block with a power-of-two scale, one binade lower
+ * so that no fp32 value rounds out of range).  dev_status: Q4_ERR_NONFINITE when an h is not finite.
+ */
+int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_t m, const q4_weight* w, void* y,
+                           int32_t out_dtype, int32_t* dev_status, void* stream);
+
 /* Largest m that q4_linear_w4a16 serves with the GEMV kernel. */
 int q4_linear_w4a16_max_gemv_m(void);
 

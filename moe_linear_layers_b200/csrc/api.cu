@@ -2,7 +2,8 @@
 #include "q4_common.cuh"
 
 int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, const q4_weight* w, void* const* y,
-                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream);
+                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream,
+                               const float* const* g = nullptr, const float* const* u = nullptr);
 int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                       int32_t out_dtype, int32_t* acc_dbg, bool int8_path, int32_t* dev_status,
                       cudaStream_t stream);
@@ -85,6 +86,23 @@ extern "C" int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, 
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (w[0].k % 64 || w[0].k > 16384) return Q4_ERR_UNSUPPORTED;
     return q4_gemv_w4a16_launch_group(count, x, m, w, y, out_dtype, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_t m, const q4_weight* w, void* y,
+                                      int32_t out_dtype, int32_t* dev_status, void* stream)
+{
+    int rc = check_weight(w, false);
+    if (rc) return rc;
+    if (!gate || !up || !y) return Q4_ERR_NULL;
+    if (m < 1 || m > kMaxGemvM) return Q4_ERR_SHAPE;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(gate) || !q4_aligned16(up) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
+    if (w->k % 64 || w->k > 16384) return Q4_ERR_UNSUPPORTED;
+    if (w->n == 0) return Q4_OK;
+    void* ys[1] = {y};
+    const float* gs[1] = {gate};
+    const float* us[1] = {up};
+    return q4_gemv_w4a16_launch_group(1, nullptr, m, w, ys, out_dtype, dev_status, (cudaStream_t)stream, gs, us);
 }
 
 extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,

@@ -56,7 +56,9 @@ constexpr int kWarpK = 32 * kLaneK;                 // 2048
 constexpr int kRedBytesMax = 16384;                 // split-k partial sums per CTA
 
 struct Problem {
-    const uint16_t* x;       // [m][k] bf16
+    const uint16_t* x;       // [m][k] bf16 (unused when g is set)
+    const float* g;          // fused SwiGLU input: x = silu(g) * u, fp32 [m][k] each (or null)
+    const float* u;
     const uint8_t* packed;   // [n][k/2]
     const __half* scales;    // [n][k/group]
     const __half* zeros;     // [n][k/group] or null
@@ -176,6 +178,73 @@ __device__ __forceinline__ uint4 x_ints(const uint4& v, float scale)
     return o;
 }
 
+// Fused SwiGLU input (the dense FFN's down projection): x = silu(g) * u = g / (1 + e^-g) * u in fp32,
+// staged like bf16 x but from fp32 values, with the block scale one binade lower (max * 2^e in
+// [2^13, 2^14)) so that rounding an fp32 value can never reach 2^15.
+__device__ __forceinline__ uint4 x_ints_f32(const float (&h)[8], float scale)
+{
+    constexpr float kMagic = 12582912.0f;
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) b[i] = __float_as_uint(fmaf(h[i], scale, kMagic));
+    uint4 o;
+    o.x = prmt(b[0], b[2], 0x5410u);
+    o.y = prmt(b[4], b[6], 0x5410u);
+    o.z = prmt(b[1], b[3], 0x5410u);
+    o.w = prmt(b[5], b[7], 0x5410u);
+    return o;
+}
+
+__device__ __forceinline__ float2 block_scale_f32(uint32_t amax_bits)
+{
+    const int ex = (int)((amax_bits >> 23) & 0xFFu);
+    if (amax_bits == 0 || ex == 0xFF) return make_float2(1.0f, 1.0f);
+    const int e = min(126, max(-126, 140 - ex));
+    return make_float2(__uint_as_float((uint32_t)(127 + e) << 23), __uint_as_float((uint32_t)(127 - e) << 23));
+}
+
+template <int MT>
+__device__ __noinline__ void stage_swiglu(const float* g, const float* u, int k, int nw, uint4* xs, float* xinv,
+                                             int32_t* status)
+{
+    bool bad = false;
+#pragma unroll
+    for (int mm = 0; mm < MT; mm++) {
+        const float4* gr = reinterpret_cast<const float4*>(g + (int64_t)mm * k);
+        const float4* ur = reinterpret_cast<const float4*>(u + (int64_t)mm * k);
+        for (int i = 0; i * kComputeThreads < nw; i++) {   // uniform; nw % 8 == 0 keeps blocks together
+            const int w = i * kComputeThreads + threadIdx.x;
+            float h[8];
+            uint32_t a = 0;
+            if (w < nw) {
+                const float4 g0 = __ldg(gr + 2 * w), g1 = __ldg(gr + 2 * w + 1);
+                const float4 u0 = __ldg(ur + 2 * w), u1 = __ldg(ur + 2 * w + 1);
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    h[j] = gv[j] * __frcp_rn(1.0f + __expf(-gv[j])) * uv[j];
+                    bad |= !isfinite(h[j]);
+                    a = max(a, __float_as_uint(h[j]) & 0x7FFFFFFFu);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) h[j] = 0.0f;
+            }
+            a = max(a, __shfl_xor_sync(0xffffffffu, a, 1));
+            a = max(a, __shfl_xor_sync(0xffffffffu, a, 2));
+            a = max(a, __shfl_xor_sync(0xffffffffu, a, 4));
+            const float2 sc = block_scale_f32(a);
+            if (w < nw) {
+                const int L = w >> 3, j = w & 7;
+                xs[mm * nw + (L << 3) + (j ^ (L & 7))] = x_ints_f32(h, sc.x);
+                if (j == 0) xinv[mm * (nw / 8) + L] = sc.y;
+            }
+        }
+    }
+    if (bad) q4_set_status(status, Q4_ERR_NONFINITE);
+}
+
 // Per-halfword max of the bf16 magnitudes of a word (integer order = magnitude order for non-NaN),
 // and a flag for an all-ones exponent (inf or NaN) in any of its 8 values.
 __device__ __forceinline__ uint32_t bf16_mag_max(const uint4& v, uint32_t& bad)
@@ -280,7 +349,12 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
             const int pre = min(nstages, kStages);
             for (int st = 0; st < pre; st++) issue(st);
             // x too: an L2 prefetch is coherent, so it is safe before the wait and shortens the read after it
-            prefetch_l2(P.x, (uint32_t)(p.m * p.k * 2));
+            if (P.g) {
+                prefetch_l2(P.g, (uint32_t)(p.m * p.k * 4));
+                prefetch_l2(P.u, (uint32_t)(p.m * p.k * 4));
+            } else {
+                prefetch_l2(P.x, (uint32_t)(p.m * p.k * 2));
+            }
             if (nstages > kStages) {
                 const int rl = r0 + kStages * rps;
                 prefetch_l2_range(P.packed + (int64_t)rl * rowbytes, P.packed + (int64_t)r1 * rowbytes);
@@ -304,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
     // thread and pass (coalesced), all loads issued first and the passes independent of one another;
     // the 8 threads of a block share its scale.  Word w of block L is staged at 8L + ((w % 8) ^ (L % 8)):
     // conflict-free lane loads.
-    {
+    if (P.g) {
+        stage_swiglu<MT>(P.g, P.u, p.k, nw, xs, xinv, p.status);
+    } else {
         constexpr int kMaxPasses = 16384 / 8 / kComputeThreads;
         uint32_t bad = 0;
 #pragma unroll
@@ -480,8 +556,10 @@ int launch_m(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStre
 
 // Host entry used by q4_linear_w4a16 (count == 1) and q4_linear_w4a16_grouped: m <= 4, and every
 // problem with the same k (a multiple of 64, at most 16384), group and symmetry.
+// g, u (nullable, both or neither): the problems' inputs are silu(g[i]) * u[i] instead of x[i].
 int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, const q4_weight* w, void* const* y,
-                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream)
+                               int32_t out_dtype, int32_t* dev_status, cudaStream_t stream,
+                               const float* const* g, const float* const* u)
 {
     if (count < 1 || count > kMaxProblems || m < 1 || m > kMaxM) return Q4_ERR_UNSUPPORTED;
     const int k = w[0].k, group = w[0].group, sym = w[0].symmetric;
@@ -524,7 +602,9 @@ int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, c
     int ctas = 0;
     for (int i = 0; i < count; i++) {
         Problem& P = p.prob[i];
-        P.x = x[i];
+        P.x = x ? x[i] : nullptr;
+        P.g = g ? g[i] : nullptr;
+        P.u = u ? u[i] : nullptr;
         P.packed = w[i].packed;
         P.scales = reinterpret_cast<const __half*>(w[i].scales);
         P.zeros = reinterpret_cast<const __half*>(w[i].zeros);

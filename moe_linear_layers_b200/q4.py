@@ -32,7 +32,7 @@ Q4_OUT_F32 = 0
 Q4_OUT_BF16 = 1
 
 EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
-            "q4_linear_w4a16_grouped",
+            "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -52,6 +52,7 @@ _lib.q4_last_cuda_error_string.restype = ctypes.c_char_p
 _lib.q4_linear_w4a16_max_gemv_m.restype = ctypes.c_int
 _lib.q4_quantize_pack.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p]
 _lib.q4_linear_w4a16.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p]
+_lib.q4_linear_w4a16_swiglu.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p]
 _lib.q4_linear_w4a16_grouped.argtypes = [_i32, ctypes.POINTER(_p), _i32, ctypes.POINTER(q4_weight),
                                          ctypes.POINTER(_p), _i32, _p, _p]
 _lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
@@ -144,6 +145,21 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
     od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
     _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
            "q4_linear_w4a16")
+    return y
+
+
+def q4_linear_w4a16_swiglu(gate: torch.Tensor, up: torch.Tensor, w: Q4Weight, out_dtype=torch.float32,
+                           y: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """y[m][n] = h[m][k] . dequant(W)^T with h = silu(gate) * up (fp32 CUDA tensors [m][k], m <= 4)."""
+    _dev(gate, torch.float32, "gate")
+    _dev(up, torch.float32, "up")
+    m = gate.numel() // w.k
+    if y is None:
+        y = torch.empty((m, w.n), dtype=out_dtype, device=gate.device)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    _check(_lib.q4_linear_w4a16_swiglu(_ptr(gate), _ptr(up), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status),
+                                       _stream(stream)), "q4_linear_w4a16_swiglu")
     return y
 
 

@@ -208,3 +208,37 @@ def test_act_quant_nonfinite_sets_status(q4):
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     q4.act_quant_per_token(x, dev_status=st)
     assert int(st.item()) == q4.Q4_ERR_NONFINITE
+
+
+# ---------------------------------------------------------------------------------------------- #
+# dense SwiGLU FFN down projection with the gating fused into the GEMV's input
+# ---------------------------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("m,n,k,group,sym", [(1, 2048, 8192, 128, False), (2, 333, 1024, 64, True),
+                                             (4, 512, 2048, 128, False), (1, 130, 64, 64, False)])
+def test_w4a16_swiglu_fused_input(q4, m, n, k, group, sym):
+    W = synth.weights(("test", "swiglu", n, k, group, sym), n, k)
+    pk, sc, zr = oracle.quantize(W, group, sym)
+    gate = (synth.normal(synth.stream_key("test", "swiglu-g", m, k), m * k) * 2.0).astype(np.float32).reshape(m, k)
+    up = synth.normal(synth.stream_key("test", "swiglu-u", m, k), m * k).astype(np.float32).reshape(m, k)
+    ref = oracle.linear_w4a16_swiglu(gate, up, pk, sc, zr, n, k, group, sym)
+    w = upload_weight(q4, pk, sc, None if sym else zr, n, k, group, sym)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.q4_linear_w4a16_swiglu(torch.from_numpy(gate).cuda(), torch.from_numpy(up).cuda(), w, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close(y.cpu().numpy(), ref, what=f"swiglu gemv {m}x{n}x{k}")
+
+
+def test_w4a16_swiglu_nonfinite_status(q4):
+    n, k = 128, 256
+    W = synth.weights(("test", "swiglu-nf"), n, k)
+    pk, sc, zr = oracle.quantize(W, 128, True)
+    w = upload_weight(q4, pk, sc, None, n, k, 128, True)
+    gate = torch.ones((1, k), dtype=torch.float32, device="cuda")
+    up = torch.ones((1, k), dtype=torch.float32, device="cuda")
+    up[0, 77] = float("inf")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.q4_linear_w4a16_swiglu(gate, up, w, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == q4.Q4_ERR_NONFINITE
