@@ -256,6 +256,19 @@ def run_decode(q4, args, ws, weights, dev):
         for w, x, y in zip(weights, xs, ys):
             q4.q4_linear_w4a16(x, w, y=y)
 
+    # the same step with the dense FFN chained: down consumes silu(gate) * up of this layer's [gate, up]
+    # outputs through q4_linear_w4a16_swiglu (the gating fused into the GEMV's input)
+    calls_fused = []
+    for l in range(synth.LLAMA_1B_LAYERS):
+        b = 7 * l
+        calls_fused += [calls[4 * l], calls[4 * l + 1], calls[4 * l + 2],
+                        lambda b=b: q4.q4_linear_w4a16_swiglu(ys[b + 4], ys[b + 5], weights[b + 6], y=ys[b + 6])]
+    bytes_fused = bytes_step + synth.LLAMA_1B_LAYERS * (2 * 4 * 8192 - 2 * 8192)   # down reads fp32 g, u
+
+    def step_fused():
+        for c in calls_fused:
+            c()
+
     g = graph_of(step)
     for _ in range(args.warmup):
         g.replay()
@@ -269,6 +282,10 @@ def run_decode(q4, args, ws, weights, dev):
     for _ in range(args.warmup):
         gu.replay()
     ms_u = time_replays(gu, args.steps, ws) / args.steps
+    gf = graph_of(step_fused)
+    for _ in range(args.warmup):
+        gf.replay()
+    ms_f = time_replays(gf, args.steps, ws) / args.steps
 
     # end to end through the public calls with host buffers: the step's x (pinned host memory) copied
     # in, the 64 calls issued eagerly, every y copied back to pinned host memory
@@ -311,6 +328,10 @@ def run_decode(q4, args, ws, weights, dev):
                              "q4_linear_w4a16: 64 launches (programmatic dependent launch)",
                    "ungrouped": {"ms_per_step": round(ms_u, 5), "value": round(bytes_step / (ms_u * 1e-3) / 1e9, 2),
                                  "launch": "112 single q4_linear_w4a16 calls"},
+                   "fused_swiglu_ffn": {"ms_per_step": round(ms_f, 5),
+                                        "value": round(bytes_fused / (ms_f * 1e-3) / 1e9, 2),
+                                        "launch": "as the headline, but down = q4_linear_w4a16_swiglu on this "
+                                                  "layer's gate/up outputs (a real dependency chain)"},
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(per_gpu / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles("gemv_decode"),

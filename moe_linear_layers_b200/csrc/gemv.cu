@@ -204,7 +204,7 @@ __device__ __forceinline__ float2 block_scale_f32(uint32_t amax_bits)
 }
 
 template <int MT>
-__device__ __noinline__ void stage_swiglu(const float* g, const float* u, int k, int nw, uint4* xs, float* xinv,
+__device__ __forceinline__ void stage_swiglu(const float* g, const float* u, int k, int nw, uint4* xs, float* xinv,
                                              int32_t* status)
 {
     bool bad = false;
@@ -293,7 +293,7 @@ __device__ __forceinline__ void store_y(void* y, int64_t o, float v, int out_bf1
     else reinterpret_cast<float*>(y)[o] = v;
 }
 
-template <int KSPLIT, int MT, bool SYM>
+template <int KSPLIT, int MT, bool SYM, bool SWIGLU>
 __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4a16_gemv_kernel(const __grid_constant__ GemvParams p)
 {
     constexpr int TEAMS = kComputeWarps / KSPLIT;
@@ -349,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
             const int pre = min(nstages, kStages);
             for (int st = 0; st < pre; st++) issue(st);
             // x too: an L2 prefetch is coherent, so it is safe before the wait and shortens the read after it
-            if (P.g) {
+            if constexpr (SWIGLU) {
                 prefetch_l2(P.g, (uint32_t)(p.m * p.k * 4));
                 prefetch_l2(P.u, (uint32_t)(p.m * p.k * 4));
             } else {
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
     // thread and pass (coalesced), all loads issued first and the passes independent of one another;
     // the 8 threads of a block share its scale.  Word w of block L is staged at 8L + ((w % 8) ^ (L % 8)):
     // conflict-free lane loads.
-    if (P.g) {
+    if constexpr (SWIGLU) {
         stage_swiglu<MT>(P.g, P.u, p.k, nw, xs, xinv, p.status);
     } else {
         constexpr int kMaxPasses = 16384 / 8 / kComputeThreads;
@@ -513,18 +513,20 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
 }
 
 template <int KSPLIT, int MT>
-int launch(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStream_t s)
+int launch(const GemvParams& p, int symmetric, bool swiglu, int grid, size_t smem, cudaStream_t s)
 {
-    auto kern = symmetric ? w4a16_gemv_kernel<KSPLIT, MT, true> : w4a16_gemv_kernel<KSPLIT, MT, false>;
+    auto kern = swiglu ? (symmetric ? w4a16_gemv_kernel<KSPLIT, MT, true, true> : w4a16_gemv_kernel<KSPLIT, MT, false, true>)
+                       : (symmetric ? w4a16_gemv_kernel<KSPLIT, MT, true, false> : w4a16_gemv_kernel<KSPLIT, MT, false, false>);
     // the shared-memory opt-in is set once per device and instantiation (it does not affect occupancy)
-    static uint64_t opted[2] = {0, 0};
+    static uint64_t opted[4] = {0, 0, 0, 0};
+    const int slot = (symmetric ? 1 : 0) + (swiglu ? 2 : 0);
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
-    if (!(opted[symmetric ? 1 : 0] & bit)) {
+    if (!(opted[slot] & bit)) {
         if (const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024))
             return q4_cuda_status(e);
-        opted[symmetric ? 1 : 0] |= bit;
+        opted[slot] |= bit;
     }
     // Programmatic stream serialization: the kernel may start, and fill its weight ring, while the
     // previous kernel on the stream runs; x is read only after griddepcontrol.wait.
@@ -542,13 +544,13 @@ int launch(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStream
 }
 
 template <int KSPLIT>
-int launch_m(const GemvParams& p, int symmetric, int grid, size_t smem, cudaStream_t s)
+int launch_m(const GemvParams& p, int symmetric, bool swiglu, int grid, size_t smem, cudaStream_t s)
 {
     switch (p.m) {
-        case 1: return launch<KSPLIT, 1>(p, symmetric, grid, smem, s);
-        case 2: return launch<KSPLIT, 2>(p, symmetric, grid, smem, s);
-        case 3: return launch<KSPLIT, 3>(p, symmetric, grid, smem, s);
-        default: return launch<KSPLIT, 4>(p, symmetric, grid, smem, s);
+        case 1: return launch<KSPLIT, 1>(p, symmetric, swiglu, grid, smem, s);
+        case 2: return launch<KSPLIT, 2>(p, symmetric, swiglu, grid, smem, s);
+        case 3: return launch<KSPLIT, 3>(p, symmetric, swiglu, grid, smem, s);
+        default: return launch<KSPLIT, 4>(p, symmetric, swiglu, grid, smem, s);
     }
 }
 
@@ -615,9 +617,9 @@ int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, c
     }
     if (ctas == 0) return Q4_OK;
     switch (ksplit) {
-        case 1: return launch_m<1>(p, sym, ctas, smem, stream);
-        case 2: return launch_m<2>(p, sym, ctas, smem, stream);
-        case 4: return launch_m<4>(p, sym, ctas, smem, stream);
-        default: return launch_m<8>(p, sym, ctas, smem, stream);
+        case 1: return launch_m<1>(p, sym, g != nullptr, ctas, smem, stream);
+        case 2: return launch_m<2>(p, sym, g != nullptr, ctas, smem, stream);
+        case 4: return launch_m<4>(p, sym, g != nullptr, ctas, smem, stream);
+        default: return launch_m<8>(p, sym, g != nullptr, ctas, smem, stream);
     }
 }
