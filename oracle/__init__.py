@@ -191,6 +191,16 @@ def permute(ids, E: int):
     return offsets, perm
 
 
+def shared_expert(x_bf16_bits, H: int, gate, up, down, I_s: int, group: int, symmetric: bool, tokens=None):
+    """A shared expert every token passes through (the MoE architecture sections of the W4A8 and
+    INT4+MoE pages): one SwiGLU FFN with routing weight 1, i.e. the routed-expert computation with a
+    single expert chosen by every token.  Returns fp64 [n_tok][H]."""
+    T = np.asarray(x_bf16_bits).reshape(-1, H).shape[0]
+    ids = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1), np.float64)
+    return moe_experts(x_bf16_bits, H, ids, w, gate, up, down, I_s, group, symmetric, tokens=tokens)
+
+
 def moe_experts(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int, symmetric: bool,
                 tokens=None):
     """gate/up/down: (packed, scales, zeros) of the stacked expert matrices.  Returns fp64 [n_tok][H]."""

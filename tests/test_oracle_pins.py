@@ -372,6 +372,22 @@ def test_swiglu_linear_reduces_to_plain_linear_for_saturated_gate():
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
 
 
+def test_shared_expert_is_the_dense_swiglu_ffn():
+    """The shared expert (one SwiGLU FFN every token passes through, weight 1) equals the dense FFN computed
+    another way: the two W4A16 products from linear_w4a16, silu(g) * u, and the down product of the
+    dequantized matrix."""
+    T, H, I_s, group = 5, 256, 128, 128
+    x = synth.activations(("pins", "shared-x"), T, H)
+    qs = [oracle.quantize(synth.weights(("pins", "shared", nm), n, k), group, False)
+          for nm, n, k in (("g", I_s, H), ("u", I_s, H), ("d", H, I_s))]
+    y = oracle.shared_expert(x, H, qs[0], qs[1], qs[2], I_s, group, False)
+    g = oracle.linear_w4a16(x, *qs[0], I_s, H, group, False)
+    u = oracle.linear_w4a16(x, *qs[1], I_s, H, group, False)
+    h = g / (1.0 + np.exp(-g)) * u
+    wd = oracle.dequant(*qs[2], I_s, group, False).astype(np.float64)
+    np.testing.assert_allclose(y, h @ wd.T, rtol=1e-11, atol=1e-12 * np.abs(y).max())
+
+
 # ---------------------------------------------------------------------------------------------- #
 # router and permutation
 # ---------------------------------------------------------------------------------------------- #
