@@ -208,6 +208,26 @@ int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H,
                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_q4_forward_ex -- moe_q4_forward with an optional shared expert.
+ * Source: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" and "高效大语言模型推理实践" MoE architecture
+ * sections (a shared expert that every token passes through, beside the routed ones).
+ *   y[t] = sum_j w[t][j] * o_(t,j) + S(x_t),  S(x) = (SiLU(x . Wg_s^T) * (x . Wu_s^T)) . Wd_s^T,
+ * the shared expert a SwiGLU FFN of intermediate I_shared computed like a routed expert (h in fp16,
+ * fp32 accumulation into the same output sums) with routing weight 1.
+ * shared[3] = {gate, up, down} of one expert: gate and up [I_shared][H], down [H][I_shared], the
+ * same group and symmetry as the routed experts; NULL (with I_shared ignored) = no shared expert.
+ * I_shared % 128 == 0.  Every other argument as moe_q4_forward; the workspace must hold
+ * moe_q4_workspace_size_ex(T, H, I, E, topk, I_shared) bytes.
+ */
+size_t moe_q4_workspace_size_ex(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t I_shared);
+int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H,
+                      const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                      const q4_weight* experts, int32_t I, const q4_weight* shared, int32_t I_shared,
+                      void* y, int32_t out_dtype,
+                      int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                      void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate device memory.
  * No counterpart in the source pages: this is a library convenience, not part of the method.
  *

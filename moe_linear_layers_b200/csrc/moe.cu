@@ -324,6 +324,10 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ a, __nv_bfloat16* _
 struct Workspace {
     uint16_t* xperm;
     __half* h;
+    // shared expert (I_shared > 0): its h, and the one-expert bookkeeping the grouped GEMMs read
+    __half* h_s;
+    int32_t *offsets_s, *tiles_gu_s, *tiles_dn_s, *row_tok_s;
+    float* row_w_s;
     float* y32;
     int32_t *ids, *perm, *offsets, *counts, *hist, *chunk_base, *tiles_gu, *tiles_dn, *row_tok;
     float *wts, *row_w;
@@ -332,7 +336,28 @@ struct Workspace {
 
 inline size_t al(size_t v) { return (v + 255) & ~(size_t)255; }
 
-Workspace carve(void* base, int T, int H, int I, int E, int topk)
+// The shared expert is a one-expert grouped GEMM over every token in order, with routing weight 1.
+__global__ void moe_shared_setup_kernel(int T, int H, int I_s, int32_t* __restrict__ offsets,
+                                        int32_t* __restrict__ tiles_gu, int32_t* __restrict__ tiles_dn,
+                                        int32_t* __restrict__ row_tok, float* __restrict__ row_w)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) {
+        const int mt = (T + tcg::BN - 1) / tcg::BN;
+        offsets[0] = 0;
+        offsets[1] = T;
+        tiles_gu[0] = 0;
+        tiles_gu[1] = mt * (I_s / 64);
+        tiles_dn[0] = 0;
+        tiles_dn[1] = mt * (H / tcg::BM);
+    }
+    if (i < T) {
+        row_tok[i] = i;
+        row_w[i] = 1.0f;
+    }
+}
+
+Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0)
 {
     Workspace w = {};
     const size_t P = (size_t)T * topk;
@@ -354,6 +379,14 @@ Workspace carve(void* base, int T, int H, int I, int E, int topk)
     w.chunk_base = reinterpret_cast<int32_t*>(take(nch * E * 4));
     w.tiles_gu = reinterpret_cast<int32_t*>(take((E + 1) * 4));
     w.tiles_dn = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    if (I_s > 0) {
+        w.h_s = reinterpret_cast<__half*>(take((size_t)T * I_s * 2));
+        w.offsets_s = reinterpret_cast<int32_t*>(take(2 * 4));
+        w.tiles_gu_s = reinterpret_cast<int32_t*>(take(2 * 4));
+        w.tiles_dn_s = reinterpret_cast<int32_t*>(take(2 * 4));
+        w.row_tok_s = reinterpret_cast<int32_t*>(take((size_t)T * 4));
+        w.row_w_s = reinterpret_cast<float*>(take((size_t)T * 4));
+    }
     w.bytes = o;
     return w;
 }
@@ -411,10 +444,34 @@ extern "C" size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t
     return carve(nullptr, T, H, I, E, topk).bytes;
 }
 
+extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                 const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts, int32_t I,
+                                 const q4_weight* shared, int32_t I_shared, void* y, int32_t out_dtype,
+                                 int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets,
+                                 int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                 void* stream);
+
 extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                               int32_t E, int32_t topk, const q4_weight* experts, int32_t I, void* y, int32_t out_dtype,
                               int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
                               void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    return moe_q4_forward_ex(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, y, out_dtype, topk_ids,
+                             topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
+}
+
+extern "C" size_t moe_q4_workspace_size_ex(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t I_shared)
+{
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || topk <= 0 || I_shared < 0) return 0;
+    return carve(nullptr, T, H, I, E, topk, I_shared).bytes;
+}
+
+extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                 const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts, int32_t I,
+                                 const q4_weight* shared, int32_t I_shared, void* y, int32_t out_dtype,
+                                 int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets,
+                                 int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                 void* stream)
 {
     if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
@@ -433,9 +490,25 @@ extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const flo
     }
     if (g.group != 64 && g.group != 128) return Q4_ERR_UNSUPPORTED;
     if (g.n != E * I || g.k != H || u.n != E * I || u.k != H || d.n != E * H || d.k != I) return Q4_ERR_SHAPE;
+    if (shared) {   // the same group and symmetry as the routed experts
+        if (I_shared <= 0) return Q4_ERR_SHAPE;
+        if (I_shared % 128) return Q4_ERR_UNSUPPORTED;
+        for (int i = 0; i < 3; i++) {
+            const q4_weight& w = shared[i];
+            if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
+            if (w.group != g.group || w.symmetric != g.symmetric) return Q4_ERR_UNSUPPORTED;
+            if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
+                return Q4_ERR_ALIGN;
+        }
+        if (shared[0].n != I_shared || shared[0].k != H || shared[1].n != I_shared || shared[1].k != H ||
+            shared[2].n != H || shared[2].k != I_shared)
+            return Q4_ERR_SHAPE;
+    } else {
+        I_shared = 0;
+    }
     if (!q4_aligned16(x) || !q4_aligned16(y) || ((uintptr_t)workspace & 255u) || ((uintptr_t)router_w & 15u))
         return Q4_ERR_ALIGN;
-    Workspace ws = carve(workspace, T, H, I, E, topk);
+    Workspace ws = carve(workspace, T, H, I, E, topk, I_shared);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
     if (T == 0) return Q4_OK;
     if (topk_ids) ws.ids = topk_ids;
@@ -470,6 +543,27 @@ extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const flo
     else rc = g.symmetric ? launch_experts<64, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)
                           : launch_experts<64, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s);
     if (rc) return rc;
+    if (I_shared > 0) {
+        // the shared expert: every token, weight 1, its output added into the same fp32 sums
+        moe_shared_setup_kernel<<<(T + 255) / 256, 256, 0, s>>>(T, H, I_shared, ws.offsets_s, ws.tiles_gu_s,
+                                                                  ws.tiles_dn_s, ws.row_tok_s, ws.row_w_s);
+        if ((rc = q4_launch_status())) return rc;
+        Workspace w1 = ws;
+        w1.xperm = const_cast<uint16_t*>(x);
+        w1.h = ws.h_s;
+        w1.offsets = ws.offsets_s;
+        w1.tiles_gu = ws.tiles_gu_s;
+        w1.tiles_dn = ws.tiles_dn_s;
+        w1.row_tok = ws.row_tok_s;
+        w1.row_w = ws.row_w_s;
+        if (g.group == 128)
+            rc = g.symmetric ? launch_experts<128, true>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s)
+                             : launch_experts<128, false>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s);
+        else
+            rc = g.symmetric ? launch_experts<64, true>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s)
+                             : launch_experts<64, false>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s);
+        if (rc) return rc;
+    }
     if (out_dtype == Q4_OUT_BF16) {
         const int64_t n = (int64_t)T * H;
         f32_to_bf16_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, s>>>(y32, reinterpret_cast<__nv_bfloat16*>(y), n);

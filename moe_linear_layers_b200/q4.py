@@ -34,7 +34,7 @@ Q4_OUT_BF16 = 1
 EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
-            "moe_q4_forward_noalloc")
+            "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -61,6 +61,10 @@ _lib.moe_q4_workspace_size.restype = _sz
 _lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p, _i32,
                                 _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_workspace_size_ex.restype = _sz
+_lib.moe_q4_workspace_size_ex.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
+_lib.moe_q4_forward_ex.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32,
+                                   ctypes.POINTER(q4_weight), _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -220,15 +224,18 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
     return y
 
 
-def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int) -> int:
+def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int, I_shared: int = 0) -> int:
+    if I_shared:
+        return int(_lib.moe_q4_workspace_size_ex(T, H, I, E, topk, I_shared))
     return int(_lib.moe_q4_workspace_size(T, H, I, E, topk))
 
 
 def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
                    experts: tuple, I: int, out_dtype=torch.float32, y: torch.Tensor | None = None,
                    workspace: torch.Tensor | None = None, want_routing: bool = False,
-                   dev_status: torch.Tensor | None = None, stream=None):
-    """Top-k routed MoE SwiGLU layer with INT4 experts.  experts = (gate, up, down) Q4Weight, stacked by expert.
+                   dev_status: torch.Tensor | None = None, stream=None, shared: tuple | None = None):
+    """Top-k routed MoE SwiGLU layer with INT4 experts.  experts = (gate, up, down) Q4Weight, stacked by expert;
+    shared (optional) = (gate, up, down) Q4Weight of a shared expert every token passes through.
     Returns y, or (y, topk_ids, topk_w, perm, offsets, counts) when want_routing."""
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
@@ -238,10 +245,12 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
     od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
-    ws_bytes = moe_q4_workspace_size(T, H, I, E, topk)
+    I_s = shared[0].n if shared is not None else 0
+    ws_bytes = moe_q4_workspace_size(T, H, I, E, topk, I_s)
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
+    sdescs = (q4_weight * 3)(*[e.desc for e in shared]) if shared is not None else None
     ids = wts = perm = offs = cnts = None
     if want_routing:
         ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
@@ -249,9 +258,10 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
         perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
         offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
         cnts = torch.empty((E,), dtype=torch.int32, device=dev)
-    _check(_lib.moe_q4_forward(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, _ptr(y), od,
-                               _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts), _ptr(workspace),
-                               workspace.numel(), _ptr(dev_status), _stream(stream)), "moe_q4_forward")
+    _check(_lib.moe_q4_forward_ex(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, sdescs, I_s,
+                                  _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
+                                  _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
+           "moe_q4_forward")
     if want_routing:
         return y, ids, wts, perm, offs, cnts
     return y

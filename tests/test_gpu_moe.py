@@ -95,3 +95,30 @@ def test_moe_workspace_too_small(q4):
     with pytest.raises(Q4Error) as ei:
         q4.moe_q4_forward(x, Wr, None, topk, ex, I, workspace=ws)
     assert ei.value.status == Q4_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("T,H,I,E,topk,I_s,group,sym", [
+    (64, 256, 128, 8, 2, 256, 128, False),       # shared expert wider than the routed ones
+    (37, 256, 256, 5, 3, 128, 64, True),         # ragged token count, group 64, symmetric
+    (300, 512, 256, 16, 4, 512, 128, False),     # several token tiles for the shared expert
+])
+def test_moe_with_shared_expert(q4, T, H, I, E, topk, I_s, group, sym):
+    tag = f"sh{T}-{E}"
+    x = synth.activations(("moe", tag, "x"), T, H)
+    Wr, bias = synth.router(("moe", tag), E, H, skew=1.1)
+    qs = _experts(tag, E, H, I, group, sym)
+    qsh = [oracle.quantize(synth.weights(("moe", tag, "shared", nm), n, k), group, sym)
+           for nm, n, k in (("gate", I_s, H), ("up", I_s, H), ("down", H, I_s))]
+    logits, ids, w, counts = oracle.route(x, H, Wr, bias, topk)
+    ref = oracle.moe_experts(x, H, ids, w, qs[0], qs[1], qs[2], I, group, sym)
+    ref = ref + oracle.shared_expert(x, H, qsh[0], qsh[1], qsh[2], I_s, group, sym)
+    ex = (upload_weight(q4, *qs[0], E * I, H, group, sym), upload_weight(q4, *qs[1], E * I, H, group, sym),
+          upload_weight(q4, *qs[2], E * H, I, group, sym))
+    sh = (upload_weight(q4, *qsh[0], I_s, H, group, sym), upload_weight(q4, *qsh[1], I_s, H, group, sym),
+          upload_weight(q4, *qsh[2], H, I_s, group, sym))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = q4.moe_q4_forward(cuda_u16_as(x, torch.bfloat16), torch.from_numpy(Wr).cuda(), torch.from_numpy(bias).cuda(),
+                          topk, ex, I, dev_status=st, shared=sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close(y.cpu().numpy(), np.asarray(ref).reshape(T, H), what="moe + shared expert")
