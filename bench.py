@@ -436,6 +436,20 @@ def run_moe(q4, args, dev):
     flops = 2 * T * topk * 3 * H * I
     tf = flops / (ms * 1e-3) / 1e12
     peaks = load_peaks()
+
+    # the same layer with one shared expert of intermediate I (every token, weight 1)
+    sh = []
+    for nm, n, k in (("shared-gate", I, H), ("shared-up", I, H), ("shared-down", H, I)):
+        W = torch.from_numpy(synth.weights((0, "moe", nm), n, k)).to(dev)
+        sh.append(q4.q4_quantize_pack(W, 128, False))
+        del W
+    sh = tuple(sh)
+    ws_s = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk, I), dtype=torch.uint8, device=dev)
+    gs = graph_of(lambda: q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_s, shared=sh))
+    for _ in range(3):
+        gs.replay()
+    ms_s = time_replays(gs, steps, 1) / steps
+    flops_s = flops + 2 * T * 3 * H * I
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "workload": "MoE layer: 4096 tokens, hidden 2048, 64 SwiGLU experts of intermediate 1024, top-8, "
                         "asymmetric INT4 g128, fp32 router with Zipf-skewed logits (bias -1.1 ln(e+1)), fp32 out",
@@ -446,6 +460,10 @@ def run_moe(q4, args, dev):
                          "algorithmic_flop": flops},
             "expert_counts": {"max": int(c.max()), "mean": float(c.mean()), "min": int(c.min()),
                               "empty": int((c == 0).sum())},
+            "with_shared_expert": {"ms_per_step": round(ms_s, 4), "tokens_per_s": round(T / (ms_s * 1e-3), 1),
+                                   "tflops": round(flops_s / (ms_s * 1e-3) / 1e12, 1),
+                                   "workload": "the same layer plus one shared SwiGLU expert of intermediate "
+                                               "1024 (moe_q4_forward_ex)"},
             "gpu_launches": 6 * steps, "clocks": clk.summary()}
 
 
