@@ -143,6 +143,15 @@ int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, int32_t m, 
 int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_t m, const q4_weight* w, void* y,
                            int32_t out_dtype, int32_t* dev_status, void* stream);
 
+/*
+ * q4_selftest_bounded_wait -- exercises the bounded waits the kernels rely on (no counterpart in the
+ * source pages; a test hook for the failure-detection path).  Launches one small kernel whose wait is
+ * never satisfied: which = 0 an mbarrier phase no thread completes, 1 a progress counter no thread
+ * raises (the issuers' weak-load polling).  After limit_us microseconds (1 .. 1000000) the wait gives
+ * up and records Q4_ERR_TIMEOUT in *dev_status (required); the context stays usable.
+ */
+int q4_selftest_bounded_wait(int32_t which, int32_t limit_us, int32_t* dev_status, void* stream);
+
 /* Largest m that q4_linear_w4a16 serves with the GEMV kernel. */
 int q4_linear_w4a16_max_gemv_m(void);
 

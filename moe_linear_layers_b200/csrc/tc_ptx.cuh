@@ -275,7 +275,7 @@ __device__ __forceinline__ void sts_publish(void* p, uint32_t v)
 // few thousand unsuccessful rounds it also watches the wall clock (2 s: Q4_ERR_TIMEOUT, raise the abort
 // flag, return false) and the abort flag.
 __device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uint32_t target, int32_t* status,
-                                                   volatile int* abort_flag)
+                                                   volatile int* abort_flag, uint64_t limit_ns = 2000000000ull)
 {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -283,7 +283,7 @@ __device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uin
         for (int i = 0; i < n; i++) ok &= lds_weak(c + i) >= target;
         if (ok) return true;
         if (abort_flag && *abort_flag) return false;
-        if (globaltimer_ns() - t0 > 2000000000ull) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             q4_set_status(status, Q4_ERR_TIMEOUT);
             if (abort_flag) *abort_flag = 1;
             return false;

@@ -34,7 +34,7 @@ Q4_OUT_BF16 = 1
 EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
-            "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex")
+            "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -61,6 +61,7 @@ _lib.moe_q4_workspace_size.restype = _sz
 _lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p, _i32,
                                 _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.q4_selftest_bounded_wait.argtypes = [_i32, _i32, _p, _p]
 _lib.moe_q4_workspace_size_ex.restype = _sz
 _lib.moe_q4_workspace_size_ex.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward_ex.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32,
@@ -222,6 +223,11 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
     _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
                                _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
     return y
+
+
+def q4_selftest_bounded_wait(which: int, limit_us: int, dev_status: torch.Tensor, stream=None) -> None:
+    """Launch a wait that nothing satisfies; it records Q4_ERR_TIMEOUT in dev_status after limit_us."""
+    _check(_lib.q4_selftest_bounded_wait(which, limit_us, _ptr(dev_status), _stream(stream)), "q4_selftest_bounded_wait")
 
 
 def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int, I_shared: int = 0) -> int:

@@ -242,3 +242,25 @@ def test_w4a16_swiglu_nonfinite_status(q4):
     q4.q4_linear_w4a16_swiglu(gate, up, w, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == q4.Q4_ERR_NONFINITE
+
+
+# ---------------------------------------------------------------------------------------------- #
+# failure detection: a wait that nothing satisfies gives up, records Q4_ERR_TIMEOUT, and the context
+# stays usable (no fault, no hang)
+# ---------------------------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_bounded_wait_times_out_cleanly(q4, which):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.q4_selftest_bounded_wait(which, 2000, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == q4.Q4_ERR_TIMEOUT
+    # the context still works: a small linear afterwards is correct
+    n, k = 64, 256
+    W = synth.weights(("test", "after-timeout"), n, k)
+    pk, sc, zr = oracle.quantize(W, 128, True)
+    w = upload_weight(q4, pk, sc, None, n, k, 128, True)
+    x = synth.activations(("test", "after-timeout-x"), 1, k)
+    y = q4.q4_linear_w4a16(cuda_u16_as(x, torch.bfloat16), w)
+    torch.cuda.synchronize()
+    assert_close(y.cpu().numpy(), oracle.linear_w4a16(x, pk, sc, None, n, k, 128, True), what="after timeout")
