@@ -141,6 +141,18 @@ def act_quant(x_bf16_bits, k: int):
     return q, s
 
 
+def act_quant_f16(x_f16_bits, k: int):
+    """Per-token INT8 quantization of fp16 rows (given as fp16 bit patterns, uint16 [M][k])."""
+    x = _c(x_f16_bits, np.uint16).reshape(-1, k)
+    m = x.shape[0]
+    q = np.empty((m, k), np.int8)
+    s = np.empty((m,), np.float32)
+    rc = lib().orc_act_quant_f16(_p(x), m, k, _p(q), _p(s))
+    if rc != 0:
+        raise OracleError(f"orc_act_quant_f16 returned {rc}")
+    return q, s
+
+
 def linear_w4a8(xq, s_a, packed, scales, n: int, k: int, group: int, rows_m=None, rows_n=None,
                 want_acc: bool = False, zeros=None, symmetric: bool = True):
     xq = _c(xq, np.int8).reshape(-1, k)
@@ -216,4 +228,25 @@ def moe_experts(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int,
         args += [_p(_c(pk, np.uint8)), _p(_c(sc, np.uint16)), _p(_c(zr, np.uint16))]
     lib().orc_moe_experts(_p(x), T, H, _p(ids), _p(w), topk, *args, I, group, int(bool(symmetric)),
                           _p(tk), 0 if tk is None else len(tk), _p(y))
+    return y
+
+
+def moe_experts_a8(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int, symmetric: bool,
+                   a8_mask: int, tokens=None):
+    """The expert FFN with INT8 activations: a8_mask bit 0 = gate/up W4A8 on the token's INT8 codes,
+    bit 1 = down W4A8 on the INT8 codes of h (stored as fp16).  Returns fp64 [n_tok][H]."""
+    x = _c(x_bf16_bits, np.uint16).reshape(-1, H)
+    ids = _c(ids, np.int32)
+    w = _c(w, np.float64)
+    T, topk = ids.shape
+    tk = _c(tokens, np.int32)
+    cnt = T if tk is None else len(tk)
+    y = np.empty((cnt, H), np.float64)
+    args = []
+    for (pk, sc, zr) in (gate, up, down):
+        args += [_p(_c(pk, np.uint8)), _p(_c(sc, np.uint16)), _p(_c(zr, np.uint16))]
+    rc = lib().orc_moe_experts_a8(_p(x), T, H, _p(ids), _p(w), topk, *args, I, group, int(bool(symmetric)),
+                                  int(a8_mask), _p(tk), 0 if tk is None else len(tk), _p(y))
+    if rc != 0:
+        raise OracleError(f"orc_moe_experts_a8 returned {rc}")
     return y

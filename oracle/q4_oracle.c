@@ -254,24 +254,43 @@ void orc_linear_w4a16(const uint16_t* x, int M, int k,
  * amax/127, round half to even, clamp to [-128, 127].  The division is fp32.
  * x: bf16 bits [M][k] -> q int8 [M][k], s fp32 [M].
  * ------------------------------------------------------------------------------------------- */
+/* One token's row, already widened to fp32 (exactly): returns the scale, writes the codes. */
+static float act_quant_row(const float* v, int k, int8_t* q, int* bad)
+{
+    float amax = 0.0f;
+    for (int kk = 0; kk < k; kk++) {
+        if (!isfinite(v[kk])) *bad = 1;
+        if (fabsf(v[kk]) > amax) amax = fabsf(v[kk]);
+    }
+    float sc = amax / 127.0f;
+    for (int kk = 0; kk < k; kk++)
+        q[kk] = sc == 0.0f ? 0 : (int8_t)clampf(rne(v[kk] / sc), -128.0f, 127.0f);
+    return sc;
+}
+
 int orc_act_quant(const uint16_t* x, int M, int k, int8_t* q, float* s)
 {
     int bad = 0;
+    float* v = (float*)malloc(sizeof(float) * (size_t)k);
     for (int mi = 0; mi < M; mi++) {
-        const uint16_t* xr = x + (size_t)mi * k;
-        float amax = 0.0f;
-        for (int kk = 0; kk < k; kk++) {
-            float v = orc_bf16_to_f32(xr[kk]);
-            if (!isfinite(v)) bad = 1;
-            if (fabsf(v) > amax) amax = fabsf(v);
-        }
-        float sc = amax / 127.0f;
-        s[mi] = sc;
-        for (int kk = 0; kk < k; kk++) {
-            float v = orc_bf16_to_f32(xr[kk]);
-            q[(size_t)mi * k + kk] = sc == 0.0f ? 0 : (int8_t)clampf(rne(v / sc), -128.0f, 127.0f);
-        }
+        for (int kk = 0; kk < k; kk++) v[kk] = orc_bf16_to_f32(x[(size_t)mi * k + kk]);
+        s[mi] = act_quant_row(v, k, q + (size_t)mi * k, &bad);
     }
+    free(v);
+    return bad ? ORC_ERR_NONFINITE : ORC_OK;
+}
+
+/* The same quantization of fp16 rows (the MoE's intermediate activations h are stored as fp16):
+ * x: fp16 bits [M][k], widened to fp32 exactly. */
+int orc_act_quant_f16(const uint16_t* x, int M, int k, int8_t* q, float* s)
+{
+    int bad = 0;
+    float* v = (float*)malloc(sizeof(float) * (size_t)k);
+    for (int mi = 0; mi < M; mi++) {
+        for (int kk = 0; kk < k; kk++) v[kk] = orc_f16_to_f32(x[(size_t)mi * k + kk]);
+        s[mi] = act_quant_row(v, k, q + (size_t)mi * k, &bad);
+    }
+    free(v);
     return bad ? ORC_ERR_NONFINITE : ORC_OK;
 }
 
@@ -459,6 +478,110 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
         free(xr);
         free(h);
     }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * MoE expert FFN with INT8 activations.  [W4A8] §3.1 (per-token INT8 activations), §2.3 (INT8 x
+ * INT4-widened-to-INT8 products in INT32, rescaled by scale_w * scale_a), §3.2 (the router stays in
+ * high precision: routing ids and weights come in from orc_route unchanged), §5.1 (the projections
+ * of an FFN can take different precisions: the down projection is the first to go W4A8).
+ * a8_mask bit 0: gate and up run W4A8 on the token's INT8 codes (one quantization of x_t serves every
+ * expert the token visits); bit 1: down runs W4A8 on the INT8 codes of h.  For token t, slot j,
+ * e = ids[t][j]:
+ *   bit 0 set:   xq, sa = act_quant(x_t);
+ *                g_i = sum_g sa * sg[i][g] * sum_{k in g} xq[k] * (qg[i][k] - zg[i][g])   (fp64
+ *                of the exact INT32 partials), u_i likewise with the up matrix;
+ *   bit 0 clear: g, u as in orc_moe_experts (fp64 over the dequantized weights);
+ *   h = g / (1 + exp(-g)) * u (fp64);
+ *   bit 1 set:   h is stored as fp16 (rounded through fp32: h16 = fp16(fp32(h))), then
+ *                hq, sh = act_quant(h16) over the row's I values, and
+ *                o_c = sum_g sh * sd[c][g] * sum_{i in g} hq[i] * (qd[c][i] - zd[c][g]);
+ *   bit 1 clear: o = h . dequant(Wd_e)^T (fp64);
+ *   y_t = sum_j w[t][j] * o (fp64).
+ * Returns ORC_ERR_NONFINITE when a quantized row holds a non-finite value.
+ * ------------------------------------------------------------------------------------------- */
+static double w4a8_dot(const int8_t* aq, double sa, const uint8_t* packed, const uint16_t* scales,
+                       const uint16_t* zeros, int symmetric, int k, int group, int r)
+{
+    int ng = k / group;
+    double sum = 0.0;
+    for (int g = 0; g < ng; g++) {
+        int32_t acc = 0;
+        const int32_t z = (symmetric || !zeros) ? 0 : (int32_t)orc_f16_to_f32(zeros[(size_t)r * ng + g]);
+        for (int kk = g * group; kk < (g + 1) * group; kk++)
+            acc += (int32_t)aq[kk] * ((int32_t)code_at(packed, k, r, kk, symmetric) - z);
+        sum += (double)acc * (double)orc_f16_to_f32(scales[(size_t)r * ng + g]) * sa;
+    }
+    return sum;
+}
+
+int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, const double* w, int topk,
+                       const uint8_t* g_packed, const uint16_t* g_scales, const uint16_t* g_zeros,
+                       const uint8_t* u_packed, const uint16_t* u_scales, const uint16_t* u_zeros,
+                       const uint8_t* d_packed, const uint16_t* d_scales, const uint16_t* d_zeros,
+                       int I, int group, int symmetric, int a8_mask,
+                       const int32_t* tokens, int n_tok, double* y)
+{
+    int cnt = tokens ? n_tok : T;
+    size_t gH = (size_t)(H / group), gI = (size_t)(I / group);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int it = 0; it < cnt; it++) {
+        int t = tokens ? tokens[it] : it;
+        float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+        int8_t* xq = (int8_t*)malloc((size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        float* h16 = (float*)malloc(sizeof(float) * (size_t)I);
+        int8_t* hq = (int8_t*)malloc((size_t)I);
+        double* yr = y + (size_t)it * H;
+        int rb = 0;
+        for (int c = 0; c < H; c++) { xf[c] = orc_bf16_to_f32(x[(size_t)t * H + c]); yr[c] = 0.0; }
+        double sa = (a8_mask & 1) ? (double)act_quant_row(xf, H, xq, &rb) : 0.0;
+        for (int j = 0; j < topk; j++) {
+            int e = ids[(size_t)t * topk + j];
+            const uint8_t* gp = g_packed + (size_t)e * I * (H / 2);
+            const uint8_t* up = u_packed + (size_t)e * I * (H / 2);
+            const uint16_t* gs = g_scales + (size_t)e * I * gH;
+            const uint16_t* us = u_scales + (size_t)e * I * gH;
+            const uint16_t* gz = g_zeros ? g_zeros + (size_t)e * I * gH : NULL;
+            const uint16_t* uz = u_zeros ? u_zeros + (size_t)e * I * gH : NULL;
+            for (int i = 0; i < I; i++) {
+                double gv = 0.0, uv = 0.0;
+                if (a8_mask & 1) {
+                    gv = w4a8_dot(xq, sa, gp, gs, gz, symmetric, H, group, i);
+                    uv = w4a8_dot(xq, sa, up, us, uz, symmetric, H, group, i);
+                } else {
+                    for (int c = 0; c < H; c++) {
+                        gv += (double)xf[c] * (double)deq_at(gp, gs, gz, H, group, symmetric, i, c);
+                        uv += (double)xf[c] * (double)deq_at(up, us, uz, H, group, symmetric, i, c);
+                    }
+                }
+                h[i] = gv / (1.0 + exp(-gv)) * uv;
+            }
+            const uint8_t* dp = d_packed + (size_t)e * H * (I / 2);
+            const uint16_t* ds = d_scales + (size_t)e * H * gI;
+            const uint16_t* dz = d_zeros ? d_zeros + (size_t)e * H * gI : NULL;
+            double wj = w[(size_t)t * topk + j];
+            double sh = 0.0;
+            if (a8_mask & 2) {
+                for (int i = 0; i < I; i++) h16[i] = orc_f16_to_f32(orc_f32_to_f16((float)h[i]));
+                sh = (double)act_quant_row(h16, I, hq, &rb);
+            }
+            for (int c = 0; c < H; c++) {
+                double o = 0.0;
+                if (a8_mask & 2) o = w4a8_dot(hq, sh, dp, ds, dz, symmetric, I, group, c);
+                else for (int i = 0; i < I; i++) o += h[i] * (double)deq_at(dp, ds, dz, I, group, symmetric, c, i);
+                yr[c] += wj * o;
+            }
+        }
+        bad |= rb;
+        free(xf);
+        free(xq);
+        free(h);
+        free(h16);
+        free(hq);
+    }
+    return bad ? ORC_ERR_NONFINITE : ORC_OK;
 }
 
 int orc_version(void) { return 1; }

@@ -476,6 +476,101 @@ def test_moe_all_experts_equal_logits_is_average():
 
 
 # ---------------------------------------------------------------------------------------------- #
+# the expert FFN with INT8 activations (W4A8 page §3.1 per-token codes, §2.3 INT32 partials and the
+# scale_w * scale_a rescale, §5.1 the down projection as the first W4A8 candidate)
+# ---------------------------------------------------------------------------------------------- #
+
+def test_act_quant_f16_hand_worked():
+    """Per-token quantization of fp16 rows, worked by hand from amax/127 and round-half-even:
+    [127, -63.5, 0.5, 2] -> s = 1, codes [127, -64 (tie), 0 (tie), 2];
+    [254, 1 + 2^-10, -3, 0] -> s = 2, codes [127, 1 (0.50049 rounds up), -2 (tie -1.5), 0] -- 1 + 2^-10
+    exists in fp16 but not in bf16, so a wrong widening of the input fails here."""
+    q, s = oracle.act_quant_f16(_f16_bits([[127.0, -63.5, 0.5, 2.0], [254.0, 1.0 + 2.0 ** -10, -3.0, 0.0]]), 4)
+    assert list(s) == [1.0, 2.0]
+    assert q.tolist() == [[127, -64, 0, 2], [127, 1, -2, 0]]
+    z, sz = oracle.act_quant_f16(np.zeros((1, 8), np.uint16), 8)
+    assert sz[0] == 0.0 and not z.any()
+
+
+def test_act_quant_f16_properties():
+    rng = np.random.default_rng(7)
+    h = (rng.standard_normal((32, 1024)) * 3.0).astype(np.float16)
+    q, s = oracle.act_quant_f16(h.view(np.uint16), 1024)
+    hf = h.astype(np.float64)
+    assert np.array_equal(s, (np.abs(hf).max(axis=1).astype(np.float32) / np.float32(127.0)))
+    assert np.all(np.abs(hf - q * s[:, None].astype(np.float64)) <= s[:, None] * (0.5 + 1e-6))
+    assert np.all(np.abs(q).max(axis=1) == 127)
+
+
+def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
+    """The same layer assembled from the separately pinned pieces: act_quant, linear_w4a8 on each
+    expert's row block, linear_w4a16, numpy's fp16 rounding and act_quant_f16."""
+    T, topk = ids.shape
+    xq, sa = oracle.act_quant(x, H)
+    y = np.zeros((T, H))
+
+    def block(q, e, rows):
+        pk, sc, zr = q
+        sl = slice(e * rows, (e + 1) * rows)
+        return pk[sl], sc[sl], (None if zr is None else zr[sl])
+
+    for t in range(T):
+        for j in range(topk):
+            e = ids[t, j]
+            gq, uq, dq = block(stack[0], e, I), block(stack[1], e, I), block(stack[2], e, H)
+            if mask & 1:
+                g = oracle.linear_w4a8(xq[t:t + 1], sa[t:t + 1], gq[0], gq[1], I, H, group, zeros=gq[2], symmetric=sym)[0]
+                u = oracle.linear_w4a8(xq[t:t + 1], sa[t:t + 1], uq[0], uq[1], I, H, group, zeros=uq[2], symmetric=sym)[0]
+            else:
+                g = oracle.linear_w4a16(x[t:t + 1], *gq, I, H, group, sym)[0]
+                u = oracle.linear_w4a16(x[t:t + 1], *uq, I, H, group, sym)[0]
+            h = g / (1.0 + np.exp(-g)) * u
+            if mask & 2:
+                h16 = h.astype(np.float32).astype(np.float16)
+                hq, sh = oracle.act_quant_f16(h16.view(np.uint16)[None, :], I)
+                o = oracle.linear_w4a8(hq, sh, dq[0], dq[1], H, I, group, zeros=dq[2], symmetric=sym)[0]
+            else:
+                o = h @ oracle.dequant(*dq, I, group, sym).astype(np.float64).T
+            y[t] += w[t, j] * o
+    return y
+
+
+@pytest.mark.parametrize("mask", [1, 2, 3])
+@pytest.mark.parametrize("sym,group", [(False, 64), (True, 128)])
+def test_moe_a8_equals_composition(mask, sym, group):
+    T, H, I, E, topk = 5, 256, 128, 3, 2
+    x = synth.activations(("pins", "moe-a8", mask), T, H)
+    Wr, bias = synth.router(("pins", "moe-a8"), E, H)
+    _, ids, w, _ = oracle.route(x, H, Wr, bias, topk)
+    stack = [oracle.quantize(synth.weights(("pins", "moe-a8", nm), n, k), group, sym)
+             for nm, n, k in (("g", E * I, H), ("u", E * I, H), ("d", E * H, I))]
+    y = oracle.moe_experts_a8(x, H, ids, w, stack[0], stack[1], stack[2], I, group, sym, mask)
+    ref = _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+    sub = oracle.moe_experts_a8(x, H, ids, w, stack[0], stack[1], stack[2], I, group, sym, mask,
+                                tokens=np.array([3, 1]))
+    assert np.array_equal(sub, y[[3, 1]])
+
+
+def test_moe_a8_mask0_is_the_w4a16_layer_and_a8_stays_close():
+    """Mask 0 is the W4A16 expert FFN exactly; with INT8 activations the layer moves by the activation
+    quantization error only (per-token steps of amax/127: a few per mille of the output's rms)."""
+    T, H, I, E, topk, group = 6, 256, 128, 4, 2, 128
+    x = synth.activations(("pins", "moe-a8-close"), T, H)
+    Wr, bias = synth.router(("pins", "moe-a8"), E, H)
+    _, ids, w, _ = oracle.route(x, H, Wr, bias, topk)
+    stack = [oracle.quantize(synth.weights(("pins", "moe-a8c", nm), n, k), group, False)
+             for nm, n, k in (("g", E * I, H), ("u", E * I, H), ("d", E * H, I))]
+    y16 = oracle.moe_experts(x, H, ids, w, stack[0], stack[1], stack[2], I, group, False)
+    y0 = oracle.moe_experts_a8(x, H, ids, w, stack[0], stack[1], stack[2], I, group, False, 0)
+    assert np.array_equal(y0, y16)
+    rms = np.sqrt(np.mean(y16 ** 2))
+    for mask in (1, 2, 3):
+        y8 = oracle.moe_experts_a8(x, H, ids, w, stack[0], stack[1], stack[2], I, group, False, mask)
+        assert 0 < np.sqrt(np.mean((y8 - y16) ** 2)) / rms < 0.03
+
+
+# ---------------------------------------------------------------------------------------------- #
 # the generator itself: SplitMix64's published output for state 0
 # ---------------------------------------------------------------------------------------------- #
 
