@@ -450,6 +450,18 @@ def run_moe(q4, args, dev):
         gs.replay()
     ms_s = time_replays(gs, steps, 1) / steps
     flops_s = flops + 2 * T * 3 * H * I
+    # the same layer with the expert projections on per-row INT8 activation codes (moe_q4_forward_a8):
+    # all three projections, and the down projection alone
+    a8 = {}
+    for name, mask in (("w4a8_experts", 3), ("w4a8_down_only", 2)):
+        ws_a = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk, a8_mask=mask), dtype=torch.uint8, device=dev)
+        ga = graph_of(lambda: q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_a, a8_mask=mask))
+        for _ in range(3):
+            ga.replay()
+        ms_a = time_replays(ga, steps, 1) / steps
+        a8[name] = {"ms_per_step": round(ms_a, 4), "tokens_per_s": round(T / (ms_a * 1e-3), 1),
+                    "tops": round(flops / (ms_a * 1e-3) / 1e12, 1), "a8_mask": mask}
+        del ga, ws_a
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "workload": "MoE layer: 4096 tokens, hidden 2048, 64 SwiGLU experts of intermediate 1024, top-8, "
                         "asymmetric INT4 g128, fp32 router with Zipf-skewed logits (bias -1.1 ln(e+1)), fp32 out",
@@ -464,6 +476,10 @@ def run_moe(q4, args, dev):
                                    "tflops": round(flops_s / (ms_s * 1e-3) / 1e12, 1),
                                    "workload": "the same layer plus one shared SwiGLU expert of intermediate "
                                                "1024 (moe_q4_forward_ex)"},
+            "w4a8_experts": dict(a8["w4a8_experts"], workload="the same layer, gate/up and down on per-row INT8 "
+                                 "activation codes, INT32 group partials (moe_q4_forward_a8, mask 3)"),
+            "w4a8_down_only": dict(a8["w4a8_down_only"], workload="the same layer, only the down projection on "
+                                   "INT8 codes of h (moe_q4_forward_a8, mask 2)"),
             "gpu_launches": 6 * steps, "clocks": clk.summary()}
 
 
@@ -571,6 +587,14 @@ def ncu_case(case):
         torch.cuda.synchronize()
         for _ in range(2):
             q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_t)
+    elif case == "moe-a8":
+        T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+        x, Wr, bias, ex = build_moe(q4, dev)
+        ws_t = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk, a8_mask=3), dtype=torch.uint8, device=dev)
+        y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_t, a8_mask=3)
     torch.cuda.synchronize()
     print(f"ncu case {case}: done", flush=True)
 
@@ -583,7 +607,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode-layer", "gemm", "moe"],
+    ap.add_argument("--ncu-case", choices=["decode-layer", "gemm", "moe", "moe-a8"],
                     help="run a small fixed launch sequence for an ncu capture and exit (no JSON line)")
     args = ap.parse_args()
     if args.ncu_case:

@@ -167,6 +167,14 @@ int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, flo
                         int32_t* dev_status, void* stream);
 
 /*
+ * act_quant_per_token_f16 -- act_quant_per_token for fp16 rows (the same arithmetic on values widened
+ * exactly from fp16).  The MoE layer's intermediate activations h are fp16; this quantizes them for a
+ * W4A8 down projection.  x [m][k] fp16 bits; everything else as act_quant_per_token.
+ */
+int act_quant_per_token_f16(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                            int32_t* dev_status, void* stream);
+
+/*
  * q4_linear_w4a8 -- INT8 activations x INT4 weights widened to INT8, INT32 accumulation, rescale.
  * Source: the W4A8 page §2.3 (three steps and the pseudo-code: dequant_int4_to_int8, int8 matmul
  * into int32, rescale by scale_w * scale_a).  With one weight scale per group of 128 (or 64) the
@@ -232,6 +240,30 @@ size_t moe_q4_workspace_size_ex(int32_t T, int32_t H, int32_t I, int32_t E, int3
 int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H,
                       const float* router_w, const float* router_bias, int32_t E, int32_t topk,
                       const q4_weight* experts, int32_t I, const q4_weight* shared, int32_t I_shared,
+                      void* y, int32_t out_dtype,
+                      int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                      void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * moe_q4_forward_a8 -- moe_q4_forward with the expert projections on INT8 activation codes (W4A8).
+ * Source: the W4A8 page §3.1 (per-token INT8 activations: scale = amax/127, round half to even),
+ * §2.3 (INT4 codes widened to INT8, INT8 x INT8 products in INT32, rescale by scale_w * scale_a),
+ * §3.2 (the router is not quantized: routing is exactly moe_q4_forward's) and §5.1 (the projections
+ * of an FFN take their own precision; the down projection is the first candidate for W4A8).
+ *   a8_mask bit 0 (gate/up): xq_t, sa_t = act_quant(x_t) once per token;
+ *                g_i = sa_t * sum_g sg[i][g] * P_g, P_g = sum_{k in g} xq_t[k] * (code_g[i][k] - zero_g[i][g])
+ *                (exact INT32 partials, fp32 rescale), u likewise;
+ *   a8_mask bit 1 (down): h (fp16, as stored) -> hq, sh = act_quant(h) per permuted row (I values), and
+ *                o_c = sh * sum_g sd[c][g] * sum_{i in g} hq[i] * (code_d[c][i] - zero_d[c][g]);
+ *   a clear bit keeps that projection W4A16 as in moe_q4_forward.  a8_mask in 0..3 (0 = moe_q4_forward).
+ * Arguments as moe_q4_forward; the workspace must hold moe_q4_workspace_size_a8(T, H, I, E, topk,
+ * a8_mask) bytes.  dev_status also receives Q4_ERR_NONFINITE when a quantized row (x, or h after an
+ * fp16 overflow) holds a non-finite value.
+ */
+size_t moe_q4_workspace_size_a8(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t a8_mask);
+int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H,
+                      const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                      const q4_weight* experts, int32_t I, int32_t a8_mask,
                       void* y, int32_t out_dtype,
                       int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);

@@ -2,7 +2,8 @@
 //
 // Source: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" §3.1: per-token amax, scale = amax/127,
 // round half to even, clamp to [-128, 127].  The division by the scale is IEEE fp32; a token whose
-// amax is 0 gets scale 0 and all-zero codes.
+// amax is 0 gets scale 0 and all-zero codes.  Inputs are bf16 (the layer inputs) or fp16 (the MoE's
+// intermediate activations h); both widen to fp32 exactly.
 //
 // HBM-bound (2 B read + 1 B written per element): one CTA per token, the row held in registers between
 // the max pass and the coding pass (one read of x), 16-byte loads and 8-byte stores.  The quotient
@@ -29,36 +30,52 @@ __device__ __forceinline__ int code8(float x, float s, float r, bool exact_div)
     return (int)fminf(fmaxf(rintf(q), -128.0f), 127.0f);
 }
 
-// codes of one 16-byte word (8 bf16 values) as 8 bytes
+// low / high 16-bit value of a word as fp32
+template <bool F16> __device__ __forceinline__ float lo16(uint32_t w)
+{
+    if constexpr (F16) return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+    return __uint_as_float(w << 16);
+}
+template <bool F16> __device__ __forceinline__ float hi16(uint32_t w)
+{
+    if constexpr (F16) return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    return __uint_as_float(w & 0xFFFF0000u);
+}
+
+// codes of one 16-byte word (8 values) as 8 bytes
+template <bool F16>
 __device__ __forceinline__ uint2 code_word(const uint4& v, float s, float r, bool exact_div)
 {
     const uint32_t e[4] = {v.x, v.y, v.z, v.w};
     uint32_t packed[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        const int qa = code8(__uint_as_float(e[j] << 16), s, r, exact_div);
-        const int qb = code8(__uint_as_float(e[j] & 0xFFFF0000u), s, r, exact_div);
+        const int qa = code8(lo16<F16>(e[j]), s, r, exact_div);
+        const int qb = code8(hi16<F16>(e[j]), s, r, exact_div);
         packed[j / 2] |= ((uint32_t)(qa & 0xFF) | ((uint32_t)(qb & 0xFF) << 8)) << (16 * (j & 1));
     }
     return make_uint2(packed[0], packed[1]);
 }
 
-// per-halfword max of bf16 magnitudes (integer order = magnitude order for non-NaN) and a flag for an
-// all-ones exponent (inf or NaN) anywhere in the word
+// per-halfword max of bf16 / fp16 magnitudes (for both formats the integer order of the magnitude bits
+// is the order of the values, NaN aside) and a flag for an all-ones exponent (inf or NaN) in the word
+template <bool F16>
 __device__ __forceinline__ uint32_t word_amax(const uint4& v, uint32_t& bad)
 {
+    constexpr uint32_t expo = F16 ? 0x7C007C00u : 0x7F807F80u;     // exponent field of both halves
+    constexpr uint32_t one = F16 ? 0x04000400u : 0x00800080u;      // its lowest bit
     const uint32_t e[4] = {v.x, v.y, v.z, v.w};
     uint32_t a = 0;
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         a = __vmaxu2(a, e[j] & 0x7FFF7FFFu);
-        bad |= ((e[j] & 0x7F807F80u) + 0x00800080u) & 0x80008000u;
+        bad |= ((e[j] & expo) + one) & 0x80008000u;
     }
     return a;
 }
 
 // W = 16-byte words per thread kept in registers (k <= 8 * kThreads * W); W = 0: any k, two passes.
-template <int W>
+template <int W, bool F16>
 __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __restrict__ x, int k,
                                                              int8_t* __restrict__ xq, float* __restrict__ scale_a,
                                                              int32_t* status)
@@ -77,9 +94,9 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
             v[i] = w < n8 ? __ldg(xr + w) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int i = 0; i < W; i++) a = __vmaxu2(a, word_amax(v[i], bad));
+        for (int i = 0; i < W; i++) a = __vmaxu2(a, word_amax<F16>(v[i], bad));
     } else {
-        for (int w = threadIdx.x; w < n8; w += kThreads) a = __vmaxu2(a, word_amax(__ldg(xr + w), bad));
+        for (int w = threadIdx.x; w < n8; w += kThreads) a = __vmaxu2(a, word_amax<F16>(__ldg(xr + w), bad));
     }
     if (bad) q4_set_status(status, Q4_ERR_NONFINITE);
     a = max(a & 0xFFFFu, a >> 16);
@@ -90,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
     uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < kThreads / 32; i++) mb = max(mb, red[i]);
-    const float m = __uint_as_float(mb << 16);
+    const float m = F16 ? __half2float(__ushort_as_half((unsigned short)mb)) : __uint_as_float(mb << 16);
     const float s = m / 127.0f;
     if (threadIdx.x == 0) scale_a[row] = s;
     const bool exact_div = !(s >= 0x1p-100f);           // tiny (or zero / NaN) scale: divide directly
@@ -99,29 +116,48 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
 #pragma unroll
         for (int i = 0; i < W; i++) {
             const int w = i * kThreads + threadIdx.x;
-            if (w < n8) out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word(v[i], s, r, exact_div);
+            if (w < n8) out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word<F16>(v[i], s, r, exact_div);
         }
     } else {
         for (int w = threadIdx.x; w < n8; w += kThreads)
-            out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word(__ldg(xr + w), s, r, exact_div);
+            out[w] = s == 0.0f ? make_uint2(0u, 0u) : code_word<F16>(__ldg(xr + w), s, r, exact_div);
     }
 }
 
-}  // namespace
-
-extern "C" int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
-                                   int32_t* dev_status, void* stream)
+template <bool F16>
+int act_quant_launch(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a, int32_t* dev_status,
+                     cudaStream_t s)
 {
     if (!x || !xq || !scale_a) return Q4_ERR_NULL;
     if (m < 0 || k <= 0 || k % 8) return Q4_ERR_SHAPE;
     if (!q4_aligned16(x) || !q4_aligned16(xq) || ((uintptr_t)scale_a & 3u)) return Q4_ERR_ALIGN;
     if (m == 0) return Q4_OK;
     const int n8 = k / 8;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (n8 <= kThreads) act_quant_kernel<1><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 2 * kThreads) act_quant_kernel<2><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 4 * kThreads) act_quant_kernel<4><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 8 * kThreads) act_quant_kernel<8><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else act_quant_kernel<0><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    if (n8 <= kThreads) act_quant_kernel<1, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 2 * kThreads) act_quant_kernel<2, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 4 * kThreads) act_quant_kernel<4, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else if (n8 <= 8 * kThreads) act_quant_kernel<8, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
+    else act_quant_kernel<0, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
     return q4_launch_status();
+}
+
+}  // namespace
+
+int q4_act_quant_rows(const uint16_t* x, bool f16, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                      int32_t* dev_status, cudaStream_t s)
+{
+    return f16 ? act_quant_launch<true>(x, m, k, xq, scale_a, dev_status, s)
+               : act_quant_launch<false>(x, m, k, xq, scale_a, dev_status, s);
+}
+
+extern "C" int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                                   int32_t* dev_status, void* stream)
+{
+    return act_quant_launch<false>(x, m, k, xq, scale_a, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" int act_quant_per_token_f16(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                                       int32_t* dev_status, void* stream)
+{
+    return act_quant_launch<true>(x, m, k, xq, scale_a, dev_status, (cudaStream_t)stream);
 }

@@ -270,13 +270,17 @@ __global__ void __launch_bounds__(kScanThreads) moe_scan_kernel(const int32_t* _
 }
 
 // ---------------------------------------------------------------------------------------------- //
-// 3. scatter + gather (one CTA per chunk of 16 tokens)
+// 3. scatter + gather (one CTA per chunk of 16 tokens).  Rows are row_bytes long (bf16 activations,
+//    or their int8 codes, whose per-token scales tok_scale then follow them into row_scale).
 // ---------------------------------------------------------------------------------------------- //
-__global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __restrict__ x, int T, int H, int E, int topk,
-                                                          const int32_t* __restrict__ ids, const float* __restrict__ wts,
+__global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restrict__ x, int T, int row_bytes, int E,
+                                                          int topk, const int32_t* __restrict__ ids,
+                                                          const float* __restrict__ wts,
                                                           const int32_t* __restrict__ chunk_base,
                                                           int32_t* __restrict__ perm, int32_t* __restrict__ row_tok,
-                                                          float* __restrict__ row_w, uint16_t* __restrict__ xperm)
+                                                          float* __restrict__ row_w, uint8_t* __restrict__ xperm,
+                                                          const float* __restrict__ tok_scale,
+                                                          float* __restrict__ row_scale)
 {
     __shared__ int pos[kRouteTok * kMaxTopk];
     __shared__ int cid[kRouteTok * kMaxTopk];   // the chunk's expert ids, token-major
@@ -295,14 +299,15 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint16_t* __rest
         perm[p] = (t0 + tl) * topk + j;
         row_tok[p] = t0 + tl;
         row_w[p] = wts[(int64_t)(t0 + tl) * topk + j];
+        if (tok_scale) row_scale[p] = tok_scale[t0 + tl];
     }
     __syncthreads();
     // gather: a warp copies whole rows, eight 16-byte loads in flight per lane before the stores
-    const int vec = H / 8;  // 16-byte units per row
+    const int vec = row_bytes / 16;  // 16-byte units per row
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nwarps = blockDim.x / 32;
     for (int q = warp; q < npairs; q += nwarps) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + q / topk) * H);
-        uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * H);
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + q / topk) * row_bytes);
+        uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * row_bytes);
         int u = lane;
         for (; u + 7 * 32 < vec; u += 8 * 32) {
             uint4 r[8];
@@ -322,7 +327,7 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ a, __nv_bfloat16* _
 }
 
 struct Workspace {
-    uint16_t* xperm;
+    uint16_t* xperm;          // permuted activations: bf16 rows, or int8 codes (W4A8 gate/up)
     __half* h;
     // shared expert (I_shared > 0): its h, and the one-expert bookkeeping the grouped GEMMs read
     __half* h_s;
@@ -331,6 +336,10 @@ struct Workspace {
     float* y32;
     int32_t *ids, *perm, *offsets, *counts, *hist, *chunk_base, *tiles_gu, *tiles_dn, *row_tok;
     float *wts, *row_w;
+    // INT8 activations (W4A8 expert GEMMs): the tokens' codes and scales, the permuted rows' scales,
+    // and the codes and scales of h
+    int8_t *xq_tok, *hq;
+    float *sa_tok, *sa_row, *sh_row;
     size_t bytes;
 };
 
@@ -357,7 +366,7 @@ __global__ void moe_shared_setup_kernel(int T, int H, int I_s, int32_t* __restri
     }
 }
 
-Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0)
+Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0, int a8_mask = 0)
 {
     Workspace w = {};
     const size_t P = (size_t)T * topk;
@@ -387,38 +396,61 @@ Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0)
         w.row_tok_s = reinterpret_cast<int32_t*>(take((size_t)T * 4));
         w.row_w_s = reinterpret_cast<float*>(take((size_t)T * 4));
     }
+    if (a8_mask & 1) {
+        w.xq_tok = reinterpret_cast<int8_t*>(take((size_t)T * H));
+        w.sa_tok = reinterpret_cast<float*>(take((size_t)T * 4));
+        w.sa_row = reinterpret_cast<float*>(take(P * 4));
+    }
+    if (a8_mask & 2) {
+        w.hq = reinterpret_cast<int8_t*>(take(P * I));
+        w.sh_row = reinterpret_cast<float*>(take(P * 4));
+    }
     w.bytes = o;
     return w;
 }
 
 template <int G, bool SYM>
 int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I, int E, int topk, float* y32,
-                   int32_t* status, cudaStream_t s)
+                   int32_t* status, cudaStream_t s, int a8_mask = 0)
 {
     using namespace tcg;
     const int P = T * topk;
     const int sms = q4_num_sms();
-    CUtensorMap mx, mg, mu, mh, md;
-    if (!make_act_map(&mx, ws.xperm, H, P, 2, false) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
-        !make_packed_map(&mu, ex[1].packed, H, (uint64_t)E * I, 64) || !make_act_map(&mh, ws.h, I, P, 2, true) ||
-        !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
-        return Q4_ERR_CUDA;
-    Args a = {};
-    a.M = P;
-    a.N = I;
-    a.K = H;
-    a.scales_a = reinterpret_cast<const __half*>(ex[0].scales);
-    a.zeros_a = reinterpret_cast<const __half*>(ex[0].zeros);
-    a.scales_b = reinterpret_cast<const __half*>(ex[1].scales);
-    a.zeros_b = reinterpret_cast<const __half*>(ex[1].zeros);
-    a.status = status;
-    a.expert_tiles = ws.tiles_gu;
-    a.offsets = ws.offsets;
-    a.h = ws.h;
-    a.E = E;
-    a.topk = topk;
-    int rc = launch<false, G, SYM, Mode::GateUp>(mx, mg, mu, a, sms, s);
+    int rc;
+    if (a8_mask & 1) {   // gate/up on the permuted rows' int8 codes
+        rc = q4_moe_gateup_a8(reinterpret_cast<const int8_t*>(ws.xperm), ws.sa_row, &ex[0], &ex[1], P, H, I, E,
+                              ws.offsets, ws.tiles_gu, ws.h, status, s);
+    } else {
+        CUtensorMap mx, mg, mu;
+        if (!make_act_map(&mx, ws.xperm, H, P, 2, false) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
+            !make_packed_map(&mu, ex[1].packed, H, (uint64_t)E * I, 64))
+            return Q4_ERR_CUDA;
+        Args a = {};
+        a.M = P;
+        a.N = I;
+        a.K = H;
+        a.scales_a = reinterpret_cast<const __half*>(ex[0].scales);
+        a.zeros_a = reinterpret_cast<const __half*>(ex[0].zeros);
+        a.scales_b = reinterpret_cast<const __half*>(ex[1].scales);
+        a.zeros_b = reinterpret_cast<const __half*>(ex[1].zeros);
+        a.status = status;
+        a.expert_tiles = ws.tiles_gu;
+        a.offsets = ws.offsets;
+        a.h = ws.h;
+        a.E = E;
+        a.topk = topk;
+        rc = launch<false, G, SYM, Mode::GateUp>(mx, mg, mu, a, sms, s);
+    }
     if (rc) return rc;
+    if (a8_mask & 2) {   // h -> per-row int8 codes, then down on them
+        if ((rc = q4_act_quant_rows(reinterpret_cast<const uint16_t*>(ws.h), true, P, I, ws.hq, ws.sh_row, status, s)))
+            return rc;
+        return q4_moe_down_a8(ws.hq, ws.sh_row, &ex[2], P, H, I, E, ws.offsets, ws.tiles_dn, ws.row_tok, ws.row_w,
+                              y32, status, s);
+    }
+    CUtensorMap mh, md;
+    if (!make_act_map(&mh, ws.h, I, P, 2, true) || !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
+        return Q4_ERR_CUDA;
     Args d = {};
     d.M = P;
     d.N = H;
@@ -444,20 +476,19 @@ extern "C" size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t
     return carve(nullptr, T, H, I, E, topk).bytes;
 }
 
-extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
-                                 const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts, int32_t I,
-                                 const q4_weight* shared, int32_t I_shared, void* y, int32_t out_dtype,
-                                 int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets,
-                                 int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                                 void* stream);
+static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
+                        int32_t E, int32_t topk, const q4_weight* experts, int32_t I, const q4_weight* shared,
+                        int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
+                        int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                               int32_t E, int32_t topk, const q4_weight* experts, int32_t I, void* y, int32_t out_dtype,
                               int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
                               void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
-    return moe_q4_forward_ex(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, y, out_dtype, topk_ids,
-                             topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
+    return forward_impl(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, 0, y, out_dtype, topk_ids,
+                        topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
 }
 
 extern "C" size_t moe_q4_workspace_size_ex(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t I_shared)
@@ -466,12 +497,39 @@ extern "C" size_t moe_q4_workspace_size_ex(int32_t T, int32_t H, int32_t I, int3
     return carve(nullptr, T, H, I, E, topk, I_shared).bytes;
 }
 
+extern "C" size_t moe_q4_workspace_size_a8(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t a8_mask)
+{
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || topk <= 0 || a8_mask < 0 || a8_mask > 3) return 0;
+    return carve(nullptr, T, H, I, E, topk, 0, a8_mask).bytes;
+}
+
 extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
                                  const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts, int32_t I,
                                  const q4_weight* shared, int32_t I_shared, void* y, int32_t out_dtype,
                                  int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets,
                                  int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                                  void* stream)
+{
+    return forward_impl(x, T, H, router_w, router_bias, E, topk, experts, I, shared, I_shared, 0, y, out_dtype,
+                        topk_ids, topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
+}
+
+extern "C" int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                 const float* router_bias, int32_t E, int32_t topk, const q4_weight* experts, int32_t I,
+                                 int32_t a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
+                                 int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (a8_mask < 0 || a8_mask > 3) return Q4_ERR_UNSUPPORTED;
+    return forward_impl(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, a8_mask, y, out_dtype,
+                        topk_ids, topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
+}
+
+static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
+                        int32_t E, int32_t topk, const q4_weight* experts, int32_t I, const q4_weight* shared,
+                        int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
+                        int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
     if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
@@ -508,7 +566,7 @@ extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const 
     }
     if (!q4_aligned16(x) || !q4_aligned16(y) || ((uintptr_t)workspace & 255u) || ((uintptr_t)router_w & 15u))
         return Q4_ERR_ALIGN;
-    Workspace ws = carve(workspace, T, H, I, E, topk, I_shared);
+    Workspace ws = carve(workspace, T, H, I, E, topk, I_shared, a8_mask);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
     if (T == 0) return Q4_OK;
     if (topk_ids) ws.ids = topk_ids;
@@ -533,15 +591,28 @@ extern "C" int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H, const 
                                                             ws.hist, dev_status);
     moe_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
                                                    ws.tiles_gu, ws.tiles_dn);
-    moe_scatter_kernel<<<nch, 256, 0, s>>>(x, T, H, E, topk, ws.ids, ws.wts, ws.chunk_base, ws.perm, ws.row_tok,
-                                           ws.row_w, ws.xperm);
+    int rc;
+    if (a8_mask & 1) {
+        // one per-token quantization of x serves every expert the token visits; the codes and their
+        // scales are permuted together
+        if ((rc = q4_act_quant_rows(x, false, T, H, ws.xq_tok, ws.sa_tok, dev_status, s))) return rc;
+        moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(ws.xq_tok), T, H, E, topk, ws.ids,
+                                               ws.wts, ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
+                                               reinterpret_cast<uint8_t*>(ws.xperm), ws.sa_tok, ws.sa_row);
+    } else {
+        moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x), T, 2 * H, E, topk, ws.ids,
+                                               ws.wts, ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
+                                               reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr);
+    }
     if (const cudaError_t e = cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s)) return q4_cuda_status(e);
-    int rc = q4_launch_status();
+    rc = q4_launch_status();
     if (rc) return rc;
-    if (g.group == 128) rc = g.symmetric ? launch_experts<128, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)
-                                         : launch_experts<128, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s);
-    else rc = g.symmetric ? launch_experts<64, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s)
-                          : launch_experts<64, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s);
+    if (g.group == 128)
+        rc = g.symmetric ? launch_experts<128, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask)
+                         : launch_experts<128, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask);
+    else
+        rc = g.symmetric ? launch_experts<64, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask)
+                         : launch_experts<64, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask);
     if (rc) return rc;
     if (I_shared > 0) {
         // the shared expert: every token, weight 1, its output added into the same fp32 sums

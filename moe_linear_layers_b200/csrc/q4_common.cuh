@@ -62,6 +62,21 @@ static inline int q4_launch_status() { return q4_cuda_status(cudaGetLastError())
 
 static inline bool q4_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Per-token INT8 quantization of bf16 (f16 = false) or fp16 rows, the kernel behind act_quant_per_token
+// and act_quant_per_token_f16 (act_quant.cu); same arguments and return codes.
+int q4_act_quant_rows(const uint16_t* x, bool f16, int32_t m, int32_t k, int8_t* xq, float* scale_a,
+                      int32_t* dev_status, cudaStream_t s);
+
+// The MoE layer's grouped expert GEMMs on int8 activation codes (moe_a8.cu): gate/up with the SwiGLU
+// epilogue into h (fp16), and down with the weighted reduction into y32.  P permuted rows; offsets and
+// tiles as the 16-bit grouped GEMMs take them; sa / sh the per-permuted-row activation scales.
+int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H,
+                     int I, int E, const int32_t* offsets, const int32_t* tiles, __half* h, int32_t* status,
+                     cudaStream_t s);
+int q4_moe_down_a8(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E,
+                   const int32_t* offsets, const int32_t* tiles, const int32_t* row_tok, const float* row_w,
+                   float* y32, int32_t* status, cudaStream_t s);
+
 // Number of SMs of the current device (cached per device).
 static inline int q4_num_sms()
 {

@@ -23,9 +23,11 @@
 //   Dense   y[m][n] = sum_g s[n][g] * D_g (W4A16, bf16 MMA) or y = s_a[m] * sum_g s[n][g] * D_g / 16
 //           (W4A8, int8 MMA on 16*code).
 //   GateUp  A rows 0-63 = gate rows i0..i0+63 of expert e, rows 64-127 = the same rows of up; B = the
-//           expert's rows of the permuted activations; epilogue h = SiLU(gate) * up -> fp16.
-//   Down    A = 128 rows of the expert's down projection (fp16 codes), B = h (fp16); epilogue
-//           y[token][n] += w[token][slot] * out (fp32 reduction into the output).
+//           expert's rows of the permuted activations (bf16, or int8 codes with per-row scales s_a);
+//           epilogue h = SiLU(gate) * up -> fp16 (gate and up each times s_a first with int8 codes).
+//   Down    A = 128 rows of the expert's down projection (fp16 codes, or int8), B = h (fp16, or its
+//           int8 codes and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
+//           (fp32 reduction into the output).
 //
 // Warp roles (640 threads = 5 warpgroups, launched at 96 registers and re-partitioned with setmaxnreg):
 //   warps 0-3    MMA issuers, one thread each, stage it issued by warp it % 4 (warp 1 also owns TMEM);
@@ -92,7 +94,7 @@ template <bool INT8, Mode MODE, bool PRING> struct Cfg {
     static constexpr int PARAMS = PRING ? 2 * PSLOT * PTENS : 0;
     // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
     // in flight to cover the latency of the activation copies
-    static constexpr int NS = INT8 ? 8 : (MODE == Mode::GateUp ? 4 : 5);
+    static constexpr int NS = INT8 ? (MODE == Mode::GateUp ? 7 : 8) : (MODE == Mode::GateUp ? 4 : 5);
     static_assert(NS <= kMaxStages, "ring depth");
     static_assert(NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144 <= 227 * 1024, "shared memory");
     static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144;
@@ -105,7 +107,7 @@ struct Args {
     const __half* zeros_a;
     const __half* scales_b;   // GateUp: up
     const __half* zeros_b;
-    const float* scale_a;     // W4A8 per-token scales
+    const float* scale_a;     // W4A8 per-activation-row scales (Dense: token; GateUp / Down: permuted row)
     void* y;                  // Dense: [M][N]; Down: fp32 [T][N] (reduction target)
     int32_t* acc_dbg;         // W4A8 debug partials (nullable)
     int32_t* status;
@@ -627,7 +629,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const int m = T.m0 + half * 64 + j;
                     const bool ok = m < T.m_end;
                     comb_tok[ew * 64 + j] = ok ? p.row_tok[m] : 0;
-                    comb_w[ew * 64 + j] = ok ? p.row_w[m] : 0.0f;
+                    float cw = ok ? p.row_w[m] : 0.0f;
+                    if constexpr (INT8) cw = ok ? cw * p.scale_a[m] : 0.0f;   // the row's activation scale
+                    comb_w[ew * 64 + j] = cw;
                 }
             }
             for (int gl = 0; gl < ngroups; gl++) {
@@ -656,7 +660,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tc::tmem_ld32(tbase + lane_field + db * BN + half * 64 + 32 * h, v);
                     tc::tmem_wait_ld();
                     if constexpr (INT8) {
-                        if (p.acc_dbg && srow) {
+                        if (MODE == Mode::Dense && p.acc_dbg && srow) {
 #pragma unroll
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
@@ -749,7 +753,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const int rows = min(64, T.m_end - mb);
                     __half* hb = p.h + (int64_t)mb * p.N + i;
                     auto swiglu = [&](int j) {
-                        const float gv = accv(j), uv = xb[j * 64 + r];
+                        float gv = accv(j), uv = xb[j * 64 + r];
+                        if constexpr (INT8) {   // the row's activation scale
+                            const float sa = __ldg(p.scale_a + mb + j);
+                            gv *= sa;
+                            uv *= sa;
+                        }
                         return __float2half_rn(gv * __frcp_rn(1.0f + __expf(-gv)) * uv);
                     };
                     if (rows == 64) {

@@ -69,6 +69,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// True once more than limit_ns of wall time separates now from t0 AND at least min_rounds polls were
+// made.  The difference is taken signed, so a global timer stepped back while a wait runs (the timer is
+// kept in step with the host clock) cannot make a fresh wait look expired through unsigned wrap-around,
+// and the poll count keeps a forward step from ending a wait that has barely started.
+__device__ __forceinline__ bool wait_expired(uint64_t t0, uint64_t limit_ns, uint32_t rounds, uint32_t min_rounds)
+{
+    return rounds >= min_rounds && (int64_t)(globaltimer_ns() - t0) > (int64_t)limit_ns;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after `limit_ns` of wall time:
 // records Q4_ERR_TIMEOUT in the status word, raises the CTA's abort flag (nullable) and returns false.
 __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int32_t* status,
@@ -79,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, i
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u) {
             if (abort_flag && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
+            if (wait_expired(t0, limit_ns, i >> 8, 64)) {
                 q4_set_status(status, Q4_ERR_TIMEOUT);
                 if (abort_flag) *abort_flag = 1;
                 return false;
@@ -278,12 +287,12 @@ __device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uin
                                                    volatile int* abort_flag, uint64_t limit_ns = 2000000000ull)
 {
     const uint64_t t0 = globaltimer_ns();
-    for (;;) {
+    for (uint32_t round = 0;; round++) {
         bool ok = true;
         for (int i = 0; i < n; i++) ok &= lds_weak(c + i) >= target;
         if (ok) return true;
         if (abort_flag && *abort_flag) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
+        if (wait_expired(t0, limit_ns, round, 1u << 16)) {
             q4_set_status(status, Q4_ERR_TIMEOUT);
             if (abort_flag) *abort_flag = 1;
             return false;

@@ -34,7 +34,8 @@ Q4_OUT_BF16 = 1
 EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
-            "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait")
+            "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
+            "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -56,6 +57,7 @@ _lib.q4_linear_w4a16_swiglu.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight),
 _lib.q4_linear_w4a16_grouped.argtypes = [_i32, ctypes.POINTER(_p), _i32, ctypes.POINTER(q4_weight),
                                          ctypes.POINTER(_p), _i32, _p, _p]
 _lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
+_lib.act_quant_per_token_f16.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
 _lib.q4_linear_w4a8.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _p]
 _lib.moe_q4_workspace_size.restype = _sz
 _lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
@@ -66,6 +68,10 @@ _lib.moe_q4_workspace_size_ex.restype = _sz
 _lib.moe_q4_workspace_size_ex.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward_ex.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32,
                                    ctypes.POINTER(q4_weight), _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_workspace_size_a8.restype = _sz
+_lib.moe_q4_workspace_size_a8.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
+_lib.moe_q4_forward_a8.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _i32,
+                                   _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -200,13 +206,15 @@ def q4_linear_w4a16_max_gemv_m() -> int:
 
 def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a: torch.Tensor | None = None,
                         dev_status: torch.Tensor | None = None, stream=None):
-    """Per-token INT8 quantization of a bf16 [m][k] CUDA tensor -> (xq int8 [m][k], scale_a fp32 [m])."""
-    _dev(x, torch.bfloat16, "x")
+    """Per-token INT8 quantization of a bf16 (or fp16) [m][k] CUDA tensor -> (xq int8 [m][k], scale_a fp32 [m])."""
+    f16 = isinstance(x, torch.Tensor) and x.dtype == torch.float16
+    _dev(x, torch.float16 if f16 else torch.bfloat16, "x")
     m, k = x.shape
     xq = torch.empty((m, k), dtype=torch.int8, device=x.device) if xq is None else xq
     scale_a = torch.empty((m,), dtype=torch.float32, device=x.device) if scale_a is None else scale_a
-    _check(_lib.act_quant_per_token(_ptr(x), m, k, _ptr(xq), _ptr(scale_a), _ptr(dev_status), _stream(stream)),
-           "act_quant_per_token")
+    fn = _lib.act_quant_per_token_f16 if f16 else _lib.act_quant_per_token
+    _check(fn(_ptr(x), m, k, _ptr(xq), _ptr(scale_a), _ptr(dev_status), _stream(stream)),
+           "act_quant_per_token_f16" if f16 else "act_quant_per_token")
     return xq, scale_a
 
 
@@ -230,7 +238,11 @@ def q4_selftest_bounded_wait(which: int, limit_us: int, dev_status: torch.Tensor
     _check(_lib.q4_selftest_bounded_wait(which, limit_us, _ptr(dev_status), _stream(stream)), "q4_selftest_bounded_wait")
 
 
-def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int, I_shared: int = 0) -> int:
+def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int, I_shared: int = 0, a8_mask: int = 0) -> int:
+    if a8_mask:
+        if I_shared:
+            raise ValueError("the W4A8 expert path takes no shared expert")
+        return int(_lib.moe_q4_workspace_size_a8(T, H, I, E, topk, a8_mask))
     if I_shared:
         return int(_lib.moe_q4_workspace_size_ex(T, H, I, E, topk, I_shared))
     return int(_lib.moe_q4_workspace_size(T, H, I, E, topk))
@@ -239,9 +251,11 @@ def moe_q4_workspace_size(T: int, H: int, I: int, E: int, topk: int, I_shared: i
 def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
                    experts: tuple, I: int, out_dtype=torch.float32, y: torch.Tensor | None = None,
                    workspace: torch.Tensor | None = None, want_routing: bool = False,
-                   dev_status: torch.Tensor | None = None, stream=None, shared: tuple | None = None):
+                   dev_status: torch.Tensor | None = None, stream=None, shared: tuple | None = None,
+                   a8_mask: int = 0):
     """Top-k routed MoE SwiGLU layer with INT4 experts.  experts = (gate, up, down) Q4Weight, stacked by expert;
     shared (optional) = (gate, up, down) Q4Weight of a shared expert every token passes through.
+    a8_mask: bit 0 runs gate/up, bit 1 runs down on per-row INT8 activation codes (W4A8; no shared expert).
     Returns y, or (y, topk_ids, topk_w, perm, offsets, counts) when want_routing."""
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
@@ -252,7 +266,7 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
     od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
     I_s = shared[0].n if shared is not None else 0
-    ws_bytes = moe_q4_workspace_size(T, H, I, E, topk, I_s)
+    ws_bytes = moe_q4_workspace_size(T, H, I, E, topk, I_s, a8_mask)
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
@@ -264,10 +278,16 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
         perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
         offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
         cnts = torch.empty((E,), dtype=torch.int32, device=dev)
-    _check(_lib.moe_q4_forward_ex(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, sdescs, I_s,
-                                  _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
-                                  _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
-           "moe_q4_forward")
+    if a8_mask:
+        _check(_lib.moe_q4_forward_a8(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, a8_mask,
+                                      _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
+                                      _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
+               "moe_q4_forward_a8")
+    else:
+        _check(_lib.moe_q4_forward_ex(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, sdescs,
+                                      I_s, _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
+                                      _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
+               "moe_q4_forward")
     if want_routing:
         return y, ids, wts, perm, offs, cnts
     return y

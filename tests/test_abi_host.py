@@ -85,6 +85,28 @@ def test_act_quant_validation():
     assert L.act_quant_per_token(None, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_NULL
     assert L.act_quant_per_token(FAKE, 4, 12, FAKE, FAKE, None, None) == q4.Q4_ERR_SHAPE
     assert L.act_quant_per_token(FAKE + 2, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_ALIGN
+    assert L.act_quant_per_token_f16(None, 4, 128, FAKE, FAKE, None, None) == q4.Q4_ERR_NULL
+    assert L.act_quant_per_token_f16(FAKE, 4, 12, FAKE, FAKE, None, None) == q4.Q4_ERR_SHAPE
+    assert L.act_quant_per_token_f16(FAKE, 4, 128, FAKE + 8, FAKE, None, None) == q4.Q4_ERR_ALIGN
+
+
+def test_moe_a8_validation_and_workspace():
+    L = q4._lib
+    T, H, I, E, topk = 64, 256, 128, 8, 2
+    base = L.moe_q4_workspace_size(T, H, I, E, topk)
+    # each INT8 path adds its codes and scales: x codes + token and row scales; h codes + row scales
+    assert L.moe_q4_workspace_size_a8(T, H, I, E, topk, 0) == base
+    assert L.moe_q4_workspace_size_a8(T, H, I, E, topk, 1) >= base + T * H + 4 * T + 4 * T * topk
+    assert L.moe_q4_workspace_size_a8(T, H, I, E, topk, 2) >= base + T * topk * I + 4 * T * topk
+    assert L.moe_q4_workspace_size_a8(T, H, I, E, topk, 4) == 0
+    ex = (q4.q4_weight * 3)(_w(n=E * I, k=H), _w(n=E * I, k=H), _w(n=E * H, k=I))
+    args = (FAKE, T, H, FAKE, None, E, topk, ex, I)
+    assert L.moe_q4_forward_a8(*args, 4, FAKE, 0, None, None, None, None, None, FAKE, 1 << 30, None, None) == q4.Q4_ERR_UNSUPPORTED
+    assert L.moe_q4_forward_a8(*args, -1, FAKE, 0, None, None, None, None, None, FAKE, 1 << 30, None, None) == q4.Q4_ERR_UNSUPPORTED
+    need = L.moe_q4_workspace_size_a8(T, H, I, E, topk, 3)
+    assert L.moe_q4_forward_a8(*args, 3, FAKE, 0, None, None, None, None, None, FAKE, need - 1, None, None) == q4.Q4_ERR_WORKSPACE
+    assert L.moe_q4_forward_a8(None, T, H, FAKE, None, E, topk, ex, I, 3, FAKE, 0, None, None, None, None, None, FAKE,
+                               need, None, None) == q4.Q4_ERR_NULL
 
 
 def test_grouped_validation():

@@ -165,6 +165,33 @@ def test_act_quant_bitexact(q4, m, k):
     assert np.array_equal(xq.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("m,k", [(33, 1024), (256, 2048), (5, 8192), (3, 20000), (1, 8)])
+def test_act_quant_f16_bitexact(q4, m, k):
+    """fp16 rows (the MoE's intermediate activations): codes and scales bit-exact against the oracle.
+    Rows span fp16's range: subnormal-only rows, ordinary rows, rows near the fp16 maximum."""
+    rng = np.random.default_rng(m * 7919 + k)
+    mags = [2.0 ** -20, 2.0 ** -14, 1e-3, 0.5, 3.0, 100.0, 8e3]
+    h = np.stack([np.clip(rng.standard_normal(k) * mags[i % len(mags)], -65000.0, 65000.0)
+                  for i in range(m)]).astype(np.float16)
+    if m > 2:
+        h[1] = 0
+    bits = h.view(np.uint16)
+    q_ref, s_ref = oracle.act_quant_f16(bits, k)
+    xq, sc = q4.act_quant_per_token(cuda_u16_as(bits, torch.float16))
+    torch.cuda.synchronize()
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+
+
+def test_act_quant_f16_nonfinite_status(q4):
+    h = np.ones((4, 64), np.float16)
+    h[2, 5] = np.inf
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.act_quant_per_token(cuda_u16_as(h.view(np.uint16), torch.float16), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == q4.Q4_ERR_NONFINITE
+
+
 def test_act_quant_rounding_stress(q4):
     """Quotients at and next to half-integers, scales with full mantissas, and extreme magnitudes (tiny
     rows take the kernel's division path, the rest the reciprocal-and-FMA path): codes and scales

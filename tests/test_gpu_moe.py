@@ -122,3 +122,65 @@ def test_moe_with_shared_expert(q4, T, H, I, E, topk, I_s, group, sym):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert_close(y.cpu().numpy(), np.asarray(ref).reshape(T, H), what="moe + shared expert")
+
+
+# ---------------------------------------------------------------------------------------------- #
+# the expert projections on INT8 activation codes (W4A8): a8_mask bit 0 = gate/up, bit 1 = down
+# ---------------------------------------------------------------------------------------------- #
+
+def _run_a8(q4, T, H, I, E, topk, group, sym, mask, tag, tokens=None):
+    x = synth.activations(("moe", tag, "x"), T, H)
+    Wr, bias = synth.router(("moe", tag), E, H, skew=1.1)
+    qs = _experts(tag, E, H, I, group, sym)
+    logits, ids, w, counts = oracle.route(x, H, Wr, bias, topk)
+    offsets, perm = oracle.permute(ids, E)
+    ref = oracle.moe_experts_a8(x, H, ids, w, qs[0], qs[1], qs[2], I, group, sym, mask, tokens=tokens)
+    ex = (upload_weight(q4, *qs[0], E * I, H, group, sym), upload_weight(q4, *qs[1], E * I, H, group, sym),
+          upload_weight(q4, *qs[2], E * H, I, group, sym))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y, ids_d, w_d, perm_d, off_d, cnt_d = q4.moe_q4_forward(
+        cuda_u16_as(x, torch.bfloat16), torch.from_numpy(Wr).cuda(), torch.from_numpy(bias).cuda(), topk, ex, I,
+        want_routing=True, dev_status=st, a8_mask=mask)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(ids_d.cpu().numpy(), ids), "expert ids differ"
+    assert np.array_equal(perm_d.cpu().numpy(), perm)
+    assert np.array_equal(off_d.cpu().numpy(), offsets)
+    yn = y.cpu().numpy()
+    return (yn if tokens is None else yn[tokens]), ref
+
+
+@pytest.mark.parametrize("mask", [1, 2, 3])
+@pytest.mark.parametrize("T,H,I,E,topk,group,sym", [
+    (64, 256, 128, 8, 2, 128, False),     # every expert busy
+    (37, 256, 256, 5, 3, 64, True),       # ragged token count, group 64, symmetric
+    (200, 512, 256, 64, 8, 128, False),   # 64 experts / top-8, skewed: some experts empty
+    (300, 512, 384, 4, 2, 64, False),     # several 128-row tiles per expert, group 64 asymmetric
+])
+def test_moe_a8(q4, T, H, I, E, topk, group, sym, mask):
+    yn, ref = _run_a8(q4, T, H, I, E, topk, group, sym, mask, f"a8-{T}-{E}")
+    assert_close(yn, ref, what=f"moe a8 mask {mask}")
+
+
+def test_moe_a8_workload_full_size(q4):
+    """The full layer (4096 tokens, 64 experts of 1024, top-8, asymmetric group 128) with every expert
+    projection on INT8 activations: routing for every token, outputs on a sample of tokens."""
+    tokens = np.arange(0, 4096, 131)
+    yn, ref = _run_a8(q4, 4096, 2048, 1024, 64, 8, 128, False, 3, "full", tokens=tokens)
+    assert_close(yn, ref, what="moe a8 full")
+
+
+def test_moe_a8_rejects_shared_expert_and_bad_mask(q4):
+    from moe_linear_layers_b200.q4 import Q4Error, Q4_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        q4.moe_q4_workspace_size(16, 128, 128, 4, 2, I_shared=128, a8_mask=1)
+    assert q4._lib.moe_q4_workspace_size_a8(16, 128, 128, 4, 2, 4) == 0
+    T, H, I, E, topk = 16, 128, 128, 4, 2
+    qs = _experts("a8bad", E, H, I, 128, True)
+    ex = tuple(upload_weight(q4, *qq, n, k, 128, True) for qq, n, k in zip(qs, (E * I, E * I, E * H), (H, H, I)))
+    x = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    Wr = torch.zeros((E, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk, a8_mask=3), dtype=torch.uint8, device="cuda")
+    with pytest.raises(Q4Error) as ei:
+        q4.moe_q4_forward(x, Wr, None, topk, ex, I, workspace=ws, a8_mask=5)
+    assert ei.value.status == Q4_ERR_UNSUPPORTED
