@@ -250,3 +250,22 @@ def moe_experts_a8(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: i
     if rc != 0:
         raise OracleError(f"orc_moe_experts_a8 returned {rc}")
     return y
+
+
+def moe_experts_classes(x_bf16_bits, H: int, ids, w, class_begin, classes, I: int, tokens=None):
+    """The expert FFN with per-class quantization (the W4A8 page §5.3: group size chosen by how often an
+    expert is used).  class c = experts class_begin[c] .. class_begin[c+1]-1; classes[c] = (gate, up, down,
+    group, symmetric) with gate/up/down = (packed, scales, zeros) stacked over the class's experts.  Each
+    class is evaluated by moe_experts on the slots routed to it (the other slots get weight 0, so they add
+    exact zeros) and the classes' outputs are summed.  Returns fp64 [n_tok][H]."""
+    ids = np.asarray(ids, np.int32)
+    w = np.asarray(w, np.float64)
+    y = None
+    for c, (gate, up, down, group, symmetric) in enumerate(classes):
+        e0, e1 = int(class_begin[c]), int(class_begin[c + 1])
+        mine = (ids >= e0) & (ids < e1)
+        ids_c = np.where(mine, ids - e0, 0).astype(np.int32)
+        w_c = np.where(mine, w, 0.0)
+        yc = moe_experts(x_bf16_bits, H, ids_c, w_c, gate, up, down, I, group, symmetric, tokens=tokens)
+        y = yc if y is None else y + yc
+    return y

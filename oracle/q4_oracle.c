@@ -425,7 +425,11 @@ void orc_permute(const int32_t* ids, int T, int topk, int E, int32_t* offsets, i
  * (proportional recombination).  For token t and each chosen expert e = ids[t][j]:
  *   g = x_t . dequant(Wg_e)^T,  u = x_t . dequant(Wu_e)^T           (length I, fp64)
  *   h = g / (1 + exp(-g)) * u                                       (SiLU(g) * u, fp64)
- *   o = h . dequant(Wd_e)^T                                         (length H, fp64)
+ *   h16 = fp16(fp32(h))      the layer's intermediate is STORED as fp16 (reading: the interface between
+ *                            the two expert projections holds h in fp16, as the library documents it;
+ *                            the rounding through fp32 can differ from a direct rounding only when the
+ *                            fp32 value lies exactly halfway between two fp16 values)
+ *   o = h16 . dequant(Wd_e)^T                                       (length H, fp64)
  *   y_t = sum_j w[t][j] * o                                         (fp64)
  * Expert weights are stacked: gate/up packed [E*I][H/2], scales/zeros [E*I][H/group];
  * down packed [E*H][I/2], scales/zeros [E*H][I/group].
@@ -464,6 +468,7 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
                     uv += xr[c] * (double)deq_at(up, us, uz, H, group, symmetric, i, c);
                 }
                 h[i] = gv / (1.0 + exp(-gv)) * uv;
+                h[i] = (double)orc_f16_to_f32(orc_f32_to_f16((float)h[i]));   /* stored as fp16 */
             }
             const uint8_t* dp = d_packed + (size_t)e * H * (I / 2);
             const uint16_t* ds = d_scales + (size_t)e * H * gI;
@@ -492,11 +497,10 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
  *                g_i = sum_g sa * sg[i][g] * sum_{k in g} xq[k] * (qg[i][k] - zg[i][g])   (fp64
  *                of the exact INT32 partials), u_i likewise with the up matrix;
  *   bit 0 clear: g, u as in orc_moe_experts (fp64 over the dequantized weights);
- *   h = g / (1 + exp(-g)) * u (fp64);
- *   bit 1 set:   h is stored as fp16 (rounded through fp32: h16 = fp16(fp32(h))), then
- *                hq, sh = act_quant(h16) over the row's I values, and
+ *   h = g / (1 + exp(-g)) * u (fp64), stored as fp16 as in orc_moe_experts: h16 = fp16(fp32(h));
+ *   bit 1 set:   hq, sh = act_quant(h16) over the row's I values, and
  *                o_c = sum_g sh * sd[c][g] * sum_{i in g} hq[i] * (qd[c][i] - zd[c][g]);
- *   bit 1 clear: o = h . dequant(Wd_e)^T (fp64);
+ *   bit 1 clear: o = h16 . dequant(Wd_e)^T (fp64);
  *   y_t = sum_j w[t][j] * o (fp64).
  * Returns ORC_ERR_NONFINITE when a quantized row holds a non-finite value.
  * ------------------------------------------------------------------------------------------- */
@@ -563,14 +567,12 @@ int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, cons
             const uint16_t* dz = d_zeros ? d_zeros + (size_t)e * H * gI : NULL;
             double wj = w[(size_t)t * topk + j];
             double sh = 0.0;
-            if (a8_mask & 2) {
-                for (int i = 0; i < I; i++) h16[i] = orc_f16_to_f32(orc_f32_to_f16((float)h[i]));
-                sh = (double)act_quant_row(h16, I, hq, &rb);
-            }
+            for (int i = 0; i < I; i++) h16[i] = orc_f16_to_f32(orc_f32_to_f16((float)h[i]));
+            if (a8_mask & 2) sh = (double)act_quant_row(h16, I, hq, &rb);
             for (int c = 0; c < H; c++) {
                 double o = 0.0;
                 if (a8_mask & 2) o = w4a8_dot(hq, sh, dp, ds, dz, symmetric, I, group, c);
-                else for (int i = 0; i < I; i++) o += h[i] * (double)deq_at(dp, ds, dz, I, group, symmetric, c, i);
+                else for (int i = 0; i < I; i++) o += (double)h16[i] * (double)deq_at(dp, ds, dz, I, group, symmetric, c, i);
                 yr[c] += wj * o;
             }
         }

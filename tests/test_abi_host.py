@@ -120,3 +120,31 @@ def test_grouped_validation():
     assert L.q4_linear_w4a16_grouped(2, xs, 5, ws2, ys, 0, None, None) == q4.Q4_ERR_SHAPE  # m > 4
     xs_bad = (ctypes.c_void_p * 2)(FAKE, FAKE + 2)
     assert L.q4_linear_w4a16_grouped(2, xs_bad, 1, ws2, ys, 0, None, None) == q4.Q4_ERR_ALIGN
+
+
+def test_moe_classes_validation():
+    L = q4._lib
+    T, H, I, E, topk = 64, 256, 128, 8, 2
+    ws = L.moe_q4_workspace_size(T, H, I, E, topk)
+
+    def call(begin, ex):
+        b = (ctypes.c_int32 * len(begin))(*begin)
+        n = len(begin) - 1
+        return L.moe_q4_forward_classes(FAKE, T, H, FAKE, None, E, topk, n, b, ex, I, FAKE, 0, None, None, None,
+                                        None, None, FAKE, ws, None, None)
+
+    two = (q4.q4_weight * 6)(_w(n=3 * I, k=H), _w(n=3 * I, k=H), _w(n=3 * H, k=I),
+                             _w(n=5 * I, k=H, group=128, sym=0, zeros=FAKE), _w(n=5 * I, k=H, group=128, sym=0, zeros=FAKE),
+                             _w(n=5 * H, k=I, group=128, sym=0, zeros=FAKE))
+    assert call([0, 3, 9], two) == q4.Q4_ERR_SHAPE          # last bound != E
+    assert call([0, 4, 8], two) == q4.Q4_ERR_SHAPE          # class sizes do not match the weights
+    assert call([1, 3, 8], two) == q4.Q4_ERR_SHAPE          # first bound != 0
+    assert call([0, 0, 8], two) == q4.Q4_ERR_SHAPE          # empty class
+    mixed = (q4.q4_weight * 6)(*two)
+    mixed[4] = _w(n=5 * I, k=H, group=64, sym=0, zeros=FAKE)  # up of class 1 with another group
+    assert call([0, 3, 8], mixed) == q4.Q4_ERR_UNSUPPORTED
+    assert L.moe_q4_forward_classes(FAKE, T, H, FAKE, None, E, topk, 2, None, two, I, FAKE, 0, None, None, None,
+                                    None, None, FAKE, ws, None, None) == q4.Q4_ERR_NULL
+    ok = (ctypes.c_int32 * 3)(0, 3, 8)
+    assert L.moe_q4_forward_classes(FAKE, T, H, FAKE, None, E, topk, 2, ok, two, I, FAKE, 0, None, None, None,
+                                    None, None, FAKE, ws - 1, None, None) == q4.Q4_ERR_WORKSPACE

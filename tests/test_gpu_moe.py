@@ -184,3 +184,53 @@ def test_moe_a8_rejects_shared_expert_and_bad_mask(q4):
     with pytest.raises(Q4Error) as ei:
         q4.moe_q4_forward(x, Wr, None, topk, ex, I, workspace=ws, a8_mask=5)
     assert ei.value.status == Q4_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------------------------- #
+# expert classes with their own group size and symmetry (moe_q4_forward_classes)
+# ---------------------------------------------------------------------------------------------- #
+
+def _run_classes(q4, T, H, I, E, topk, begin, params, tag, tokens=None):
+    x = synth.activations(("moe", tag, "x"), T, H)
+    Wr, bias = synth.router(("moe", tag), E, H, skew=1.1)
+    logits, ids, w, counts = oracle.route(x, H, Wr, bias, topk)
+    offsets, perm = oracle.permute(ids, E)
+    classes, dev_classes = [], []
+    for c, (group, sym) in enumerate(params):
+        Ec = begin[c + 1] - begin[c]
+        qs = [oracle.quantize(synth.weights(("moe", tag, c, nm), n, k), group, sym)
+              for nm, n, k in (("gate", Ec * I, H), ("up", Ec * I, H), ("down", Ec * H, I))]
+        classes.append((qs[0], qs[1], qs[2], group, sym))
+        dev_classes.append(tuple(upload_weight(q4, *q, n, k, group, sym)
+                                 for q, n, k in zip(qs, (Ec * I, Ec * I, Ec * H), (H, H, I))))
+    ref = oracle.moe_experts_classes(x, H, ids, w, begin, classes, I, tokens=tokens)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y, ids_d, w_d, perm_d, off_d, cnt_d = q4.moe_q4_forward_classes(
+        cuda_u16_as(x, torch.bfloat16), torch.from_numpy(Wr).cuda(), torch.from_numpy(bias).cuda(), topk, begin,
+        dev_classes, I, want_routing=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(ids_d.cpu().numpy(), ids)
+    assert np.array_equal(perm_d.cpu().numpy(), perm)
+    assert np.array_equal(off_d.cpu().numpy(), offsets)
+    yn = y.cpu().numpy()
+    return (yn if tokens is None else yn[tokens]), ref
+
+
+@pytest.mark.parametrize("T,H,I,E,topk,begin,params", [
+    (200, 512, 256, 16, 4, [0, 2, 8, 16], [(64, True), (128, False), (64, False)]),
+    (37, 256, 128, 5, 3, [0, 1, 5], [(64, False), (128, True)]),
+    (300, 256, 128, 8, 2, [0, 8], [(128, False)]),          # one class = the plain layer
+])
+def test_moe_classes(q4, T, H, I, E, topk, begin, params):
+    yn, ref = _run_classes(q4, T, H, I, E, topk, begin, params, f"cls{T}-{E}")
+    assert_close(yn, ref, what="moe classes")
+
+
+def test_moe_classes_workload_full_size(q4):
+    """The 4096-token layer with the four most chosen experts (6 % of 64; expert 0 is the hottest under the
+    Zipf-skewed logits) quantized at group 64 and the other 60 at group 128, asymmetric."""
+    tokens = np.arange(0, 4096, 173)
+    yn, ref = _run_classes(q4, 4096, 2048, 1024, 64, 8, [0, 4, 64], [(64, False), (128, False)], "clsfull",
+                           tokens=tokens)
+    assert_close(yn, ref, what="moe classes full")

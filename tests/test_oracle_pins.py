@@ -383,7 +383,7 @@ def test_shared_expert_is_the_dense_swiglu_ffn():
     y = oracle.shared_expert(x, H, qs[0], qs[1], qs[2], I_s, group, False)
     g = oracle.linear_w4a16(x, *qs[0], I_s, H, group, False)
     u = oracle.linear_w4a16(x, *qs[1], I_s, H, group, False)
-    h = g / (1.0 + np.exp(-g)) * u
+    h = _f16_store(g / (1.0 + np.exp(-g)) * u)
     wd = oracle.dequant(*qs[2], I_s, group, False).astype(np.float64)
     np.testing.assert_allclose(y, h @ wd.T, rtol=1e-11, atol=1e-12 * np.abs(y).max())
 
@@ -432,10 +432,15 @@ def test_permute_is_stable_sort():
 # MoE special cases: one expert = dense SwiGLU; k = E with equal logits = uniform average
 # ---------------------------------------------------------------------------------------------- #
 
+def _f16_store(h):
+    """The MoE intermediate as the layer stores it: fp64 -> fp32 -> fp16 (numpy's conversions), back to fp64."""
+    return np.asarray(h, np.float64).astype(np.float32).astype(np.float16).astype(np.float64)
+
+
 def _dense_swiglu(xf, Wg, Wu, Wd):
     g = xf @ Wg.T
     u = xf @ Wu.T
-    return (g / (1.0 + np.exp(-g)) * u) @ Wd.T
+    return _f16_store(g / (1.0 + np.exp(-g)) * u) @ Wd.T
 
 
 def _stacked_experts(E, H, I, group, sym, seed):
@@ -530,7 +535,7 @@ def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
                 hq, sh = oracle.act_quant_f16(h16.view(np.uint16)[None, :], I)
                 o = oracle.linear_w4a8(hq, sh, dq[0], dq[1], H, I, group, zeros=dq[2], symmetric=sym)[0]
             else:
-                o = h @ oracle.dequant(*dq, I, group, sym).astype(np.float64).T
+                o = _f16_store(h) @ oracle.dequant(*dq, I, group, sym).astype(np.float64).T
             y[t] += w[t, j] * o
     return y
 
@@ -568,6 +573,58 @@ def test_moe_a8_mask0_is_the_w4a16_layer_and_a8_stays_close():
     for mask in (1, 2, 3):
         y8 = oracle.moe_experts_a8(x, H, ids, w, stack[0], stack[1], stack[2], I, group, False, mask)
         assert 0 < np.sqrt(np.mean((y8 - y16) ** 2)) / rms < 0.03
+
+
+# ---------------------------------------------------------------------------------------------- #
+# expert classes with their own group size (W4A8 page §5.3)
+# ---------------------------------------------------------------------------------------------- #
+
+def test_moe_classes_one_class_and_equal_classes_are_the_layer():
+    T, H, I, E, topk, group = 6, 256, 128, 6, 2, 64
+    x = synth.activations(("pins", "cls-x"), T, H)
+    Wr, bias = synth.router(("pins", "cls"), E, H)
+    _, ids, w, _ = oracle.route(x, H, Wr, bias, topk)
+    stack = [oracle.quantize(synth.weights(("pins", "cls", nm), n, k), group, False)
+             for nm, n, k in (("g", E * I, H), ("u", E * I, H), ("d", E * H, I))]
+    ref = oracle.moe_experts(x, H, ids, w, stack[0], stack[1], stack[2], I, group, False)
+    one = oracle.moe_experts_classes(x, H, ids, w, [0, E], [(stack[0], stack[1], stack[2], group, False)], I)
+    assert np.array_equal(one, ref)
+    # the same quantized stack cut into classes {0,1}, {2..5}: row blocks of the stacked matrices
+    def cut(q, rows_per, e0, e1):
+        pk, sc, zr = q
+        sl = slice(e0 * rows_per, e1 * rows_per)
+        return pk[sl], sc[sl], (None if zr is None else zr[sl])
+    classes = [tuple(cut(q, r, a, b) for q, r in zip(stack, (I, I, H))) + (group, False) for a, b in ((0, 2), (2, E))]
+    two = oracle.moe_experts_classes(x, H, ids, w, [0, 2, E], classes, I)
+    np.testing.assert_allclose(two, ref, rtol=1e-12, atol=1e-14 * np.abs(ref).max())
+
+
+def test_moe_classes_each_expert_uses_its_class_quantization():
+    """Classes with different group sizes and symmetry: every token's output equals the dense SwiGLU FFNs
+    of its chosen experts built from each class's own dequantized matrices (numpy), weighted."""
+    T, H, I, E, topk = 5, 256, 128, 5, 2
+    x = synth.activations(("pins", "cls2-x"), T, H)
+    Wr, bias = synth.router(("pins", "cls2"), E, H)
+    _, ids, w, _ = oracle.route(x, H, Wr, bias, topk)
+    begin = [0, 1, 3, E]
+    params = [(64, True), (128, False), (64, False)]
+    classes, dense = [], {}
+    for c, (group, sym) in enumerate(params):
+        Ec = begin[c + 1] - begin[c]
+        qs = [oracle.quantize(synth.weights(("pins", "cls2", c, nm), n, k), group, sym)
+              for nm, n, k in (("g", Ec * I, H), ("u", Ec * I, H), ("d", Ec * H, I))]
+        classes.append((qs[0], qs[1], qs[2], group, sym))
+        deq = [oracle.dequant(*q, k, group, sym).astype(np.float64) for q, k in zip(qs, (H, H, I))]
+        for le in range(Ec):
+            dense[begin[c] + le] = (deq[0][le * I:(le + 1) * I], deq[1][le * I:(le + 1) * I], deq[2][le * H:(le + 1) * H])
+    y = oracle.moe_experts_classes(x, H, ids, w, begin, classes, I)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    ref = np.zeros((T, H))
+    for t in range(T):
+        for j in range(topk):
+            Wg, Wu, Wd = dense[ids[t, j]]
+            ref[t] += w[t, j] * _dense_swiglu(xf[t:t + 1], Wg, Wu, Wd)[0]
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
 
 
 # ---------------------------------------------------------------------------------------------- #
