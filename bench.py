@@ -462,6 +462,21 @@ def run_moe(q4, args, dev):
         a8[name] = {"ms_per_step": round(ms_a, 4), "tokens_per_s": round(T / (ms_a * 1e-3), 1),
                     "tops": round(flops / (ms_a * 1e-3) / 1e12, 1), "a8_mask": mask}
         del ga, ws_a
+    # the same layer with per-class group sizes: the 4 most chosen experts (expert 0 is the hottest under the
+    # skew) at group 64, the other 60 at group 128 (moe_q4_forward_classes)
+    hot = 4
+    cls = [[], []]
+    for nm, n_per, k in (("gate", I, H), ("up", I, H), ("down", H, I)):
+        W = torch.from_numpy(synth.weights((0, "moe", nm), E * n_per, k)).to(dev)
+        cls[0].append(q4.q4_quantize_pack(W[:hot * n_per].contiguous(), 64, False))
+        cls[1].append(q4.q4_quantize_pack(W[hot * n_per:].contiguous(), 128, False))
+        del W
+    gc = graph_of(lambda: q4.moe_q4_forward_classes(x, Wr, bias, topk, [0, hot, E], [tuple(cls[0]), tuple(cls[1])],
+                                                    I, y=y, workspace=ws_t))
+    for _ in range(3):
+        gc.replay()
+    ms_c = time_replays(gc, steps, 1) / steps
+    del gc
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "workload": "MoE layer: 4096 tokens, hidden 2048, 64 SwiGLU experts of intermediate 1024, top-8, "
                         "asymmetric INT4 g128, fp32 router with Zipf-skewed logits (bias -1.1 ln(e+1)), fp32 out",
@@ -480,6 +495,10 @@ def run_moe(q4, args, dev):
                                  "activation codes, INT32 group partials (moe_q4_forward_a8, mask 3)"),
             "w4a8_down_only": dict(a8["w4a8_down_only"], workload="the same layer, only the down projection on "
                                    "INT8 codes of h (moe_q4_forward_a8, mask 2)"),
+            "group64_hot_experts": {"ms_per_step": round(ms_c, 4), "tokens_per_s": round(T / (ms_c * 1e-3), 1),
+                                    "tflops": round(flops / (ms_c * 1e-3) / 1e12, 1),
+                                    "workload": "the same layer with the 4 most chosen experts quantized at group 64 "
+                                                "and the other 60 at group 128 (moe_q4_forward_classes)"},
             "gpu_launches": 6 * steps, "clocks": clk.summary()}
 
 

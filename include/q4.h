@@ -269,6 +269,27 @@ int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H,
                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_q4_forward_classes -- moe_q4_forward with the experts split into classes, each with its own
+ * quantization group size and symmetry.
+ * Source: the W4A8 page §5.3 (group size by how often an expert is chosen: smaller groups, i.e. more
+ * scales and less error, for the experts most tokens go to, larger groups for rarely chosen ones) and
+ * §5.2 (rarely chosen experts can take coarser quantization).
+ * Class c holds experts class_begin[c] .. class_begin[c+1]-1 (expert ids as the router numbers them;
+ * order the experts so that each class is a contiguous id range); its weights are experts[3c],
+ * experts[3c+1], experts[3c+2] = gate [E_c*I][H], up [E_c*I][H], down [E_c*H][I] stacked by the
+ * class's experts in id order, with one group (64 or 128) and symmetry shared by the three.
+ * class_begin: host array of n_classes + 1 ints, class_begin[0] = 0 < ... < class_begin[n_classes] = E.
+ * The layer computes exactly moe_q4_forward's function with each expert's matrices dequantized with
+ * its class's parameters.  Every other argument, the workspace size and the limits as moe_q4_forward.
+ */
+int moe_q4_forward_classes(const uint16_t* x, int32_t T, int32_t H,
+                           const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                           int32_t n_classes, const int32_t* class_begin, const q4_weight* experts, int32_t I,
+                           void* y, int32_t out_dtype,
+                           int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate device memory.
  * No counterpart in the source pages: this is a library convenience, not part of the method.
  *

@@ -480,7 +480,8 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
                         int32_t E, int32_t topk, const q4_weight* experts, int32_t I, const q4_weight* shared,
                         int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
                         int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
-                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+                        size_t workspace_bytes, int32_t* dev_status, void* stream, int n_classes = 1,
+                        const int32_t* class_begin = nullptr);
 
 extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                               int32_t E, int32_t topk, const q4_weight* experts, int32_t I, void* y, int32_t out_dtype,
@@ -525,29 +526,54 @@ extern "C" int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H, const 
                         topk_ids, topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream);
 }
 
+extern "C" int moe_q4_forward_classes(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                      const float* router_bias, int32_t E, int32_t topk, int32_t n_classes,
+                                      const int32_t* class_begin, const q4_weight* experts, int32_t I, void* y,
+                                      int32_t out_dtype, int32_t* topk_ids, float* topk_w, int32_t* perm,
+                                      int32_t* offsets, int32_t* expert_counts, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (!class_begin) return Q4_ERR_NULL;
+    return forward_impl(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, 0, y, out_dtype, topk_ids,
+                        topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream,
+                        n_classes, class_begin);
+}
+
 static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                         int32_t E, int32_t topk, const q4_weight* experts, int32_t I, const q4_weight* shared,
                         int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
                         int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
-                        size_t workspace_bytes, int32_t* dev_status, void* stream)
+                        size_t workspace_bytes, int32_t* dev_status, void* stream, int n_classes,
+                        const int32_t* class_begin)
 {
     if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
         return Q4_ERR_SHAPE;
     if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
-    const q4_weight& g = experts[0];
-    const q4_weight& u = experts[1];
-    const q4_weight& d = experts[2];
-    for (int i = 0; i < 3; i++) {
-        const q4_weight& w = experts[i];
-        if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
-        if (w.group != g.group || w.symmetric != g.symmetric) return Q4_ERR_UNSUPPORTED;
-        if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
-            return Q4_ERR_ALIGN;
+    // expert classes: experts [begin[c], begin[c+1]) share one stacked weight triple (one class = all)
+    int32_t single[2] = {0, E};
+    if (!class_begin) {
+        n_classes = 1;
+        class_begin = single;
     }
-    if (g.group != 64 && g.group != 128) return Q4_ERR_UNSUPPORTED;
-    if (g.n != E * I || g.k != H || u.n != E * I || u.k != H || d.n != E * H || d.k != I) return Q4_ERR_SHAPE;
+    if (n_classes < 1 || n_classes > E || class_begin[0] != 0 || class_begin[n_classes] != E) return Q4_ERR_SHAPE;
+    for (int c = 0; c < n_classes; c++) {
+        const int Ec = class_begin[c + 1] - class_begin[c];
+        if (Ec < 1) return Q4_ERR_SHAPE;
+        const q4_weight* cw = experts + 3 * c;
+        for (int i = 0; i < 3; i++) {
+            const q4_weight& w = cw[i];
+            if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
+            if (w.group != cw[0].group || w.symmetric != cw[0].symmetric) return Q4_ERR_UNSUPPORTED;
+            if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
+                return Q4_ERR_ALIGN;
+        }
+        if (cw[0].group != 64 && cw[0].group != 128) return Q4_ERR_UNSUPPORTED;
+        if (cw[0].n != Ec * I || cw[0].k != H || cw[1].n != Ec * I || cw[1].k != H || cw[2].n != Ec * H || cw[2].k != I)
+            return Q4_ERR_SHAPE;
+    }
+    const q4_weight& g = experts[0];
     if (shared) {   // the same group and symmetry as the routed experts
         if (I_shared <= 0) return Q4_ERR_SHAPE;
         if (I_shared % 128) return Q4_ERR_UNSUPPORTED;
@@ -607,12 +633,21 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
     if (const cudaError_t e = cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s)) return q4_cuda_status(e);
     rc = q4_launch_status();
     if (rc) return rc;
-    if (g.group == 128)
-        rc = g.symmetric ? launch_experts<128, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask)
-                         : launch_experts<128, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask);
-    else
-        rc = g.symmetric ? launch_experts<64, true>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask)
-                         : launch_experts<64, false>(ws, experts, T, H, I, E, topk, y32, dev_status, s, a8_mask);
+    for (int c = 0; c < n_classes && !rc; c++) {
+        // the class's slice of the routing bookkeeping: its experts' row offsets and tile prefix sums
+        const int e0 = class_begin[c], Ec = class_begin[c + 1] - e0;
+        const q4_weight* cw = experts + 3 * c;
+        Workspace wc = ws;
+        wc.offsets = ws.offsets + e0;
+        wc.tiles_gu = ws.tiles_gu + e0;
+        wc.tiles_dn = ws.tiles_dn + e0;
+        if (cw[0].group == 128)
+            rc = cw[0].symmetric ? launch_experts<128, true>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask)
+                                 : launch_experts<128, false>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask);
+        else
+            rc = cw[0].symmetric ? launch_experts<64, true>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask)
+                                 : launch_experts<64, false>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask);
+    }
     if (rc) return rc;
     if (I_shared > 0) {
         // the shared expert: every token, weight 1, its output added into the same fp32 sums

@@ -112,7 +112,7 @@ struct Args {
     int32_t* acc_dbg;         // W4A8 debug partials (nullable)
     int32_t* status;
     // MoE
-    const int32_t* expert_tiles;   // [E+1] prefix sums of tiles per expert
+    const int32_t* expert_tiles;   // [E+1] prefix sums of tiles per expert (taken relative to [0])
     const int32_t* offsets;        // [E+1] first permuted row of each expert
     const int32_t* row_tok;        // Down: [P] token of each permuted row
     const float* row_w;            // Down: [P] routing weight of each permuted row
@@ -365,11 +365,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
         if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
-        else sh->total_tiles = p.expert_tiles[p.E];
+        else sh->total_tiles = p.expert_tiles[p.E] - p.expert_tiles[0];
         tc::fence_mbar_init();
     }
+    // (a class of experts passes its slice of the layer's tile prefix sums: counted from its first expert)
     if constexpr (MODE != Mode::Dense)
-        for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sh->expert_tiles[i] = p.expert_tiles[i];
+        for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sh->expert_tiles[i] = p.expert_tiles[i] - p.expert_tiles[0];
     if (warp == 0 && lane == 0) {
         tc::tma_prefetch_desc(&tm_x);
         tc::tma_prefetch_desc(&tm_wa);

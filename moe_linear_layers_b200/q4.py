@@ -35,7 +35,7 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_q
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
-            "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8")
+            "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -72,6 +72,8 @@ _lib.moe_q4_workspace_size_a8.restype = _sz
 _lib.moe_q4_workspace_size_a8.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward_a8.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _i32,
                                    _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_forward_classes.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _i32, ctypes.POINTER(_i32),
+                                        ctypes.POINTER(q4_weight), _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -288,6 +290,44 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
                                       I_s, _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
                                       _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
                "moe_q4_forward")
+    if want_routing:
+        return y, ids, wts, perm, offs, cnts
+    return y
+
+
+def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                           class_begin, class_experts, I: int, out_dtype=torch.float32, y: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, want_routing: bool = False,
+                           dev_status: torch.Tensor | None = None, stream=None):
+    """moe_q4_forward with expert classes: class c = experts class_begin[c] .. class_begin[c+1]-1, whose
+    (gate, up, down) Q4Weight triple class_experts[c] is stacked over the class's experts and has its own
+    group size and symmetry."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    dev = x.device
+    n = len(class_experts)
+    if len(class_begin) != n + 1:
+        raise ValueError("class_begin needs one more entry than there are classes")
+    if y is None:
+        y = torch.empty((T, H), dtype=out_dtype, device=dev)
+    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    if workspace is None:
+        workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=dev)
+    begin = (_i32 * (n + 1))(*[int(v) for v in class_begin])
+    descs = (q4_weight * (3 * n))(*[w.desc for trip in class_experts for w in trip])
+    ids = wts = perm = offs = cnts = None
+    if want_routing:
+        ids = torch.empty((T, topk), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, topk), dtype=torch.float32, device=dev)
+        perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
+        offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+        cnts = torch.empty((E,), dtype=torch.int32, device=dev)
+    _check(_lib.moe_q4_forward_classes(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, n, begin, descs,
+                                       I, _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
+                                       _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
+           "moe_q4_forward_classes")
     if want_routing:
         return y, ids, wts, perm, offs, cnts
     return y
