@@ -606,6 +606,22 @@ def ncu_case(case):
         torch.cuda.synchronize()
         for _ in range(2):
             q4.moe_q4_forward(x, Wr, bias, topk, ex, I, y=y, workspace=ws_t)
+    elif case == "moe-classes":
+        T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+        x, Wr, bias, _ = build_moe(q4, dev)
+        hot = 4
+        cls = [[], []]
+        for nm, n_per, k in (("gate", I, H), ("up", I, H), ("down", H, I)):
+            W = torch.from_numpy(synth.weights((0, "moe", nm), E * n_per, k)).to(dev)
+            cls[0].append(q4.q4_quantize_pack(W[:hot * n_per].contiguous(), 64, False))
+            cls[1].append(q4.q4_quantize_pack(W[hot * n_per:].contiguous(), 128, False))
+            del W
+        ws_t = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk), dtype=torch.uint8, device=dev)
+        y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            q4.moe_q4_forward_classes(x, Wr, bias, topk, [0, hot, E], [tuple(cls[0]), tuple(cls[1])], I, y=y,
+                                      workspace=ws_t)
     elif case == "moe-a8":
         T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
         x, Wr, bias, ex = build_moe(q4, dev)
@@ -626,7 +642,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode-layer", "gemm", "moe", "moe-a8"],
+    ap.add_argument("--ncu-case", choices=["decode-layer", "gemm", "moe", "moe-a8", "moe-classes"],
                     help="run a small fixed launch sequence for an ncu capture and exit (no JSON line)")
     args = ap.parse_args()
     if args.ncu_case:
