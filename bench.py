@@ -419,6 +419,22 @@ def build_moe(q4, dev, seed=0):
     return x, torch.from_numpy(Wr).to(dev), torch.from_numpy(bias).to(dev), tuple(ex)
 
 
+MOE_TIERS = ((0, 3, 32), (3, 32, 64), (32, 64, 128))   # (first expert, end, group): hot, ordinary, cold
+
+
+def tiered_classes(q4, dev):
+    """The MoE workload's expert weights (the same fp32 matrices build_moe quantizes) cut into the hotness
+    tiers, each quantized with its own group size (asymmetric)."""
+    T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
+    cls = [[] for _ in MOE_TIERS]
+    for nm, n_per, k in (("gate", I, H), ("up", I, H), ("down", H, I)):
+        W = torch.from_numpy(synth.weights((0, "moe", nm), E * n_per, k)).to(dev)
+        for c, (e0, e1, group) in enumerate(MOE_TIERS):
+            cls[c].append(q4.q4_quantize_pack(W[e0 * n_per:e1 * n_per].contiguous(), group, False))
+        del W
+    return [t[0] for t in MOE_TIERS] + [E], [tuple(c) for c in cls]
+
+
 def run_moe(q4, args, dev):
     T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
     x, Wr, bias, ex = build_moe(q4, dev)
@@ -462,17 +478,10 @@ def run_moe(q4, args, dev):
         a8[name] = {"ms_per_step": round(ms_a, 4), "tokens_per_s": round(T / (ms_a * 1e-3), 1),
                     "tops": round(flops / (ms_a * 1e-3) / 1e12, 1), "a8_mask": mask}
         del ga, ws_a
-    # the same layer with per-class group sizes: the 4 most chosen experts (expert 0 is the hottest under the
-    # skew) at group 64, the other 60 at group 128 (moe_q4_forward_classes)
-    hot = 4
-    cls = [[], []]
-    for nm, n_per, k in (("gate", I, H), ("up", I, H), ("down", H, I)):
-        W = torch.from_numpy(synth.weights((0, "moe", nm), E * n_per, k)).to(dev)
-        cls[0].append(q4.q4_quantize_pack(W[:hot * n_per].contiguous(), 64, False))
-        cls[1].append(q4.q4_quantize_pack(W[hot * n_per:].contiguous(), 128, False))
-        del W
-    gc = graph_of(lambda: q4.moe_q4_forward_classes(x, Wr, bias, topk, [0, hot, E], [tuple(cls[0]), tuple(cls[1])],
-                                                    I, y=y, workspace=ws_t))
+    # the same layer with group sizes by expert hotness, the pages' three tiers: the 3 most chosen experts
+    # (5 %; expert 0 is the hottest under the skew) at group 32, experts 3-31 at 64, 32-63 at 128
+    begin, cls = tiered_classes(q4, dev)
+    gc = graph_of(lambda: q4.moe_q4_forward_classes(x, Wr, bias, topk, begin, cls, I, y=y, workspace=ws_t))
     for _ in range(3):
         gc.replay()
     ms_c = time_replays(gc, steps, 1) / steps
@@ -495,10 +504,10 @@ def run_moe(q4, args, dev):
                                  "activation codes, INT32 group partials (moe_q4_forward_a8, mask 3)"),
             "w4a8_down_only": dict(a8["w4a8_down_only"], workload="the same layer, only the down projection on "
                                    "INT8 codes of h (moe_q4_forward_a8, mask 2)"),
-            "group64_hot_experts": {"ms_per_step": round(ms_c, 4), "tokens_per_s": round(T / (ms_c * 1e-3), 1),
-                                    "tflops": round(flops / (ms_c * 1e-3) / 1e12, 1),
-                                    "workload": "the same layer with the 4 most chosen experts quantized at group 64 "
-                                                "and the other 60 at group 128 (moe_q4_forward_classes)"},
+            "group_by_hotness": {"ms_per_step": round(ms_c, 4), "tokens_per_s": round(T / (ms_c * 1e-3), 1),
+                                 "tflops": round(flops / (ms_c * 1e-3) / 1e12, 1),
+                                 "workload": "the same layer with group sizes by expert hotness: experts 0-2 at "
+                                             "group 32, 3-31 at 64, 32-63 at 128 (moe_q4_forward_classes)"},
             "gpu_launches": 6 * steps, "clocks": clk.summary()}
 
 
@@ -609,19 +618,12 @@ def ncu_case(case):
     elif case == "moe-classes":
         T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
         x, Wr, bias, _ = build_moe(q4, dev)
-        hot = 4
-        cls = [[], []]
-        for nm, n_per, k in (("gate", I, H), ("up", I, H), ("down", H, I)):
-            W = torch.from_numpy(synth.weights((0, "moe", nm), E * n_per, k)).to(dev)
-            cls[0].append(q4.q4_quantize_pack(W[:hot * n_per].contiguous(), 64, False))
-            cls[1].append(q4.q4_quantize_pack(W[hot * n_per:].contiguous(), 128, False))
-            del W
+        begin, cls = tiered_classes(q4, dev)
         ws_t = torch.empty(q4.moe_q4_workspace_size(T, H, I, E, topk), dtype=torch.uint8, device=dev)
         y = torch.empty((T, H), dtype=torch.float32, device=dev)
         torch.cuda.synchronize()
         for _ in range(2):
-            q4.moe_q4_forward_classes(x, Wr, bias, topk, [0, hot, E], [tuple(cls[0]), tuple(cls[1])], I, y=y,
-                                      workspace=ws_t)
+            q4.moe_q4_forward_classes(x, Wr, bias, topk, begin, cls, I, y=y, workspace=ws_t)
     elif case == "moe-a8":
         T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
         x, Wr, bias, ex = build_moe(q4, dev)

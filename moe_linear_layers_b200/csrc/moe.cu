@@ -468,6 +468,27 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     return launch<false, G, SYM, Mode::Down>(mh, md, md, d, sms, s);
 }
 
+// group 32 is built for the 16-bit expert GEMMs only (the INT8 paths take 64 and 128)
+int launch_experts_any(const Workspace& ws, const q4_weight* ex, int T, int H, int I, int E, int topk, float* y32,
+                       int32_t* status, cudaStream_t s, int a8_mask)
+{
+    const bool sym = ex[0].symmetric != 0;
+    switch (ex[0].group) {
+    case 128:
+        return sym ? launch_experts<128, true>(ws, ex, T, H, I, E, topk, y32, status, s, a8_mask)
+                   : launch_experts<128, false>(ws, ex, T, H, I, E, topk, y32, status, s, a8_mask);
+    case 64:
+        return sym ? launch_experts<64, true>(ws, ex, T, H, I, E, topk, y32, status, s, a8_mask)
+                   : launch_experts<64, false>(ws, ex, T, H, I, E, topk, y32, status, s, a8_mask);
+    case 32:
+        if (a8_mask) return Q4_ERR_UNSUPPORTED;
+        return sym ? launch_experts<32, true>(ws, ex, T, H, I, E, topk, y32, status, s, 0)
+                   : launch_experts<32, false>(ws, ex, T, H, I, E, topk, y32, status, s, 0);
+    default:
+        return Q4_ERR_UNSUPPORTED;
+    }
+}
+
 }  // namespace
 
 extern "C" size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk)
@@ -569,7 +590,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
             if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
                 return Q4_ERR_ALIGN;
         }
-        if (cw[0].group != 64 && cw[0].group != 128) return Q4_ERR_UNSUPPORTED;
+        if (cw[0].group != 64 && cw[0].group != 128 && !(cw[0].group == 32 && a8_mask == 0)) return Q4_ERR_UNSUPPORTED;
         if (cw[0].n != Ec * I || cw[0].k != H || cw[1].n != Ec * I || cw[1].k != H || cw[2].n != Ec * H || cw[2].k != I)
             return Q4_ERR_SHAPE;
     }
@@ -641,12 +662,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         wc.offsets = ws.offsets + e0;
         wc.tiles_gu = ws.tiles_gu + e0;
         wc.tiles_dn = ws.tiles_dn + e0;
-        if (cw[0].group == 128)
-            rc = cw[0].symmetric ? launch_experts<128, true>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask)
-                                 : launch_experts<128, false>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask);
-        else
-            rc = cw[0].symmetric ? launch_experts<64, true>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask)
-                                 : launch_experts<64, false>(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask);
+        rc = launch_experts_any(wc, cw, T, H, I, Ec, topk, y32, dev_status, s, a8_mask);
     }
     if (rc) return rc;
     if (I_shared > 0) {
@@ -662,12 +678,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         w1.tiles_dn = ws.tiles_dn_s;
         w1.row_tok = ws.row_tok_s;
         w1.row_w = ws.row_w_s;
-        if (g.group == 128)
-            rc = g.symmetric ? launch_experts<128, true>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s)
-                             : launch_experts<128, false>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s);
-        else
-            rc = g.symmetric ? launch_experts<64, true>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s)
-                             : launch_experts<64, false>(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s);
+        rc = launch_experts_any(w1, shared, T, H, I_shared, 1, 1, y32, dev_status, s, 0);
         if (rc) return rc;
     }
     if (out_dtype == Q4_OUT_BF16) {

@@ -93,7 +93,7 @@ extern "C" int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t gr
                                 void* stream)
 {
     if (!w || !packed || !scales || (!symmetric && !zeros)) return Q4_ERR_NULL;
-    if (n < 0 || k <= 0 || (group != 64 && group != 128) || k % group) return Q4_ERR_SHAPE;
+    if (n < 0 || k <= 0 || (group != 32 && group != 64 && group != 128) || k % group) return Q4_ERR_SHAPE;
     if (!q4_aligned16(w) || !q4_aligned16(packed) || !q4_aligned16(scales) || (!symmetric && !q4_aligned16(zeros)))
         return Q4_ERR_ALIGN;
     if (n == 0) return Q4_OK;
@@ -107,9 +107,12 @@ extern "C" int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t gr
     if (group == 128) {
         if (symmetric) quantize_pack_kernel<128, true><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
         else quantize_pack_kernel<128, false><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
-    } else {
+    } else if (group == 64) {
         if (symmetric) quantize_pack_kernel<64, true><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
         else quantize_pack_kernel<64, false><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
+    } else {
+        if (symmetric) quantize_pack_kernel<32, true><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
+        else quantize_pack_kernel<32, false><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
     }
     return q4_launch_status();
 }

@@ -48,7 +48,7 @@ def _w(n=128, k=256, group=64, sym=1, packed=FAKE, scales=FAKE, zeros=None):
     (dict(w=None), q4.Q4_ERR_NULL),
     (dict(w=_w(packed=None)), q4.Q4_ERR_NULL),
     (dict(w=_w(sym=0, zeros=None)), q4.Q4_ERR_NULL),
-    (dict(w=_w(group=32)), q4.Q4_ERR_SHAPE),
+    (dict(w=_w(group=32)), q4.Q4_ERR_SHAPE),      # group 32 serves the MoE expert GEMMs only
     (dict(w=_w(k=200)), q4.Q4_ERR_SHAPE),
     (dict(w=_w(packed=FAKE + 4)), q4.Q4_ERR_ALIGN),
     (dict(x=FAKE + 2), q4.Q4_ERR_ALIGN),
@@ -75,6 +75,8 @@ def test_quantize_validation():
     L = q4._lib
     assert L.q4_quantize_pack(None, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_NULL
     assert L.q4_quantize_pack(FAKE, 4, 128, 48, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_quantize_pack(FAKE, 4, 128, 256, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_quantize_pack(FAKE, 4, 96, 32, 1, FAKE + 8, FAKE, None, None, None) == q4.Q4_ERR_ALIGN  # 32 accepted
     assert L.q4_quantize_pack(FAKE, 4, 100, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
     assert L.q4_quantize_pack(FAKE + 8, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_ALIGN
     assert L.q4_quantize_pack(FAKE, 4, 128, 64, 0, FAKE, FAKE, None, None, None) == q4.Q4_ERR_NULL
@@ -148,3 +150,12 @@ def test_moe_classes_validation():
     ok = (ctypes.c_int32 * 3)(0, 3, 8)
     assert L.moe_q4_forward_classes(FAKE, T, H, FAKE, None, E, topk, 2, ok, two, I, FAKE, 0, None, None, None,
                                     None, None, FAKE, ws - 1, None, None) == q4.Q4_ERR_WORKSPACE
+
+
+def test_moe_group32_only_on_the_16bit_path():
+    L = q4._lib
+    T, H, I, E, topk = 64, 256, 128, 8, 2
+    ex = (q4.q4_weight * 3)(_w(n=E * I, k=H, group=32), _w(n=E * I, k=H, group=32), _w(n=E * H, k=I, group=32))
+    need = L.moe_q4_workspace_size_a8(T, H, I, E, topk, 3)
+    assert L.moe_q4_forward_a8(FAKE, T, H, FAKE, None, E, topk, ex, I, 3, FAKE, 0, None, None, None, None, None, FAKE,
+                               need, None, None) == q4.Q4_ERR_UNSUPPORTED

@@ -31,6 +31,8 @@ def q4():
     (3, 8192, 128, True),      # down projection width
     (1, 64, 64, False),        # a single group
     (8192, 2048, 128, False),  # a full gate projection
+    (300, 1024, 32, False),    # group 32 (the hottest MoE experts' tier), asymmetric
+    (64, 2048, 32, True),      # group 32, symmetric
 ])
 def test_quantize_bitexact(q4, n, k, group, sym):
     W = synth.weights(("test", "quant", n, k, group, sym), n, k)

@@ -61,6 +61,8 @@ def _run(q4, T, H, I, E, topk, group, sym, tag, skew=1.1, tokens=None, out=torch
     (37, 256, 256, 5, 3, 64, True),       # ragged token count, group 64, symmetric
     (16, 128, 128, 1, 1, 128, False),     # a single expert: a dense SwiGLU FFN
     (200, 512, 256, 64, 8, 128, False),   # the workload's expert count / top-8, skewed: some experts empty
+    (150, 256, 256, 6, 2, 32, False),     # group 32, asymmetric
+    (90, 512, 128, 4, 2, 32, True),       # group 32, symmetric
 ])
 def test_moe_small(q4, T, H, I, E, topk, group, sym):
     yn, ref, counts = _run(q4, T, H, I, E, topk, group, sym, f"s{T}-{E}")
@@ -221,6 +223,7 @@ def _run_classes(q4, T, H, I, E, topk, begin, params, tag, tokens=None):
     (200, 512, 256, 16, 4, [0, 2, 8, 16], [(64, True), (128, False), (64, False)]),
     (37, 256, 128, 5, 3, [0, 1, 5], [(64, False), (128, True)]),
     (300, 256, 128, 8, 2, [0, 8], [(128, False)]),          # one class = the plain layer
+    (256, 512, 256, 16, 4, [0, 1, 6, 16], [(32, False), (64, False), (128, False)]),   # the pages' three tiers
 ])
 def test_moe_classes(q4, T, H, I, E, topk, begin, params):
     yn, ref = _run_classes(q4, T, H, I, E, topk, begin, params, f"cls{T}-{E}")
@@ -228,9 +231,9 @@ def test_moe_classes(q4, T, H, I, E, topk, begin, params):
 
 
 def test_moe_classes_workload_full_size(q4):
-    """The 4096-token layer with the four most chosen experts (6 % of 64; expert 0 is the hottest under the
-    Zipf-skewed logits) quantized at group 64 and the other 60 at group 128, asymmetric."""
+    """The 4096-token layer in the pages' three tiers: the 3 most chosen experts (5 % of 64; expert 0 is the
+    hottest under the Zipf-skewed logits) at group 32, experts 3-31 at group 64, the rest at group 128."""
     tokens = np.arange(0, 4096, 173)
-    yn, ref = _run_classes(q4, 4096, 2048, 1024, 64, 8, [0, 4, 64], [(64, False), (128, False)], "clsfull",
-                           tokens=tokens)
+    yn, ref = _run_classes(q4, 4096, 2048, 1024, 64, 8, [0, 3, 32, 64], [(32, False), (64, False), (128, False)],
+                           "clsfull", tokens=tokens)
     assert_close(yn, ref, what="moe classes full")
