@@ -290,6 +290,25 @@ int moe_q4_forward_classes(const uint16_t* x, int32_t T, int32_t H,
                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * moe_q4_forward_range -- the part of the MoE layer that one range of experts contributes: the unit of
+ * expert parallelism.
+ * Source: "大模型之Dense、MoE与量化" 混合专家架构 MoE (the layer is a routing-weighted sum over experts, so
+ * it splits into per-expert terms); the W4A8 page §1 (spreading experts over devices trades memory for
+ * communication).
+ *   y[t] = sum over slots j with e_begin <= ids[t][j] < e_end of w[t][j] * o_(t,j)   (fp32, [T][H])
+ * Routing and the permutation are the whole layer's (every token is routed over all E experts);
+ * experts[3] = {gate [n*I][H], up [n*I][H], down [n*H][I]} stacked over the n = e_end - e_begin experts
+ * of the range.  Ranks that own disjoint ranges covering 0 .. E-1 and sum their y (an all-reduce) obtain
+ * moe_q4_forward's output.  0 <= e_begin < e_end <= E; group 32, 64 or 128; everything else as
+ * moe_q4_forward (fp32 output only, the workspace of moe_q4_workspace_size).
+ */
+int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H,
+                         const float* router_w, const float* router_bias, int32_t E, int32_t topk,
+                         int32_t e_begin, int32_t e_end, const q4_weight* experts, int32_t I, float* y,
+                         int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate device memory.
  * No counterpart in the source pages: this is a library convenience, not part of the method.
  *

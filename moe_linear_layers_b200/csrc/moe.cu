@@ -502,7 +502,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
                         int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
                         int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
                         size_t workspace_bytes, int32_t* dev_status, void* stream, int n_classes = 1,
-                        const int32_t* class_begin = nullptr);
+                        const int32_t* class_begin = nullptr, bool expert_range = false);
 
 extern "C" int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                               int32_t E, int32_t topk, const q4_weight* experts, int32_t I, void* y, int32_t out_dtype,
@@ -560,12 +560,25 @@ extern "C" int moe_q4_forward_classes(const uint16_t* x, int32_t T, int32_t H, c
                         n_classes, class_begin);
 }
 
+extern "C" int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H, const float* router_w,
+                                    const float* router_bias, int32_t E, int32_t topk, int32_t e_begin, int32_t e_end,
+                                    const q4_weight* experts, int32_t I, float* y, int32_t* topk_ids, float* topk_w,
+                                    int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (e_begin < 0 || e_end > E || e_begin >= e_end) return Q4_ERR_SHAPE;
+    const int32_t range[2] = {e_begin, e_end};
+    return forward_impl(x, T, H, router_w, router_bias, E, topk, experts, I, nullptr, 0, 0, y, Q4_OUT_F32, topk_ids,
+                        topk_w, perm, offsets, expert_counts, workspace, workspace_bytes, dev_status, stream, 1, range,
+                        true);
+}
+
 static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
                         int32_t E, int32_t topk, const q4_weight* experts, int32_t I, const q4_weight* shared,
                         int32_t I_shared, int a8_mask, void* y, int32_t out_dtype, int32_t* topk_ids, float* topk_w,
                         int32_t* perm, int32_t* offsets, int32_t* expert_counts, void* workspace,
                         size_t workspace_bytes, int32_t* dev_status, void* stream, int n_classes,
-                        const int32_t* class_begin)
+                        const int32_t* class_begin, bool expert_range)
 {
     if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
@@ -578,7 +591,11 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         n_classes = 1;
         class_begin = single;
     }
-    if (n_classes < 1 || n_classes > E || class_begin[0] != 0 || class_begin[n_classes] != E) return Q4_ERR_SHAPE;
+    // the classes cover every expert, or (expert_range) one contiguous range of them
+    if (n_classes < 1 || n_classes > E) return Q4_ERR_SHAPE;
+    if (expert_range ? (class_begin[0] < 0 || class_begin[n_classes] > E)
+                     : (class_begin[0] != 0 || class_begin[n_classes] != E))
+        return Q4_ERR_SHAPE;
     for (int c = 0; c < n_classes; c++) {
         const int Ec = class_begin[c + 1] - class_begin[c];
         if (Ec < 1) return Q4_ERR_SHAPE;

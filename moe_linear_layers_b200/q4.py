@@ -35,7 +35,8 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_q
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
-            "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes")
+            "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes",
+            "moe_q4_forward_range")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -74,6 +75,8 @@ _lib.moe_q4_forward_a8.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.PO
                                    _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_classes.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _i32, ctypes.POINTER(_i32),
                                         ctypes.POINTER(q4_weight), _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_forward_range.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _i32, _i32, ctypes.POINTER(q4_weight), _i32,
+                                      _p, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -330,6 +333,49 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
            "moe_q4_forward_classes")
     if want_routing:
         return y, ids, wts, perm, offs, cnts
+    return y
+
+
+def moe_q4_forward_range(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                         e_begin: int, e_end: int, experts: tuple, I: int, y: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """The contribution of experts e_begin .. e_end-1 (weights stacked over that range) to the MoE layer,
+    fp32 [T][H]; disjoint ranges covering every expert sum to the layer."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _dev(y, torch.float32, "y")
+    if workspace is None:
+        workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=x.device)
+    descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _check(_lib.moe_q4_forward_range(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, e_begin, e_end, descs,
+                                     I, _ptr(y), None, None, None, None, None, _ptr(workspace), workspace.numel(),
+                                     _ptr(dev_status), _stream(stream)), "moe_q4_forward_range")
+    return y
+
+
+def expert_range(rank: int, world: int, E: int) -> tuple:
+    """The experts rank `rank` of `world` owns under expert parallelism: a contiguous, near-equal split."""
+    return (rank * E) // world, ((rank + 1) * E) // world
+
+
+def moe_q4_forward_expert_parallel(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None,
+                                   topk: int, local_experts: tuple, I: int, group=None, range_fn=None,
+                                   **kw) -> torch.Tensor:
+    """Expert-parallel MoE layer: this rank holds the weights of expert_range(rank, world, E) only; every
+    rank routes the same tokens, computes its experts' contribution and the contributions are summed by an
+    all-reduce (fp32) over `group` (torch.distributed; NCCL on GPUs).  range_fn replaces
+    moe_q4_forward_range (tests on CPU ranks)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    e0, e1 = expert_range(rank, world, router_w.shape[0])
+    y = (range_fn or moe_q4_forward_range)(x, router_w, router_bias, topk, e0, e1, local_experts, I, **kw)
+    dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
     return y
 
 

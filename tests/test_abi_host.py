@@ -159,3 +159,20 @@ def test_moe_group32_only_on_the_16bit_path():
     need = L.moe_q4_workspace_size_a8(T, H, I, E, topk, 3)
     assert L.moe_q4_forward_a8(FAKE, T, H, FAKE, None, E, topk, ex, I, 3, FAKE, 0, None, None, None, None, None, FAKE,
                                need, None, None) == q4.Q4_ERR_UNSUPPORTED
+
+
+def test_moe_range_validation():
+    L = q4._lib
+    T, H, I, E, topk = 64, 256, 128, 8, 2
+    ws = L.moe_q4_workspace_size(T, H, I, E, topk)
+    ex3 = (q4.q4_weight * 3)(_w(n=3 * I, k=H), _w(n=3 * I, k=H), _w(n=3 * H, k=I))
+
+    def call(e0, e1, ex=ex3, wsb=ws):
+        return L.moe_q4_forward_range(FAKE, T, H, FAKE, None, E, topk, e0, e1, ex, I, FAKE, None, None, None, None,
+                                      None, FAKE, wsb, None, None)
+
+    assert call(3, 3) == q4.Q4_ERR_SHAPE          # empty range
+    assert call(6, 9) == q4.Q4_ERR_SHAPE          # past the last expert
+    assert call(-1, 2) == q4.Q4_ERR_SHAPE
+    assert call(2, 4) == q4.Q4_ERR_SHAPE          # 2 experts, weights stacked for 3
+    assert call(2, 5, wsb=ws - 1) == q4.Q4_ERR_WORKSPACE

@@ -237,3 +237,47 @@ def test_moe_classes_workload_full_size(q4):
     yn, ref = _run_classes(q4, 4096, 2048, 1024, 64, 8, [0, 3, 32, 64], [(32, False), (64, False), (128, False)],
                            "clsfull", tokens=tokens)
     assert_close(yn, ref, what="moe classes full")
+
+
+# ---------------------------------------------------------------------------------------------- #
+# expert ranges (moe_q4_forward_range): the unit of expert parallelism
+# ---------------------------------------------------------------------------------------------- #
+
+def test_moe_expert_ranges_sum_to_the_layer(q4):
+    T, H, I, E, topk, group, sym = 300, 512, 256, 16, 4, 128, False
+    tag = "ranges"
+    x = synth.activations(("moe", tag, "x"), T, H)
+    Wr, bias = synth.router(("moe", tag), E, H, skew=1.1)
+    qs = _experts(tag, E, H, I, group, sym)
+    _, ids, w, _ = oracle.route(x, H, Wr, bias, topk)
+    xd = cuda_u16_as(x, torch.bfloat16)
+    Wrd, bd = torch.from_numpy(Wr).cuda(), torch.from_numpy(bias).cuda()
+    full = q4.moe_q4_forward(xd, Wrd, bd, topk, tuple(upload_weight(q4, *q, n, k, group, sym) for q, n, k in
+                                                     zip(qs, (E * I, E * I, E * H), (H, H, I))), I)
+
+    def sliced(e0, e1):
+        out = []
+        for (pk, sc, zr), rows, k in zip(qs, (I, I, H), (H, H, I)):
+            sl = slice(e0 * rows, e1 * rows)
+            out.append(upload_weight(q4, pk[sl], sc[sl], None if zr is None else zr[sl], (e1 - e0) * rows, k, group, sym))
+        return tuple(out)
+
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for world in (2, 4, 5):
+        parts = []
+        for r in range(world):
+            e0, e1 = q4.expert_range(r, world, E)
+            parts.append(q4.moe_q4_forward_range(xd, Wrd, bd, topk, e0, e1, sliced(e0, e1), I, dev_status=st))
+            if r == 1:   # one range against the oracle over the slots routed into it
+                mine = (ids >= e0) & (ids < e1)
+                ref = oracle.moe_experts(x, H, np.where(mine, ids - e0, 0).astype(np.int32), np.where(mine, w, 0.0),
+                                         *[(pk[e0 * rows:e1 * rows], sc[e0 * rows:e1 * rows],
+                                            None if zr is None else zr[e0 * rows:e1 * rows])
+                                           for (pk, sc, zr), rows in zip(qs, (I, I, H))], I, group, sym)
+                torch.cuda.synchronize()
+                assert_close(parts[-1].cpu().numpy(), ref, what=f"range {e0}-{e1}")
+        total = sum(parts)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        d = (total - full).abs().max().item() / full.pow(2).mean().sqrt().item()
+        assert d <= 1e-5, f"ranges of {world} ranks differ from the layer by {d:.2e} of rms"
