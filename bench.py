@@ -294,9 +294,18 @@ def run_decode(q4, args, ws, weights, dev):
     h2d = hx.numel() * hx.element_size()
     d2h = hy.numel() * hy.element_size()
 
+    # the calls prepared once (q4.GroupedGemv: the argument arrays of q4_linear_w4a16_grouped built ahead,
+    # one problem for o and down), as a decode loop that serves many steps would hold them
+    calls_e2e = []
+    for l in range(synth.LLAMA_1B_LAYERS):
+        b = 7 * l
+        for idx in ((b, b + 1, b + 2), (b + 3,), (b + 4, b + 5), (b + 6,)):
+            calls_e2e.append(q4.GroupedGemv([xs[i] for i in idx], [weights[i] for i in idx], [ys[i] for i in idx]))
+
     def e2e_step():
         x_all.copy_(hx, non_blocking=True)
-        step()
+        for c in calls_e2e:
+            c()
         hy.copy_(y_all, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -340,8 +349,8 @@ def run_decode(q4, args, ws, weights, dev):
                                "bytes per launch / mean launch duration (graph replay, gaps included)",
                      "mean_launch_us": round(1e3 * ms_step / len(calls), 3)},
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "eager public-API calls (64 per step); all x of the step copied in from pinned host memory "
-                       "and all y copied back to pinned host memory every step"},
+                "how": "eager public-API calls (64 prepared q4.GroupedGemv calls per step); all x of the step copied "
+                       "in from pinned host memory and all y copied back to pinned host memory every step"},
         "gpu_launches": len(calls) * args.steps,
         "clocks": clk.summary(),
     }

@@ -99,9 +99,18 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_current_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    """The cudaStream_t handle of `stream`, or of torch's current stream on the current device (looked up
+    without building a Stream object: a decode step makes dozens of calls, each paying this)."""
+    if stream is None:
+        if _raw_current_stream is not None and _current_device is not None:
+            return _raw_current_stream(_current_device())
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
 
 
 def _dev(t, dtype, name):
