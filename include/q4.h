@@ -190,28 +190,6 @@ int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_w
                    int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream);
 
 /*
- * q4_linear_workspace_size / q4_linear_w4a16_ws / q4_linear_w4a8_ws -- the linear layers with a caller
- * workspace that lets the tensor-core GEMM split K when the output has too few 128 x 128 tiles to
- * occupy the GPU (small m: e.g. m = 64 with n = 2048 gives 16 tiles for 148 SMs).  No counterpart in the
- * source pages: the arithmetic is q4_linear_w4a16's / q4_linear_w4a8's; only the summation of the
- * per-group terms is cut into K ranges whose fp32 partial sums are added in range order (the result
- * does not depend on which range finishes last).
- *   workspace: NULL (no split: exactly q4_linear_w4a16 / q4_linear_w4a8), or device memory of at least
- *   q4_linear_workspace_size(m, w) bytes, 256-byte aligned, owned by the caller; its first 512 bytes
- *   (tile counters, at the same place for every shape) must be zero before the first call — zero-fill
- *   the buffer once — and every call that completes leaves them zero again, so one workspace of the
- *   largest size needed serves every shape.  After a call that reported an error through dev_status,
- *   zero it again.  Calls that share a workspace must not run concurrently.
- * q4_linear_workspace_size returns 0 when the shape is not split (the workspace is then ignored).
- */
-size_t q4_linear_workspace_size(int32_t m, const q4_weight* w);
-int q4_linear_w4a16_ws(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
-                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
-int q4_linear_w4a8_ws(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
-                      int32_t out_dtype, int32_t* acc_dbg, void* workspace, size_t workspace_bytes,
-                      int32_t* dev_status, void* stream);
-
-/*
  * moe_q4_workspace_size -- bytes of device workspace moe_q4_forward needs for these sizes.
  */
 size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk);

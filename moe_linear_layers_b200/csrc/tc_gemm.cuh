@@ -118,12 +118,6 @@ struct Args {
     const float* row_w;            // Down: [P] routing weight of each permuted row
     __half* h;                     // GateUp output [P][N]
     int E, topk;
-    // Dense split-K (splits > 1): split s of a tile covers K stages [s*sps, min((s+1)*sps, K/128)) and
-    // stores its fp32 partial sums in ws [splits][M][N]; the split that completes a tile's count in
-    // tile_ctr adds the partials in split order (deterministic), writes y and sets the counter back to 0
-    int splits, sps;
-    float* ws;
-    int32_t* tile_ctr;
 };
 
 struct Tile {
@@ -131,8 +125,6 @@ struct Tile {
     int n0;           // Dense/Down: first weight row of the tile inside the (expert) matrix; GateUp: i0
     int wrow_a, wrow_b;  // packed rows of the TMA boxes
     int e;
-    int kb0, kb1;     // K stages of this work item (all of them unless split-K)
-    int tile, split;  // Dense: output tile index and split (split-K bookkeeping)
 };
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr)
@@ -224,8 +216,6 @@ struct Shared {
     int expert_tiles[kMaxExperts + 1];
     int comb_tok[8 * 64];      // Down: token of each activation row of the tile, per epilogue warp
     float comb_w[8 * 64];      // Down: its routing weight
-    uint32_t out_done[8];      // split-K: work items whose partials an epilogue warp has added
-    uint32_t fix_seq, fix_last;  // split-K: decision of warp 12 whether this CTA finishes the tile
 };
 static_assert(sizeof(Shared) <= 6144, "Shared must fit the space reserved in Cfg::SMEM");
 
@@ -234,18 +224,7 @@ template <Mode MODE>
 __device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
 {
     Tile T;
-    T.kb0 = 0;
-    T.kb1 = p.K / KBLK;
-    T.tile = 0;
-    T.split = 0;
     if constexpr (MODE == Mode::Dense) {
-        if (p.splits > 1) {   // work item t = (tile, split), splits of a tile adjacent
-            T.split = t % p.splits;
-            t /= p.splits;
-            T.kb0 = T.split * p.sps;
-            T.kb1 = min(T.kb1, T.kb0 + p.sps);
-        }
-        T.tile = t;
         T.e = 0;
         T.m0 = (t % tiles_m) * BN;
         T.m_end = p.M;
@@ -300,7 +279,7 @@ struct QuadRing {
     uint2 cur, nxt, pre;
     __device__ __forceinline__ void preload(const __half* r, int count)
     {
-        pre_row = (r && (count & 3) == 0 && ((uintptr_t)r & 7) == 0) ? r : nullptr;
+        pre_row = (r && (count & 3) == 0) ? r : nullptr;
         if (pre_row) pre = __ldg(reinterpret_cast<const uint2*>(r));
     }
     __device__ __forceinline__ void start(const __half* r, int count)
@@ -308,13 +287,12 @@ struct QuadRing {
         row = r;
         n = count;
         cur = nxt = make_uint2(0u, 0u);
-        if (row && (n & 3) == 0 && ((uintptr_t)row & 7) == 0) nxt = row == pre_row ? pre : __ldg(reinterpret_cast<const uint2*>(row));
-        else if (row) n = n | 0x40000000;   // unaligned start (a split-K slice of the row): direct loads
+        if (row && (n & 3) == 0) nxt = row == pre_row ? pre : __ldg(reinterpret_cast<const uint2*>(row));
     }
     __device__ __forceinline__ float get(int i)   // positions in increasing order, from 0
     {
         if (!row) return 0.0f;
-        if (n & 0x40000003) return __half2float(row[i]);
+        if (n & 3) return __half2float(row[i]);
         if ((i & 3) == 0) {
             cur = nxt;
             nxt = i + 4 < n ? __ldg(reinterpret_cast<const uint2*>(row + i + 4)) : make_uint2(0u, 0u);
@@ -379,15 +357,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         }
         for (int i = 0; i < C::ND; i++) tc::mbar_init(&sh->d_full[i], 1);
         for (int i = 0; i < 4; i++) sh->conv_done[i] = 0;
-        for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = sh->out_done[i] = 0;
-        sh->fix_seq = sh->fix_last = 0;
+        for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
         tc::mbar_init(&sh->done, kIssuers);
         // consumers: the converters, and the epilogue unless it is W4A8's
         for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->p_full[i], 32); tc::mbar_init(&sh->p_empty[i], INT8 ? 4 : 4 + 8); }
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
-        if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM) * max(p.splits, 1);
+        if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
         else sh->total_tiles = p.expert_tiles[p.E] - p.expert_tiles[0];
         tc::fence_mbar_init();
     }
@@ -419,7 +396,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-                for (int kb = T.kb0; kb < T.kb1; kb++, it++) {
+                for (int kb = 0; kb < kblocks; kb++, it++) {
                     if ((it & 1u) != parity) continue;
                     const int s = it % NS;
                     if (!(ok = tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag))) break;
@@ -449,11 +426,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // -------------------------------------------------------------- parameter loader (warp 10)
             // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
             // ahead of the converters and the epilogue, so that their loops make no global loads.
+            const int nwin = (ngroups + PW - 1) / PW;
             uint32_t wi = 0;
             for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-                const int g_first = T.kb0 * GPK, ng_t = (T.kb1 - T.kb0) * GPK;   // this work item's groups
-                const int nwin = (ng_t + PW - 1) / PW;
                 for (int w = 0; w < nwin; w++, wi++) {
                     if (!tc::mbar_wait(&sh->p_empty[wi & 1], ((wi >> 1) & 1) ^ 1, p.status, abort_flag)) goto load_done;
                     __half* ps = params + (wi & 1) * C::PTENS * PW * BM;
@@ -462,8 +438,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         const int r = 32 * i + lane;
                         const __half *srow, *zrow;
                         row_params<MODE>(p, T, r, ngroups, srow, zrow);
-                        stage_params(srow ? srow + g_first : nullptr, w * PW, ng_t, ps + r);
-                        if constexpr (!SYM) stage_params(zrow ? zrow + g_first : nullptr, w * PW, ng_t, ps + PW * BM + r);
+                        stage_params(srow, w * PW, ngroups, ps + r);
+                        if constexpr (!SYM) stage_params(zrow, w * PW, ngroups, ps + PW * BM + r);
                     }
                     tc::mbar_arrive(&sh->p_full[wi & 1]);   // every lane: its stores are visible
                 }
@@ -482,12 +458,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             bool ok = true;
             if constexpr (INT8) ok = tc::poll_counters<8>(sh->epi_init, 1, p.status, abort_flag);
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                int nkb = kblocks;
-                if constexpr (MODE == Mode::Dense) {
-                    const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-                    nkb = T.kb1 - T.kb0;
-                }
-                for (int kb = 0; kb < nkb && ok; kb++, it++) {
+                for (int kb = 0; kb < kblocks && ok; kb++, it++) {
                     if (it % kIssuers != (uint32_t)warp) {   // another issuer's stage
                         g += GPK;
                         continue;
@@ -531,13 +502,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         constexpr float kMagic = F16 ? 1024.0f : 128.0f;
         uint32_t it = 0, wi = 0;   // stage and parameter-window counters (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            int nkb = kblocks;
-            if constexpr (MODE == Mode::Dense) {
-                const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-                nkb = T.kb1 - T.kb0;
-            }
-            const int ng_t = nkb * GPK;   // groups of this work item
-            for (int kb = 0; kb < nkb; kb++) {
+            for (int kb = 0; kb < kblocks; kb++) {
                 const int s = it % NS, sa = it % NA;
                 // zero points of the stage's groups from the parameter ring
                 float zcur[GPK];
@@ -549,7 +514,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
-                    if ((g0 + GPK) % PW == 0 || g0 + GPK >= ng_t) {   // the window's last stage: release it
+                    if ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups) {   // the window's last stage: release it
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
                         wi++;
@@ -646,16 +611,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         QuadRing sr;       // W4A8: group scales read a few groups ahead
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-            const int g_first = T.kb0 * GPK, ng_t = (T.kb1 - T.kb0) * GPK;   // this work item's groups
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
             if constexpr (INT8) {
-                sr.start(srow ? srow + g_first : nullptr, ng_t);
+                sr.start(srow, ngroups);
                 if (t + (int)gridDim.x < total) {   // load the next tile's first block of scales now
                     const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
                     const __half *sn, *zn;
                     row_params<MODE>(p, Tn, r, ngroups, sn, zn);
-                    sr.preload(sn ? sn + Tn.kb0 * GPK : nullptr, (Tn.kb1 - Tn.kb0) * GPK);
+                    sr.preload(sn, ngroups);
                 }
             }
 #pragma unroll
@@ -671,7 +635,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     comb_w[ew * 64 + j] = cw;
                 }
             }
-            for (int gl = 0; gl < ng_t; gl++) {
+            for (int gl = 0; gl < ngroups; gl++) {
                 const uint32_t db = g % C::ND;
                 // group scale: W4A8 from its read-ahead ring, 16-bit modes from the parameter ring
                 float s;
@@ -680,7 +644,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 } else {
                     if (gl % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto epi_done;
                     s = __half2float(params[(wi & 1) * C::PTENS * PW * BM + (gl % PW) * BM + r]);
-                    if ((gl + 1) % PW == 0 || gl + 1 == ng_t) {   // the window's last group: release it
+                    if ((gl + 1) % PW == 0 || gl + 1 == ngroups) {   // the window's last group: release it
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
                         wi++;
@@ -702,7 +666,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
                                 if (m < T.m_end)
-                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + g_first + gl] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
+                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
                             }
                         }
                         const uint64_t nb2 = tc::f2_pack(__float_as_uint(-kAccBiasF), __float_as_uint(-kAccBiasF));
@@ -729,56 +693,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // ---------------------------------------------------------- tile output
             // (every loop below has a branch-free path for a full 64-row block: a conditional branch per
             // row costs more than the store it guards)
-            if (MODE == Mode::Dense && p.splits > 1) {
-                // split-K: store this split's partial (times the row's activation scale for W4A8) in ws
-                const int n = T.n0 + r;
-                const int mb = T.m0 + half * 64;
-                const int rows = min(64, p.M - mb);
-                if (n < p.N && rows > 0) {
-                    float* wr = p.ws + ((int64_t)T.split * p.M + mb) * p.N + n;
-#pragma unroll
-                    for (int j = 0; j < 64; j++)
-                        if (j < rows) {
-                            float v = accv(j);
-                            if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
-                            __stcg(wr + (int64_t)j * p.N, v);
-                        }
-                }
-                // every epilogue warp's stores are visible device-wide before warp 12 counts this split in;
-                // the split that completes the count sums the partials and writes y
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) tc::sts_volatile(&sh->out_done[ew], tl + 1);
-                if (ew == 0 && lane == 0) {
-                    uint32_t last = 0;
-                    if (tc::poll_volatile(sh->out_done, 8, tl + 1, p.status, abort_flag)) {
-                        __threadfence();
-                        last = atomicAdd(p.tile_ctr + T.tile, 1) == p.splits - 1;
-                        if (last) {
-                            __threadfence();
-                            atomicExch(p.tile_ctr + T.tile, 0);
-                        }
-                    }
-                    tc::sts_volatile(&sh->fix_seq, 2 * (tl + 1) + last);
-                }
-                __syncwarp();
-                if (!tc::poll_volatile(&sh->fix_seq, 1, 2 * (tl + 1), p.status, abort_flag)) goto epi_done;
-                if (tc::lds_volatile(&sh->fix_seq) & 1u) {
-                    __threadfence();
-                    if (n < p.N && rows > 0) {
-                        const int64_t split_stride = (int64_t)p.M * p.N;
-                        const float* wr = p.ws + (int64_t)mb * p.N + n;
-                        for (int j = 0; j < rows; j++) {
-                            float v = 0.0f;
-                            for (int sp = 0; sp < p.splits; sp++) v += __ldcg(wr + sp * split_stride + (int64_t)j * p.N);
-                            if (p.out_bf16)
-                                reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)(mb + j) * p.N + n] = __float2bfloat16_rn(v);
-                            else
-                                reinterpret_cast<float*>(p.y)[(int64_t)(mb + j) * p.N + n] = v;
-                        }
-                    }
-                }
-            } else if constexpr (MODE == Mode::Dense) {
+            if constexpr (MODE == Mode::Dense) {
                 const int n = T.n0 + r;
                 const int mb = T.m0 + half * 64;
                 const int rows = min(64, p.M - mb);

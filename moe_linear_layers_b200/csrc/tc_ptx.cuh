@@ -300,32 +300,6 @@ __device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uin
     }
 }
 
-// Volatile (relaxed, morally strong) shared-memory word access, for hand-offs that carry data between
-// warps that are not MMA issuers (a weak load suffices for the issuers' progress counters, whose
-// consumers then order through tcgen05 fences).
-__device__ __forceinline__ void sts_volatile(uint32_t* p, uint32_t v) { *reinterpret_cast<volatile uint32_t*>(p) = v; }
-__device__ __forceinline__ uint32_t lds_volatile(const uint32_t* p) { return *reinterpret_cast<const volatile uint32_t*>(p); }
-
-// Spin until each of the n words at c is >= target (volatile loads); bounded like poll_counters_slow.
-__device__ __forceinline__ bool poll_volatile(const uint32_t* c, int n, uint32_t target, int32_t* status,
-                                              volatile int* abort_flag, uint64_t limit_ns = 2000000000ull)
-{
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t round = 0;; round++) {
-        bool ok = true;
-        for (int i = 0; i < n; i++) ok &= lds_volatile(c + i) >= target;
-        if (ok) return true;
-        if ((round & 63u) == 63u) {
-            if (abort_flag && *abort_flag) return false;
-            if (wait_expired(t0, limit_ns, round, 1u << 16)) {
-                q4_set_status(status, Q4_ERR_TIMEOUT);
-                if (abort_flag) *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-}
-
 template <int N>
 __device__ __forceinline__ bool poll_counters(const uint32_t* c, uint32_t target, int32_t* status,
                                               volatile int* abort_flag)

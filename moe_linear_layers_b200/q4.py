@@ -36,7 +36,7 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_q
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
             "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes",
-            "moe_q4_forward_range", "q4_linear_workspace_size", "q4_linear_w4a16_ws", "q4_linear_w4a8_ws")
+            "moe_q4_forward_range")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -58,10 +58,6 @@ _lib.q4_linear_w4a16_swiglu.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight),
 _lib.q4_linear_w4a16_grouped.argtypes = [_i32, ctypes.POINTER(_p), _i32, ctypes.POINTER(q4_weight),
                                          ctypes.POINTER(_p), _i32, _p, _p]
 _lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
-_lib.q4_linear_workspace_size.restype = _sz
-_lib.q4_linear_workspace_size.argtypes = [_i32, ctypes.POINTER(q4_weight)]
-_lib.q4_linear_w4a16_ws.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _sz, _p, _p]
-_lib.q4_linear_w4a8_ws.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _sz, _p, _p]
 _lib.act_quant_per_token_f16.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
 _lib.q4_linear_w4a8.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _p]
 _lib.moe_q4_workspace_size.restype = _sz
@@ -164,41 +160,16 @@ def q4_quantize_pack(w: torch.Tensor, group: int, symmetric: bool, dev_status: t
     return q
 
 
-_gemm_ws = {}   # device index -> zero-initialised split-K workspace (grown on demand)
-
-
-def linear_workspace(m: int, w: "Q4Weight", device) -> torch.Tensor | None:
-    """A workspace for q4_linear_w4a16_ws / q4_linear_w4a8_ws of this shape, shared per device (calls
-    using it must stay on one stream), or None when the shape is not split."""
-    need = int(_lib.q4_linear_workspace_size(m, ctypes.byref(w.desc)))
-    if need == 0:
-        return None
-    dev = torch.device(device)
-    key = dev.index if dev.index is not None else torch.cuda.current_device()
-    t = _gemm_ws.get(key)
-    if t is None or t.numel() < need:
-        t = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=dev)
-        _gemm_ws[key] = t
-    return t
-
-
 def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: torch.Tensor | None = None,
-                    dev_status: torch.Tensor | None = None, stream=None, workspace="auto") -> torch.Tensor:
-    """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor.  workspace: "auto" (the per-device split-K
-    workspace when the shape splits), None (no split) or a caller tensor."""
+                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor."""
     _dev(x, torch.bfloat16, "x")
     m = x.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
     od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
-    if isinstance(workspace, str):
-        workspace = linear_workspace(m, w, x.device) if m > 4 else None
-    if workspace is None:
-        _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status),
-                                    _stream(stream)), "q4_linear_w4a16")
-    else:
-        _check(_lib.q4_linear_w4a16_ws(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(workspace),
-                                       workspace.numel(), _ptr(dev_status), _stream(stream)), "q4_linear_w4a16_ws")
+    _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
+           "q4_linear_w4a16")
     return y
 
 
@@ -263,24 +234,16 @@ def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a
 
 def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dtype=torch.float32,
                    y: torch.Tensor | None = None, acc_dbg: torch.Tensor | None = None,
-                   dev_status: torch.Tensor | None = None, stream=None, workspace="auto") -> torch.Tensor:
-    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . (code - zero))_g; zero = 0 for symmetric W.
-    workspace as in q4_linear_w4a16."""
+                   dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . (code - zero))_g; zero = 0 for symmetric W."""
     _dev(xq, torch.int8, "xq")
     _dev(scale_a, torch.float32, "scale_a")
     m = xq.shape[0]
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
     od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
-    if isinstance(workspace, str):
-        workspace = linear_workspace(m, w, xq.device)
-    if workspace is None:
-        _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
-                                   _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
-    else:
-        _check(_lib.q4_linear_w4a8_ws(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
-                                      _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
-               "q4_linear_w4a8_ws")
+    _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
+                               _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
     return y
 
 

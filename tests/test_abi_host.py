@@ -176,15 +176,3 @@ def test_moe_range_validation():
     assert call(-1, 2) == q4.Q4_ERR_SHAPE
     assert call(2, 4) == q4.Q4_ERR_SHAPE          # 2 experts, weights stacked for 3
     assert call(2, 5, wsb=ws - 1) == q4.Q4_ERR_WORKSPACE
-
-
-def test_linear_workspace_entry_points():
-    L = q4._lib
-    w = _w(n=2048, k=2048, group=128, sym=1)
-    assert L.q4_linear_workspace_size(64, w) > 64 * 2048 * 4          # split: partials of several K ranges
-    assert L.q4_linear_workspace_size(4096, w) == 0                   # 512 tiles: never split
-    need = L.q4_linear_workspace_size(64, w)
-    assert L.q4_linear_w4a16_ws(FAKE, 64, w, FAKE, 0, FAKE, need - 1, None, None) == q4.Q4_ERR_WORKSPACE
-    assert L.q4_linear_w4a16_ws(FAKE, 64, w, FAKE, 0, FAKE + 16, need, None, None) == q4.Q4_ERR_ALIGN
-    assert L.q4_linear_w4a8_ws(FAKE, FAKE, 64, w, FAKE, 0, None, FAKE, need - 1, None, None) == q4.Q4_ERR_WORKSPACE
-    assert L.q4_linear_w4a16_ws(None, 64, w, FAKE, 0, None, 0, None, None) == q4.Q4_ERR_NULL

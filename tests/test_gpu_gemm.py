@@ -115,58 +115,3 @@ def test_w4a8_asym_workload_shapes(q4, m, n, k):
     rows = np.arange(0, m, max(1, m // 32))
     ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, 128, rows_m=rows, zeros=zr, symmetric=False)
     assert_close(y.cpu().numpy()[rows], ref, what=f"w4a8 asym {m}x{n}x{k}")
-
-
-# ---------------------------------------------------------------------------------------------- #
-# split-K (q4_linear_*_ws): few output tiles, K cut into ranges whose partials meet in the workspace
-# ---------------------------------------------------------------------------------------------- #
-
-@pytest.mark.parametrize("m,n,k,group,sym", [
-    (64, 2048, 8192, 128, False),     # down-projection shape at m = 64: 16 tiles, 64 K stages
-    (33, 512, 2048, 64, True),        # ragged m, 4 tiles
-    (130, 256, 1024, 128, False),     # two m tiles, ragged
-])
-def test_w4a16_split_k(q4, m, n, k, group, sym):
-    from moe_linear_layers_b200 import q4 as mod
-    yn, ref, w, xd, y = _w4a16(q4, m, n, k, group, sym, tag="splitk")
-    assert mod._lib.q4_linear_workspace_size(m, w.desc) > 0, "this shape should split"
-    assert_close(yn, ref, what=f"split-K {m}x{n}x{k}")
-    y0 = q4.q4_linear_w4a16(xd, w, workspace=None)           # the unsplit kernel
-    y2 = q4.q4_linear_w4a16(xd, w)                           # split again: same bits (fixed summation order)
-    y16 = q4.q4_linear_w4a16(xd, w, out_dtype=torch.bfloat16)
-    torch.cuda.synchronize()
-    assert torch.equal(y2, y)
-    assert_close(y0.cpu().numpy(), ref, what="unsplit")
-    assert np.array_equal(cpu_u16(y16), bf16_rne(y.cpu().numpy()))
-
-
-@pytest.mark.parametrize("m,n,k,group,sym", [(16, 2048, 2048, 128, True), (64, 256, 2048, 64, False)])
-def test_w4a8_split_k_partials_bitexact(q4, m, n, k, group, sym):
-    y, acc, (xq, sa, pk, sc, zr), w, xqd, sad = _w4a8(q4, m, n, k, group, "splitk", want_acc=True, sym=sym)
-    assert q4._lib.q4_linear_workspace_size(m, w.desc) > 0, "this shape should split"
-    ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True,
-                                      zeros=None if sym else zr, symmetric=sym)
-    assert np.array_equal(acc.cpu().numpy(), acc_ref)
-    assert_close(y.cpu().numpy(), ref, what="w4a8 split-K")
-
-
-def test_split_k_workspace_contract(q4):
-    from moe_linear_layers_b200.q4 import Q4Error, Q4_ERR_WORKSPACE
-    m, n, k = 64, 2048, 2048
-    yn, ref, w, xd, y = _w4a16(q4, m, n, k, 128, False, tag="ws")
-    need = q4._lib.q4_linear_workspace_size(m, w.desc)
-    small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
-    with pytest.raises(Q4Error) as ei:
-        q4.q4_linear_w4a16(xd, w, workspace=small)
-    assert ei.value.status == Q4_ERR_WORKSPACE
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    for _ in range(3):                                       # the counters come back to zero every call
-        y1 = q4.q4_linear_w4a16(xd, w, workspace=ws)
-    torch.cuda.synchronize()
-    assert torch.equal(y1, y)
-    assert int(ws[:512].view(torch.int32).abs().sum().item()) == 0   # the tile counters (offset 0)
-    # the same workspace serves another split shape afterwards (the counters stay where they are)
-    yb, refb, wb, xb, _ = _w4a16(q4, 40, 640, 1024, 64, True, tag="ws2")
-    yb2 = q4.q4_linear_w4a16(xb, wb, workspace=ws)
-    torch.cuda.synchronize()
-    assert_close(yb2.cpu().numpy(), refb, what="reused workspace")
