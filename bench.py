@@ -376,7 +376,7 @@ def run_prefill(q4, args, weights, dev, m=2048):
     tf = flops / (ms * 1e-3) / 1e12
     peaks = load_peaks()
     return {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 3), "m": m,
-            "workload": "W4A16 GEMM over the 112 decode-step matrices at m=2048, x with 1% channels x10, bf16 out",
+            "workload": f"W4A16 GEMM over the 112 decode-step matrices at m={m}, x with 1% channels x10, bf16 out",
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
                          "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4),
@@ -409,11 +409,30 @@ def run_w4a8(q4, args, weights_sym, dev, m=4096):
     int8_peak = 2 * peaks["bf16_tflops_sustained"]
     return {"value": round(tops, 1), "unit": "TOPS", "ms_per_step": round(ms, 3), "m": m,
             "workload": "per-token INT8 act-quant + W4A8 GEMM over the 112 matrices (symmetric INT4 g128), "
-                        "m=4096, Student-t(3) activations, bf16 out; act-quant time included",
+                        f"m={m}, Student-t(3) activations, bf16 out; act-quant time included",
             "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
                          "frac": round(tops / int8_peak, 4),
                          "peak_source": peaks["source"] + " bf16 sustained x 2 (nominal int8:bf16 dense ratio)"},
             "gpu_launches": 2 * len(layers) * steps, "clocks": clk.summary()}
+
+
+def with_attainable(r, m, a8: bool):
+    """Adds the bound that the step's bytes put on a small-m GEMM: attainable = min(tensor peak, HBM
+    bandwidth x arithmetic intensity), bytes = packed weights + scales (+ zeros) + activations in + bf16
+    out, over the 112 matrices."""
+    layers = decode_layers()
+    peaks = load_peaks()
+    g = 128
+    wbytes = sum(n * k // 2 + n * (k // g) * 2 * (1 if a8 else 2) for (_, n, k) in layers)
+    abytes = sum(m * k * (1 if a8 else 2) + (4 * m if a8 else 0) + 2 * m * n for (_, n, k) in layers)
+    ops = 2 * m * sum(n * k for (_, n, k) in layers)
+    inten = ops / (wbytes + abytes)
+    peak = r["roofline"]["peak"]
+    attain = min(peak, peaks["hbm_gbs"] * inten / 1e3)
+    r["roofline"].update({"bytes_per_step": wbytes + abytes, "intensity_ops_per_byte": round(inten, 1),
+                          "attainable": round(attain, 1), "frac_of_attainable": round(r["value"] / attain, 4),
+                          "bound_at_this_m": "hbm" if attain < peak else "tensor"})
+    return r
 
 
 def build_moe(q4, dev, seed=0):
@@ -676,6 +695,11 @@ def main():
     if components:
         line["components"] = {"prefill_w4a16_m2048": run_prefill(q4, args, asym, dev),
                               "w4a8_m4096": run_w4a8(q4, args, sym, dev)}
+        # the other token counts of the prefill and W4A8 workloads, each against the bound its bytes set
+        for m in (64, 512):
+            line["components"][f"prefill_w4a16_m{m}"] = with_attainable(run_prefill(q4, args, asym, dev, m=m), m, False)
+        for m in (16, 256):
+            line["components"][f"w4a8_m{m}"] = with_attainable(run_w4a8(q4, args, sym, dev, m=m), m, True)
         del sym
         torch.cuda.empty_cache()
         line["components"]["moe_layer"] = run_moe(q4, args, dev)
