@@ -45,3 +45,27 @@ def test_decode_bytes_per_step():
     assert sum(n * k for (_, n, k) in layers) // 2 == 486539264
     b = bench.decode_bytes(layers)
     assert 0.5e9 < b < 0.53e9
+
+
+def test_small_m_attainable_bound(monkeypatch):
+    """The bound a small-m GEMM's bytes set: min(tensor peak, HBM bandwidth x ops per byte)."""
+    monkeypatch.setattr(bench, "load_peaks", lambda: {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0,
+                                                      "bf16_tflops_sustained": 1400.0, "source": "test"})
+    layers = bench.decode_layers()
+    ops = 2 * 64 * sum(n * k for (_, n, k) in layers)
+    r = bench.with_attainable({"value": 50.0, "roofline": {"peak": 1400.0}}, 64, False)
+    rf = r["roofline"]
+    wbytes = sum(n * k // 2 + n * (k // 128) * 4 for (_, n, k) in layers)
+    abytes = sum(64 * k * 2 + 2 * 64 * n for (_, n, k) in layers)
+    assert rf["bytes_per_step"] == wbytes + abytes
+    assert abs(rf["attainable"] - min(1400.0, 6000.0 * ops / (wbytes + abytes) / 1e3)) < 0.1
+    assert rf["bound_at_this_m"] == "hbm" and abs(rf["frac_of_attainable"] - 50.0 / rf["attainable"]) < 1e-3
+    big = bench.with_attainable({"value": 700.0, "roofline": {"peak": 1400.0}}, 4096, False)["roofline"]
+    assert big["bound_at_this_m"] == "tensor" and big["attainable"] == 1400.0
+
+
+def test_moe_hotness_tiers_cover_the_experts():
+    tiers = bench.MOE_TIERS
+    assert tiers[0][0] == 0 and tiers[-1][1] == bench.MOE["E"]
+    assert all(a[1] == b[0] for a, b in zip(tiers, tiers[1:]))
+    assert [t[2] for t in tiers] == [32, 64, 128]          # hot, ordinary, cold
