@@ -491,7 +491,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
             }
             tc::mma_commit(&sh->done);   // every MMA of this thread has completed once `done` flips
-            tc::mbar_wait(&sh->done, 0, p.status, abort_flag, 100000000ull);
+            tc::mbar_wait(&sh->done, 0, p.status, abort_flag);
         }
     } else if (wg == 1) {
         tc::setmaxnreg_dec<kRegsConv>();

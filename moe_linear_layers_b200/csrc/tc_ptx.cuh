@@ -69,6 +69,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// Wall-time limit of the kernels' waits.  Long enough that a context time-sliced with other work on a
+// shared GPU does not read as stuck, short enough that a wait nothing will satisfy ends the kernel
+// with Q4_ERR_TIMEOUT instead of hanging it.
+constexpr uint64_t kWaitLimitNs = 10000000000ull;
+
 // True once more than limit_ns of wall time separates now from t0 AND at least min_rounds polls were
 // made.  The difference is taken signed, so a global timer stepped back while a wait runs (the timer is
 // kept in step with the host clock) cannot make a fresh wait look expired through unsigned wrap-around,
@@ -98,7 +103,7 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, i
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort_flag,
-                                          uint64_t limit_ns = 2000000000ull)
+                                          uint64_t limit_ns = kWaitLimitNs)
 {
 #pragma unroll 1
     for (int i = 0; i < 64; i++)
@@ -281,10 +286,10 @@ __device__ __forceinline__ void sts_publish(void* p, uint32_t v)
 }
 
 // Spin until each of the n counters at c is >= target.  The fast path makes weak loads only; after a
-// few thousand unsuccessful rounds it also watches the wall clock (2 s: Q4_ERR_TIMEOUT, raise the abort
-// flag, return false) and the abort flag.
+// few thousand unsuccessful rounds it also watches the wall clock (kWaitLimitNs: Q4_ERR_TIMEOUT, raise
+// the abort flag, return false) and the abort flag.
 __device__ __forceinline__ bool poll_counters_slow(const uint32_t* c, int n, uint32_t target, int32_t* status,
-                                                   volatile int* abort_flag, uint64_t limit_ns = 2000000000ull)
+                                                   volatile int* abort_flag, uint64_t limit_ns = kWaitLimitNs)
 {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t round = 0;; round++) {
