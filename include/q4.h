@@ -17,8 +17,9 @@
  *
  * Conventions for every call:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The caller owns every
- *     buffer; the library allocates no device memory.  Scratch space of the MoE layer is the
- *     caller's workspace.
+ *     buffer and no call allocates device memory: scratch space of the MoE layer is the caller's
+ *     workspace (the one exception, moe_q4_forward_noalloc, uses a fixed array that exists from the
+ *     moment the library is loaded).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every call is
  *     asynchronous on it.
  *   - The return value reports errors the host can see before launching (null pointers, shapes,
