@@ -82,7 +82,7 @@ def max_over_ranks(v: float, ws: int) -> float:
 # ------------------------------------------------------------------------------------------------ #
 
 class ClockSampler:
-    def __init__(self, device: int, period_s: float = 0.01):
+    def __init__(self, device: int, period_s: float = 0.002):
         self.period, self.samples, self.reasons, self.handle, self.max_mhz = period_s, [], set(), None, None
         self.power = []
         try:
