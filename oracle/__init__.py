@@ -5,7 +5,9 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the 
 ``--impl reference`` legs of ``bench.py`` may import this package.  The product path (the CUDA
 library under ``moe_linear_layers_b200``) never imports it, and the two share no code.
 
-This module only marshals numpy arrays into the C functions; it holds none of the arithmetic.
+This module marshals numpy arrays into the C functions.  Apart from the composition helpers below
+(``silu_mul``, ``linear_w4a16_swiglu``, ``moe_experts_classes``), which combine the pinned C functions
+with plain fp64 numpy arithmetic, the arithmetic is in q4_oracle.c.
 """
 from __future__ import annotations
 
@@ -234,7 +236,7 @@ def moe_experts(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int,
 def moe_experts_a8(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int, symmetric: bool,
                    a8_mask: int, tokens=None):
     """The expert FFN with INT8 activations: a8_mask bit 0 = gate/up W4A8 on the token's INT8 codes,
-    bit 1 = down W4A8 on the INT8 codes of h (stored as fp16).  Returns fp64 [n_tok][H]."""
+    bit 1 = down W4A8 on the INT8 codes of h (quantized per row from fp32(h)).  Returns fp64 [n_tok][H]."""
     x = _c(x_bf16_bits, np.uint16).reshape(-1, H)
     ids = _c(ids, np.int32)
     w = _c(w, np.float64)

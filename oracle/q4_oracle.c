@@ -280,7 +280,7 @@ int orc_act_quant(const uint16_t* x, int M, int k, int8_t* q, float* s)
     return bad ? ORC_ERR_NONFINITE : ORC_OK;
 }
 
-/* The same quantization of fp16 rows (the MoE's intermediate activations h are stored as fp16):
+/* The same quantization of fp16 rows (the library's act_quant_per_token_f16 entry point):
  * x: fp16 bits [M][k], widened to fp32 exactly. */
 int orc_act_quant_f16(const uint16_t* x, int M, int k, int8_t* q, float* s)
 {
@@ -425,11 +425,10 @@ void orc_permute(const int32_t* ids, int T, int topk, int E, int32_t* offsets, i
  * (proportional recombination).  For token t and each chosen expert e = ids[t][j]:
  *   g = x_t . dequant(Wg_e)^T,  u = x_t . dequant(Wu_e)^T           (length I, fp64)
  *   h = g / (1 + exp(-g)) * u                                       (SiLU(g) * u, fp64)
- *   h16 = fp16(fp32(h))      the layer's intermediate is STORED as fp16 (reading: the interface between
- *                            the two expert projections holds h in fp16, as the library documents it;
- *                            the rounding through fp32 can differ from a direct rounding only when the
- *                            fp32 value lies exactly halfway between two fp16 values)
- *   o = h16 . dequant(Wd_e)^T                                       (length H, fp64)
+ *   o = h . dequant(Wd_e)^T                                         (length H, fp64)
+ * h stays fp64 between the two projections: the pages define the expert as a SwiGLU FFN and fix no
+ * storage precision for its intermediate, so the plain reading is the mathematical value; how a
+ * kernel carries h is its own choice, held to the output tolerance.
  *   y_t = sum_j w[t][j] * o                                         (fp64)
  * Expert weights are stacked: gate/up packed [E*I][H/2], scales/zeros [E*I][H/group];
  * down packed [E*H][I/2], scales/zeros [E*H][I/group].
@@ -468,7 +467,6 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
                     uv += xr[c] * (double)deq_at(up, us, uz, H, group, symmetric, i, c);
                 }
                 h[i] = gv / (1.0 + exp(-gv)) * uv;
-                h[i] = (double)orc_f16_to_f32(orc_f32_to_f16((float)h[i]));   /* stored as fp16 */
             }
             const uint8_t* dp = d_packed + (size_t)e * H * (I / 2);
             const uint16_t* ds = d_scales + (size_t)e * H * gI;
@@ -497,10 +495,11 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
  *                g_i = sum_g sa * sg[i][g] * sum_{k in g} xq[k] * (qg[i][k] - zg[i][g])   (fp64
  *                of the exact INT32 partials), u_i likewise with the up matrix;
  *   bit 0 clear: g, u as in orc_moe_experts (fp64 over the dequantized weights);
- *   h = g / (1 + exp(-g)) * u (fp64), stored as fp16 as in orc_moe_experts: h16 = fp16(fp32(h));
- *   bit 1 set:   hq, sh = act_quant(h16) over the row's I values, and
+ *   h = g / (1 + exp(-g)) * u (fp64), as in orc_moe_experts;
+ *   bit 1 set:   hq, sh = act_quant(hf) over the row's I values, hf = fp32(h) (the §3.1 arithmetic is
+ *                fp32: amax, amax/127 and the quotient are fp32 operations on the row's values), and
  *                o_c = sum_g sh * sd[c][g] * sum_{i in g} hq[i] * (qd[c][i] - zd[c][g]);
- *   bit 1 clear: o = h16 . dequant(Wd_e)^T (fp64);
+ *   bit 1 clear: o = h . dequant(Wd_e)^T (fp64, as orc_moe_experts);
  *   y_t = sum_j w[t][j] * o (fp64).
  * Returns ORC_ERR_NONFINITE when a quantized row holds a non-finite value.
  * ------------------------------------------------------------------------------------------- */
@@ -535,7 +534,7 @@ int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, cons
         float* xf = (float*)malloc(sizeof(float) * (size_t)H);
         int8_t* xq = (int8_t*)malloc((size_t)H);
         double* h = (double*)malloc(sizeof(double) * (size_t)I);
-        float* h16 = (float*)malloc(sizeof(float) * (size_t)I);
+        float* hf = (float*)malloc(sizeof(float) * (size_t)I);
         int8_t* hq = (int8_t*)malloc((size_t)I);
         double* yr = y + (size_t)it * H;
         int rb = 0;
@@ -567,12 +566,12 @@ int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, cons
             const uint16_t* dz = d_zeros ? d_zeros + (size_t)e * H * gI : NULL;
             double wj = w[(size_t)t * topk + j];
             double sh = 0.0;
-            for (int i = 0; i < I; i++) h16[i] = orc_f16_to_f32(orc_f32_to_f16((float)h[i]));
-            if (a8_mask & 2) sh = (double)act_quant_row(h16, I, hq, &rb);
+            for (int i = 0; i < I; i++) hf[i] = (float)h[i];
+            if (a8_mask & 2) sh = (double)act_quant_row(hf, I, hq, &rb);
             for (int c = 0; c < H; c++) {
                 double o = 0.0;
                 if (a8_mask & 2) o = w4a8_dot(hq, sh, dp, ds, dz, symmetric, I, group, c);
-                else for (int i = 0; i < I; i++) o += (double)h16[i] * (double)deq_at(dp, ds, dz, I, group, symmetric, c, i);
+                else for (int i = 0; i < I; i++) o += h[i] * (double)deq_at(dp, ds, dz, I, group, symmetric, c, i);
                 yr[c] += wj * o;
             }
         }
@@ -580,7 +579,7 @@ int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, cons
         free(xf);
         free(xq);
         free(h);
-        free(h16);
+        free(hf);
         free(hq);
     }
     return bad ? ORC_ERR_NONFINITE : ORC_OK;

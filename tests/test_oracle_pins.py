@@ -383,7 +383,7 @@ def test_shared_expert_is_the_dense_swiglu_ffn():
     y = oracle.shared_expert(x, H, qs[0], qs[1], qs[2], I_s, group, False)
     g = oracle.linear_w4a16(x, *qs[0], I_s, H, group, False)
     u = oracle.linear_w4a16(x, *qs[1], I_s, H, group, False)
-    h = _f16_store(g / (1.0 + np.exp(-g)) * u)
+    h = g / (1.0 + np.exp(-g)) * u
     wd = oracle.dequant(*qs[2], I_s, group, False).astype(np.float64)
     np.testing.assert_allclose(y, h @ wd.T, rtol=1e-11, atol=1e-12 * np.abs(y).max())
 
@@ -432,15 +432,23 @@ def test_permute_is_stable_sort():
 # MoE special cases: one expert = dense SwiGLU; k = E with equal logits = uniform average
 # ---------------------------------------------------------------------------------------------- #
 
-def _f16_store(h):
-    """The MoE intermediate as the layer stores it: fp64 -> fp32 -> fp16 (numpy's conversions), back to fp64."""
-    return np.asarray(h, np.float64).astype(np.float32).astype(np.float16).astype(np.float64)
-
-
 def _dense_swiglu(xf, Wg, Wu, Wd):
+    """A SwiGLU FFN in fp64 numpy: (silu(x Wg^T) * (x Wu^T)) Wd^T, the intermediate kept in fp64."""
     g = xf @ Wg.T
     u = xf @ Wu.T
-    return _f16_store(g / (1.0 + np.exp(-g)) * u) @ Wd.T
+    return (g / (1.0 + np.exp(-g)) * u) @ Wd.T
+
+
+def _act_quant_f32_numpy(hf):
+    """Per-token INT8 codes of one fp32 row restated in numpy (the W4A8 page §3.1): amax, scale = amax/127
+    and the quotient as IEEE fp32 operations, round half to even, clamp to [-128, 127]; scale 0 gives
+    all-zero codes."""
+    hf = np.asarray(hf, np.float32)
+    s = np.float32(np.abs(hf).max()) / np.float32(127.0)
+    if s == 0:
+        return np.zeros(hf.shape, np.int8), np.float32(0.0)
+    q = np.clip(np.rint(hf / s), -128, 127).astype(np.int8)
+    return q, s
 
 
 def _stacked_experts(E, H, I, group, sym, seed):
@@ -509,7 +517,7 @@ def test_act_quant_f16_properties():
 
 def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
     """The same layer assembled from the separately pinned pieces: act_quant, linear_w4a8 on each
-    expert's row block, linear_w4a16, numpy's fp16 rounding and act_quant_f16."""
+    expert's row block, linear_w4a16, and the codes of h restated in numpy from fp32(h)."""
     T, topk = ids.shape
     xq, sa = oracle.act_quant(x, H)
     y = np.zeros((T, H))
@@ -531,11 +539,11 @@ def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
                 u = oracle.linear_w4a16(x[t:t + 1], *uq, I, H, group, sym)[0]
             h = g / (1.0 + np.exp(-g)) * u
             if mask & 2:
-                h16 = h.astype(np.float32).astype(np.float16)
-                hq, sh = oracle.act_quant_f16(h16.view(np.uint16)[None, :], I)
-                o = oracle.linear_w4a8(hq, sh, dq[0], dq[1], H, I, group, zeros=dq[2], symmetric=sym)[0]
+                hq, sh = _act_quant_f32_numpy(h.astype(np.float32))
+                o = oracle.linear_w4a8(hq[None, :], np.array([sh], np.float32), dq[0], dq[1], H, I, group,
+                                       zeros=dq[2], symmetric=sym)[0]
             else:
-                o = _f16_store(h) @ oracle.dequant(*dq, I, group, sym).astype(np.float64).T
+                o = h @ oracle.dequant(*dq, I, group, sym).astype(np.float64).T
             y[t] += w[t, j] * o
     return y
 
