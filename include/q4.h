@@ -170,8 +170,8 @@ int act_quant_per_token(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, flo
 
 /*
  * act_quant_per_token_f16 -- act_quant_per_token for fp16 rows (the same arithmetic on values widened
- * exactly from fp16).  The MoE layer's intermediate activations h are fp16; this quantizes them for a
- * W4A8 down projection.  x [m][k] fp16 bits; everything else as act_quant_per_token.
+ * exactly from fp16), for activations a caller keeps in fp16.  x [m][k] fp16 bits; everything else as
+ * act_quant_per_token.
  */
 int act_quant_per_token_f16(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a,
                             int32_t* dev_status, void* stream);
@@ -208,7 +208,9 @@ size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t
  *   ids[t][j]    = the topk experts by (logit descending, id ascending), slot j = j-th best;
  *   w[t][j]      = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the chosen (= softmax, renormalised);
  *   perm/offsets = stable counting sort of the pairs (t, j) by expert (tokens ascending);
- *   h            = SiLU(x . Wg_e^T) * (x . Wu_e^T), kept as fp16;  o = h . Wd_e^T;
+ *   h            = SiLU(x . Wg_e^T) * (x . Wu_e^T) in fp32, carried to the down projection as two bf16
+ *                  values hi = bf16(h), lo = bf16(h - hi) (h to about 2^-17 of its magnitude; the down
+ *                  projection multiplies both);  o = h . Wd_e^T;
  *   y[t]         = sum_j w[t][j] * o_(t,j).
  * x [T][H] bf16; router_w [E][H] fp32; router_bias [E] fp32 or NULL.
  * experts[3] = {gate, up, down}: gate and up are [E*I][H] stacked by expert (rows e*I .. e*I+I-1),
@@ -231,8 +233,8 @@ int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H,
  * Source: "MoE推理优化实战：4bit存储+INT8计算的W4A8路线解析" and "高效大语言模型推理实践" MoE architecture
  * sections (a shared expert that every token passes through, beside the routed ones).
  *   y[t] = sum_j w[t][j] * o_(t,j) + S(x_t),  S(x) = (SiLU(x . Wg_s^T) * (x . Wu_s^T)) . Wd_s^T,
- * the shared expert a SwiGLU FFN of intermediate I_shared computed like a routed expert (h in fp16,
- * fp32 accumulation into the same output sums) with routing weight 1.
+ * the shared expert a SwiGLU FFN of intermediate I_shared computed like a routed expert (h as a bf16
+ * hi/lo pair, fp32 accumulation into the same output sums) with routing weight 1.
  * shared[3] = {gate, up, down} of one expert: gate and up [I_shared][H], down [H][I_shared], the
  * same group and symmetry as the routed experts; NULL (with I_shared ignored) = no shared expert.
  * I_shared % 128 == 0.  Every other argument as moe_q4_forward; the workspace must hold
@@ -255,13 +257,13 @@ int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H,
  *   a8_mask bit 0 (gate/up): xq_t, sa_t = act_quant(x_t) once per token;
  *                g_i = sa_t * sum_g sg[i][g] * P_g, P_g = sum_{k in g} xq_t[k] * (code_g[i][k] - zero_g[i][g])
  *                (exact INT32 partials, fp32 rescale), u likewise;
- *   a8_mask bit 1 (down): h (fp16, as stored) -> hq, sh = act_quant(h) per permuted row (I values), and
+ *   a8_mask bit 1 (down): h (the fp32 value hi + lo) -> hq, sh = act_quant(h) per permuted row (I values), and
  *                o_c = sh * sum_g sd[c][g] * sum_{i in g} hq[i] * (code_d[c][i] - zero_d[c][g]);
  *   a clear bit keeps that projection W4A16 as in moe_q4_forward.  a8_mask in 0..3 (0 = moe_q4_forward).
  *   The INT8 projections take groups 64 and 128 (group 32 only with a8_mask 0: Q4_ERR_UNSUPPORTED).
  * Arguments as moe_q4_forward; the workspace must hold moe_q4_workspace_size_a8(T, H, I, E, topk,
- * a8_mask) bytes.  dev_status also receives Q4_ERR_NONFINITE when a quantized row (x, or h after an
- * fp16 overflow) holds a non-finite value.
+ * a8_mask) bytes.  dev_status also receives Q4_ERR_NONFINITE when a quantized row (x or h) holds a
+ * non-finite value.
  */
 size_t moe_q4_workspace_size_a8(int32_t T, int32_t H, int32_t I, int32_t E, int32_t topk, int32_t a8_mask);
 int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H,
@@ -323,11 +325,12 @@ int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H,
  * 256-byte aligned).  Every GPU on which the library is loaded holds that array until the process
  * exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - Sizes whose moe_q4_workspace_size(T, H, I, E, topk) exceeds Q4_MOE_NOALLOC_SCRATCH_BYTES are
- *     rejected with Q4_ERR_WORKSPACE before anything is launched (for H = 2048, I = 1024, top-8 that
- *     is roughly T > 580 tokens).
+ *     rejected with Q4_ERR_WORKSPACE before anything is launched (for H = 2048, I = 1024, E = 64,
+ *     top-8 that is T > 453 tokens).
  *   - The first call on a device looks up the array's device address with cudaGetSymbolAddress while
- *     that device is current, and caches it; make that first call on each device before any stream
- *     capture begins.
+ *     that device is current, and caches it (per device and driver context: after a device reset the
+ *     next call looks it up again); make that first call on each device before any stream capture
+ *     begins.
  *   - All calls share the one array, which keeps the last call's contents (every call overwrites
  *     what it reads).  Calls that overlap on the GPU (for example on two streams) race on it: keep
  *     them ordered on one stream or serialise them.

@@ -9,7 +9,7 @@ int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_w
     using namespace tcg;
     if (w->k % KBLK) return Q4_ERR_UNSUPPORTED;
     CUtensorMap mx, mw;
-    if (!make_act_map(&mx, x, (uint64_t)w->k, (uint64_t)m, int8_path ? 1 : 2, false) ||
+    if (!make_act_map(&mx, x, (uint64_t)w->k, (uint64_t)m, int8_path ? 1 : 2) ||
         !make_packed_map(&mw, w->packed, (uint64_t)w->k, (uint64_t)w->n, BM))
         return Q4_ERR_CUDA;
     Args p = {};

@@ -14,7 +14,7 @@
 //   3. scatter   stable counting sort: every (token, slot) pair gets its row in the permuted order
 //                (expert, token ascending), and the token's activation row is gathered there;
 //   4. gate/up   grouped tcgen05 GEMM over (expert, token tile, 64 intermediate rows) tiles with the
-//                SwiGLU epilogue, h in fp16;
+//                SwiGLU epilogue, h as bf16 hi/lo pairs (h to about 2^-17 of its magnitude);
 //   5. down      grouped tcgen05 GEMM over (expert, token tile, 128 hidden rows) tiles whose epilogue
 //                adds w[t][j] * out into the fp32 output (float atomics: the sum order is not fixed);
 //   6. (bf16 output) a conversion pass.
@@ -328,9 +328,9 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ a, __nv_bfloat16* _
 
 struct Workspace {
     uint16_t* xperm;          // permuted activations: bf16 rows, or int8 codes (W4A8 gate/up)
-    __half* h;
+    __nv_bfloat16* h;         // [P][I/64][hi 64 | lo 64]
     // shared expert (I_shared > 0): its h, and the one-expert bookkeeping the grouped GEMMs read
-    __half* h_s;
+    __nv_bfloat16* h_s;
     int32_t *offsets_s, *tiles_gu_s, *tiles_dn_s, *row_tok_s;
     float* row_w_s;
     float* y32;
@@ -375,7 +375,7 @@ Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0, i
     size_t o = 0;
     auto take = [&](size_t bytes) { uint8_t* q = p ? p + o : nullptr; o += al(bytes); return q; };
     w.xperm = reinterpret_cast<uint16_t*>(take(P * H * 2));
-    w.h = reinterpret_cast<__half*>(take(P * I * 2));
+    w.h = reinterpret_cast<__nv_bfloat16*>(take(P * I * 4));
     w.y32 = reinterpret_cast<float*>(take((size_t)T * H * 4));
     w.ids = reinterpret_cast<int32_t*>(take(P * 4));
     w.wts = reinterpret_cast<float*>(take(P * 4));
@@ -389,7 +389,7 @@ Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0, i
     w.tiles_gu = reinterpret_cast<int32_t*>(take((E + 1) * 4));
     w.tiles_dn = reinterpret_cast<int32_t*>(take((E + 1) * 4));
     if (I_s > 0) {
-        w.h_s = reinterpret_cast<__half*>(take((size_t)T * I_s * 2));
+        w.h_s = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * I_s * 4));
         w.offsets_s = reinterpret_cast<int32_t*>(take(2 * 4));
         w.tiles_gu_s = reinterpret_cast<int32_t*>(take(2 * 4));
         w.tiles_dn_s = reinterpret_cast<int32_t*>(take(2 * 4));
@@ -422,7 +422,7 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
                               ws.offsets, ws.tiles_gu, ws.h, status, s);
     } else {
         CUtensorMap mx, mg, mu;
-        if (!make_act_map(&mx, ws.xperm, H, P, 2, false) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
+        if (!make_act_map(&mx, ws.xperm, H, P, 2) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
             !make_packed_map(&mu, ex[1].packed, H, (uint64_t)E * I, 64))
             return Q4_ERR_CUDA;
         Args a = {};
@@ -443,13 +443,12 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     }
     if (rc) return rc;
     if (a8_mask & 2) {   // h -> per-row int8 codes, then down on them
-        if ((rc = q4_act_quant_rows(reinterpret_cast<const uint16_t*>(ws.h), true, P, I, ws.hq, ws.sh_row, status, s)))
-            return rc;
+        if ((rc = q4_act_quant_hilo_rows(ws.h, P, I, ws.hq, ws.sh_row, status, s))) return rc;
         return q4_moe_down_a8(ws.hq, ws.sh_row, &ex[2], P, H, I, E, ws.offsets, ws.tiles_dn, ws.row_tok, ws.row_w,
                               y32, status, s);
     }
     CUtensorMap mh, md;
-    if (!make_act_map(&mh, ws.h, I, P, 2, true) || !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
+    if (!make_act_map(&mh, ws.h, 2 * (uint64_t)I, P, 2, 4) || !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
         return Q4_ERR_CUDA;
     Args d = {};
     d.M = P;
@@ -714,17 +713,36 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
 // ---------------------------------------------------------------------------------------------- //
 static __device__ __align__(256) uint8_t q4_moe_noalloc_scratch[Q4_MOE_NOALLOC_SCRATCH_BYTES];
 
+// The current driver context (nullptr when the entry point is unavailable): a device reset makes a new
+// primary context, in which the module and its array may sit elsewhere, so the cache is keyed on it too.
+static void* current_context()
+{
+    using GetCurrent = CUresult (*)(CUcontext*);
+    static GetCurrent fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess) ? reinterpret_cast<GetCurrent>(f) : nullptr;
+    }();
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
 static int noalloc_scratch_address(void** out)
 {
     static void* cache[64] = {nullptr};
+    static const void* cache_ctx[64] = {nullptr};
     static std::mutex lock;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return Q4_ERR_CUDA;
+    const void* ctx = current_context();   // nullptr until the runtime has made a context current here
     std::lock_guard<std::mutex> guard(lock);
-    if (!cache[dev]) {
-        void* p = nullptr;
+    if (!cache[dev] || !ctx || cache_ctx[dev] != ctx) {
+        void* p = nullptr;   // the lookup makes the device's primary context current on this thread
         if (cudaGetSymbolAddress(&p, q4_moe_noalloc_scratch) != cudaSuccess || !p) return Q4_ERR_CUDA;
         cache[dev] = p;
+        cache_ctx[dev] = current_context();
     }
     *out = cache[dev];
     return Q4_OK;

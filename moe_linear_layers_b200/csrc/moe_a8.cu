@@ -9,11 +9,11 @@ namespace {
 
 template <int G, bool SYM>
 int gateup(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H, int I, int E,
-           const int32_t* offsets, const int32_t* tiles, __half* h, int32_t* status, cudaStream_t s)
+           const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, int32_t* status, cudaStream_t s)
 {
     using namespace tcg;
     CUtensorMap mx, mg, mu;
-    if (!make_act_map(&mx, xq, H, P, 1, false) || !make_packed_map(&mg, gate->packed, H, (uint64_t)E * I, 64) ||
+    if (!make_act_map(&mx, xq, H, P, 1) || !make_packed_map(&mg, gate->packed, H, (uint64_t)E * I, 64) ||
         !make_packed_map(&mu, up->packed, H, (uint64_t)E * I, 64))
         return Q4_ERR_CUDA;
     Args a = {};
@@ -40,7 +40,7 @@ int down(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, i
 {
     using namespace tcg;
     CUtensorMap mh, md;
-    if (!make_act_map(&mh, hq, I, P, 1, false) || !make_packed_map(&md, dn->packed, I, (uint64_t)E * H, BM))
+    if (!make_act_map(&mh, hq, I, P, 1) || !make_packed_map(&md, dn->packed, I, (uint64_t)E * H, BM))
         return Q4_ERR_CUDA;
     Args d = {};
     d.M = P;
@@ -62,7 +62,7 @@ int down(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, i
 }  // namespace
 
 int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H,
-                     int I, int E, const int32_t* offsets, const int32_t* tiles, __half* h, int32_t* status,
+                     int I, int E, const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, int32_t* status,
                      cudaStream_t s)
 {
     if (gate->group == 128)

@@ -24,9 +24,12 @@
 //           (W4A8, int8 MMA on 16*code).
 //   GateUp  A rows 0-63 = gate rows i0..i0+63 of expert e, rows 64-127 = the same rows of up; B = the
 //           expert's rows of the permuted activations (bf16, or int8 codes with per-row scales s_a);
-//           epilogue h = SiLU(gate) * up -> fp16 (gate and up each times s_a first with int8 codes).
-//   Down    A = 128 rows of the expert's down projection (fp16 codes, or int8), B = h (fp16, or its
-//           int8 codes and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
+//           epilogue h = SiLU(gate) * up in fp32, stored as a pair of bf16 values hi = bf16(h) and
+//           lo = bf16(h - hi), which together hold h to about 2^-17 of its magnitude (gate and up each
+//           times s_a first with int8 codes).  Row layout of h: [I/64][hi 64 | lo 64].
+//   Down    A = 128 rows of the expert's down projection (bf16 codes, or int8), B = h: per K step one
+//           MMA on the hi values and one on the lo values into the same accumulator (or, int8, the
+//           codes of h and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
 //           (fp32 reduction into the output).
 //
 // Warp roles (640 threads = 5 warpgroups, launched at 96 registers and re-partitioned with setmaxnreg):
@@ -71,13 +74,15 @@ constexpr int kRegsEpi = 144;            // epilogue (two warpgroups)
 static_assert(128 * (kRegsIssue + kRegsProd + kRegsConv) + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
-constexpr int PW = 16;                   // quantization groups per window of the parameter ring
 constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
 constexpr float kAccBiasF = 12582912.0f;
 
 // PRING: the group parameters go through the shared-memory ring (every mode except symmetric W4A8)
 template <bool INT8, Mode MODE, bool PRING> struct Cfg {
-    static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2);   // activation bytes per stage
+    // the 16-bit down projection reads h as hi and lo halves: twice the activation bytes per stage
+    static constexpr bool HILO = MODE == Mode::Down && !INT8;
+    static constexpr int XBLK = HILO ? 4 : 2;                   // 64-column blocks per stage (16-bit)
+    static constexpr int XSTAGE = BN * KBLK * (INT8 ? 1 : 2) * (HILO ? 2 : 1);   // activation bytes per stage
     static constexpr int ACOLS = KBLK / (INT8 ? 4 : 2);         // TMEM columns of one widened stage
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     // group accumulators in TMEM: three for W4A8 (its MMAs are twice as fast, so the epilogue needs more
@@ -90,11 +95,12 @@ template <bool INT8, Mode MODE, bool PRING> struct Cfg {
     // zero points, group-major so a warp reads 32 consecutive rows (W4A8's epilogue reads its scales
     // through a register read-ahead instead, so symmetric W4A8 needs no ring at all)
     static constexpr int PTENS = 2;                             // scales, zero points
+    static constexpr int PW = HILO ? 4 : 16;                    // quantization groups per window
     static constexpr int PSLOT = PW * BM * 2;                   // bytes of one tensor in one slot
     static constexpr int PARAMS = PRING ? 2 * PSLOT * PTENS : 0;
     // shared-memory stages (activations + packed weights): as many as fit, so that enough MMA work is
     // in flight to cover the latency of the activation copies
-    static constexpr int NS = INT8 ? (MODE == Mode::GateUp ? 7 : 8) : (MODE == Mode::GateUp ? 4 : 5);
+    static constexpr int NS = INT8 ? (MODE == Mode::GateUp ? 7 : 8) : (MODE == Mode::GateUp ? 4 : (HILO ? 3 : 5));
     static_assert(NS <= kMaxStages, "ring depth");
     static_assert(NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144 <= 227 * 1024, "shared memory");
     static constexpr int SMEM = NS * (XSTAGE + WSTAGE) + XCHG + PARAMS + 1024 + 6144;
@@ -116,7 +122,7 @@ struct Args {
     const int32_t* offsets;        // [E+1] first permuted row of each expert
     const int32_t* row_tok;        // Down: [P] token of each permuted row
     const float* row_w;            // Down: [P] routing weight of each permuted row
-    __half* h;                     // GateUp output [P][N]
+    __nv_bfloat16* h;              // GateUp output [P][N/64][hi 64 | lo 64]
     int E, topk;
 };
 
@@ -141,29 +147,22 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
     return d;
 }
 
-__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// 8 nibbles (k = 0..7, even k in the low nibble of each byte) -> 4 words of 16-bit pairs holding the
+// 8 nibbles (k = 0..7, even k in the low nibble of each byte) -> 4 words of bf16 pairs holding the
 // exact integers (code - zero) in natural k order.  A PRMT puts nibble 2b at bits 0-3 and nibble 2b+1
-// at bits 16-19; one LOP3 ORs in the exponent of 128.0 (bf16) or 1024.0 (fp16), which makes the
-// nibble the low mantissa bits, and flips bit 3 of symmetric two's-complement codes (code + 8); one
-// packed subtract removes the magic plus the zero point (bias2 = magic + zero in both halves).
-template <bool SYM, bool F16>
+// at bits 16-19; one LOP3 ORs in the exponent of 128.0, which makes the nibble the low mantissa bits,
+// and flips bit 3 of symmetric two's-complement codes (code + 8); one packed subtract removes the
+// magic plus the zero point (bias2 = magic + zero in both halves).
+template <bool SYM>
 __device__ __forceinline__ void widen16(uint32_t w, uint32_t bias2, uint32_t (&o)[4])
 {
-    constexpr uint32_t magic = F16 ? 0x64006400u : 0x43004300u;
+    constexpr uint32_t magic = 0x43004300u;
     constexpr uint32_t key = SYM ? (magic ^ 0x00080008u) : magic;
     const uint32_t u = w >> 4;
 #pragma unroll
     for (int b = 0; b < 4; b++) {
         const uint32_t sel = (uint32_t)b | ((uint32_t)b << 4) | ((uint32_t)(4 + b) << 8) | ((uint32_t)(4 + b) << 12);
         const uint32_t t = lop3_and_xor(prmt(w, u, sel), 0x000F000Fu, key);
-        o[b] = F16 ? f16x2_sub(t, bias2) : bf16x2_sub(t, bias2);
+        o[b] = bf16x2_sub(t, bias2);
     }
 }
 
@@ -190,12 +189,8 @@ __device__ __forceinline__ void widen_s8_asym(uint32_t w, uint32_t zb, uint32_t&
     o1 = prmt(lo, hi, 0x7362u) ^ 0x80808080u;
 }
 
-__device__ __forceinline__ uint32_t pair16_bits(float v, bool f16)
+__device__ __forceinline__ uint32_t pair16_bits(float v)
 {
-    if (f16) {
-        const __half2 h = __floats2half2_rn(v, v);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    }
     const __nv_bfloat162 h = __floats2bfloat162_rn(v, v);
     return *reinterpret_cast<const uint32_t*>(&h);
 }
@@ -304,10 +299,11 @@ struct QuadRing {
 
 // PW consecutive fp16 group parameters of one row, from group g0 (zeros past the row's end or for a
 // missing row), stored group-major at dst[j * BM].
+template <int PW>
 __device__ __forceinline__ void stage_params(const __half* row, int g0, int ng, __half* dst)
 {
     uint16_t* d = reinterpret_cast<uint16_t*>(dst);
-    if (row && (ng & 7) == 0 && ((uintptr_t)row & 15) == 0) {
+    if (PW % 8 == 0 && row && (ng & 7) == 0 && ((uintptr_t)row & 15) == 0) {
 #pragma unroll
         for (int q = 0; q < PW / 8; q++) {
             const uint4 u = g0 + 8 * q < ng ? __ldg(reinterpret_cast<const uint4*>(row + g0 + 8 * q)) : make_uint4(0u, 0u, 0u, 0u);
@@ -331,8 +327,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 {
     constexpr bool PRING = !INT8 || !SYM;
     using C = Cfg<INT8, MODE, PRING>;
-    constexpr bool F16 = MODE == Mode::Down;   // the down projection consumes fp16 h
     constexpr int GPK = KBLK / G;               // groups per K stage
+    constexpr int PW = C::PW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     constexpr int NS = C::NS;
@@ -412,7 +408,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tc::mbar_arrive_expect_tx(&sh->x_full[s], C::XSTAGE);
                     uint8_t* xdst = xs + s * C::XSTAGE;
                     if constexpr (INT8) tc::tma_load_2d(xdst, &tm_x, &sh->x_full[s], kb * KBLK, T.m0);
-                    else tc::tma_load_3d(xdst, &tm_x, &sh->x_full[s], 0, T.m0, kb * 2);   // both 64-column halves
+                    else tc::tma_load_3d(xdst, &tm_x, &sh->x_full[s], 0, T.m0, kb * C::XBLK);   // the stage's 64-column blocks
                 }
             }
             if (!ok || *abort_flag) {  // let every copy this thread issued land before the CTA can exit
@@ -438,8 +434,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         const int r = 32 * i + lane;
                         const __half *srow, *zrow;
                         row_params<MODE>(p, T, r, ngroups, srow, zrow);
-                        stage_params(srow, w * PW, ngroups, ps + r);
-                        if constexpr (!SYM) stage_params(zrow, w * PW, ngroups, ps + PW * BM + r);
+                        stage_params<PW>(srow, w * PW, ngroups, ps + r);
+                        if constexpr (!SYM) stage_params<PW>(zrow, w * PW, ngroups, ps + PW * BM + r);
                     }
                     tc::mbar_arrive(&sh->p_full[wi & 1]);   // every lane: its stores are visible
                 }
@@ -453,7 +449,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // pipe never drains between stages; their completions go out through tcgen05.commit, which tracks
         // the issuing thread's own MMAs: every stage is issued and committed by one thread.
         if (lane == 0) {
-            constexpr uint32_t idesc = INT8 ? tc::idesc_s8_s32(BN) : (F16 ? tc::idesc_f16_f32(BN) : tc::idesc_bf16_f32(BN));
+            constexpr uint32_t idesc = INT8 ? tc::idesc_s8_s32(BN) : tc::idesc_bf16_f32(BN);
             uint32_t it = 0, g = 0;
             bool ok = true;
             if constexpr (INT8) ok = tc::poll_counters<8>(sh->epi_init, 1, p.status, abort_flag);
@@ -480,10 +476,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             const uint32_t a_tmem = tbase + C::A_COL0 + sa * C::ACOLS + (INT8 ? kk / 4 : kk / 2);
                             uint32_t boff;
                             if constexpr (INT8) boff = kk;                              // one 128-byte row box
-                            else boff = (kk / 64) * (BN * 128) + (kk % 64) * 2;          // two 64-column boxes
+                            else boff = (kk / 64) * (C::HILO ? 2 : 1) * (BN * 128) + (kk % 64) * 2;   // 64-column boxes
                             const uint64_t bdesc = tc::smem_desc_sw128(xaddr + (boff & ~127u)) + ((boff & 127u) >> 4);
-                            if constexpr (INT8) tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, true);
-                            else tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                            if constexpr (INT8) {
+                                tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, true);
+                            } else {
+                                tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                                if constexpr (C::HILO)   // the lo half of h: the next 64-column box
+                                    tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc + ((BN * 128) >> 4), idesc, 1);
+                            }
                         }
                         tc::mma_commit(&sh->d_full[db]);
                     }
@@ -491,7 +492,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
             }
             tc::mma_commit(&sh->done);   // every MMA of this thread has completed once `done` flips
-            tc::mbar_wait(&sh->done, 0, p.status, abort_flag);
+            // This wait must not honour the abort flag: after another role gave up, the MMAs already
+            // issued still read shared memory and write TMEM, and the CTA may leave (and free TMEM) only
+            // once they have completed.  Their operands are in place, so they finish; the wall-time limit
+            // still bounds the wait.
+            tc::mbar_wait(&sh->done, 0, p.status, nullptr);
         }
     } else if (wg == 1) {
         tc::setmaxnreg_dec<kRegsConv>();
@@ -499,7 +504,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int sub = warp & 3;
         const int r = 32 * sub + lane;                 // row in tile == TMEM lane
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
-        constexpr float kMagic = F16 ? 1024.0f : 128.0f;
+        constexpr float kMagic = 128.0f;
         uint32_t it = 0, wi = 0;   // stage and parameter-window counters (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             for (int kb = 0; kb < kblocks; kb++) {
@@ -559,7 +564,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 } else {
                     uint32_t bias[GPK];
 #pragma unroll
-                    for (int gi = 0; gi < GPK; gi++) bias[gi] = pair16_bits(kMagic + zcur[gi], F16);
+                    for (int gi = 0; gi < GPK; gi++) bias[gi] = pair16_bits(kMagic + zcur[gi]);
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
                         uint32_t o[32];
@@ -567,7 +572,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         for (int w = 0; w < 8; w++) {
                             const int ww = 8 * h + w;                  // word: k = 8*ww .. 8*ww+7
                             uint32_t q[4];
-                            widen16<SYM, F16>(words[ww], bias[(8 * ww) / G], q);
+                            widen16<SYM>(words[ww], bias[(8 * ww) / G], q);
 #pragma unroll
                             for (int b = 0; b < 4; b++) o[4 * w + b] = q[b];
                         }
@@ -749,10 +754,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if (lane == 0) tc::mbar_arrive(&sh->up_ready);
                 } else {
                     if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
-                    const int i = T.n0 + r;
                     const int mb = T.m0 + half * 64;
                     const int rows = min(64, T.m_end - mb);
-                    __half* hb = p.h + (int64_t)mb * p.N + i;
+                    // intermediate index i = n0 + r: its hi value in block n0 / 64 of the row, lo 64 later
+                    __nv_bfloat16* hb = p.h + (int64_t)mb * (2 * p.N) + 2 * T.n0 + r;
                     auto swiglu = [&](int j) {
                         float gv = accv(j), uv = xb[j * 64 + r];
                         if constexpr (INT8) {   // the row's activation scale
@@ -760,15 +765,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             gv *= sa;
                             uv *= sa;
                         }
-                        return __float2half_rn(gv * __frcp_rn(1.0f + __expf(-gv)) * uv);
+                        const float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+                        hb[(int64_t)j * (2 * p.N)] = hi;
+                        hb[(int64_t)j * (2 * p.N) + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
                     };
                     if (rows == 64) {
 #pragma unroll
-                        for (int j = 0; j < 64; j++) hb[(int64_t)j * p.N] = swiglu(j);
+                        for (int j = 0; j < 64; j++) swiglu(j);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 64; j++)
-                            if (j < rows) hb[(int64_t)j * p.N] = swiglu(j);
+                            if (j < rows) swiglu(j);
                     }
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&sh->gate_done);

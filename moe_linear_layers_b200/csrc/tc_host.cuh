@@ -36,11 +36,12 @@ inline bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Activation tile map.  int8 [rows][k]: one 128 x 128 box per stage.  bf16 / fp16 [rows][k]: viewed as
-// 3-D (64 columns, rows, k / 64 column blocks; the last stride is 128 bytes) so that the 128 x 128 tile
-// of a stage -- two 64-column halves of 128 rows, each 128-byte swizzled -- is ONE copy (a thread's
-// bulk copies are throughput-limited per instruction, not per byte).
-inline bool make_act_map(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, int elem_bytes, bool f16)
+// Activation tile map.  int8 [rows][k]: one 128 x 128 box per stage.  bf16 [rows][k]: viewed as 3-D
+// (64 columns, rows, k / 64 column blocks; the last stride is 128 bytes) so that the tile of a stage --
+// `blocks` 64-column blocks of 128 rows, each 128-byte swizzled -- is ONE copy (a thread's bulk copies
+// are throughput-limited per instruction, not per byte).  blocks = 2: a 128-column stage; blocks = 4:
+// the MoE intermediate h, whose rows interleave 64-column blocks of hi and lo values (k = 2 I).
+inline bool make_act_map(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, int elem_bytes, int blocks = 2)
 {
     if (elem_bytes == 1)
         return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, k, rows, k, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -48,9 +49,9 @@ inline bool make_act_map(CUtensorMap* map, const void* base, uint64_t k, uint64_
     if (!enc || k % 64) return false;
     cuuint64_t dims[3] = {64, rows, k / 64};
     cuuint64_t strides[2] = {2 * k, 128};
-    cuuint32_t box[3] = {64, BN, 2};
+    cuuint32_t box[3] = {64, BN, (cuuint32_t)blocks};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

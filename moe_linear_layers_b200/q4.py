@@ -123,6 +123,24 @@ def _dev(t, dtype, name):
     return t
 
 
+def _out(y, shape, device, name="y"):
+    """Check a caller-supplied output: fp32 or bf16 (the two output dtypes of the ABI), the expected shape,
+    contiguous, on the inputs' device.  Returns the ABI's out_dtype code."""
+    if not isinstance(y, torch.Tensor):
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if y.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"{name} must be torch.float32 or torch.bfloat16, got {y.dtype}")
+    if tuple(y.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(y.shape)}")
+    if not y.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not y.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if y.device != device:
+        raise ValueError(f"{name} is on {y.device}, the inputs on {device}")
+    return Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+
+
 def status_string(status: int) -> str:
     return _lib.q4_status_string(status).decode()
 
@@ -167,7 +185,7 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
     m = x.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (m, w.n), x.device)
     _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
            "q4_linear_w4a16")
     return y
@@ -182,7 +200,7 @@ def q4_linear_w4a16_swiglu(gate: torch.Tensor, up: torch.Tensor, w: Q4Weight, ou
     m = gate.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=gate.device)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (m, w.n), gate.device)
     _check(_lib.q4_linear_w4a16_swiglu(_ptr(gate), _ptr(up), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status),
                                        _stream(stream)), "q4_linear_w4a16_swiglu")
     return y
@@ -199,7 +217,10 @@ class GroupedGemv:
         self.x = (_p * self.count)(*[t.data_ptr() for t in xs])
         self.w = (q4_weight * self.count)(*[w.desc for w in ws])
         self.y = (_p * self.count)(*[t.data_ptr() for t in ys])
-        self.od = Q4_OUT_BF16 if ys[0].dtype == torch.bfloat16 else Q4_OUT_F32
+        ods = {_out(y, (self.m, w.n), xs[0].device) for y, w in zip(ys, ws)}
+        if len(ods) != 1:
+            raise TypeError("every y of a grouped call must have the same dtype")
+        self.od = ods.pop()
 
     def __call__(self, dev_status: torch.Tensor | None = None, stream=None):
         _check(_lib.q4_linear_w4a16_grouped(self.count, self.x, self.m, self.w, self.y, self.od, _ptr(dev_status),
@@ -241,7 +262,7 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
     m = xq.shape[0]
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (m, w.n), xq.device)
     _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
                                _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
     return y
@@ -278,7 +299,7 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
     dev = x.device
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (T, H), dev)
     I_s = shared[0].n if shared is not None else 0
     ws_bytes = moe_q4_workspace_size(T, H, I, E, topk, I_s, a8_mask)
     if workspace is None:
@@ -324,7 +345,7 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
         raise ValueError("class_begin needs one more entry than there are classes")
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (T, H), dev)
     if workspace is None:
         workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=dev)
     begin = (_i32 * (n + 1))(*[int(v) for v in class_begin])
@@ -358,6 +379,7 @@ def moe_q4_forward_range(x: torch.Tensor, router_w: torch.Tensor, router_bias: t
     if y is None:
         y = torch.empty((T, H), dtype=torch.float32, device=x.device)
     _dev(y, torch.float32, "y")
+    _out(y, (T, H), x.device)
     if workspace is None:
         workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=x.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
@@ -401,7 +423,7 @@ def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     E = router_w.shape[0]
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=x.device)
-    od = Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
+    od = _out(y, (T, H), x.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
     _check(_lib.moe_q4_forward_noalloc(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, _ptr(y),
                                        od, None, None, None, None, None, _ptr(dev_status), _stream(stream)),

@@ -176,3 +176,18 @@ def test_moe_range_validation():
     assert call(-1, 2) == q4.Q4_ERR_SHAPE
     assert call(2, 4) == q4.Q4_ERR_SHAPE          # 2 experts, weights stacked for 3
     assert call(2, 5, wsb=ws - 1) == q4.Q4_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("y,err", [
+    (lambda: __import__("torch").empty((4, 8), dtype=__import__("torch").float16), TypeError),   # fp16: no ABI code
+    (lambda: __import__("torch").empty((4, 7), dtype=__import__("torch").float32), ValueError),  # smaller than [T][H]
+    (lambda: __import__("torch").empty((8, 4), dtype=__import__("torch").float32).t(), ValueError),  # not contiguous
+    (lambda: __import__("torch").empty((4, 8), dtype=__import__("torch").float32), TypeError),   # host memory
+    (lambda: [0.0] * 32, TypeError),
+])
+def test_output_checked_before_any_launch(y, err):
+    """A caller-supplied output of the wrong dtype, shape, layout or memory is refused by the binding (the
+    ABI would read an fp16 buffer as fp32 and write past a short one)."""
+    import torch
+    with pytest.raises(err):
+        q4._out(y(), (4, 8), torch.device("cuda", 0))

@@ -410,6 +410,57 @@ def test_route_selection_and_weights():
     assert np.array_equal(counts, np.bincount(ids.ravel(), minlength=E))
 
 
+def _fp32_round(q):
+    """The fp32 nearest to the rational q, ties to even (an exact rounding: fp64 conversion can round twice)."""
+    from fractions import Fraction
+    if q == 0:
+        return np.float32(0.0)
+    f = np.float32(float(q))
+    best = None
+    for c in (f, np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf))):
+        d = abs(Fraction(float(c)) - q)
+        key = (d, int(np.array(c, np.float32).view(np.uint32)) & 1)   # on a tie the even significand wins
+        if best is None or key < best[0]:
+            best = (key, c)
+    return np.float32(best[1])
+
+
+def _fma32(a, b, c):
+    """fp32 fused multiply-add with one rounding: a * b + c formed exactly as a rational, then rounded."""
+    from fractions import Fraction
+    return _fp32_round(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def test_router_logit_pinned_order_bit_exact():
+    """The pinned fp32 order of the router logits, restated independently: 32 lane partials, each a chain
+    of correctly rounded fp32 fmas over k = l, l + 32, ... from +0, then the xor butterfly p_l + p_(l^s) for
+    s = 16, 8, 4, 2, 1 in fp32, logit = lane 0 (+ bias in fp32).  Bit-exact against the oracle; a plain
+    sequential fp32 sum of the same products differs for some logits, so the check sees the order."""
+    T, H, E = 3, 256, 4
+    x = synth.activations(("pins", "router-order"), T, H)
+    Wr, bias = synth.router(("pins", "router-order"), E, H)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float32)
+    logits, _, _, _ = oracle.route(x, H, Wr, bias, 1)
+    differs = 0
+    for t in range(T):
+        for e in range(E):
+            p = np.zeros(32, np.float32)
+            for lane in range(32):
+                for kk in range(lane, H, 32):
+                    p[lane] = _fma32(xf[t, kk], Wr[e, kk], p[lane])
+            for sft in (16, 8, 4, 2, 1):
+                p = np.array([p[lane] + p[lane ^ sft] for lane in range(32)], np.float32)
+            want = np.float32(p[0] + bias[e])
+            got = np.float32(oracle.router_logit(x[t], Wr[e]) + bias[e])
+            assert np.array_equal(np.array(want).view(np.uint32), np.array(got).view(np.uint32)), (t, e)
+            assert np.array_equal(np.array(want).view(np.uint32), np.array(logits[t, e]).view(np.uint32)), (t, e)
+            seq = np.float32(0.0)
+            for kk in range(H):
+                seq = np.float32(seq + np.float32(xf[t, kk] * Wr[e, kk]))
+            differs += int(seq != p[0])
+    assert differs > 0
+
+
 def test_route_ties_and_degenerate():
     T, H, E, topk = 5, 64, 8, 3
     x = synth.activations(("pins", "tie"), T, H)
