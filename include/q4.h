@@ -146,6 +146,35 @@ int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_t m, const 
                            int32_t out_dtype, int32_t* dev_status, void* stream);
 
 /*
+ * q4_linear_w4a16_chain -- a chain of DEPENDENT stages of m = 1 W4A16 GEMVs in one launch (a decode step:
+ * per layer [q, k, v], o, [gate, up], down).
+ * Source: the W4A8 page §2.1 (4-bit storage restored before the multiply) and §1 (small model, small
+ * batch: memory bound); "高效大语言模型推理实践：INT4量化与MoE架构的融合探索" MoE架构设计 (the FFN is
+ * SwiGLU: a stage may take silu(gate) * up as its input).  Each problem computes exactly what
+ * q4_linear_w4a16 computes at m = 1; the chain only orders the work: stage s reads its inputs only after
+ * every output of stages 0 .. s-1 is written, so an input may be (or be gated from) an earlier output.
+ * Inside the launch the weights of later stages are already streaming while a stage waits.
+ *   stage_begin: HOST array of n_stages + 1 ints, 0 = stage_begin[0] < ... ; stage s holds problems
+ *                stage_begin[s] .. stage_begin[s+1]-1 (1 to 8 problems with the same k).
+ *   x, gate, up, w, y: HOST arrays of count = stage_begin[n_stages] entries (device pointers / descriptors).
+ *                x[i]: bf16 [k]; or, when gate and up are given and gate[i] != NULL, problem i's input is
+ *                silu(gate[i]) * up[i] from fp32 [k] vectors (then x may be NULL or x[i] ignored).
+ *                gate and up may be NULL (no gated problem).  y[i]: [n] in out_dtype.
+ *   Every w[i] has the same group and symmetry, k % 64 == 0, k <= 16384, n >= 1.  n_stages <= 128,
+ *   count <= 256.
+ *   sync: device memory of q4_linear_w4a16_chain_sync_bytes(n_stages) bytes, 4-byte aligned, ZERO before
+ *   the first call; the kernel leaves it zero on completion, so calls (and graph replays) on one stream can
+ *   reuse it.  Calls sharing a sync buffer must not overlap on the GPU.
+ * The launch is cooperative (every CTA resident at once: one per SM); the library's other launches need
+ * not be.  dev_status: Q4_ERR_NONFINITE for a non-finite input; Q4_ERR_TIMEOUT when a stage wait ran out
+ * (the other CTAs then stop too) -- outputs are undefined and the sync buffer must be zeroed again.
+ */
+size_t q4_linear_w4a16_chain_sync_bytes(int32_t n_stages);
+int q4_linear_w4a16_chain(int32_t n_stages, const int32_t* stage_begin, const uint16_t* const* x,
+                          const float* const* gate, const float* const* up, const q4_weight* w, void* const* y,
+                          int32_t out_dtype, uint32_t* sync, int32_t* dev_status, void* stream);
+
+/*
  * q4_selftest_bounded_wait -- exercises the bounded waits the kernels rely on (no counterpart in the
  * source pages; a test hook for the failure-detection path).  Launches one small kernel whose wait is
  * never satisfied: which = 0 an mbarrier phase no thread completes, 1 a progress counter no thread

@@ -119,3 +119,56 @@ extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m,
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
     return q4_gemm_tc_launch(xq, scale_a, m, w, y, out_dtype, acc_dbg, true, dev_status, (cudaStream_t)stream);
 }
+
+int q4_gemv_w4a16_chain_launch(int n_stages, const int32_t* stage_begin, const uint16_t* const* x,
+                               const float* const* g, const float* const* u, const q4_weight* w, void* const* y,
+                               int32_t out_dtype, uint32_t* sync, int32_t* dev_status, cudaStream_t stream);
+
+extern "C" size_t q4_linear_w4a16_chain_sync_bytes(int32_t n_stages)
+{
+    return n_stages < 1 ? 0 : (size_t)(n_stages + 1) * sizeof(uint32_t);
+}
+
+extern "C" int q4_linear_w4a16_chain(int32_t n_stages, const int32_t* stage_begin, const uint16_t* const* x,
+                                     const float* const* gate, const float* const* up, const q4_weight* w,
+                                     void* const* y, int32_t out_dtype, uint32_t* sync, int32_t* dev_status,
+                                     void* stream)
+{
+    if (!stage_begin || !w || !y || !sync) return Q4_ERR_NULL;
+    if (n_stages < 1 || n_stages > 128 || stage_begin[0] != 0) return Q4_ERR_SHAPE;
+    for (int s = 0; s < n_stages; s++) {
+        const int np = stage_begin[s + 1] - stage_begin[s];
+        if (np < 1 || np > 8) return Q4_ERR_SHAPE;
+    }
+    const int count = stage_begin[n_stages];
+    if (count > 256) return Q4_ERR_SHAPE;
+    if ((uintptr_t)sync & 3u) return Q4_ERR_ALIGN;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    for (int i = 0; i < count; i++) {
+        const int rc = check_weight(&w[i], false);
+        if (rc) return rc;
+        if (w[i].group != w[0].group || w[i].symmetric != w[0].symmetric) return Q4_ERR_UNSUPPORTED;
+        if (w[i].n < 1) return Q4_ERR_SHAPE;
+        if (w[i].k % 64 || w[i].k > 16384) return Q4_ERR_UNSUPPORTED;
+        const bool gated = gate && up && gate[i];
+        if (gated) {
+            if (!up[i]) return Q4_ERR_NULL;
+            if (!q4_aligned16(gate[i]) || !q4_aligned16(up[i])) return Q4_ERR_ALIGN;
+        } else {
+            if (!x || !x[i]) return Q4_ERR_NULL;
+            if (!q4_aligned16(x[i])) return Q4_ERR_ALIGN;
+        }
+        if (!y[i]) return Q4_ERR_NULL;
+        if (!q4_aligned16(y[i])) return Q4_ERR_ALIGN;
+    }
+    // entries of gate/up that are NULL take x (a problem is gated only when both are given)
+    const float* gs[256];
+    const float* us[256];
+    for (int i = 0; i < count; i++) {
+        const bool gated = gate && up && gate[i];
+        gs[i] = gated ? gate[i] : nullptr;
+        us[i] = gated ? up[i] : nullptr;
+    }
+    return q4_gemv_w4a16_chain_launch(n_stages, stage_begin, x, gs, us, w, y, out_dtype, sync, dev_status,
+                                      (cudaStream_t)stream);
+}

@@ -32,10 +32,11 @@
 //           codes of h and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
 //           (fp32 reduction into the output).
 //
-// Warp roles (640 threads = 5 warpgroups, launched at 96 registers and re-partitioned with setmaxnreg):
+// Warp roles (768 threads = 6 warpgroups, launched at 80 registers and re-partitioned with setmaxnreg):
 //   warps 0-3    MMA issuers, one thread each, stage it issued by warp it % 4 (warp 1 also owns TMEM);
-//   warps 4-7    converters (TMEM lanes 32*(warp%4) ...);
-//   warps 8-9    TMA producers (alternate stages); warps 10-11 idle;
+//   warps 4-7    converters of the even stages, warps 20-23 converters of the odd stages (TMEM lanes
+//                32*(warp%4) ...): a converter warp's loop is latency-bound, so two sets alternate;
+//   warps 8-9    TMA producers (alternate stages); warp 10 parameter loader; warp 11 idle;
 //   warps 12-19  epilogue (two warps per TMEM lane quarter, each draining 64 of the 128 columns).
 // Measured on B200: one thread issues an M128 N128 K16 MMA only every ~120 cycles, half the tensor
 // pipe's rate, and any strong memory operation in that thread (an mbarrier wait included) stalls it
@@ -62,16 +63,18 @@ constexpr int KBLK = 128;                // K per stage
 constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
-constexpr int kThreads = 640;            // 20 warps = 5 warpgroups
+constexpr int kThreads = 768;            // 24 warps = 6 warpgroups
 constexpr int kIssuers = 4;              // MMA issuer threads (warps 0-3)
-// registers per thread: the launch allocation (65536 / 640, rounded down to a multiple of 8) and the
+constexpr int kConvSets = 2;             // converter warpgroups, alternate stages
+// registers per thread: the launch allocation (65536 / 768, rounded down to a multiple of 8) and the
 // per-warpgroup split after setmaxnreg; the split may not exceed the launch allocation
-constexpr int kLaunchRegs = 96;
+constexpr int kLaunchRegs = 80;
 constexpr int kRegsIssue = 48;           // MMA issuers
-constexpr int kRegsProd = 56;            // TMA producers, parameter loader
-constexpr int kRegsConv = 88;            // converters
-constexpr int kRegsEpi = 144;            // epilogue (two warpgroups)
-static_assert(128 * (kRegsIssue + kRegsProd + kRegsConv) + 256 * kRegsEpi <= kThreads * kLaunchRegs, "register split");
+constexpr int kRegsProd = 40;            // TMA producers, parameter loader
+constexpr int kRegsConv = 64;            // converters (each set)
+constexpr int kRegsEpi = 128;            // epilogue (two warpgroups)
+static_assert(128 * (kRegsIssue + kRegsProd + kConvSets * kRegsConv) + 256 * kRegsEpi <= kThreads * kLaunchRegs,
+              "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxExperts = 256;
 constexpr uint32_t kAccBias = 0x4B400000u;   // bits of 1.5 * 2^23: preloaded int32 accumulators (W4A8)
@@ -197,12 +200,16 @@ __device__ __forceinline__ uint32_t pair16_bits(float v)
 
 struct Shared {
     // per stage: packed weights landed, activations landed (converters wait on both), and the slot
-    // free again (MMA commit + the four converter warps; it also frees the stage's TMEM A slot)
+    // free again (MMA commit + the four converter warps of the stage's set)
     uint64_t w_full[kMaxStages], x_full[kMaxStages], xw_empty[kMaxStages];
+    // per TMEM slot of widened weights: the MMAs of the slot's last stage have completed.  (The ring's
+    // xw_empty cannot stand in for it: with fewer ring stages than TMEM slots, or two converter sets, the
+    // ring barrier of stage it - NA can complete a second phase before the converter of stage it looks.)
+    uint64_t tmem_free[NA];
     uint64_t d_full[3], done;
     // progress counters read by the MMA issuer (weak loads): stages converted (and activations landed)
-    // per converter warp, groups drained per epilogue warp, W4A8 accumulator preload done per epilogue warp
-    uint32_t conv_done[4], epi_done[8], epi_init[8];
+    // per converter warp of each set, groups drained per epilogue warp, W4A8 accumulator preload done
+    uint32_t conv_done[4 * kConvSets], epi_done[8], epi_init[8];
     uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
     uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
@@ -352,11 +359,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->xw_empty[i], 1 + 4);
         }
         for (int i = 0; i < C::ND; i++) tc::mbar_init(&sh->d_full[i], 1);
-        for (int i = 0; i < 4; i++) sh->conv_done[i] = 0;
+        for (int i = 0; i < NA; i++) tc::mbar_init(&sh->tmem_free[i], 1);
+        for (int i = 0; i < 4 * kConvSets; i++) sh->conv_done[i] = 0;
         for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
         tc::mbar_init(&sh->done, kIssuers);
         // consumers: the converters, and the epilogue unless it is W4A8's
-        for (int i = 0; i < 2; i++) { tc::mbar_init(&sh->p_full[i], 32); tc::mbar_init(&sh->p_empty[i], INT8 ? 4 : 4 + 8); }
+        // parameter windows are released by every converter warp of both sets (and the 16-bit epilogue)
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&sh->p_full[i], 32);
+            tc::mbar_init(&sh->p_empty[i], 4 * kConvSets + (INT8 ? 0 : 8));
+        }
         tc::mbar_init(&sh->up_ready, 4);
         tc::mbar_init(&sh->gate_done, 4);
         sh->abort_flag = 0;
@@ -461,7 +473,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                     const int s = it % NS, sa = it % NA;
                     // the stage's weights are widened into TMEM and its activations have landed
-                    if (!(ok = tc::poll_counters<4>(sh->conv_done, it + 1, p.status, abort_flag))) break;
+                    if (!(ok = tc::poll_counters<4>(sh->conv_done + 4 * (it % kConvSets), it + 1, p.status, abort_flag))) break;
                     tc::fence_after_sync();
                     const uint32_t xaddr = tc::smem_u32(xs + s * C::XSTAGE);
 #pragma unroll
@@ -489,6 +501,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tc::mma_commit(&sh->d_full[db]);
                     }
                     tc::mma_commit(&sh->xw_empty[s]);
+                    tc::mma_commit(&sh->tmem_free[sa]);
                 }
             }
             tc::mma_commit(&sh->done);   // every MMA of this thread has completed once `done` flips
@@ -498,9 +511,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // still bounds the wait.
             tc::mbar_wait(&sh->done, 0, p.status, nullptr);
         }
-    } else if (wg == 1) {
+    } else if (wg == 1 || wg == 5) {
         tc::setmaxnreg_dec<kRegsConv>();
-        // ------------------------------------------------------------------ converters (warps 4-7)
+        // ------------------------------------------------------------------ converters (warps 4-7, 20-23)
+        // Set cs converts the stages it with it % 2 == cs; both sets walk every stage for the parameter
+        // windows, so each releases every window once.
+        const int cs = wg == 5 ? 1 : 0;
         const int sub = warp & 3;
         const int r = 32 * sub + lane;                 // row in tile == TMEM lane
         const uint32_t lane_field = (uint32_t)(32 * sub) << 16;
@@ -525,14 +541,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         wi++;
                     }
                 }
+                if (it % kConvSets != (uint32_t)cs) {   // the other set's stage
+                    it++;
+                    continue;
+                }
                 // one combined wait: the stage's packed weights and activations have landed, and TMEM slot
-                // sa is free -- the MMAs of stage it - NA have completed, i.e. that stage's slot of the ring
-                // has been released (its phase cannot be older: this warp has converted stage it - NA, so the
-                // producer refilled it; nor newer: that needs this warp's arrival for it - NA + NS)
+                // sa is free -- the MMAs of stage it - NA, the slot's previous stage, have completed (that
+                // phase cannot be older: this set converted stage it - NA; nor can a newer one have completed:
+                // the slot's next stage is this one)
                 {
-                    const uint32_t j = it >= (uint32_t)NA ? it - NA : it;
-                    uint64_t* slot_bar = it >= (uint32_t)NA ? &sh->xw_empty[j % NS] : &sh->w_full[s];
-                    const uint32_t slot_par = it >= (uint32_t)NA ? (j / NS) & 1 : (it / NS) & 1;
+                    uint64_t* slot_bar = it >= (uint32_t)NA ? &sh->tmem_free[sa] : &sh->w_full[s];
+                    const uint32_t slot_par = it >= (uint32_t)NA ? ((it / NA) - 1) & 1 : (it / NS) & 1;
                     if (!tc::mbar_wait3(&sh->w_full[s], (it / NS) & 1, &sh->x_full[s], (it / NS) & 1, slot_bar, slot_par,
                                         p.status, abort_flag))
                         goto conv_done;
@@ -583,7 +602,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tc::fence_before_sync();
                 // publish: this warp's rows of the stage are in TMEM, and the stage's activations landed
                 __syncwarp();
-                if (lane == 0) tc::sts_publish(&sh->conv_done[sub], it + 1);
+                if (lane == 0) tc::sts_publish(&sh->conv_done[4 * cs + sub], it + 1);
                 it++;
             }
         }

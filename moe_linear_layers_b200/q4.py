@@ -36,7 +36,7 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_q
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
             "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes",
-            "moe_q4_forward_range")
+            "moe_q4_forward_range", "q4_linear_w4a16_chain_sync_bytes", "q4_linear_w4a16_chain")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -77,6 +77,11 @@ _lib.moe_q4_forward_classes.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _i32
                                         ctypes.POINTER(q4_weight), _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
 _lib.moe_q4_forward_range.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _i32, _i32, ctypes.POINTER(q4_weight), _i32,
                                       _p, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.q4_linear_w4a16_chain_sync_bytes.restype = _sz
+_lib.q4_linear_w4a16_chain_sync_bytes.argtypes = [_i32]
+_lib.q4_linear_w4a16_chain.argtypes = [_i32, ctypes.POINTER(_i32), ctypes.POINTER(_p), ctypes.POINTER(_p),
+                                       ctypes.POINTER(_p), ctypes.POINTER(q4_weight), ctypes.POINTER(_p), _i32, _p, _p,
+                                       _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -225,6 +230,60 @@ class GroupedGemv:
     def __call__(self, dev_status: torch.Tensor | None = None, stream=None):
         _check(_lib.q4_linear_w4a16_grouped(self.count, self.x, self.m, self.w, self.y, self.od, _ptr(dev_status),
                                             _stream(stream)), "q4_linear_w4a16_grouped")
+
+
+class GemvChain:
+    """A chain of dependent GEMV stages at m = 1 in one launch (q4_linear_w4a16_chain), its argument arrays
+    and its stage counters built once.  stages: a list of stages, each a list of problems (x, w, y): x a bf16
+    CUDA tensor of w.k values, or a pair (gate, up) of fp32 CUDA tensors of w.k values (the input is then
+    silu(gate) * up); w a Q4Weight; y an fp32 (or bf16, the same for every problem) CUDA tensor of w.n values.
+    Stage s starts reading its inputs only once every output of the stages before it is written."""
+
+    def __init__(self, stages):
+        probs = [pr for st in stages for pr in st]
+        if not stages or not probs:
+            raise ValueError("a chain needs at least one stage with one problem")
+        self.n_stages = len(stages)
+        self.count = len(probs)
+        begin = [0]
+        for st in stages:
+            begin.append(begin[-1] + len(st))
+        dev = probs[0][2].device
+        ods = set()
+        xs, gs, us = [], [], []
+        for x, w, y in probs:
+            ods.add(_out(y.view(-1), (w.n,), dev))
+            if isinstance(x, (tuple, list)):
+                _dev(x[0], torch.float32, "gate")
+                _dev(x[1], torch.float32, "up")
+                xs.append(None)
+                gs.append(x[0].data_ptr())
+                us.append(x[1].data_ptr())
+            else:
+                _dev(x, torch.bfloat16, "x")
+                xs.append(x.data_ptr())
+                gs.append(None)
+                us.append(None)
+        if len(ods) != 1:
+            raise TypeError("every y of a chain must have the same dtype")
+        self.od = ods.pop()
+        self.keep = stages
+        self.begin = (_i32 * (self.n_stages + 1))(*begin)
+        self.x = (_p * self.count)(*xs)
+        self.g = (_p * self.count)(*gs)
+        self.u = (_p * self.count)(*us)
+        self.w = (q4_weight * self.count)(*[w.desc for _, w, _ in probs])
+        self.y = (_p * self.count)(*[y.data_ptr() for _, _, y in probs])
+        nbytes = int(_lib.q4_linear_w4a16_chain_sync_bytes(self.n_stages))
+        self.sync = torch.zeros((nbytes // 4,), dtype=torch.int32, device=dev)
+
+    def reset(self):
+        """Zero the stage counters (needed only after a call that reported Q4_ERR_TIMEOUT)."""
+        self.sync.zero_()
+
+    def __call__(self, dev_status: torch.Tensor | None = None, stream=None):
+        _check(_lib.q4_linear_w4a16_chain(self.n_stages, self.begin, self.x, self.g, self.u, self.w, self.y, self.od,
+                                          _ptr(self.sync), _ptr(dev_status), _stream(stream)), "q4_linear_w4a16_chain")
 
 
 def q4_linear_w4a16_grouped(xs, ws, ys, dev_status: torch.Tensor | None = None, stream=None):

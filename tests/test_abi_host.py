@@ -191,3 +191,31 @@ def test_output_checked_before_any_launch(y, err):
     import torch
     with pytest.raises(err):
         q4._out(y(), (4, 8), torch.device("cuda", 0))
+
+
+def test_chain_validation():
+    L = q4._lib
+    P = ctypes.c_void_p
+    assert L.q4_linear_w4a16_chain_sync_bytes(64) == 65 * 4 and L.q4_linear_w4a16_chain_sync_bytes(0) == 0
+
+    def call(begin, ws, xs=None, ys=None, sync=FAKE, gate=None, up=None, out=0):
+        n = len(ws)
+        b = (ctypes.c_int32 * len(begin))(*begin)
+        w = (q4.q4_weight * n)(*ws)
+        x = xs if xs is not None else (P * n)(*([FAKE] * n))
+        y = ys if ys is not None else (P * n)(*([FAKE] * n))
+        return L.q4_linear_w4a16_chain(len(begin) - 1, b, x, gate, up, w, y, out, sync, None, None)
+
+    w2 = [_w(group=128, sym=0, zeros=FAKE), _w(group=128, sym=0, zeros=FAKE)]
+    assert call([0, 1, 2], w2, sync=None) == q4.Q4_ERR_NULL
+    assert call([0, 1, 2], w2, sync=FAKE + 2) == q4.Q4_ERR_ALIGN
+    assert call([1, 2], w2) == q4.Q4_ERR_SHAPE                    # stage_begin[0] != 0
+    assert call([0, 0, 2], w2) == q4.Q4_ERR_SHAPE                 # an empty stage
+    assert call([0, 9] + [9] * 0, [w2[0]] * 9) == q4.Q4_ERR_SHAPE  # 9 problems in one stage
+    assert call([0, 1, 2], [w2[0], _w(group=64)]) == q4.Q4_ERR_UNSUPPORTED   # group/symmetry differ
+    assert call([0, 1, 2], w2, out=5) == q4.Q4_ERR_UNSUPPORTED
+    assert call([0, 1, 2], w2, xs=(P * 2)(FAKE, None)) == q4.Q4_ERR_NULL
+    assert call([0, 1, 2], w2, ys=(P * 2)(FAKE, FAKE + 4)) == q4.Q4_ERR_ALIGN
+    g = (P * 2)(None, FAKE)
+    assert call([0, 1, 2], w2, gate=g, up=(P * 2)(None, None)) == q4.Q4_ERR_NULL   # gated without up
+    assert call([0, 1, 2], w2, gate=g, up=(P * 2)(None, FAKE + 8)) == q4.Q4_ERR_ALIGN
