@@ -236,7 +236,7 @@ def moe_experts(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int,
 def moe_experts_a8(x_bf16_bits, H: int, ids, w, gate, up, down, I: int, group: int, symmetric: bool,
                    a8_mask: int, tokens=None):
     """The expert FFN with INT8 activations: a8_mask bit 0 = gate/up W4A8 on the token's INT8 codes,
-    bit 1 = down W4A8 on the INT8 codes of h (quantized per row from fp32(h)).  Returns fp64 [n_tok][H]."""
+    bit 1 = down W4A8 on the INT8 codes of h (quantized per row as an fp16 activation).  Returns fp64 [n_tok][H]."""
     x = _c(x_bf16_bits, np.uint16).reshape(-1, H)
     ids = _c(ids, np.int32)
     w = _c(w, np.float64)

@@ -496,8 +496,10 @@ void orc_moe_experts(const uint16_t* x, int T, int H, const int32_t* ids, const 
  *                of the exact INT32 partials), u_i likewise with the up matrix;
  *   bit 0 clear: g, u as in orc_moe_experts (fp64 over the dequantized weights);
  *   h = g / (1 + exp(-g)) * u (fp64), as in orc_moe_experts;
- *   bit 1 set:   hq, sh = act_quant(hf) over the row's I values, hf = fp32(h) (the §3.1 arithmetic is
- *                fp32: amax, amax/127 and the quotient are fp32 operations on the row's values), and
+ *   bit 1 set:   hq, sh = act_quant(h16) over the row's I values, h16 = fp16(fp32(h)): §3.1's per-token
+ *                quantizer takes the layer's 16-bit activation tensor (fp16, the pages' activation
+ *                format) as its input, so the down projection's INT8 activations are the codes of h as an
+ *                fp16 activation; then
  *                o_c = sum_g sh * sd[c][g] * sum_{i in g} hq[i] * (qd[c][i] - zd[c][g]);
  *   bit 1 clear: o = h . dequant(Wd_e)^T (fp64, as orc_moe_experts);
  *   y_t = sum_j w[t][j] * o (fp64).
@@ -566,7 +568,7 @@ int orc_moe_experts_a8(const uint16_t* x, int T, int H, const int32_t* ids, cons
             const uint16_t* dz = d_zeros ? d_zeros + (size_t)e * H * gI : NULL;
             double wj = w[(size_t)t * topk + j];
             double sh = 0.0;
-            for (int i = 0; i < I; i++) hf[i] = (float)h[i];
+            for (int i = 0; i < I; i++) hf[i] = orc_f16_to_f32(orc_f32_to_f16((float)h[i]));
             if (a8_mask & 2) sh = (double)act_quant_row(hf, I, hq, &rb);
             for (int c = 0; c < H; c++) {
                 double o = 0.0;

@@ -568,7 +568,7 @@ def test_act_quant_f16_properties():
 
 def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
     """The same layer assembled from the separately pinned pieces: act_quant, linear_w4a8 on each
-    expert's row block, linear_w4a16, and the codes of h restated in numpy from fp32(h)."""
+    expert's row block, linear_w4a16, and the codes of h (as an fp16 activation) restated in numpy."""
     T, topk = ids.shape
     xq, sa = oracle.act_quant(x, H)
     y = np.zeros((T, H))
@@ -589,8 +589,9 @@ def _moe_a8_by_composition(x, H, ids, w, stack, I, group, sym, mask):
                 g = oracle.linear_w4a16(x[t:t + 1], *gq, I, H, group, sym)[0]
                 u = oracle.linear_w4a16(x[t:t + 1], *uq, I, H, group, sym)[0]
             h = g / (1.0 + np.exp(-g)) * u
-            if mask & 2:
-                hq, sh = _act_quant_f32_numpy(h.astype(np.float32))
+            if mask & 2:   # the codes of h as an fp16 activation (numpy's IEEE conversions)
+                h16 = h.astype(np.float32).astype(np.float16)
+                hq, sh = _act_quant_f32_numpy(h16.astype(np.float32))
                 o = oracle.linear_w4a8(hq[None, :], np.array([sh], np.float32), dq[0], dq[1], H, I, group,
                                        zeros=dq[2], symmetric=sym)[0]
             else:
