@@ -212,8 +212,14 @@ def traffic_from_profiles(name):
 
 
 def graph_of(fn):
+    """Capture fn in a CUDA graph after one eager call.  The eager call must finish within seconds: a call
+    that takes longer ran into a kernel's bounded wait (10 s, Q4_ERR_TIMEOUT), and timing it would only
+    measure the limit, so the run stops there."""
+    t0 = time.time()
     fn()
     torch.cuda.synchronize()
+    if time.time() - t0 > 5.0:
+        raise SystemExit(f"bench: an eager call took {time.time() - t0:.1f} s (a bounded wait ran out?); not timing it")
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         fn()
@@ -539,7 +545,11 @@ def run_moe(q4, args, dev):
     steps = max(3, min(args.steps, 20))
     clk = ClockSampler(torch.cuda.current_device())
     ms = time_replays(g, steps, 1, clk) / steps
-    _, ids, _, _, _, counts = q4.moe_q4_forward(x, Wr, bias, topk, ex, I, workspace=ws_t, want_routing=True)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    _, ids, _, _, _, counts = q4.moe_q4_forward(x, Wr, bias, topk, ex, I, workspace=ws_t, want_routing=True,
+                                                dev_status=st)
+    if int(st.item()) != 0:
+        raise SystemExit(f"bench: the MoE layer reported device status {int(st.item())}")
     c = counts.cpu().numpy()
     flops = 2 * T * topk * 3 * H * I
     tf = flops / (ms * 1e-3) / 1e12

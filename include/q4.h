@@ -286,7 +286,8 @@ int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H,
  *   a8_mask bit 0 (gate/up): xq_t, sa_t = act_quant(x_t) once per token;
  *                g_i = sa_t * sum_g sg[i][g] * P_g, P_g = sum_{k in g} xq_t[k] * (code_g[i][k] - zero_g[i][g])
  *                (exact INT32 partials, fp32 rescale), u likewise;
- *   a8_mask bit 1 (down): h (the fp32 value hi + lo) -> hq, sh = act_quant(h) per permuted row (I values), and
+ *   a8_mask bit 1 (down): h as an fp16 activation (§3.1 quantizes the layer's 16-bit activations) ->
+ *                hq, sh = act_quant(fp16(h)) per permuted row (I values), and
  *                o_c = sh * sum_g sd[c][g] * sum_{i in g} hq[i] * (code_d[c][i] - zero_d[c][g]);
  *   a clear bit keeps that projection W4A16 as in moe_q4_forward.  a8_mask in 0..3 (0 = moe_q4_forward).
  *   The INT8 projections take groups 64 and 128 (group 32 only with a8_mask 0: Q4_ERR_UNSUPPORTED).
@@ -341,6 +342,53 @@ int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H,
                          int32_t e_begin, int32_t e_end, const q4_weight* experts, int32_t I, float* y,
                          int32_t* topk_ids, float* topk_w, int32_t* perm, int32_t* offsets, int32_t* expert_counts,
                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * The MoE layer's steps as separate calls: the units of expert parallelism in its all-to-all form (each
+ * rank routes its own tokens, sends every routed row to the rank that owns its expert, runs its experts
+ * on the rows it receives and sends the results back, where they are combined in token order).
+ * Source: "大模型之Dense、MoE与量化" 混合专家架构 MoE and its 缺点 paragraph (tokens are dispatched to
+ * different experts, whose outputs are recombined in proportion); the W4A8 page §1 (dispatch and merge
+ * cost extra).  Together the three calls compute exactly moe_q4_forward's function.
+ *
+ * moe_q4_route -- routing (as moe_q4_forward: pinned fp32 logits, top-k with ties to the lower id,
+ * softmax over the chosen) and the permutation (stable counting sort of the (token, slot) pairs by expert).
+ *   Outputs (required): topk_ids [T][topk] int32, topk_w [T][topk] fp32, offsets [E+1] int32 (the
+ *   permuted rows of expert e are offsets[e] .. offsets[e+1]-1), pair_pos [T*topk] int32 (the permuted
+ *   position of pair (t, j) at index t*topk + j).  Optional (nullable): x_perm [T*topk][H] bf16 (token rows
+ *   in permuted order: the dispatch buffer, whose rows for the experts e0 .. e1-1 are one contiguous block),
+ *   row_expert [T*topk] int32 (the expert of each permuted row), perm [T*topk] int32 (value t*topk + j),
+ *   expert_counts [E].  workspace: moe_q4_route_workspace_size(T, E, topk) bytes, 256-byte aligned.
+ *   Limits as moe_q4_forward (E <= 256, topk <= 16, H % 128 == 0).
+ */
+size_t moe_q4_route_workspace_size(int32_t T, int32_t E, int32_t topk);
+int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
+                 int32_t E, int32_t topk, int32_t* topk_ids, float* topk_w, int32_t* offsets, int32_t* pair_pos,
+                 uint16_t* x_perm, int32_t* row_expert, int32_t* perm, int32_t* expert_counts,
+                 void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * moe_q4_forward_rows -- the expert FFN on R rows that were routed elsewhere:
+ *   y_rows[r] = row_weight[r] * (SiLU(x_r . Wg_e^T) * (x_r . Wu_e^T)) . Wd_e^T,  e = row_expert[r] - e_base,
+ * computed exactly as moe_q4_forward's expert GEMMs compute a routed row (h as a bf16 hi/lo pair).
+ * x_rows [R][H] bf16; row_expert [R] int32 in [e_base, e_base + E); row_weight [R] fp32 or NULL (1);
+ * experts[3] = {gate [E*I][H], up [E*I][H], down [E*H][I]} stacked over the E local experts; y_rows [R][H]
+ * fp32.  workspace: moe_q4_rows_workspace_size(R, H, I, E) bytes, 256-byte aligned.  dev_status:
+ * Q4_ERR_SHAPE when a row's expert id is outside the range (that row then contributes zeros).
+ */
+size_t moe_q4_rows_workspace_size(int32_t R, int32_t H, int32_t I, int32_t E);
+int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H, const int32_t* row_expert, int32_t e_base,
+                        const float* row_weight, int32_t E, const q4_weight* experts, int32_t I, float* y_rows,
+                        void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * moe_q4_combine -- the weighted combine in token order: y[t] = sum_j topk_w[t][j] * o_rows[pair_pos[t*topk+j]]
+ * (fp32, slot order j, deterministic).  o_rows [P][H] fp32 (the expert outputs in permuted order);
+ * pair_pos, topk_w as moe_q4_route returns them; y [T][H] fp32 or bf16.  H % 4 == 0.  dev_status:
+ * Q4_ERR_SHAPE when a position is outside [0, P) (that term is left out).
+ */
+int moe_q4_combine(const float* o_rows, int32_t P, int32_t H, const int32_t* pair_pos, const float* topk_w,
+                   int32_t T, int32_t topk, void* y, int32_t out_dtype, int32_t* dev_status, void* stream);
 
 /*
  * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate device memory.

@@ -185,105 +185,7 @@ int act_quant_launch(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float*
     return q4_launch_status();
 }
 
-// The MoE intermediate h as the gate/up GEMM stores it: each row [k/64][hi 64 | lo 64] bf16, value
-// hi + lo (exact in fp32: lo is at most half an ulp of hi).  One warp per row; 16-byte word w of values
-// 8w .. 8w+7 has its hi values at uint4 (w / 8) * 16 + w % 8 of the row and its lo values 8 uint4 later.
-// W: words per lane kept in registers (k <= 256 W); W = 0: any k, read twice.
-template <int W>
-__global__ void __launch_bounds__(256) act_quant_hilo_kernel(const __nv_bfloat16* __restrict__ h, int m, int k,
-                                                             int8_t* __restrict__ xq, float* __restrict__ scale_a,
-                                                             int32_t* status)
-{
-    const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
-    const int lane = threadIdx.x & 31;
-    if (row >= m) return;
-    const uint4* hr = reinterpret_cast<const uint4*>(h + row * 2 * k);
-    uint2* out = reinterpret_cast<uint2*>(xq + row * k);
-    const int n8 = k / 8;
-    auto values = [&](int w, float (&v)[8]) {
-        const int hi = (w >> 3) * 16 + (w & 7);
-        const uint4 a = __ldg(hr + hi), b = __ldg(hr + hi + 8);
-        const uint32_t ea[4] = {a.x, a.y, a.z, a.w}, eb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            v[2 * j] = __uint_as_float(ea[j] << 16) + __uint_as_float(eb[j] << 16);
-            v[2 * j + 1] = __uint_as_float(ea[j] & 0xFFFF0000u) + __uint_as_float(eb[j] & 0xFFFF0000u);
-        }
-    };
-    auto codes = [&](const float (&v)[8], float s, float r, bool exact_div) {
-        uint32_t pk[2] = {0u, 0u};
-#pragma unroll
-        for (int j = 0; j < 8; j++) pk[j / 4] |= (uint32_t)(code8(v[j], s, r, exact_div) & 0xFF) << (8 * (j & 3));
-        return make_uint2(pk[0], pk[1]);
-    };
-    uint32_t a = 0;
-    bool bad = false;
-    float v[W > 0 ? W : 1][8];
-    if constexpr (W > 0) {
-#pragma unroll
-        for (int i = 0; i < W; i++) {
-            const int w = i * 32 + lane;
-            if (w < n8) values(w, v[i]);
-            else
-#pragma unroll
-                for (int j = 0; j < 8; j++) v[i][j] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                bad |= !isfinite(v[i][j]);
-                a = max(a, __float_as_uint(v[i][j]) & 0x7FFFFFFFu);
-            }
-        }
-    } else {
-        for (int w = lane; w < n8; w += 32) {
-            float t[8];
-            values(w, t);
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                bad |= !isfinite(t[j]);
-                a = max(a, __float_as_uint(t[j]) & 0x7FFFFFFFu);
-            }
-        }
-    }
-    if (bad) q4_set_status(status, Q4_ERR_NONFINITE);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, off));
-    const float s = __uint_as_float(a) / 127.0f;
-    if (lane == 0) scale_a[row] = s;
-    const bool exact_div = !(s >= 0x1p-100f);
-    const float r = exact_div ? 0.0f : 1.0f / s;
-    if constexpr (W > 0) {
-#pragma unroll
-        for (int i = 0; i < W; i++) {
-            const int w = i * 32 + lane;
-            if (w < n8) out[w] = s == 0.0f ? make_uint2(0u, 0u) : codes(v[i], s, r, exact_div);
-        }
-    } else {
-        for (int w = lane; w < n8; w += 32) {
-            float t[8];
-            values(w, t);
-            out[w] = s == 0.0f ? make_uint2(0u, 0u) : codes(t, s, r, exact_div);
-        }
-    }
-}
-
 }  // namespace
-
-int q4_act_quant_hilo_rows(const __nv_bfloat16* h, int32_t m, int32_t k, int8_t* xq, float* scale_a,
-                           int32_t* dev_status, cudaStream_t s)
-{
-    if (!h || !xq || !scale_a) return Q4_ERR_NULL;
-    if (m < 0 || k <= 0 || k % 64) return Q4_ERR_SHAPE;
-    if (!q4_aligned16(h) || !q4_aligned16(xq) || ((uintptr_t)scale_a & 3u)) return Q4_ERR_ALIGN;
-    if (m == 0) return Q4_OK;
-    const int n8 = k / 8;
-    const int grid = (m + 7) / 8;
-    if (n8 <= 32) act_quant_hilo_kernel<1><<<grid, 256, 0, s>>>(h, m, k, xq, scale_a, dev_status);
-    else if (n8 <= 64) act_quant_hilo_kernel<2><<<grid, 256, 0, s>>>(h, m, k, xq, scale_a, dev_status);
-    else if (n8 <= 128) act_quant_hilo_kernel<4><<<grid, 256, 0, s>>>(h, m, k, xq, scale_a, dev_status);
-    else if (n8 <= 256) act_quant_hilo_kernel<8><<<grid, 256, 0, s>>>(h, m, k, xq, scale_a, dev_status);
-    else act_quant_hilo_kernel<0><<<grid, 256, 0, s>>>(h, m, k, xq, scale_a, dev_status);
-    return q4_launch_status();
-}
 
 int q4_act_quant_rows(const uint16_t* x, bool f16, int32_t m, int32_t k, int8_t* xq, float* scale_a,
                       int32_t* dev_status, cudaStream_t s)

@@ -39,7 +39,12 @@ constexpr int kMaxProblems = 256;
 constexpr int kMaxStages = 128;
 constexpr int kMaxStageProblems = 8;
 constexpr int kRedFloats = 2048;           // split-k partial sums per CTA and stage
-constexpr int kL2Ahead = 8;                // chunks prefetched into L2 beyond the ring
+#ifndef Q4_CHAIN_L2_AHEAD
+#define Q4_CHAIN_L2_AHEAD 0
+#endif
+// chunks prefetched into L2 beyond the ring (by the producer thread: its mbarrier waits then also wait for
+// the prefetches, so the default is none)
+constexpr int kL2Ahead = Q4_CHAIN_L2_AHEAD;
 
 struct ChainProblem {
     const uint16_t* x;       // bf16 [k] (null when g is set)
@@ -268,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                         bulk_g2s_hint(dst + wbytes + sbytes, P.zeros + (int64_t)c.lr * ng, (uint32_t)(c.rows * ng * 2),
                                       &full[slot], pol);
                 }
-                l2_advance(it + 1 + p.nslots + kL2Ahead);
+                if constexpr (kL2Ahead > 0) l2_advance(it + 1 + p.nslots + kL2Ahead);
                 r += c.rows;
             }
         }

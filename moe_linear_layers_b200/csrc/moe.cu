@@ -280,7 +280,9 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restr
                                                           int32_t* __restrict__ perm, int32_t* __restrict__ row_tok,
                                                           float* __restrict__ row_w, uint8_t* __restrict__ xperm,
                                                           const float* __restrict__ tok_scale,
-                                                          float* __restrict__ row_scale)
+                                                          float* __restrict__ row_scale,
+                                                          int32_t* __restrict__ pair_pos = nullptr,
+                                                          int32_t* __restrict__ row_exp = nullptr)
 {
     __shared__ int pos[kRouteTok * kMaxTopk];
     __shared__ int cid[kRouteTok * kMaxTopk];   // the chunk's expert ids, token-major
@@ -300,8 +302,11 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restr
         row_tok[p] = t0 + tl;
         row_w[p] = wts[(int64_t)(t0 + tl) * topk + j];
         if (tok_scale) row_scale[p] = tok_scale[t0 + tl];
+        if (pair_pos) pair_pos[(int64_t)t0 * topk + q] = p;   // the inverse permutation
+        if (row_exp) row_exp[p] = e;
     }
     __syncthreads();
+    if (!xperm) return;
     // gather: a warp copies whole rows, eight 16-byte loads in flight per lane before the stores
     const int vec = row_bytes / 16;  // 16-byte units per row
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nwarps = blockDim.x / 32;
@@ -419,7 +424,7 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     int rc;
     if (a8_mask & 1) {   // gate/up on the permuted rows' int8 codes
         rc = q4_moe_gateup_a8(reinterpret_cast<const int8_t*>(ws.xperm), ws.sa_row, &ex[0], &ex[1], P, H, I, E,
-                              ws.offsets, ws.tiles_gu, ws.h, status, s);
+                              ws.offsets, ws.tiles_gu, ws.h, (a8_mask & 2) != 0, status, s);
     } else {
         CUtensorMap mx, mg, mu;
         if (!make_act_map(&mx, ws.xperm, H, P, 2) || !make_packed_map(&mg, ex[0].packed, H, (uint64_t)E * I, 64) ||
@@ -437,13 +442,15 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
         a.expert_tiles = ws.tiles_gu;
         a.offsets = ws.offsets;
         a.h = ws.h;
+        a.h_f16 = (a8_mask & 2) != 0;   // an INT8 down projection quantizes h as an fp16 activation
         a.E = E;
         a.topk = topk;
         rc = launch<false, G, SYM, Mode::GateUp>(mx, mg, mu, a, sms, s);
     }
     if (rc) return rc;
-    if (a8_mask & 2) {   // h -> per-row int8 codes, then down on them
-        if ((rc = q4_act_quant_hilo_rows(ws.h, P, I, ws.hq, ws.sh_row, status, s))) return rc;
+    if (a8_mask & 2) {   // h (fp16) -> per-row int8 codes, then down on them
+        if ((rc = q4_act_quant_rows(reinterpret_cast<const uint16_t*>(ws.h), true, P, I, ws.hq, ws.sh_row, status, s)))
+            return rc;
         return q4_moe_down_a8(ws.hq, ws.sh_row, &ex[2], P, H, I, E, ws.offsets, ws.tiles_dn, ws.row_tok, ws.row_w,
                               y32, status, s);
     }
@@ -703,6 +710,198 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         rc = q4_launch_status();
     }
     return rc;
+}
+
+// ---------------------------------------------------------------------------------------------- //
+// The layer's steps as separate calls, the units of expert parallelism in its all-to-all form: routing
+// with the permutation and the dispatch buffer (moe_q4_route), the expert FFN on rows routed elsewhere
+// (moe_q4_forward_rows) and the weighted combine back into token order (moe_q4_combine).
+// ---------------------------------------------------------------------------------------------- //
+
+// Pre-routed rows: one CTA per chunk of kRouteTok rows writes the rows' local expert ids and weights
+// (topk = 1) and the chunk's expert histogram, as the route kernel does for routed tokens.  A row whose
+// expert id lies outside [e_base, e_base + E) is reported (Q4_ERR_SHAPE) and counted as expert 0 with
+// weight 0, so it contributes nothing.
+__global__ void __launch_bounds__(64) moe_rows_setup_kernel(const int32_t* __restrict__ row_expert,
+                                                            const float* __restrict__ row_weight, int R, int E,
+                                                            int e_base, int32_t* __restrict__ ids,
+                                                            float* __restrict__ wts, int32_t* __restrict__ hist,
+                                                            int32_t* status)
+{
+    __shared__ int hc[tcg::kMaxExperts];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hc[e] = 0;
+    __syncthreads();
+    const int r = blockIdx.x * kRouteTok + threadIdx.x;
+    if (threadIdx.x < kRouteTok && r < R) {
+        int e = row_expert[r] - e_base;
+        float w = row_weight ? row_weight[r] : 1.0f;
+        if (e < 0 || e >= E) {
+            q4_set_status(status, Q4_ERR_SHAPE);
+            e = 0;
+            w = 0.0f;
+        }
+        ids[r] = e;
+        wts[r] = w;
+        atomicAdd(&hc[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = hc[e];
+}
+
+// y[t] = sum_j w[t][j] * o[pair_pos[t*topk + j]] in slot order (deterministic): one CTA per token.
+__global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ o, const int32_t* __restrict__ pair_pos,
+                                                          const float* __restrict__ w, int H, int topk, int P,
+                                                          void* __restrict__ y, int out_bf16, int32_t* status)
+{
+    const int64_t t = blockIdx.x;
+    for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int j = 0; j < topk; j++) {
+            const int p = pair_pos[t * topk + j];
+            if (p < 0 || p >= P) {   // not a position of the permuted rows: report, contribute nothing
+                if (c == threadIdx.x) q4_set_status(status, Q4_ERR_SHAPE);
+                continue;
+            }
+            const float wj = w[t * topk + j];
+            const float4 v = __ldg(reinterpret_cast<const float4*>(o + (int64_t)p * H) + c);
+            acc.x = fmaf(wj, v.x, acc.x);
+            acc.y = fmaf(wj, v.y, acc.y);
+            acc.z = fmaf(wj, v.z, acc.z);
+            acc.w = fmaf(wj, v.w, acc.w);
+        }
+        if (out_bf16) {
+            __nv_bfloat162* yb = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(y) + t * H) + 2 * c;
+            yb[0] = __floats2bfloat162_rn(acc.x, acc.y);
+            yb[1] = __floats2bfloat162_rn(acc.z, acc.w);
+        } else {
+            reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + t * H)[c] = acc;
+        }
+    }
+}
+
+struct RouteWorkspace {
+    int32_t *hist, *chunk_base, *tiles_gu, *tiles_dn, *counts, *perm, *row_tok;
+    float* row_w;
+    size_t bytes;
+};
+
+static RouteWorkspace carve_route(void* base, int T, int E, int topk)
+{
+    RouteWorkspace w = {};
+    const size_t P = (size_t)T * topk, nch = (size_t)(T + kRouteTok - 1) / kRouteTok;
+    uint8_t* p = reinterpret_cast<uint8_t*>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { uint8_t* q = p ? p + o : nullptr; o += al(bytes); return q; };
+    w.hist = reinterpret_cast<int32_t*>(take(nch * E * 4));
+    w.chunk_base = reinterpret_cast<int32_t*>(take(nch * E * 4));
+    w.tiles_gu = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    w.tiles_dn = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    w.counts = reinterpret_cast<int32_t*>(take(E * 4));
+    w.perm = reinterpret_cast<int32_t*>(take(P * 4));
+    w.row_tok = reinterpret_cast<int32_t*>(take(P * 4));
+    w.row_w = reinterpret_cast<float*>(take(P * 4));
+    w.bytes = o;
+    return w;
+}
+
+extern "C" size_t moe_q4_route_workspace_size(int32_t T, int32_t E, int32_t topk)
+{
+    if (T < 0 || E <= 0 || topk <= 0) return 0;
+    return carve_route(nullptr, T, E, topk).bytes;
+}
+
+extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,
+                            int32_t E, int32_t topk, int32_t* topk_ids, float* topk_w, int32_t* offsets,
+                            int32_t* pair_pos, uint16_t* x_perm, int32_t* row_expert, int32_t* perm,
+                            int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream)
+{
+    if (!x || !router_w || !topk_ids || !topk_w || !offsets || !pair_pos || !workspace) return Q4_ERR_NULL;
+    if (T < 0 || H <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E) return Q4_ERR_SHAPE;
+    if (H % 128) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(x) || (x_perm && !q4_aligned16(x_perm)) || ((uintptr_t)workspace & 255u) ||
+        ((uintptr_t)router_w & 15u))
+        return Q4_ERR_ALIGN;
+    RouteWorkspace ws = carve_route(workspace, T, E, topk);
+    if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
+    if (T == 0) return cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream) ? Q4_ERR_CUDA : Q4_OK;
+    if (perm) ws.perm = perm;
+    if (expert_counts) ws.counts = expert_counts;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int nch = (T + kRouteTok - 1) / kRouteTok;
+    CUtensorMap mrx, mrw;
+    if (!tcg::make_map(&mrx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, T, (uint64_t)H * 2, kRouteKC, kRouteTok,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !tcg::make_map(&mrw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, router_w, H, E, (uint64_t)H * 4, kRouteKC, 64,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    constexpr int route_smem = kRouteStages * (kRouteWTile + kRouteXTile);
+    if (const cudaError_t e = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, route_smem))
+        return q4_cuda_status(e);
+    moe_route_kernel<<<nch, kRouteThreads, route_smem, s>>>(mrx, mrw, T, H, router_bias, E, topk, topk_ids, topk_w,
+                                                            ws.hist, dev_status);
+    moe_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.hist, nch, E, 128, H, ws.chunk_base, offsets, ws.counts,
+                                                   ws.tiles_gu, ws.tiles_dn);
+    moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x), T, 2 * H, E, topk, topk_ids, topk_w,
+                                           ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
+                                           reinterpret_cast<uint8_t*>(x_perm), nullptr, nullptr, pair_pos, row_expert);
+    return q4_launch_status();
+}
+
+extern "C" size_t moe_q4_rows_workspace_size(int32_t R, int32_t H, int32_t I, int32_t E)
+{
+    if (R < 0 || H <= 0 || I <= 0 || E <= 0) return 0;
+    return carve(nullptr, R, H, I, E, 1).bytes;
+}
+
+extern "C" int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H, const int32_t* row_expert,
+                                   int32_t e_base, const float* row_weight, int32_t E, const q4_weight* experts,
+                                   int32_t I, float* y_rows, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream)
+{
+    if (!x_rows || !row_expert || !experts || !y_rows || !workspace) return Q4_ERR_NULL;
+    if (R < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts) return Q4_ERR_SHAPE;
+    if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
+    for (int i = 0; i < 3; i++) {
+        const q4_weight& w = experts[i];
+        if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
+        if (w.group != experts[0].group || w.symmetric != experts[0].symmetric) return Q4_ERR_UNSUPPORTED;
+        if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
+            return Q4_ERR_ALIGN;
+    }
+    if (experts[0].group != 32 && experts[0].group != 64 && experts[0].group != 128) return Q4_ERR_UNSUPPORTED;
+    if (experts[0].n != E * I || experts[0].k != H || experts[1].n != E * I || experts[1].k != H ||
+        experts[2].n != E * H || experts[2].k != I)
+        return Q4_ERR_SHAPE;
+    if (!q4_aligned16(x_rows) || !q4_aligned16(y_rows) || ((uintptr_t)workspace & 255u)) return Q4_ERR_ALIGN;
+    Workspace ws = carve(workspace, R, H, I, E, 1);
+    if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
+    if (R == 0) return Q4_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int nch = (R + kRouteTok - 1) / kRouteTok;
+    moe_rows_setup_kernel<<<nch, 64, 0, s>>>(row_expert, row_weight, R, E, e_base, ws.ids, ws.wts, ws.hist, dev_status);
+    moe_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.hist, nch, E, I, H, ws.chunk_base, ws.offsets, ws.counts,
+                                                   ws.tiles_gu, ws.tiles_dn);
+    moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x_rows), R, 2 * H, E, 1, ws.ids, ws.wts,
+                                           ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
+                                           reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr);
+    if (const cudaError_t e = cudaMemsetAsync(y_rows, 0, (size_t)R * H * sizeof(float), s)) return q4_cuda_status(e);
+    int rc = q4_launch_status();
+    if (rc) return rc;
+    return launch_experts_any(ws, experts, R, H, I, E, 1, y_rows, dev_status, s, 0);
+}
+
+extern "C" int moe_q4_combine(const float* o_rows, int32_t P, int32_t H, const int32_t* pair_pos, const float* topk_w,
+                              int32_t T, int32_t topk, void* y, int32_t out_dtype, int32_t* dev_status, void* stream)
+{
+    if (!o_rows || !pair_pos || !topk_w || !y) return Q4_ERR_NULL;
+    if (T < 0 || P < 0 || H <= 0 || topk < 1 || topk > kMaxTopk || H % 4) return Q4_ERR_SHAPE;
+    if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (!q4_aligned16(o_rows) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
+    if (T == 0) return Q4_OK;
+    moe_combine_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(o_rows, pair_pos, topk_w, H, topk, P, y,
+                                                            out_dtype == Q4_OUT_BF16, dev_status);
+    return q4_launch_status();
 }
 
 // ---------------------------------------------------------------------------------------------- //

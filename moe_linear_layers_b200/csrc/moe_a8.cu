@@ -9,7 +9,7 @@ namespace {
 
 template <int G, bool SYM>
 int gateup(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H, int I, int E,
-           const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, int32_t* status, cudaStream_t s)
+           const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, bool h_f16, int32_t* status, cudaStream_t s)
 {
     using namespace tcg;
     CUtensorMap mx, mg, mu;
@@ -29,6 +29,7 @@ int gateup(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_we
     a.expert_tiles = tiles;
     a.offsets = offsets;
     a.h = h;
+    a.h_f16 = h_f16;
     a.E = E;
     return launch<true, G, SYM, Mode::GateUp>(mx, mg, mu, a, q4_num_sms(), s);
 }
@@ -62,14 +63,14 @@ int down(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, i
 }  // namespace
 
 int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H,
-                     int I, int E, const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, int32_t* status,
-                     cudaStream_t s)
+                     int I, int E, const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, bool h_f16,
+                     int32_t* status, cudaStream_t s)
 {
     if (gate->group == 128)
-        return gate->symmetric ? gateup<128, true>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, status, s)
-                               : gateup<128, false>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, status, s);
-    return gate->symmetric ? gateup<64, true>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, status, s)
-                           : gateup<64, false>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, status, s);
+        return gate->symmetric ? gateup<128, true>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, h_f16, status, s)
+                               : gateup<128, false>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, h_f16, status, s);
+    return gate->symmetric ? gateup<64, true>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, h_f16, status, s)
+                           : gateup<64, false>(xq, sa, gate, up, P, H, I, E, offsets, tiles, h, h_f16, status, s);
 }
 
 int q4_moe_down_a8(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E,

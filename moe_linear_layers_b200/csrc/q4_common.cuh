@@ -67,18 +67,13 @@ static inline bool q4_aligned16(const void* p) { return (reinterpret_cast<uintpt
 int q4_act_quant_rows(const uint16_t* x, bool f16, int32_t m, int32_t k, int8_t* xq, float* scale_a,
                       int32_t* dev_status, cudaStream_t s);
 
-// Per-row INT8 quantization of the MoE intermediate h stored as bf16 hi/lo pairs ([m][k/64][hi 64 | lo
-// 64], value hi + lo), the input of the INT8 down projection (act_quant.cu).  Same arithmetic and status
-// as act_quant_per_token on the fp32 values hi + lo; k % 64 == 0.
-int q4_act_quant_hilo_rows(const __nv_bfloat16* h, int32_t m, int32_t k, int8_t* xq, float* scale_a,
-                           int32_t* dev_status, cudaStream_t s);
-
 // The MoE layer's grouped expert GEMMs on int8 activation codes (moe_a8.cu): gate/up with the SwiGLU
-// epilogue into h (bf16 hi/lo pairs), and down with the weighted reduction into y32.  P permuted rows;
+// epilogue into h (bf16 hi/lo pairs, or fp16 when h_f16: the activation an INT8 down projection
+// quantizes), and down with the weighted reduction into y32.  P permuted rows;
 // offsets and tiles as the 16-bit grouped GEMMs take them; sa / sh the per-permuted-row activation scales.
 int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_weight* up, int P, int H,
-                     int I, int E, const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, int32_t* status,
-                     cudaStream_t s);
+                     int I, int E, const int32_t* offsets, const int32_t* tiles, __nv_bfloat16* h, bool h_f16,
+                     int32_t* status, cudaStream_t s);
 int q4_moe_down_a8(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E,
                    const int32_t* offsets, const int32_t* tiles, const int32_t* row_tok, const float* row_w,
                    float* y32, int32_t* status, cudaStream_t s);

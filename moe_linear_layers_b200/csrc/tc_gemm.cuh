@@ -26,7 +26,8 @@
 //           expert's rows of the permuted activations (bf16, or int8 codes with per-row scales s_a);
 //           epilogue h = SiLU(gate) * up in fp32, stored as a pair of bf16 values hi = bf16(h) and
 //           lo = bf16(h - hi), which together hold h to about 2^-17 of its magnitude (gate and up each
-//           times s_a first with int8 codes).  Row layout of h: [I/64][hi 64 | lo 64].
+//           times s_a first with int8 codes).  Row layout of h: [I/64][hi 64 | lo 64].  For a down
+//           projection on INT8 activations, h is stored instead as the fp16 activation it quantizes.
 //   Down    A = 128 rows of the expert's down projection (bf16 codes, or int8), B = h: per K step one
 //           MMA on the hi values and one on the lo values into the same accumulator (or, int8, the
 //           codes of h and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
@@ -63,16 +64,19 @@ constexpr int KBLK = 128;                // K per stage
 constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
-constexpr int kThreads = 768;            // 24 warps = 6 warpgroups
+#ifndef Q4_CONV_SETS
+#define Q4_CONV_SETS 2
+#endif
+constexpr int kConvSets = Q4_CONV_SETS;  // converter warpgroups, alternate stages
+constexpr int kThreads = 640 + 128 * (kConvSets - 1);   // 20 or 24 warps
 constexpr int kIssuers = 4;              // MMA issuer threads (warps 0-3)
-constexpr int kConvSets = 2;             // converter warpgroups, alternate stages
-// registers per thread: the launch allocation (65536 / 768, rounded down to a multiple of 8) and the
+// registers per thread: the launch allocation (65536 / threads, rounded down to a multiple of 8) and the
 // per-warpgroup split after setmaxnreg; the split may not exceed the launch allocation
-constexpr int kLaunchRegs = 80;
-constexpr int kRegsIssue = 48;           // MMA issuers
-constexpr int kRegsProd = 40;            // TMA producers, parameter loader
-constexpr int kRegsConv = 64;            // converters (each set)
-constexpr int kRegsEpi = 128;            // epilogue (two warpgroups)
+constexpr int kLaunchRegs = kConvSets == 1 ? 96 : 80;
+constexpr int kRegsIssue = 48;                           // MMA issuers
+constexpr int kRegsProd = kConvSets == 1 ? 56 : 40;      // TMA producers, parameter loader
+constexpr int kRegsConv = kConvSets == 1 ? 88 : 64;      // converters (each set)
+constexpr int kRegsEpi = kConvSets == 1 ? 144 : 128;     // epilogue (two warpgroups)
 static_assert(128 * (kRegsIssue + kRegsProd + kConvSets * kRegsConv) + 256 * kRegsEpi <= kThreads * kLaunchRegs,
               "register split");
 constexpr uint32_t kTmemCols = 512;
@@ -125,7 +129,8 @@ struct Args {
     const int32_t* offsets;        // [E+1] first permuted row of each expert
     const int32_t* row_tok;        // Down: [P] token of each permuted row
     const float* row_w;            // Down: [P] routing weight of each permuted row
-    __nv_bfloat16* h;              // GateUp output [P][N/64][hi 64 | lo 64]
+    __nv_bfloat16* h;              // GateUp output [P][N/64][hi 64 | lo 64], or fp16 [P][N] when h_f16
+    int h_f16;                     // GateUp: h for an INT8 down projection, stored as the fp16 activation
     int E, topk;
 };
 
@@ -776,7 +781,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const int mb = T.m0 + half * 64;
                     const int rows = min(64, T.m_end - mb);
                     // intermediate index i = n0 + r: its hi value in block n0 / 64 of the row, lo 64 later
-                    __nv_bfloat16* hb = p.h + (int64_t)mb * (2 * p.N) + 2 * T.n0 + r;
+                    // (or its fp16 value at column i of an [P][N] row)
+                    const bool f16 = p.h_f16;
+                    const int64_t hstride = f16 ? p.N : 2 * p.N;
+                    __nv_bfloat16* hb = p.h + (int64_t)mb * hstride + (f16 ? T.n0 : 2 * T.n0) + r;
                     auto swiglu = [&](int j) {
                         float gv = accv(j), uv = xb[j * 64 + r];
                         if constexpr (INT8) {   // the row's activation scale
@@ -785,9 +793,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             uv *= sa;
                         }
                         const float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-                        hb[(int64_t)j * (2 * p.N)] = hi;
-                        hb[(int64_t)j * (2 * p.N) + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+                        if (f16) {
+                            reinterpret_cast<__half*>(hb)[(int64_t)j * hstride] = __float2half_rn(hv);
+                        } else {
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+                            hb[(int64_t)j * hstride] = hi;
+                            hb[(int64_t)j * hstride + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+                        }
                     };
                     if (rows == 64) {
 #pragma unroll

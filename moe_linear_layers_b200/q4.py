@@ -36,7 +36,9 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_q
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
             "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes",
-            "moe_q4_forward_range", "q4_linear_w4a16_chain_sync_bytes", "q4_linear_w4a16_chain")
+            "moe_q4_forward_range", "q4_linear_w4a16_chain_sync_bytes", "q4_linear_w4a16_chain",
+            "moe_q4_route_workspace_size", "moe_q4_route", "moe_q4_rows_workspace_size", "moe_q4_forward_rows",
+            "moe_q4_combine")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -82,6 +84,14 @@ _lib.q4_linear_w4a16_chain_sync_bytes.argtypes = [_i32]
 _lib.q4_linear_w4a16_chain.argtypes = [_i32, ctypes.POINTER(_i32), ctypes.POINTER(_p), ctypes.POINTER(_p),
                                        ctypes.POINTER(_p), ctypes.POINTER(q4_weight), ctypes.POINTER(_p), _i32, _p, _p,
                                        _p]
+_lib.moe_q4_route_workspace_size.restype = _sz
+_lib.moe_q4_route_workspace_size.argtypes = [_i32, _i32, _i32]
+_lib.moe_q4_route.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p, _p]
+_lib.moe_q4_rows_workspace_size.restype = _sz
+_lib.moe_q4_rows_workspace_size.argtypes = [_i32, _i32, _i32, _i32]
+_lib.moe_q4_forward_rows.argtypes = [_p, _i32, _i32, _p, _i32, _p, _i32, ctypes.POINTER(q4_weight), _i32, _p, _p, _sz,
+                                     _p, _p]
+_lib.moe_q4_combine.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, _p, _i32, _p, _p]
 _lib.moe_q4_forward_noalloc.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p,
                                         _i32, _p, _p, _p, _p, _p, _p, _p]
 
@@ -488,3 +498,115 @@ def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias:
                                        od, None, None, None, None, None, _ptr(dev_status), _stream(stream)),
            "moe_q4_forward_noalloc")
     return y
+
+
+# ---------------------------------------------------------------------------------------------- #
+# the layer's steps as separate calls, and expert parallelism in its all-to-all form
+# ---------------------------------------------------------------------------------------------- #
+
+def moe_q4_route(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                 dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """Routing and the permutation of the MoE layer (moe_q4_route): returns a dict of device tensors
+    topk_ids [T][topk] i32, topk_w [T][topk] f32, offsets [E+1] i32, pair_pos [T*topk] i32 (the permuted
+    position of each (token, slot) pair), x_perm [T*topk][H] bf16 (the rows in expert order: the dispatch
+    buffer), row_expert [T*topk] i32 (the expert of each permuted row)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    dev = x.device
+    P = T * topk
+    out = {"topk_ids": torch.empty((T, topk), dtype=torch.int32, device=dev),
+           "topk_w": torch.empty((T, topk), dtype=torch.float32, device=dev),
+           "offsets": torch.empty((E + 1,), dtype=torch.int32, device=dev),
+           "pair_pos": torch.empty((P,), dtype=torch.int32, device=dev),
+           "x_perm": torch.empty((P, H), dtype=torch.bfloat16, device=dev),
+           "row_expert": torch.empty((P,), dtype=torch.int32, device=dev)}
+    ws = torch.empty((max(int(_lib.moe_q4_route_workspace_size(T, E, topk)), 1),), dtype=torch.uint8, device=dev)
+    _check(_lib.moe_q4_route(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, _ptr(out["topk_ids"]),
+                             _ptr(out["topk_w"]), _ptr(out["offsets"]), _ptr(out["pair_pos"]), _ptr(out["x_perm"]),
+                             _ptr(out["row_expert"]), None, None, _ptr(ws), ws.numel(), _ptr(dev_status),
+                             _stream(stream)), "moe_q4_route")
+    return out
+
+
+def moe_q4_forward_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, e_base: int, experts: tuple, I: int,
+                        row_weight: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """The expert FFN on rows routed elsewhere (moe_q4_forward_rows): y[r] = row_weight[r] *
+    FFN_{row_expert[r] - e_base}(x_rows[r]), fp32 [R][H]; experts = (gate, up, down) stacked over the E
+    local experts (E = gate.n / I)."""
+    _dev(x_rows, torch.bfloat16, "x_rows")
+    _dev(row_expert, torch.int32, "row_expert")
+    R, H = x_rows.shape
+    E = experts[0].n // I
+    if y is None:
+        y = torch.empty((R, H), dtype=torch.float32, device=x_rows.device)
+    _dev(y, torch.float32, "y")
+    _out(y, (R, H), x_rows.device)
+    if workspace is None:
+        workspace = torch.empty((max(int(_lib.moe_q4_rows_workspace_size(R, H, I, E)), 1),), dtype=torch.uint8,
+                                device=x_rows.device)
+    descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _check(_lib.moe_q4_forward_rows(_ptr(x_rows), R, H, _ptr(row_expert), int(e_base), _ptr(row_weight), E, descs, I,
+                                    _ptr(y), _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
+           "moe_q4_forward_rows")
+    return y
+
+
+def moe_q4_combine(o_rows: torch.Tensor, pair_pos: torch.Tensor, topk_w: torch.Tensor, out_dtype=torch.float32,
+                   y: torch.Tensor | None = None, dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[t] = sum_j topk_w[t][j] * o_rows[pair_pos[t*topk + j]] (moe_q4_combine), slot order j."""
+    _dev(o_rows, torch.float32, "o_rows")
+    _dev(pair_pos, torch.int32, "pair_pos")
+    _dev(topk_w, torch.float32, "topk_w")
+    P, H = o_rows.shape
+    T, topk = topk_w.shape
+    if y is None:
+        y = torch.empty((T, H), dtype=out_dtype, device=o_rows.device)
+    od = _out(y, (T, H), o_rows.device)
+    _check(_lib.moe_q4_combine(_ptr(o_rows), P, H, _ptr(pair_pos), _ptr(topk_w), T, topk, _ptr(y), od,
+                               _ptr(dev_status), _stream(stream)), "moe_q4_combine")
+    return y
+
+
+def moe_q4_forward_ep(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Tensor | None, topk: int,
+                      local_experts: tuple, I: int, group=None, out_dtype=torch.float32, fns: dict | None = None,
+                      dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Expert-parallel MoE layer, all-to-all form.  Every rank holds its own tokens x [T_r][H] and the weights
+    of its experts expert_range(rank, world, E) only.  Per rank: route its tokens (the permutation puts the
+    rows in expert order, so the rows for rank d are one contiguous block); exchange the block sizes; send
+    each block to the rank that owns its experts and receive the rows routed to this rank's experts (one
+    all-to-all of bf16 rows and one of their expert ids); run the local experts on the received rows; send
+    the fp32 results back (the reverse all-to-all) and combine them with the routing weights in token
+    order.  Each routed row crosses the interconnect once each way.  fns replaces the three device steps
+    (route, rows, combine) with host implementations for tests on CPU ranks."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    E = router_w.shape[0]
+    T, H = x.shape
+    fns = fns or {}
+    route = fns.get("route", lambda: moe_q4_route(x, router_w, router_bias, topk, dev_status=dev_status))
+    r = route()
+    bounds = [expert_range(d, world, E) for d in range(world)]
+    off = r["offsets"].to("cpu")
+    send = [int(off[e1] - off[e0]) for (e0, e1) in bounds]
+    cdev = r["offsets"].device if dist.get_backend(group) == "nccl" else torch.device("cpu")
+    send_t = torch.tensor(send, dtype=torch.int64, device=cdev)
+    recv_t = torch.empty_like(send_t)
+    dist.all_to_all_single(recv_t, send_t, group=group)
+    recv = [int(v) for v in recv_t.to("cpu")]
+    # rows travel as bytes (2 H per row), which every backend moves as they are
+    rows_in = torch.empty((sum(recv), 2 * H), dtype=torch.uint8, device=r["x_perm"].device)
+    dist.all_to_all_single(rows_in, r["x_perm"].contiguous().view(torch.uint8), recv, send, group=group)
+    exp_in = torch.empty((sum(recv),), dtype=torch.int32, device=r["row_expert"].device)
+    dist.all_to_all_single(exp_in, r["row_expert"], recv, send, group=group)
+    e0, e1 = bounds[rank]
+    rows_fn = fns.get("rows", lambda xr, er, eb: moe_q4_forward_rows(xr, er, eb, local_experts, I, dev_status=dev_status))
+    o_in = rows_fn(rows_in.view(torch.bfloat16), exp_in, e0)
+    o_back = torch.empty((T * topk, H), dtype=torch.float32, device=o_in.device)
+    dist.all_to_all_single(o_back, o_in, send, recv, group=group)
+    combine = fns.get("combine", lambda o, pp, w: moe_q4_combine(o, pp, w, out_dtype=out_dtype, dev_status=dev_status))
+    return combine(o_back, r["pair_pos"], r["topk_w"])

@@ -219,3 +219,36 @@ def test_chain_validation():
     g = (P * 2)(None, FAKE)
     assert call([0, 1, 2], w2, gate=g, up=(P * 2)(None, None)) == q4.Q4_ERR_NULL   # gated without up
     assert call([0, 1, 2], w2, gate=g, up=(P * 2)(None, FAKE + 8)) == q4.Q4_ERR_ALIGN
+
+
+def test_moe_steps_validation():
+    L = q4._lib
+    T, H, I, E, topk = 64, 256, 128, 8, 2
+    rws = L.moe_q4_route_workspace_size(T, E, topk)
+    assert rws > 0 and L.moe_q4_route_workspace_size(T, 0, topk) == 0
+
+    def route(x=FAKE, ids=FAKE, pp=FAKE, e=E, k=topk, ws=FAKE, wsb=rws, xp=None):
+        return L.moe_q4_route(x, T, H, FAKE, None, e, k, ids, FAKE, FAKE, pp, xp, None, None, None, ws, wsb, None, None)
+
+    assert route(ids=None) == q4.Q4_ERR_NULL
+    assert route(pp=None) == q4.Q4_ERR_NULL
+    assert route(k=9, e=8) == q4.Q4_ERR_SHAPE
+    assert route(e=300) == q4.Q4_ERR_SHAPE
+    assert route(x=FAKE + 2) == q4.Q4_ERR_ALIGN
+    assert route(xp=FAKE + 8) == q4.Q4_ERR_ALIGN
+    assert route(ws=FAKE + 16) == q4.Q4_ERR_ALIGN
+    assert route(wsb=rws - 1) == q4.Q4_ERR_WORKSPACE
+    ex = (q4.q4_weight * 3)(_w(n=E * I, k=H), _w(n=E * I, k=H), _w(n=E * H, k=I))
+    need = L.moe_q4_rows_workspace_size(T, H, I, E)
+
+    def rows(exw=ex, y=FAKE, wsb=need, e=E):
+        return L.moe_q4_forward_rows(FAKE, T, H, FAKE, 0, None, e, exw, I, y, FAKE, wsb, None, None)
+
+    assert rows(y=None) == q4.Q4_ERR_NULL
+    assert rows(e=7) == q4.Q4_ERR_SHAPE            # weights stacked for 8 experts
+    assert rows(y=FAKE + 4) == q4.Q4_ERR_ALIGN
+    assert rows(wsb=need - 1) == q4.Q4_ERR_WORKSPACE
+    assert L.moe_q4_combine(None, 10, H, FAKE, FAKE, 5, 2, FAKE, 0, None, None) == q4.Q4_ERR_NULL
+    assert L.moe_q4_combine(FAKE, 10, 6, FAKE, FAKE, 5, 2, FAKE, 0, None, None) == q4.Q4_ERR_SHAPE
+    assert L.moe_q4_combine(FAKE, 10, H, FAKE, FAKE, 5, 2, FAKE, 3, None, None) == q4.Q4_ERR_UNSUPPORTED
+    assert L.moe_q4_combine(FAKE, 10, H, FAKE, FAKE, 5, 2, FAKE + 8, 0, None, None) == q4.Q4_ERR_ALIGN
