@@ -59,7 +59,8 @@ typedef enum {
     Q4_ERR_WORKSPACE = -5,   /* workspace too small */
     Q4_ERR_CUDA = -6,        /* a CUDA call failed (launch error) */
     Q4_ERR_NONFINITE = -7,   /* (device) non-finite input, or a scale that overflows fp16 */
-    Q4_ERR_TIMEOUT = -8      /* (device) a bounded wait inside a kernel gave up */
+    Q4_ERR_TIMEOUT = -8,     /* (device) a bounded wait inside a kernel gave up */
+    Q4_ERR_BOUNDS = -9       /* (device, debug build only) a computed index fell outside its buffer */
 } q4_status;
 
 enum { Q4_OUT_F32 = 0, Q4_OUT_BF16 = 1 };
@@ -82,6 +83,14 @@ int q4_version(void);
 
 /* Description of the last CUDA error behind a Q4_ERR_CUDA return on the calling host thread. */
 const char* q4_last_cuda_error_string(void);
+
+/*
+ * Build flags of the loaded library: bit 0 set in the debug build (libq4_debug.so, compiled with
+ * Q4_DEBUG), whose kernels check every global-memory index they compute against the extent of its buffer
+ * and, instead of making the access, record Q4_ERR_BOUNDS in dev_status.  The debug build stands in for
+ * a memory checker; it computes the same results as the release build, more slowly.
+ */
+int q4_build_flags(void);
 
 /*
  * q4_quantize_pack -- round-to-nearest group quantization and packing of an fp32 matrix.

@@ -35,11 +35,21 @@ extern "C" const char* q4_status_string(int status)
         case Q4_ERR_CUDA: return "CUDA error";
         case Q4_ERR_NONFINITE: return "non-finite input or scale";
         case Q4_ERR_TIMEOUT: return "bounded wait timed out";
+        case Q4_ERR_BOUNDS: return "index out of bounds (debug build)";
         default: return "unknown status";
     }
 }
 
 extern "C" int q4_version(void) { return 1; }
+
+extern "C" int q4_build_flags(void)
+{
+#ifdef Q4_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
 
 static thread_local cudaError_t q4_last_error = cudaSuccess;
 

@@ -311,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
                     const int rr = hi ? rb : ra;
 #pragma unroll
                     for (int mm = 0; mm < MT; mm++) {
-                        if constexpr (KSPLIT == 1) store_y(P.y, (int64_t)mm * P.n + rs + rr, pa[mm], p.out_bf16);
+                        if constexpr (KSPLIT == 1)
+                            store_y(P.y, (int64_t)mm * P.n + rs + rr, pa[mm], p.out_bf16, (int64_t)p.m * P.n, p.status);
                         else red[((rs - r0 + rr) * KSPLIT + ks) * MT + mm] = pa[mm];
                     }
                 }
@@ -324,7 +325,8 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
                     float v = pa[0];
 #pragma unroll
                     for (int mm = 1; mm < MT; mm++) if (lane == mm) v = pa[mm];
-                    if constexpr (KSPLIT == 1) store_y(P.y, (int64_t)lane * P.n + rs + ra, v, p.out_bf16);
+                    if constexpr (KSPLIT == 1)
+                        store_y(P.y, (int64_t)lane * P.n + rs + ra, v, p.out_bf16, (int64_t)p.m * P.n, p.status);
                     else red[((rs - r0 + ra) * KSPLIT + ks) * MT + lane] = v;
                 }
             }
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
             float v = 0.0f;
 #pragma unroll
             for (int t = 0; t < KSPLIT; t++) v += red[(rr * KSPLIT + t) * MT + mm];
-            store_y(P.y, (int64_t)mm * P.n + r0 + rr, v, p.out_bf16);
+            store_y(P.y, (int64_t)mm * P.n + r0 + rr, v, p.out_bf16, (int64_t)p.m * P.n, p.status);
         }
     }
 }

@@ -13,8 +13,11 @@
 //  * one CTA per SM (cooperative launch: every CTA is resident), 16 compute warps and a producer warp;
 //  * each stage's weight rows (the concatenation of its problems' rows) are split evenly over the CTAs;
 //  * the producer streams the CTA's rows of every stage, in stage order, through a shared-memory ring
-//    with cp.async.bulk (evict-first in L2, so that activations and outputs stay cached), and prefetches
-//    rows further ahead into L2.  It never waits for the dependency: weights do not depend on it;
+//    with cp.async.bulk (evict-first in L2, so that activations and outputs stay cached).  It never waits
+//    for the dependency: weights do not depend on it.  Nor does it wait on an mbarrier for a free slot:
+//    on this GPU a thread's mbarrier wait also waits for that thread's own bulk copies in flight, which
+//    would leave one chunk in flight per HBM round trip; the compute warps publish the chunks they have
+//    finished in per-warp shared-memory counters, which the producer polls with plain loads;
 //  * the compute warps of stage s wait until every CTA has finished stage s-1 (one thread polls the
 //    stage's arrival counter with acquire loads, bounded in time), then read x -- which may be an output of
 //    an earlier stage -- and reduce the rows already waiting in the ring; they then publish their own
@@ -80,13 +83,6 @@ struct ChainParams {
 
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p)
 {
     uint32_t v;
@@ -105,6 +101,28 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
                  ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar)), "l"(pol) : "memory");
+}
+
+// Wait (plain shared-memory loads, a short sleep between rounds so the compute warps on the producer's
+// scheduler keep their issue slots) until every compute warp has finished `target` chunks.  Bounded: after
+// tc::kWaitLimitNs, or when the CTA's abort flag rises, it records Q4_ERR_TIMEOUT / returns false.
+__device__ __forceinline__ bool poll_consumed(const uint32_t* consumed, uint32_t target, int32_t* status,
+                                              volatile int* abort_cta)
+{
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (uint32_t round = 0;; round++) {
+        bool ok = true;
+#pragma unroll
+        for (int i = 0; i < kCW; i++) ok &= tc::lds_weak(consumed + i) >= target;
+        if (ok) return true;
+        if (*abort_cta) return false;
+        if (tc::wait_expired(t0, tc::kWaitLimitNs, round, 1u << 12)) {
+            q4_set_status(status, Q4_ERR_TIMEOUT);
+            *abort_cta = 1;
+            return false;
+        }
+        __nanosleep(64);
+    }
 }
 
 // The CTA's rows [a, b) of stage s, and its chunks: a chunk is at most rps rows of one problem.
@@ -209,8 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
 {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
-    uint64_t* empty = full + p.nslots;
-    volatile int* abort_cta = reinterpret_cast<volatile int*>(empty + p.nslots);
+    uint32_t* consumed = reinterpret_cast<uint32_t*>(full + p.nslots);   // [kCW] chunks finished per warp
+    volatile int* abort_cta = reinterpret_cast<volatile int*>(consumed + kCW);
     uint4* xs = reinterpret_cast<uint4*>(smem + p.xs_off);
     float* xinv = reinterpret_cast<float*>(smem + p.xinv_off);
     float* red = reinterpret_cast<float*>(smem + p.red_off);
@@ -219,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
     const int ng_of = p.group;   // k / group per stage below
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < p.nslots; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kCW); }
+        for (int i = 0; i < p.nslots; i++) tc::mbar_init(&full[i], 1);
+        for (int i = 0; i < kCW; i++) consumed[i] = 0;
         *abort_cta = 0;
         tc::fence_mbar_init();
     }
@@ -258,9 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                 const Chunk c = chunk_at(p, S, r, a, b);
                 const ChainProblem& P = p.prob[c.pi];
                 const int slot = it % p.nslots;
-                if (it >= (uint32_t)p.nslots &&
-                    !(ok = tc::mbar_wait(&empty[slot], ((it / p.nslots) & 1) ^ 1, p.status, abort_cta)))
-                    break;
+                if (it >= (uint32_t)p.nslots) {
+                    // chunk it - nslots, the slot's previous one, is finished by every compute warp
+                    if (!(ok = poll_consumed(consumed, it - p.nslots + 1, p.status, abort_cta))) break;
+                    // the warps' reads of the slot (generic proxy) before the copy's writes (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
                 uint8_t* dst = ring + slot * p.slot_bytes;
                 const uint32_t wb = (uint32_t)(c.rows * rowbytes);
                 uint32_t bytes = wb;
@@ -301,7 +323,11 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                 const uint32_t* cnt = p.sync + s;   // arrivals at stage s - 1
                 const uint64_t t0 = tc::globaltimer_ns();
                 for (uint32_t i = 0;; i++) {
-                    if (ld_acquire_gpu(cnt) >= gridDim.x) break;
+                    if (ld_relaxed_gpu(cnt) >= gridDim.x) {
+                        // acquire: the arrivals' released writes (stage s-1's outputs) are visible from here
+                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                        break;
+                    }
                     if ((i & 7u) == 7u && ld_relaxed_gpu(p.sync)) { *abort_cta = 1; break; }
                     if ((i & 63u) == 63u) {
                         if (tc::wait_expired(t0, tc::kWaitLimitNs, i >> 6, 64)) {
@@ -359,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
             // (after an expired wait the warp skips its rows but keeps to the barriers below, so that every
             // compute warp leaves together at the end of the stage; the abort word stops the other CTAs)
             const bool have = !*abort_cta && tc::mbar_wait(&full[slot], (it / p.nslots) & 1, p.status, abort_cta);
-            if (!have && !*abort_cta) {
+            if (!have) {   // (the producer may have given up first: the other CTAs must learn of it too)
                 *abort_cta = 1;
                 atomicExch(p.sync, 1u);
             }
@@ -387,12 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                 for (int off = 8; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
                 if ((lane & 15) == 0 && (!hi || hasb)) {
                     const int rr = hi ? rb : ra;
-                    if (ks == 1) store_y(P.y, c.lr + rr, v, p.out_bf16);
+                    if (ks == 1) store_y(P.y, c.lr + rr, v, p.out_bf16, P.n, p.status);
                     else red[(c.cr + rr) * ks + kq] = v;
                 }
             }
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[slot]);
+            if (lane == 0) tc::sts_publish(&consumed[warp], it + 1);   // this warp is done with the slot
             r += c.rows;
         }
         compute_bar();   // every row of the stage is reduced (and, ksplit 1, stored)
@@ -402,17 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                 float v = 0.0f;
                 for (int t = 0; t < ks; t++) v += red[i * ks + t];
                 const Chunk c = chunk_at(p, S, a + i, a, b);
-                store_y(p.prob[c.pi].y, c.lr, v, p.out_bf16);
+                store_y(p.prob[c.pi].y, c.lr, v, p.out_bf16, p.prob[c.pi].n, p.status);
             }
             compute_bar();
         }
-        // publish: this CTA's outputs of stage s are written
+        // publish: this CTA's outputs of stage s are written (the barrier above orders every compute
+        // thread's stores before thread 0's release, which carries them to the other CTAs' acquire)
         if (threadIdx.x == 0) {
-            __threadfence();
-            const uint32_t old = atomicAdd(p.sync + 1 + s, 1u);
-            if (s == p.nstages - 1 && old == gridDim.x - 1) {
-                // the last arrival of the last stage: every CTA is past every wait; leave the counters zero
-                for (int i = 1; i <= p.nstages; i++) p.sync[i] = 0u;
+            if (s < p.nstages - 1) {
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.sync + 1 + s) : "memory");
+            } else {
+                uint32_t old;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.sync + 1 + s) : "memory");
+                if (old == gridDim.x - 1) {
+                    // the last arrival of the last stage: every CTA is past every wait; leave the counters zero
+                    for (int i = 1; i <= p.nstages; i++) p.sync[i] = 0u;
+                }
             }
         }
     }
@@ -482,7 +513,7 @@ int q4_gemv_w4a16_chain_launch(int n_stages, const int32_t* stage_begin, const u
     P.xinv_off = kmax * 2;
     P.red_off = P.xinv_off + (kmax / 64) * 4;
     P.bar_off = (P.red_off + redmax * 4 + 127) & ~127;
-    const int bar_bytes = 2 * 8 * 8 + 16;   // up to 8 slots' full and empty barriers, the CTA abort flag
+    const int bar_bytes = 8 * 8 + 4 * kCW + 16;   // up to 8 slots' full barriers, consumed counters, abort flag
     P.ring_off = (P.bar_off + bar_bytes + 127) & ~127;
     const int avail = 227 * 1024 - P.ring_off;
     P.nslots = std::min(8, avail / slot_bytes);

@@ -173,8 +173,10 @@ __device__ __forceinline__ void row_dot(const uint8_t* wrow, const __half* srow,
     }
 }
 
-__device__ __forceinline__ void store_y(void* y, int64_t o, float v, int out_bf16)
+// y[o] of a buffer of n values (the debug build checks o against n)
+__device__ __forceinline__ void store_y(void* y, int64_t o, float v, int out_bf16, int64_t n, int32_t* status)
 {
+    if (!q4_in_bounds(o, n, status)) return;
     if (out_bf16) reinterpret_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
     else reinterpret_cast<float*>(y)[o] = v;
 }

@@ -452,7 +452,7 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
         if ((rc = q4_act_quant_rows(reinterpret_cast<const uint16_t*>(ws.h), true, P, I, ws.hq, ws.sh_row, status, s)))
             return rc;
         return q4_moe_down_a8(ws.hq, ws.sh_row, &ex[2], P, H, I, E, ws.offsets, ws.tiles_dn, ws.row_tok, ws.row_w,
-                              y32, status, s);
+                              y32, T, status, s);
     }
     CUtensorMap mh, md;
     if (!make_act_map(&mh, ws.h, 2 * (uint64_t)I, P, 2, 4) || !make_packed_map(&md, ex[2].packed, I, (uint64_t)E * H, BM))
@@ -471,6 +471,7 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     d.row_w = ws.row_w;
     d.E = E;
     d.topk = topk;
+    d.T = T;
     return launch<false, G, SYM, Mode::Down>(mh, md, md, d, sms, s);
 }
 

@@ -36,7 +36,7 @@ int gateup(const int8_t* xq, const float* sa, const q4_weight* gate, const q4_we
 
 template <int G, bool SYM>
 int down(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E, const int32_t* offsets,
-         const int32_t* tiles, const int32_t* row_tok, const float* row_w, float* y32, int32_t* status,
+         const int32_t* tiles, const int32_t* row_tok, const float* row_w, float* y32, int T, int32_t* status,
          cudaStream_t s)
 {
     using namespace tcg;
@@ -57,6 +57,7 @@ int down(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, i
     d.row_tok = row_tok;
     d.row_w = row_w;
     d.E = E;
+    d.T = T;
     return launch<true, G, SYM, Mode::Down>(mh, md, md, d, q4_num_sms(), s);
 }
 
@@ -75,11 +76,11 @@ int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, c
 
 int q4_moe_down_a8(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E,
                    const int32_t* offsets, const int32_t* tiles, const int32_t* row_tok, const float* row_w,
-                   float* y32, int32_t* status, cudaStream_t s)
+                   float* y32, int T, int32_t* status, cudaStream_t s)
 {
     if (dn->group == 128)
-        return dn->symmetric ? down<128, true>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, status, s)
-                             : down<128, false>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, status, s);
-    return dn->symmetric ? down<64, true>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, status, s)
-                         : down<64, false>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, status, s);
+        return dn->symmetric ? down<128, true>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, T, status, s)
+                             : down<128, false>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, T, status, s);
+    return dn->symmetric ? down<64, true>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, T, status, s)
+                         : down<64, false>(hq, sh, dn, P, H, I, E, offsets, tiles, row_tok, row_w, y32, T, status, s);
 }

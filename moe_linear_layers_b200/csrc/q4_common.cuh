@@ -18,6 +18,23 @@ __device__ __forceinline__ void q4_set_status(int32_t* status, int32_t code)
     if (status) atomicCAS(status, 0, code);
 }
 
+// Debug build (Q4_DEBUG): a global-memory index a kernel computes is checked against its buffer's extent
+// before the access; a failed check records Q4_ERR_BOUNDS and the access is skipped.  In the release build
+// the check is the constant true and costs nothing.
+__device__ __forceinline__ bool q4_in_bounds(int64_t i, int64_t n, int32_t* status)
+{
+#ifdef Q4_DEBUG
+    if (i >= 0 && i < n) return true;
+    q4_set_status(status, Q4_ERR_BOUNDS);
+    return false;
+#else
+    (void)i;
+    (void)n;
+    (void)status;
+    return true;
+#endif
+}
+
 // (a & b) ^ c in one LOP3.
 __device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c)
 {
@@ -76,7 +93,7 @@ int q4_moe_gateup_a8(const int8_t* xq, const float* sa, const q4_weight* gate, c
                      int32_t* status, cudaStream_t s);
 int q4_moe_down_a8(const int8_t* hq, const float* sh, const q4_weight* dn, int P, int H, int I, int E,
                    const int32_t* offsets, const int32_t* tiles, const int32_t* row_tok, const float* row_w,
-                   float* y32, int32_t* status, cudaStream_t s);
+                   float* y32, int T, int32_t* status, cudaStream_t s);
 
 // Number of SMs of the current device (cached per device).
 static inline int q4_num_sms()

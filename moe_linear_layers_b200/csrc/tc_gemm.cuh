@@ -33,10 +33,10 @@
 //           codes of h and per-row scales s_a); epilogue y[token][n] += w[token][slot] * (s_a) * out
 //           (fp32 reduction into the output).
 //
-// Warp roles (768 threads = 6 warpgroups, launched at 80 registers and re-partitioned with setmaxnreg):
+// Warp roles (640 threads = 5 warpgroups, launched at 96 registers and re-partitioned with setmaxnreg):
 //   warps 0-3    MMA issuers, one thread each, stage it issued by warp it % 4 (warp 1 also owns TMEM);
-//   warps 4-7    converters of the even stages, warps 20-23 converters of the odd stages (TMEM lanes
-//                32*(warp%4) ...): a converter warp's loop is latency-bound, so two sets alternate;
+//   warps 4-7    converters (TMEM lanes 32*(warp%4) ...); a build with Q4_CONV_SETS=2 adds warps 20-23 for
+//                the odd stages (measured slower on B200: 683 against 880 TFLOP/s, so one set is the default);
 //   warps 8-9    TMA producers (alternate stages); warp 10 parameter loader; warp 11 idle;
 //   warps 12-19  epilogue (two warps per TMEM lane quarter, each draining 64 of the 128 columns).
 // Measured on B200: one thread issues an M128 N128 K16 MMA only every ~120 cycles, half the tensor
@@ -65,7 +65,7 @@ constexpr int NA = 4;                    // TMEM stages of widened weights
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
 #ifndef Q4_CONV_SETS
-#define Q4_CONV_SETS 2
+#define Q4_CONV_SETS 1
 #endif
 constexpr int kConvSets = Q4_CONV_SETS;  // converter warpgroups, alternate stages
 constexpr int kThreads = 640 + 128 * (kConvSets - 1);   // 20 or 24 warps
@@ -132,6 +132,7 @@ struct Args {
     __nv_bfloat16* h;              // GateUp output [P][N/64][hi 64 | lo 64], or fp16 [P][N] when h_f16
     int h_f16;                     // GateUp: h for an INT8 down projection, stored as the fp16 activation
     int E, topk;
+    int T;                         // Down: rows of the output y (tokens)
 };
 
 struct Tile {
@@ -694,8 +695,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
-                                if (m < T.m_end)
-                                    p.acc_dbg[((int64_t)m * p.N + T.n0 + r) * ngroups + gl] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
+                                const int64_t o = ((int64_t)m * p.N + T.n0 + r) * ngroups + gl;
+                                if (m < T.m_end && q4_in_bounds(o, (int64_t)p.M * p.N * ngroups, p.status))
+                                    p.acc_dbg[o] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
                             }
                         }
                         const uint64_t nb2 = tc::f2_pack(__float_as_uint(-kAccBiasF), __float_as_uint(-kAccBiasF));
@@ -735,7 +737,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             for (int j = 0; j < 64; j++) {
                                 float v = accv(j);
                                 if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
-                                yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
+                                if (q4_in_bounds(base + (int64_t)j * p.N, (int64_t)p.M * p.N, p.status))
+                                    yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
                             }
                         } else {
 #pragma unroll
@@ -743,7 +746,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                 if (j < rows) {
                                     float v = accv(j);
                                     if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
-                                    yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
+                                    if (q4_in_bounds(base + (int64_t)j * p.N, (int64_t)p.M * p.N, p.status))
+                                        yb[(int64_t)j * p.N] = __float2bfloat16_rn(v);
                                 }
                         }
                     } else {
@@ -753,7 +757,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             for (int j = 0; j < 64; j++) {
                                 float v = accv(j);
                                 if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
-                                yf[(int64_t)j * p.N] = v;
+                                if (q4_in_bounds(base + (int64_t)j * p.N, (int64_t)p.M * p.N, p.status))
+                                    yf[(int64_t)j * p.N] = v;
                             }
                         } else {
 #pragma unroll
@@ -761,7 +766,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                 if (j < rows) {
                                     float v = accv(j);
                                     if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
-                                    yf[(int64_t)j * p.N] = v;
+                                    if (q4_in_bounds(base + (int64_t)j * p.N, (int64_t)p.M * p.N, p.status))
+                                        yf[(int64_t)j * p.N] = v;
                                 }
                         }
                     }
@@ -793,6 +799,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             uv *= sa;
                         }
                         const float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
+                        const int64_t o = (hb - p.h) + (int64_t)j * hstride + (f16 ? 0 : 64);
+                        if (!q4_in_bounds(o, (int64_t)p.M * hstride, p.status)) return;
                         if (f16) {
                             reinterpret_cast<__half*>(hb)[(int64_t)j * hstride] = __float2half_rn(hv);
                         } else {
@@ -820,11 +828,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 if (rows == 64) {
 #pragma unroll
                     for (int j = 0; j < 64; j++)
-                        atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
+                        if (q4_in_bounds((int64_t)comb_tok[ew * 64 + j] * p.N + n, (int64_t)p.T * p.N, p.status))
+                            atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
                 } else {
 #pragma unroll
                     for (int j = 0; j < 64; j++)
-                        if (j < rows) atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
+                        if (j < rows &&
+                            q4_in_bounds((int64_t)comb_tok[ew * 64 + j] * p.N + n, (int64_t)p.T * p.N, p.status))
+                            atomicAdd(yv + (int64_t)comb_tok[ew * 64 + j] * p.N, comb_w[ew * 64 + j] * accv(j));
                 }
                 __syncwarp();
             }

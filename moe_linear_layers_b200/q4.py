@@ -12,7 +12,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libq4.so")
+# Q4_DEBUG_LIBRARY=1 loads the debug build (bounds-checked kernels, Q4_ERR_BOUNDS) instead of the release one
+LIB_PATH = os.path.join(_HERE, "libq4_debug.so" if os.environ.get("Q4_DEBUG_LIBRARY") == "1" else "libq4.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_linear_layers_b200.build_lib`")
@@ -28,10 +29,11 @@ Q4_ERR_WORKSPACE = -5
 Q4_ERR_CUDA = -6
 Q4_ERR_NONFINITE = -7
 Q4_ERR_TIMEOUT = -8
+Q4_ERR_BOUNDS = -9
 Q4_OUT_F32 = 0
 Q4_OUT_BF16 = 1
 
-EXPORTED = ("q4_status_string", "q4_version", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
+EXPORTED = ("q4_status_string", "q4_version", "q4_build_flags", "q4_last_cuda_error_string", "q4_quantize_pack", "q4_linear_w4a16", "q4_linear_w4a16_max_gemv_m",
             "q4_linear_w4a16_grouped", "q4_linear_w4a16_swiglu",
             "act_quant_per_token", "q4_linear_w4a8", "moe_q4_workspace_size", "moe_q4_forward",
             "moe_q4_forward_noalloc", "moe_q4_workspace_size_ex", "moe_q4_forward_ex", "q4_selftest_bounded_wait",
@@ -52,6 +54,7 @@ _i32, _p, _sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
 _lib.q4_status_string.restype = ctypes.c_char_p
 _lib.q4_status_string.argtypes = [ctypes.c_int]
 _lib.q4_version.restype = ctypes.c_int
+_lib.q4_build_flags.restype = ctypes.c_int
 _lib.q4_last_cuda_error_string.restype = ctypes.c_char_p
 _lib.q4_linear_w4a16_max_gemv_m.restype = ctypes.c_int
 _lib.q4_quantize_pack.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p]
