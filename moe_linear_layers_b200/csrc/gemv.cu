@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
     constexpr bool PAIR = MT <= 2;                  // two rows per warp iteration
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + kStages;
+    uint32_t* consumed = reinterpret_cast<uint32_t*>(full + kStages);   // [kComputeWarps] stages finished per warp
     uint4* xs = reinterpret_cast<uint4*>(smem + p.xs_off);      // [MT][k/8] int16 x pairs, swizzled
     float* xinv = reinterpret_cast<float*>(smem + p.ips_off);   // [MT][k/64] 2^-e of each block
     float* red = reinterpret_cast<float*>(smem + p.red_off);    // [rows_per_cta][KSPLIT][MT]
@@ -155,7 +155,8 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
     const int sbytes = rps * ng * 2;                            // scale part of a stage
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kComputeWarps); }
+        for (int i = 0; i < kStages; i++) tc::mbar_init(&full[i], 1);
+        for (int i = 0; i < kComputeWarps; i++) consumed[i] = 0;
         tc::fence_mbar_init();
     }
     __syncthreads();
@@ -197,8 +198,11 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
                     if constexpr (!SYM) prefetch_l2_range(P.zeros + (int64_t)rl * ng, P.zeros + (int64_t)r1 * ng);
                 }
             }
+            // beyond the first fill the producer polls the compute warps' counters with plain loads: an
+            // mbarrier wait would also wait for this thread's own bulk copies in flight
             for (int st = kStages; st < nstages; st++) {
-                if (!tc::mbar_wait(&empty[st % kStages], ((st / kStages) & 1) ^ 1, p.status, nullptr)) break;
+                if (!tc::poll_counters<kComputeWarps>(consumed, st - kStages + 1, p.status, nullptr)) break;
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 issue(st);
             }
         }
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, MT == 1 ? Q4_GEMV_MIN_BLOCKS : 2) w4
             }
         }
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&empty[s]);
+        if (lane == 0) tc::sts_publish(&consumed[warp], st + 1);   // this warp is done with the stage
     }
 
     if constexpr (KSPLIT > 1) {

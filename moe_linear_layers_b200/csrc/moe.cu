@@ -42,7 +42,7 @@ constexpr int kMaxTopk = 16;
 // reproduces bit for bit.  A producer warp streams 64-column tiles of Wr (fp32) and x (bf16) through a
 // 4-stage TMA ring.
 constexpr int kRouteStages = 4;
-constexpr int kRouteThreads = (kRouteWarps + 1) * 32;
+constexpr int kRouteThreads = (kRouteWarps + 2) * 32;   // + producer warp + ring-slot watcher warp
 constexpr int kRouteWTile = 64 * kRouteKC * 4;       // 64 experts x 64 columns, fp32
 constexpr int kRouteXTile = kRouteTok * kRouteKC * 2;  // 16 tokens x 64 columns, bf16
 
@@ -68,6 +68,7 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     __shared__ float logits[kRouteTok][tcg::kMaxExperts];
     __shared__ int hcount[tcg::kMaxExperts];
     __shared__ uint64_t full[kRouteStages], empty[kRouteStages];
+    __shared__ uint32_t slot_free;   // ring stages released so far (published by the watcher)
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kRouteTok;
     const int nk = H / kRouteKC;
@@ -76,17 +77,30 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRouteStages; i++) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], kRouteWarps); }
+        slot_free = 0;
         tc::fence_mbar_init();
     }
     for (int e = threadIdx.x; e < E; e += blockDim.x) hcount[e] = 0;
     __syncthreads();
 
-    if (warp == kRouteWarps) {
+    if (warp == kRouteWarps + 1) {
+        // ------------------------------------------------------------------ ring-slot watcher: waits for each
+        // stage's slot to be released and publishes the count (the producer, which issues the copies, must
+        // not wait on an mbarrier: such a wait also waits for the thread's own bulk copies in flight)
+        if (lane == 0)
+            for (int st = 0; st < nsteps; st++) {
+                if (!tc::mbar_wait(&empty[st % kRouteStages], (st / kRouteStages) & 1, status, nullptr)) break;
+                tc::sts_publish(&slot_free, st + 1);
+            }
+    } else if (warp == kRouteWarps) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             for (int st = 0; st < nsteps; st++) {
                 const int s = st % kRouteStages;
-                if (!tc::mbar_wait(&empty[s], ((st / kRouteStages) & 1) ^ 1, status, nullptr)) break;
+                if (st >= kRouteStages) {
+                    if (!tc::poll_counters<1>(&slot_free, st - kRouteStages + 1, status, nullptr)) break;
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
                 const int eb = st / nk, kc = st % nk;
                 tc::mbar_arrive_expect_tx(&full[s], kRouteWTile + kRouteXTile);
                 tc::tma_load_2d(wst + s * (kRouteWTile / 4), &tm_w, &full[s], kc * kRouteKC, eb * 64);
@@ -161,8 +175,8 @@ moe_route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
     __syncthreads();
 
-    // top-k per token (warp w handles tokens w, w + 9 of the chunk)
-    for (int tt = warp; tt < kRouteTok; tt += kRouteWarps + 1) {
+    // top-k per token (warp w handles tokens w, w + 10 of the chunk)
+    for (int tt = warp; tt < kRouteTok; tt += kRouteWarps + 2) {
         const int t = t0 + tt;
         if (t >= T) break;
         constexpr int PER = tcg::kMaxExperts / 32;

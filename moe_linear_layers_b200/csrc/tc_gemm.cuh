@@ -37,14 +37,15 @@
 //   warps 0-3    MMA issuers, one thread each, stage it issued by warp it % 4 (warp 1 also owns TMEM);
 //   warps 4-7    converters (TMEM lanes 32*(warp%4) ...); a build with Q4_CONV_SETS=2 adds warps 20-23 for
 //                the odd stages (measured slower on B200: 683 against 880 TFLOP/s, so one set is the default);
-//   warps 8-9    TMA producers (alternate stages); warp 10 parameter loader; warp 11 idle;
+//   warp 8       TMA producer (issues every copy, never waits on an mbarrier); warp 9 ring-slot watcher;
+//                warp 10 parameter loader; warp 11 idle;
 //   warps 12-19  epilogue (two warps per TMEM lane quarter, each draining 64 of the 128 columns).
 // Measured on B200: one thread issues an M128 N128 K16 MMA only every ~120 cycles, half the tensor
 // pipe's rate, and any strong memory operation in that thread (an mbarrier wait included) stalls it
 // until its MMAs have retired; four issuer threads in different warps that only poll progress counters
 // with weak loads keep the pipe at one MMA per 64 cycles, commits included.  A thread that waits on an
-// mbarrier also stalls until its own bulk copies have landed, so the TMA stream is split over two
-// producer threads too.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their
+// mbarrier also stalls until its own bulk copies have landed, so the thread that issues the TMA copies
+// polls a counter that another thread publishes after the mbarrier wait.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their
 // phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
 //
 // Epilogue arithmetic runs on packed fp32 pairs (FFMA2).  For W4A8 every int32 accumulator is preloaded
@@ -216,6 +217,7 @@ struct Shared {
     // progress counters read by the MMA issuer (weak loads): stages converted (and activations landed)
     // per converter warp of each set, groups drained per epilogue warp, W4A8 accumulator preload done
     uint32_t conv_done[4 * kConvSets], epi_done[8], epi_init[8];
+    uint32_t slot_free;             // ring stages released so far (published by the slot watcher)
     uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
     uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
@@ -367,6 +369,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = 0; i < C::ND; i++) tc::mbar_init(&sh->d_full[i], 1);
         for (int i = 0; i < NA; i++) tc::mbar_init(&sh->tmem_free[i], 1);
         for (int i = 0; i < 4 * kConvSets; i++) sh->conv_done[i] = 0;
+        sh->slot_free = 0;
         for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
         tc::mbar_init(&sh->done, kIssuers);
         // consumers: the converters, and the epilogue unless it is W4A8's
@@ -400,20 +403,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const int wg = warp / 4;
     if (wg == 2) {
         tc::setmaxnreg_dec<kRegsProd>();
-        // ------------------------------------------------------------------ TMA producers (warps 8, 9)
-        // Two producer threads in different warps take alternate stages: a thread that waits on an
-        // mbarrier stalls until its own outstanding bulk copies have landed, so one thread alone would
-        // issue only one stage per L2 round trip.
-        if (lane == 0 && warp < 10) {
-            const uint32_t parity = warp - 8;
+        // ------------------------------------------------------------------ TMA producer (warp 8) and
+        // ring-slot watcher (warp 9).  A thread that waits on an mbarrier also waits for its own bulk copies
+        // in flight, so the thread that issues the copies never waits on one: the watcher (which issues no
+        // copies) waits for each stage's slot to be released (MMA commit + converters) and publishes the
+        // count in shared memory, and the producer polls that count with plain loads.
+        if (lane == 0 && warp == 9) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x)
+                for (int kb = 0; kb < kblocks; kb++, it++) {
+                    if (!tc::mbar_wait(&sh->xw_empty[it % NS], (it / NS) & 1, p.status, abort_flag)) goto watch_done;
+                    tc::sts_publish(&sh->slot_free, it + 1);
+                }
+        watch_done:;
+        } else if (lane == 0 && warp == 8) {
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
                 for (int kb = 0; kb < kblocks; kb++, it++) {
-                    if ((it & 1u) != parity) continue;
                     const int s = it % NS;
-                    if (!(ok = tc::mbar_wait(&sh->xw_empty[s], ((it / NS) & 1) ^ 1, p.status, abort_flag))) break;
+                    if (it >= (uint32_t)NS) {
+                        // stage it - NS, the slot's previous one, has been released
+                        if (!(ok = tc::poll_counters<1>(&sh->slot_free, it - NS + 1, p.status, abort_flag))) break;
+                        // its readers' accesses (generic and tensor) before this copy's writes (async proxy)
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    }
                     // weights first (small; the converters start on them while the activations land)
                     tc::mbar_arrive_expect_tx(&sh->w_full[s], WSTAGE);
                     uint8_t* wdst = wsm + s * WSTAGE;
@@ -430,11 +445,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
             }
             if (!ok || *abort_flag) {  // let every copy this thread issued land before the CTA can exit
-                for (uint32_t j = it > (uint32_t)NS ? it - NS : 0; j < it; j++)
-                    if ((j & 1u) == parity) {
-                        tc::mbar_wait(&sh->w_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
-                        tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
-                    }
+                for (uint32_t j = it > (uint32_t)NS ? it - NS : 0; j < it; j++) {
+                    tc::mbar_wait(&sh->w_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
+                    tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
+                }
             }
         } else if (PRING && warp == 10) {
             // -------------------------------------------------------------- parameter loader (warp 10)
