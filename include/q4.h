@@ -68,7 +68,7 @@ enum { Q4_OUT_F32 = 0, Q4_OUT_BF16 = 1 };
 /* Descriptor of one INT4 weight matrix (all pointers device pointers, 16-byte aligned). */
 typedef struct q4_weight {
     int32_t n, k;        /* rows (output features) and columns (input features) */
-    int32_t group;       /* 64 or 128 (32 for the MoE entry points' 16-bit expert GEMMs); k % group == 0 */
+    int32_t group;       /* 64 or 128 (32 and 256 for the MoE entry points' 16-bit expert GEMMs); k % group == 0 */
     int32_t symmetric;   /* 1: codes -8..7, zeros == NULL; 0: codes 0..15 with zeros */
     const uint8_t* packed;
     const uint16_t* scales;
@@ -102,8 +102,8 @@ int q4_build_flags(void);
  * All divisions are IEEE fp32; rne = round half to even; the STORED fp16 scale codes the group;
  * a group whose scale is 0 codes to its zero point.
  * w [n][k] fp32 (16-byte aligned); packed [n][k/2]; scales [n][k/group]; zeros [n][k/group]
- * (required when symmetric == 0, ignored otherwise).  group in {32, 64, 128}; k % group == 0 (group 32
- * serves the MoE layer's expert matrices; the dense linear entry points take 64 and 128).
+ * (required when symmetric == 0, ignored otherwise).  group in {32, 64, 128, 256}; k % group == 0 (groups
+ * 32 and 256 serve the MoE layer's expert matrices; the dense linear entry points take 64 and 128).
  * dev_status: Q4_ERR_NONFINITE when a group holds a non-finite value or its scale overflows fp16.
  */
 int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t group, int32_t symmetric,
@@ -171,7 +171,8 @@ int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_t m, const 
  *                gate and up may be NULL (no gated problem).  y[i]: [n] in out_dtype.
  *   Every w[i] has the same group and symmetry, k % 64 == 0, k <= 16384, n >= 1.  n_stages <= 128,
  *   count <= 256.
- *   sync: device memory of q4_linear_w4a16_chain_sync_bytes(n_stages) bytes, 4-byte aligned, ZERO before
+ *   sync: device memory of q4_linear_w4a16_chain_sync_bytes(n_stages) bytes (a 128-byte line per stage
+ *   counter, so that the stages' counters do not share cache lines), 4-byte aligned, ZERO before
  *   the first call; the kernel leaves it zero on completion, so calls (and graph replays) on one stream can
  *   reuse it.  Calls sharing a sync buffer must not overlap on the GPU.
  * The launch is cooperative (every CTA resident at once: one per SM); the library's other launches need
@@ -252,7 +253,7 @@ size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t
  *   y[t]         = sum_j w[t][j] * o_(t,j).
  * x [T][H] bf16; router_w [E][H] fp32; router_bias [E] fp32 or NULL.
  * experts[3] = {gate, up, down}: gate and up are [E*I][H] stacked by expert (rows e*I .. e*I+I-1),
- * down is [E*H][I]; all three with the same group (128, 64, or 32) and symmetry.
+ * down is [E*H][I]; all three with the same group (256, 128, 64, or 32) and symmetry.
  * y [T][H] fp32 or bf16.  Optional outputs (nullable): topk_ids [T][topk] int32, topk_w [T][topk]
  * fp32, perm [T*topk] int32 (value t*topk+j), offsets [E+1] int32, expert_counts [E] int32.
  * workspace: device memory of at least moe_q4_workspace_size(T, H, I, E, topk) bytes, 256-byte
@@ -299,7 +300,7 @@ int moe_q4_forward_ex(const uint16_t* x, int32_t T, int32_t H,
  *                hq, sh = act_quant(fp16(h)) per permuted row (I values), and
  *                o_c = sh * sum_g sd[c][g] * sum_{i in g} hq[i] * (code_d[c][i] - zero_d[c][g]);
  *   a clear bit keeps that projection W4A16 as in moe_q4_forward.  a8_mask in 0..3 (0 = moe_q4_forward).
- *   The INT8 projections take groups 64 and 128 (group 32 only with a8_mask 0: Q4_ERR_UNSUPPORTED).
+ *   The INT8 projections take groups 64 and 128 (groups 32 and 256 only with a8_mask 0: Q4_ERR_UNSUPPORTED).
  * Arguments as moe_q4_forward; the workspace must hold moe_q4_workspace_size_a8(T, H, I, E, topk,
  * a8_mask) bytes.  dev_status also receives Q4_ERR_NONFINITE when a quantized row (x or h) holds a
  * non-finite value.
@@ -321,7 +322,7 @@ int moe_q4_forward_a8(const uint16_t* x, int32_t T, int32_t H,
  * Class c holds experts class_begin[c] .. class_begin[c+1]-1 (expert ids as the router numbers them;
  * order the experts so that each class is a contiguous id range); its weights are experts[3c],
  * experts[3c+1], experts[3c+2] = gate [E_c*I][H], up [E_c*I][H], down [E_c*H][I] stacked by the
- * class's experts in id order, with one group (128, 64 or 32) and symmetry shared by the three.
+ * class's experts in id order, with one group (256, 128, 64 or 32) and symmetry shared by the three.
  * class_begin: host array of n_classes + 1 ints, class_begin[0] = 0 < ... < class_begin[n_classes] = E.
  * The layer computes exactly moe_q4_forward's function with each expert's matrices dequantized with
  * its class's parameters.  Every other argument, the workspace size and the limits as moe_q4_forward.
@@ -343,7 +344,7 @@ int moe_q4_forward_classes(const uint16_t* x, int32_t T, int32_t H,
  * Routing and the permutation are the whole layer's (every token is routed over all E experts);
  * experts[3] = {gate [n*I][H], up [n*I][H], down [n*H][I]} stacked over the n = e_end - e_begin experts
  * of the range.  Ranks that own disjoint ranges covering 0 .. E-1 and sum their y (an all-reduce) obtain
- * moe_q4_forward's output.  0 <= e_begin < e_end <= E; group 32, 64 or 128; everything else as
+ * moe_q4_forward's output.  0 <= e_begin < e_end <= E; group 32, 64, 128 or 256; everything else as
  * moe_q4_forward (fp32 output only, the workspace of moe_q4_workspace_size).
  */
 int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H,

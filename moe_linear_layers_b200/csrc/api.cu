@@ -136,7 +136,7 @@ int q4_gemv_w4a16_chain_launch(int n_stages, const int32_t* stage_begin, const u
 
 extern "C" size_t q4_linear_w4a16_chain_sync_bytes(int32_t n_stages)
 {
-    return n_stages < 1 ? 0 : (size_t)(n_stages + 1) * sizeof(uint32_t);
+    return n_stages < 1 ? 0 : (size_t)(n_stages + 1) * 128;   // one 128-byte line per counter
 }
 
 extern "C" int q4_linear_w4a16_chain(int32_t n_stages, const int32_t* stage_begin, const uint16_t* const* x,

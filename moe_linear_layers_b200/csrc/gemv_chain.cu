@@ -11,13 +11,16 @@
 // launch dependency latency (about 2 us on this GPU) 64 times per step, which alone caps a 64-stage step
 // far below HBM bandwidth.  Here the dependency is a counter per stage in global memory:
 //  * one CTA per SM (cooperative launch: every CTA is resident), 16 compute warps and a producer warp;
-//  * each stage's weight rows (the concatenation of its problems' rows) are split evenly over the CTAs;
+//  * each stage's weight rows are split over the CTAs, each problem of the stage getting CTAs in proportion
+//    to its rows, so that a CTA serves one problem (stages one x) per stage;
 //  * the producer streams the CTA's rows of every stage, in stage order, through a shared-memory ring
 //    with cp.async.bulk (evict-first in L2, so that activations and outputs stay cached).  It never waits
 //    for the dependency: weights do not depend on it.  Nor does it wait on an mbarrier for a free slot:
 //    on this GPU a thread's mbarrier wait also waits for that thread's own bulk copies in flight, which
 //    would leave one chunk in flight per HBM round trip; the compute warps publish the chunks they have
 //    finished in per-warp shared-memory counters, which the producer polls with plain loads;
+//  * a prefetch warp pulls the rows of the next ~1.3 layers (and their x) into L2, paced by the same
+//    counters, so that HBM keeps streaming while the compute warps wait at stage boundaries;
 //  * the compute warps of stage s wait until every CTA has finished stage s-1 (one thread polls the
 //    stage's arrival counter with acquire loads, bounded in time), then read x -- which may be an output of
 //    an earlier stage -- and reduce the rows already waiting in the ring; they then publish their own
@@ -35,7 +38,7 @@ using namespace gemv;
 
 constexpr int kCW = 16;                    // compute warps
 constexpr int kCT = kCW * 32;
-constexpr int kThreads = kCT + 32;         // + one producer warp
+constexpr int kThreads = kCT + 64;         // + a producer warp and an L2 prefetch warp
 constexpr int kChunkW = 32768;             // packed weight bytes per ring chunk
 constexpr int kMaxK = 16384;
 constexpr int kMaxProblems = 256;
@@ -43,10 +46,10 @@ constexpr int kMaxStages = 128;
 constexpr int kMaxStageProblems = 8;
 constexpr int kRedFloats = 2048;           // split-k partial sums per CTA and stage
 #ifndef Q4_CHAIN_L2_AHEAD
-#define Q4_CHAIN_L2_AHEAD 0
+#define Q4_CHAIN_L2_AHEAD 12
 #endif
-// chunks prefetched into L2 beyond the ring (by the producer thread: its mbarrier waits then also wait for
-// the prefetches, so the default is none)
+// chunks the prefetch warp keeps in L2 ahead of the compute warps (about 1.3 decode layers of a CTA's rows:
+// some 60 MB of the 126 MB L2 over all SMs)
 constexpr int kL2Ahead = Q4_CHAIN_L2_AHEAD;
 
 struct ChainProblem {
@@ -59,13 +62,13 @@ struct ChainProblem {
     void* y;                 // [n]
     int n;
     int row0;                // first row of the problem in its stage's row concatenation
+    int cta0, ncta, rpc;     // the CTAs that share its rows (a CTA serves one problem per stage), rows each
 };
 
 struct ChainStage {
     int k;                   // reduction length of every problem of the stage
     int p0, np;              // problems p0 .. p0+np-1
     int rows;                // sum of their n
-    int rpc;                 // rows per CTA
     int rps;                 // rows per ring chunk
     int ksplit;              // warps per row (k > 2048 * ksplit never)
     int bulk_scales;         // scales (and zeros) travel in the chunks
@@ -77,7 +80,7 @@ struct ChainParams {
     int nstages, group, out_bf16;
     int slot_bytes, nslots;
     int xs_off, xinv_off, red_off, ring_off, bar_off;
-    uint32_t* sync;          // [0] abort word, [1 + s] arrivals at stage s
+    uint32_t* sync;          // [0] abort word, [32 (1 + s)] arrivals at stage s (a 128-byte line each)
     int32_t* status;
 };
 
@@ -133,10 +136,19 @@ struct Chunk {
     int cr;       // first row relative to the CTA's range (split-k partial sums)
 };
 
-__device__ __forceinline__ void cta_range(const ChainStage& S, int& a, int& b)
+// The CTA's rows [a, b) of stage S (concatenated row numbers): a block of one problem's rows, so that the CTA
+// stages one x per stage; a CTA beyond the stage's CTAs gets none.
+__device__ __forceinline__ void cta_range(const ChainParams& p, const ChainStage& S, int& a, int& b)
 {
-    a = min(S.rows, (int)blockIdx.x * S.rpc);
-    b = min(S.rows, a + S.rpc);
+    a = b = S.rows;
+    for (int pi = S.p0; pi < S.p0 + S.np; pi++) {
+        const ChainProblem& P = p.prob[pi];
+        const int c = (int)blockIdx.x - P.cta0;
+        if (c >= 0 && c < P.ncta) {
+            a = min(P.row0 + P.n, P.row0 + c * P.rpc);
+            b = min(P.row0 + P.n, a + P.rpc);
+        }
+    }
 }
 
 // Chunk starting at concatenated row r (< b) of stage S.
@@ -244,32 +256,54 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
     }
     __syncthreads();
 
+    if (warp == kCW + 1) {
+        // -------------------------------------------------------------- L2 prefetch warp
+        // Walks the same chunks as the producer and pulls each into L2 (weights, scales, zeros, and the
+        // stage's x) once the compute warps are within kL2Ahead chunks of it, so that HBM keeps streaming
+        // while the compute warps wait at a stage boundary and the ring refills from L2.  It issues no
+        // copy into shared memory and waits on no mbarrier.
+        if (lane != 0 || kL2Ahead <= 0) return;
+        uint32_t j = 0;
+        for (int s = 0; s < p.nstages; s++) {
+            const ChainStage& S = p.st[s];
+            int a, b;
+            cta_range(p, S, a, b);
+            const int64_t rowbytes = S.k / 2;
+            const int ng = S.k / ng_of;
+            int cur = -1;
+            for (int r = a; r < b; j++) {
+                const Chunk c = chunk_at(p, S, r, a, b);
+                const ChainProblem& P = p.prob[c.pi];
+                if (j > (uint32_t)kL2Ahead && !poll_consumed(consumed, j - kL2Ahead, p.status, abort_cta)) return;
+                prefetch_l2(P.packed + (int64_t)c.lr * rowbytes, (uint32_t)(c.rows * rowbytes));
+                if (S.bulk_scales) {
+                    prefetch_l2(P.scales + (int64_t)c.lr * ng, (uint32_t)(c.rows * ng * 2));
+                    if constexpr (!SYM) prefetch_l2(P.zeros + (int64_t)c.lr * ng, (uint32_t)(c.rows * ng * 2));
+                }
+                if (c.pi != cur) {   // the problem's input (a hint only: L2 serves the latest writes)
+                    cur = c.pi;
+                    if (P.g) {
+                        prefetch_l2(P.g, (uint32_t)(S.k * 4));
+                        prefetch_l2(P.u, (uint32_t)(S.k * 4));
+                    } else {
+                        prefetch_l2(P.x, (uint32_t)(S.k * 2));
+                    }
+                }
+                r += c.rows;
+            }
+        }
+        return;
+    }
     if (warp == kCW) {
         // -------------------------------------------------------------- producer (weights only)
         if (lane != 0) return;
         const uint64_t pol = evict_first_policy();
         uint32_t it = 0;          // chunks issued
         bool ok = true;
-        // L2 look-ahead cursor: runs kL2Ahead chunks in front of the ring's issue point
-        int ls = 0, lr = -1, la = 0, lb = 0;
-        uint32_t lit = 0;
-        auto l2_advance = [&](uint32_t target) {
-            while (lit < target && ls < p.nstages) {
-                const ChainStage& S = p.st[ls];
-                if (lr < 0) { cta_range(S, la, lb); lr = la; }
-                if (lr >= lb) { ls++; lr = -1; continue; }
-                const Chunk c = chunk_at(p, S, lr, la, lb);
-                const ChainProblem& P = p.prob[c.pi];
-                const int64_t rowbytes = S.k / 2;
-                prefetch_l2(P.packed + (int64_t)c.lr * rowbytes, (uint32_t)(c.rows * rowbytes));
-                lr += c.rows;
-                lit++;
-            }
-        };
         for (int s = 0; s < p.nstages && ok; s++) {
             const ChainStage& S = p.st[s];
             int a, b;
-            cta_range(S, a, b);
+            cta_range(p, S, a, b);
             const int64_t rowbytes = S.k / 2;
             const int ng = S.k / ng_of;
             const int wbytes = S.rps * (int)rowbytes, sbytes = S.rps * ng * 2;
@@ -295,7 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                         bulk_g2s_hint(dst + wbytes + sbytes, P.zeros + (int64_t)c.lr * ng, (uint32_t)(c.rows * ng * 2),
                                       &full[slot], pol);
                 }
-                if constexpr (kL2Ahead > 0) l2_advance(it + 1 + p.nslots + kL2Ahead);
                 r += c.rows;
             }
         }
@@ -320,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
         // wait for every CTA to have finished stage s - 1 (its outputs may be this stage's inputs)
         if (s > 0) {
             if (threadIdx.x == 0) {
-                const uint32_t* cnt = p.sync + s;   // arrivals at stage s - 1
+                const uint32_t* cnt = p.sync + 32 * s;   // arrivals at stage s - 1
                 const uint64_t t0 = tc::globaltimer_ns();
                 for (uint32_t i = 0;; i++) {
                     if (ld_relaxed_gpu(cnt) >= gridDim.x) {
@@ -328,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                         asm volatile("fence.acq_rel.gpu;" ::: "memory");
                         break;
                     }
-                    if ((i & 7u) == 7u && ld_relaxed_gpu(p.sync)) { *abort_cta = 1; break; }
+                    if ((i & 63u) == 63u && ld_relaxed_gpu(p.sync)) { *abort_cta = 1; break; }
                     if ((i & 63u) == 63u) {
                         if (tc::wait_expired(t0, tc::kWaitLimitNs, i >> 6, 64)) {
                             q4_set_status(p.status, Q4_ERR_TIMEOUT);
@@ -346,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
             }
         }
         int a, b;
-        cta_range(S, a, b);
+        cta_range(p, S, a, b);
         const int k = S.k, ks = S.ksplit, teams = kCW / ks;
         const int team = warp / ks, kq = warp % ks;
         const int64_t rowbytes = k / 2;
@@ -436,13 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
         // thread's stores before thread 0's release, which carries them to the other CTAs' acquire)
         if (threadIdx.x == 0) {
             if (s < p.nstages - 1) {
-                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.sync + 1 + s) : "memory");
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.sync + 32 * (1 + s)) : "memory");
             } else {
                 uint32_t old;
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.sync + 1 + s) : "memory");
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.sync + 32 * (1 + s)) : "memory");
                 if (old == gridDim.x - 1) {
                     // the last arrival of the last stage: every CTA is past every wait; leave the counters zero
-                    for (int i = 1; i <= p.nstages; i++) p.sync[i] = 0u;
+                    for (int i = 1; i <= p.nstages; i++) p.sync[32 * i] = 0u;
                 }
             }
         }
@@ -494,18 +527,46 @@ int q4_gemv_w4a16_chain_launch(int n_stages, const int32_t* stage_begin, const u
         }
         if (S.k % 64 || S.k > kMaxK) return Q4_ERR_UNSUPPORTED;
         S.rows = rows;
+        // CTAs per problem in proportion to its rows (at least one each), rows per CTA within the problem
+        {
+            int nc[kMaxStageProblems], tot = 0;
+            for (int i = 0; i < S.np; i++) {
+                nc[i] = std::max(1, (int)((int64_t)w[S.p0 + i].n * grid / rows));
+                tot += nc[i];
+            }
+            while (tot > grid) {   // (only with many tiny problems) take from the problem with the most CTAs
+                int j = 0;
+                for (int i = 1; i < S.np; i++) if (nc[i] > nc[j]) j = i;
+                nc[j]--; tot--;
+            }
+            while (tot < grid) {   // give the rest to the problem with the most rows per CTA
+                int j = 0;
+                for (int i = 1; i < S.np; i++)
+                    if ((int64_t)w[S.p0 + i].n * nc[j] > (int64_t)w[S.p0 + j].n * nc[i]) j = i;
+                nc[j]++; tot++;
+            }
+            int c0 = 0;
+            for (int i = 0; i < S.np; i++) {
+                ChainProblem& Q = P.prob[S.p0 + i];
+                Q.cta0 = c0;
+                Q.ncta = nc[i];
+                Q.rpc = (Q.n + nc[i] - 1) / nc[i];
+                c0 += nc[i];
+            }
+        }
         int ks = 1;
         while (ks * 2048 < S.k) ks *= 2;
         S.ksplit = ks;
         const int rowbytes = S.k / 2, ng = S.k / group;
         S.rps = std::max(1, kChunkW / rowbytes);
-        S.rpc = std::max(1, (rows + grid - 1) / grid);
-        if (ks > 1 && S.rpc * ks > kRedFloats) return Q4_ERR_UNSUPPORTED;
+        int rpc_max = 1;
+        for (int i = S.p0; i < S.p0 + S.np; i++) rpc_max = std::max(rpc_max, P.prob[i].rpc);
+        if (ks > 1 && rpc_max * ks > kRedFloats) return Q4_ERR_UNSUPPORTED;
         S.bulk_scales = (ng * 2) % 16 == 0;
         const int sb = S.rps * rowbytes + (S.bulk_scales ? S.rps * ng * 2 * (sym ? 1 : 2) : 0);
         slot_bytes = std::max(slot_bytes, sb);
         kmax = std::max(kmax, S.k);
-        redmax = std::max(redmax, ks > 1 ? S.rpc * ks : 0);
+        redmax = std::max(redmax, ks > 1 ? rpc_max * ks : 0);
     }
     slot_bytes = (slot_bytes + 127) & ~127;
     // shared memory: x (int16) | per-block inverse scales | split-k partials | barriers | ring

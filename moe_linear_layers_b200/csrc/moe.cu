@@ -489,7 +489,7 @@ int launch_experts(const Workspace& ws, const q4_weight* ex, int T, int H, int I
     return launch<false, G, SYM, Mode::Down>(mh, md, md, d, sms, s);
 }
 
-// group 32 is built for the 16-bit expert GEMMs only (the INT8 paths take 64 and 128)
+// groups 32 and 256 are built for the 16-bit expert GEMMs only (the INT8 paths take 64 and 128)
 int launch_experts_any(const Workspace& ws, const q4_weight* ex, int T, int H, int I, int E, int topk, float* y32,
                        int32_t* status, cudaStream_t s, int a8_mask)
 {
@@ -505,6 +505,10 @@ int launch_experts_any(const Workspace& ws, const q4_weight* ex, int T, int H, i
         if (a8_mask) return Q4_ERR_UNSUPPORTED;
         return sym ? launch_experts<32, true>(ws, ex, T, H, I, E, topk, y32, status, s, 0)
                    : launch_experts<32, false>(ws, ex, T, H, I, E, topk, y32, status, s, 0);
+    case 256:
+        if (a8_mask) return Q4_ERR_UNSUPPORTED;
+        return sym ? launch_experts<256, true>(ws, ex, T, H, I, E, topk, y32, status, s, 0)
+                   : launch_experts<256, false>(ws, ex, T, H, I, E, topk, y32, status, s, 0);
     default:
         return Q4_ERR_UNSUPPORTED;
     }
@@ -625,10 +629,12 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
             const q4_weight& w = cw[i];
             if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
             if (w.group != cw[0].group || w.symmetric != cw[0].symmetric) return Q4_ERR_UNSUPPORTED;
+            if (w.group <= 0 || w.k % w.group) return Q4_ERR_SHAPE;
             if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
                 return Q4_ERR_ALIGN;
         }
-        if (cw[0].group != 64 && cw[0].group != 128 && !(cw[0].group == 32 && a8_mask == 0)) return Q4_ERR_UNSUPPORTED;
+        if (cw[0].group != 64 && cw[0].group != 128 && !((cw[0].group == 32 || cw[0].group == 256) && a8_mask == 0))
+            return Q4_ERR_UNSUPPORTED;
         if (cw[0].n != Ec * I || cw[0].k != H || cw[1].n != Ec * I || cw[1].k != H || cw[2].n != Ec * H || cw[2].k != I)
             return Q4_ERR_SHAPE;
     }
@@ -881,10 +887,12 @@ extern "C" int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H,
         const q4_weight& w = experts[i];
         if (!w.packed || !w.scales || (!w.symmetric && !w.zeros)) return Q4_ERR_NULL;
         if (w.group != experts[0].group || w.symmetric != experts[0].symmetric) return Q4_ERR_UNSUPPORTED;
+        if (w.group <= 0 || w.k % w.group) return Q4_ERR_SHAPE;
         if (!q4_aligned16(w.packed) || !q4_aligned16(w.scales) || (!w.symmetric && !q4_aligned16(w.zeros)))
             return Q4_ERR_ALIGN;
     }
-    if (experts[0].group != 32 && experts[0].group != 64 && experts[0].group != 128) return Q4_ERR_UNSUPPORTED;
+    if (experts[0].group != 32 && experts[0].group != 64 && experts[0].group != 128 && experts[0].group != 256)
+        return Q4_ERR_UNSUPPORTED;
     if (experts[0].n != E * I || experts[0].k != H || experts[1].n != E * I || experts[1].k != H ||
         experts[2].n != E * H || experts[2].k != I)
         return Q4_ERR_SHAPE;

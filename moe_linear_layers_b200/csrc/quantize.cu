@@ -93,7 +93,7 @@ extern "C" int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t gr
                                 void* stream)
 {
     if (!w || !packed || !scales || (!symmetric && !zeros)) return Q4_ERR_NULL;
-    if (n < 0 || k <= 0 || (group != 32 && group != 64 && group != 128) || k % group) return Q4_ERR_SHAPE;
+    if (n < 0 || k <= 0 || (group != 32 && group != 64 && group != 128 && group != 256) || k % group) return Q4_ERR_SHAPE;
     if (!q4_aligned16(w) || !q4_aligned16(packed) || !q4_aligned16(scales) || (!symmetric && !q4_aligned16(zeros)))
         return Q4_ERR_ALIGN;
     if (n == 0) return Q4_OK;
@@ -104,7 +104,10 @@ extern "C" int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t gr
     uint32_t* pk = reinterpret_cast<uint32_t*>(packed);
     __half* sc = reinterpret_cast<__half*>(scales);
     __half* zr = reinterpret_cast<__half*>(zeros);
-    if (group == 128) {
+    if (group == 256) {
+        if (symmetric) quantize_pack_kernel<256, true><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
+        else quantize_pack_kernel<256, false><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
+    } else if (group == 128) {
         if (symmetric) quantize_pack_kernel<128, true><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
         else quantize_pack_kernel<128, false><<<(int)blocks, 256, 0, s>>>(w, total8, pk, sc, zr, dev_status);
     } else if (group == 64) {

@@ -342,7 +342,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 {
     constexpr bool PRING = !INT8 || !SYM;
     using C = Cfg<INT8, MODE, PRING>;
-    constexpr int GPK = KBLK / G;               // groups per K stage
+    // a group narrower than a stage: GPK groups per stage; a wider one (group 256): SPG stages per group
+    constexpr int GPK = G <= KBLK ? KBLK / G : 1;
+    constexpr int SPG = G > KBLK ? G / KBLK : 1;
+    constexpr int GK = G <= KBLK ? G : KBLK;    // K of one group inside one stage
     constexpr int PW = C::PW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -487,24 +490,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             if constexpr (INT8) ok = tc::poll_counters<8>(sh->epi_init, 1, p.status, abort_flag);
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 for (int kb = 0; kb < kblocks && ok; kb++, it++) {
-                    if (it % kIssuers != (uint32_t)warp) {   // another issuer's stage
-                        g += GPK;
+                    // (the SPG stages of one group go to one issuer, whose MMAs into the group's accumulator
+                    // are then ordered)
+                    if ((it / SPG) % kIssuers != (uint32_t)warp) {   // another issuer's stage
+                        if (it % SPG == SPG - 1) g += GPK;
                         continue;
                     }
+                    const bool g_first = it % SPG == 0, g_last = it % SPG == SPG - 1;
                     const int s = it % NS, sa = it % NA;
                     // the stage's weights are widened into TMEM and its activations have landed
                     if (!(ok = tc::poll_counters<4>(sh->conv_done + 4 * (it % kConvSets), it + 1, p.status, abort_flag))) break;
                     tc::fence_after_sync();
                     const uint32_t xaddr = tc::smem_u32(xs + s * C::XSTAGE);
 #pragma unroll
-                    for (int gi = 0; gi < GPK; gi++, g++) {
-                        const uint32_t db = g % C::ND;
-                        // accumulator db is free once group g-ND has been drained
-                        if (!(ok = tc::poll_counters<8>(sh->epi_done, g >= (uint32_t)C::ND ? g - C::ND + 1 : 0, p.status, abort_flag))) break;
-                        tc::fence_after_sync();
+                    for (int gi = 0; gi < GPK; gi++) {
+                        const uint32_t gg = g + gi;
+                        const uint32_t db = gg % C::ND;
+                        // accumulator db is free once group gg-ND has been drained
+                        if (g_first) {
+                            if (!(ok = tc::poll_counters<8>(sh->epi_done, gg >= (uint32_t)C::ND ? gg - C::ND + 1 : 0, p.status,
+                                                            abort_flag)))
+                                break;
+                            tc::fence_after_sync();
+                        }
 #pragma unroll
-                        for (int i = 0; i < G / C::KI; i++) {
-                            const int kk = gi * G + i * C::KI;   // k offset inside the stage
+                        for (int i = 0; i < GK / C::KI; i++) {
+                            const int kk = gi * GK + i * C::KI;   // k offset inside the stage
                             const uint32_t a_tmem = tbase + C::A_COL0 + sa * C::ACOLS + (INT8 ? kk / 4 : kk / 2);
                             uint32_t boff;
                             if constexpr (INT8) boff = kk;                              // one 128-byte row box
@@ -513,13 +524,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             if constexpr (INT8) {
                                 tc::mma_i8_ts(tbase + db * BN, a_tmem, bdesc, idesc, true);
                             } else {
-                                tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0);
+                                tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc, idesc, i > 0 || !g_first);
                                 if constexpr (C::HILO)   // the lo half of h: the next 64-column box
                                     tc::mma_16_ts(tbase + db * BN, a_tmem, bdesc + ((BN * 128) >> 4), idesc, 1);
                             }
                         }
-                        tc::mma_commit(&sh->d_full[db]);
+                        if (g_last) tc::mma_commit(&sh->d_full[db]);
                     }
+                    if (g_last) g += GPK;
                     tc::mma_commit(&sh->xw_empty[s]);
                     tc::mma_commit(&sh->tmem_free[sa]);
                 }
@@ -550,12 +562,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                 for (int gi = 0; gi < GPK; gi++) zcur[gi] = 8.0f;
                 if constexpr (PRING) {
-                    const int g0 = kb * GPK;
-                    if (g0 % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto conv_done;
+                    const int g0 = SPG > 1 ? kb / SPG : kb * GPK;   // the first group of the stage
+                    const bool gf = kb % SPG == 0, gl_ = kb % SPG == SPG - 1;   // first / last stage of its group
+                    if (g0 % PW == 0 && gf && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag))
+                        goto conv_done;
                     const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
-                    if ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups) {   // the window's last stage: release it
+                    if (gl_ && ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups)) {   // the window's last stage: release it
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
                         wi++;

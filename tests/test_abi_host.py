@@ -75,7 +75,9 @@ def test_quantize_validation():
     L = q4._lib
     assert L.q4_quantize_pack(None, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_NULL
     assert L.q4_quantize_pack(FAKE, 4, 128, 48, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
-    assert L.q4_quantize_pack(FAKE, 4, 128, 256, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_quantize_pack(FAKE, 4, 128, 256, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE   # k % 256
+    assert L.q4_quantize_pack(FAKE, 4, 512, 256, 1, FAKE + 8, FAKE, None, None, None) == q4.Q4_ERR_ALIGN  # 256 accepted
+    assert L.q4_quantize_pack(FAKE, 4, 1024, 512, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
     assert L.q4_quantize_pack(FAKE, 4, 96, 32, 1, FAKE + 8, FAKE, None, None, None) == q4.Q4_ERR_ALIGN  # 32 accepted
     assert L.q4_quantize_pack(FAKE, 4, 100, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_SHAPE
     assert L.q4_quantize_pack(FAKE + 8, 4, 128, 64, 1, FAKE, FAKE, None, None, None) == q4.Q4_ERR_ALIGN
@@ -196,7 +198,7 @@ def test_output_checked_before_any_launch(y, err):
 def test_chain_validation():
     L = q4._lib
     P = ctypes.c_void_p
-    assert L.q4_linear_w4a16_chain_sync_bytes(64) == 65 * 4 and L.q4_linear_w4a16_chain_sync_bytes(0) == 0
+    assert L.q4_linear_w4a16_chain_sync_bytes(64) == 65 * 128 and L.q4_linear_w4a16_chain_sync_bytes(0) == 0
 
     def call(begin, ws, xs=None, ys=None, sync=FAKE, gate=None, up=None, out=0):
         n = len(ws)

@@ -33,6 +33,8 @@ def q4():
     (8192, 2048, 128, False),  # a full gate projection
     (300, 1024, 32, False),    # group 32 (the hottest MoE experts' tier), asymmetric
     (64, 2048, 32, True),      # group 32, symmetric
+    (300, 1024, 256, False),   # group 256 (the coldest MoE experts' tier), asymmetric
+    (64, 2048, 256, True),     # group 256, symmetric
 ])
 def test_quantize_bitexact(q4, n, k, group, sym):
     W = synth.weights(("test", "quant", n, k, group, sym), n, k)

@@ -63,6 +63,8 @@ def _run(q4, T, H, I, E, topk, group, sym, tag, skew=1.1, tokens=None, out=torch
     (200, 512, 256, 64, 8, 128, False),   # the workload's expert count / top-8, skewed: some experts empty
     (150, 256, 256, 6, 2, 32, False),     # group 32, asymmetric
     (90, 512, 128, 4, 2, 32, True),       # group 32, symmetric
+    (150, 512, 256, 6, 2, 256, False),    # group 256 (a group spans two 128-K stages), asymmetric
+    (64, 1024, 512, 8, 2, 256, True),     # group 256, symmetric, several groups per row
 ])
 def test_moe_small(q4, T, H, I, E, topk, group, sym):
     yn, ref, counts = _run(q4, T, H, I, E, topk, group, sym, f"s{T}-{E}")
@@ -224,6 +226,7 @@ def _run_classes(q4, T, H, I, E, topk, begin, params, tag, tokens=None):
     (37, 256, 128, 5, 3, [0, 1, 5], [(64, False), (128, True)]),
     (300, 256, 128, 8, 2, [0, 8], [(128, False)]),          # one class = the plain layer
     (256, 512, 256, 16, 4, [0, 1, 6, 16], [(32, False), (64, False), (128, False)]),   # the pages' three tiers
+    (256, 512, 512, 16, 4, [0, 1, 6, 16], [(32, False), (64, False), (256, False)]),   # the coldest tier at 256
 ])
 def test_moe_classes(q4, T, H, I, E, topk, begin, params):
     yn, ref = _run_classes(q4, T, H, I, E, topk, begin, params, f"cls{T}-{E}")

@@ -131,7 +131,7 @@ def _exact_grid(n, k, group, symmetric, seed):
 
 
 @pytest.mark.parametrize("symmetric", [True, False])
-@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("group", [32, 64, 128, 256])
 def test_exact_grid_roundtrip(symmetric, group):
     n, k = 37, 512
     W, q, sbits, z = _exact_grid(n, k, group, symmetric, seed=group + symmetric)
@@ -151,7 +151,7 @@ def test_exact_grid_roundtrip(symmetric, group):
 # ---------------------------------------------------------------------------------------------- #
 
 @pytest.mark.parametrize("symmetric", [True, False])
-@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("group", [32, 64, 128, 256])
 def test_quant_invariants(symmetric, group):
     n, k = 64, 1024
     W = synth.weights(("pins", "inv", group, symmetric), n, k)
