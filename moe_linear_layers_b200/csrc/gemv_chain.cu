@@ -401,9 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_gemv_chain_kernel(const __g
                 stage_x(P, k, xs, xinv, p.status);
                 compute_bar();
                 cur = c.pi;
+                // (a warp with no rows in this stage's range skips its share of x: 4 KB of shared-memory
+                // reads per warp and problem)
+                const bool xwarp = cvalid && team < b - a;
 #pragma unroll
-                for (int i = 0; i < 8; i++) X[0][i] = cvalid ? xs[(L << 3) + (i ^ (L & 7))] : make_uint4(0, 0, 0, 0);
-                inv_xs[0] = cvalid ? xinv[L] : 0.0f;
+                for (int i = 0; i < 8; i++) X[0][i] = xwarp ? xs[(L << 3) + (i ^ (L & 7))] : make_uint4(0, 0, 0, 0);
+                inv_xs[0] = xwarp ? xinv[L] : 0.0f;
                 int s4[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
