@@ -36,7 +36,10 @@ namespace {
 
 using namespace gemv;
 
-constexpr int kCW = 16;                    // compute warps
+#ifndef Q4_CHAIN_WARPS
+#define Q4_CHAIN_WARPS 16
+#endif
+constexpr int kCW = Q4_CHAIN_WARPS;        // compute warps
 constexpr int kCT = kCW * 32;
 constexpr int kThreads = kCT + 64;         // + a producer warp and an L2 prefetch warp
 constexpr int kChunkW = 32768;             // packed weight bytes per ring chunk
