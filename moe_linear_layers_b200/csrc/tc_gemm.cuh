@@ -62,7 +62,14 @@ enum class Mode { Dense, GateUp, Down };
 constexpr int BM = 128;                  // weight rows per tile
 constexpr int BN = 128;                  // activation rows per tile
 constexpr int KBLK = 128;                // K per stage
-constexpr int NA = 4;                    // TMEM stages of widened weights
+constexpr int kMaxNA = 4;                // TMEM stages of widened weights (at most)
+// 16-bit modes: group accumulators and TMEM stages of widened weights (ND16 * 128 + NA16 * 64 <= 512)
+#ifndef Q4_ND16
+#define Q4_ND16 2
+#endif
+#ifndef Q4_NA16
+#define Q4_NA16 4
+#endif
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
 #ifndef Q4_CONV_SETS
@@ -95,7 +102,9 @@ template <bool INT8, Mode MODE, bool PRING> struct Cfg {
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     // group accumulators in TMEM: three for W4A8 (its MMAs are twice as fast, so the epilogue needs more
     // slack), two otherwise; the widened weights follow them (NA * ACOLS columns)
-    static constexpr int ND = INT8 ? 3 : 2;
+    static constexpr int ND = INT8 ? 3 : Q4_ND16;
+    static constexpr int NA = INT8 ? 4 : Q4_NA16;
+    static_assert(ND >= 2 && ND <= 3 && NA >= 2 && NA <= kMaxNA, "accumulator / TMEM stage counts");
     static constexpr uint32_t A_COL0 = ND * BN;
     static_assert(ND * BN + NA * ACOLS <= (int)kTmemCols, "TMEM columns");
     static constexpr int XCHG = MODE == Mode::GateUp ? 2 * 64 * 64 * 4 : 0;  // up -> gate exchange
@@ -212,7 +221,7 @@ struct Shared {
     // per TMEM slot of widened weights: the MMAs of the slot's last stage have completed.  (The ring's
     // xw_empty cannot stand in for it: with fewer ring stages than TMEM slots, or two converter sets, the
     // ring barrier of stage it - NA can complete a second phase before the converter of stage it looks.)
-    uint64_t tmem_free[NA];
+    uint64_t tmem_free[kMaxNA];
     uint64_t d_full[3], done;
     // progress counters read by the MMA issuer (weak loads): stages converted (and activations landed)
     // per converter warp of each set, groups drained per epilogue warp, W4A8 accumulator preload done
@@ -370,7 +379,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->xw_empty[i], 1 + 4);
         }
         for (int i = 0; i < C::ND; i++) tc::mbar_init(&sh->d_full[i], 1);
-        for (int i = 0; i < NA; i++) tc::mbar_init(&sh->tmem_free[i], 1);
+        for (int i = 0; i < C::NA; i++) tc::mbar_init(&sh->tmem_free[i], 1);
         for (int i = 0; i < 4 * kConvSets; i++) sh->conv_done[i] = 0;
         sh->slot_free = 0;
         for (int i = 0; i < 8; i++) sh->epi_done[i] = sh->epi_init[i] = 0;
@@ -497,7 +506,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         continue;
                     }
                     const bool g_first = it % SPG == 0, g_last = it % SPG == SPG - 1;
-                    const int s = it % NS, sa = it % NA;
+                    const int s = it % NS, sa = it % C::NA;
                     // the stage's weights are widened into TMEM and its activations have landed
                     if (!(ok = tc::poll_counters<4>(sh->conv_done + 4 * (it % kConvSets), it + 1, p.status, abort_flag))) break;
                     tc::fence_after_sync();
@@ -556,7 +565,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         uint32_t it = 0, wi = 0;   // stage and parameter-window counters (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             for (int kb = 0; kb < kblocks; kb++) {
-                const int s = it % NS, sa = it % NA;
+                const int s = it % NS, sa = it % C::NA;
                 // zero points of the stage's groups from the parameter ring
                 float zcur[GPK];
 #pragma unroll
@@ -584,8 +593,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 // phase cannot be older: this set converted stage it - NA; nor can a newer one have completed:
                 // the slot's next stage is this one)
                 {
-                    uint64_t* slot_bar = it >= (uint32_t)NA ? &sh->tmem_free[sa] : &sh->w_full[s];
-                    const uint32_t slot_par = it >= (uint32_t)NA ? ((it / NA) - 1) & 1 : (it / NS) & 1;
+                    uint64_t* slot_bar = it >= (uint32_t)C::NA ? &sh->tmem_free[sa] : &sh->w_full[s];
+                    const uint32_t slot_par = it >= (uint32_t)C::NA ? ((it / C::NA) - 1) & 1 : (it / NS) & 1;
                     if (!tc::mbar_wait3(&sh->w_full[s], (it / NS) & 1, &sh->x_full[s], (it / NS) & 1, slot_bar, slot_par,
                                         p.status, abort_flag))
                         goto conv_done;
