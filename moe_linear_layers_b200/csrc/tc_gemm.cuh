@@ -24,7 +24,8 @@
 //           (W4A8, int8 MMA on 16*code).
 //   GateUp  A rows 0-63 = gate rows i0..i0+63 of expert e, rows 64-127 = the same rows of up; B = the
 //           expert's rows of the permuted activations (bf16, or int8 codes with per-row scales s_a);
-//           epilogue h = SiLU(gate) * up in fp32, stored as a pair of bf16 values hi = bf16(h) and
+//           epilogue h = SiLU(gate) * up in fp32 (gate and up rows each evaluate it for half of the
+//           tokens, after exchanging the other half through shared memory), stored as bf16 hi = bf16(h) and
 //           lo = bf16(h - hi), which together hold h to about 2^-17 of its magnitude (gate and up each
 //           times s_a first with int8 codes).  Row layout of h: [I/64][hi 64 | lo 64].  For a down
 //           projection on INT8 activations, h is stored instead as the fp16 activation it quantizes.
@@ -227,7 +228,7 @@ struct Shared {
     // per converter warp of each set, groups drained per epilogue warp, W4A8 accumulator preload done
     uint32_t conv_done[4 * kConvSets], epi_done[8], epi_init[8];
     uint32_t slot_free;             // ring stages released so far (published by the slot watcher)
-    uint64_t up_ready, gate_done;   // GateUp: hand-over of the up rows to the gate rows
+    uint64_t up_ready, gate_done;   // GateUp: gate/up hand-over written (all 8 epilogue warps), and consumed
     uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
     int abort_flag;
@@ -390,8 +391,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->p_full[i], 32);
             tc::mbar_init(&sh->p_empty[i], 4 * kConvSets + (INT8 ? 0 : 8));
         }
-        tc::mbar_init(&sh->up_ready, 4);
-        tc::mbar_init(&sh->gate_done, 4);
+        // GateUp exchange: every epilogue warp writes its half of the hand-over (up_ready) and consumes
+        // the other side's (gate_done)
+        tc::mbar_init(&sh->up_ready, 8);
+        tc::mbar_init(&sh->gate_done, 8);
         sh->abort_flag = 0;
         if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
         else sh->total_tiles = p.expert_tiles[p.E] - p.expert_tiles[0];
@@ -810,53 +813,72 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                 }
             } else if constexpr (MODE == Mode::GateUp) {
-                // rows 64..127 (up) hand their values to rows 0..63 (gate) of the same intermediate index
+                // Rows 0-63 hold gate, rows 64-127 up, of the same 64 intermediate indices.  Both sides
+                // share the SwiGLU work: the up rows hand u of tokens 0-31 to the gate rows, the gate rows
+                // hand g of tokens 32-63 to the up rows (through shared memory, [token][index]), and each
+                // side then evaluates h for its 32 tokens of this warp's 64.
                 float* xb = xchg + half * 64 * 64;
-                if (r >= 64) {
-                    // the buffer is free once the gate rows consumed the previous tile's values
-                    if (!tc::mbar_wait(&sh->gate_done, (tl & 1) ^ 1, p.status, abort_flag)) goto epi_done;
+                const int ii = r & 63;              // intermediate index within the tile
+                const bool up = r >= 64;
+                // the buffer is free once both sides consumed the previous tile's values
+                if (!tc::mbar_wait(&sh->gate_done, (tl & 1) ^ 1, p.status, abort_flag)) goto epi_done;
+                if (up) {
 #pragma unroll
-                    for (int j = 0; j < 64; j++) xb[j * 64 + (r - 64)] = accv(j);
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&sh->up_ready);
+                    for (int j = 0; j < 32; j++) xb[j * 64 + ii] = accv(j);
                 } else {
-                    if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
-                    const int mb = T.m0 + half * 64;
-                    const int rows = min(64, T.m_end - mb);
-                    // intermediate index i = n0 + r: its hi value in block n0 / 64 of the row, lo 64 later
-                    // (or its fp16 value at column i of an [P][N] row)
-                    const bool f16 = p.h_f16;
-                    const int64_t hstride = f16 ? p.N : 2 * p.N;
-                    __nv_bfloat16* hb = p.h + (int64_t)mb * hstride + (f16 ? T.n0 : 2 * T.n0) + r;
-                    auto swiglu = [&](int j) {
-                        float gv = accv(j), uv = xb[j * 64 + r];
-                        if constexpr (INT8) {   // the row's activation scale
-                            const float sa = __ldg(p.scale_a + mb + j);
-                            gv *= sa;
-                            uv *= sa;
-                        }
-                        const float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
-                        const int64_t o = (hb - p.h) + (int64_t)j * hstride + (f16 ? 0 : 64);
-                        if (!q4_in_bounds(o, (int64_t)p.M * hstride, p.status)) return;
-                        if (f16) {
-                            reinterpret_cast<__half*>(hb)[(int64_t)j * hstride] = __float2half_rn(hv);
-                        } else {
-                            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-                            hb[(int64_t)j * hstride] = hi;
-                            hb[(int64_t)j * hstride + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
-                        }
-                    };
+#pragma unroll
+                    for (int j = 32; j < 64; j++) xb[j * 64 + ii] = accv(j);
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->up_ready);
+                if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
+                const int mb = T.m0 + half * 64;
+                const int rows = min(64, T.m_end - mb);
+                // intermediate index i = n0 + ii: its hi value in block n0 / 64 of the row, lo 64 later
+                // (or its fp16 value at column i of an [P][N] row)
+                const bool f16 = p.h_f16;
+                const int64_t hstride = f16 ? p.N : 2 * p.N;
+                __nv_bfloat16* hb = p.h + (int64_t)mb * hstride + (f16 ? T.n0 : 2 * T.n0) + ii;
+                auto swiglu = [&](int j, float gv, float uv) {
+                    if constexpr (INT8) {   // the row's activation scale
+                        const float sa = __ldg(p.scale_a + mb + j);
+                        gv *= sa;
+                        uv *= sa;
+                    }
+                    // SiLU(g) = g / (1 + e^-g); the fast quotient's error (~1e-7 relative) is far below the
+                    // bf16 hi/lo resolution of h; for g << 0 the divisor is +inf and the quotient -0
+                    const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                    const int64_t o = (hb - p.h) + (int64_t)j * hstride + (f16 ? 0 : 64);
+                    if (!q4_in_bounds(o, (int64_t)p.M * hstride, p.status)) return;
+                    if (f16) {
+                        reinterpret_cast<__half*>(hb)[(int64_t)j * hstride] = __float2half_rn(hv);
+                    } else {
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+                        hb[(int64_t)j * hstride] = hi;
+                        hb[(int64_t)j * hstride + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+                    }
+                };
+                if (up) {
                     if (rows == 64) {
 #pragma unroll
-                        for (int j = 0; j < 64; j++) swiglu(j);
+                        for (int j = 32; j < 64; j++) swiglu(j, xb[j * 64 + ii], accv(j));
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 64; j++)
-                            if (j < rows) swiglu(j);
+                        for (int j = 32; j < 64; j++)
+                            if (j < rows) swiglu(j, xb[j * 64 + ii], accv(j));
                     }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&sh->gate_done);
+                } else {
+                    if (rows >= 32) {
+#pragma unroll
+                        for (int j = 0; j < 32; j++) swiglu(j, accv(j), xb[j * 64 + ii]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (j < rows) swiglu(j, accv(j), xb[j * 64 + ii]);
+                    }
                 }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->gate_done);
             } else {
                 const int n = T.n0 + r;
                 float* yv = reinterpret_cast<float*>(p.y) + n;
