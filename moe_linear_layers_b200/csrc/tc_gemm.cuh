@@ -229,6 +229,7 @@ struct Shared {
     uint32_t conv_done[4 * kConvSets], epi_done[8], epi_init[8];
     uint32_t slot_free;             // ring stages released so far (published by the slot watcher)
     uint64_t up_ready, gate_done;   // GateUp: gate/up hand-over written (all 8 epilogue warps), and consumed
+    uint64_t h_ready[2];            // GateUp: a half's h values are in the exchange buffer (its 4 warps)
     uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
     int abort_flag;
@@ -395,6 +396,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // the other side's (gate_done)
         tc::mbar_init(&sh->up_ready, 8);
         tc::mbar_init(&sh->gate_done, 8);
+        tc::mbar_init(&sh->h_ready[0], 4);
+        tc::mbar_init(&sh->h_ready[1], 4);
         sh->abort_flag = 0;
         if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
         else sh->total_tiles = p.expert_tiles[p.E] - p.expert_tiles[0];
@@ -834,47 +837,54 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 if (!tc::mbar_wait(&sh->up_ready, tl & 1, p.status, abort_flag)) goto epi_done;
                 const int mb = T.m0 + half * 64;
                 const int rows = min(64, T.m_end - mb);
-                // intermediate index i = n0 + ii: its hi value in block n0 / 64 of the row, lo 64 later
-                // (or its fp16 value at column i of an [P][N] row)
-                const bool f16 = p.h_f16;
-                const int64_t hstride = f16 ? p.N : 2 * p.N;
-                __nv_bfloat16* hb = p.h + (int64_t)mb * hstride + (f16 ? T.n0 : 2 * T.n0) + ii;
-                auto swiglu = [&](int j, float gv, float uv) {
-                    if constexpr (INT8) {   // the row's activation scale
-                        const float sa = __ldg(p.scale_a + mb + j);
+                // h of this thread's 32 tokens, written back over the exchanged values it read
+                auto silu_mul = [&](int j, float gv, float uv) {
+                    if constexpr (INT8) {   // the row's activation scale (rows past the expert's end: none)
+                        const float sa = j < rows ? __ldg(p.scale_a + mb + j) : 0.0f;
                         gv *= sa;
                         uv *= sa;
                     }
                     // SiLU(g) = g / (1 + e^-g); the fast quotient's error (~1e-7 relative) is far below the
                     // bf16 hi/lo resolution of h; for g << 0 the divisor is +inf and the quotient -0
-                    const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-                    const int64_t o = (hb - p.h) + (int64_t)j * hstride + (f16 ? 0 : 64);
-                    if (!q4_in_bounds(o, (int64_t)p.M * hstride, p.status)) return;
-                    if (f16) {
-                        reinterpret_cast<__half*>(hb)[(int64_t)j * hstride] = __float2half_rn(hv);
-                    } else {
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-                        hb[(int64_t)j * hstride] = hi;
-                        hb[(int64_t)j * hstride + 64] = __float2bfloat16_rn(hv - __bfloat162float(hi));
-                    }
+                    xb[j * 64 + ii] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
                 };
                 if (up) {
-                    if (rows == 64) {
 #pragma unroll
-                        for (int j = 32; j < 64; j++) swiglu(j, xb[j * 64 + ii], accv(j));
-                    } else {
-#pragma unroll
-                        for (int j = 32; j < 64; j++)
-                            if (j < rows) swiglu(j, xb[j * 64 + ii], accv(j));
-                    }
+                    for (int j = 32; j < 64; j++) silu_mul(j, xb[j * 64 + ii], accv(j));
                 } else {
-                    if (rows >= 32) {
 #pragma unroll
-                        for (int j = 0; j < 32; j++) swiglu(j, accv(j), xb[j * 64 + ii]);
+                    for (int j = 0; j < 32; j++) silu_mul(j, accv(j), xb[j * 64 + ii]);
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->h_ready[half]);
+                if (!tc::mbar_wait(&sh->h_ready[half], tl & 1, p.status, abort_flag)) goto epi_done;
+                // Stores by token row: the 4 warps of this half take token pairs q, q + 4, ...; in a pair, lanes
+                // 0-15 write token j and lanes 16-31 token j + 1, each lane 4 consecutive intermediate indices:
+                // a row's 64 hi values (128 bytes) in one pass and its 64 lo values in a second, or its 64 fp16
+                // values (intermediate index i = n0 + ii: hi in block n0 / 64 of the row, lo 64 later; fp16 at
+                // column i of an [P][N] row)
+                const bool f16 = p.h_f16;
+                const int64_t hstride = f16 ? p.N : 2 * p.N;
+                const int q = ew & 3, c4 = 4 * (lane & 15);
+                for (int pr = q; pr < 32; pr += 4) {
+                    const int j = 2 * pr + (lane >> 4);
+                    if (j >= rows) continue;
+                    const float4 hv = *reinterpret_cast<const float4*>(xb + j * 64 + c4);
+                    const int64_t o = (int64_t)(mb + j) * hstride + (f16 ? T.n0 : 2 * T.n0) + c4;
+                    if (!q4_in_bounds(o + (f16 ? 3 : 67), (int64_t)p.M * hstride, p.status)) continue;
+                    if (f16) {
+                        const __half2 a = __floats2half2_rn(hv.x, hv.y), b = __floats2half2_rn(hv.z, hv.w);
+                        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.h) + o) =
+                            make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
                     } else {
-#pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            if (j < rows) swiglu(j, accv(j), xb[j * 64 + ii]);
+                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(hv.x, hv.y), h1 = __floats2bfloat162_rn(hv.z, hv.w);
+                        const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+                        const __nv_bfloat162 l0 = __floats2bfloat162_rn(hv.x - f0.x, hv.y - f0.y);
+                        const __nv_bfloat162 l1 = __floats2bfloat162_rn(hv.z - f1.x, hv.w - f1.y);
+                        *reinterpret_cast<uint2*>(p.h + o) =
+                            make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+                        *reinterpret_cast<uint2*>(p.h + o + 64) =
+                            make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
                     }
                 }
                 __syncwarp();
