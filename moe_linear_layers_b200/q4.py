@@ -159,6 +159,42 @@ def _out(y, shape, device, name="y"):
     return Q4_OUT_BF16 if y.dtype == torch.bfloat16 else Q4_OUT_F32
 
 
+def _router(router_w, router_bias, H, device):
+    """Check the router of a MoE call: router_w fp32 [E][H] and router_bias (fp32 [E], or None) on the
+    inputs' device.  Returns E."""
+    if router_w.dim() != 2 or router_w.shape[1] != H:
+        raise ValueError(f"router_w must have shape [E][{H}], got {tuple(router_w.shape)}")
+    if router_w.device != device:
+        raise ValueError(f"router_w is on {router_w.device}, the inputs on {device}")
+    E = router_w.shape[0]
+    if router_bias is not None:
+        if not isinstance(router_bias, torch.Tensor) or router_bias.dtype != torch.float32:
+            raise TypeError("router_bias must be a torch.float32 tensor (or None)")
+        if router_bias.numel() != E or not router_bias.is_contiguous():
+            raise ValueError(f"router_bias must be a contiguous tensor of {E} values")
+        if router_bias.device != device:
+            raise ValueError(f"router_bias is on {router_bias.device}, the inputs on {device}")
+    return E
+
+
+def _workspace(ws, device):
+    """Check a caller-supplied workspace: a contiguous uint8 tensor (its numel is its size in bytes) on the
+    inputs' device."""
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8:
+        raise TypeError("workspace must be a torch.uint8 tensor")
+    if not ws.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    if ws.device != device:
+        raise ValueError(f"workspace is on {ws.device}, the inputs on {device}")
+    return ws
+
+
+def _numel(t, n, name):
+    if t.numel() != n:
+        raise ValueError(f"{name} must hold {n} elements, got {t.numel()}")
+    return t
+
+
 def status_string(status: int) -> str:
     return _lib.q4_status_string(status).decode()
 
@@ -228,9 +264,14 @@ class GroupedGemv:
     """Host-side argument arrays for q4_linear_w4a16_grouped, built once and reused (e.g. per layer)."""
 
     def __init__(self, xs, ws, ys):
-        assert len(xs) == len(ws) == len(ys) and 1 <= len(xs) <= 8
+        if not (len(xs) == len(ws) == len(ys) and 1 <= len(xs) <= 8):
+            raise ValueError("a grouped call takes 1 to 8 problems, as many x, w and y")
         self.count = len(xs)
         self.m = xs[0].numel() // ws[0].k
+        for x, w in zip(xs, ws):
+            _numel(x, self.m * w.k, "x")   # every problem has the same m
+            if x.device != xs[0].device:
+                raise ValueError("every x of a grouped call must be on one device")
         self.keep = (xs, ws, ys)
         self.x = (_p * self.count)(*[t.data_ptr() for t in xs])
         self.w = (q4_weight * self.count)(*[w.desc for w in ws])
@@ -266,6 +307,10 @@ class GemvChain:
         xs, gs, us = [], [], []
         for x, w, y in probs:
             ods.add(_out(y.view(-1), (w.n,), dev))
+            for t in (x if isinstance(x, (tuple, list)) else (x,)):
+                _numel(t, w.k, "a chain input")   # m = 1: one row of k values
+                if t.device != dev:
+                    raise ValueError(f"a chain input is on {t.device}, the outputs on {dev}")
             if isinstance(x, (tuple, list)):
                 _dev(x[0], torch.float32, "gate")
                 _dev(x[1], torch.float32, "up")
@@ -367,8 +412,8 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
-    E = router_w.shape[0]
     dev = x.device
+    E = _router(router_w, router_bias, H, dev)
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
     od = _out(y, (T, H), dev)
@@ -376,6 +421,7 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
     ws_bytes = moe_q4_workspace_size(T, H, I, E, topk, I_s, a8_mask)
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _workspace(workspace, dev)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
     sdescs = (q4_weight * 3)(*[e.desc for e in shared]) if shared is not None else None
     ids = wts = perm = offs = cnts = None
@@ -410,8 +456,8 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
-    E = router_w.shape[0]
     dev = x.device
+    E = _router(router_w, router_bias, H, dev)
     n = len(class_experts)
     if len(class_begin) != n + 1:
         raise ValueError("class_begin needs one more entry than there are classes")
@@ -420,6 +466,7 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     od = _out(y, (T, H), dev)
     if workspace is None:
         workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=dev)
+    _workspace(workspace, dev)
     begin = (_i32 * (n + 1))(*[int(v) for v in class_begin])
     descs = (q4_weight * (3 * n))(*[w.desc for trip in class_experts for w in trip])
     ids = wts = perm = offs = cnts = None
@@ -447,13 +494,14 @@ def moe_q4_forward_range(x: torch.Tensor, router_w: torch.Tensor, router_bias: t
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
-    E = router_w.shape[0]
+    E = _router(router_w, router_bias, H, x.device)
     if y is None:
         y = torch.empty((T, H), dtype=torch.float32, device=x.device)
     _dev(y, torch.float32, "y")
     _out(y, (T, H), x.device)
     if workspace is None:
         workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=x.device)
+    _workspace(workspace, x.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
     _check(_lib.moe_q4_forward_range(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, e_begin, e_end, descs,
                                      I, _ptr(y), None, None, None, None, None, _ptr(workspace), workspace.numel(),
@@ -492,7 +540,7 @@ def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
-    E = router_w.shape[0]
+    E = _router(router_w, router_bias, H, x.device)
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=x.device)
     od = _out(y, (T, H), x.device)
@@ -516,8 +564,8 @@ def moe_q4_route(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Ten
     _dev(x, torch.bfloat16, "x")
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
-    E = router_w.shape[0]
     dev = x.device
+    E = _router(router_w, router_bias, H, dev)
     P = T * topk
     out = {"topk_ids": torch.empty((T, topk), dtype=torch.int32, device=dev),
            "topk_w": torch.empty((T, topk), dtype=torch.float32, device=dev),
@@ -544,6 +592,9 @@ def moe_q4_forward_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, e_base: 
     _dev(row_expert, torch.int32, "row_expert")
     R, H = x_rows.shape
     E = experts[0].n // I
+    _numel(row_expert, R, "row_expert")
+    if row_weight is not None:
+        _numel(_dev(row_weight, torch.float32, "row_weight"), R, "row_weight")
     if y is None:
         y = torch.empty((R, H), dtype=torch.float32, device=x_rows.device)
     _dev(y, torch.float32, "y")
@@ -551,6 +602,7 @@ def moe_q4_forward_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, e_base: 
     if workspace is None:
         workspace = torch.empty((max(int(_lib.moe_q4_rows_workspace_size(R, H, I, E)), 1),), dtype=torch.uint8,
                                 device=x_rows.device)
+    _workspace(workspace, x_rows.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
     _check(_lib.moe_q4_forward_rows(_ptr(x_rows), R, H, _ptr(row_expert), int(e_base), _ptr(row_weight), E, descs, I,
                                     _ptr(y), _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
@@ -566,6 +618,7 @@ def moe_q4_combine(o_rows: torch.Tensor, pair_pos: torch.Tensor, topk_w: torch.T
     _dev(topk_w, torch.float32, "topk_w")
     P, H = o_rows.shape
     T, topk = topk_w.shape
+    _numel(pair_pos, T * topk, "pair_pos")
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=o_rows.device)
     od = _out(y, (T, H), o_rows.device)

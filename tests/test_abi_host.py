@@ -254,3 +254,37 @@ def test_moe_steps_validation():
     assert L.moe_q4_combine(FAKE, 10, 6, FAKE, FAKE, 5, 2, FAKE, 0, None, None) == q4.Q4_ERR_SHAPE
     assert L.moe_q4_combine(FAKE, 10, H, FAKE, FAKE, 5, 2, FAKE, 3, None, None) == q4.Q4_ERR_UNSUPPORTED
     assert L.moe_q4_combine(FAKE, 10, H, FAKE, FAKE, 5, 2, FAKE + 8, 0, None, None) == q4.Q4_ERR_ALIGN
+
+
+def test_binding_argument_checks():
+    """The binding's checks of MoE arguments the C ABI cannot see (it takes pointers and sizes): the router's
+    shape, the bias's dtype, length and device, a caller workspace's dtype and device, and input lengths;
+    each raises before any library call."""
+    import torch
+    cpu = torch.device("cpu")
+    w = torch.zeros((8, 256), dtype=torch.float32)
+    assert q4._router(w, None, 256, cpu) == 8
+    assert q4._router(w, torch.zeros(8, dtype=torch.float32), 256, cpu) == 8
+    with pytest.raises(ValueError):
+        q4._router(w, None, 512, cpu)                                    # x is [T][512]
+    with pytest.raises(ValueError):
+        q4._router(torch.zeros(8 * 256, dtype=torch.float32), None, 256, cpu)   # not 2-D
+    with pytest.raises(TypeError):
+        q4._router(w, torch.zeros(8, dtype=torch.float64), 256, cpu)
+    with pytest.raises(ValueError):
+        q4._router(w, torch.zeros(7, dtype=torch.float32), 256, cpu)
+    with pytest.raises(ValueError):
+        q4._router(w, torch.zeros(16, dtype=torch.float32)[::2], 256, cpu)     # not contiguous
+    with pytest.raises(ValueError):
+        q4._router(w, None, 256, torch.device("meta"))                   # on another device than x
+    ws = torch.zeros(64, dtype=torch.uint8)
+    assert q4._workspace(ws, cpu) is ws
+    with pytest.raises(TypeError):
+        q4._workspace(torch.zeros(16, dtype=torch.float32), cpu)        # numel would not be bytes
+    with pytest.raises(ValueError):
+        q4._workspace(ws, torch.device("meta"))
+    with pytest.raises(ValueError):
+        q4._workspace(torch.zeros(128, dtype=torch.uint8)[::2], cpu)
+    assert q4._numel(torch.zeros(6), 6, "t") is not None
+    with pytest.raises(ValueError):
+        q4._numel(torch.zeros(5), 6, "pair_pos")
