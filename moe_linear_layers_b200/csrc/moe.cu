@@ -296,8 +296,10 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restr
                                                           const float* __restrict__ tok_scale,
                                                           float* __restrict__ row_scale,
                                                           int32_t* __restrict__ pair_pos = nullptr,
-                                                          int32_t* __restrict__ row_exp = nullptr)
+                                                          int32_t* __restrict__ row_exp = nullptr,
+                                                          int32_t* status = nullptr)
 {
+    const int64_t P = (int64_t)T * topk;   // permuted rows
     __shared__ int pos[kRouteTok * kMaxTopk];
     __shared__ int cid[kRouteTok * kMaxTopk];   // the chunk's expert ids, token-major
     const int c = blockIdx.x;
@@ -311,7 +313,8 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restr
         int rank = 0;  // earlier tokens of this chunk that chose the same expert (a token picks an expert once)
         for (int u = 0; u < tl * topk; u++) rank += cid[u] == e;
         const int p = chunk_base[(int64_t)c * E + e] + rank;
-        pos[q] = p;
+        pos[q] = q4_in_bounds(p, P, status) ? p : -1;   // (debug build: a position outside the rows is not used)
+        if (pos[q] < 0) continue;
         perm[p] = (t0 + tl) * topk + j;
         row_tok[p] = t0 + tl;
         row_w[p] = wts[(int64_t)(t0 + tl) * topk + j];
@@ -321,21 +324,30 @@ __global__ void __launch_bounds__(256) moe_scatter_kernel(const uint8_t* __restr
     }
     __syncthreads();
     if (!xperm) return;
-    // gather: a warp copies whole rows, eight 16-byte loads in flight per lane before the stores
+    // gather: a warp takes a token, reads its row once (eight 16-byte loads in flight per lane) and writes
+    // it to the permuted rows of all its topk slots
     const int vec = row_bytes / 16;  // 16-byte units per row
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31, nwarps = blockDim.x / 32;
-    for (int q = warp; q < npairs; q += nwarps) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + q / topk) * row_bytes);
-        uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)pos[q] * row_bytes);
+    const int ntok = npairs / topk;
+    for (int tl = warp; tl < ntok; tl += nwarps) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + tl) * row_bytes);
         int u = lane;
         for (; u + 7 * 32 < vec; u += 8 * 32) {
             uint4 r[8];
 #pragma unroll
             for (int j = 0; j < 8; j++) r[j] = __ldg(src + u + 32 * j);
+            for (int k = 0; k < topk; k++) {
+                if (pos[tl * topk + k] < 0) continue;
+                uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)pos[tl * topk + k] * row_bytes);
 #pragma unroll
-            for (int j = 0; j < 8; j++) dst[u + 32 * j] = r[j];
+                for (int j = 0; j < 8; j++) dst[u + 32 * j] = r[j];
+            }
         }
-        for (; u < vec; u += 32) dst[u] = __ldg(src + u);
+        for (; u < vec; u += 32) {
+            const uint4 r = __ldg(src + u);
+            for (int k = 0; k < topk; k++)
+                if (pos[tl * topk + k] >= 0) reinterpret_cast<uint4*>(xperm + (int64_t)pos[tl * topk + k] * row_bytes)[u] = r;
+        }
     }
 }
 
@@ -689,11 +701,13 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         if ((rc = q4_act_quant_rows(x, false, T, H, ws.xq_tok, ws.sa_tok, dev_status, s))) return rc;
         moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(ws.xq_tok), T, H, E, topk, ws.ids,
                                                ws.wts, ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
-                                               reinterpret_cast<uint8_t*>(ws.xperm), ws.sa_tok, ws.sa_row);
+                                               reinterpret_cast<uint8_t*>(ws.xperm), ws.sa_tok, ws.sa_row, nullptr, nullptr,
+                                               dev_status);
     } else {
         moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x), T, 2 * H, E, topk, ws.ids,
                                                ws.wts, ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
-                                               reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr);
+                                               reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr, nullptr, nullptr,
+                                               dev_status);
     }
     if (const cudaError_t e = cudaMemsetAsync(y32, 0, (size_t)T * H * sizeof(float), s)) return q4_cuda_status(e);
     rc = q4_launch_status();
@@ -865,7 +879,8 @@ extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float
                                                    ws.tiles_gu, ws.tiles_dn);
     moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x), T, 2 * H, E, topk, topk_ids, topk_w,
                                            ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
-                                           reinterpret_cast<uint8_t*>(x_perm), nullptr, nullptr, pair_pos, row_expert);
+                                           reinterpret_cast<uint8_t*>(x_perm), nullptr, nullptr, pair_pos, row_expert,
+                                           dev_status);
     return q4_launch_status();
 }
 
@@ -907,7 +922,8 @@ extern "C" int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H,
                                                    ws.tiles_gu, ws.tiles_dn);
     moe_scatter_kernel<<<nch, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(x_rows), R, 2 * H, E, 1, ws.ids, ws.wts,
                                            ws.chunk_base, ws.perm, ws.row_tok, ws.row_w,
-                                           reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr);
+                                           reinterpret_cast<uint8_t*>(ws.xperm), nullptr, nullptr, nullptr, nullptr,
+                                           dev_status);
     if (const cudaError_t e = cudaMemsetAsync(y_rows, 0, (size_t)R * H * sizeof(float), s)) return q4_cuda_status(e);
     int rc = q4_launch_status();
     if (rc) return rc;

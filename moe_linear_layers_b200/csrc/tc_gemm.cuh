@@ -71,12 +71,20 @@ constexpr int kMaxNA = 4;                // TMEM stages of widened weights (at m
 #ifndef Q4_NA16
 #define Q4_NA16 4
 #endif
-// the hi/lo down projection (two MMAs per K step, so fewer widened stages ahead suffice)
+// the hi/lo down projection: two MMAs per K step, so two widened stages ahead suffice and a third
+// accumulator covers its tile output (the atomic combine): 0.6-1 % on the MoE layer
 #ifndef Q4_ND_HILO
-#define Q4_ND_HILO 2
+#define Q4_ND_HILO 3
 #endif
 #ifndef Q4_NA_HILO
-#define Q4_NA_HILO 4
+#define Q4_NA_HILO 2
+#endif
+// the MoE gate/up projection (its tile output, the SwiGLU epilogue, is the longest)
+#ifndef Q4_ND_GU
+#define Q4_ND_GU 2
+#endif
+#ifndef Q4_NA_GU
+#define Q4_NA_GU 4
 #endif
 constexpr int kMaxStages = 8;            // barrier slots of the shared-memory ring
 constexpr int WSTAGE = BM * KBLK / 2;    // packed bytes per stage
@@ -110,8 +118,8 @@ template <bool INT8, Mode MODE, bool PRING> struct Cfg {
     static constexpr int KI = INT8 ? 32 : 16;                   // K per MMA instruction
     // group accumulators in TMEM: three for W4A8 (its MMAs are twice as fast, so the epilogue needs more
     // slack), two otherwise; the widened weights follow them (NA * ACOLS columns)
-    static constexpr int ND = INT8 ? 3 : (HILO ? Q4_ND_HILO : Q4_ND16);
-    static constexpr int NA = INT8 ? 4 : (HILO ? Q4_NA_HILO : Q4_NA16);
+    static constexpr int ND = INT8 ? 3 : (HILO ? Q4_ND_HILO : (MODE == Mode::GateUp ? Q4_ND_GU : Q4_ND16));
+    static constexpr int NA = INT8 ? 4 : (HILO ? Q4_NA_HILO : (MODE == Mode::GateUp ? Q4_NA_GU : Q4_NA16));
     static_assert(ND >= 2 && ND <= 3 && NA >= 2 && NA <= kMaxNA, "accumulator / TMEM stage counts");
     static constexpr uint32_t A_COL0 = ND * BN;
     static_assert(ND * BN + NA * ACOLS <= (int)kTmemCols, "TMEM columns");
