@@ -18,7 +18,7 @@ At one GPU the line also carries "components", the other rows of the hot path on
   moe      the MoE layer: 4096 tokens, hidden 2048, 64 experts of intermediate 1024, top-8 (tokens/s).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
-    python bench.py --ncu-case {decode-chain,decode-layer,gemm,moe,moe-a8,moe-classes}
+    python bench.py --ncu-case {decode-chain,decode-layer,gemm,prefill-m64,moe,moe-a8,moe-classes}
                                                (small launch sequences for ncu captures)
 
 Multi-GPU (torchrun): every rank runs an independent replica of the decode step (the step has no data
@@ -729,6 +729,18 @@ def ncu_case(case):
         for _ in range(2):
             xq, sa = q4.act_quant_per_token(x8)
             q4.q4_linear_w4a8(xq, sa, ws_, y=y8)
+    elif case == "prefill-m64":
+        # one decoder layer's seven W4A16 GEMMs at m = 64 (split along K), twice
+        layers = decode_layers(1)
+        ws = [q4.q4_quantize_pack(torch.from_numpy(synth.weights((0, "llama1b", name), n, k)).to(dev), 128, False)
+              for (name, n, k) in layers]
+        xs = {k: dev_bf16(synth.activations((0, "llama1b-prefill-x", k), 64, k, "outlier_channels"), dev)
+              for (_, _, k) in layers}
+        ys = [torch.empty((64, n), dtype=torch.bfloat16, device=dev) for (_, n, _) in layers]
+        torch.cuda.synchronize()
+        for _ in range(2):
+            for w, (_, n, k), y in zip(ws, layers, ys):
+                q4.q4_linear_w4a16(xs[k], w, y=y)
     elif case == "moe":
         T, H, I, E, topk = (MOE[k] for k in ("T", "H", "I", "E", "topk"))
         x, Wr, bias, ex = build_moe(q4, dev)
@@ -766,7 +778,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode-chain", "decode-layer", "gemm", "moe", "moe-a8", "moe-classes"],
+    ap.add_argument("--ncu-case", choices=["decode-chain", "decode-layer", "gemm", "prefill-m64", "moe", "moe-a8",
+                                           "moe-classes"],
                     help="run a small fixed launch sequence for an ncu capture and exit (no JSON line)")
     args = ap.parse_args()
     if args.ncu_case:

@@ -131,6 +131,26 @@ int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, i
                     int32_t* dev_status, void* stream);
 
 /*
+ * q4_linear_workspace_size -- bytes of device workspace with which q4_linear_w4a16_ws and
+ * q4_linear_w4a8_ws split a tensor-core GEMM of these sizes along K (0: the shape is not split; a
+ * library convenience, not a step of the pages' method).  A problem whose 128 x 128 output tiles fill
+ * fewer than half of the GPU's SMs is cut into K ranges of at least two 128-K blocks, so that every SM
+ * gets work; each range stores its fp32 partial sums in the workspace and a second kernel adds them
+ * in range order (the result does not depend on the timing).  0 for m < 1, n < 1 or k % 128 != 0.
+ */
+size_t q4_linear_workspace_size(int32_t m, const q4_weight* w);
+
+/*
+ * q4_linear_w4a16_ws -- q4_linear_w4a16 with a caller workspace (nullable; device memory, 256-byte
+ * aligned, at least q4_linear_workspace_size(m, w) bytes, else Q4_ERR_ALIGN / Q4_ERR_WORKSPACE).  The
+ * library owns it during the call (kernels on `stream`); it needs no initial contents.  Without a
+ * workspace, or for a shape that is not split, this is q4_linear_w4a16.  The split form computes the
+ * same per-group products; only the order of the fp32 additions across K ranges differs.
+ */
+int q4_linear_w4a16_ws(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * q4_linear_w4a16_grouped -- up to 8 independent small-m W4A16 products in one launch:
  * y[i] = x[i] . dequant(W[i])^T for i < count, each exactly as q4_linear_w4a16 with m <= 4 computes it.
  * Source: as q4_linear_w4a16; the grouping is a launch-level choice (independent linears of one layer
@@ -229,6 +249,14 @@ int act_quant_per_token_f16(const uint16_t* x, int32_t m, int32_t k, int8_t* xq,
  */
 int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                    int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream);
+
+/*
+ * q4_linear_w4a8_ws -- q4_linear_w4a8 with a caller workspace, exactly as q4_linear_w4a16_ws (the INT32
+ * partials are unchanged: each group lies in one K range; the ranges' sums are times scale_a already).
+ */
+int q4_linear_w4a8_ws(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
+                      int32_t out_dtype, int32_t* acc_dbg, void* workspace, size_t workspace_bytes,
+                      int32_t* dev_status, void* stream);
 
 /*
  * moe_q4_workspace_size -- bytes of device workspace moe_q4_forward needs for these sizes.

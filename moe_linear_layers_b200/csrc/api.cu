@@ -4,9 +4,10 @@
 int q4_gemv_w4a16_launch_group(int count, const uint16_t* const* x, int32_t m, const q4_weight* w, void* const* y,
                                int32_t out_dtype, int32_t* dev_status, cudaStream_t stream,
                                const float* const* g = nullptr, const float* const* u = nullptr);
+size_t q4_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k);
 int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                       int32_t out_dtype, int32_t* acc_dbg, bool int8_path, int32_t* dev_status,
-                      cudaStream_t stream);
+                      cudaStream_t stream, void* workspace);
 
 namespace {
 constexpr int kMaxGemvM = 4;
@@ -62,8 +63,30 @@ extern "C" const char* q4_last_cuda_error_string(void)
 
 extern "C" int q4_linear_w4a16_max_gemv_m(void) { return kMaxGemvM; }
 
+extern "C" size_t q4_linear_workspace_size(int32_t m, const q4_weight* w)
+{
+    if (!w || m < 1 || w->n < 1 || w->k < 1 || w->k % 128) return 0;
+    return q4_gemm_workspace_bytes(m, w->n, w->k);   // (a W4A16 call the GEMV serves leaves it unused)
+}
+
+namespace {
+// a caller workspace (nullable): 256-byte aligned, at least q4_linear_workspace_size bytes
+int check_workspace(const void* workspace, size_t bytes, int32_t m, const q4_weight* w)
+{
+    if (!workspace) return Q4_OK;
+    if ((uintptr_t)workspace & 255u) return Q4_ERR_ALIGN;
+    return bytes < q4_linear_workspace_size(m, w) ? Q4_ERR_WORKSPACE : Q4_OK;
+}
+}  // namespace
+
 extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
                                int32_t* dev_status, void* stream)
+{
+    return q4_linear_w4a16_ws(x, m, w, y, out_dtype, nullptr, 0, dev_status, stream);
+}
+
+extern "C" int q4_linear_w4a16_ws(const uint16_t* x, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
     int rc = check_weight(w, false);
     if (rc) return rc;
@@ -71,6 +94,7 @@ extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w,
     if (m < 0) return Q4_ERR_SHAPE;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(x) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
+    if ((rc = check_workspace(workspace, workspace_bytes, m, w))) return rc;
     if (m == 0 || w->n == 0) return Q4_OK;
     if (m <= kMaxGemvM && w->k % 64 == 0) {
         void* ys[1] = {y};
@@ -78,7 +102,8 @@ extern "C" int q4_linear_w4a16(const uint16_t* x, int32_t m, const q4_weight* w,
         if (rc != Q4_ERR_UNSUPPORTED) return rc;  // shapes the GEMV cannot stage go to the GEMM
     }
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
-    return q4_gemm_tc_launch(x, nullptr, m, w, y, out_dtype, nullptr, false, dev_status, (cudaStream_t)stream);
+    return q4_gemm_tc_launch(x, nullptr, m, w, y, out_dtype, nullptr, false, dev_status, (cudaStream_t)stream,
+                             workspace);
 }
 
 extern "C" int q4_linear_w4a16_grouped(int32_t count, const uint16_t* const* x, int32_t m, const q4_weight* w,
@@ -118,6 +143,13 @@ extern "C" int q4_linear_w4a16_swiglu(const float* gate, const float* up, int32_
 extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
                               int32_t out_dtype, int32_t* acc_dbg, int32_t* dev_status, void* stream)
 {
+    return q4_linear_w4a8_ws(xq, scale_a, m, w, y, out_dtype, acc_dbg, nullptr, 0, dev_status, stream);
+}
+
+extern "C" int q4_linear_w4a8_ws(const int8_t* xq, const float* scale_a, int32_t m, const q4_weight* w, void* y,
+                                 int32_t out_dtype, int32_t* acc_dbg, void* workspace, size_t workspace_bytes,
+                                 int32_t* dev_status, void* stream)
+{
     int rc = check_weight(w, false);
     if (rc) return rc;
     if (!xq || !scale_a || !y) return Q4_ERR_NULL;
@@ -125,9 +157,11 @@ extern "C" int q4_linear_w4a8(const int8_t* xq, const float* scale_a, int32_t m,
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(xq) || !q4_aligned16(y) || ((uintptr_t)scale_a & 3u) || ((uintptr_t)acc_dbg & 3u))
         return Q4_ERR_ALIGN;
+    if ((rc = check_workspace(workspace, workspace_bytes, m, w))) return rc;
     if (m == 0 || w->n == 0) return Q4_OK;
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
-    return q4_gemm_tc_launch(xq, scale_a, m, w, y, out_dtype, acc_dbg, true, dev_status, (cudaStream_t)stream);
+    return q4_gemm_tc_launch(xq, scale_a, m, w, y, out_dtype, acc_dbg, true, dev_status, (cudaStream_t)stream,
+                             workspace);
 }
 
 int q4_gemv_w4a16_chain_launch(int n_stages, const int32_t* stage_begin, const uint16_t* const* x,

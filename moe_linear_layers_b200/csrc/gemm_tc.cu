@@ -2,9 +2,43 @@
 // The kernel itself is tcg::tc_gemm_kernel (tc_gemm.cuh) in Dense mode.
 #include "tc_host.cuh"
 
-// m >= 1, k % 128 == 0, group in {64, 128}.
+// Split-K: a problem whose output tiles fill fewer than half the SMs is cut along K into splits of sps
+// 128-K blocks each (at least two), so that splits x tiles approaches the SM count; 1 = no split.
+static int choose_splits(int32_t m, int32_t n, int32_t k, int sms, int* sps)
+{
+    const int tiles = ((m + tcg::BN - 1) / tcg::BN) * ((n + tcg::BM - 1) / tcg::BM);
+    const int kblocks = k / tcg::KBLK;
+    *sps = kblocks;
+    if (tiles < 1 || 2 * tiles > sms || kblocks < 4) return 1;
+    const int want = std::min(kblocks / 2, sms / tiles);
+    if (want < 2) return 1;
+    *sps = (kblocks + want - 1) / want;
+    return (kblocks + *sps - 1) / *sps;
+}
+
+size_t q4_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k)
+{
+    int sps;
+    const int splits = choose_splits(m, n, k, q4_num_sms(), &sps);
+    return splits < 2 ? 0 : (((size_t)splits * m * n * 4 + 255) & ~(size_t)255);
+}
+
+// y = the sum of the splits' partial sums, in split order (the same bits on every run)
+__global__ void split_reduce_kernel(const float* __restrict__ part, int splits, int64_t mn, void* y, int out_bf16)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = part[i];
+        for (int sp = 1; sp < splits; sp++) v += part[(int64_t)sp * mn + i];
+        if (out_bf16) reinterpret_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
+        else reinterpret_cast<float*>(y)[i] = v;
+    }
+}
+
+// m >= 1, k % 128 == 0, group in {64, 128}.  With a workspace of q4_gemm_workspace_bytes, a problem of few
+// output tiles is split along K (the splits' partial sums meet in the workspace and a second kernel adds
+// them up); without one, or when the shape is not split, one kernel writes y.
 int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_weight* w, void* y, int32_t out_dtype,
-                      int32_t* acc_dbg, bool int8_path, int32_t* dev_status, cudaStream_t stream)
+                      int32_t* acc_dbg, bool int8_path, int32_t* dev_status, cudaStream_t stream, void* workspace)
 {
     using namespace tcg;
     if (w->k % KBLK) return Q4_ERR_UNSUPPORTED;
@@ -24,17 +58,34 @@ int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_w
     p.acc_dbg = acc_dbg;
     p.status = dev_status;
     const int tiles = ((m + BN - 1) / BN) * ((w->n + BM - 1) / BM);
-    const int grid = std::min(tiles, q4_num_sms());
+    const int sms = q4_num_sms();
+    p.splits = 1;
+    p.sps = w->k / KBLK;
+    if (workspace) {
+        p.splits = choose_splits(m, w->n, w->k, sms, &p.sps);
+        p.part = reinterpret_cast<float*>(workspace);
+    }
+    if (p.splits < 2) p.splits = 1;
+    const int grid = std::min(tiles * p.splits, sms);
+    int rc;
     if (int8_path) {
         if (w->group == 128)
-            return w->symmetric ? launch<true, 128, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
-                                : launch<true, 128, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
-        return w->symmetric ? launch<true, 64, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
-                            : launch<true, 64, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
+            rc = w->symmetric ? launch<true, 128, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
+                              : launch<true, 128, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
+        else
+            rc = w->symmetric ? launch<true, 64, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
+                              : launch<true, 64, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
+    } else {
+        if (w->group == 128)
+            rc = w->symmetric ? launch<false, 128, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
+                              : launch<false, 128, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
+        else
+            rc = w->symmetric ? launch<false, 64, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
+                              : launch<false, 64, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
     }
-    if (w->group == 128)
-        return w->symmetric ? launch<false, 128, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
-                            : launch<false, 128, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
-    return w->symmetric ? launch<false, 64, true, Mode::Dense>(mx, mw, mw, p, grid, stream)
-                        : launch<false, 64, false, Mode::Dense>(mx, mw, mw, p, grid, stream);
+    if (rc || p.splits == 1) return rc;
+    const int64_t mn = (int64_t)m * w->n;
+    split_reduce_kernel<<<(int)std::min<int64_t>((mn + 255) / 256, 4 * sms), 256, 0, stream>>>(
+        p.part, p.splits, mn, y, out_dtype == Q4_OUT_BF16);
+    return q4_launch_status();
 }

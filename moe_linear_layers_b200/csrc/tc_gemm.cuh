@@ -159,6 +159,11 @@ struct Args {
     int h_f16;                     // GateUp: h for an INT8 down projection, stored as the fp16 activation
     int E, topk;
     int T;                         // Down: rows of the output y (tokens)
+    // Dense split-K (splits > 1): work item t is split t % splits of output tile t / splits and covers the
+    // K blocks [split * sps, min(K / 128, (split + 1) * sps)); it stores its fp32 partial sums (times s_a
+    // for W4A8) in part[split][M][N], which a second kernel adds up in split order
+    int splits, sps;
+    float* part;
 };
 
 struct Tile {
@@ -166,7 +171,25 @@ struct Tile {
     int n0;           // Dense/Down: first weight row of the tile inside the (expert) matrix; GateUp: i0
     int wrow_a, wrow_b;  // packed rows of the TMA boxes
     int e;
+    int kb0, kb1;     // the work item's 128-K blocks (all of them unless the K dimension is split)
+    int split;
 };
+
+// The K blocks of work item t (Dense split-K) or of every tile.
+template <Mode MODE>
+__device__ __forceinline__ void item_blocks(int t, const Args& p, int kblocks, int& kb0, int& kb1, int& split)
+{
+    kb0 = 0;
+    kb1 = kblocks;
+    split = 0;
+    if constexpr (MODE == Mode::Dense) {
+        if (p.splits > 1) {
+            split = t % p.splits;
+            kb0 = split * p.sps;
+            kb1 = min(kblocks, kb0 + p.sps);
+        }
+    }
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr)
 {
@@ -260,7 +283,9 @@ template <Mode MODE>
 __device__ __forceinline__ Tile map_tile(int t, const Args& p, const Shared* sh, int tiles_m)
 {
     Tile T;
+    item_blocks<MODE>(t, p, p.K / KBLK, T.kb0, T.kb1, T.split);
     if constexpr (MODE == Mode::Dense) {
+        if (p.splits > 1) t /= p.splits;   // the output tile
         T.e = 0;
         T.m0 = (t % tiles_m) * BN;
         T.m_end = p.M;
@@ -306,16 +331,18 @@ __device__ __forceinline__ void row_params(const Args& p, const Tile& T, int r, 
 
 // W4A8 epilogue: fp16 scales of one row, n of them, read 4 at a time, one 8-byte block ahead: the
 // block for positions [4j, 4j+4) is loaded when position 4j-4 is taken, so a register that is still
-// loading is touched (moved) only 4 positions later.  n % 4 != 0 falls back to direct loads.
+// loading is touched (moved) only 4 positions later.  n % 4 != 0 or a row that is not 8-byte aligned (a
+// split-K item's slice of the row) falls back to direct loads.
 // preload() issues the first block of the next row one tile early, so start() does not wait for it.
 struct QuadRing {
     const __half* row = nullptr;
     const __half* pre_row = nullptr;
     int n = 0;
     uint2 cur, nxt, pre;
+    bool vec = false;   // 8-byte blocks (count % 4 == 0 and an 8-byte aligned row; else direct loads)
     __device__ __forceinline__ void preload(const __half* r, int count)
     {
-        pre_row = (r && (count & 3) == 0) ? r : nullptr;
+        pre_row = (r && (count & 3) == 0 && ((uintptr_t)r & 7) == 0) ? r : nullptr;
         if (pre_row) pre = __ldg(reinterpret_cast<const uint2*>(r));
     }
     __device__ __forceinline__ void start(const __half* r, int count)
@@ -323,12 +350,13 @@ struct QuadRing {
         row = r;
         n = count;
         cur = nxt = make_uint2(0u, 0u);
-        if (row && (n & 3) == 0) nxt = row == pre_row ? pre : __ldg(reinterpret_cast<const uint2*>(row));
+        vec = row && (n & 3) == 0 && ((uintptr_t)row & 7) == 0;
+        if (vec) nxt = row == pre_row ? pre : __ldg(reinterpret_cast<const uint2*>(row));
     }
     __device__ __forceinline__ float get(int i)   // positions in increasing order, from 0
     {
         if (!row) return 0.0f;
-        if (n & 3) return __half2float(row[i]);
+        if (!vec) return __half2float(row[i]);
         if ((i & 3) == 0) {
             cur = nxt;
             nxt = i + 4 < n ? __ldg(reinterpret_cast<const uint2*>(row + i + 4)) : make_uint2(0u, 0u);
@@ -414,13 +442,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         tc::mbar_init(&sh->h_ready[0], 4);
         tc::mbar_init(&sh->h_ready[1], 4);
         sh->abort_flag = 0;
-        if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM);
+        if constexpr (MODE == Mode::Dense) sh->total_tiles = tiles_m * ((p.N + BM - 1) / BM) * max(p.splits, 1);
         else sh->total_tiles = p.expert_tiles[p.E] - p.expert_tiles[0];
         tc::fence_mbar_init();
     }
     // (a class of experts passes its slice of the layer's tile prefix sums: counted from its first expert)
     if constexpr (MODE != Mode::Dense)
         for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sh->expert_tiles[i] = p.expert_tiles[i] - p.expert_tiles[0];
+    // Dense: the first work item's first parameter window is staged here by every thread, one group row
+    // piece each, so its global reads are one round trip instead of the loader warp's one per row it
+    // stages (which delayed every launch's first stage by ~2.5 us); the loader then only publishes it
+    if constexpr (MODE == Mode::Dense && PRING) {
+        const int total0 = tiles_m * ((p.N + BM - 1) / BM) * max(p.splits, 1);
+        if ((int)blockIdx.x < total0) {
+            const Tile T0 = map_tile<MODE>(blockIdx.x, p, sh, tiles_m);
+            const int grp0 = T0.kb0 * GPK, ngr = (T0.kb1 - T0.kb0) * GPK;   // (Dense: SPG == 1)
+            constexpr int kPieces = C::PTENS * BM * (PW / 8);                 // tensor x row x 8 groups
+            for (int i = threadIdx.x; i < kPieces; i += kThreads) {
+                const int ten = i / (BM * (PW / 8)), r = (i / (PW / 8)) % BM, q = i % (PW / 8);
+                if (SYM && ten == 1) continue;
+                const __half *srow, *zrow;
+                row_params<MODE>(p, T0, r, ngroups, srow, zrow);
+                const __half* row = ten == 0 ? srow : zrow;
+                uint16_t* d = reinterpret_cast<uint16_t*>(params + ten * PW * BM + r);   // window slot 0
+                uint16_t v[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int gg = 8 * q + j;
+                    v[j] = (row && gg < ngr) ? __half_as_ushort(row[grp0 + gg]) : (uint16_t)0;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; j++) d[(8 * q + j) * BM] = v[j];
+            }
+        }
+    }
     if (warp == 0 && lane == 0) {
         tc::tma_prefetch_desc(&tm_x);
         tc::tma_prefetch_desc(&tm_wa);
@@ -443,18 +498,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // count in shared memory, and the producer polls that count with plain loads.
         if (lane == 0 && warp == 9) {
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x)
-                for (int kb = 0; kb < kblocks; kb++, it++) {
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                int kb0, kb1, sp;
+                item_blocks<MODE>(t, p, kblocks, kb0, kb1, sp);
+                for (int kb = kb0; kb < kb1; kb++, it++) {
                     if (!tc::mbar_wait(&sh->xw_empty[it % NS], (it / NS) & 1, p.status, abort_flag)) goto watch_done;
                     tc::sts_publish(&sh->slot_free, it + 1);
                 }
+            }
         watch_done:;
         } else if (lane == 0 && warp == 8) {
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
-                for (int kb = 0; kb < kblocks; kb++, it++) {
+                for (int kb = T.kb0; kb < T.kb1; kb++, it++) {
                     const int s = it % NS;
                     if (it >= (uint32_t)NS) {
                         // stage it - NS, the slot's previous one, has been released
@@ -487,20 +545,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             // -------------------------------------------------------------- parameter loader (warp 10)
             // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
             // ahead of the converters and the epilogue, so that their loops make no global loads.
-            const int nwin = (ngroups + PW - 1) / PW;
             uint32_t wi = 0;
             for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+                // the item's groups (all of the tile's unless K is split)
+                const int grp0 = SPG > 1 ? T.kb0 / SPG : T.kb0 * GPK;
+                const int ngr = SPG > 1 ? (T.kb1 - T.kb0) / SPG : (T.kb1 - T.kb0) * GPK;
+                const int nwin = (ngr + PW - 1) / PW;
                 for (int w = 0; w < nwin; w++, wi++) {
                     if (!tc::mbar_wait(&sh->p_empty[wi & 1], ((wi >> 1) & 1) ^ 1, p.status, abort_flag)) goto load_done;
                     __half* ps = params + (wi & 1) * C::PTENS * PW * BM;
 #pragma unroll 1
-                    for (int i = 0; i < BM / 32; i++) {
+                    for (int i = 0; i < BM / 32 && !(MODE == Mode::Dense && wi == 0); i++) {   // (window 0: staged above)
                         const int r = 32 * i + lane;
                         const __half *srow, *zrow;
                         row_params<MODE>(p, T, r, ngroups, srow, zrow);
-                        stage_params<PW>(srow, w * PW, ngroups, ps + r);
-                        if constexpr (!SYM) stage_params<PW>(zrow, w * PW, ngroups, ps + PW * BM + r);
+                        stage_params<PW>(srow ? srow + grp0 : nullptr, w * PW, ngr, ps + r);
+                        if constexpr (!SYM) stage_params<PW>(zrow ? zrow + grp0 : nullptr, w * PW, ngr, ps + PW * BM + r);
                     }
                     tc::mbar_arrive(&sh->p_full[wi & 1]);   // every lane: its stores are visible
                 }
@@ -519,7 +580,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             bool ok = true;
             if constexpr (INT8) ok = tc::poll_counters<8>(sh->epi_init, 1, p.status, abort_flag);
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                for (int kb = 0; kb < kblocks && ok; kb++, it++) {
+                int kb0, kb1, sp;
+                item_blocks<MODE>(t, p, kblocks, kb0, kb1, sp);
+                for (int kb = kb0; kb < kb1 && ok; kb++, it++) {
                     // (the SPG stages of one group go to one issuer, whose MMAs into the group's accumulator
                     // are then ordered)
                     if ((it / SPG) % kIssuers != (uint32_t)warp) {   // another issuer's stage
@@ -585,21 +648,25 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         constexpr float kMagic = 128.0f;
         uint32_t it = 0, wi = 0;   // stage and parameter-window counters (running across tiles)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            for (int kb = 0; kb < kblocks; kb++) {
+            int kb0, kb1, sp;
+            item_blocks<MODE>(t, p, kblocks, kb0, kb1, sp);
+            const int ngr = SPG > 1 ? (kb1 - kb0) / SPG : (kb1 - kb0) * GPK;   // the item's groups
+            for (int kb = kb0; kb < kb1; kb++) {
                 const int s = it % NS, sa = it % C::NA;
                 // zero points of the stage's groups from the parameter ring
                 float zcur[GPK];
 #pragma unroll
                 for (int gi = 0; gi < GPK; gi++) zcur[gi] = 8.0f;
                 if constexpr (PRING) {
-                    const int g0 = SPG > 1 ? kb / SPG : kb * GPK;   // the first group of the stage
+                    // the first group of the stage, counted from the item's first group
+                    const int g0 = SPG > 1 ? (kb - kb0) / SPG : (kb - kb0) * GPK;
                     const bool gf = kb % SPG == 0, gl_ = kb % SPG == SPG - 1;   // first / last stage of its group
                     if (g0 % PW == 0 && gf && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag))
                         goto conv_done;
                     const __half* pz = params + (wi & 1) * C::PTENS * PW * BM + PW * BM + r;
 #pragma unroll
                     for (int gi = 0; gi < GPK; gi++) zcur[gi] = SYM ? 8.0f : __half2float(pz[((g0 + gi) % PW) * BM]);
-                    if (gl_ && ((g0 + GPK) % PW == 0 || g0 + GPK >= ngroups)) {   // the window's last stage: release it
+                    if (gl_ && ((g0 + GPK) % PW == 0 || g0 + GPK >= ngr)) {   // the window's last stage: release it
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
                         wi++;
@@ -699,15 +766,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         QuadRing sr;       // W4A8: group scales read a few groups ahead
         for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
             const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+            // the item's groups (all of the tile's unless K is split)
+            const int grp0 = SPG > 1 ? T.kb0 / SPG : T.kb0 * GPK;
+            const int ngr = SPG > 1 ? (T.kb1 - T.kb0) / SPG : (T.kb1 - T.kb0) * GPK;
             const __half *srow, *zrow;
             row_params<MODE>(p, T, r, ngroups, srow, zrow);
             if constexpr (INT8) {
-                sr.start(srow, ngroups);
+                sr.start(srow ? srow + grp0 : nullptr, ngr);
                 if (t + (int)gridDim.x < total) {   // load the next tile's first block of scales now
                     const Tile Tn = map_tile<MODE>(t + gridDim.x, p, sh, tiles_m);
                     const __half *sn, *zn;
                     row_params<MODE>(p, Tn, r, ngroups, sn, zn);
-                    sr.preload(sn, ngroups);
+                    const int g0n = SPG > 1 ? Tn.kb0 / SPG : Tn.kb0 * GPK;
+                    sr.preload(sn ? sn + g0n : nullptr, SPG > 1 ? (Tn.kb1 - Tn.kb0) / SPG : (Tn.kb1 - Tn.kb0) * GPK);
                 }
             }
 #pragma unroll
@@ -723,7 +794,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     comb_w[ew * 64 + j] = cw;
                 }
             }
-            for (int gl = 0; gl < ngroups; gl++) {
+            for (int gl = 0; gl < ngr; gl++) {
                 const uint32_t db = g % C::ND;
                 // group scale: W4A8 from its read-ahead ring, 16-bit modes from the parameter ring
                 float s;
@@ -732,7 +803,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 } else {
                     if (gl % PW == 0 && !tc::mbar_wait(&sh->p_full[wi & 1], (wi >> 1) & 1, p.status, abort_flag)) goto epi_done;
                     s = __half2float(params[(wi & 1) * C::PTENS * PW * BM + (gl % PW) * BM + r]);
-                    if ((gl + 1) % PW == 0 || gl + 1 == ngroups) {   // the window's last group: release it
+                    if ((gl + 1) % PW == 0 || gl + 1 == ngr) {   // the window's last group: release it
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh->p_empty[wi & 1]);
                         wi++;
@@ -753,7 +824,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                             for (int j = 0; j < 32; j++) {
                                 const int m = T.m0 + half * 64 + 32 * h + j;
-                                const int64_t o = ((int64_t)m * p.N + T.n0 + r) * ngroups + gl;
+                                const int64_t o = ((int64_t)m * p.N + T.n0 + r) * ngroups + grp0 + gl;
                                 if (m < T.m_end && q4_in_bounds(o, (int64_t)p.M * p.N * ngroups, p.status))
                                     p.acc_dbg[o] = ((int32_t)(v[j] - kAccBias)) >> (SYM ? 4 : 0);
                             }
@@ -788,7 +859,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const int rows = min(64, p.M - mb);
                 if (n < p.N && rows > 0) {
                     const int64_t base = (int64_t)mb * p.N + n;
-                    if (p.out_bf16) {
+                    if (p.splits > 1) {   // this split's partial sums, for the split reduction
+                        float* pf = p.part + (int64_t)T.split * p.M * p.N + base;
+                        const int64_t lim = (int64_t)p.splits * p.M * p.N - ((int64_t)T.split * p.M * p.N + base);
+#pragma unroll
+                        for (int j = 0; j < 64; j++)
+                            if (j < rows) {
+                                float v = accv(j);
+                                if constexpr (INT8) v *= __ldg(p.scale_a + mb + j);
+                                if (q4_in_bounds((int64_t)j * p.N, lim, p.status)) pf[(int64_t)j * p.N] = v;
+                            }
+                    } else if (p.out_bf16) {
                         __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(p.y) + base;
                         if (rows == 64) {
 #pragma unroll

@@ -40,7 +40,7 @@ EXPORTED = ("q4_status_string", "q4_version", "q4_build_flags", "q4_last_cuda_er
             "act_quant_per_token_f16", "moe_q4_workspace_size_a8", "moe_q4_forward_a8", "moe_q4_forward_classes",
             "moe_q4_forward_range", "q4_linear_w4a16_chain_sync_bytes", "q4_linear_w4a16_chain",
             "moe_q4_route_workspace_size", "moe_q4_route", "moe_q4_rows_workspace_size", "moe_q4_forward_rows",
-            "moe_q4_combine")
+            "moe_q4_combine", "q4_linear_workspace_size", "q4_linear_w4a16_ws", "q4_linear_w4a8_ws")
 Q4_MOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -65,6 +65,10 @@ _lib.q4_linear_w4a16_grouped.argtypes = [_i32, ctypes.POINTER(_p), _i32, ctypes.
 _lib.act_quant_per_token.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
 _lib.act_quant_per_token_f16.argtypes = [_p, _i32, _i32, _p, _p, _p, _p]
 _lib.q4_linear_w4a8.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _p]
+_lib.q4_linear_workspace_size.restype = _sz
+_lib.q4_linear_workspace_size.argtypes = [_i32, ctypes.POINTER(q4_weight)]
+_lib.q4_linear_w4a16_ws.argtypes = [_p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _sz, _p, _p]
+_lib.q4_linear_w4a8_ws.argtypes = [_p, _p, _i32, ctypes.POINTER(q4_weight), _p, _i32, _p, _p, _sz, _p, _p]
 _lib.moe_q4_workspace_size.restype = _sz
 _lib.moe_q4_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.moe_q4_forward.argtypes = [_p, _i32, _i32, _p, _p, _i32, _i32, ctypes.POINTER(q4_weight), _i32, _p, _i32,
@@ -232,16 +236,39 @@ def q4_quantize_pack(w: torch.Tensor, group: int, symmetric: bool, dev_status: t
     return q
 
 
+_SPLIT_WS = {}   # device -> the workspace of split-K GEMMs, grown to the largest size asked for
+
+
+def linear_workspace(m: int, w: Q4Weight, device) -> torch.Tensor | None:
+    """A device workspace for q4_linear_w4a16_ws / q4_linear_w4a8_ws at these sizes (None when the shape
+    is not split along K), kept per device and grown as needed.  Calls that share it must be ordered on
+    one stream; pass your own to run on several streams at once."""
+    need = int(_lib.q4_linear_workspace_size(int(m), ctypes.byref(w.desc)))
+    if need == 0:
+        return None
+    ws = _SPLIT_WS.get(device)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty((need,), dtype=torch.uint8, device=device)
+        _SPLIT_WS[device] = ws
+    return ws
+
+
 def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: torch.Tensor | None = None,
-                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor."""
+                    dev_status: torch.Tensor | None = None, stream=None, workspace="auto") -> torch.Tensor:
+    """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor.  workspace: "auto" (the per-device one of
+    linear_workspace: a GEMM of few output tiles is split along K), None (never split) or a uint8 tensor."""
     _dev(x, torch.bfloat16, "x")
     m = x.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
     od = _out(y, (m, w.n), x.device)
-    _check(_lib.q4_linear_w4a16(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status), _stream(stream)),
-           "q4_linear_w4a16")
+    if isinstance(workspace, str):
+        workspace = linear_workspace(m, w, x.device) if m > q4_linear_w4a16_max_gemv_m() else None
+    if workspace is not None:
+        _workspace(workspace, x.device)
+    _check(_lib.q4_linear_w4a16_ws(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(workspace),
+                                   workspace.numel() if workspace is not None else 0, _ptr(dev_status),
+                                   _stream(stream)), "q4_linear_w4a16")
     return y
 
 
@@ -372,16 +399,22 @@ def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a
 
 def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dtype=torch.float32,
                    y: torch.Tensor | None = None, acc_dbg: torch.Tensor | None = None,
-                   dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . (code - zero))_g; zero = 0 for symmetric W."""
+                   dev_status: torch.Tensor | None = None, stream=None, workspace="auto") -> torch.Tensor:
+    """y[m][n] = scale_a[m] * sum_g scale_w[n][g] * (xq . (code - zero))_g; zero = 0 for symmetric W.
+    workspace: as q4_linear_w4a16's."""
     _dev(xq, torch.int8, "xq")
     _dev(scale_a, torch.float32, "scale_a")
     m = xq.shape[0]
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
     od = _out(y, (m, w.n), xq.device)
-    _check(_lib.q4_linear_w4a8(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
-                               _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
+    if isinstance(workspace, str):
+        workspace = linear_workspace(m, w, xq.device)
+    if workspace is not None:
+        _workspace(workspace, xq.device)
+    _check(_lib.q4_linear_w4a8_ws(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
+                                  _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                  _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
     return y
 
 

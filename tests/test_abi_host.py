@@ -288,3 +288,23 @@ def test_binding_argument_checks():
     assert q4._numel(torch.zeros(6), 6, "t") is not None
     with pytest.raises(ValueError):
         q4._numel(torch.zeros(5), 6, "pair_pos")
+
+
+def test_linear_workspace_validation():
+    """Split-K workspace of the dense GEMM: its size rule and the checks of a caller workspace."""
+    L = q4._lib
+    w = _w(n=2048, k=2048, group=128, sym=1)
+    need = L.q4_linear_workspace_size(64, ctypes.byref(w))
+    assert need > 0 and need % 256 == 0                          # 16 output tiles: split
+    assert L.q4_linear_workspace_size(4096, ctypes.byref(_w(n=8192, k=2048, group=128))) == 0   # enough tiles
+    assert L.q4_linear_workspace_size(64, ctypes.byref(_w(n=2048, k=256, group=128))) == 0      # 2 K blocks
+    assert L.q4_linear_workspace_size(0, ctypes.byref(w)) == 0
+    P = ctypes.c_void_p
+    call = lambda ws, nb: L.q4_linear_w4a16_ws(P(FAKE), 64, ctypes.byref(w), P(FAKE), 0, P(ws) if ws else None, nb,
+                                               None, None)
+    assert call(FAKE + 16, need) == q4.Q4_ERR_ALIGN
+    assert call(FAKE, need - 1) == q4.Q4_ERR_WORKSPACE
+    call8 = lambda ws, nb: L.q4_linear_w4a8_ws(P(FAKE), P(FAKE), 64, ctypes.byref(w), P(FAKE), 0, None,
+                                               P(ws) if ws else None, nb, None, None)
+    assert call8(FAKE + 16, need) == q4.Q4_ERR_ALIGN
+    assert call8(FAKE, need - 1) == q4.Q4_ERR_WORKSPACE

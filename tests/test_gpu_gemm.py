@@ -2,6 +2,8 @@
 
 Floating outputs: max|err| <= 1e-2 * rms(fp64 oracle).  bf16 outputs equal the round-to-nearest-even of
 the fp32 outputs bit for bit.  W4A8's per-group INT32 partials (debug output) are bit-exact."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -115,3 +117,43 @@ def test_w4a8_asym_workload_shapes(q4, m, n, k):
     rows = np.arange(0, m, max(1, m // 32))
     ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, 128, rows_m=rows, zeros=zr, symmetric=False)
     assert_close(y.cpu().numpy()[rows], ref, what=f"w4a8 asym {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k,group,sym", [
+    (64, 2048, 1408, 128, False),   # 11 K blocks in splits of 3: a ragged last split
+    (64, 2048, 1408, 64, True),     # two groups per K block
+    (96, 640, 4096, 128, True),     # 5 output tiles, many splits
+])
+def test_w4a16_split_k(q4, m, n, k, group, sym):
+    """A GEMM of few output tiles split along K (q4_linear_w4a16_ws): against the oracle, and against the
+    unsplit form of the same call (the same per-group products, summed in another order)."""
+    W = synth.weights(("test", "splitk", n, k, group, sym), n, k)
+    pk, sc, zr = oracle.quantize(W, group, sym)
+    x = synth.activations(("test", "splitk-x", m, k), m, k)
+    ref = oracle.linear_w4a16(x, pk, sc, zr, n, k, group, sym)
+    w = upload_weight(q4, pk, sc, zr, n, k, group, sym)
+    assert q4._lib.q4_linear_workspace_size(m, ctypes.byref(w.desc)) > 0, "the shape should be split"
+    xd = cuda_u16_as(x, torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ys = q4.q4_linear_w4a16(xd, w, dev_status=st)
+    yu = q4.q4_linear_w4a16(xd, w, dev_status=st, workspace=None)
+    y16 = q4.q4_linear_w4a16(xd, w, out_dtype=torch.bfloat16, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close(ys.cpu().numpy(), ref, what="split")
+    assert_close(yu.cpu().numpy(), ref, what="unsplit")
+    d = np.abs(ys.cpu().numpy() - yu.cpu().numpy()).max() / np.sqrt(np.mean(ref * ref))
+    assert d < 1e-5, f"split and unsplit differ by {d} of rms"
+    assert np.array_equal(cpu_u16(y16), bf16_rne(ys.cpu().numpy()))
+
+
+@pytest.mark.parametrize("m,n,k,group,sym", [(16, 1024, 1408, 128, True), (32, 640, 2048, 64, False)])
+def test_w4a8_split_k_partials_bitexact(q4, m, n, k, group, sym):
+    """W4A8 split along K: every group's INT32 partial bit-exact (each group lies in one K range), y within
+    tolerance of the oracle."""
+    y, acc, (xq, sa, pk, sc, zr), w, *_ = _w4a8(q4, m, n, k, group, "split", want_acc=True, sym=sym)
+    assert q4._lib.q4_linear_workspace_size(m, ctypes.byref(w.desc)) > 0, "the shape should be split"
+    kw = {} if sym else dict(zeros=zr, symmetric=False)
+    ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True, **kw)
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_close(y.cpu().numpy(), ref, what="w4a8 split")
