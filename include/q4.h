@@ -119,8 +119,8 @@ int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t group, int32_
  * dequant); larger m runs the tcgen05 tensor-core GEMM (exact integer codes in bf16, fp32
  * accumulation per group, scale applied per group in the epilogue).  The choice is by shape only.
  * The GEMV serves k % 64 == 0, k <= 16384; the GEMM serves k % 128 == 0 (see q4_linear_w4a16_max_gemv_m).
- * The GEMV may start, and read W (packed, scales, zeros) into shared memory and L2, before the
- * previous kernel on the stream has finished (programmatic dependent launch); it reads x and writes y
+ * Both kernels may start, and read W (packed, scales, zeros) into shared memory, TMEM and L2, before the
+ * previous kernel on the stream has finished (programmatic dependent launch); they read x and write y
  * only after that kernel's writes are visible.  So W must not be written by the immediately preceding
  * kernel when that kernel releases its dependents early (none of this library's kernels that write
  * weights does).  Inside the GEMV, x is taken per 64-value block as int16 with a power-of-two scale

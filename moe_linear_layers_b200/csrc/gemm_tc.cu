@@ -26,6 +26,9 @@ size_t q4_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k)
 // y = the sum of the splits' partial sums, in split order (the same bits on every run)
 __global__ void split_reduce_kernel(const float* __restrict__ part, int splits, int64_t mn, void* y, int out_bf16)
 {
+    // launched as a programmatic dependent of the GEMM: the partials are read after its completion
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += (int64_t)gridDim.x * blockDim.x) {
         float v = part[i];
         for (int sp = 1; sp < splits; sp++) v += part[(int64_t)sp * mn + i];
@@ -85,7 +88,15 @@ int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_w
     }
     if (rc || p.splits == 1) return rc;
     const int64_t mn = (int64_t)m * w->n;
-    split_reduce_kernel<<<(int)std::min<int64_t>((mn + 255) / 256, 4 * sms), 256, 0, stream>>>(
-        p.part, p.splits, mn, y, out_dtype == Q4_OUT_BF16);
-    return q4_launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((mn + 255) / 256, 4 * sms));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return q4_cuda_status(cudaLaunchKernelEx(&cfg, split_reduce_kernel, (const float*)p.part, p.splits, mn, y,
+                                             (int)(out_dtype == Q4_OUT_BF16)));
 }

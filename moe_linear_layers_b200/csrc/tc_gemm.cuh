@@ -487,6 +487,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tc::fence_after_sync();
     const uint32_t tbase = sh->tmem_base;
     const int total = sh->total_tiles;
+    // Dense launches use programmatic dependent launch: the next kernel on the stream may start (its
+    // prologue and weight copies) while this one runs; it reads this one's outputs only after its own
+    // griddepcontrol.wait, which waits for this grid's completion and memory flush
+    if constexpr (MODE == Mode::Dense)
+        if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int wg = warp / 4;
     if (wg == 2) {
@@ -510,6 +515,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         } else if (lane == 0 && warp == 8) {
             uint32_t it = 0;
             bool ok = true;
+            bool dep_ready = MODE != Mode::Dense;   // (Dense: x may come from the previous kernel)
             for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
                 const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
                 for (int kb = T.kb0; kb < T.kb1; kb++, it++) {
@@ -531,6 +537,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                     tc::mbar_arrive_expect_tx(&sh->x_full[s], C::XSTAGE);
                     uint8_t* xdst = xs + s * C::XSTAGE;
+                    if (!dep_ready) {   // the weights above may be read early; the activations only now
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        dep_ready = true;
+                    }
                     if constexpr (INT8) tc::tma_load_2d(xdst, &tm_x, &sh->x_full[s], kb * KBLK, T.m0);
                     else tc::tma_load_3d(xdst, &tm_x, &sh->x_full[s], 0, T.m0, kb * C::XBLK);   // the stage's 64-column blocks
                 }

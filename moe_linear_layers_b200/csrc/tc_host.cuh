@@ -78,8 +78,23 @@ int launch(const CUtensorMap& mx, const CUtensorMap& ma, const CUtensorMap& mb, 
         return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
     }();
     if (nregs != kLaunchRegs) return Q4_ERR_UNSUPPORTED;
-    kern<<<grid, kThreads, smem, s>>>(mx, ma, mb, p);
-    return q4_launch_status();
+    if constexpr (MODE == Mode::Dense) {
+        // programmatic dependent launch (see the kernel: only the activation copies wait)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return q4_cuda_status(cudaLaunchKernelEx(&cfg, kern, mx, ma, mb, p));
+    } else {
+        kern<<<grid, kThreads, smem, s>>>(mx, ma, mb, p);
+        return q4_launch_status();
+    }
 }
 
 }  // namespace tcg
