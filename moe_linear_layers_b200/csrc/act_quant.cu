@@ -75,6 +75,29 @@ __device__ __forceinline__ uint32_t word_amax(const uint4& v, uint32_t& bad)
     return a;
 }
 
+// The kernels are launched as programmatic dependents (launch_pdl): a kernel lets the next one on the
+// stream launch at once, and reads x and writes its outputs only after the previous kernel's completion.
+__device__ __forceinline__ void pdl_start()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... P, typename... A>
+int launch_pdl(void (*kern)(P...), int grid, int block, cudaStream_t s, A... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return q4_cuda_status(cudaLaunchKernelEx(&cfg, kern, args...));
+}
+
 // W = 16-byte words per thread kept in registers (k <= 8 * kThreads * W); W = 0: any k, two passes.
 template <int W, bool F16>
 __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __restrict__ x, int k,
@@ -82,6 +105,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
                                                              int32_t* status)
 {
     __shared__ uint32_t red[kThreads / 32];
+    pdl_start();
     const int64_t row = blockIdx.x;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * k);
     uint2* out = reinterpret_cast<uint2*>(xq + row * k);
@@ -134,6 +158,7 @@ __global__ void __launch_bounds__(256) act_quant_warp_kernel(const uint16_t* __r
                                                              int8_t* __restrict__ xq, float* __restrict__ scale_a,
                                                              int32_t* status)
 {
+    pdl_start();
     const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= m) return;
@@ -175,14 +200,13 @@ int act_quant_launch(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float*
     if (m == 0) return Q4_OK;
     const int n8 = k / 8;
     const int wgrid = (m + 7) / 8;
-    if (n8 <= 32 * 2) act_quant_warp_kernel<2, F16><<<wgrid, 256, 0, s>>>(x, m, k, xq, scale_a, dev_status);
-    else if (n8 <= 32 * 4) act_quant_warp_kernel<4, F16><<<wgrid, 256, 0, s>>>(x, m, k, xq, scale_a, dev_status);
-    else if (n8 <= kThreads) act_quant_kernel<1, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 2 * kThreads) act_quant_kernel<2, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 4 * kThreads) act_quant_kernel<4, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else if (n8 <= 8 * kThreads) act_quant_kernel<8, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    else act_quant_kernel<0, F16><<<m, kThreads, 0, s>>>(x, k, xq, scale_a, dev_status);
-    return q4_launch_status();
+    if (n8 <= 32 * 2) return launch_pdl(act_quant_warp_kernel<2, F16>, wgrid, 256, s, x, m, k, xq, scale_a, dev_status);
+    if (n8 <= 32 * 4) return launch_pdl(act_quant_warp_kernel<4, F16>, wgrid, 256, s, x, m, k, xq, scale_a, dev_status);
+    if (n8 <= kThreads) return launch_pdl(act_quant_kernel<1, F16>, m, kThreads, s, x, k, xq, scale_a, dev_status);
+    if (n8 <= 2 * kThreads) return launch_pdl(act_quant_kernel<2, F16>, m, kThreads, s, x, k, xq, scale_a, dev_status);
+    if (n8 <= 4 * kThreads) return launch_pdl(act_quant_kernel<4, F16>, m, kThreads, s, x, k, xq, scale_a, dev_status);
+    if (n8 <= 8 * kThreads) return launch_pdl(act_quant_kernel<8, F16>, m, kThreads, s, x, k, xq, scale_a, dev_status);
+    return launch_pdl(act_quant_kernel<0, F16>, m, kThreads, s, x, k, xq, scale_a, dev_status);
 }
 
 }  // namespace
