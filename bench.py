@@ -12,9 +12,11 @@ Metric: HBM GB/s = algorithmic bytes (packed weights + fp16 scales + fp16 zeros 
 of the step / device time of the step.
 
 At one GPU the line also carries "components", the other rows of the hot path on their workloads:
-  prefill  W4A16 GEMM, m = 2048, the same 112 weight matrices, x with 1% of channels x10 (TFLOP/s);
-  w4a8     per-token INT8 act-quant + W4A8 GEMM, m = 4096, the same shapes quantized symmetrically,
-           Student-t(3) activations (TOPS);
+  prefill  W4A16 GEMM, m = 2048, the same 112 weight matrices issued as a decoder layer can issue them
+           at m > 4 ([q,k,v] and [gate,up] each one GEMM over stacked weights: 64 GEMMs), x with 1%
+           of channels x10 (TFLOP/s); also at m = 64 and m = 512;
+  w4a8     per-token INT8 act-quant + W4A8 GEMM, m = 4096, the same shapes quantized symmetrically and
+           stacked the same way, Student-t(3) activations (TOPS); also at m = 16 and m = 256;
   moe      the MoE layer: 4096 tokens, hidden 2048, 64 experts of intermediate 1024, top-8 (tokens/s).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
@@ -27,6 +29,7 @@ exchange); value = bytes of all ranks / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -428,15 +431,32 @@ def run_decode(q4, args, ws, weights, dev):
     }
 
 
+def layer_gemms(q4, weights):
+    """The 112 matrices issued the way a decoder layer can issue them at m > 4: [q,k,v] and [gate,up] (which
+    read the same input) each as ONE GEMM over their stacked weights (Q4Weight.stack: the parts' quantized
+    rows one after another, so the products are exactly the parts'), o and down alone: 64 GEMMs per step."""
+    out = []
+    for l in range(synth.LLAMA_1B_LAYERS):
+        w = weights[7 * l: 7 * l + 7]
+        out += [q4.Q4Weight.stack(w[0:3]), w[3], q4.Q4Weight.stack(w[4:6]), w[6]]
+    return out
+
+
+def gemm_launches(q4, gemms, m):
+    """Kernel launches of one step: one per GEMM, plus the reduction of those split along K."""
+    return sum(1 + (q4._lib.q4_linear_workspace_size(m, ctypes.byref(w.desc)) > 0) for w in gemms)
+
+
 def run_prefill(q4, args, weights, dev, m=2048):
     layers = decode_layers()
+    gemms = layer_gemms(q4, weights)
     xk = {k: dev_bf16(synth.activations((0, "llama1b-prefill-x", k), m, k, "outlier_channels"), dev)
           for k in sorted({k for (_, _, k) in layers})}
-    yn = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in sorted({n for (_, n, _) in layers})}
+    yn = {w.n: torch.empty((m, w.n), dtype=torch.bfloat16, device=dev) for w in gemms}
 
     def step():
-        for w, (_, n, k) in zip(weights, layers):
-            q4.q4_linear_w4a16(xk[k], w, y=yn[n])
+        for w in gemms:
+            q4.q4_linear_w4a16(xk[w.k], w, y=yn[w.n])
 
     g = graph_of(step)
     for _ in range(3):
@@ -450,25 +470,27 @@ def run_prefill(q4, args, weights, dev, m=2048):
     cl = clk.summary()
     pk, src = tensor_peak(peaks, cl)
     return {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 3), "m": m,
-            "workload": f"W4A16 GEMM over the 112 decode-step matrices at m={m}, x with 1% channels x10, bf16 out",
+            "workload": f"W4A16 GEMM over the 112 decode-step matrices at m={m} ([q,k,v] and [gate,up] each one "
+                        "GEMM over stacked weights: 64 GEMMs), x with 1% channels x10, bf16 out",
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk, "unit": "TFLOP/s",
                          "frac": round(tf / pk, 4), "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4),
                          "peak_source": src},
-            "gpu_launches": len(layers) * steps, "clocks": cl}
+            "gpu_launches": gemm_launches(q4, gemms, m) * steps, "clocks": cl}
 
 
 def run_w4a8(q4, args, weights_sym, dev, m=4096):
     layers = decode_layers()
     xk = {k: dev_bf16(synth.activations((0, "llama1b-w4a8-x", k), m, k, "student_t3"), dev)
           for k in sorted({k for (_, _, k) in layers})}
+    gemms = layer_gemms(q4, weights_sym)
     xq = {k: torch.empty((m, k), dtype=torch.int8, device=dev) for k in xk}
     sa = torch.empty((m,), dtype=torch.float32, device=dev)
-    yn = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in sorted({n for (_, n, _) in layers})}
+    yn = {w.n: torch.empty((m, w.n), dtype=torch.bfloat16, device=dev) for w in gemms}
 
     def step():
-        for w, (_, n, k) in zip(weights_sym, layers):
-            q4.act_quant_per_token(xk[k], xq=xq[k], scale_a=sa)
-            q4.q4_linear_w4a8(xq[k], sa, w, y=yn[n])
+        for w in gemms:   # one quantization of the GEMM's input, then the GEMM
+            q4.act_quant_per_token(xk[w.k], xq=xq[w.k], scale_a=sa)
+            q4.q4_linear_w4a8(xq[w.k], sa, w, y=yn[w.n])
 
     g = graph_of(step)
     for _ in range(3):
@@ -482,11 +504,12 @@ def run_w4a8(q4, args, weights_sym, dev, m=4096):
     cl = clk.summary()
     int8_peak, src = tensor_peak(peaks, cl, int8=True)
     return {"value": round(tops, 1), "unit": "TOPS", "ms_per_step": round(ms, 3), "m": m,
-            "workload": "per-token INT8 act-quant + W4A8 GEMM over the 112 matrices (symmetric INT4 g128), "
-                        f"m={m}, Student-t(3) activations, bf16 out; act-quant time included",
+            "workload": "per-token INT8 act-quant + W4A8 GEMM over the 112 matrices (symmetric INT4 g128; [q,k,v] "
+                        f"and [gate,up] each one GEMM over stacked weights: 64 GEMMs), m={m}, Student-t(3) "
+                        "activations, bf16 out; act-quant time included",
             "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
                          "frac": round(tops / int8_peak, 4), "peak_source": src},
-            "gpu_launches": 2 * len(layers) * steps, "clocks": cl}
+            "gpu_launches": (gemm_launches(q4, gemms, m) + len(gemms)) * steps, "clocks": cl}
 
 
 def with_attainable(r, m, a8: bool):

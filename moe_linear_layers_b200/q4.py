@@ -218,6 +218,20 @@ class Q4Weight:
                               zeros.data_ptr() if zeros is not None else None)
 
     @staticmethod
+    def stack(ws) -> "Q4Weight":
+        """The weights of several linears with the same k, group and symmetry stacked by rows (e.g. a layer's
+        q, k and v projections, which read the same input): y of the stack = the parts' outputs side by
+        side.  Quantization is per row and per group along k, so the stack's codes, scales and zero points
+        are exactly the parts' rows one after another (copied, no arithmetic)."""
+        ws = list(ws)
+        w0 = ws[0]
+        if any(w.k != w0.k or w.group != w0.group or w.symmetric != w0.symmetric for w in ws):
+            raise ValueError("stacked weights must share k, group and symmetry")
+        zeros = None if w0.symmetric else torch.cat([w.zeros for w in ws], 0).contiguous()
+        return Q4Weight(torch.cat([w.packed for w in ws], 0).contiguous(), torch.cat([w.scales for w in ws], 0).contiguous(),
+                        zeros, sum(w.n for w in ws), w0.k, w0.group, w0.symmetric)
+
+    @staticmethod
     def empty(n: int, k: int, group: int, symmetric: bool, device="cuda") -> "Q4Weight":
         packed = torch.empty((n, k // 2), dtype=torch.uint8, device=device)
         scales = torch.empty((n, k // group), dtype=torch.float16, device=device)

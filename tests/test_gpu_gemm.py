@@ -157,3 +157,32 @@ def test_w4a8_split_k_partials_bitexact(q4, m, n, k, group, sym):
     ref, acc_ref = oracle.linear_w4a8(xq, sa, pk, sc, n, k, group, want_acc=True, **kw)
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert_close(y.cpu().numpy(), ref, what="w4a8 split")
+
+
+def test_stacked_weights_equal_their_parts(q4):
+    """Q4Weight.stack: one GEMM over a layer's stacked projections (here q, k, v shaped, asymmetric g128)
+    gives each part's output in its column range: equal to the part's own GEMM up to the fp32 order of
+    its K sums, and to the oracle."""
+    m, k = 64, 1024
+    parts = []
+    for tag, n in (("q", 512), ("k", 128), ("v", 128)):
+        W = synth.weights(("test", "stack", tag, n, k), n, k)
+        pk, sc, zr = oracle.quantize(W, 128, False)
+        parts.append(((pk, sc, zr), upload_weight(q4, pk, sc, zr, n, k, 128, False), n))
+    st = q4.Q4Weight.stack([w for _, w, _ in parts])
+    assert st.n == 768 and st.k == k
+    x = synth.activations(("test", "stack-x", m, k), m, k)
+    xd = cuda_u16_as(x, torch.bfloat16)
+    ys = q4.q4_linear_w4a16(xd, st)
+    c0 = 0
+    for (pk, sc, zr), w, n in parts:
+        yp = q4.q4_linear_w4a16(xd, w)
+        torch.cuda.synchronize()
+        ref = oracle.linear_w4a16(x, pk, sc, zr, n, k, 128, False)
+        part = ys[:, c0:c0 + n].cpu().numpy()
+        assert_close(part, ref, what=f"stacked part at column {c0}")
+        d = np.abs(part - yp.cpu().numpy()).max() / np.sqrt(np.mean(ref * ref))
+        assert d < 1e-5, f"stacked and separate differ by {d} of rms"
+        c0 += n
+    with pytest.raises(ValueError):
+        q4.Q4Weight.stack([parts[0][1], q4.q4_quantize_pack(torch.zeros((64, 512), device="cuda"), 128, False)])
