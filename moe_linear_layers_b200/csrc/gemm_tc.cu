@@ -10,7 +10,7 @@ static int choose_splits(int32_t m, int32_t n, int32_t k, int sms, int* sps)
     const int kblocks = k / tcg::KBLK;
     *sps = kblocks;
     if (tiles < 1 || 2 * tiles > sms || kblocks < 4) return 1;
-    const int want = std::min(kblocks / 2, sms / tiles);
+    const int want = std::min(std::min(kblocks / 2, sms / tiles), 16);   // (the reduction takes at most 16)
     if (want < 2) return 1;
     *sps = (kblocks + want - 1) / want;
     return (kblocks + *sps - 1) / *sps;
@@ -23,13 +23,44 @@ size_t q4_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k)
     return splits < 2 ? 0 : (((size_t)splits * m * n * 4 + 255) & ~(size_t)255);
 }
 
-// y = the sum of the splits' partial sums, in split order (the same bits on every run)
+// y = the sum of the splits' partial sums, in split order (the same bits on every run).  Four values a
+// thread when m * n % 4 == 0 (16-byte loads; every split's load goes out before the sum), else one.
+constexpr int kMaxSplits = 16;
+
 __global__ void split_reduce_kernel(const float* __restrict__ part, int splits, int64_t mn, void* y, int out_bf16)
 {
     // launched as a programmatic dependent of the GEMM: the partials are read after its completion
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (mn % 4 == 0) {
+        const int64_t n4 = mn / 4;
+        const float4* p4 = reinterpret_cast<const float4*>(part);
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+            float4 v[kMaxSplits];
+#pragma unroll
+            for (int sp = 0; sp < kMaxSplits; sp++)
+                if (sp < splits) v[sp] = __ldg(p4 + (int64_t)sp * n4 + i);
+            float4 a = v[0];
+#pragma unroll
+            for (int sp = 1; sp < kMaxSplits; sp++)
+                if (sp < splits) {
+                    a.x += v[sp].x;
+                    a.y += v[sp].y;
+                    a.z += v[sp].z;
+                    a.w += v[sp].w;
+                }
+            if (out_bf16) {
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+                reinterpret_cast<uint2*>(y)[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                                            *reinterpret_cast<const uint32_t*>(&hi));
+            } else {
+                reinterpret_cast<float4*>(y)[i] = a;
+            }
+        }
+        return;
+    }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn; i += stride) {
         float v = part[i];
         for (int sp = 1; sp < splits; sp++) v += part[(int64_t)sp * mn + i];
         if (out_bf16) reinterpret_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
@@ -89,7 +120,8 @@ int q4_gemm_tc_launch(const void* x, const float* scale_a, int32_t m, const q4_w
     if (rc || p.splits == 1) return rc;
     const int64_t mn = (int64_t)m * w->n;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)std::min<int64_t>((mn + 255) / 256, 4 * sms));
+    const int64_t units = mn % 4 == 0 ? mn / 4 : mn;
+    cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((units + 255) / 256, 4 * sms)));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
