@@ -186,3 +186,38 @@ def test_stacked_weights_equal_their_parts(q4):
         c0 += n
     with pytest.raises(ValueError):
         q4.Q4Weight.stack([parts[0][1], q4.q4_quantize_pack(torch.zeros((64, 512), device="cuda"), 128, False)])
+
+
+@pytest.mark.parametrize("ws", ["auto", None])
+def test_dependent_launches_keep_their_order(q4, ws):
+    """The dense GEMM, its split-K reduction and the INT8 quantizer start early (programmatic dependent
+    launch) and wait only before reading what the previous kernel wrote.  Read after write: y2 = GEMM(y1)
+    right after y1 = GEMM(x) (bf16 y1).  Write after read: the quantizer overwrites the INT8 codes the
+    previous W4A8 GEMM reads; each result must still be the oracle's for its own input."""
+    m, k = 64, 1024
+    W1 = synth.weights(("test", "pdl", 1), k, k)
+    W2 = synth.weights(("test", "pdl", 2), k, k)
+    q1, q2 = oracle.quantize(W1, 128, False), oracle.quantize(W2, 128, False)
+    w1, w2 = upload_weight(q4, *q1, k, k, 128, False), upload_weight(q4, *q2, k, k, 128, False)
+    x = synth.activations(("test", "pdl-x", m, k), m, k)
+    y1 = q4.q4_linear_w4a16(cuda_u16_as(x, torch.bfloat16), w1, out_dtype=torch.bfloat16, workspace=ws)
+    y2 = q4.q4_linear_w4a16(y1, w2, workspace=ws)
+    torch.cuda.synchronize()
+    y1u = cpu_u16(y1).reshape(m, k)
+    assert_close(y1.float().cpu().numpy(), oracle.linear_w4a16(x, *q1, k, k, 128, False), what="first GEMM")
+    assert_close(y2.cpu().numpy(), oracle.linear_w4a16(y1u, *q2, k, k, 128, False), what="GEMM on its output")
+    # write after read through the quantizer and W4A8 (symmetric weights), one INT8 buffer for both inputs
+    qs = oracle.quantize(W1, 128, True)
+    ws8 = upload_weight(q4, qs[0], qs[1], None, k, k, 128, True)
+    xa = synth.activations(("test", "pdl-xa", m, k), m, k, "student_t3")
+    xb = synth.activations(("test", "pdl-xb", m, k), m, k, "student_t3")
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sa = torch.empty((m,), dtype=torch.float32, device="cuda")
+    q4.act_quant_per_token(cuda_u16_as(xa, torch.bfloat16), xq=xq, scale_a=sa)
+    ya = q4.q4_linear_w4a8(xq, sa, ws8, workspace=ws)
+    q4.act_quant_per_token(cuda_u16_as(xb, torch.bfloat16), xq=xq, scale_a=sa)
+    yb = q4.q4_linear_w4a8(xq, sa, ws8, workspace=ws)
+    torch.cuda.synchronize()
+    for xin, y, tag in ((xa, ya, "first"), (xb, yb, "second")):
+        xq_ref, sa_ref = oracle.act_quant(xin, k)
+        assert_close(y.cpu().numpy(), oracle.linear_w4a8(xq_ref, sa_ref, qs[0], qs[1], k, k, 128), what=f"{tag} W4A8")
