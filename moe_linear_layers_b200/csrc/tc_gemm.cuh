@@ -39,7 +39,7 @@
 //   warps 4-7    converters (TMEM lanes 32*(warp%4) ...); a build with Q4_CONV_SETS=2 adds warps 20-23 for
 //                the odd stages (measured slower on B200: 683 against 880 TFLOP/s, so one set is the default);
 //   warp 8       TMA producer (issues every copy, never waits on an mbarrier); warp 9 ring-slot watcher;
-//                warp 10 parameter loader; warp 11 idle;
+//                warp 10 parameter loader; warp 11 the MoE gate/up's h stores (else idle);
 //   warps 12-19  epilogue (two warps per TMEM lane quarter, each draining 64 of the 128 columns).
 // Measured on B200: one thread issues an M128 N128 K16 MMA only every ~120 cycles, half the tensor
 // pipe's rate, and any strong memory operation in that thread (an mbarrier wait included) stalls it
@@ -266,7 +266,7 @@ struct Shared {
     // per converter warp of each set, groups drained per epilogue warp, W4A8 accumulator preload done
     uint32_t conv_done[4 * kConvSets], epi_done[8], epi_init[8];
     uint32_t slot_free;             // ring stages released so far (published by the slot watcher)
-    uint64_t up_ready, gate_done;   // GateUp: gate/up hand-over written (all 8 epilogue warps), and consumed
+    uint64_t up_ready, gate_done;   // GateUp: gate/up hand-over written (8 epilogue warps); buffer free again (warp 11)
     uint64_t h_ready[2];            // GateUp: a half's h values are in the exchange buffer (its 4 warps)
     uint64_t p_full[2], p_empty[2]; // parameter ring: window staged (loader lanes), window consumed
     uint32_t tmem_base;
@@ -435,10 +435,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tc::mbar_init(&sh->p_full[i], 32);
             tc::mbar_init(&sh->p_empty[i], 4 * kConvSets + (INT8 ? 0 : 8));
         }
-        // GateUp exchange: every epilogue warp writes its half of the hand-over (up_ready) and consumes
-        // the other side's (gate_done)
+        // GateUp exchange: every epilogue warp writes its half of the hand-over (up_ready); warp 11 stores
+        // the h values and frees the buffer (gate_done)
         tc::mbar_init(&sh->up_ready, 8);
-        tc::mbar_init(&sh->gate_done, 8);
+        tc::mbar_init(&sh->gate_done, 1);
         tc::mbar_init(&sh->h_ready[0], 4);
         tc::mbar_init(&sh->h_ready[1], 4);
         sh->abort_flag = 0;
@@ -551,6 +551,52 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tc::mbar_wait(&sh->x_full[j % NS], (j / NS) & 1, p.status, nullptr, 100000000ull);
                 }
             }
+        } else if (MODE == Mode::GateUp && warp == 11) {
+            // -------------------------------------------------------------- h stores (warp 11, GateUp)
+            // Once both halves of a tile's h are in the exchange buffer, store them by token rows (lanes 0-15
+            // token j, lanes 16-31 token j + 1, each lane 4 consecutive intermediate indices: a row's 64 hi
+            // values, one 128-byte line, in one store and its 64 lo values in a second, or its 64 fp16
+            // values; intermediate index i = n0 + c: hi in block n0 / 64 of the row, lo 64 later, fp16 at
+            // column i of an [P][N] row), then free the buffer.  The epilogue warps meanwhile drain the next
+            // tile's groups.
+            const bool f16 = p.h_f16;
+            const int64_t hstride = f16 ? p.N : 2 * p.N;
+            const int c4 = 4 * (lane & 15);
+            uint32_t tl = 0;
+            for (int t = blockIdx.x; t < total; t += gridDim.x, tl++) {
+                const Tile T = map_tile<MODE>(t, p, sh, tiles_m);
+                for (int hf = 0; hf < 2; hf++) {
+                    if (!tc::mbar_wait(&sh->h_ready[hf], tl & 1, p.status, abort_flag)) goto hstore_done;
+                    const float* xb = xchg + hf * 64 * 64;
+                    const int mb = T.m0 + hf * 64;
+                    const int rows = min(64, T.m_end - mb);
+#pragma unroll 4
+                    for (int pr = 0; pr < 32; pr++) {
+                        const int j = 2 * pr + (lane >> 4);
+                        if (j >= rows) continue;
+                        const float4 hv = *reinterpret_cast<const float4*>(xb + j * 64 + c4);
+                        const int64_t o = (int64_t)(mb + j) * hstride + (f16 ? T.n0 : 2 * T.n0) + c4;
+                        if (!q4_in_bounds(o + (f16 ? 3 : 67), (int64_t)p.M * hstride, p.status)) continue;
+                        if (f16) {
+                            const __half2 a = __floats2half2_rn(hv.x, hv.y), b = __floats2half2_rn(hv.z, hv.w);
+                            *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.h) + o) =
+                                make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+                        } else {
+                            const __nv_bfloat162 h0 = __floats2bfloat162_rn(hv.x, hv.y), h1 = __floats2bfloat162_rn(hv.z, hv.w);
+                            const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+                            const __nv_bfloat162 l0 = __floats2bfloat162_rn(hv.x - f0.x, hv.y - f0.y);
+                            const __nv_bfloat162 l1 = __floats2bfloat162_rn(hv.z - f1.x, hv.w - f1.y);
+                            *reinterpret_cast<uint2*>(p.h + o) =
+                                make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+                            *reinterpret_cast<uint2*>(p.h + o + 64) =
+                                make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sh->gate_done);
+            }
+        hstore_done:;
         } else if (PRING && warp == 10) {
             // -------------------------------------------------------------- parameter loader (warp 10)
             // Stages each window of PW groups of the tile's scales (and zero points) in shared memory,
@@ -961,40 +1007,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 32; j++) silu_mul(j, accv(j), xb[j * 64 + ii]);
                 }
+                // the h values of this warp's tokens are in the buffer: warp 11 stores them by token rows
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sh->h_ready[half]);
-                if (!tc::mbar_wait(&sh->h_ready[half], tl & 1, p.status, abort_flag)) goto epi_done;
-                // Stores by token row: the 4 warps of this half take token pairs q, q + 4, ...; in a pair, lanes
-                // 0-15 write token j and lanes 16-31 token j + 1, each lane 4 consecutive intermediate indices:
-                // a row's 64 hi values (128 bytes) in one pass and its 64 lo values in a second, or its 64 fp16
-                // values (intermediate index i = n0 + ii: hi in block n0 / 64 of the row, lo 64 later; fp16 at
-                // column i of an [P][N] row)
-                const bool f16 = p.h_f16;
-                const int64_t hstride = f16 ? p.N : 2 * p.N;
-                const int q = ew & 3, c4 = 4 * (lane & 15);
-                for (int pr = q; pr < 32; pr += 4) {
-                    const int j = 2 * pr + (lane >> 4);
-                    if (j >= rows) continue;
-                    const float4 hv = *reinterpret_cast<const float4*>(xb + j * 64 + c4);
-                    const int64_t o = (int64_t)(mb + j) * hstride + (f16 ? T.n0 : 2 * T.n0) + c4;
-                    if (!q4_in_bounds(o + (f16 ? 3 : 67), (int64_t)p.M * hstride, p.status)) continue;
-                    if (f16) {
-                        const __half2 a = __floats2half2_rn(hv.x, hv.y), b = __floats2half2_rn(hv.z, hv.w);
-                        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.h) + o) =
-                            make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
-                    } else {
-                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(hv.x, hv.y), h1 = __floats2bfloat162_rn(hv.z, hv.w);
-                        const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
-                        const __nv_bfloat162 l0 = __floats2bfloat162_rn(hv.x - f0.x, hv.y - f0.y);
-                        const __nv_bfloat162 l1 = __floats2bfloat162_rn(hv.z - f1.x, hv.w - f1.y);
-                        *reinterpret_cast<uint2*>(p.h + o) =
-                            make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
-                        *reinterpret_cast<uint2*>(p.h + o + 64) =
-                            make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sh->gate_done);
             } else {
                 const int n = T.n0 + r;
                 float* yv = reinterpret_cast<float*>(p.y) + n;
