@@ -308,3 +308,23 @@ def test_linear_workspace_validation():
                                                P(ws) if ws else None, nb, None, None)
     assert call8(FAKE + 16, need) == q4.Q4_ERR_ALIGN
     assert call8(FAKE, need - 1) == q4.Q4_ERR_WORKSPACE
+
+
+def test_weight_stack_is_a_row_concatenation():
+    """Q4Weight.stack copies the parts' packed rows, scales and zero points one after another (CPU tensors:
+    no library call) and refuses parts of different k, group or symmetry."""
+    import torch
+    def part(n, k=256, group=128, sym=False, fill=0):
+        packed = torch.full((n, k // 2), fill, dtype=torch.uint8)
+        scales = torch.full((n, k // group), float(fill), dtype=torch.float16)
+        zeros = None if sym else torch.full((n, k // group), float(fill + 1), dtype=torch.float16)
+        return q4.Q4Weight(packed, scales, zeros, n, k, group, sym)
+    a, b, c = part(64, fill=1), part(16, fill=2), part(16, fill=3)
+    st = q4.Q4Weight.stack([a, b, c])
+    assert (st.n, st.k, st.group, st.symmetric) == (96, 256, 128, False)
+    assert torch.equal(st.packed[64:80], b.packed) and torch.equal(st.scales[80:], c.scales)
+    assert torch.equal(st.zeros[:64], a.zeros)
+    assert q4.Q4Weight.stack([part(8, sym=True), part(8, sym=True)]).zeros is None
+    for bad in (part(8, k=512), part(8, group=64), part(8, sym=True)):
+        with pytest.raises(ValueError):
+            q4.Q4Weight.stack([a, bad])
