@@ -69,3 +69,12 @@ def test_moe_hotness_tiers_cover_the_experts():
     assert tiers[0][0] == 0 and tiers[-1][1] == bench.MOE["E"]
     assert all(a[1] == b[0] for a, b in zip(tiers, tiers[1:]))
     assert [t[2] for t in tiers] == [32, 64, 128]          # hot, ordinary, cold
+
+
+def test_memory_footprint_closed_form():
+    """Every decode-step k is a multiple of 128, so per weight the INT4 layout holds half a byte of code
+    plus 2 (sym) or 4 (asym) bytes of fp16 scale and zero per 128 weights, against 2 bytes of fp16."""
+    f = bench.footprint(bench.decode_layers())
+    assert f["int4_asym_g128_bytes"] / f["fp16_bytes"] == (0.5 + 4 / 128) / 2 == 0.265625
+    assert f["int4_sym_g128_bytes"] / f["fp16_bytes"] == (0.5 + 2 / 128) / 2 == 0.2578125
+    assert f["ratio_asym_g128"] == 0.2656 and f["ratio_sym_g128"] == 0.2578
