@@ -41,7 +41,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        # Q4_ORACLE_LIB substitutes a library built from a modified copy of q4_oracle.c: the test that
+        # plants mistakes in the oracle checks that the pins reject each one
+        _lib = ctypes.CDLL(os.environ.get("Q4_ORACLE_LIB") or build())
         _lib.orc_f32_to_f16.restype = ctypes.c_uint16
         _lib.orc_f32_to_f16.argtypes = [ctypes.c_float]
         _lib.orc_f16_to_f32.restype = ctypes.c_float
