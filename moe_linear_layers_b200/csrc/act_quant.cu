@@ -194,10 +194,10 @@ template <bool F16>
 int act_quant_launch(const uint16_t* x, int32_t m, int32_t k, int8_t* xq, float* scale_a, int32_t* dev_status,
                      cudaStream_t s)
 {
-    if (!x || !xq || !scale_a) return Q4_ERR_NULL;
     if (m < 0 || k <= 0 || k % 8) return Q4_ERR_SHAPE;
+    if (m == 0) return Q4_OK;                 // no rows: x, xq, scale_a may be NULL
+    if (!x || !xq || !scale_a) return Q4_ERR_NULL;
     if (!q4_aligned16(x) || !q4_aligned16(xq) || ((uintptr_t)scale_a & 3u)) return Q4_ERR_ALIGN;
-    if (m == 0) return Q4_OK;
     const int n8 = k / 8;
     const int wgrid = (m + 7) / 8;
     if (n8 <= 32 * 2) return launch_pdl(act_quant_warp_kernel<2, F16>, wgrid, 256, s, x, m, k, xq, scale_a, dev_status);

@@ -90,12 +90,12 @@ extern "C" int q4_linear_w4a16_ws(const uint16_t* x, int32_t m, const q4_weight*
 {
     int rc = check_weight(w, false);
     if (rc) return rc;
-    if (!x || !y) return Q4_ERR_NULL;
     if (m < 0) return Q4_ERR_SHAPE;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (m == 0 || w->n == 0) return Q4_OK;   // an empty product reads and writes nothing: x, y may be NULL
+    if (!x || !y) return Q4_ERR_NULL;
     if (!q4_aligned16(x) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
     if ((rc = check_workspace(workspace, workspace_bytes, m, w))) return rc;
-    if (m == 0 || w->n == 0) return Q4_OK;
     if (m <= kMaxGemvM && w->k % 64 == 0) {
         void* ys[1] = {y};
         const int rc = q4_gemv_w4a16_launch_group(1, &x, m, w, ys, out_dtype, dev_status, (cudaStream_t)stream);
@@ -152,13 +152,13 @@ extern "C" int q4_linear_w4a8_ws(const int8_t* xq, const float* scale_a, int32_t
 {
     int rc = check_weight(w, false);
     if (rc) return rc;
-    if (!xq || !scale_a || !y) return Q4_ERR_NULL;
     if (m < 0) return Q4_ERR_SHAPE;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
+    if (m == 0 || w->n == 0) return Q4_OK;   // an empty product: xq, scale_a, y may be NULL
+    if (!xq || !scale_a || !y) return Q4_ERR_NULL;
     if (!q4_aligned16(xq) || !q4_aligned16(y) || ((uintptr_t)scale_a & 3u) || ((uintptr_t)acc_dbg & 3u))
         return Q4_ERR_ALIGN;
     if ((rc = check_workspace(workspace, workspace_bytes, m, w))) return rc;
-    if (m == 0 || w->n == 0) return Q4_OK;
     if (w->k % 128) return Q4_ERR_UNSUPPORTED;
     return q4_gemm_tc_launch(xq, scale_a, m, w, y, out_dtype, acc_dbg, true, dev_status, (cudaStream_t)stream,
                              workspace);

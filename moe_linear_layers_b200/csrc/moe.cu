@@ -617,7 +617,8 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
                         size_t workspace_bytes, int32_t* dev_status, void* stream, int n_classes,
                         const int32_t* class_begin, bool expert_range)
 {
-    if (!x || !router_w || !experts || !y || !workspace) return Q4_ERR_NULL;
+    // x and y hold T rows: with no tokens they may be NULL
+    if (!router_w || !experts || !workspace || (T > 0 && (!x || !y))) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
         return Q4_ERR_SHAPE;
     if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
@@ -671,7 +672,10 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
         return Q4_ERR_ALIGN;
     Workspace ws = carve(workspace, T, H, I, E, topk, I_shared, a8_mask);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
-    if (T == 0) return Q4_OK;
+    if (T == 0)   // no tokens: the optional routing outputs are empty ranges and zero counts
+        return ((offsets && cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream)) ||
+                (expert_counts && cudaMemsetAsync(expert_counts, 0, E * sizeof(int32_t), (cudaStream_t)stream)))
+                   ? Q4_ERR_CUDA : Q4_OK;
     if (topk_ids) ws.ids = topk_ids;
     if (topk_w) ws.wts = topk_w;
     if (perm) ws.perm = perm;
@@ -851,7 +855,8 @@ extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float
                             int32_t* expert_counts, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                             void* stream)
 {
-    if (!x || !router_w || !topk_ids || !topk_w || !offsets || !pair_pos || !workspace) return Q4_ERR_NULL;
+    // the per-token and per-pair arrays hold T and T*topk entries: with no tokens they may be NULL
+    if (!router_w || !offsets || !workspace || (T > 0 && (!x || !topk_ids || !topk_w || !pair_pos))) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E) return Q4_ERR_SHAPE;
     if (H % 128) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(x) || (x_perm && !q4_aligned16(x_perm)) || ((uintptr_t)workspace & 255u) ||
@@ -859,7 +864,10 @@ extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float
         return Q4_ERR_ALIGN;
     RouteWorkspace ws = carve_route(workspace, T, E, topk);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
-    if (T == 0) return cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream) ? Q4_ERR_CUDA : Q4_OK;
+    if (T == 0)   // no pairs: every expert's range is empty and its count 0
+        return (cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream) ||
+                (expert_counts && cudaMemsetAsync(expert_counts, 0, E * sizeof(int32_t), (cudaStream_t)stream)))
+                   ? Q4_ERR_CUDA : Q4_OK;
     if (perm) ws.perm = perm;
     if (expert_counts) ws.counts = expert_counts;
     cudaStream_t s = (cudaStream_t)stream;
@@ -895,7 +903,8 @@ extern "C" int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H,
                                    int32_t I, float* y_rows, void* workspace, size_t workspace_bytes,
                                    int32_t* dev_status, void* stream)
 {
-    if (!x_rows || !row_expert || !experts || !y_rows || !workspace) return Q4_ERR_NULL;
+    // the row arrays hold R entries: with no rows they may be NULL
+    if (!experts || !workspace || (R > 0 && (!x_rows || !row_expert || !y_rows))) return Q4_ERR_NULL;
     if (R < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts) return Q4_ERR_SHAPE;
     if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
     for (int i = 0; i < 3; i++) {
@@ -933,7 +942,8 @@ extern "C" int moe_q4_forward_rows(const uint16_t* x_rows, int32_t R, int32_t H,
 extern "C" int moe_q4_combine(const float* o_rows, int32_t P, int32_t H, const int32_t* pair_pos, const float* topk_w,
                               int32_t T, int32_t topk, void* y, int32_t out_dtype, int32_t* dev_status, void* stream)
 {
-    if (!o_rows || !pair_pos || !topk_w || !y) return Q4_ERR_NULL;
+    // with no tokens nothing is read or written and the arrays may be NULL
+    if (T > 0 && (!o_rows || !pair_pos || !topk_w || !y)) return Q4_ERR_NULL;
     if (T < 0 || P < 0 || H <= 0 || topk < 1 || topk > kMaxTopk || H % 4) return Q4_ERR_SHAPE;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(o_rows) || !q4_aligned16(y)) return Q4_ERR_ALIGN;

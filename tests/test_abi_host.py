@@ -328,3 +328,38 @@ def test_weight_stack_is_a_row_concatenation():
     for bad in (part(8, k=512), part(8, group=64), part(8, sym=True)):
         with pytest.raises(ValueError):
             q4.Q4Weight.stack([a, bad])
+
+
+def test_empty_problems_launch_nothing():
+    """A problem without rows is valid: its sizes, options and weights are still checked, then the call
+    returns Q4_OK without launching, and the arrays that hold no elements may be NULL (a zero-element
+    tensor has no storage).  No call below reaches the device: every pointer given is a placeholder."""
+    L = q4._lib
+    w = _w(n=128, k=256, group=64)
+    assert L.q4_linear_w4a16(None, 0, ctypes.byref(w), None, 0, None, None) == q4.Q4_OK
+    assert L.q4_linear_w4a16_ws(None, 0, ctypes.byref(w), None, 1, None, 0, None, None) == q4.Q4_OK
+    assert L.q4_linear_w4a8(None, None, 0, ctypes.byref(w), None, 0, None, None, None) == q4.Q4_OK
+    assert L.act_quant_per_token(None, 0, 128, None, None, None, None) == q4.Q4_OK
+    assert L.act_quant_per_token_f16(None, 0, 128, None, None, None, None) == q4.Q4_OK
+    # what an empty problem can still get wrong is still reported
+    assert L.q4_linear_w4a16(None, 0, ctypes.byref(_w(k=200)), None, 0, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_linear_w4a16(None, 0, ctypes.byref(w), None, 7, None, None) == q4.Q4_ERR_UNSUPPORTED
+    assert L.q4_linear_w4a16(None, -1, ctypes.byref(w), None, 0, None, None) == q4.Q4_ERR_SHAPE
+    assert L.act_quant_per_token(None, 0, 12, None, None, None, None) == q4.Q4_ERR_SHAPE
+    assert L.q4_linear_w4a16(None, 1, ctypes.byref(w), FAKE, 0, None, None) == q4.Q4_ERR_NULL   # one row needs x
+    # the MoE layer and its steps with no tokens / rows (no optional routing outputs: nothing to zero)
+    H, I, E, topk = 256, 128, 8, 2
+    ex = (q4.q4_weight * 3)(_w(n=E * I, k=H), _w(n=E * I, k=H), _w(n=E * H, k=I))
+    ws = L.moe_q4_workspace_size(0, H, I, E, topk)
+    assert L.moe_q4_forward(None, 0, H, FAKE, None, E, topk, ex, I, None, 0, None, None, None, None, None, FAKE, ws,
+                            None, None) == q4.Q4_OK
+    assert L.moe_q4_forward(None, 0, 200, FAKE, None, E, topk, ex, I, None, 0, None, None, None, None, None, FAKE,
+                            ws, None, None) == q4.Q4_ERR_UNSUPPORTED           # H % 128
+    assert L.moe_q4_forward(None, 0, H, None, None, E, topk, ex, I, None, 0, None, None, None, None, None, FAKE, ws,
+                            None, None) == q4.Q4_ERR_NULL                      # the router is still needed
+    assert L.moe_q4_forward(None, 1, H, FAKE, None, E, topk, ex, I, FAKE, 0, None, None, None, None, None, FAKE,
+                            L.moe_q4_workspace_size(1, H, I, E, topk), None, None) == q4.Q4_ERR_NULL
+    rws = L.moe_q4_rows_workspace_size(0, H, I, E)
+    assert L.moe_q4_forward_rows(None, 0, H, None, 0, None, E, ex, I, None, FAKE, rws, None, None) == q4.Q4_OK
+    assert L.moe_q4_combine(None, 0, H, None, None, 0, topk, None, 0, None, None) == q4.Q4_OK
+    assert L.moe_q4_combine(None, 0, H, None, None, 0, 0, None, 0, None, None) == q4.Q4_ERR_SHAPE   # topk 0
