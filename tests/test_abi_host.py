@@ -363,3 +363,26 @@ def test_empty_problems_launch_nothing():
     assert L.moe_q4_forward_rows(None, 0, H, None, 0, None, E, ex, I, None, FAKE, rws, None, None) == q4.Q4_OK
     assert L.moe_q4_combine(None, 0, H, None, None, 0, topk, None, 0, None, None) == q4.Q4_OK
     assert L.moe_q4_combine(None, 0, H, None, None, 0, 0, None, 0, None, None) == q4.Q4_ERR_SHAPE   # topk 0
+
+
+def test_size_limits_are_refused_before_any_launch():
+    """The largest problems a call takes: 256 experts and top-16 in the MoE layer (top-k <= E), k <= 16384
+    for the decode GEMV calls.  Beyond them the call reports the size and launches nothing (every case
+    here fails validation; none would reach the placeholder pointers)."""
+    L = q4._lib
+    T, H, I = 64, 256, 128
+
+    def moe(E, topk):
+        ex = (q4.q4_weight * 3)(_w(n=E * I, k=H), _w(n=E * I, k=H), _w(n=E * H, k=I))
+        return L.moe_q4_forward(FAKE, T, H, FAKE, None, E, topk, ex, I, FAKE, 0, None, None, None, None, None, FAKE,
+                                1 << 40, None, None)
+
+    assert moe(257, 8) == q4.Q4_ERR_SHAPE      # more experts than one launch holds
+    assert moe(64, 17) == q4.Q4_ERR_SHAPE      # top-k above 16
+    assert moe(4, 5) == q4.Q4_ERR_SHAPE        # top-k above the expert count
+    assert moe(4, 0) == q4.Q4_ERR_SHAPE
+    wide = _w(n=128, k=16384 + 64, group=64)
+    assert L.q4_linear_w4a16_swiglu(FAKE, FAKE, 1, ctypes.byref(wide), FAKE, 0, None, None) == q4.Q4_ERR_UNSUPPORTED
+    xs, ys = (ctypes.c_void_p * 1)(FAKE), (ctypes.c_void_p * 1)(FAKE)
+    assert L.q4_linear_w4a16_grouped(1, xs, 1, (q4.q4_weight * 1)(wide), ys, 0, None, None) == q4.Q4_ERR_UNSUPPORTED
+    assert L.q4_linear_w4a16_swiglu(FAKE, FAKE, 5, ctypes.byref(_w()), FAKE, 0, None, None) == q4.Q4_ERR_SHAPE  # m > 4
