@@ -135,6 +135,17 @@ def _stream(stream=None):
     return stream.cuda_stream
 
 
+def _hold(stream, *tensors):
+    """A call on a stream other than the current one: the caching allocator ties a tensor's memory to the
+    stream it was allocated on, so a workspace or output that this wrapper made (and that may be dropped
+    while the work is still queued) is marked in use by `stream` too, and is not handed out again before
+    that work is done."""
+    if stream is not None:
+        for t in tensors:
+            if t is not None:
+                t.record_stream(stream)
+
+
 def _dev(t, dtype, name):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -245,6 +256,7 @@ def q4_quantize_pack(w: torch.Tensor, group: int, symmetric: bool, dev_status: t
     _dev(w, torch.float32, "w")
     n, k = w.shape
     q = out or Q4Weight.empty(n, k, group, symmetric, device=w.device)
+    _hold(stream, q.packed, q.scales, q.zeros)
     _check(_lib.q4_quantize_pack(_ptr(w), n, k, group, int(bool(symmetric)), _ptr(q.packed), _ptr(q.scales),
                                  _ptr(q.zeros), _ptr(dev_status), _stream(stream)), "q4_quantize_pack")
     return q
@@ -280,6 +292,7 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
         workspace = linear_workspace(m, w, x.device) if m > q4_linear_w4a16_max_gemv_m() else None
     if workspace is not None:
         _workspace(workspace, x.device)
+    _hold(stream, y, workspace)
     _check(_lib.q4_linear_w4a16_ws(_ptr(x), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(workspace),
                                    workspace.numel() if workspace is not None else 0, _ptr(dev_status),
                                    _stream(stream)), "q4_linear_w4a16")
@@ -296,6 +309,7 @@ def q4_linear_w4a16_swiglu(gate: torch.Tensor, up: torch.Tensor, w: Q4Weight, ou
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=gate.device)
     od = _out(y, (m, w.n), gate.device)
+    _hold(stream, y)
     _check(_lib.q4_linear_w4a16_swiglu(_ptr(gate), _ptr(up), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(dev_status),
                                        _stream(stream)), "q4_linear_w4a16_swiglu")
     return y
@@ -406,6 +420,7 @@ def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a
     xq = torch.empty((m, k), dtype=torch.int8, device=x.device) if xq is None else xq
     scale_a = torch.empty((m,), dtype=torch.float32, device=x.device) if scale_a is None else scale_a
     fn = _lib.act_quant_per_token_f16 if f16 else _lib.act_quant_per_token
+    _hold(stream, xq, scale_a)
     _check(fn(_ptr(x), m, k, _ptr(xq), _ptr(scale_a), _ptr(dev_status), _stream(stream)),
            "act_quant_per_token_f16" if f16 else "act_quant_per_token")
     return xq, scale_a
@@ -426,6 +441,7 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
         workspace = linear_workspace(m, w, xq.device)
     if workspace is not None:
         _workspace(workspace, xq.device)
+    _hold(stream, y, workspace)
     _check(_lib.q4_linear_w4a8_ws(_ptr(xq), _ptr(scale_a), m, ctypes.byref(w.desc), _ptr(y), od, _ptr(acc_dbg),
                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                   _ptr(dev_status), _stream(stream)), "q4_linear_w4a8")
@@ -478,6 +494,7 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
         perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
         offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
         cnts = torch.empty((E,), dtype=torch.int32, device=dev)
+    _hold(stream, y, workspace, ids, wts, perm, offs, cnts)
     if a8_mask:
         _check(_lib.moe_q4_forward_a8(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, a8_mask,
                                       _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
@@ -523,6 +540,7 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
         perm = torch.empty((T * topk,), dtype=torch.int32, device=dev)
         offs = torch.empty((E + 1,), dtype=torch.int32, device=dev)
         cnts = torch.empty((E,), dtype=torch.int32, device=dev)
+    _hold(stream, y, workspace, ids, wts, perm, offs, cnts)
     _check(_lib.moe_q4_forward_classes(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, n, begin, descs,
                                        I, _ptr(y), od, _ptr(ids), _ptr(wts), _ptr(perm), _ptr(offs), _ptr(cnts),
                                        _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
@@ -550,6 +568,7 @@ def moe_q4_forward_range(x: torch.Tensor, router_w: torch.Tensor, router_bias: t
         workspace = torch.empty((max(moe_q4_workspace_size(T, H, I, E, topk), 1),), dtype=torch.uint8, device=x.device)
     _workspace(workspace, x.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _hold(stream, y, workspace)
     _check(_lib.moe_q4_forward_range(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, e_begin, e_end, descs,
                                      I, _ptr(y), None, None, None, None, None, _ptr(workspace), workspace.numel(),
                                      _ptr(dev_status), _stream(stream)), "moe_q4_forward_range")
@@ -592,6 +611,7 @@ def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias:
         y = torch.empty((T, H), dtype=out_dtype, device=x.device)
     od = _out(y, (T, H), x.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _hold(stream, y)
     _check(_lib.moe_q4_forward_noalloc(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, descs, I, _ptr(y),
                                        od, None, None, None, None, None, _ptr(dev_status), _stream(stream)),
            "moe_q4_forward_noalloc")
@@ -621,6 +641,7 @@ def moe_q4_route(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.Ten
            "x_perm": torch.empty((P, H), dtype=torch.bfloat16, device=dev),
            "row_expert": torch.empty((P,), dtype=torch.int32, device=dev)}
     ws = torch.empty((max(int(_lib.moe_q4_route_workspace_size(T, E, topk)), 1),), dtype=torch.uint8, device=dev)
+    _hold(stream, ws, *out.values())
     _check(_lib.moe_q4_route(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, topk, _ptr(out["topk_ids"]),
                              _ptr(out["topk_w"]), _ptr(out["offsets"]), _ptr(out["pair_pos"]), _ptr(out["x_perm"]),
                              _ptr(out["row_expert"]), None, None, _ptr(ws), ws.numel(), _ptr(dev_status),
@@ -651,6 +672,7 @@ def moe_q4_forward_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, e_base: 
                                 device=x_rows.device)
     _workspace(workspace, x_rows.device)
     descs = (q4_weight * 3)(*[e.desc for e in experts])
+    _hold(stream, y, workspace)
     _check(_lib.moe_q4_forward_rows(_ptr(x_rows), R, H, _ptr(row_expert), int(e_base), _ptr(row_weight), E, descs, I,
                                     _ptr(y), _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)),
            "moe_q4_forward_rows")
@@ -669,6 +691,7 @@ def moe_q4_combine(o_rows: torch.Tensor, pair_pos: torch.Tensor, topk_w: torch.T
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=o_rows.device)
     od = _out(y, (T, H), o_rows.device)
+    _hold(stream, y)
     _check(_lib.moe_q4_combine(_ptr(o_rows), P, H, _ptr(pair_pos), _ptr(topk_w), T, topk, _ptr(y), od,
                                _ptr(dev_status), _stream(stream)), "moe_q4_combine")
     return y

@@ -386,3 +386,21 @@ def test_size_limits_are_refused_before_any_launch():
     xs, ys = (ctypes.c_void_p * 1)(FAKE), (ctypes.c_void_p * 1)(FAKE)
     assert L.q4_linear_w4a16_grouped(1, xs, 1, (q4.q4_weight * 1)(wide), ys, 0, None, None) == q4.Q4_ERR_UNSUPPORTED
     assert L.q4_linear_w4a16_swiglu(FAKE, FAKE, 5, ctypes.byref(_w()), FAKE, 0, None, None) == q4.Q4_ERR_SHAPE  # m > 4
+
+
+def test_wrapper_tensors_are_held_for_the_callers_stream():
+    """A call given a stream marks the tensors its wrapper made as in use by that stream (the allocator
+    would otherwise hand their memory out again while the work there is queued); without a stream the
+    current stream orders everything and nothing is marked."""
+    class T:
+        def __init__(self):
+            self.streams = []
+
+        def record_stream(self, s):
+            self.streams.append(s)
+
+    a, b = T(), T()
+    q4._hold(None, a, b)
+    assert a.streams == [] and b.streams == []
+    q4._hold("side", a, None, b)
+    assert a.streams == ["side"] and b.streams == ["side"]
