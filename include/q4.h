@@ -120,9 +120,9 @@ int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t group, int32_
  * Source: the W4A8 page §2.1 (4-bit storage restored to a 16-bit compute type) and §1 (small batch:
  * memory bound; larger batch: compute bound).
  * x [m][k] bf16; y [m][n] fp32 (out_dtype Q4_OUT_F32) or bf16 (Q4_OUT_BF16, round to nearest even of
- * the fp32 result).  m >= 1.  Small m runs the memory-bound GEMV kernel (CUDA cores, in-register
- * dequant); larger m runs the tcgen05 tensor-core GEMM (exact integer codes in bf16, fp32
- * accumulation per group, scale applied per group in the epilogue).  The choice is by shape only.
+ * the fp32 result).  m >= 0 (m = 0 launches nothing).  Small m runs the memory-bound GEMV kernel
+ * (CUDA cores, in-register dequant); larger m runs the tcgen05 tensor-core GEMM (exact integer codes
+ * in bf16, fp32 accumulation per group, scale applied per group in the epilogue).  The choice is by shape only.
  * The GEMV serves k % 64 == 0, k <= 16384; the GEMM serves k % 128 == 0 (see q4_linear_w4a16_max_gemv_m).
  * Both kernels may start, and read W (packed, scales, zeros) into shared memory, TMEM and L2, before the
  * previous kernel on the stream has finished (programmatic dependent launch); they read x and write y
@@ -291,7 +291,8 @@ size_t moe_q4_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t
  * fp32, perm [T*topk] int32 (value t*topk+j), offsets [E+1] int32, expert_counts [E] int32.
  * workspace: device memory of at least moe_q4_workspace_size(T, H, I, E, topk) bytes, 256-byte
  * aligned, owned by the caller; contents on entry are ignored.
- * Limits: E <= 256, topk <= 16, H % 128 == 0, I % 128 == 0.
+ * Limits: E <= 256, topk <= 16, T * topk <= 2^31 - 1 (pair positions are int32), H % 128 == 0,
+ * I % 128 == 0.
  */
 int moe_q4_forward(const uint16_t* x, int32_t T, int32_t H,
                    const float* router_w, const float* router_bias, int32_t E, int32_t topk,
@@ -402,7 +403,7 @@ int moe_q4_forward_range(const uint16_t* x, int32_t T, int32_t H,
  *   in permuted order: the dispatch buffer, whose rows for the experts e0 .. e1-1 are one contiguous block),
  *   row_expert [T*topk] int32 (the expert of each permuted row), perm [T*topk] int32 (value t*topk + j),
  *   expert_counts [E].  workspace: moe_q4_route_workspace_size(T, E, topk) bytes, 256-byte aligned.
- *   Limits as moe_q4_forward (E <= 256, topk <= 16, H % 128 == 0).
+ *   Limits as moe_q4_forward (E <= 256, topk <= 16, T * topk <= 2^31 - 1, H % 128 == 0).
  */
 size_t moe_q4_route_workspace_size(int32_t T, int32_t E, int32_t topk);
 int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float* router_w, const float* router_bias,

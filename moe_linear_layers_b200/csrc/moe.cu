@@ -28,6 +28,8 @@ constexpr int kRouteTok = 16;           // tokens per route CTA (= one histogram
 constexpr int kRouteWarps = 8;
 constexpr int kRouteKC = 64;            // K columns staged per step
 constexpr int kMaxTopk = 16;
+// (token, slot) pairs of one call: their positions t * topk + j are int32
+constexpr int64_t kMaxPairs = INT32_MAX;
 
 // ---------------------------------------------------------------------------------------------- //
 // 1. route
@@ -621,6 +623,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
     if (!router_w || !experts || !workspace || (T > 0 && (!x || !y))) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E)
         return Q4_ERR_SHAPE;
+    if ((int64_t)T * topk > kMaxPairs) return Q4_ERR_SHAPE;
     if (H % 128 || I % 128) return Q4_ERR_UNSUPPORTED;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     // expert classes: experts [begin[c], begin[c+1]) share one stacked weight triple (one class = all)
@@ -858,6 +861,7 @@ extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float
     // the per-token and per-pair arrays hold T and T*topk entries: with no tokens they may be NULL
     if (!router_w || !offsets || !workspace || (T > 0 && (!x || !topk_ids || !topk_w || !pair_pos))) return Q4_ERR_NULL;
     if (T < 0 || H <= 0 || E < 1 || E > tcg::kMaxExperts || topk < 1 || topk > kMaxTopk || topk > E) return Q4_ERR_SHAPE;
+    if ((int64_t)T * topk > kMaxPairs) return Q4_ERR_SHAPE;
     if (H % 128) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(x) || (x_perm && !q4_aligned16(x_perm)) || ((uintptr_t)workspace & 255u) ||
         ((uintptr_t)router_w & 15u))
@@ -944,7 +948,8 @@ extern "C" int moe_q4_combine(const float* o_rows, int32_t P, int32_t H, const i
 {
     // with no tokens nothing is read or written and the arrays may be NULL
     if (T > 0 && (!o_rows || !pair_pos || !topk_w || !y)) return Q4_ERR_NULL;
-    if (T < 0 || P < 0 || H <= 0 || topk < 1 || topk > kMaxTopk || H % 4) return Q4_ERR_SHAPE;
+    if (T < 0 || P < 0 || H <= 0 || topk < 1 || topk > kMaxTopk || H % 4 || (int64_t)T * topk > kMaxPairs)
+        return Q4_ERR_SHAPE;
     if (out_dtype != Q4_OUT_F32 && out_dtype != Q4_OUT_BF16) return Q4_ERR_UNSUPPORTED;
     if (!q4_aligned16(o_rows) || !q4_aligned16(y)) return Q4_ERR_ALIGN;
     if (T == 0) return Q4_OK;

@@ -404,3 +404,17 @@ def test_wrapper_tensors_are_held_for_the_callers_stream():
     assert a.streams == [] and b.streams == []
     q4._hold("side", a, None, b)
     assert a.streams == ["side"] and b.streams == ["side"]
+
+
+def test_pair_positions_fit_int32():
+    """Positions of (token, slot) pairs are int32: a call with T * topk above 2^31 - 1 is refused before
+    anything is launched (a route workspace of 12 bytes per pair and the tokens themselves would still fit
+    in a B200's memory at 2^28 tokens of hidden 128)."""
+    L = q4._lib
+    T, H, E, topk = 1 << 28, 128, 16, 16
+    assert L.moe_q4_route(FAKE, T, H, FAKE, None, E, topk, FAKE, FAKE, FAKE, FAKE, None, None, None, None, FAKE,
+                          1 << 40, None, None) == q4.Q4_ERR_SHAPE
+    assert L.moe_q4_combine(FAKE, 0, H, FAKE, FAKE, T, topk, FAKE, 0, None, None) == q4.Q4_ERR_SHAPE
+    ex = (q4.q4_weight * 3)(_w(n=E * 128, k=H), _w(n=E * 128, k=H), _w(n=E * H, k=128))
+    assert L.moe_q4_forward(FAKE, T, H, FAKE, None, E, topk, ex, 128, FAKE, 0, None, None, None, None, None, FAKE,
+                            1 << 40, None, None) == q4.Q4_ERR_SHAPE
