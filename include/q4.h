@@ -29,11 +29,12 @@
  *     they detect a problem in the data: Q4_ERR_NONFINITE for a non-finite input group/row,
  *     Q4_ERR_TIMEOUT when a bounded wait inside a kernel ran out.  The library never clears it;
  *     the caller zeroes it and reads it when convenient.  Outputs are undefined when it is set.
- *   - A problem without rows (m = 0 in the linear and activation calls, T = 0 tokens, R = 0 rows) is
- *     valid: the call checks its sizes, options and weights, zeroes the expert offsets and counts it
- *     is given, and launches nothing else.  Pointers to arrays that then hold no elements (x, y, the
- *     per-token and per-row arrays) may be NULL.  The decode GEMV calls (q4_linear_w4a16_grouped,
- *     q4_linear_w4a16_swiglu, q4_linear_w4a16_chain) take 1 <= m <= 4.
+ *   - A problem without rows (m = 0 in the linear and activation calls, n = 0 in the quantizer,
+ *     T = 0 tokens, R = 0 rows) is valid: the call checks its sizes, options and weights, zeroes the
+ *     expert offsets and counts it is given, and launches nothing else.  Pointers to arrays that then
+ *     hold no elements (x, y, the per-token and per-row arrays, the quantizer's four) may be NULL.
+ *     The decode GEMV calls (q4_linear_w4a16_grouped, q4_linear_w4a16_swiglu, q4_linear_w4a16_chain)
+ *     take 1 <= m <= 4.
  *   - fp16 and bf16 values are passed as their 16-bit patterns (uint16_t).
  *   - Matrices are row-major.
  *

@@ -92,11 +92,11 @@ extern "C" int q4_quantize_pack(const float* w, int32_t n, int32_t k, int32_t gr
                                 uint8_t* packed, uint16_t* scales, uint16_t* zeros, int32_t* dev_status,
                                 void* stream)
 {
-    if (!w || !packed || !scales || (!symmetric && !zeros)) return Q4_ERR_NULL;
     if (n < 0 || k <= 0 || (group != 32 && group != 64 && group != 128 && group != 256) || k % group) return Q4_ERR_SHAPE;
+    if (n == 0) return Q4_OK;   // no rows: the four arrays hold nothing and may be NULL
+    if (!w || !packed || !scales || (!symmetric && !zeros)) return Q4_ERR_NULL;
     if (!q4_aligned16(w) || !q4_aligned16(packed) || !q4_aligned16(scales) || (!symmetric && !q4_aligned16(zeros)))
         return Q4_ERR_ALIGN;
-    if (n == 0) return Q4_OK;
     const int64_t total8 = (int64_t)n * k / 8;
     const int64_t warps = (total8 + 31) / 32;
     const int64_t blocks = std::min<int64_t>((warps + 7) / 8, (int64_t)q4_num_sms() * 16);

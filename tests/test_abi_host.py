@@ -341,6 +341,8 @@ def test_empty_problems_launch_nothing():
     assert L.q4_linear_w4a8(None, None, 0, ctypes.byref(w), None, 0, None, None, None) == q4.Q4_OK
     assert L.act_quant_per_token(None, 0, 128, None, None, None, None) == q4.Q4_OK
     assert L.act_quant_per_token_f16(None, 0, 128, None, None, None, None) == q4.Q4_OK
+    assert L.q4_quantize_pack(None, 0, 128, 64, 0, None, None, None, None, None) == q4.Q4_OK
+    assert L.q4_quantize_pack(None, 0, 100, 64, 0, None, None, None, None, None) == q4.Q4_ERR_SHAPE
     # what an empty problem can still get wrong is still reported
     assert L.q4_linear_w4a16(None, 0, ctypes.byref(_w(k=200)), None, 0, None, None) == q4.Q4_ERR_SHAPE
     assert L.q4_linear_w4a16(None, 0, ctypes.byref(w), None, 7, None, None) == q4.Q4_ERR_UNSUPPORTED
