@@ -113,6 +113,24 @@ MUTANTS = [
     ("a8: combine weight dropped", "int orc_moe_experts_a8(", "yr[c] += wj * o;", "yr[c] += o;"),
     ("a8: zero point added in the INT8 dot", "static double w4a8_dot(",
      "((int32_t)code_at(packed, k, r, kk, symmetric) - z)", "((int32_t)code_at(packed, k, r, kk, symmetric) + z)"),
+    ("a8: down projection's activation scale dropped", "int orc_moe_experts_a8(",
+     "o = w4a8_dot(hq, sh, dp, ds, dz, symmetric, I, group, c);", "o = w4a8_dot(hq, 1.0, dp, ds, dz, symmetric, I, group, c);"),
+    ("a8: gate codes rescaled by the up matrix's scales", "int orc_moe_experts_a8(",
+     "gv = w4a8_dot(xq, sa, gp, gs, gz, symmetric, H, group, i);", "gv = w4a8_dot(xq, sa, gp, us, gz, symmetric, H, group, i);"),
+    ("router: top-k takes the smallest logits", "int orc_route(", "l[e] > l[best]", "l[e] < l[best]"),
+    ("two's complement by 8 instead of 16", "static int code_at(", "if (symmetric && v >= 8) v -= 16;",
+     "if (symmetric && v >= 8) v -= 8;"),
+    ("symmetric codes truncated, not rounded", "int orc_quantize(",
+     "(int)clampf(rne(src[i] / S), -8.0f, 7.0f)", "(int)clampf(truncf(src[i] / S), -8.0f, 7.0f)"),
+    ("W4A8: symmetric codes read as unsigned", "void orc_linear_w4a8(",
+     "((int32_t)code_at(packed, k, r, kk, symmetric) - z)", "((int32_t)code_at(packed, k, r, kk, 0) - z)"),
+    ("bf16 widening shifted by 15", "float orc_bf16_to_f32(uint16_t b)", "(uint32_t)b << 16", "(uint32_t)b << 15"),
+    ("act quant: amax over the first half of the row", "static float act_quant_row(",
+     "for (int kk = 0; kk < k; kk++) {\n        if (!isfinite(v[kk])) *bad = 1;",
+     "for (int kk = 0; kk < k / 2; kk++) {\n        if (!isfinite(v[kk])) *bad = 1;"),
+    ("MoE: the last chosen expert left out", "void orc_moe_experts(",
+     "for (int j = 0; j < topk; j++) {\n            int e = ids[(size_t)t * topk + j];\n            /* the expert's row blocks",
+     "for (int j = 0; j < topk - 1; j++) {\n            int e = ids[(size_t)t * topk + j];\n            /* the expert's row blocks"),
 ]
 
 
