@@ -11,10 +11,11 @@
 // activation rows (the MMA's N), D_g = sum_{k in g} (code - zero)[row][k] * act[m][k] exactly (integer
 // codes are exact in bf16 / fp16 / int8) one quantization group at a time, and the epilogue
 // accumulates s[row][g] * D_g in fp32.  Group accumulators rotate through two TMEM buffers (three for
-// W4A8) so the MMAs of the next groups overlap the epilogue's drain of group g.
+// W4A8 and for the hi/lo down projection) so the MMAs of the next groups overlap the epilogue's drain
+// of group g.
 //
 // Data flow: TMA brings the packed nibbles (64-byte swizzle) and the activation tile (128-byte
-// swizzle, K-major, the MMA's B operand) into a 4-stage shared-memory ring.  Converter warps widen the
+// swizzle, K-major, the MMA's B operand) into a shared-memory ring of 3 to 8 stages (Cfg::NS, by mode).  Converter warps widen the
 // nibbles in registers and write them into TMEM with tcgen05.st (the MMA's A operand), so widened
 // weights never use shared-memory bandwidth.  Four threads in four warps issue tcgen05.mma for
 // alternate K stages and commit to mbarriers.
@@ -46,8 +47,9 @@
 // until its MMAs have retired; four issuer threads in different warps that only poll progress counters
 // with weak loads keep the pipe at one MMA per 64 cycles, commits included.  A thread that waits on an
 // mbarrier also stalls until its own bulk copies have landed, so the thread that issues the TMA copies
-// polls a counter that another thread publishes after the mbarrier wait.  Persistent CTAs walk tiles with a stride of gridDim.x; the rings carry their
-// phases across tiles.  Every wait is bounded (Q4_ERR_TIMEOUT, then a clean exit).
+// polls a counter that another thread publishes after the mbarrier wait.  Persistent CTAs walk tiles
+// with a stride of gridDim.x; the rings carry their phases across tiles.  Every wait is bounded
+// (Q4_ERR_TIMEOUT, then a clean exit).
 //
 // Epilogue arithmetic runs on packed fp32 pairs (FFMA2).  For W4A8 every int32 accumulator is preloaded
 // with the bit pattern of 1.5 * 2^23, so the accumulated bits are the float 1.5 * 2^23 + acc and one
