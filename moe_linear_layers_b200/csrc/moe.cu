@@ -399,6 +399,16 @@ __global__ void moe_shared_setup_kernel(int T, int H, int I_s, int32_t* __restri
     }
 }
 
+// The routing outputs of a call without tokens: offsets [E + 1] and counts [E] all 0 (each nullable).
+int zero_routing(int32_t* offsets, int32_t* counts, int E, cudaStream_t s)
+{
+    if (offsets)
+        if (const cudaError_t e = cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s)) return q4_cuda_status(e);
+    if (counts)
+        if (const cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s)) return q4_cuda_status(e);
+    return Q4_OK;
+}
+
 Workspace carve(void* base, int T, int H, int I, int E, int topk, int I_s = 0, int a8_mask = 0)
 {
     Workspace w = {};
@@ -676,9 +686,7 @@ static int forward_impl(const uint16_t* x, int32_t T, int32_t H, const float* ro
     Workspace ws = carve(workspace, T, H, I, E, topk, I_shared, a8_mask);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
     if (T == 0)   // no tokens: the optional routing outputs are empty ranges and zero counts
-        return ((offsets && cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream)) ||
-                (expert_counts && cudaMemsetAsync(expert_counts, 0, E * sizeof(int32_t), (cudaStream_t)stream)))
-                   ? Q4_ERR_CUDA : Q4_OK;
+        return zero_routing(offsets, expert_counts, E, (cudaStream_t)stream);
     if (topk_ids) ws.ids = topk_ids;
     if (topk_w) ws.wts = topk_w;
     if (perm) ws.perm = perm;
@@ -869,9 +877,7 @@ extern "C" int moe_q4_route(const uint16_t* x, int32_t T, int32_t H, const float
     RouteWorkspace ws = carve_route(workspace, T, E, topk);
     if (workspace_bytes < ws.bytes) return Q4_ERR_WORKSPACE;
     if (T == 0)   // no pairs: every expert's range is empty and its count 0
-        return (cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), (cudaStream_t)stream) ||
-                (expert_counts && cudaMemsetAsync(expert_counts, 0, E * sizeof(int32_t), (cudaStream_t)stream)))
-                   ? Q4_ERR_CUDA : Q4_OK;
+        return zero_routing(offsets, expert_counts, E, (cudaStream_t)stream);
     if (perm) ws.perm = perm;
     if (expert_counts) ws.counts = expert_counts;
     cudaStream_t s = (cudaStream_t)stream;
