@@ -10,6 +10,8 @@ import re
 import subprocess
 import sys
 
+import numpy as np
+
 import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -176,3 +178,84 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
             (survivors if rc == 0 else crashed).append((name, rc, out[-400:]))
     assert not crashed, f"mutants that did not run to a pin failure: {crashed}"
     assert not survivors, f"mistakes no pin catches: {[s[0] for s in survivors]}"
+
+
+# The compositions the oracle does in numpy (oracle/__init__.py): each replaced, in this process, by a
+# plausible wrong version; the pins that cover it must fail.  (Only mistakes that stay inside the arrays:
+# the C functions they call are not bounds-checked.)
+def _silu_wrong_sign(g, u):
+    g = np.asarray(g, np.float32).astype(np.float64)
+    return g / (1.0 + np.exp(g)) * np.asarray(u, np.float32).astype(np.float64)
+
+
+def _sigmoid_not_silu(g, u):
+    g = np.asarray(g, np.float32).astype(np.float64)
+    return 1.0 / (1.0 + np.exp(-g)) * np.asarray(u, np.float32).astype(np.float64)
+
+
+def _silu_in_fp32(g, u):
+    g, u = np.asarray(g, np.float32), np.asarray(u, np.float32)
+    return (g / (np.float32(1.0) + np.exp(-g)) * u).astype(np.float64)
+
+
+def _swiglu_gate_only(gate, up, packed, scales, zeros, n, k, group, symmetric):
+    h = _REAL["silu_mul"](gate, np.ones_like(np.asarray(up, np.float32))).reshape(-1, k)
+    return h @ oracle.dequant(packed, scales, zeros, k, group, symmetric).astype(np.float64).T
+
+
+def _swiglu_untransposed(gate, up, packed, scales, zeros, n, k, group, symmetric):
+    h = _REAL["silu_mul"](gate, up).reshape(-1, k)
+    return h @ oracle.dequant(packed, scales, zeros, k, group, symmetric).astype(np.float64)
+
+
+def _shared_half_weight(x, H, gate, up, down, I_s, group, symmetric, tokens=None):
+    return 0.5 * _REAL["shared_expert"](x, H, gate, up, down, I_s, group, symmetric, tokens=tokens)
+
+
+def _classes_foreign_slots_kept(x, H, ids, w, class_begin, classes, I, tokens=None):
+    ids = np.asarray(ids, np.int32)
+    y = None
+    for c, (gate, up, down, group, symmetric) in enumerate(classes):
+        e0, e1 = int(class_begin[c]), int(class_begin[c + 1])
+        mine = (ids >= e0) & (ids < e1)
+        ids_c = np.where(mine, ids - e0, 0).astype(np.int32)
+        yc = oracle.moe_experts(x, H, ids_c, np.asarray(w, np.float64), gate, up, down, I, group, symmetric,
+                                tokens=tokens)
+        y = yc if y is None else y + yc
+    return y
+
+
+_REAL = {name: getattr(oracle, name) for name in ("silu_mul", "shared_expert")}
+
+
+def test_every_planted_mistake_in_the_numpy_compositions_fails_a_pin(monkeypatch):
+    from tests import test_oracle_pins as pins
+    swiglu_pins = [pins.test_silu_mul_identities, pins.test_swiglu_linear_reduces_to_plain_linear_for_saturated_gate]
+    class_pins = [pins.test_moe_classes_one_class_and_equal_classes_are_the_layer,
+                  pins.test_moe_classes_each_expert_uses_its_class_quantization]
+    cases = [
+        ("silu_mul", _silu_wrong_sign, swiglu_pins),
+        ("silu_mul", _sigmoid_not_silu, swiglu_pins),
+        ("silu_mul", _silu_in_fp32, swiglu_pins),
+        ("linear_w4a16_swiglu", _swiglu_gate_only, swiglu_pins),
+        ("linear_w4a16_swiglu", _swiglu_untransposed, swiglu_pins),
+        ("shared_expert", _shared_half_weight, [pins.test_shared_expert_is_the_dense_swiglu_ffn]),
+        ("moe_experts_classes", _classes_foreign_slots_kept, class_pins),
+    ]
+    for _, _, checks in cases:          # the real compositions pass their pins
+        for check in checks:
+            check()
+    survivors = []
+    for name, wrong, checks in cases:
+        monkeypatch.setattr(oracle, name, wrong)
+        caught = False
+        for check in checks:
+            try:
+                check()
+            except Exception:
+                caught = True
+                break
+        monkeypatch.undo()
+        if not caught:
+            survivors.append(f"{name}: {wrong.__name__}")
+    assert not survivors, f"mistakes no pin catches: {survivors}"
