@@ -1,4 +1,6 @@
-"""The 16-bit expert path carries the SwiGLU intermediate h as two bf16 values, hi = bf16(h) and
+"""Arithmetic facts the kernels rely on, checked on the CPU.
+
+The 16-bit expert path carries the SwiGLU intermediate h as two bf16 values, hi = bf16(h) and
 lo = bf16(h - hi), both rounded to nearest even.  bf16 keeps 8 significant bits, so hi is within half a
 bf16 ulp (at most 2^-8 relative) of h, the difference h - hi is exact in fp32, and lo is within 2^-8 of
 it: hi + lo is within 2^-16 |h| of h (about 2^-17 at worst in practice, as both worst cases rarely meet),
@@ -39,3 +41,20 @@ def test_hi_lo_pair_holds_h_to_2_pow_minus_16():
     assert np.max(rel) < 1.05 * 2.0 ** -17       # the figure quoted for the pair
     # a single bf16 is off by up to 2^-8 |h|: the second half is what meets the bar
     assert np.max(np.abs(hi - h) / np.abs(h)) > 2.0 ** -9
+
+
+def test_w4a8_accumulator_preload_is_exact_for_every_group_sum():
+    """The W4A8 epilogue preloads each int32 accumulator with the bits of 1.5 * 2^23; after the integer
+    MMAs add acc, the bits read as the float 1.5 * 2^23 + acc exactly while 1.5 * 2^23 + acc stays in
+    [2^23, 2^24), i.e. |acc| < 2^22, and one subtraction recovers acc.  The largest group sum W4A8 forms
+    (group 128, |activation code| <= 128, |16 * weight code| <= 128 on the symmetric path, |code - zero|
+    <= 15 on the asymmetric one) is 128 * 128 * 128 = 2^21."""
+    bias_bits, bias = 0x4B400000, 1.5 * 2.0 ** 23
+    acc = np.concatenate([np.arange(-(1 << 21), (1 << 21) + 1, 997), [-(1 << 21), (1 << 21), -1, 0, 1]]).astype(np.int64)
+    bits = (bias_bits + acc).astype(np.uint32)
+    got = bits.view(np.float32).astype(np.float64) - bias
+    assert np.array_equal(got, acc.astype(np.float64))
+    assert 128 * 128 * 128 == 1 << 21 and 128 * (16 * 8) * 128 == 1 << 21 and 128 * 15 * 128 < 1 << 21
+    # past 2^22 the sum leaves the binade and the identity fails: the bound is the real limit
+    over = np.array([bias_bits + (1 << 22) + 1], np.int64).astype(np.uint32).view(np.float32).astype(np.float64)
+    assert over[0] - bias != (1 << 22) + 1
