@@ -395,6 +395,7 @@ class GemvChain:
         self.sync.zero_()
 
     def __call__(self, dev_status: torch.Tensor | None = None, stream=None):
+        _hold(stream, self.sync)
         _check(_lib.q4_linear_w4a16_chain(self.n_stages, self.begin, self.x, self.g, self.u, self.w, self.y, self.od,
                                           _ptr(self.sync), _ptr(dev_status), _stream(stream)), "q4_linear_w4a16_chain")
 
