@@ -15,7 +15,8 @@ def _declared_functions():
     names = []
     for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
         if fn.endswith(".h"):
-            src = open(os.path.join(ROOT, "include", fn)).read()
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                src = f.read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
             names += re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(\w+)\s*\(", src, flags=re.M)
     return names

@@ -75,7 +75,7 @@ def test_expert_parallel_sum_equals_the_layer_on_gloo_ranks():
     _, ids, w, _ = oracle.route(x, H, Wr, bias, TOPK)
     ref = oracle.moe_experts(x, H, ids, w, stack[0], stack[1], stack[2], I, GROUP, SYM)
     for world in (2, 3):
-        out = mp.Manager().dict()
+        out = mp.get_context("spawn").Manager().dict()   # no fork of this threaded process
         mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
         for r in range(world):
             e0, e1, y = out[r]

@@ -105,7 +105,7 @@ def _worker(rank, world, port, out):
 def test_expert_parallel_all_to_all_on_gloo_ranks():
     Wr, bias, stack = _layer()
     for world in (2, 3):
-        out = mp.Manager().dict()
+        out = mp.get_context("spawn").Manager().dict()   # no fork of this threaded process
         mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
         for r in range(world):
             x = _tokens(r)
