@@ -78,3 +78,38 @@ def test_memory_footprint_closed_form():
     assert f["int4_asym_g128_bytes"] / f["fp16_bytes"] == (0.5 + 4 / 128) / 2 == 0.265625
     assert f["int4_sym_g128_bytes"] / f["fp16_bytes"] == (0.5 + 2 / 128) / 2 == 0.2578125
     assert f["ratio_asym_g128"] == 0.2656 and f["ratio_sym_g128"] == 0.2578
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The clock record the bench line carries: the median SM clock of the samples, the throttle reasons
+    seen (NVML's bitmask mapped to names), the highest power; and an 'unavailable' record without NVML.
+    The fake only answers reads, as the real sampler only reads."""
+    import sys
+    import time
+    import types
+
+    clocks = iter([1965, 1965, 1800] + [1965] * 10000)
+    nv = types.ModuleType("pynvml")
+    nv.NVML_CLOCK_SM = 1
+    nv.nvmlClocksEventReasonSwPowerCap = 0x4
+    nv.nvmlClocksEventReasonHwSlowdown = 0x8
+    nv.nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nv.nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nv.nvmlInit = lambda: None
+    nv.nvmlDeviceGetHandleByUUID = lambda u: "gpu0"
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    nv.nvmlDeviceGetClockInfo = lambda h, c: next(clocks)
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 | 0x1   # power cap and an unnamed bit
+    nv.nvmlDeviceGetPowerUsage = lambda h: 712_300                    # mW
+    monkeypatch.setitem(sys.modules, "pynvml", nv)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: types.SimpleNamespace(uuid="1234"))
+    with bench.ClockSampler(0, period_s=0.001) as cs:
+        time.sleep(0.05)
+    s = cs.summary()
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["samples"] >= 3
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 712.3
+
+    monkeypatch.setitem(sys.modules, "pynvml", None)                  # import fails: no NVML
+    with bench.ClockSampler(0) as cs:
+        pass
+    assert cs.summary()["reasons"] == ["unavailable"] and cs.summary()["samples"] == 0
