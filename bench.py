@@ -143,7 +143,8 @@ class ClockSampler:
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
+        with open(p) as f:
+            d = json.load(f)
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
                 "bf16_tflops_sustained": d.get("bf16_tflops_sustained") or d["bf16_tflops"], "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
@@ -206,12 +207,16 @@ def traffic_from_profiles(name):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    for line in open(p):
+    with open(p) as fh:
+        lines = fh.readlines()
+    for line in lines:
         f = line.split()
         if len(f) == 4 and f[0] == name:
             src = os.path.join(ROOT, f[3])
-            if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == f[2]:
-                return int(float(f[1]))
+            if os.path.exists(src):
+                with open(src, "rb") as fs:
+                    if hashlib.sha256(fs.read()).hexdigest() == f[2]:
+                        return int(float(f[1]))
     return None
 
 

@@ -113,3 +113,19 @@ def test_clock_sampler_with_a_fake_nvml(monkeypatch):
     with bench.ClockSampler(0) as cs:
         pass
     assert cs.summary()["reasons"] == ["unavailable"] and cs.summary()["samples"] == 0
+
+
+def test_traffic_figure_is_dropped_when_its_kernel_source_changes(tmp_path, monkeypatch):
+    """profiles/traffic.txt keys each ncu DRAM figure to the SHA-256 of the kernel source it was captured
+    from: the bench reports it while the source is unchanged and null once it differs."""
+    import hashlib
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "kern.cu"
+    src.write_text("__global__ void k() {}\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles" / "traffic.txt").write_text(f"k_launch 123456 {digest} kern.cu\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profiles("k_launch") == 123456
+    assert bench.traffic_from_profiles("other") is None
+    src.write_text("__global__ void k() { }\n")
+    assert bench.traffic_from_profiles("k_launch") is None
