@@ -135,6 +135,14 @@ def _stream(stream=None):
     return stream.cuda_stream
 
 
+def _weights_on(device, *weights):
+    """Every Q4Weight of a call lives on the inputs' device (a host or other-device buffer would be read
+    through a pointer the kernels cannot use)."""
+    for w in weights:
+        if w is not None and w.packed.device != device:
+            raise ValueError(f"a weight is on {w.packed.device}, the inputs on {device}")
+
+
 def _hold(stream, *tensors):
     """A call on a stream other than the current one: the caching allocator ties a tensor's memory to the
     stream it was allocated on, so a workspace or output that this wrapper made (and that may be dropped
@@ -223,6 +231,23 @@ class Q4Weight:
 
     def __init__(self, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor | None, n: int, k: int,
                  group: int, symmetric: bool):
+        # the library trusts these sizes: a buffer that is short, strided, of another type or on another
+        # device than the sizes say would be read past its end (or from the host) by the kernels
+        if n < 0 or k <= 0 or k % 2 or group <= 0 or k % group:
+            raise ValueError(f"an INT4 weight needs n >= 0, an even k > 0 and k % group == 0 (n={n}, k={k}, group={group})")
+        for t, dt, cnt, name in ((packed, torch.uint8, n * (k // 2), "packed"),
+                                 (scales, torch.float16, n * (k // group), "scales"),
+                                 (zeros, torch.float16, n * (k // group), "zeros")):
+            if t is None:
+                if name == "zeros" and not symmetric:
+                    raise ValueError("an asymmetric INT4 weight needs its zero points")
+                continue
+            if not isinstance(t, torch.Tensor) or t.dtype != dt:
+                raise TypeError(f"{name} must be a {dt} tensor")
+            if not t.is_contiguous() or t.numel() != cnt:
+                raise ValueError(f"{name} must be contiguous with {cnt} elements, got {tuple(t.shape)}")
+            if t.device != packed.device:
+                raise ValueError(f"{name} is on {t.device}, packed on {packed.device}")
         self.packed, self.scales, self.zeros = packed, scales, zeros
         self.n, self.k, self.group, self.symmetric = n, k, group, bool(symmetric)
         self.desc = q4_weight(n, k, group, int(bool(symmetric)), packed.data_ptr(), scales.data_ptr(),
@@ -255,7 +280,10 @@ def q4_quantize_pack(w: torch.Tensor, group: int, symmetric: bool, dev_status: t
     """RTN group quantization + packing of an fp32 [n][k] CUDA tensor."""
     _dev(w, torch.float32, "w")
     n, k = w.shape
+    if out is not None and (out.n, out.k, out.group, out.symmetric) != (n, k, group, bool(symmetric)):
+        raise ValueError(f"out holds a [{out.n}][{out.k}] group-{out.group} weight, not [{n}][{k}] group-{group}")
     q = out or Q4Weight.empty(n, k, group, symmetric, device=w.device)
+    _weights_on(w.device, q)
     _hold(stream, q.packed, q.scales, q.zeros)
     _check(_lib.q4_quantize_pack(_ptr(w), n, k, group, int(bool(symmetric)), _ptr(q.packed), _ptr(q.scales),
                                  _ptr(q.zeros), _ptr(dev_status), _stream(stream)), "q4_quantize_pack")
@@ -284,6 +312,7 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
     """y[m][n] = x[m][k] . dequant(W)^T; x bf16 CUDA tensor.  workspace: "auto" (the per-device one of
     linear_workspace: a GEMM of few output tiles is split along K), None (never split) or a uint8 tensor."""
     _dev(x, torch.bfloat16, "x")
+    _weights_on(x.device, w)
     m = x.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
@@ -305,6 +334,7 @@ def q4_linear_w4a16_swiglu(gate: torch.Tensor, up: torch.Tensor, w: Q4Weight, ou
     """y[m][n] = h[m][k] . dequant(W)^T with h = silu(gate) * up (fp32 CUDA tensors [m][k], m <= 4)."""
     _dev(gate, torch.float32, "gate")
     _dev(up, torch.float32, "up")
+    _weights_on(gate.device, w)
     m = gate.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=gate.device)
@@ -322,6 +352,7 @@ class GroupedGemv:
         if not (len(xs) == len(ws) == len(ys) and 1 <= len(xs) <= 8):
             raise ValueError("a grouped call takes 1 to 8 problems, as many x, w and y")
         self.count = len(xs)
+        _weights_on(xs[0].device, *ws)
         self.m = xs[0].numel() // ws[0].k
         for x, w in zip(xs, ws):
             _numel(x, self.m * w.k, "x")   # every problem has the same m
@@ -358,6 +389,7 @@ class GemvChain:
         for st in stages:
             begin.append(begin[-1] + len(st))
         dev = probs[0][2].device
+        _weights_on(dev, *[w for _, w, _ in probs])
         ods = set()
         xs, gs, us = [], [], []
         for x, w, y in probs:
@@ -434,6 +466,7 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
     workspace: as q4_linear_w4a16's."""
     _dev(xq, torch.int8, "xq")
     _dev(scale_a, torch.float32, "scale_a")
+    _weights_on(xq.device, w)
     m = xq.shape[0]
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
@@ -478,6 +511,7 @@ def moe_q4_forward(x: torch.Tensor, router_w: torch.Tensor, router_bias: torch.T
     T, H = x.shape
     dev = x.device
     E = _router(router_w, router_bias, H, dev)
+    _weights_on(dev, *experts, *(shared or ()))
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=dev)
     od = _out(y, (T, H), dev)
@@ -524,6 +558,7 @@ def moe_q4_forward_classes(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     dev = x.device
     E = _router(router_w, router_bias, H, dev)
     n = len(class_experts)
+    _weights_on(dev, *[w for trip in class_experts for w in trip])
     if len(class_begin) != n + 1:
         raise ValueError("class_begin needs one more entry than there are classes")
     if y is None:
@@ -561,6 +596,7 @@ def moe_q4_forward_range(x: torch.Tensor, router_w: torch.Tensor, router_bias: t
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
     E = _router(router_w, router_bias, H, x.device)
+    _weights_on(x.device, *experts)
     if y is None:
         y = torch.empty((T, H), dtype=torch.float32, device=x.device)
     _dev(y, torch.float32, "y")
@@ -608,6 +644,7 @@ def moe_q4_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_bias:
     _dev(router_w, torch.float32, "router_w")
     T, H = x.shape
     E = _router(router_w, router_bias, H, x.device)
+    _weights_on(x.device, *experts)
     if y is None:
         y = torch.empty((T, H), dtype=out_dtype, device=x.device)
     od = _out(y, (T, H), x.device)
@@ -660,6 +697,7 @@ def moe_q4_forward_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, e_base: 
     _dev(x_rows, torch.bfloat16, "x_rows")
     _dev(row_expert, torch.int32, "row_expert")
     R, H = x_rows.shape
+    _weights_on(x_rows.device, *experts)
     E = experts[0].n // I
     _numel(row_expert, R, "row_expert")
     if row_weight is not None:

@@ -421,3 +421,40 @@ def test_pair_positions_fit_int32():
     ex = (q4.q4_weight * 3)(_w(n=E * 128, k=H), _w(n=E * 128, k=H), _w(n=E * H, k=128))
     assert L.moe_q4_forward(FAKE, T, H, FAKE, None, E, topk, ex, 128, FAKE, 0, None, None, None, None, None, FAKE,
                             1 << 40, None, None) == q4.Q4_ERR_SHAPE
+
+
+def test_weight_buffers_are_checked_against_their_sizes():
+    """The kernels trust a weight's n, k and group: a Q4Weight whose buffers are of another type, short,
+    strided, split across devices or missing its zero points is refused when it is made, and a weight on
+    another device than a call's inputs is refused at the call."""
+    import torch
+    n, k, g = 8, 256, 64
+
+    def make(packed=None, scales=None, zeros="default", sym=False, **kw):
+        packed = torch.zeros((n, k // 2), dtype=torch.uint8) if packed is None else packed
+        scales = torch.zeros((n, k // g), dtype=torch.float16) if scales is None else scales
+        zeros = torch.zeros((n, k // g), dtype=torch.float16) if isinstance(zeros, str) else zeros
+        return q4.Q4Weight(packed, scales, zeros, kw.get("n", n), kw.get("k", k), kw.get("group", g), sym)
+
+    w = make()
+    assert (w.n, w.k, w.group) == (n, k, g)
+    make(zeros=None, sym=True)                                             # symmetric: no zero points
+    q4.Q4Weight(torch.zeros((0, k // 2), dtype=torch.uint8), torch.zeros((0, k // g), dtype=torch.float16),
+                None, 0, k, g, True)                                        # an empty weight
+    bad = [
+        (TypeError, dict(packed=torch.zeros((n, k // 2), dtype=torch.int8))),
+        (TypeError, dict(scales=torch.zeros((n, k // g), dtype=torch.float32))),
+        (ValueError, dict(packed=torch.zeros((n, k // 2 - 1), dtype=torch.uint8))),     # short
+        (ValueError, dict(scales=torch.zeros((k // g, n), dtype=torch.float16).t())),   # strided
+        (ValueError, dict(zeros=None)),                                                 # asymmetric, no zeros
+        (ValueError, dict(zeros=torch.zeros((n, k // g), dtype=torch.float16, device="meta"))),
+        (ValueError, dict(k=255)),
+        (ValueError, dict(group=0)),
+        (ValueError, dict(k=192, group=128)),
+    ]
+    for err, kw in bad:
+        with pytest.raises(err):
+            make(**kw)
+    q4._weights_on(torch.device("cpu"), w, None)
+    with pytest.raises(ValueError):
+        q4._weights_on(torch.device("meta"), w)
