@@ -313,6 +313,8 @@ def q4_linear_w4a16(x: torch.Tensor, w: Q4Weight, out_dtype=torch.float32, y: to
     linear_workspace: a GEMM of few output tiles is split along K), None (never split) or a uint8 tensor."""
     _dev(x, torch.bfloat16, "x")
     _weights_on(x.device, w)
+    if x.numel() % w.k:
+        raise ValueError(f"x holds {x.numel()} values, not whole rows of k = {w.k}")
     m = x.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=x.device)
@@ -335,6 +337,9 @@ def q4_linear_w4a16_swiglu(gate: torch.Tensor, up: torch.Tensor, w: Q4Weight, ou
     _dev(gate, torch.float32, "gate")
     _dev(up, torch.float32, "up")
     _weights_on(gate.device, w)
+    if gate.numel() % w.k:
+        raise ValueError(f"gate holds {gate.numel()} values, not whole rows of k = {w.k}")
+    _numel(up, gate.numel(), "up")
     m = gate.numel() // w.k
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=gate.device)
@@ -452,6 +457,10 @@ def act_quant_per_token(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a
     m, k = x.shape
     xq = torch.empty((m, k), dtype=torch.int8, device=x.device) if xq is None else xq
     scale_a = torch.empty((m,), dtype=torch.float32, device=x.device) if scale_a is None else scale_a
+    for t, dt, cnt, name in ((xq, torch.int8, m * k, "xq"), (scale_a, torch.float32, m, "scale_a")):
+        _numel(_dev(t, dt, name), cnt, name)
+        if t.device != x.device:
+            raise ValueError(f"{name} is on {t.device}, x on {x.device}")
     fn = _lib.act_quant_per_token_f16 if f16 else _lib.act_quant_per_token
     _hold(stream, xq, scale_a)
     _check(fn(_ptr(x), m, k, _ptr(xq), _ptr(scale_a), _ptr(dev_status), _stream(stream)),
@@ -467,7 +476,14 @@ def q4_linear_w4a8(xq: torch.Tensor, scale_a: torch.Tensor, w: Q4Weight, out_dty
     _dev(xq, torch.int8, "xq")
     _dev(scale_a, torch.float32, "scale_a")
     _weights_on(xq.device, w)
-    m = xq.shape[0]
+    if xq.numel() % w.k:
+        raise ValueError(f"xq holds {xq.numel()} codes, not whole rows of k = {w.k}")
+    m = xq.numel() // w.k
+    _numel(scale_a, m, "scale_a")
+    if acc_dbg is not None:
+        _numel(_dev(acc_dbg, torch.int32, "acc_dbg"), m * w.n * (w.k // w.group), "acc_dbg")
+    if scale_a.device != xq.device or (acc_dbg is not None and acc_dbg.device != xq.device):
+        raise ValueError("xq, scale_a and acc_dbg must be on one device")
     if y is None:
         y = torch.empty((m, w.n), dtype=out_dtype, device=xq.device)
     od = _out(y, (m, w.n), xq.device)
